@@ -1,0 +1,257 @@
+/*
+ * imq.h -- C ABI of the IM-Unpack exact low-bit integer GEMM for NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "IM-Unpack: Training and Inference with Arbitrarily Low Precision Integers"
+ * (atlas.scime.ai summary page), sections "Approach", "Problem", "Key results", the measured-effects
+ * table and "Limitations".  The page states the method in prose only; every point it leaves open is
+ * fixed below and marked READING.
+ *
+ * The hot path has three stages, one entry point each:
+ *   1. imq_rtn_quantize   round-to-nearest quantisation: the p-th percentile of |x| of each group maps
+ *                         to the bound beta, heavy hitters are kept unclipped   ("Approach", "Problem",
+ *                         measured-effects rows on beta and p)
+ *   2. imq_plan           per-line outlier statistics and the per-matrix choice of row or column
+ *                         unpacking ("Approach": chosen per matrix from outlier counts; the Mix row and
+ *                         the four fixed-strategy rows of the measured-effects table)
+ *   3. imq_unpacked_gemm  digit-split unpacking into b-bit integers, b-bit integer GEMMs on the tensor
+ *                         cores, then bit-shift scaling and accumulation that give back the exact
+ *                         integer product ("Approach"), plus an fp32 dequantised copy.
+ *
+ * Conventions shared by every call
+ *   - Matrices are dense and row-major with a leading dimension (elements between consecutive rows).
+ *   - Every tensor pointer is DEVICE memory owned by the caller unless a parameter says "host".
+ *   - Every call is asynchronous on the given stream except imq_plan (it reads a small summary back
+ *     to the host to size the unpacked operands) and the imq_plan_* query calls.
+ *   - Argument errors are returned at once and launch nothing.  Errors found by a kernel (a non-finite
+ *     input, an integer that leaves its type) are written to a per-device status word; the next
+ *     imq_plan call or imq_device_status() returns it.  No call aborts the process.
+ *   - Every wait inside a kernel is bounded; a wait that runs out sets IMQ_ERR_TIMEOUT and the kernel
+ *     returns instead of hanging the device.
+ *   - GEMM notation: C = A * B with A logically M x K, B logically K x N, unpack width b in [2, 8],
+ *     radix R = 2^(b-1).  The b-bit in-range set is |v| <= R-1 (READING: symmetric sign-magnitude
+ *     digits, so every digit of an entry has the entry's sign).
+ */
+#ifndef IMQ_H
+#define IMQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL selects the legacy default stream. */
+typedef struct CUstream_st *imq_stream_t;
+
+typedef enum {
+  IMQ_OK = 0,
+  IMQ_ERR_ARG = 1,         /* null pointer, bad size, stride, dtype, b outside [2,8], p outside (0,1]   */
+  IMQ_ERR_NONFINITE = 2,   /* NaN or Inf in a quantiser input                                           */
+  IMQ_ERR_RANGE = 3,       /* |x*s| >= 2^31, an int16 output above 32767, or an int32 C requested while */
+                           /* the plan's bound says the product may leave int32                          */
+  IMQ_ERR_BUFFER = 4,      /* workspace smaller than imq_plan_info.workspace_bytes                      */
+  IMQ_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out                                    */
+  IMQ_ERR_CUDA = 6,        /* a CUDA runtime call failed                                                 */
+  IMQ_ERR_UNSUPPORTED = 7  /* legal input outside what the kernels implement (see imq_plan)             */
+} imq_status;
+
+typedef enum { IMQ_F32 = 0, IMQ_BF16 = 1, IMQ_I16 = 2, IMQ_I32 = 3, IMQ_I64 = 4 } imq_dtype;
+
+/* Quantisation groups, relative to the STORED matrix passed to imq_rtn_quantize. */
+typedef enum { IMQ_PER_TENSOR = 0, IMQ_PER_ROW = 1, IMQ_PER_COL = 2 } imq_gran;
+
+/* Unpack strategy: Mix decides per matrix; the fixed ones force (A direction)/(B direction), named
+ * for the C = A*B convention: "row" of A = an output row (OUTER), "col" of A = an inner index (INNER),
+ * "row" of B = an inner index (INNER), "col" of B = an output column (OUTER).
+ * READING: the page never says whether its GEMM is A*B or A*B^T; the directions are therefore named
+ * by axis (OUTER/INNER) in imq_plan_info. */
+typedef enum { IMQ_MIX = 0, IMQ_ROW_ROW = 1, IMQ_ROW_COL = 2, IMQ_COL_ROW = 3, IMQ_COL_COL = 4 } imq_strategy;
+
+/* Direction a matrix is unpacked in.  NONE: the matrix has no out-of-range entry (Mix only). */
+typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2 } imq_dir;
+
+#define IMQ_MAX_GROUPS 64   /* exponent groups e = lA + lB of the inner dimension                         */
+#define IMQ_INNER_PAD 128   /* each exponent group of the unpacked inner dimension is padded to this      */
+#define IMQ_A_GROUP 128     /* OUTER-unpacked rows of A are packed in groups of this many unpacked rows   */
+#define IMQ_B_GROUP 32      /* OUTER-unpacked columns of B are packed in groups of this many columns      */
+
+/* ------------------------------------------------------------------------------------------------ */
+/* 1. Round-to-nearest quantisation                                                                  */
+/* ------------------------------------------------------------------------------------------------ */
+/*
+ * imq_rtn_quantize -- per group g (the whole tensor, one stored row or one stored column):
+ *   q_g   = nearest-rank p-quantile of |x| over the group: sort |x| ascending into v_1..v_n,
+ *           k = clamp(ceil(p*n), 1, n), q = v_k  (READING: nearest rank, so q is an element of the
+ *           data and p = 1 gives the maximum, as the p=100% ablation row of the measured-effects
+ *           table requires).  If q == 0 the group's maximum is used; if that is 0 too, s = Delta = 1.
+ *   s_g   = (float)beta / q_g              fp32, correctly rounded
+ *   x_int = rint_half_even(fp32(x * s_g))  no clipping: heavy hitters stay outside +-beta
+ *           ("Problem" and "Approach"; clipping is the separate 99.5% ablation row)
+ *   Delta_g = q_g / (float)beta            fp32, the dequantisation step (x ~= Delta * x_int)
+ *
+ * X       device, rows x cols, row-major with leading dimension ld (>= cols), dtype xt (F32 or BF16).
+ * Xint    device, rows x cols, leading dimension ldq (>= cols), dtype it (I16 or I32).
+ * delta   device, fp32, 1 / rows / cols entries for PER_TENSOR / PER_ROW / PER_COL.
+ * qval    device or NULL, fp32, same length as delta: the selected percentile values q_g.
+ * rowmax  device or NULL, int32[rows]: max |Xint| of each stored row.
+ * colmax  device or NULL, int32[cols]: max |Xint| of each stored column.
+ * Errors: IMQ_ERR_ARG at once; IMQ_ERR_NONFINITE / IMQ_ERR_RANGE through the device status word.
+ * Scratch: PER_TENSOR uses a small per-device buffer the library allocates once on first use.
+ */
+imq_status imq_rtn_quantize(const void *X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                            imq_gran g, double p, int32_t beta,
+                            void *Xint, imq_dtype it, int64_t ldq,
+                            float *delta, float *qval, int32_t *rowmax, int32_t *colmax,
+                            imq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------------ */
+/* 2. Unpack plan                                                                                    */
+/* ------------------------------------------------------------------------------------------------ */
+typedef struct imq_plan imq_plan_t;   /* opaque, owned by the library, freed by imq_plan_destroy */
+
+typedef struct {
+  int32_t e;            /* scale exponent of the group: its products are weighted by R^e            */
+  int32_t pad_;
+  int64_t k_offset;     /* first unpacked inner index of the group (a multiple of IMQ_INNER_PAD)   */
+  int64_t k_len;        /* number of real (t, lA, lB) pairs in the group                            */
+  int64_t k_len_padded; /* k_len rounded up to IMQ_INNER_PAD                                          */
+} imq_group;
+
+typedef struct {
+  int32_t b;                 /* unpack bit width                                                   */
+  int32_t strategy;          /* imq_strategy the plan was made with                                */
+  int32_t dir_a, dir_b;      /* imq_dir chosen for A and B                                         */
+  int64_t M, K, N;           /* original GEMM shape                                                */
+  int64_t M_unp;             /* rows of the unpacked A' (OUTER: a multiple of IMQ_A_GROUP)         */
+  int64_t N_unp;             /* rows of the unpacked B'^T (OUTER: a multiple of IMQ_B_GROUP)       */
+  int64_t K_unp;             /* unpacked inner length including padding                           */
+  int64_t M_eff, N_eff, K_eff; /* unpadded sizes: sum of row levels, column levels, inner pairs    */
+  double  ratio;             /* unpack ratio M_eff*N_eff*K_eff / (M*N*K)  (READING: executed MACs   */
+                             /* over original MACs; the page names the metric without a formula)  */
+  double  bound;             /* sum_t max_i|A[i,t]| * max_j|B[t,j]|: bounds |C| and every partial  */
+                             /* sum of the fold-back (exact below 2^53)                            */
+  int32_t acc_bits;          /* 32 when bound < 2^31 (int32 C is exact), else 64                   */
+  int32_t n_groups;          /* exponent groups of the inner dimension                             */
+  int32_t lmax_a_row, lmax_a_col, lmax_b_row, lmax_b_col;  /* largest level per line kind         */
+  int64_t sum_l_a_row, sum_l_a_col, sum_l_b_row, sum_l_b_col; /* sums of levels per line kind       */
+  int64_t oor_lines_a_row, oor_lines_a_col, oor_lines_b_row, oor_lines_b_col; /* lines with level>1 */
+  size_t  workspace_bytes;   /* device bytes imq_unpacked_gemm needs for A' and B'^T               */
+} imq_plan_info;
+
+/*
+ * imq_plan -- levels, outlier counts, the direction of each matrix and the unpacked layout
+ * ("Approach": row or column unpacking chosen per matrix from outlier counts).
+ *
+ *   L(v) = 1 if |v| <= R-1, else the number of base-R digits of |v|.
+ *   Level of a line = L(max |v| over the line).  A line "holds outliers" when its level is > 1.
+ *   Expansion factors: A outer (row unpack) = sum_i L(A row i) / M, A inner (column unpack)
+ *   = sum_t L(A col t) / K; B inner (row unpack) = sum_t L(B row t) / K, B outer (column unpack)
+ *   = sum_j L(B col j) / N.
+ *   Mix (READING of "chosen per matrix via outlier counts"): per matrix, the direction with the
+ *   smaller factor; on a tie the one with fewer lines holding outliers; then row unpacking.  A matrix
+ *   without any out-of-range entry is not unpacked (IMQ_DIR_NONE).
+ *
+ * A       device, logical M x K.  transA = 0: stored M x K with leading dim lda; transA = 1: stored
+ *         K x M (A^T row-major) with leading dim lda.   dtype it (I16 or I32), as written by
+ *         imq_rtn_quantize.
+ * B       device, logical K x N.  transB = 0: stored K x N; transB = 1: stored N x K (B^T row-major).
+ * a_rowmax, a_colmax, b_rowmax, b_colmax
+ *         device or NULL, int32 max |v| per logical line (A rows: M, A cols: K, B rows: K, B cols: N),
+ *         e.g. the rowmax/colmax side outputs of imq_rtn_quantize.  When all four are given the plan
+ *         skips its own pass over A and B; when any is NULL all four are computed.
+ * plan    out: a new plan object.
+ * Synchronises the stream once (reads a summary of a few hundred bytes).  Returns any pending device
+ * status (e.g. IMQ_ERR_NONFINITE from a preceding quantisation) before planning.
+ * IMQ_ERR_UNSUPPORTED: more than IMQ_MAX_GROUPS exponent groups, a line level above 31, an exponent
+ * group whose raw int32 accumulation could overflow (k_len*(R-1)^2 >= 2^31), or a bound so large that
+ * two TMEM accumulators cannot hold the exact sum (bound / R^e1 >= 2^31 with e1 the smallest
+ * non-zero exponent present).
+ */
+imq_status imq_plan(const void *A, const void *B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                    int32_t transA, int64_t lda, int32_t transB, int64_t ldb,
+                    int32_t b, imq_strategy strategy,
+                    const int32_t *a_rowmax, const int32_t *a_colmax,
+                    const int32_t *b_rowmax, const int32_t *b_colmax,
+                    imq_plan_t **plan, imq_stream_t stream);
+
+/* Copies the plan summary to *info (host).  No device work. */
+imq_status imq_plan_info_get(const imq_plan_t *plan, imq_plan_info *info);
+
+/* Copies the per-line levels to HOST buffers (int8): a_row[M], a_col[K], b_row[K], b_col[N].
+ * Any pointer may be NULL.  Synchronous. */
+imq_status imq_plan_levels(const imq_plan_t *plan, int8_t *a_row, int8_t *a_col,
+                           int8_t *b_row, int8_t *b_col);
+
+/* Copies the exponent-group table (HOST, up to max_groups entries; *n_out gets the count). */
+imq_status imq_plan_groups(const imq_plan_t *plan, imq_group *groups, int32_t max_groups,
+                           int32_t *n_out);
+
+/* Frees the plan and its device arrays.  Call only after work that uses it has finished. */
+imq_status imq_plan_destroy(imq_plan_t *plan);
+
+/* ------------------------------------------------------------------------------------------------ */
+/* 3. Unpack and low-bit GEMM                                                                        */
+/* ------------------------------------------------------------------------------------------------ */
+/*
+ * imq_unpack -- digit split of A and B into b-bit integers stored as int8 ("Approach": out-of-range
+ * entries become several in-range entries by row or column unpacking).
+ *   digit d_l(v) = sgn(v) * ((|v| >> (l*(b-1))) & (R-1)), so sum_l R^l d_l(v) = v and |d_l| <= R-1.
+ * Layout (READING: the page fixes no operand order; this one is the library's):
+ *   inner index p enumerates pairs (t, lA, lB) with lA < la_t, lB < lb_t (la_t = level of A column t
+ *   when A is INNER else 1, lb_t = level of B row t when B is INNER else 1), ordered by exponent
+ *   e = lA + lB, then lA, then t; each exponent group padded with zeros to IMQ_INNER_PAD.
+ *   OUTER rows of A: source rows sorted by level L (stable), floor(IMQ_A_GROUP / L) source rows per
+ *   group of IMQ_A_GROUP unpacked rows, lines (source, level) consecutive, unused rows zero.
+ *   OUTER columns of B: the same with IMQ_B_GROUP.
+ * A_unp   device int8, M_unp x K_unp row-major (K contiguous), written in full.
+ * B_unp_t device int8, N_unp x K_unp row-major (K contiguous, i.e. B'^T), written in full.
+ * A, B must be the matrices (same pointers and layouts) the plan was made from.  Asynchronous.
+ */
+imq_status imq_unpack(const imq_plan_t *plan, const void *A, const void *B,
+                      int8_t *A_unp, int8_t *B_unp_t, imq_stream_t stream);
+
+/*
+ * imq_gemm_unpacked -- the low-bit GEMM on already unpacked operands with the fold-back epilogue:
+ *   C = sum over exponent groups e of R^e * (A'_e * B'_e), then every OUTER line folded back with its
+ *   level weight R^l ("Approach": bit-shift scaling and accumulation reproduce the integer product
+ *   exactly).  s8 x s8 -> s32 products run on the tcgen05 tensor cores; partial sums never leave
+ *   int32 inside one accumulator (the plan checks the bounds), the fold runs in int32 or int64.
+ *   Cf[i,j] = (float)C[i,j] * (deltaA[i] * deltaB[j])  (fp32; READING: the page implies dequantised
+ *   outputs but gives no formula).
+ * deltaA  device fp32: 1 value (gA = IMQ_PER_TENSOR) or M values (IMQ_PER_ROW: one per row of A).
+ * deltaB  device fp32: 1 value (IMQ_PER_TENSOR) or N values (IMQ_PER_COL: one per column of B).
+ *         Both may be NULL when Cf is NULL.
+ * Cint    device or NULL, M x N, leading dim ldc, dtype ct (I32 or I64).  I32 with
+ *         plan acc_bits == 64 returns IMQ_ERR_RANGE.
+ * Cf      device or NULL, fp32 M x N, leading dim ldcf.
+ * Asynchronous.
+ */
+imq_status imq_gemm_unpacked(const imq_plan_t *plan, const int8_t *A_unp, const int8_t *B_unp_t,
+                             const float *deltaA, imq_gran gA, const float *deltaB, imq_gran gB,
+                             void *Cint, imq_dtype ct, int64_t ldc, float *Cf, int64_t ldcf,
+                             imq_stream_t stream);
+
+/*
+ * imq_unpacked_gemm -- imq_unpack into the caller's workspace followed by imq_gemm_unpacked.
+ * workspace  device, at least imq_plan_info.workspace_bytes bytes, 1024-byte aligned.
+ */
+imq_status imq_unpacked_gemm(const imq_plan_t *plan, const void *A, const void *B,
+                             const float *deltaA, imq_gran gA, const float *deltaB, imq_gran gB,
+                             void *Cint, imq_dtype ct, int64_t ldc, float *Cf, int64_t ldcf,
+                             void *workspace, size_t workspace_bytes, imq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------------ */
+/* Status                                                                                            */
+/* ------------------------------------------------------------------------------------------------ */
+/* Synchronises the stream, returns the device status word of the current device and, when clear is
+ * non-zero, resets it to IMQ_OK. */
+imq_status imq_device_status(imq_stream_t stream, int32_t clear);
+
+/* Static, never NULL. */
+const char *imq_status_str(imq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* IMQ_H */

@@ -1,0 +1,91 @@
+/*
+ * oracle.h -- declarations of the CPU oracle for the IM-Unpack exact low-bit integer GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline leg
+ * (and its --impl reference arm) may load or call this code.  It shares no code, header, table or
+ * constant with the CUDA library under bit_integer_gemm_b200/, and neither side includes the other.
+ *
+ * Source of the method: "IM-Unpack: Training and Inference with Arbitrarily Low Precision Integers"
+ * (atlas.scime.ai summary page).  Each function cites the section it follows.  Points the page leaves
+ * open are marked READING and are the same readings the library documents in include/imq.h.
+ *
+ * Parity pins: every function here is checked by tests/test_oracle_pins.py against something other
+ * than itself (sorting, brute force, closed forms, invariants, exact library arithmetic).
+ */
+#ifndef IMQ_ORACLE_H
+#define IMQ_ORACLE_H
+#include <stdint.h>
+
+#define OR_OK 0
+#define OR_ERR_ARG 1
+#define OR_ERR_NONFINITE 2
+#define OR_ERR_RANGE 3
+
+#define OR_PER_TENSOR 0
+#define OR_PER_ROW 1
+#define OR_PER_COL 2
+
+#define OR_MIX 0
+#define OR_ROW_ROW 1
+#define OR_ROW_COL 2
+#define OR_COL_ROW 3
+#define OR_COL_COL 4
+
+#define OR_DIR_NONE 0
+#define OR_DIR_OUTER 1
+#define OR_DIR_INNER 2
+
+#define OR_MAX_GROUPS 64
+#define OR_INNER_PAD 128
+#define OR_A_GROUP 128
+#define OR_B_GROUP 32
+
+typedef struct {
+  int32_t b, strategy, dir_a, dir_b;
+  int64_t M, K, N;
+  int64_t M_unp, N_unp, K_unp;
+  int64_t M_eff, N_eff, K_eff;
+  double ratio;
+  double bound;            /* sum_t max_i|A_it| * max_j|B_tj|, rounded to double          */
+  int32_t bound_lt_2_31;   /* exact comparison of the bound with 2^31                     */
+  int32_t n_groups;
+  int32_t lmax[4];         /* A rows, A cols, B rows, B cols                              */
+  int64_t suml[4];
+  int64_t oor_lines[4];
+  int32_t group_e[OR_MAX_GROUPS];
+  int64_t group_off[OR_MAX_GROUPS];
+  int64_t group_len[OR_MAX_GROUPS];
+  int64_t group_padded[OR_MAX_GROUPS];
+} oracle_plan_t;
+
+/* percentile.c */
+float oracle_percentile_abs(const float *v, int64_t n, double p);
+/* rtn.c */
+int oracle_rtn_quantize(const float *x, int64_t rows, int64_t cols, int gran, double p, int beta,
+                        int64_t *xint, float *delta, float *qval);
+/* digits.c */
+int oracle_level(int64_t v, int b);
+int64_t oracle_digit(int64_t v, int l, int b);
+void oracle_digits_array(const int64_t *v, int64_t n, int b, int nl, int64_t *out, int32_t *lev);
+/* plan.c */
+int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N, int b,
+                int strategy, int32_t *LrA, int32_t *LcA, int32_t *LrB, int32_t *LcB,
+                oracle_plan_t *out);
+int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcA,
+                     const int32_t *LrB, const int32_t *LcB, int32_t *tK, int32_t *lAk,
+                     int32_t *lBk, int32_t *srcA, int32_t *lvlA, int32_t *srcB, int32_t *lvlB);
+/* unpack.c */
+int oracle_unpack(const oracle_plan_t *pl, const int32_t *tK, const int32_t *lAk,
+                  const int32_t *lBk, const int32_t *srcA, const int32_t *lvlA,
+                  const int32_t *srcB, const int32_t *lvlB, const int64_t *A, const int64_t *B,
+                  int8_t *Aunp, int8_t *Bunp_t);
+/* gemm.c */
+void oracle_gemm_i64(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N,
+                     int64_t *C, int nthreads);
+int oracle_unpacked_gemm(const oracle_plan_t *pl, const int32_t *srcA, const int32_t *lvlA,
+                         const int32_t *srcB, const int32_t *lvlB, const int8_t *Aunp,
+                         const int8_t *Bunp_t, int64_t *C);
+/* dequant.c */
+void oracle_dequant(const int64_t *C, int64_t M, int64_t N, const float *dA, int gA,
+                    const float *dB, int gB, double *Cf);
+#endif

@@ -1,0 +1,252 @@
+/*
+ * plan.c -- oracle step 3-4 and the unpacked layout: levels, outlier counts, the per-matrix direction
+ * (the Mix strategy or a fixed one), the unpack ratio and the index maps of the unpacked operands.
+ * TEST INFRASTRUCTURE ONLY (see oracle.h).
+ *
+ * IM-Unpack summary page:
+ *   "Approach"  -- rows or columns that hold out-of-bound entries are unpacked; the choice between row
+ *                  and column unpacking is made per matrix from outlier counts.
+ *   measured-effects table -- the Mix strategy against fixed row/row, row/col, col/row and col/col
+ *                  unpacking, compared by unpack ratio (beta = 15, b = 5).
+ *   "Experimental setup" -- the unpack ratio is one of the reported metrics (no formula given).
+ * READINGs (the page gives no formulas):
+ *   level of a line = number of base-R digits of its largest |entry|; it "holds outliers" if > 1.
+ *   expansion factor of a direction = mean level of the lines unpacked in that direction.
+ *   Mix: per matrix the smaller factor; tie -> fewer lines holding outliers; tie -> row unpacking;
+ *        a matrix without any out-of-range entry is not unpacked.
+ *   unpack ratio = M_eff * N_eff * K_eff / (M * N * K): executed multiply-adds over original ones.
+ *   layout: inner pairs (t, lA, lB) ordered by e = lA + lB, then lA, then t, each exponent group padded
+ *   with zeros to OR_INNER_PAD; OUTER lines sorted by level (stable), floor(G / L) source lines per
+ *   group of G unpacked lines (G = OR_A_GROUP for rows of A, OR_B_GROUP for columns of B), the L lines
+ *   of one source consecutive, unused lines empty.
+ */
+#include <stdlib.h>
+#include <string.h>
+#include "oracle.h"
+
+static int64_t iabs64(int64_t v) { return v < 0 ? -v : v; }
+
+int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N, int b,
+                int strategy, int32_t *LrA, int32_t *LcA, int32_t *LrB, int32_t *LcB,
+                oracle_plan_t *out) {
+  if (b < 2 || b > 8 || M < 0 || K < 0 || N < 0 || strategy < 0 || strategy > 4) return OR_ERR_ARG;
+  memset(out, 0, sizeof(*out));
+  out->b = b;
+  out->strategy = strategy;
+  out->M = M;
+  out->K = K;
+  out->N = N;
+
+  /* levels of every line */
+  for (int64_t i = 0; i < M; ++i) LrA[i] = 1;
+  for (int64_t t = 0; t < K; ++t) { LcA[t] = 1; LrB[t] = 1; }
+  for (int64_t j = 0; j < N; ++j) LcB[j] = 1;
+  for (int64_t i = 0; i < M; ++i)
+    for (int64_t t = 0; t < K; ++t) {
+      int l = oracle_level(A[i * K + t], b);
+      if (l > LrA[i]) LrA[i] = l;
+      if (l > LcA[t]) LcA[t] = l;
+    }
+  for (int64_t t = 0; t < K; ++t)
+    for (int64_t j = 0; j < N; ++j) {
+      int l = oracle_level(B[t * N + j], b);
+      if (l > LrB[t]) LrB[t] = l;
+      if (l > LcB[j]) LcB[j] = l;
+    }
+  const int32_t *vecs[4] = {LrA, LcA, LrB, LcB};
+  const int64_t lens[4] = {M, K, K, N};
+  for (int v = 0; v < 4; ++v) {
+    out->lmax[v] = 1;
+    for (int64_t x = 0; x < lens[v]; ++x) {
+      out->suml[v] += vecs[v][x];
+      if (vecs[v][x] > 1) out->oor_lines[v] += 1;
+      if (vecs[v][x] > out->lmax[v]) out->lmax[v] = vecs[v][x];
+    }
+  }
+
+  /* direction of each matrix */
+  int da, db;
+  if (strategy == OR_MIX) {
+    if (out->oor_lines[0] == 0 && out->oor_lines[1] == 0) {
+      da = OR_DIR_NONE;
+    } else {
+      /* row factor suml[0]/M against column factor suml[1]/K, compared exactly */
+      int64_t row_side = out->suml[0] * K, col_side = out->suml[1] * M;
+      if (row_side < col_side) da = OR_DIR_OUTER;
+      else if (row_side > col_side) da = OR_DIR_INNER;
+      else if (out->oor_lines[0] < out->oor_lines[1]) da = OR_DIR_OUTER;
+      else if (out->oor_lines[0] > out->oor_lines[1]) da = OR_DIR_INNER;
+      else da = OR_DIR_OUTER;
+    }
+    if (out->oor_lines[2] == 0 && out->oor_lines[3] == 0) {
+      db = OR_DIR_NONE;
+    } else {
+      /* row factor suml[2]/K against column factor suml[3]/N */
+      int64_t row_side = out->suml[2] * N, col_side = out->suml[3] * K;
+      if (row_side < col_side) db = OR_DIR_INNER;
+      else if (row_side > col_side) db = OR_DIR_OUTER;
+      else if (out->oor_lines[2] < out->oor_lines[3]) db = OR_DIR_INNER;
+      else if (out->oor_lines[2] > out->oor_lines[3]) db = OR_DIR_OUTER;
+      else db = OR_DIR_INNER;
+    }
+  } else {
+    da = (strategy == OR_ROW_ROW || strategy == OR_ROW_COL) ? OR_DIR_OUTER : OR_DIR_INNER;
+    db = (strategy == OR_ROW_ROW || strategy == OR_COL_ROW) ? OR_DIR_INNER : OR_DIR_OUTER;
+  }
+  out->dir_a = da;
+  out->dir_b = db;
+
+  /* levels each index carries in the unpacked GEMM */
+  out->M_eff = 0;
+  for (int64_t i = 0; i < M; ++i) out->M_eff += (da == OR_DIR_OUTER) ? LrA[i] : 1;
+  out->N_eff = 0;
+  for (int64_t j = 0; j < N; ++j) out->N_eff += (db == OR_DIR_OUTER) ? LcB[j] : 1;
+  int maxla = (da == OR_DIR_INNER) ? out->lmax[1] : 1;
+  int maxlb = (db == OR_DIR_INNER) ? out->lmax[2] : 1;
+  out->K_eff = 0;
+  for (int64_t t = 0; t < K; ++t) {
+    int64_t la = (da == OR_DIR_INNER) ? LcA[t] : 1;
+    int64_t lb = (db == OR_DIR_INNER) ? LrB[t] : 1;
+    out->K_eff += la * lb;
+  }
+  if (M > 0 && N > 0 && K > 0)
+    out->ratio = ((double)out->M_eff / (double)M) * ((double)out->N_eff / (double)N) *
+                 ((double)out->K_eff / (double)K);
+  else
+    out->ratio = 1.0;
+
+  /* exponent groups of the inner dimension */
+  int64_t off = 0;
+  int ng = 0;
+  for (int e = 0; e <= maxla + maxlb - 2; ++e) {
+    int64_t len = 0;
+    for (int la = 0; la < maxla; ++la) {
+      int lb = e - la;
+      if (lb < 0 || lb >= maxlb) continue;
+      for (int64_t t = 0; t < K; ++t) {
+        int64_t a = (da == OR_DIR_INNER) ? LcA[t] : 1;
+        int64_t bb = (db == OR_DIR_INNER) ? LrB[t] : 1;
+        if (a > la && bb > lb) len += 1;
+      }
+    }
+    if (len == 0) continue;
+    if (ng >= OR_MAX_GROUPS) return OR_ERR_ARG;
+    int64_t padded = (len + OR_INNER_PAD - 1) / OR_INNER_PAD * OR_INNER_PAD;
+    out->group_e[ng] = e;
+    out->group_off[ng] = off;
+    out->group_len[ng] = len;
+    out->group_padded[ng] = padded;
+    off += padded;
+    ng += 1;
+  }
+  out->n_groups = ng;
+  out->K_unp = off;
+
+  /* outer sizes: groups of lines of equal level */
+  if (da == OR_DIR_OUTER) {
+    int64_t groups = 0;
+    for (int L = 1; L <= out->lmax[0]; ++L) {
+      int64_t cnt = 0;
+      for (int64_t i = 0; i < M; ++i) cnt += (LrA[i] == L);
+      int64_t per = OR_A_GROUP / L;
+      groups += (cnt + per - 1) / per;
+    }
+    out->M_unp = groups * OR_A_GROUP;
+  } else {
+    out->M_unp = M;
+  }
+  if (db == OR_DIR_OUTER) {
+    int64_t groups = 0;
+    for (int L = 1; L <= out->lmax[3]; ++L) {
+      int64_t cnt = 0;
+      for (int64_t j = 0; j < N; ++j) cnt += (LcB[j] == L);
+      int64_t per = OR_B_GROUP / L;
+      groups += (cnt + per - 1) / per;
+    }
+    out->N_unp = groups * OR_B_GROUP;
+  } else {
+    out->N_unp = N;
+  }
+
+  /* bound on |C| and on every partial sum of the fold-back */
+  __int128 bound = 0;
+  for (int64_t t = 0; t < K; ++t) {
+    int64_t ma = 0, mb = 0;
+    for (int64_t i = 0; i < M; ++i)
+      if (iabs64(A[i * K + t]) > ma) ma = iabs64(A[i * K + t]);
+    for (int64_t j = 0; j < N; ++j)
+      if (iabs64(B[t * N + j]) > mb) mb = iabs64(B[t * N + j]);
+    bound += (__int128)ma * (__int128)mb;
+  }
+  out->bound = (double)bound;
+  out->bound_lt_2_31 = bound < ((__int128)1 << 31);
+  return OR_OK;
+}
+
+/* Fills the index maps of the layout described at the top of this file.
+ * tK/lAk/lBk: K_unp entries (tK = -1 on padding).  srcA/lvlA: M_unp entries (srcA = -1 on unused
+ * lines).  srcB/lvlB: N_unp entries. */
+int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcA,
+                     const int32_t *LrB, const int32_t *LcB, int32_t *tK, int32_t *lAk,
+                     int32_t *lBk, int32_t *srcA, int32_t *lvlA, int32_t *srcB, int32_t *lvlB) {
+  const int da = pl->dir_a, db = pl->dir_b;
+  const int64_t M = pl->M, K = pl->K, N = pl->N;
+  int maxla = (da == OR_DIR_INNER) ? pl->lmax[1] : 1;
+  int maxlb = (db == OR_DIR_INNER) ? pl->lmax[2] : 1;
+
+  for (int64_t p = 0; p < pl->K_unp; ++p) { tK[p] = -1; lAk[p] = 0; lBk[p] = 0; }
+  for (int g = 0; g < pl->n_groups; ++g) {
+    int e = pl->group_e[g];
+    int64_t p = pl->group_off[g];
+    for (int la = 0; la < maxla; ++la) {
+      int lb = e - la;
+      if (lb < 0 || lb >= maxlb) continue;
+      for (int64_t t = 0; t < K; ++t) {
+        int64_t a = (da == OR_DIR_INNER) ? LcA[t] : 1;
+        int64_t bb = (db == OR_DIR_INNER) ? LrB[t] : 1;
+        if (a > la && bb > lb) {
+          tK[p] = (int32_t)t;
+          lAk[p] = la;
+          lBk[p] = lb;
+          p += 1;
+        }
+      }
+    }
+    if (p != pl->group_off[g] + pl->group_len[g]) return OR_ERR_ARG;
+  }
+
+  for (int64_t u = 0; u < pl->M_unp; ++u) { srcA[u] = -1; lvlA[u] = 0; }
+  if (da == OR_DIR_OUTER) {
+    int64_t grp = 0;
+    for (int L = 1; L <= pl->lmax[0]; ++L) {
+      int64_t per = OR_A_GROUP / L, rank = 0;
+      for (int64_t i = 0; i < M; ++i) {
+        if (LrA[i] != L) continue;
+        int64_t base = (grp + rank / per) * OR_A_GROUP + (rank % per) * L;
+        for (int l = 0; l < L; ++l) { srcA[base + l] = (int32_t)i; lvlA[base + l] = l; }
+        rank += 1;
+      }
+      grp += (rank + per - 1) / per;
+    }
+  } else {
+    for (int64_t i = 0; i < M; ++i) srcA[i] = (int32_t)i;
+  }
+
+  for (int64_t w = 0; w < pl->N_unp; ++w) { srcB[w] = -1; lvlB[w] = 0; }
+  if (db == OR_DIR_OUTER) {
+    int64_t grp = 0;
+    for (int L = 1; L <= pl->lmax[3]; ++L) {
+      int64_t per = OR_B_GROUP / L, rank = 0;
+      for (int64_t j = 0; j < N; ++j) {
+        if (LcB[j] != L) continue;
+        int64_t base = (grp + rank / per) * OR_B_GROUP + (rank % per) * L;
+        for (int l = 0; l < L; ++l) { srcB[base + l] = (int32_t)j; lvlB[base + l] = l; }
+        rank += 1;
+      }
+      grp += (rank + per - 1) / per;
+    }
+  } else {
+    for (int64_t j = 0; j < N; ++j) srcB[j] = (int32_t)j;
+  }
+  return OR_OK;
+}

@@ -1,0 +1,397 @@
+"""CPU pins of the oracle against facts that do not come from the oracle itself.
+
+Each test names what fixes the expected value: sorting / counting (percentile), exact rational
+arithmetic (rounding, dequantisation), the defining properties of sign-magnitude base-R digits,
+brute-force integer products, closed forms of the unpack ratio, and the Mix rule re-derived from the
+line levels.  Method source: "IM-Unpack: Training and Inference with Arbitrarily Low Precision
+Integers" (atlas.scime.ai summary): "Approach", "Problem", measured-effects table.
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+BF16_FINITE = None
+
+
+def _all_finite_bf16():
+    global BF16_FINITE
+    if BF16_FINITE is None:
+        bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+        exp = (bits >> 7) & 0xFF
+        BF16_FINITE = bits[exp != 0xFF]
+    return BF16_FINITE
+
+
+# ------------------------------------------------------------------------------------------------
+# percentile (measured-effects table: p = 95% default, p = 100% ablation)
+# ------------------------------------------------------------------------------------------------
+def _rank_by_counting(v, p):
+    """Smallest |x| such that at least ceil(p*n) values are <= it (nearest-rank, by counting)."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    k = oracle.nearest_rank(a.size, p)
+    for c in sorted(set(a.tolist())):
+        if (a <= c).sum() >= k:
+            return c
+    raise AssertionError
+
+
+@pytest.mark.parametrize("p", [0.01, 0.5, 0.95, 0.999, 1.0])
+def test_percentile_matches_counting_definition(p):
+    rng = np.random.default_rng(11)
+    for n in (1, 2, 3, 7, 20, 101):
+        v = rng.standard_normal(n).astype(np.float32) * np.float32(rng.uniform(0.1, 100))
+        assert float(oracle.percentile_abs(v, p)) == _rank_by_counting(v, p)
+
+
+def test_percentile_order_invariant_bruteforce():
+    rng = np.random.default_rng(12)
+    for _ in range(20):
+        n = int(rng.integers(1, 7))
+        v = (rng.integers(-4, 5, size=n)).astype(np.float32)  # many ties
+        p = float(rng.choice([0.2, 0.5, 0.95, 1.0]))
+        want = _rank_by_counting(v, p)
+        for perm in itertools.permutations(range(n)):
+            assert float(oracle.percentile_abs(v[list(perm)], p)) == want
+
+
+def test_percentile_p1_is_max_and_ranks_of_configs():
+    rng = np.random.default_rng(13)
+    v = rng.standard_normal(1000).astype(np.float32)
+    assert oracle.percentile_abs(v, 1.0) == np.abs(v).max()
+    # ranks k = ceil(0.95 n) for the group sizes of the workloads (nearest rank, double arithmetic)
+    want = {128: 122, 2048: 1946, 4096: 3892, 8192: 7783, 11008: 10458,
+            8388608: 7969178, 33554432: 31876711}
+    for n, k in want.items():
+        assert oracle.nearest_rank(n, 0.95) == k
+
+
+# ------------------------------------------------------------------------------------------------
+# RTN ("Problem"/"Approach": heavy hitters kept, not clipped)
+# ------------------------------------------------------------------------------------------------
+def _rne_int(fr: Fraction) -> int:
+    """Round a rational to the nearest integer, ties to even, in exact arithmetic."""
+    fl = math.floor(fr)
+    rem = fr - fl
+    if rem > Fraction(1, 2):
+        return fl + 1
+    if rem < Fraction(1, 2):
+        return fl
+    return fl if fl % 2 == 0 else fl + 1
+
+
+def test_rtn_exhaustive_bf16_against_exact_rounding():
+    bits = _all_finite_bf16()
+    x = oracle.bf16_bits_to_f32(bits).reshape(1, -1)
+    for beta in (15, 31, 255):
+        xint, delta, q = oracle.rtn_quantize(x, oracle.PER_TENSOR, 0.95, beta)
+        s = np.float32(beta) / np.float32(q[0])  # IEEE fp32 division, correctly rounded
+        # a bf16 value has 8 significant bits and s 24, so x*s is exact in float64; casting that
+        # float64 to float32 is the single correct rounding of the fp32 product
+        prod32 = (x.astype(np.float64) * np.float64(s)).astype(np.float32)
+        want = np.array([_rne_int(Fraction(float(v))) for v in prod32.ravel()], dtype=np.int64)
+        assert np.array_equal(xint.ravel(), want)
+        assert delta[0] == np.float32(q[0]) / np.float32(beta)
+
+
+def test_rtn_rank_k_maps_to_beta_and_sign_symmetry():
+    g = workloads.q_proj()[0]
+    X = oracle.as_f32(g.A.data[:64], "bf16")
+    for beta in (15, 31):
+        xint, delta, q = oracle.rtn_quantize(X, oracle.PER_ROW, 0.95, beta)
+        n = X.shape[1]
+        k = oracle.nearest_rank(n, 0.95)
+        for r in range(X.shape[0]):
+            row = X[r]
+            idx = np.flatnonzero(np.abs(row) == q[r])
+            assert idx.size > 0, "q must be an element of the group"
+            assert np.all(np.abs(xint[r, idx]) == beta)
+            assert (np.abs(xint[r]) <= beta).sum() >= k
+        # heavy hitters are not clipped: the x60 channels exceed beta
+        assert np.abs(xint).max() > 10 * beta
+        xneg, dneg, qneg = oracle.rtn_quantize(-X, oracle.PER_ROW, 0.95, beta)
+        assert np.array_equal(xneg, -xint) and np.array_equal(dneg, delta)
+
+
+def test_rtn_granularities_agree_with_per_group_calls():
+    rng = np.random.default_rng(14)
+    X = rng.standard_normal((9, 13)).astype(np.float32)
+    xr, dr, qr = oracle.rtn_quantize(X, oracle.PER_ROW, 0.9, 15)
+    xc, dc, qc = oracle.rtn_quantize(X, oracle.PER_COL, 0.9, 15)
+    for r in range(9):
+        a, d, q = oracle.rtn_quantize(X[r:r + 1], oracle.PER_TENSOR, 0.9, 15)
+        assert np.array_equal(a[0], xr[r]) and d[0] == dr[r] and q[0] == qr[r]
+    for c in range(13):
+        a, d, q = oracle.rtn_quantize(X[:, c:c + 1].copy(), oracle.PER_TENSOR, 0.9, 15)
+        assert np.array_equal(a[:, 0], xc[:, c]) and d[0] == dc[c]
+
+
+def test_rtn_zero_groups_and_errors():
+    x = np.zeros((2, 40), np.float32)
+    x[1, 3] = 2.0  # 39 zeros: the 95% rank is 0, so the maximum is used
+    xi, d, q = oracle.rtn_quantize(x, oracle.PER_ROW, 0.95, 15)
+    assert d[0] == 1.0 and q[0] == 0.0 and not xi[0].any()
+    assert q[1] == 2.0 and xi[1, 3] == 15
+    bad = np.ones((1, 4), np.float32)
+    bad[0, 2] = np.nan
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.rtn_quantize(bad, oracle.PER_TENSOR, 0.95, 15)
+    assert e.value.status == oracle.ERR_NONFINITE
+    big = np.full((1, 100), 1e-3, np.float32)
+    big[0, 0] = 1e8  # 1e8 / 1e-3 * 15 >= 2^31
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.rtn_quantize(big, oracle.PER_TENSOR, 0.95, 15)
+    assert e.value.status == oracle.ERR_RANGE
+
+
+# ------------------------------------------------------------------------------------------------
+# digits ("Approach": an out-of-bound integer becomes several in-bound b-bit integers)
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("b", range(2, 9))
+def test_digits_exhaustive(b):
+    R = 1 << (b - 1)
+    nl = math.ceil(21 / (b - 1)) + 1
+    v = np.arange(-(1 << 20) + 1, 1 << 20, dtype=np.int64)
+    d, lev = oracle.digits_array(v, b, nl)
+    w = np.array([R ** l for l in range(nl)], dtype=np.int64)
+    assert np.array_equal(d @ w, v)                          # reconstruction
+    assert np.abs(d).max() <= R - 1                          # in range
+    assert np.all(d * np.sign(v)[:, None] >= 0)              # every digit carries v's sign
+    # level: 1 for |v| <= R-1, else the smallest L with |v| < R^L
+    a = np.abs(v)
+    want = np.ones_like(a)
+    for L in range(2, nl + 1):
+        want[a >= R ** (L - 1)] = L
+    assert np.array_equal(lev, want)
+    # digits above the level are zero
+    cols = np.arange(nl)[None, :]
+    assert not d[cols >= lev[:, None]].any()
+
+
+# ------------------------------------------------------------------------------------------------
+# unpacked product == direct product ("Approach": the original GEMM is reproduced exactly)
+# ------------------------------------------------------------------------------------------------
+def _brute(A, B):
+    M, K = A.shape
+    N = B.shape[1]
+    return np.array([[sum(int(A[i, t]) * int(B[t, j]) for t in range(K)) for j in range(N)]
+                     for i in range(M)], dtype=np.int64)
+
+
+def test_unpacked_equals_direct_random_tiny():
+    rng = np.random.default_rng(21)
+    for case in range(1000):
+        M, K, N = (int(x) for x in rng.integers(1, 10, size=3))
+        b = int(rng.integers(2, 9))
+        A, B = workloads.random_case(rng, M, K, N, big=5000, frac=float(rng.choice([0.0, 0.05, 0.3])))
+        direct = _brute(A, B) if case < 100 else oracle.gemm_i64(A, B)
+        if case < 100:
+            assert np.array_equal(direct, oracle.gemm_i64(A, B))
+        R = 1 << (b - 1)
+        for st in range(5):
+            pl = oracle.plan(A, B, b, st)
+            Au, Bu = oracle.unpack(pl, A, B)
+            assert np.abs(Au.astype(np.int64)).max(initial=0) <= R - 1
+            assert np.abs(Bu.astype(np.int64)).max(initial=0) <= R - 1
+            assert np.array_equal(oracle.unpacked_gemm(pl, Au, Bu), direct), (case, st, b)
+            # the bound covers |C|
+            assert np.abs(direct).max(initial=0) <= pl.bound
+
+
+def test_direct_product_against_numpy_int64():
+    rng = np.random.default_rng(22)
+    for M, K, N in [(1, 1, 1), (3, 5, 7), (64, 128, 64), (512, 512, 512), (37, 511, 129)]:
+        A, B = workloads.random_case(rng, M, K, N, big=30000)
+        want = np.matmul(A, B)  # exact here: |C| < 2^63
+        assert np.array_equal(oracle.gemm_i64(A, B), want)
+        assert np.array_equal(oracle.gemm_exact(A, B), want)
+
+
+def test_tiny_config_int64_against_brute_force():
+    g = workloads.tiny()[0]
+    A, dA, _ = oracle.rtn_quantize(oracle.as_f32(g.A.data, "f32"), oracle.PER_TENSOR, 0.95, 15)
+    B, dB, _ = oracle.rtn_quantize(oracle.as_f32(g.B.data, "f32"), oracle.PER_TENSOR, 0.95, 15)
+    direct = _brute(A, B)
+    assert np.array_equal(oracle.gemm_i64(A, B), direct)
+    pl = oracle.plan(A, B, 5, oracle.MIX)
+    Au, Bu = oracle.unpack(pl, A, B)
+    assert np.array_equal(oracle.unpacked_gemm(pl, Au, Bu), direct)
+    assert pl.ratio > 1.0  # the planted heavy hitters need unpacking
+
+
+# ------------------------------------------------------------------------------------------------
+# unpack ratio (named as a metric; no formula on the page) -- closed forms
+# ------------------------------------------------------------------------------------------------
+def test_ratio_closed_forms():
+    K, M, N, b = 40, 6, 5, 5
+    A = np.full((M, K), 3, np.int64)
+    A[:, 7] = 100          # one column, every row, level 2 at b=5 (16 <= 100 < 256)
+    B = np.full((K, N), -2, np.int64)
+    pl = oracle.plan(A, B, b, oracle.COL_ROW)
+    assert pl.K_eff == K + 1 and pl.ratio == pytest.approx((K + 1) / K, rel=0, abs=1e-15)
+    pl = oracle.plan(A, B, b, oracle.ROW_ROW)
+    assert pl.M_eff == 2 * M and pl.ratio == 2.0
+    # Mix picks the column for A (factor (K+1)/K < 2) and does not unpack B
+    pl = oracle.plan(A, B, b, oracle.MIX)
+    assert (pl.dir_a, pl.dir_b) == (oracle.DIR_INNER, oracle.DIR_NONE)
+    # nothing out of range: identity plan, ratio exactly 1, product is a plain int8 GEMM
+    rng = np.random.default_rng(23)
+    A8 = rng.integers(-127, 128, size=(33, 70)).astype(np.int64)
+    B8 = rng.integers(-127, 128, size=(70, 17)).astype(np.int64)
+    pl = oracle.plan(A8, B8, 8, oracle.MIX)
+    assert (pl.dir_a, pl.dir_b, pl.ratio) == (oracle.DIR_NONE, oracle.DIR_NONE, 1.0)
+    assert pl.K_unp == 128 and pl.M_unp == 33 and pl.N_unp == 17
+    Au, Bu = oracle.unpack(pl, A8, B8)
+    assert np.array_equal(Au[:, :70], A8.astype(np.int8)) and not Au[:, 70:].any()
+    assert np.array_equal(Bu[:, :70], B8.T.astype(np.int8))
+
+
+def test_ratio_equals_counted_macs():
+    rng = np.random.default_rng(24)
+    for _ in range(200):
+        M, K, N = (int(x) for x in rng.integers(1, 12, size=3))
+        b = int(rng.integers(2, 9))
+        A, B = workloads.random_case(rng, M, K, N, big=3000, frac=0.2)
+        for st in range(5):
+            pl = oracle.plan(A, B, b, st)
+            mp = pl.maps
+            macs = int((mp["srcA"] >= 0).sum()) * int((mp["srcB"] >= 0).sum()) * int((mp["tK"] >= 0).sum())
+            assert macs == pl.M_eff * pl.N_eff * pl.K_eff
+            assert pl.ratio == pytest.approx(macs / (M * N * K), rel=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# Mix ("Approach": direction chosen per matrix from outlier counts)
+# ------------------------------------------------------------------------------------------------
+def _levels_numpy(X, b):
+    R = 1 << (b - 1)
+    a = np.abs(X)
+    L = np.ones_like(a)
+    t = a // R
+    while (t > 0).any():
+        L += (t > 0)
+        t //= R
+    return L
+
+
+def test_mix_choice_bruteforce():
+    rng = np.random.default_rng(25)
+    for _ in range(300):
+        M, K, N = (int(x) for x in rng.integers(1, 10, size=3))
+        b = int(rng.integers(2, 9))
+        A, B = workloads.random_case(rng, M, K, N, big=int(rng.choice([50, 5000])), frac=0.15)
+        pl = oracle.plan(A, B, b, oracle.MIX)
+        LA, LB = _levels_numpy(A, b), _levels_numpy(B, b)
+        lar, lac, lbr, lbc = LA.max(1), LA.max(0), LB.max(1), LB.max(0)
+        assert np.array_equal(pl.levels["a_row"], lar) and np.array_equal(pl.levels["a_col"], lac)
+        assert np.array_equal(pl.levels["b_row"], lbr) and np.array_equal(pl.levels["b_col"], lbc)
+
+        def choose(row_lv, col_lv, row_is_outer):
+            if (row_lv > 1).sum() == 0 and (col_lv > 1).sum() == 0:
+                return oracle.DIR_NONE
+            fr, fc = Fraction(int(row_lv.sum()), row_lv.size), Fraction(int(col_lv.sum()), col_lv.size)
+            nr, nc = int((row_lv > 1).sum()), int((col_lv > 1).sum())
+            row_dir = oracle.DIR_OUTER if row_is_outer else oracle.DIR_INNER
+            col_dir = oracle.DIR_INNER if row_is_outer else oracle.DIR_OUTER
+            if fr != fc:
+                return row_dir if fr < fc else col_dir
+            if nr != nc:
+                return row_dir if nr < nc else col_dir
+            return row_dir
+
+        assert pl.dir_a == choose(lar, lac, True)
+        assert pl.dir_b == choose(lbr, lbc, False)
+
+
+def test_mix_beats_fixed_on_channel_outliers():
+    """The measured-effects table reports Mix below every fixed strategy on linear layers, where
+    heavy hitters sit in channels; a channel-structured case reproduces that ordering."""
+    rng = np.random.default_rng(26)
+    M, K, N, b = 64, 96, 48, 5
+    A = rng.integers(-15, 16, size=(M, K)).astype(np.int64)
+    B = rng.integers(-15, 16, size=(K, N)).astype(np.int64)
+    A[:, [3, 50]] *= 40          # activation outlier channels: columns of A
+    B[[10, 70], :] *= 30         # weight outlier input channels: rows of B
+    ratios = {st: oracle.plan(A, B, b, st).ratio for st in range(5)}
+    mix = oracle.plan(A, B, b, oracle.MIX)
+    assert (mix.dir_a, mix.dir_b) == (oracle.DIR_INNER, oracle.DIR_INNER)  # col/row
+    assert ratios[oracle.MIX] == ratios[oracle.COL_ROW]
+    others = (oracle.ROW_ROW, oracle.ROW_COL, oracle.COL_COL)
+    assert all(ratios[oracle.MIX] < ratios[st] for st in others), ratios
+    assert ratios[oracle.MIX] < 1.1
+
+
+# ------------------------------------------------------------------------------------------------
+# dequantisation (implied by RTN GEMMs replacing FP GEMMs)
+# ------------------------------------------------------------------------------------------------
+def test_dequant_exact_rational_bound():
+    rng = np.random.default_rng(27)
+    C = rng.integers(-(1 << 40), 1 << 40, size=(7, 5)).astype(np.int64)
+    C[0, 0] = 0
+    dA = rng.uniform(1e-4, 1.0, 7).astype(np.float32)
+    dB = rng.uniform(1e-4, 1.0, 5).astype(np.float32)
+    Cf = oracle.dequant(C, dA, oracle.PER_ROW, dB, oracle.PER_COL)
+    assert Cf[0, 0] == 0.0
+    for i in range(7):
+        for j in range(5):
+            exact = Fraction(int(C[i, j])) * Fraction(float(dA[i])) * Fraction(float(dB[j]))
+            if exact != 0:
+                assert abs(Fraction(float(Cf[i, j])) - exact) / abs(exact) <= Fraction(1, 2 ** 51)
+    ones = np.ones(1, np.float32)
+    assert np.array_equal(oracle.dequant(C, ones, oracle.PER_TENSOR, ones, oracle.PER_TENSOR),
+                          C.astype(np.float64))
+
+
+# ------------------------------------------------------------------------------------------------
+# the unpacked layout (a READING: the page fixes no operand order) is the documented one
+# ------------------------------------------------------------------------------------------------
+def test_layout_follows_documented_order():
+    rng = np.random.default_rng(28)
+    for _ in range(150):
+        M, K, N = (int(x) for x in rng.integers(1, 40, size=3))
+        b = int(rng.integers(2, 9))
+        A, B = workloads.random_case(rng, M, K, N, big=4000, frac=0.2)
+        for st in range(5):
+            pl = oracle.plan(A, B, b, st)
+            mp, lv = pl.maps, pl.levels
+            la = lv["a_col"] if pl.dir_a == oracle.DIR_INNER else np.ones(K, np.int32)
+            lb = lv["b_row"] if pl.dir_b == oracle.DIR_INNER else np.ones(K, np.int32)
+            # inner: groups ascending in e, offsets multiples of 128, inside a group (lA, t) ascending
+            want = []
+            for e, off, ln, padded in pl.groups:
+                assert off % 128 == 0 and padded % 128 == 0 and padded - ln < 128
+                pairs = sorted((lA, t) for t in range(K) for lA in range(la[t]) for lB in [e - lA]
+                               if 0 <= lB < lb[t])
+                got = list(zip(mp["lAk"][off:off + ln].tolist(), mp["tK"][off:off + ln].tolist()))
+                assert got == pairs
+                assert np.all(mp["lAk"][off:off + ln] + mp["lBk"][off:off + ln] == e)
+                assert np.all(mp["tK"][off + ln:off + padded] == -1)
+                want.append(e)
+            assert want == sorted(want)
+            # outer: per group one level L, floor(G/L) sources of that level, lines (src, l) in order
+            for src, lvl, lines, G, dirv, outer in (
+                    (mp["srcA"], mp["lvlA"], lv["a_row"], 128, pl.dir_a, oracle.DIR_OUTER),
+                    (mp["srcB"], mp["lvlB"], lv["b_col"], 32, pl.dir_b, oracle.DIR_OUTER)):
+                if dirv != outer:
+                    assert np.array_equal(src, np.arange(src.size)) and not lvl.any()
+                    continue
+                assert src.size % G == 0
+                seen = []
+                for g0 in range(0, src.size, G):
+                    s, l = src[g0:g0 + G], lvl[g0:g0 + G]
+                    used = s >= 0
+                    n = int(used.sum())
+                    assert used[:n].all() and not used[n:].any()
+                    L = int(lines[s[0]])
+                    assert n % L == 0 and n // L <= G // L
+                    for k in range(n // L):
+                        assert np.all(s[k * L:(k + 1) * L] == s[k * L])
+                        assert np.array_equal(l[k * L:(k + 1) * L], np.arange(L))
+                        assert lines[s[k * L]] == L
+                        seen.append((L, int(s[k * L])))
+                assert seen == sorted(seen) and len(seen) == lines.size
