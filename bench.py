@@ -1,0 +1,382 @@
+"""Throughput of the exact unpacked integer GEMM path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole path on the q_proj-shaped workload (X 2048x4096 bf16 per-token RTN,
+W 4096x4096 bf16 per-output-channel RTN, p = 0.95, beta = 15, b = 5, Mix): percentile + RTN of X and W,
+plan, unpack, tcgen05 int8 GEMM with fold-back and dequantisation.  `value` is the effective TOPS of
+the original-shape product, 2*M*N*K / step time, with inputs resident in HBM; `e2e` is the same through
+the C ABI with the inputs copied from pinned host memory and C (int32) plus Cf (fp32) copied back inside
+the timed region.  Between timed steps L2 is flushed by writing 256 MB.  The dominant kernel (the GEMM)
+is timed with CUDA events on its stream for the roofline.  With --gpus N > 1 every rank runs its own
+replica (the path has no data exchange); time is the max over ranks.
+
+--impl reference times the CPU oracle (the reference arm of this build) on a bounded sample of the same
+workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "effective TOPS of exact unpacked int GEMM (orig. shape) and % of B200 INT8 peak"
+UNIT = "TOPS"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), \
+            float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _workload():
+    g = workloads.q_proj()[0]
+    return g
+
+
+def _config(g, extra=None):
+    c = {"workload": f"q_proj-shaped X {g.M}x{g.K} bf16 per-token RTN x W {g.K}x{g.N} bf16 "
+                     f"per-channel RTN, p={g.p}, beta={g.beta}, b={g.b}, Mix",
+         "M": g.M, "K": g.K, "N": g.N, "b": g.b, "beta": g.beta, "p": g.p, "strategy": "mix",
+         "l2": "flushed between timed steps (256 MB write)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------------
+class Clocks:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.samples = []
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                self.samples.append(f)
+
+    def summary(self):
+        if not getattr(self, "samples", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4) if s[5 + k] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+class Path:
+    """Preallocated buffers and one step of the path on the current device."""
+
+    def __init__(self, imq, torch, g, X, W):
+        self.imq, self.torch, self.g = imq, torch, g
+        dev = X.device
+        self.X, self.W = X, W
+        M, K, N = g.M, g.K, g.N
+        t = torch
+        self.Xint = t.empty((M, K), dtype=t.int16, device=dev)
+        self.Wint = t.empty((K, N), dtype=t.int16, device=dev)
+        self.dX = t.empty(M, dtype=t.float32, device=dev)
+        self.dW = t.empty(N, dtype=t.float32, device=dev)
+        self.mx = [t.empty(n, dtype=t.int32, device=dev) for n in (M, K, K, N)]
+        self.C = t.empty((M, N), dtype=t.int32, device=dev)
+        self.Cf = t.empty((M, N), dtype=t.float32, device=dev)
+        self.ws = None
+        self.info = None
+        self.launches = 0
+
+    def step(self, gemm_events=None):
+        imq, g = self.imq, self.g
+        imq.imq_rtn_quantize(self.X, imq.IMQ_PER_ROW, g.p, g.beta, Xint=self.Xint, delta=self.dX,
+                             want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
+        imq.imq_rtn_quantize(self.W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
+                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3])
+        plan = imq.imq_plan(self.Xint, self.Wint, g.b, imq.IMQ_MIX, maxes=self.mx)
+        I = plan.info
+        if self.ws is None or self.ws.numel() < I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048:
+            self.ws = self.torch.empty(I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048,
+                                       dtype=self.torch.int8, device=self.X.device)
+        na = I["M_unp"] * I["K_unp"]
+        a_off = (-self.ws.data_ptr()) % 1024
+        b_off = a_off + (na + 1023) // 1024 * 1024
+        Au = self.ws[a_off:a_off + na].view(I["M_unp"], I["K_unp"])
+        Bu = self.ws[b_off:b_off + I["N_unp"] * I["K_unp"]].view(I["N_unp"], I["K_unp"])
+        imq.imq_unpack(plan, self.Xint, self.Wint, A_unp=Au, B_unp_t=Bu)
+        if gemm_events is not None:
+            gemm_events[0].record()
+        imq.imq_gemm_unpacked(plan, Au, Bu, self.dX, imq.IMQ_PER_ROW, self.dW, imq.IMQ_PER_COL, C=self.C,
+                              Cf=self.Cf)
+        if gemm_events is not None:
+            gemm_events[1].record()
+        self.info = I
+        # kernels of this library launched by the step: 2 quantisers, levels, inner map, one outer map
+        # per OUTER operand, 2 unpack kernels, one zeroing kernel per OUTER operand, the GEMM
+        outer = int(I["dir_a"] == imq.IMQ_DIR_OUTER) + int(I["dir_b"] == imq.IMQ_DIR_OUTER)
+        self.launches = 2 + 1 + (1 if I["K_unp"] > 0 else 0) + outer + 2 + outer + 1
+        plan.destroy()
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import bit_integer_gemm_b200 as imq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    imq.lib()
+
+    g = _workload()
+    Xh = torch.from_numpy(g.A.data.view(np.int16)).view(torch.bfloat16)
+    Wh = torch.from_numpy(g.B.data.view(np.int16)).view(torch.bfloat16)
+    X = Xh.to(dev)
+    W = Wh.to(dev)
+    path = Path(imq, torch, g, X, W)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize()
+    if imq.imq_device_status() != imq.IMQ_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    # ---- device-resident timed region ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with Clocks(dev.index) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record()
+            path.step(gev[k])
+            ends[k].record()
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    gemm_ms = [a.elapsed_time(b) for a, b in gev]
+    total_ms = sum(step_ms)
+    launches = path.launches * args.steps
+
+    # ---- end to end through the C ABI with host buffers ----
+    Xp = Xh.pin_memory()
+    Wp = Wh.pin_memory()
+    Cp = torch.empty((g.M, g.N), dtype=torch.int32).pin_memory()
+    Cfp = torch.empty((g.M, g.N), dtype=torch.float32).pin_memory()
+    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        e_start[k].record()
+        X.copy_(Xp, non_blocking=True)
+        W.copy_(Wp, non_blocking=True)
+        path.step()
+        Cp.copy_(path.C, non_blocking=True)
+        Cfp.copy_(path.Cf, non_blocking=True)
+        e_end[k].record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_start, e_end))
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    I = path.info
+    ops = 2.0 * g.M * g.N * g.K
+    value = ops * world * args.steps / (total_ms * 1e-3) / 1e12
+    e2e_value = ops * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    bf16_burst, bf16_sus, hbm, src = _peaks()
+    int8_peak = 2.0 * bf16_burst  # dense int8 = 2 x dense bf16 on B200 (nominal 4.5 vs 2.25 PFLOP/s)
+    exec_ops = 2.0 * I["M_unp"] * I["N_unp"] * I["K_unp"]
+    gemm_avg_ms = sum(gemm_ms) / len(gemm_ms)
+    achieved = exec_ops / (gemm_avg_ms * 1e-3) / 1e12
+    traffic = _traffic_from_profiles()
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic (seeded, bf16)",
+        "config": _config(g, {"parallelism": f"replicas x{world}", "ratio": round(I["ratio"], 4),
+                              "dir_a": I["dir_a"], "dir_b": I["dir_b"], "M_unp": I["M_unp"],
+                              "N_unp": I["N_unp"], "K_unp": I["K_unp"], "acc_bits": I["acc_bits"],
+                              "pct_int8_peak_effective": round(100 * value / world / int8_peak, 2)}),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(achieved / int8_peak, 4), "traffic": traffic,
+                     "kernel": "k_gemm (tcgen05 kind::i8)", "peak_source": f"{src} bf16 burst x2",
+                     "gemm_ms": round(gemm_avg_ms, 4), "exec_ops_per_launch": exec_ops},
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": 2 * (g.M * g.K + g.K * g.N),
+                "d2h_bytes_per_step": 8 * g.M * g.N},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(g, target_s=args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# the oracle on the host (cpu_baseline and the reference arm)
+# ------------------------------------------------------------------------------------------------
+def _oracle_sample(g, rows: int, qW=None):
+    """Definition tier of the oracle on `rows` rows of X: RTN of those rows (per token), RTN of W (per
+    channel; once, passed in when already done), the direct int64 product and the dequantisation."""
+    import oracle
+    t0 = time.perf_counter()
+    if qW is None:
+        qW = oracle.rtn_quantize(oracle.as_f32(g.B.data, "bf16"), oracle.PER_COL, g.p, g.beta)
+    xs = oracle.as_f32(g.A.data[:rows], "bf16")
+    xi, dx, _ = oracle.rtn_quantize(xs, oracle.PER_ROW, g.p, g.beta)
+    C = oracle.gemm_i64(xi, qW[0])
+    oracle.dequant(C, dx, oracle.PER_ROW, qW[1], oracle.PER_COL)
+    return time.perf_counter() - t0, qW
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(g, target_s=15.0):
+    probe_rows = 8
+    t_probe, qW = _oracle_sample(g, probe_rows)
+    t_small, _ = _oracle_sample(g, probe_rows, qW)
+    rows = int(max(probe_rows, min(g.M, probe_rows * target_s / max(t_small, 1e-3))))
+    t_w0 = time.perf_counter()
+    import oracle
+    qW = oracle.rtn_quantize(oracle.as_f32(g.B.data, "bf16"), oracle.PER_COL, g.p, g.beta)
+    t_w = time.perf_counter() - t_w0
+    t_rows, _ = _oracle_sample(g, rows, qW)
+    t = t_w + t_rows
+    ops = 2.0 * rows * g.N * g.K
+    return {"value": round(ops / t / 1e12, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"{rows} of {g.M} rows of X: RTN of those rows + RTN of all of W + int64 product + "
+                      f"dequant; {t:.1f} s on the host", "seconds": round(t, 2)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    g = _workload()
+    import oracle
+    qW = oracle.rtn_quantize(oracle.as_f32(g.B.data, "bf16"), oracle.PER_COL, g.p, g.beta)
+    # size one step (a bounded sample of rows) so that warm-up + steps take about a minute
+    t8, _ = _oracle_sample(g, 8, qW)
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(g.M, 8 * per_step / max(t8, 1e-3))))
+    for _ in range(args.warmup):
+        _oracle_sample(g, rows, qW)
+    times = [_oracle_sample(g, rows, qW)[0] for _ in range(args.steps)]
+    total = sum(times)
+    ops = 2.0 * rows * g.N * g.K
+    value = ops * args.steps / total / 1e12
+    sample = (f"{rows} of {g.M} rows of X per step: RTN of those rows + int64 product + dequant "
+              f"(W quantised once before timing)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+            "data": "synthetic (seeded, bf16)", "config": _config(g, {"parallelism": "host cores"}),
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _traffic_from_profiles():
+    """DRAM bytes per GEMM launch from the committed ncu summary of the current kernel, if present."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f).get("bytes_per_launch")
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

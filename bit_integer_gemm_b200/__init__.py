@@ -1,0 +1,286 @@
+"""Python binding of libimq.so, the B200 (sm_100a) IM-Unpack exact low-bit integer GEMM.
+
+Every function here has the name of the C entry point it calls (include/imq.h) and only marshals
+arguments: it takes torch CUDA tensors, allocates outputs that the caller did not pass, and raises
+:class:`ImqError` on a non-OK status.  All arithmetic runs in the library's CUDA kernels.  There is no
+fallback: without the built library every call raises.
+
+Method: "IM-Unpack: Training and Inference with Arbitrarily Low Precision Integers" (atlas.scime.ai
+summary), "Approach" -- RTN quantisation, per-matrix row/column unpacking of heavy hitters into b-bit
+integers, b-bit integer GEMMs and bit-shift accumulation that reproduce the integer product exactly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from collections import namedtuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libimq.so")
+
+# status codes
+IMQ_OK, IMQ_ERR_ARG, IMQ_ERR_NONFINITE, IMQ_ERR_RANGE = 0, 1, 2, 3
+IMQ_ERR_BUFFER, IMQ_ERR_TIMEOUT, IMQ_ERR_CUDA, IMQ_ERR_UNSUPPORTED = 4, 5, 6, 7
+# dtypes
+IMQ_F32, IMQ_BF16, IMQ_I16, IMQ_I32, IMQ_I64 = 0, 1, 2, 3, 4
+# quantisation groups
+IMQ_PER_TENSOR, IMQ_PER_ROW, IMQ_PER_COL = 0, 1, 2
+# strategies
+IMQ_MIX, IMQ_ROW_ROW, IMQ_ROW_COL, IMQ_COL_ROW, IMQ_COL_COL = 0, 1, 2, 3, 4
+# directions
+IMQ_DIR_NONE, IMQ_DIR_OUTER, IMQ_DIR_INNER = 0, 1, 2
+IMQ_MAX_GROUPS = 64
+
+_TORCH_TO_IMQ = {torch.float32: IMQ_F32, torch.bfloat16: IMQ_BF16, torch.int16: IMQ_I16,
+                 torch.int32: IMQ_I32, torch.int64: IMQ_I64}
+
+
+class ImqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {imq_status_str(status)} (status {status})")
+        self.status = status
+
+
+class imq_plan_info(ctypes.Structure):
+    _fields_ = [
+        ("b", ctypes.c_int32), ("strategy", ctypes.c_int32),
+        ("dir_a", ctypes.c_int32), ("dir_b", ctypes.c_int32),
+        ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("N", ctypes.c_int64),
+        ("M_unp", ctypes.c_int64), ("N_unp", ctypes.c_int64), ("K_unp", ctypes.c_int64),
+        ("M_eff", ctypes.c_int64), ("N_eff", ctypes.c_int64), ("K_eff", ctypes.c_int64),
+        ("ratio", ctypes.c_double), ("bound", ctypes.c_double),
+        ("acc_bits", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+        ("lmax_a_row", ctypes.c_int32), ("lmax_a_col", ctypes.c_int32),
+        ("lmax_b_row", ctypes.c_int32), ("lmax_b_col", ctypes.c_int32),
+        ("sum_l_a_row", ctypes.c_int64), ("sum_l_a_col", ctypes.c_int64),
+        ("sum_l_b_row", ctypes.c_int64), ("sum_l_b_col", ctypes.c_int64),
+        ("oor_lines_a_row", ctypes.c_int64), ("oor_lines_a_col", ctypes.c_int64),
+        ("oor_lines_b_row", ctypes.c_int64), ("oor_lines_b_col", ctypes.c_int64),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+    def as_dict(self) -> dict:
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class imq_group(ctypes.Structure):
+    _fields_ = [("e", ctypes.c_int32), ("pad_", ctypes.c_int32), ("k_offset", ctypes.c_int64),
+                ("k_len", ctypes.c_int64), ("k_len_padded", ctypes.c_int64)]
+
+
+# Names and argument types of every entry point of include/imq.h.
+_VP, _I32, _I64, _F64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+SIGNATURES = {
+    "imq_rtn_quantize": [_VP, _I32, _I64, _I64, _I64, _I32, _F64, _I32, _VP, _I32, _I64, _VP, _VP, _VP, _VP, _VP],
+    "imq_plan": [_VP, _VP, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32, _VP, _VP, _VP, _VP,
+                 ctypes.POINTER(_VP), _VP],
+    "imq_plan_info_get": [_VP, ctypes.POINTER(imq_plan_info)],
+    "imq_plan_levels": [_VP, _VP, _VP, _VP, _VP],
+    "imq_plan_groups": [_VP, ctypes.POINTER(imq_group), _I32, ctypes.POINTER(_I32)],
+    "imq_plan_destroy": [_VP],
+    "imq_unpack": [_VP, _VP, _VP, _VP, _VP, _VP],
+    "imq_gemm_unpacked": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP],
+    "imq_unpacked_gemm": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP, _SZ, _VP],
+    "imq_device_status": [_VP, _I32],
+    "imq_status_str": [_I32],
+}
+
+_lib = None
+
+
+def lib():
+    """Loads libimq.so (raises when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m bit_integer_gemm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int32
+        L.imq_status_str.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def imq_status_str(status: int) -> str:
+    return lib().imq_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != IMQ_OK:
+        raise ImqError(status, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _ld(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    return t.stride(0) if t.size(0) > 1 else t.size(1)
+
+
+# ------------------------------------------------------------------------------------------------
+# 1. quantisation
+# ------------------------------------------------------------------------------------------------
+Quantized = namedtuple("Quantized", "xint delta qval rowmax colmax")
+
+
+def imq_rtn_quantize(X: torch.Tensor, gran: int, p: float, beta: int, out_dtype=torch.int16,
+                     Xint=None, delta=None, qval=None, rowmax=None, colmax=None, want_qval=True,
+                     want_max=True, stream=None) -> Quantized:
+    """RTN quantisation of a stored 2-D matrix (fp32 or bf16) per tensor / stored row / stored column."""
+    rows, cols = X.shape
+    dev = X.device
+    if Xint is None:
+        Xint = torch.empty((rows, cols), dtype=out_dtype, device=dev)
+    ng = 1 if gran == IMQ_PER_TENSOR else (rows if gran == IMQ_PER_ROW else cols)
+    if delta is None:
+        delta = torch.empty(ng, dtype=torch.float32, device=dev)
+    if qval is None and want_qval:
+        qval = torch.empty(ng, dtype=torch.float32, device=dev)
+    if rowmax is None and want_max:
+        rowmax = torch.empty(rows, dtype=torch.int32, device=dev)
+    if colmax is None and want_max:
+        colmax = torch.empty(cols, dtype=torch.int32, device=dev)
+    st = lib().imq_rtn_quantize(_ptr(X), _TORCH_TO_IMQ[X.dtype], rows, cols, _ld(X), gran, float(p), int(beta),
+                                _ptr(Xint), _TORCH_TO_IMQ[Xint.dtype], _ld(Xint), _ptr(delta), _ptr(qval),
+                                _ptr(rowmax), _ptr(colmax), _stream(stream))
+    _check(st, "imq_rtn_quantize")
+    return Quantized(Xint, delta, qval, rowmax, colmax)
+
+
+# ------------------------------------------------------------------------------------------------
+# 2. plan
+# ------------------------------------------------------------------------------------------------
+class Plan:
+    """Owns an imq_plan_t handle; `info` is the imq_plan_info summary as a dict."""
+
+    def __init__(self, handle, A, B):
+        self.handle = handle
+        self._keep = (A, B)  # the plan refers to A and B
+        inf = imq_plan_info()
+        _check(lib().imq_plan_info_get(handle, ctypes.byref(inf)), "imq_plan_info_get")
+        self.info = inf.as_dict()
+
+    def levels(self):
+        I = self.info
+        import numpy as np
+        out = [np.zeros(n, np.int8) for n in (I["M"], I["K"], I["K"], I["N"])]
+        _check(lib().imq_plan_levels(self.handle, *[o.ctypes.data_as(ctypes.c_void_p) for o in out]),
+               "imq_plan_levels")
+        return dict(zip(("a_row", "a_col", "b_row", "b_col"), out))
+
+    def groups(self):
+        arr = (imq_group * IMQ_MAX_GROUPS)()
+        n = ctypes.c_int32(0)
+        _check(lib().imq_plan_groups(self.handle, arr, IMQ_MAX_GROUPS, ctypes.byref(n)), "imq_plan_groups")
+        return [(arr[i].e, arr[i].k_offset, arr[i].k_len, arr[i].k_len_padded) for i in range(n.value)]
+
+    def destroy(self):
+        if self.handle is not None:
+            lib().imq_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def imq_plan(A: torch.Tensor, B: torch.Tensor, b: int, strategy: int = IMQ_MIX, transA: bool = False,
+             transB: bool = False, maxes=None, stream=None) -> Plan:
+    """A: stored M x K (K x M when transA); B: stored K x N (N x K when transB); int16 or int32.
+    maxes: optional (a_rowmax, a_colmax, b_rowmax, b_colmax) int32 tensors over LOGICAL lines."""
+    M = A.shape[1] if transA else A.shape[0]
+    K = A.shape[0] if transA else A.shape[1]
+    N = B.shape[0] if transB else B.shape[1]
+    if A.dtype != B.dtype:
+        raise ValueError("A and B must have the same integer dtype")
+    mx = [None] * 4 if maxes is None else list(maxes)
+    h = ctypes.c_void_p()
+    st = lib().imq_plan(_ptr(A), _ptr(B), _TORCH_TO_IMQ[A.dtype], M, K, N, int(transA), _ld(A), int(transB),
+                        _ld(B), int(b), int(strategy), *[_ptr(m) for m in mx], ctypes.byref(h), _stream(stream))
+    _check(st, "imq_plan")
+    return Plan(h, A, B)
+
+
+# ------------------------------------------------------------------------------------------------
+# 3. unpack and GEMM
+# ------------------------------------------------------------------------------------------------
+def imq_unpack(plan: Plan, A: torch.Tensor, B: torch.Tensor, A_unp=None, B_unp_t=None, stream=None):
+    I = plan.info
+    dev = A.device
+    if A_unp is None:
+        A_unp = torch.empty((I["M_unp"], I["K_unp"]), dtype=torch.int8, device=dev)
+    if B_unp_t is None:
+        B_unp_t = torch.empty((I["N_unp"], I["K_unp"]), dtype=torch.int8, device=dev)
+    _check(lib().imq_unpack(plan.handle, _ptr(A), _ptr(B), _ptr(A_unp), _ptr(B_unp_t), _stream(stream)),
+           "imq_unpack")
+    return A_unp, B_unp_t
+
+
+def _outputs(I, dev, C, c_dtype, Cf, want_int, want_f32):
+    if C is None and want_int:
+        if c_dtype is None:
+            c_dtype = torch.int32 if I["acc_bits"] == 32 else torch.int64
+        C = torch.empty((I["M"], I["N"]), dtype=c_dtype, device=dev)
+    if Cf is None and want_f32:
+        Cf = torch.empty((I["M"], I["N"]), dtype=torch.float32, device=dev)
+    return C, Cf
+
+
+def imq_gemm_unpacked(plan: Plan, A_unp, B_unp_t, deltaA=None, gA=IMQ_PER_TENSOR, deltaB=None,
+                      gB=IMQ_PER_TENSOR, C=None, c_dtype=None, Cf=None, want_int=True, want_f32=True,
+                      stream=None):
+    I = plan.info
+    C, Cf = _outputs(I, A_unp.device, C, c_dtype, Cf, want_int, want_f32 and deltaA is not None)
+    st = lib().imq_gemm_unpacked(plan.handle, _ptr(A_unp), _ptr(B_unp_t), _ptr(deltaA), gA, _ptr(deltaB), gB,
+                                 _ptr(C), _TORCH_TO_IMQ[C.dtype] if C is not None else IMQ_I32,
+                                 _ld(C) if C is not None else I["N"], _ptr(Cf),
+                                 _ld(Cf) if Cf is not None else I["N"], _stream(stream))
+    _check(st, "imq_gemm_unpacked")
+    return C, Cf
+
+
+def workspace_for(plan: Plan, device=None) -> torch.Tensor:
+    n = max(int(plan.info["workspace_bytes"]), 1) + 1024
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _aligned(ws: torch.Tensor):
+    off = (-ws.data_ptr()) % 1024
+    nbytes = ws.numel() * ws.element_size()
+    return ctypes.c_void_p(ws.data_ptr() + off), max(0, nbytes - off)
+
+
+def imq_unpacked_gemm(plan: Plan, A, B, deltaA=None, gA=IMQ_PER_TENSOR, deltaB=None, gB=IMQ_PER_TENSOR,
+                      C=None, c_dtype=None, Cf=None, workspace=None, want_int=True, want_f32=True,
+                      stream=None):
+    I = plan.info
+    if workspace is None:
+        workspace = workspace_for(plan, A.device)
+    wp, wn = _aligned(workspace)
+    C, Cf = _outputs(I, A.device, C, c_dtype, Cf, want_int, want_f32 and deltaA is not None)
+    st = lib().imq_unpacked_gemm(plan.handle, _ptr(A), _ptr(B), _ptr(deltaA), gA, _ptr(deltaB), gB, _ptr(C),
+                                 _TORCH_TO_IMQ[C.dtype] if C is not None else IMQ_I32,
+                                 _ld(C) if C is not None else I["N"], _ptr(Cf),
+                                 _ld(Cf) if Cf is not None else I["N"], wp, wn, _stream(stream))
+    _check(st, "imq_unpacked_gemm")
+    return C, Cf
+
+
+def imq_device_status(clear: bool = False, stream=None) -> int:
+    return int(lib().imq_device_status(_stream(stream), int(clear)))

@@ -1,0 +1,180 @@
+// api.cu -- the C ABI declared in include/imq.h: argument checks, per-device state, status word.
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace imq {
+imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                      int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
+                      imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                      const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out, cudaStream_t st);
+
+namespace {
+__device__ int32_t g_status;  // the per-device status word (one instance per device)
+DeviceState g_dev[64];
+std::mutex g_dev_mu;
+}  // namespace
+
+imq_status device_state(DeviceState** out) {
+  int dev = 0;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return IMQ_ERR_UNSUPPORTED;
+  DeviceState& d = g_dev[dev];
+  if (!d.init) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!d.init) {
+      void* p = nullptr;
+      IMQ_CUDA_TRY(cudaGetSymbolAddress(&p, g_status));
+      IMQ_CUDA_TRY(cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev));
+      d.status = static_cast<int32_t*>(p);
+      d.init = true;
+    }
+  }
+  *out = &d;
+  return IMQ_OK;
+}
+
+}  // namespace imq
+
+using imq::DeviceState;
+
+extern "C" {
+
+imq_status imq_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld, imq_gran g,
+                            double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq, float* delta,
+                            float* qval, int32_t* rowmax, int32_t* colmax, imq_stream_t stream) {
+  return imq::launch_rtn_quantize(X, xt, rows, cols, ld, g, p, beta, Xint, it, ldq, delta, qval, rowmax,
+                                  colmax, reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                    int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b, imq_strategy strategy,
+                    const int32_t* a_rowmax, const int32_t* a_colmax, const int32_t* b_rowmax,
+                    const int32_t* b_colmax, imq_plan_t** plan, imq_stream_t stream) {
+  if (!plan) return IMQ_ERR_ARG;
+  *plan = nullptr;
+  if (it != IMQ_I16 && it != IMQ_I32) return IMQ_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || b < 2 || b > 8) return IMQ_ERR_ARG;
+  if (M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return IMQ_ERR_UNSUPPORTED;
+  if ((int)strategy < 0 || (int)strategy > 4) return IMQ_ERR_ARG;
+  if (transA != 0 && transA != 1) return IMQ_ERR_ARG;
+  if (transB != 0 && transB != 1) return IMQ_ERR_ARG;
+  if (lda < (transA ? M : K) || ldb < (transB ? K : N)) return IMQ_ERR_ARG;
+  if ((M > 0 && K > 0 && !A) || (K > 0 && N > 0 && !B)) return IMQ_ERR_ARG;
+  return imq::build_plan(A, B, it, M, K, N, transA, lda, transB, ldb, b, strategy, a_rowmax, a_colmax, b_rowmax,
+                         b_colmax, plan, reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_plan_info_get(const imq_plan_t* plan, imq_plan_info* info) {
+  if (!plan || !info) return IMQ_ERR_ARG;
+  *info = plan->info;
+  return IMQ_OK;
+}
+
+imq_status imq_plan_levels(const imq_plan_t* plan, int8_t* a_row, int8_t* a_col, int8_t* b_row, int8_t* b_col) {
+  if (!plan) return IMQ_ERR_ARG;
+  const imq_plan_info& I = plan->info;
+  int dev = 0;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  IMQ_CUDA_TRY(cudaSetDevice(plan->device));
+  cudaError_t e = cudaSuccess;
+  if (a_row && I.M) e = cudaMemcpy(a_row, plan->lv_a_row, (size_t)I.M, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && a_col && I.K) e = cudaMemcpy(a_col, plan->lv_a_col, (size_t)I.K, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && b_row && I.K) e = cudaMemcpy(b_row, plan->lv_b_row, (size_t)I.K, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && b_col && I.N) e = cudaMemcpy(b_col, plan->lv_b_col, (size_t)I.N, cudaMemcpyDeviceToHost);
+  cudaSetDevice(dev);
+  return e == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
+imq_status imq_plan_groups(const imq_plan_t* plan, imq_group* groups, int32_t max_groups, int32_t* n_out) {
+  if (!plan || !n_out || (max_groups > 0 && !groups)) return IMQ_ERR_ARG;
+  const int n = plan->info.n_groups;
+  for (int i = 0; i < n && i < max_groups; ++i) groups[i] = plan->groups[i];
+  *n_out = n;
+  return IMQ_OK;
+}
+
+imq_status imq_plan_destroy(imq_plan_t* plan) {
+  if (!plan) return IMQ_OK;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaSetDevice(plan->device);
+  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  if (plan->dev_block) e1 = cudaFreeAsync(plan->dev_block, 0);
+  if (plan->dev_block2) e2 = cudaFreeAsync(plan->dev_block2, 0);
+  cudaSetDevice(dev);
+  free(plan->host_tables);
+  delete plan;
+  return (e1 == cudaSuccess && e2 == cudaSuccess) ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
+imq_status imq_unpack(const imq_plan_t* plan, const void* A, const void* B, int8_t* A_unp, int8_t* B_unp_t,
+                      imq_stream_t stream) {
+  if (!plan) return IMQ_ERR_ARG;
+  const imq_plan_info& I = plan->info;
+  if (I.K_unp > 0 && ((I.M_unp > 0 && !A_unp) || (I.N_unp > 0 && !B_unp_t))) return IMQ_ERR_ARG;
+  if ((I.M > 0 && I.K > 0 && !A) || (I.K > 0 && I.N > 0 && !B)) return IMQ_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(A_unp) & 15) || (reinterpret_cast<uintptr_t>(B_unp_t) & 15)) return IMQ_ERR_ARG;
+  return imq::launch_unpack(plan, A, B, A_unp, B_unp_t, reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_gemm_unpacked(const imq_plan_t* plan, const int8_t* A_unp, const int8_t* B_unp_t, const float* deltaA,
+                             imq_gran gA, const float* deltaB, imq_gran gB, void* Cint, imq_dtype ct, int64_t ldc,
+                             float* Cf, int64_t ldcf, imq_stream_t stream) {
+  if (!plan) return IMQ_ERR_ARG;
+  return imq::launch_gemm(plan, A_unp, B_unp_t, deltaA, gA, deltaB, gB, Cint, ct, ldc, Cf, ldcf,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_unpacked_gemm(const imq_plan_t* plan, const void* A, const void* B, const float* deltaA, imq_gran gA,
+                             const float* deltaB, imq_gran gB, void* Cint, imq_dtype ct, int64_t ldc, float* Cf,
+                             int64_t ldcf, void* workspace, size_t workspace_bytes, imq_stream_t stream) {
+  if (!plan) return IMQ_ERR_ARG;
+  const imq_plan_info& I = plan->info;
+  if (workspace_bytes < I.workspace_bytes) return IMQ_ERR_BUFFER;
+  if (I.workspace_bytes > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 1023))) return IMQ_ERR_ARG;
+  // argument checks of the GEMM first, so a bad call launches nothing
+  if (!Cint && !Cf) return IMQ_ERR_ARG;
+  if (Cint && ct == IMQ_I32 && I.acc_bits > 32) return IMQ_ERR_RANGE;
+  int8_t* Au = static_cast<int8_t*>(workspace);
+  const size_t a_bytes = ((size_t)(I.M_unp * I.K_unp) + 1023) / 1024 * 1024;
+  int8_t* Bu = Au ? Au + a_bytes : nullptr;
+  imq_status s = imq_unpack(plan, A, B, Au, Bu, stream);
+  if (s != IMQ_OK) return s;
+  return imq_gemm_unpacked(plan, Au, Bu, deltaA, gA, deltaB, gB, Cint, ct, ldc, Cf, ldcf, stream);
+}
+
+imq_status imq_device_status(imq_stream_t stream, int32_t clear) {
+  DeviceState* ds;
+  imq_status s = imq::device_state(&ds);
+  if (s != IMQ_OK) return s;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  IMQ_CUDA_TRY(cudaMemcpyAsync(&v, ds->status, 4, cudaMemcpyDeviceToHost, st));
+  IMQ_CUDA_TRY(cudaStreamSynchronize(st));
+  if (clear) {
+    IMQ_CUDA_TRY(cudaMemsetAsync(ds->status, 0, 4, st));
+    IMQ_CUDA_TRY(cudaStreamSynchronize(st));
+  }
+  return (imq_status)v;
+}
+
+const char* imq_status_str(imq_status s) {
+  switch (s) {
+    case IMQ_OK: return "ok";
+    case IMQ_ERR_ARG: return "invalid argument";
+    case IMQ_ERR_NONFINITE: return "non-finite input";
+    case IMQ_ERR_RANGE: return "integer range exceeded";
+    case IMQ_ERR_BUFFER: return "buffer too small";
+    case IMQ_ERR_TIMEOUT: return "bounded wait timed out in a kernel";
+    case IMQ_ERR_CUDA: return "CUDA runtime error";
+    case IMQ_ERR_UNSUPPORTED: return "unsupported input";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,93 @@
+// internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "imq.h"
+
+namespace imq {
+
+constexpr int kMaxSeq = IMQ_MAX_GROUPS;
+
+// Per-device state owned by the library: the status word address and small scratch buffers.
+struct DeviceState {
+  int32_t* status = nullptr;   // device address of the status word of this device
+  void* scratch = nullptr;     // per-tensor quantiser scratch (allocated on first use)
+  int num_sms = 0;
+  bool init = false;
+};
+imq_status device_state(DeviceState** out);
+
+// Percentile + RTN quantisation (rtn.cu).
+imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                               imq_gran g, double p, int32_t beta, void* Xint, imq_dtype it,
+                               int64_t ldq, float* delta, float* qval, int32_t* rowmax,
+                               int32_t* colmax, cudaStream_t stream);
+
+// Line maxima of an integer matrix (plan.cu): logical rows and columns of a stored matrix.
+imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t cols, int64_t ld,
+                           int32_t* rowmax, int32_t* colmax, cudaStream_t stream);
+
+}  // namespace imq
+
+// The plan object (opaque in the public header).
+struct imq_plan {
+  imq_plan_info info;
+  int device;
+  // inputs the plan was made from
+  const void* A;
+  const void* B;
+  imq_dtype it;
+  int32_t transA, transB;
+  int64_t lda, ldb;
+  // one device allocation holding every array below
+  void* dev_block;   // stage 1: line maxima, levels, summary
+  void* dev_block2;  // stage 2: index maps
+  size_t dev_bytes;
+  void* host_tables; // segment and class tables copied to the device (kept until destroy)
+  int32_t* max_a_row;
+  int32_t* max_a_col;
+  int32_t* max_b_row;
+  int32_t* max_b_col;
+  int8_t* lv_a_row;
+  int8_t* lv_a_col;
+  int8_t* lv_b_row;
+  int8_t* lv_b_col;
+  int32_t* tK;      // [K_unp] source inner index, -1 on padding
+  int8_t* lAk;      // [K_unp] digit level of A at that inner position
+  int8_t* lBk;      // [K_unp] digit level of B
+  int32_t* posA;    // [M] first unpacked row of each source row (A OUTER)
+  int32_t* srcA;    // [M_unp] source row of each unpacked row, -1 unused (A OUTER)
+  int32_t* grpA_L;  // [M_unp / IMQ_A_GROUP] level of each row group
+  int32_t* grpA_n;  // [...] number of source rows in the group
+  int32_t* posB;    // [N]
+  int32_t* srcB;    // [N_unp]
+  int32_t* grpB_L;  // [N_unp / IMQ_B_GROUP]
+  int32_t* grpB_n;
+  int64_t n_grp_a, n_grp_b;
+  imq_group groups[IMQ_MAX_GROUPS];
+  // GEMM schedule over the groups (see gemm.cu)
+  int32_t n_slots;
+  int32_t seq_len;
+  int32_t seq_group[imq::kMaxSeq];
+  int32_t seq_slot[imq::kMaxSeq];
+  int32_t seq_rescale[imq::kMaxSeq];  // left shift applied to the slot before this group, -1: first
+  int32_t slot_shift[2];              // final left shift of each slot
+  int32_t wide_stage;                 // stage the accumulators as int64 in the epilogue
+};
+
+namespace imq {
+imq_status launch_unpack(const imq_plan_t* pl, const void* A, const void* B, int8_t* Au, int8_t* Bu,
+                         cudaStream_t stream);
+imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu, const float* dA,
+                       imq_gran gA, const float* dB, imq_gran gB, void* C, imq_dtype ct,
+                       int64_t ldc, float* Cf, int64_t ldcf, cudaStream_t stream);
+}  // namespace imq
+
+#define IMQ_CUDA_TRY(expr)                                    \
+  do {                                                        \
+    cudaError_t e_ = (expr);                                  \
+    if (e_ != cudaSuccess) return IMQ_ERR_CUDA;               \
+  } while (0)

@@ -1,0 +1,652 @@
+// plan.cu -- the unpack plan: line levels, outlier counts, per-matrix direction and layout maps.
+//
+// Method: "IM-Unpack: Training and Inference with Arbitrarily Low Precision Integers" (atlas.scime.ai
+// summary), "Approach": rows or columns holding out-of-bound entries are unpacked, the choice made per
+// matrix from outlier counts; measured-effects table: Mix against fixed row/col strategies, compared by
+// unpack ratio.  The rules (levels, expansion factors, Mix tie-breaks, ratio, layout) are documented in
+// include/imq.h.
+//
+// Device work, in stream order:
+//   k_line_max     max |v| of every logical line, unless the caller passes the quantiser's side outputs
+//   k_levels       int8 level of every line plus a summary: level sums, lines with level > 1, level
+//                  histograms, the joint histogram of (level of A column t, level of B row t), and the
+//                  exact 128-bit bound sum_t max|A[:,t]| * max|B[t,:]|
+//   -- the summary (a few KB) is read back; the host fixes directions, groups and sizes --
+//   k_inner_map    one CTA per (lA, lB) segment: stream compaction of the inner indices t it holds
+//   k_outer_map    one CTA per level class: stable compaction of the lines of that level into groups
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace imq {
+namespace {
+
+constexpr int kLv = 33;  // levels 1..32
+
+struct Summary {
+  unsigned long long sum[4];
+  unsigned long long oor[4];
+  unsigned int lmax[4];
+  unsigned int hist[4][kLv];
+  unsigned int joint[kLv][kLv];
+  unsigned long long bound_lo, bound_hi;
+  int32_t status;  // copy of the device status word taken in stream order
+  int32_t pad_;
+};
+
+// ------------------------------------------------------------------------------------------------
+// line maxima of a stored integer matrix
+// ------------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_line_max(const T* __restrict__ X, int64_t rows, int64_t cols,
+                                                  int64_t ld, int32_t* __restrict__ rowmax,
+                                                  int32_t* __restrict__ colmax, int smem_cols) {
+  extern __shared__ uint32_t cmax[];
+  __shared__ uint32_t red[8];
+  const int tid = threadIdx.x;
+  if (smem_cols)
+    for (int64_t c = tid; c < cols; c += 256) cmax[c] = 0;
+  __syncthreads();
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    uint32_t m = 0;
+    for (int64_t c = tid; c < cols; c += 256) {
+      const int64_t v = X[r * ld + c];
+      const uint32_t a = (uint32_t)(v < 0 ? -v : v);
+      m = max(m, a);
+      if (colmax) {
+        if (smem_cols) cmax[c] = max(cmax[c], a);
+        else if (a) atomicMax(colmax + c, (int32_t)a);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0 && rowmax) {
+      uint32_t r2 = 0;
+      for (int w = 0; w < 8; ++w) r2 = max(r2, red[w]);
+      rowmax[r] = (int32_t)r2;
+    }
+    __syncthreads();
+  }
+  if (colmax && smem_cols)
+    for (int64_t c = tid; c < cols; c += 256)
+      if (cmax[c]) atomicMax(colmax + c, (int32_t)cmax[c]);
+}
+
+// ------------------------------------------------------------------------------------------------
+// levels and summary.  Vectors: 0 = A rows (M), 1 = A cols (K), 2 = B rows (K), 3 = B cols (N).
+// ------------------------------------------------------------------------------------------------
+struct LevelArgs {
+  const int32_t* mx[4];
+  int8_t* lv[4];
+  int64_t n[4];
+  int32_t bm1;
+  Summary* sum;
+};
+
+__global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
+  __shared__ unsigned int hist[4][kLv];
+  __shared__ unsigned int joint[kLv][kLv];
+  __shared__ unsigned long long ssum[4], soor[4];
+  __shared__ unsigned int slmax[4];
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 4 * kLv; i += 256) (&hist[0][0])[i] = 0;
+  for (int i = tid; i < kLv * kLv; i += 256) (&joint[0][0])[i] = 0;
+  if (tid < 4) {
+    ssum[tid] = 0;
+    soor[tid] = 0;
+    slmax[tid] = 0;
+  }
+  __syncthreads();
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  unsigned long long bsum[4] = {0, 0, 0, 0}, boor[4] = {0, 0, 0, 0};
+  unsigned int blmax[4] = {0, 0, 0, 0};
+  unsigned __int128 bound = 0;
+  for (int v = 0; v < 4; ++v) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + tid; i < a.n[v]; i += stride) {
+      const uint32_t m = (uint32_t)a.mx[v][i];
+      const int L = level_of(m, a.bm1);
+      a.lv[v][i] = (int8_t)L;
+      bsum[v] += (unsigned)L;
+      boor[v] += (L > 1);
+      blmax[v] = max(blmax[v], (unsigned)L);
+      atomicAdd(&hist[v][L], 1u);
+      if (v == 1) {
+        const uint32_t mb = (uint32_t)a.mx[2][i];
+        atomicAdd(&joint[L][level_of(mb, a.bm1)], 1u);
+        bound += (unsigned __int128)((unsigned long long)m * (unsigned long long)mb);
+      }
+    }
+  }
+  for (int v = 0; v < 4; ++v) {
+    if (bsum[v]) atomicAdd(&ssum[v], bsum[v]);
+    if (boor[v]) atomicAdd(&soor[v], boor[v]);
+    if (blmax[v]) atomicMax(&slmax[v], blmax[v]);
+  }
+  if (bound) {
+    const unsigned long long lo = (unsigned long long)bound, hi = (unsigned long long)(bound >> 64);
+    const unsigned long long old = atomicAdd(&a.sum->bound_lo, lo);
+    const unsigned long long carry = (old + lo < old) ? 1ull : 0ull;
+    if (hi + carry) atomicAdd(&a.sum->bound_hi, hi + carry);
+  }
+  __syncthreads();
+  if (tid < 4) {
+    if (ssum[tid]) atomicAdd(&a.sum->sum[tid], ssum[tid]);
+    if (soor[tid]) atomicAdd(&a.sum->oor[tid], soor[tid]);
+    if (slmax[tid]) atomicMax(&a.sum->lmax[tid], slmax[tid]);
+  }
+  for (int i = tid; i < 4 * kLv; i += 256)
+    if ((&hist[0][0])[i]) atomicAdd(&a.sum->hist[0][0] + i, (&hist[0][0])[i]);
+  for (int i = tid; i < kLv * kLv; i += 256)
+    if ((&joint[0][0])[i]) atomicAdd(&a.sum->joint[0][0] + i, (&joint[0][0])[i]);
+}
+
+// ------------------------------------------------------------------------------------------------
+// maps
+// ------------------------------------------------------------------------------------------------
+// Block-wide exclusive scan of a 0/1 predicate (1024 threads); returns the rank and the block total.
+__device__ __forceinline__ int block_rank(int pred, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned ball = __ballot_sync(0xffffffffu, pred);
+  const int in_warp = __popc(ball & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[warp] = __popc(ball);
+  __syncthreads();
+  if (warp == 0) {
+    const int v = warp_tot[lane];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    warp_tot[lane] = incl - v;
+    if (lane == 31) *total = incl;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + in_warp;
+  return r;
+}
+
+struct InnerSeg {
+  int32_t la, lb;
+  int64_t off;
+};
+
+__global__ void __launch_bounds__(1024) k_inner_map(const InnerSeg* __restrict__ segs, const int8_t* __restrict__ lva,
+                                                    const int8_t* __restrict__ lvb, int a_inner, int b_inner,
+                                                    int64_t K, int32_t* __restrict__ tK,
+                                                    int8_t* __restrict__ lAk, int8_t* __restrict__ lBk) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const InnerSeg sg = segs[blockIdx.x];
+  int64_t base = sg.off;
+  for (int64_t t0 = 0; t0 < K; t0 += 1024) {
+    const int64_t t = t0 + threadIdx.x;
+    int pred = 0;
+    if (t < K) {
+      const int la = a_inner ? lva[t] : 1;
+      const int lb = b_inner ? lvb[t] : 1;
+      pred = (la > sg.la) && (lb > sg.lb);
+    }
+    const int r = block_rank(pred, warp_tot, &total);
+    if (pred) {
+      tK[base + r] = (int32_t)t;
+      lAk[base + r] = (int8_t)sg.la;
+      lBk[base + r] = (int8_t)sg.lb;
+    }
+    __syncthreads();
+    base += total;
+    __syncthreads();
+  }
+}
+
+struct OuterClass {
+  int32_t L;
+  int32_t per;      // source lines per group
+  int64_t grp0;     // first group of this class
+  int64_t count;    // lines of this level
+};
+
+__global__ void __launch_bounds__(1024) k_outer_map(const OuterClass* __restrict__ cls, const int8_t* __restrict__ lv,
+                                                    int64_t n, int G, int32_t* __restrict__ pos,
+                                                    int32_t* __restrict__ src, int32_t* __restrict__ grpL,
+                                                    int32_t* __restrict__ grpN) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const OuterClass c = cls[blockIdx.x];
+  const int64_t ngrp = (c.count + c.per - 1) / c.per;
+  for (int64_t g = threadIdx.x; g < ngrp; g += blockDim.x) {
+    grpL[c.grp0 + g] = c.L;
+    grpN[c.grp0 + g] = (int32_t)(g < ngrp - 1 ? c.per : c.count - (ngrp - 1) * c.per);
+  }
+  int64_t rank0 = 0;
+  for (int64_t i0 = 0; i0 < n; i0 += 1024) {
+    const int64_t i = i0 + threadIdx.x;
+    const int pred = (i < n) && (lv[i] == c.L);
+    const int r = block_rank(pred, warp_tot, &total);
+    if (pred) {
+      const int64_t rank = rank0 + r;
+      const int64_t p = (c.grp0 + rank / c.per) * G + (rank % c.per) * c.L;
+      pos[i] = (int32_t)p;
+      for (int l = 0; l < c.L; ++l) src[p + l] = (int32_t)i;
+    }
+    __syncthreads();
+    rank0 += total;
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------------
+struct Pinned {
+  Summary* sum = nullptr;
+  std::mutex mu;
+};
+Pinned g_pinned[64];
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t cols, int64_t ld,
+                           int32_t* rowmax, int32_t* colmax, cudaStream_t st) {
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  if (rows == 0 || cols == 0) return IMQ_OK;
+  if (rowmax) IMQ_CUDA_TRY(cudaMemsetAsync(rowmax, 0, (size_t)rows * 4, st));
+  if (colmax) IMQ_CUDA_TRY(cudaMemsetAsync(colmax, 0, (size_t)cols * 4, st));
+  const int smem_cols = (colmax && cols <= 32768) ? 1 : 0;
+  const size_t smem = smem_cols ? (size_t)cols * 4 : 0;
+  const int64_t grid = rows < (int64_t)ds->num_sms * 4 ? rows : (int64_t)ds->num_sms * 4;
+  if (it == IMQ_I16) {
+    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_line_max<int16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_line_max<int16_t><<<(unsigned)grid, 256, smem, st>>>(static_cast<const int16_t*>(X), rows, cols, ld,
+                                                           rowmax, colmax, smem_cols);
+  } else {
+    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_line_max<int32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_line_max<int32_t><<<(unsigned)grid, 256, smem, st>>>(static_cast<const int32_t*>(X), rows, cols, ld,
+                                                           rowmax, colmax, smem_cols);
+  }
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
+// Builds a plan; see imq_plan in include/imq.h.
+imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                      int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
+                      imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                      const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out,
+                      cudaStream_t st) {
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  int dev;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  Pinned& pin = g_pinned[dev & 63];
+  std::lock_guard<std::mutex> lock(pin.mu);
+  if (!pin.sum) IMQ_CUDA_TRY(cudaMallocHost(&pin.sum, sizeof(Summary)));
+
+  imq_plan_t* pl = new imq_plan_t;
+  memset(pl, 0, sizeof(*pl));
+  const size_t tables_bytes = sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv;
+  pl->host_tables = malloc(tables_bytes);
+  if (!pl->host_tables) {
+    delete pl;
+    return IMQ_ERR_CUDA;
+  }
+  InnerSeg* hsegs = static_cast<InnerSeg*>(pl->host_tables);
+  OuterClass* hcls = reinterpret_cast<OuterClass*>(hsegs + kLv * kLv);
+  pl->device = dev;
+  pl->A = A;
+  pl->B = B;
+  pl->it = it;
+  pl->transA = transA;
+  pl->transB = transB;
+  pl->lda = lda;
+  pl->ldb = ldb;
+  imq_plan_info& I = pl->info;
+  I.b = b;
+  I.strategy = strategy;
+  I.M = M;
+  I.K = K;
+  I.N = N;
+
+  // ---- stage 1: maxima, levels, summary ----
+  const int64_t nvec[4] = {M, K, K, N};
+  size_t off = 0;
+  size_t o_max[4], o_lv[4];
+  for (int v = 0; v < 4; ++v) { o_max[v] = off; off = align_up(off + (size_t)nvec[v] * 4, 256); }
+  for (int v = 0; v < 4; ++v) { o_lv[v] = off; off = align_up(off + (size_t)nvec[v], 256); }
+  const size_t o_sum = off;
+  off = align_up(off + sizeof(Summary), 256);
+  const size_t o_segs = off;
+  off = align_up(off + sizeof(InnerSeg) * kLv * kLv, 256);
+  const size_t o_cls = off;
+  off = align_up(off + sizeof(OuterClass) * 2 * kLv, 256);
+  const size_t stage1 = off;
+  char* blk1 = nullptr;
+  if (cudaMallocAsync((void**)&blk1, stage1, st) != cudaSuccess) {
+    free(pl->host_tables);
+    delete pl;
+    return IMQ_ERR_CUDA;
+  }
+  pl->dev_block = blk1;
+  pl->dev_bytes = stage1;
+  int32_t* mx[4];
+  for (int v = 0; v < 4; ++v) mx[v] = reinterpret_cast<int32_t*>(blk1 + o_max[v]);
+  pl->max_a_row = mx[0];
+  pl->max_a_col = mx[1];
+  pl->max_b_row = mx[2];
+  pl->max_b_col = mx[3];
+  pl->lv_a_row = reinterpret_cast<int8_t*>(blk1 + o_lv[0]);
+  pl->lv_a_col = reinterpret_cast<int8_t*>(blk1 + o_lv[1]);
+  pl->lv_b_row = reinterpret_cast<int8_t*>(blk1 + o_lv[2]);
+  pl->lv_b_col = reinterpret_cast<int8_t*>(blk1 + o_lv[3]);
+  Summary* dsum = reinterpret_cast<Summary*>(blk1 + o_sum);
+
+  auto fail = [&](imq_status e) {
+    cudaFreeAsync(pl->dev_block, st);
+    if (pl->dev_block2) cudaFreeAsync(pl->dev_block2, st);
+    free(pl->host_tables);
+    delete pl;
+    return e;
+  };
+
+  const bool have_max = a_rowmax && a_colmax && b_rowmax && b_colmax;
+  if (have_max) {
+    const int32_t* given[4] = {a_rowmax, a_colmax, b_rowmax, b_colmax};
+    for (int v = 0; v < 4; ++v)
+      if (nvec[v] && cudaMemcpyAsync(mx[v], given[v], (size_t)nvec[v] * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return fail(IMQ_ERR_CUDA);
+  } else {
+    // A stored M x K (or K x M when transposed); B stored K x N (or N x K)
+    imq_status e = transA ? launch_line_max(A, it, K, M, lda, mx[1], mx[0], st)
+                          : launch_line_max(A, it, M, K, lda, mx[0], mx[1], st);
+    if (e != IMQ_OK) return fail(e);
+    e = transB ? launch_line_max(B, it, N, K, ldb, mx[3], mx[2], st)
+               : launch_line_max(B, it, K, N, ldb, mx[2], mx[3], st);
+    if (e != IMQ_OK) return fail(e);
+    if (M == 0 && K > 0 && cudaMemsetAsync(mx[1], 0, (size_t)K * 4, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+    if (N == 0 && K > 0 && cudaMemsetAsync(mx[2], 0, (size_t)K * 4, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+    if (K == 0) {
+      if (M && cudaMemsetAsync(mx[0], 0, (size_t)M * 4, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+      if (N && cudaMemsetAsync(mx[3], 0, (size_t)N * 4, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+    }
+  }
+  if (cudaMemsetAsync(dsum, 0, sizeof(Summary), st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  LevelArgs la;
+  for (int v = 0; v < 4; ++v) {
+    la.mx[v] = mx[v];
+    la.n[v] = nvec[v];
+  }
+  la.lv[0] = pl->lv_a_row;
+  la.lv[1] = pl->lv_a_col;
+  la.lv[2] = pl->lv_b_row;
+  la.lv[3] = pl->lv_b_col;
+  la.bm1 = b - 1;
+  la.sum = dsum;
+  {
+    const int64_t nmax = (M > K ? M : K) > N ? (M > K ? M : K) : N;
+    int64_t grid = (nmax + 255) / 256;
+    if (grid > ds->num_sms * 2) grid = ds->num_sms * 2;
+    if (grid < 1) grid = 1;
+    k_levels<<<(unsigned)grid, 256, 0, st>>>(la);
+  }
+  if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  if (cudaMemcpyAsync(&dsum->status, ds->status, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(pin.sum, dsum, sizeof(Summary), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return fail(IMQ_ERR_CUDA);
+  const Summary S = *pin.sum;
+  // a pending kernel error (e.g. a non-finite quantiser input) is reported before planning
+  if (S.status != IMQ_OK) return fail((imq_status)S.status);
+
+  // ---- host decisions ----
+  for (int v = 0; v < 4; ++v) if (S.lmax[v] > 31) return fail(IMQ_ERR_UNSUPPORTED);
+  const int64_t lmax[4] = {nvec[0] ? S.lmax[0] : 1, nvec[1] ? S.lmax[1] : 1, nvec[2] ? S.lmax[2] : 1,
+                           nvec[3] ? S.lmax[3] : 1};
+  I.lmax_a_row = (int32_t)lmax[0];
+  I.lmax_a_col = (int32_t)lmax[1];
+  I.lmax_b_row = (int32_t)lmax[2];
+  I.lmax_b_col = (int32_t)lmax[3];
+  I.sum_l_a_row = (int64_t)S.sum[0];
+  I.sum_l_a_col = (int64_t)S.sum[1];
+  I.sum_l_b_row = (int64_t)S.sum[2];
+  I.sum_l_b_col = (int64_t)S.sum[3];
+  I.oor_lines_a_row = (int64_t)S.oor[0];
+  I.oor_lines_a_col = (int64_t)S.oor[1];
+  I.oor_lines_b_row = (int64_t)S.oor[2];
+  I.oor_lines_b_col = (int64_t)S.oor[3];
+
+  int da, db;
+  if (strategy == IMQ_MIX) {
+    if (S.oor[0] == 0 && S.oor[1] == 0) {
+      da = IMQ_DIR_NONE;
+    } else {
+      const __int128 row_side = (__int128)S.sum[0] * K, col_side = (__int128)S.sum[1] * M;
+      if (row_side != col_side) da = row_side < col_side ? IMQ_DIR_OUTER : IMQ_DIR_INNER;
+      else if (S.oor[0] != S.oor[1]) da = S.oor[0] < S.oor[1] ? IMQ_DIR_OUTER : IMQ_DIR_INNER;
+      else da = IMQ_DIR_OUTER;
+    }
+    if (S.oor[2] == 0 && S.oor[3] == 0) {
+      db = IMQ_DIR_NONE;
+    } else {
+      const __int128 row_side = (__int128)S.sum[2] * N, col_side = (__int128)S.sum[3] * K;
+      if (row_side != col_side) db = row_side < col_side ? IMQ_DIR_INNER : IMQ_DIR_OUTER;
+      else if (S.oor[2] != S.oor[3]) db = S.oor[2] < S.oor[3] ? IMQ_DIR_INNER : IMQ_DIR_OUTER;
+      else db = IMQ_DIR_INNER;
+    }
+  } else {
+    da = (strategy == IMQ_ROW_ROW || strategy == IMQ_ROW_COL) ? IMQ_DIR_OUTER : IMQ_DIR_INNER;
+    db = (strategy == IMQ_ROW_ROW || strategy == IMQ_COL_ROW) ? IMQ_DIR_INNER : IMQ_DIR_OUTER;
+  }
+  I.dir_a = da;
+  I.dir_b = db;
+  const bool a_outer = da == IMQ_DIR_OUTER, a_inner = da == IMQ_DIR_INNER;
+  const bool b_outer = db == IMQ_DIR_OUTER, b_inner = db == IMQ_DIR_INNER;
+
+  // inner segments from the joint level histogram
+  const int maxla = a_inner ? (int)lmax[1] : 1;
+  const int maxlb = b_inner ? (int)lmax[2] : 1;
+  auto seg_len = [&](int sa, int sb) {
+    int64_t n = 0;
+    for (int x = 1; x < kLv; ++x)
+      for (int y = 1; y < kLv; ++y) {
+        const int ea = a_inner ? x : 1, eb = b_inner ? y : 1;
+        if (ea > sa && eb > sb) n += S.joint[x][y];
+      }
+    return n;
+  };
+  int nseg = 0;
+  int64_t koff = 0, keff = 0;
+  int ng = 0;
+  for (int e = 0; e <= maxla + maxlb - 2; ++e) {
+    int64_t glen = 0;
+    for (int sa = 0; sa < maxla; ++sa) {
+      const int sb = e - sa;
+      if (sb < 0 || sb >= maxlb) continue;
+      const int64_t n = seg_len(sa, sb);
+      if (n == 0) continue;
+      hsegs[nseg].la = sa;
+      hsegs[nseg].lb = sb;
+      hsegs[nseg].off = koff + glen;
+      ++nseg;
+      glen += n;
+    }
+    if (glen == 0) continue;
+    if (ng >= IMQ_MAX_GROUPS) return fail(IMQ_ERR_UNSUPPORTED);
+    pl->groups[ng].e = e;
+    pl->groups[ng].k_offset = koff;
+    pl->groups[ng].k_len = glen;
+    pl->groups[ng].k_len_padded = (glen + IMQ_INNER_PAD - 1) / IMQ_INNER_PAD * IMQ_INNER_PAD;
+    koff += pl->groups[ng].k_len_padded;
+    keff += glen;
+    ++ng;
+  }
+  I.n_groups = ng;
+  I.K_unp = koff;
+  I.K_eff = keff;
+
+  // outer sizes
+  int ncls = 0;
+  auto outer_classes = [&](int v, int G, int64_t* groups_out) {
+    int64_t grp = 0;
+    for (int L = 1; L <= (int)lmax[v]; ++L) {
+      const int64_t cnt = S.hist[v][L];
+      if (cnt == 0) continue;
+      const int per = G / L;
+      hcls[ncls].L = L;
+      hcls[ncls].per = per;
+      hcls[ncls].grp0 = grp;
+      hcls[ncls].count = cnt;
+      ++ncls;
+      grp += (cnt + per - 1) / per;
+    }
+    *groups_out = grp;
+  };
+  int cls_a0 = 0, cls_a1 = 0, cls_b0 = 0, cls_b1 = 0;
+  if (a_outer) {
+    cls_a0 = ncls;
+    outer_classes(0, IMQ_A_GROUP, &pl->n_grp_a);
+    cls_a1 = ncls;
+    I.M_unp = pl->n_grp_a * IMQ_A_GROUP;
+    I.M_eff = (int64_t)S.sum[0];
+  } else {
+    I.M_unp = M;
+    I.M_eff = M;
+  }
+  if (b_outer) {
+    cls_b0 = ncls;
+    outer_classes(3, IMQ_B_GROUP, &pl->n_grp_b);
+    cls_b1 = ncls;
+    I.N_unp = pl->n_grp_b * IMQ_B_GROUP;
+    I.N_eff = (int64_t)S.sum[3];
+  } else {
+    I.N_unp = N;
+    I.N_eff = N;
+  }
+  I.ratio = (M > 0 && N > 0 && K > 0)
+                ? ((double)I.M_eff / (double)M) * ((double)I.N_eff / (double)N) * ((double)I.K_eff / (double)K)
+                : 1.0;
+
+  // bound and accumulator schedule
+  const unsigned __int128 bound = ((unsigned __int128)S.bound_hi << 64) | S.bound_lo;
+  I.bound = (double)bound;
+  const unsigned __int128 two31 = (unsigned __int128)1 << 31;
+  if (bound >= ((unsigned __int128)1 << 63)) return fail(IMQ_ERR_UNSUPPORTED);  // C itself may leave int64
+  I.acc_bits = bound < two31 ? 32 : 64;
+  const int bm1 = b - 1;
+  const int64_t R1 = ((int64_t)1 << bm1) - 1;
+  pl->n_slots = 1;
+  pl->seq_len = 0;
+  pl->wide_stage = 0;
+  pl->slot_shift[0] = pl->slot_shift[1] = 0;
+  if (ng > 0) {
+    if (bound < two31 || ng == 1) {
+      if (bound >= two31 && (unsigned __int128)pl->groups[0].k_len * (unsigned __int128)(R1 * R1) >= two31)
+        return fail(IMQ_ERR_UNSUPPORTED);
+      for (int g = ng - 1; g >= 0; --g) {
+        const int i = pl->seq_len++;
+        pl->seq_group[i] = g;
+        pl->seq_slot[i] = 0;
+        pl->seq_rescale[i] = (g == ng - 1) ? -1 : (pl->groups[g + 1].e - pl->groups[g].e) * bm1;
+      }
+      pl->slot_shift[0] = pl->groups[0].e * bm1;
+    } else {
+      const int e1 = pl->groups[1].e;
+      const int sh1 = e1 * bm1;
+      const bool fits = (sh1 + 31 >= 127) || (bound < (two31 << sh1));
+      if (!fits) return fail(IMQ_ERR_UNSUPPORTED);
+      if ((unsigned __int128)pl->groups[0].k_len * (unsigned __int128)(R1 * R1) >= two31)
+        return fail(IMQ_ERR_UNSUPPORTED);
+      for (int g = ng - 1; g >= 1; --g) {
+        const int i = pl->seq_len++;
+        pl->seq_group[i] = g;
+        pl->seq_slot[i] = 1;
+        pl->seq_rescale[i] = (g == ng - 1) ? -1 : (pl->groups[g + 1].e - pl->groups[g].e) * bm1;
+      }
+      const int i = pl->seq_len++;
+      pl->seq_group[i] = 0;
+      pl->seq_slot[i] = 0;
+      pl->seq_rescale[i] = -1;
+      pl->n_slots = 2;
+      pl->slot_shift[0] = pl->groups[0].e * bm1;
+      pl->slot_shift[1] = sh1;
+      pl->wide_stage = 1;
+    }
+  }
+  I.workspace_bytes = align_up((size_t)(I.M_unp * I.K_unp), 1024) + align_up((size_t)(I.N_unp * I.K_unp), 1024);
+
+  // ---- stage 2: maps ----
+  size_t off2 = 0;
+  const size_t o_tK = off2; off2 = align_up(off2 + (size_t)I.K_unp * 4, 256);
+  const size_t o_lAk = off2; off2 = align_up(off2 + (size_t)I.K_unp, 256);
+  const size_t o_lBk = off2; off2 = align_up(off2 + (size_t)I.K_unp, 256);
+  size_t o_posA = 0, o_srcA = 0, o_gLA = 0, o_gNA = 0, o_posB = 0, o_srcB = 0, o_gLB = 0, o_gNB = 0;
+  if (a_outer) {
+    o_posA = off2; off2 = align_up(off2 + (size_t)M * 4, 256);
+    o_srcA = off2; off2 = align_up(off2 + (size_t)I.M_unp * 4, 256);
+    o_gLA = off2; off2 = align_up(off2 + (size_t)pl->n_grp_a * 4, 256);
+    o_gNA = off2; off2 = align_up(off2 + (size_t)pl->n_grp_a * 4, 256);
+  }
+  if (b_outer) {
+    o_posB = off2; off2 = align_up(off2 + (size_t)N * 4, 256);
+    o_srcB = off2; off2 = align_up(off2 + (size_t)I.N_unp * 4, 256);
+    o_gLB = off2; off2 = align_up(off2 + (size_t)pl->n_grp_b * 4, 256);
+    o_gNB = off2; off2 = align_up(off2 + (size_t)pl->n_grp_b * 4, 256);
+  }
+  char* b2 = nullptr;
+  if (cudaMallocAsync((void**)&b2, off2 > 0 ? off2 : 256, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  pl->dev_block2 = b2;
+  pl->dev_bytes = stage1 + off2;
+  InnerSeg* dsegs = reinterpret_cast<InnerSeg*>(blk1 + o_segs);
+  OuterClass* dcls = reinterpret_cast<OuterClass*>(blk1 + o_cls);
+  pl->tK = reinterpret_cast<int32_t*>(b2 + o_tK);
+  pl->lAk = reinterpret_cast<int8_t*>(b2 + o_lAk);
+  pl->lBk = reinterpret_cast<int8_t*>(b2 + o_lBk);
+  if (a_outer) {
+    pl->posA = reinterpret_cast<int32_t*>(b2 + o_posA);
+    pl->srcA = reinterpret_cast<int32_t*>(b2 + o_srcA);
+    pl->grpA_L = reinterpret_cast<int32_t*>(b2 + o_gLA);
+    pl->grpA_n = reinterpret_cast<int32_t*>(b2 + o_gNA);
+  }
+  if (b_outer) {
+    pl->posB = reinterpret_cast<int32_t*>(b2 + o_posB);
+    pl->srcB = reinterpret_cast<int32_t*>(b2 + o_srcB);
+    pl->grpB_L = reinterpret_cast<int32_t*>(b2 + o_gLB);
+    pl->grpB_n = reinterpret_cast<int32_t*>(b2 + o_gNB);
+  }
+  if (I.K_unp) {
+    if (cudaMemsetAsync(pl->tK, 0xFF, (size_t)I.K_unp * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(pl->lAk, 0, (size_t)I.K_unp, st) != cudaSuccess ||
+        cudaMemsetAsync(pl->lBk, 0, (size_t)I.K_unp, st) != cudaSuccess)
+      return fail(IMQ_ERR_CUDA);
+  }
+  if (a_outer && I.M_unp && cudaMemsetAsync(pl->srcA, 0xFF, (size_t)I.M_unp * 4, st) != cudaSuccess)
+    return fail(IMQ_ERR_CUDA);
+  if (b_outer && I.N_unp && cudaMemsetAsync(pl->srcB, 0xFF, (size_t)I.N_unp * 4, st) != cudaSuccess)
+    return fail(IMQ_ERR_CUDA);
+  if (nseg > 0 || ncls > 0) {
+    if (cudaMemcpyAsync(dsegs, hsegs, sizeof(InnerSeg) * (nseg > 0 ? nseg : 1), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dcls, hcls, sizeof(OuterClass) * (ncls > 0 ? ncls : 1), cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return fail(IMQ_ERR_CUDA);
+  }
+  if (nseg > 0)
+    k_inner_map<<<nseg, 1024, 0, st>>>(dsegs, pl->lv_a_col, pl->lv_b_row, a_inner, b_inner, K, pl->tK, pl->lAk, pl->lBk);
+  if (a_outer && cls_a1 > cls_a0)
+    k_outer_map<<<cls_a1 - cls_a0, 1024, 0, st>>>(dcls + cls_a0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
+                                                  pl->grpA_L, pl->grpA_n);
+  if (b_outer && cls_b1 > cls_b0)
+    k_outer_map<<<cls_b1 - cls_b0, 1024, 0, st>>>(dcls + cls_b0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
+                                                  pl->grpB_L, pl->grpB_n);
+  if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  *out = pl;
+  return IMQ_OK;
+}
+
+}  // namespace imq

@@ -1,0 +1,235 @@
+"""GPU parity of every stage of the path against the CPU oracle, through the C ABI.
+
+Integer results (quantised values, levels, plan sizes, unpacked bytes, the product C) must be
+bit-exact; dequantised fp32 outputs within 1e-6 relative of the oracle's float64 value.  Sizes span
+several 128 x 256 GEMM tiles and ragged edges.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_common import (assert_f32_close, logical, plan_matches, slots_needed_unsupported,
+                              to_device)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def imq():
+    import bit_integer_gemm_b200 as m
+    assert torch.cuda.is_available(), "a GPU is required"
+    m.lib()
+    m.imq_device_status(clear=True)
+    return m
+
+
+# ------------------------------------------------------------------------------------------------
+# quantisation
+# ------------------------------------------------------------------------------------------------
+def _matrix(rng, shape, heavy=True):
+    x = rng.standard_normal(shape).astype(np.float32) * np.float32(rng.uniform(0.01, 10))
+    if heavy and x.size:
+        idx = rng.choice(x.size, max(1, x.size // 200), replace=False)
+        x.reshape(-1)[idx] *= np.float32(40)
+    return x
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("gran", [oracle.PER_TENSOR, oracle.PER_ROW, oracle.PER_COL])
+@pytest.mark.parametrize("shape", [(1, 1), (3, 5), (37, 129), (128, 4096), (257, 1000), (1000, 64)])
+@pytest.mark.parametrize("p,beta", [(0.95, 15), (1.0, 31), (0.5, 255)])
+def test_quantize_parity(imq, dtype, gran, shape, p, beta):
+    rng = np.random.default_rng(zlib.crc32(repr((dtype, gran, shape, p)).encode()))
+    x = _matrix(rng, shape)
+    st = workloads.Stored("x", workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x, dtype)
+    want_i, want_d, want_q = oracle.rtn_quantize(oracle.as_f32(st.data, dtype), gran, p, beta)
+    X = to_device(st)
+    for out in (torch.int16, torch.int32):
+        if out == torch.int16 and np.abs(want_i).max() > 32767:
+            continue
+        r = imq.imq_rtn_quantize(X, gran, p, beta, out_dtype=out)
+        torch.cuda.synchronize()
+        assert imq.imq_device_status() == imq.IMQ_OK
+        assert np.array_equal(r.xint.cpu().numpy().astype(np.int64), want_i)
+        assert np.array_equal(r.delta.cpu().numpy().view(np.uint32), want_d.view(np.uint32))
+        assert np.array_equal(r.qval.cpu().numpy().view(np.uint32), want_q.view(np.uint32))
+        assert np.array_equal(r.rowmax.cpu().numpy(), np.abs(want_i).max(axis=1))
+        assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0))
+
+
+def test_quantize_strided_input(imq):
+    rng = np.random.default_rng(5)
+    x = _matrix(rng, (70, 300))
+    bits = workloads.f32_to_bf16_bits(x)
+    full = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    X = full[:, 17:17 + 211]  # leading dimension 300, 211 columns, unaligned start
+    sub = oracle.bf16_bits_to_f32(np.ascontiguousarray(bits[:, 17:228]))
+    for gran in (oracle.PER_TENSOR, oracle.PER_ROW, oracle.PER_COL):
+        want_i, want_d, _ = oracle.rtn_quantize(sub, gran, 0.95, 15)
+        out = torch.zeros((70, 256), dtype=torch.int16, device="cuda")
+        r = imq.imq_rtn_quantize(X, gran, 0.95, 15, Xint=out[:, :211])
+        assert np.array_equal(r.xint.cpu().numpy().astype(np.int64), want_i)
+        assert np.array_equal(r.delta.cpu().numpy(), want_d)
+        assert not out[:, 211:].any()
+
+
+def test_quantize_errors(imq):
+    x = torch.ones((4, 64), device="cuda")
+    x[2, 7] = float("nan")
+    imq.imq_rtn_quantize(x, imq.IMQ_PER_ROW, 0.95, 15)
+    assert imq.imq_device_status(clear=True) == imq.IMQ_ERR_NONFINITE
+    y = torch.full((1, 1000), 1e-3, device="cuda")
+    y[0, 0] = 100.0  # 100 / 1e-3 * 15 = 1.5e6: fits int32, not int16
+    imq.imq_rtn_quantize(y, imq.IMQ_PER_TENSOR, 0.95, 15, out_dtype=torch.int16)
+    assert imq.imq_device_status(clear=True) == imq.IMQ_ERR_RANGE
+    r = imq.imq_rtn_quantize(y, imq.IMQ_PER_TENSOR, 0.95, 15, out_dtype=torch.int32)
+    assert imq.imq_device_status(clear=True) == imq.IMQ_OK and int(r.xint[0, 0]) == 1500000
+    for p, beta in ((0.0, 15), (1.5, 15), (0.95, 0)):
+        with pytest.raises(imq.ImqError) as e:
+            imq.imq_rtn_quantize(y, imq.IMQ_PER_TENSOR, p, beta)
+        assert e.value.status == imq.IMQ_ERR_ARG
+
+
+def test_quantize_empty(imq):
+    x = torch.empty((0, 5), device="cuda")
+    r = imq.imq_rtn_quantize(x, imq.IMQ_PER_COL, 0.95, 15)
+    assert np.array_equal(r.delta.cpu().numpy(), np.ones(5, np.float32))
+
+
+# ------------------------------------------------------------------------------------------------
+# plan, unpack, GEMM on random integer matrices
+# ------------------------------------------------------------------------------------------------
+def _run_path(imq, A, B, b, strategy, transA, transB, dtype=torch.int16, check_unpack=True):
+    """A, B: logical int64 numpy matrices.  Runs plan -> unpack -> GEMM on the GPU and checks each
+    stage against the oracle."""
+    M, K = A.shape
+    N = B.shape[1]
+    pl = oracle.plan(A, B, b, strategy)
+    A_st = np.ascontiguousarray(A.T if transA else A)
+    B_st = np.ascontiguousarray(B.T if transB else B)
+    npdt = np.int16 if dtype == torch.int16 else np.int32
+    Ad = torch.from_numpy(A_st.astype(npdt)).cuda()
+    Bd = torch.from_numpy(B_st.astype(npdt)).cuda()
+    if slots_needed_unsupported(pl):
+        with pytest.raises(imq.ImqError) as e:
+            imq.imq_plan(Ad, Bd, b, strategy, transA, transB)
+        assert e.value.status == imq.IMQ_ERR_UNSUPPORTED
+        return None
+    plan = imq.imq_plan(Ad, Bd, b, strategy, transA, transB)
+    plan_matches(plan.info, pl)
+    lv = plan.levels()
+    for k in ("a_row", "a_col", "b_row", "b_col"):
+        assert np.array_equal(lv[k].astype(np.int32), pl.levels[k]), k
+    assert plan.groups() == [tuple(g) for g in pl.groups]
+    Au, Bu = imq.imq_unpack(plan, Ad, Bd)
+    if check_unpack:
+        oAu, oBu = oracle.unpack(pl, A, B)
+        assert np.array_equal(Au.cpu().numpy(), oAu), "A' bytes"
+        assert np.array_equal(Bu.cpu().numpy(), oBu), "B'^T bytes"
+    rng = np.random.default_rng(M * 7 + N)
+    dA = rng.uniform(1e-3, 1.0, M).astype(np.float32)
+    dB = rng.uniform(1e-3, 1.0, N).astype(np.float32)
+    C, Cf = imq.imq_gemm_unpacked(plan, Au, Bu, torch.from_numpy(dA).cuda(), imq.IMQ_PER_ROW,
+                                  torch.from_numpy(dB).cuda(), imq.IMQ_PER_COL)
+    torch.cuda.synchronize()
+    assert imq.imq_device_status() == imq.IMQ_OK
+    want = oracle.gemm_exact(A, B)
+    got = C.cpu().numpy().astype(np.int64)
+    assert np.array_equal(got, want), f"C mismatch at {np.argwhere(got != want)[:5]}"
+    assert_f32_close(Cf.cpu().numpy(), oracle.dequant(want, dA, oracle.PER_ROW, dB, oracle.PER_COL))
+    return plan
+
+
+@pytest.mark.parametrize("b", [2, 3, 5, 8])
+@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("trans", [(False, False), (True, False), (False, True), (True, True)])
+def test_path_parity_int32_regime(imq, b, strategy, trans):
+    rng = np.random.default_rng(1000 * b + 10 * strategy + 2 * trans[0] + trans[1])
+    A, B = workloads.random_case(rng, 300, 500, 700, big=300, frac=0.05)
+    _run_path(imq, A, B, b, strategy, *trans)
+
+
+@pytest.mark.parametrize("b", [3, 4, 5, 8])
+@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4])
+def test_path_parity_int64_regime(imq, b, strategy):
+    rng = np.random.default_rng(77 + 10 * b + strategy)
+    A, B = workloads.random_case(rng, 200, 384, 300, big=3000, frac=0.05)
+    plan = _run_path(imq, A, B, b, strategy, False, True)
+    if plan is not None:
+        assert plan.info["acc_bits"] == 64
+
+
+def test_path_parity_no_outliers_is_plain_int8(imq):
+    rng = np.random.default_rng(3)
+    A = rng.integers(-127, 128, size=(256 + 17, 1024 + 40)).astype(np.int64)
+    B = rng.integers(-127, 128, size=(1024 + 40, 512 + 3)).astype(np.int64)
+    plan = _run_path(imq, A, B, 8, 0, False, False)
+    assert plan.info["ratio"] == 1.0 and plan.info["dir_a"] == 0 and plan.info["dir_b"] == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (1, 300, 1), (129, 1, 257), (128, 128, 256), (5, 3000, 9)])
+def test_path_parity_edge_shapes(imq, shape):
+    rng = np.random.default_rng(sum(shape))
+    A, B = workloads.random_case(rng, *shape, big=3000, frac=0.1)
+    for st in range(5):
+        _run_path(imq, A, B, 5, st, False, False)
+
+
+def test_path_int32_inputs(imq):
+    rng = np.random.default_rng(9)
+    A, B = workloads.random_case(rng, 130, 260, 270, big=100000, frac=0.01)
+    _run_path(imq, A, B, 8, 0, True, False, dtype=torch.int32)
+
+
+def test_gemm_rejects_int32_output_when_bound_exceeds(imq):
+    rng = np.random.default_rng(10)
+    A, B = workloads.random_case(rng, 64, 256, 64, big=30000, frac=0.05)
+    pl = oracle.plan(A, B, 8, 0)
+    assert not pl.bound_lt_2_31
+    Ad = torch.from_numpy(A.astype(np.int16)).cuda()
+    Bd = torch.from_numpy(B.astype(np.int16)).cuda()
+    plan = imq.imq_plan(Ad, Bd, 8, 0)
+    with pytest.raises(imq.ImqError) as e:
+        imq.imq_unpacked_gemm(plan, Ad, Bd, c_dtype=torch.int32, want_f32=False)
+    assert e.value.status == imq.IMQ_ERR_RANGE
+
+
+def test_unpacked_gemm_workspace_checks(imq):
+    rng = np.random.default_rng(11)
+    A, B = workloads.random_case(rng, 40, 90, 50, big=200, frac=0.1)
+    Ad = torch.from_numpy(A.astype(np.int16)).cuda()
+    Bd = torch.from_numpy(B.astype(np.int16)).cuda()
+    plan = imq.imq_plan(Ad, Bd, 4, 0)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(imq.ImqError) as e:
+        imq.imq_unpacked_gemm(plan, Ad, Bd, workspace=small, want_f32=False)
+    assert e.value.status == imq.IMQ_ERR_BUFFER
+    C, _ = imq.imq_unpacked_gemm(plan, Ad, Bd, want_f32=False)
+    assert np.array_equal(C.cpu().numpy().astype(np.int64), A @ B)
+
+
+def test_plan_uses_given_line_maxima(imq):
+    rng = np.random.default_rng(12)
+    A, B = workloads.random_case(rng, 100, 200, 150, big=500, frac=0.05)
+    Ad = torch.from_numpy(A.astype(np.int16)).cuda()
+    Bd = torch.from_numpy(B.astype(np.int16)).cuda()
+    mx = [torch.from_numpy(v.astype(np.int32)).cuda() for v in
+          (np.abs(A).max(1), np.abs(A).max(0), np.abs(B).max(1), np.abs(B).max(0))]
+    p1 = imq.imq_plan(Ad, Bd, 5, 0)
+    p2 = imq.imq_plan(Ad, Bd, 5, 0, maxes=mx)
+    assert p1.info == p2.info
+
+
+def test_repeatable(imq):
+    rng = np.random.default_rng(13)
+    A, B = workloads.random_case(rng, 300, 700, 600, big=2000, frac=0.05)
+    Ad = torch.from_numpy(A.astype(np.int16)).cuda()
+    Bd = torch.from_numpy(B.astype(np.int16)).cuda()
+    plan = imq.imq_plan(Ad, Bd, 5, 0)
+    C1, _ = imq.imq_unpacked_gemm(plan, Ad, Bd, want_f32=False)
+    C2, _ = imq.imq_unpacked_gemm(plan, Ad, Bd, want_f32=False)
+    assert torch.equal(C1, C2)
