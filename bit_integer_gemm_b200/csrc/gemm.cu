@@ -9,15 +9,16 @@
 //               swizzle, into a 4-stage shared-memory ring (mbarrier complete_tx).
 //   warp 1      MMA issuer (one thread): tcgen05.mma.cta_group::1.kind::i8, M=128 N=256 K=32,
 //               s8 x s8 -> s32 accumulators in tensor memory (TMEM).
-//   warps 2-5   epilogue: tcgen05.ld of the accumulators, fold-back, dequantisation, stores.
-// The inner dimension is a sequence of exponent groups (products weighted by R^e).  The groups of one
-// accumulator slot run in descending e; between two groups the epilogue warps multiply the slot by
-// R^(e_prev - e) in TMEM (Horner's rule), so the slot ends as sum_e R^(e - e_min) C_e.  The plan proves
-// every intermediate value of a slot stays below 2^31.  When the full product may exceed int32 a second
-// slot keeps the e = 0 group apart and the two are combined in int64 in the epilogue.
-// The epilogue stages each 128 x 32 accumulator chunk in shared memory and folds the OUTER-unpacked
-// lines back (row levels of A, column levels of B) with shifts, then writes C (int32/int64) and the
-// dequantised fp32 copy with coalesced stores.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulators, fold-back, shift, accumulation into C,
+//               dequantisation.
+// The inner dimension is a sequence of exponent groups whose products carry the weight R^e.  Each group
+// of each tile is one accumulation job; jobs alternate between two 256-column TMEM slots, so the MMAs of
+// job n+1 run while the epilogue drains job n (also across tiles).  The epilogue folds the OUTER lines
+// of a job back with their level weights, shifts by e*(b-1) and adds the result into C (the first job of
+// a tile writes, later ones read-modify-write the tile they own; the last also writes the fp32 copy).
+// Every partial sum is a partial sum of the exact product, so it is bounded by the plan's bound: int32
+// when that is below 2^31, int64 otherwise.  The plan splits a group along K when its raw s32
+// accumulator could overflow.
 // Every mbarrier wait is bounded (common.cuh): a stuck pipeline ends the kernel with IMQ_ERR_TIMEOUT.
 #include <string.h>
 
@@ -37,13 +38,10 @@ constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 struct GemmArgs {
   int32_t tiles_m, tiles_n;
-  int32_t seq_len;
-  int32_t n_slots;
-  int32_t seq_kb0[kMaxSeq];
-  int32_t seq_nkb[kMaxSeq];
-  int8_t seq_slot[kMaxSeq];
-  int8_t seq_rescale[kMaxSeq];
-  int32_t slot_shift[2];
+  int32_t n_jobs;
+  int32_t job_kb0[kMaxJobs];
+  int32_t job_nkb[kMaxJobs];
+  int8_t job_shift[kMaxJobs];
   int32_t bm1;
   int32_t a_outer, b_outer;
   const int32_t* srcA;
@@ -66,16 +64,15 @@ struct GemmArgs {
   uint64_t timeout_ns;
 };
 
-template <bool kWide>
 struct Smem {
-  using Stage = typename std::conditional<kWide, int64_t, int32_t>::type;
   static constexpr size_t kA = 0;
   static constexpr size_t kB = kA + (size_t)STAGES * A_STAGE;
-  static constexpr size_t kStage = kB + (size_t)STAGES * B_STAGE;
-  static constexpr size_t kRsrc = kStage + (size_t)BM * 32 * sizeof(Stage);
+  static constexpr size_t kStage = kB + (size_t)STAGES * B_STAGE;  // int32 [128][32], XOR-swizzled
+  static constexpr size_t kRsrc = kStage + (size_t)BM * 32 * 4;
   static constexpr size_t kCsrc = kRsrc + BM * 4;
-  static constexpr size_t kBars = kCsrc + 32 * 4;  // full[S], empty[S], acc_full, acc_empty, drain
-  static constexpr size_t kMisc = kBars + (2 * STAGES + 3) * 8;  // tmem base, abort flag, epilogue flag
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain
+  static constexpr size_t kBars = kCsrc + 32 * 4;
+  static constexpr size_t kMisc = kBars + (2 * STAGES + 5) * 8;  // tmem base, abort flag, epilogue flag
   static constexpr size_t kEnd = kMisc + 16;
   static constexpr size_t kBytes = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
@@ -87,17 +84,15 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
   return true;
 }
 
-template <bool kWide>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ GemmArgs g) {
-  using L = Smem<kWide>;
-  using Stage = typename L::Stage;
+  using L = Smem;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base + L::kA;
   uint8_t* sB = base + L::kB;
-  Stage* stg = reinterpret_cast<Stage*>(base + L::kStage);
+  int32_t* stg = reinterpret_cast<int32_t*>(base + L::kStage);
   int32_t* s_rsrc = reinterpret_cast<int32_t*>(base + L::kRsrc);
   int32_t* s_csrc = reinterpret_cast<int32_t*>(base + L::kCsrc);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::kBars);
@@ -107,17 +102,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + STAGES);
-  const uint32_t acc_full = smem_addr(bars + 2 * STAGES), acc_empty = smem_addr(bars + 2 * STAGES + 1);
-  const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 2);
-  const uint32_t ncols = (uint32_t)g.n_slots * BN;
+  const uint32_t accf0 = smem_addr(bars + 2 * STAGES), acce0 = smem_addr(bars + 2 * STAGES + 2);
+  const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 4);
+  constexpr uint32_t kCols = 2 * BN;  // two accumulator slots
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, EPI_THREADS);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(accf0 + 8 * s, 1);
+      mbar_init(acce0 + 8 * s, EPI_THREADS);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -128,7 +125,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_holder), ncols);
+    tmem_alloc(smem_addr(tmem_holder), kCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -146,12 +143,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int s = 0; s < STAGES; ++s) issued[s] = 2;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
-        for (int i = 0; i < g.seq_len; ++i) {
-          for (int kb = 0; kb < g.seq_nkb[i]; ++kb) {
+        for (int j = 0; j < g.n_jobs; ++j) {
+          for (int kb = 0; kb < g.job_nkb[j]; ++kb) {
             if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
             const uint32_t fb = full0 + 8 * stage;
             mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
-            const int32_t x = (g.seq_kb0[i] + kb) * BK;
+            const int32_t x = (g.job_kb0[j] + kb) * BK;
             tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, x, mt * BM, fb);
             tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, x, nt * BN, fb);
             issued[stage] = phase;
@@ -174,22 +171,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t idesc = idesc_i8(BM, BN);
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t acc_waits = 0;
+      uint32_t empty_waits[2] = {0, 0};
+      uint32_t job_count = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(acc_empty, (acc_waits & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns)) goto mma_done;
-        ++acc_waits;
-        tc_fence_after();
-        for (int i = 0; i < g.seq_len; ++i) {
-          const uint32_t d = tmem_base + (uint32_t)g.seq_slot[i] * BN;
-          const bool first = g.seq_rescale[i] < 0;
-          if (!first) {
-            // Horner step: the epilogue multiplies this slot by R^(e_prev - e) once it is complete
-            mma_commit(acc_full);
-            if (!mbar_wait(acc_empty, (acc_waits & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns)) goto mma_done;
-            ++acc_waits;
-            tc_fence_after();
-          }
-          for (int kb = 0; kb < g.seq_nkb[i]; ++kb) {
+        for (int j = 0; j < g.n_jobs; ++j, ++job_count) {
+          const uint32_t slot = job_count & 1u;
+          // the epilogue has drained the job this slot held before
+          if (!mbar_wait(acce0 + 8 * slot, (empty_waits[slot] & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns))
+            goto mma_done;
+          ++empty_waits[slot];
+          tc_fence_after();
+          const uint32_t d = tmem_base + slot * BN;
+          for (int kb = 0; kb < g.job_nkb[j]; ++kb) {
             if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, g.status, g.timeout_ns)) goto mma_done;
             tc_fence_after();
             const uint64_t adesc = smem_desc_k_sw128(smem_addr(sA + (size_t)stage * A_STAGE));
@@ -197,7 +190,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
               // 32 bytes further along K inside the 128-byte swizzled row: +2 in the address field
-              mma_i8(d, adesc + 2 * k, bdesc + 2 * k, idesc, (first && kb == 0 && k == 0) ? 0u : 1u);
+              mma_i8(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb == 0 && k == 0) ? 0u : 1u);
             }
             mma_commit(empty0 + 8 * stage);
             if (++stage == STAGES) {
@@ -205,8 +198,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               phase ^= 1u;
             }
           }
+          mma_commit(accf0 + 8 * slot);
         }
-        mma_commit(acc_full);
       }
     mma_done:
       // every issued MMA must complete before TMEM is released
@@ -220,17 +213,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;     // accumulator row owned by this thread
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    uint32_t acc_waits = 0;
-    // One thread waits on the accumulator barrier and all 128 take its answer, so every epilogue
-    // thread passes the same named barriers even when a wait gives up.
-    auto wait_acc_full = [&]() -> bool {
-      if (et == 0) *epi_ok = mbar_wait(acc_full, acc_waits & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
-      named_bar_sync(1, EPI_THREADS);
-      const bool ok = *epi_ok != 0;
-      named_bar_sync(1, EPI_THREADS);
-      ++acc_waits;
-      return ok;
-    };
+    uint32_t full_waits[2] = {0, 0};
+    uint32_t job_count = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
       // source rows of this tile
@@ -245,98 +229,89 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         nA = rem < BM ? (int)rem : BM;
         if (et < nA) s_rsrc[et] = mt * BM + et;
       }
-      // Horner rescales
-      for (int i = 0; i < g.seq_len; ++i) {
-        if (g.seq_rescale[i] < 0) continue;
-        if (!wait_acc_full()) goto epi_done;
+      for (int j = 0; j < g.n_jobs; ++j, ++job_count) {
+        const uint32_t slot = job_count & 1u;
+        // one thread waits and all 128 take its answer, so every epilogue thread passes the same named
+        // barriers even when a wait gives up
+        if (et == 0)
+          *epi_ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
+        named_bar_sync(1, EPI_THREADS);
+        const bool ok = *epi_ok != 0;
+        named_bar_sync(1, EPI_THREADS);
+        ++full_waits[slot];
+        if (!ok) goto epi_done;
         tc_fence_after();
-        const uint32_t sbase = tmem_base + lane_off + (uint32_t)g.seq_slot[i] * BN;
-        // the plan bounds every slot value by 2^31, so a shift of 31 or more only meets zeros
-        const int32_t mul = g.seq_rescale[i] < 31 ? (1 << g.seq_rescale[i]) : 0;
+        const bool first = j == 0, last = j == g.n_jobs - 1;
+        const int64_t mul = (int64_t)1 << g.job_shift[j];
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(sbase + c * 32, v);
+          tmem_ld32(tmem_base + lane_off + slot * BN + c * 32, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = (uint32_t)((int32_t)v[j] * mul);
-          tmem_st32(sbase + c * 32, v);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(acc_empty);
-      }
-      // final accumulators
-      if (!wait_acc_full()) goto epi_done;
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v0[32];
-        tmem_ld32(tmem_base + lane_off + c * 32, v0);
-        if (kWide) {
-          uint32_t v1[32];
-          tmem_ld32(tmem_base + lane_off + BN + c * 32, v1);
-          tmem_wait_ld();
-          const int64_t m0 = (int64_t)1 << g.slot_shift[0], m1 = (int64_t)1 << g.slot_shift[1];
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            stg[row * 32 + (j ^ lane)] = (Stage)((int64_t)(int32_t)v0[j] * m0 + (int64_t)(int32_t)v1[j] * m1);
-        } else {
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) stg[row * 32 + (j ^ lane)] = (Stage)(int32_t)v0[j];
-        }
-        // source columns of this 32-column chunk
-        const int64_t gc = (int64_t)nt * (BN / 32) + c;
-        int LB, nB;
-        if (g.b_outer) {
-          if (gc < g.n_grp_b) {
-            LB = g.grpB_L[gc];
-            nB = g.grpB_n[gc];
+          for (int jj = 0; jj < 32; ++jj) stg[row * 32 + (jj ^ lane)] = (int32_t)v[jj];
+          if (c == BN / 32 - 1) {
+            // the slot is fully read: let the MMA warp start the job after next in it
+            tc_fence_before();
+            mbar_arrive(acce0 + 8 * slot);
+          }
+          // source columns of this 32-column chunk
+          const int64_t gc = (int64_t)nt * (BN / 32) + c;
+          int LB, nB;
+          if (g.b_outer) {
+            if (gc < g.n_grp_b) {
+              LB = g.grpB_L[gc];
+              nB = g.grpB_n[gc];
+            } else {
+              LB = 1;
+              nB = 0;
+            }
+            if (et < nB) s_csrc[et] = g.srcB[gc * 32 + (int64_t)et * LB];
           } else {
             LB = 1;
-            nB = 0;
+            const int64_t rem = g.N - gc * 32;
+            nB = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
+            if (et < nB) s_csrc[et] = (int32_t)(gc * 32 + et);
           }
-          if (et < nB) s_csrc[et] = g.srcB[gc * 32 + (int64_t)et * LB];
-        } else {
-          LB = 1;
-          const int64_t rem = g.N - gc * 32;
-          nB = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
-          if (et < nB) s_csrc[et] = (int32_t)(gc * 32 + et);
-        }
-        named_bar_sync(1, EPI_THREADS);
-        const int total = nA * nB;
-        for (int o = et; o < total; o += EPI_THREADS) {
-          const int r = o / nB, s = o - r * nB;
-          int64_t acc = 0;
-          for (int la = 0; la < LA; ++la) {
-            const int rr = r * LA + la;
-            for (int lb = 0; lb < LB; ++lb) {
-              const int cc = s * LB + lb;
-              acc += (int64_t)stg[rr * 32 + (cc ^ (rr & 31))] * ((int64_t)1 << ((la + lb) * g.bm1));
+          named_bar_sync(1, EPI_THREADS);
+          const int total = nA * nB;
+          for (int o = et; o < total; o += EPI_THREADS) {
+            const int r = o / nB, s = o - r * nB;
+            int64_t acc = 0;
+            for (int la = 0; la < LA; ++la) {
+              const int rr = r * LA + la;
+              for (int lb = 0; lb < LB; ++lb) {
+                const int cc = s * LB + lb;
+                acc += (int64_t)stg[rr * 32 + (cc ^ (rr & 31))] * ((int64_t)1 << ((la + lb) * g.bm1));
+              }
+            }
+            acc *= mul;
+            const int64_t i = s_rsrc[r], col = s_csrc[s];
+            // the same thread owns output (i, col) in every job of this tile
+            if (g.c64) {
+              int64_t* cp = static_cast<int64_t*>(g.C) + i * g.ldc + col;
+              if (!first) acc += *cp;
+              *cp = acc;
+            } else if (g.C) {
+              int32_t* cp = static_cast<int32_t*>(g.C) + i * g.ldc + col;
+              if (!first) acc += *cp;
+              *cp = (int32_t)acc;
+            }
+            if (last && g.Cf) {
+              const float sa = g.dA[g.dA_per_row ? i : 0], sb = g.dB[g.dB_per_col ? col : 0];
+              g.Cf[i * g.ldcf + col] = __fmul_rn(__ll2float_rn(acc), __fmul_rn(sa, sb));
             }
           }
-          const int64_t i = s_rsrc[r], jj = s_csrc[s];
-          if (g.C) {
-            if (g.c64) static_cast<int64_t*>(g.C)[i * g.ldc + jj] = acc;
-            else static_cast<int32_t*>(g.C)[i * g.ldc + jj] = (int32_t)acc;
-          }
-          if (g.Cf) {
-            const float sa = g.dA[g.dA_per_row ? i : 0], sb = g.dB[g.dB_per_col ? jj : 0];
-            g.Cf[i * g.ldcf + jj] = __fmul_rn(__ll2float_rn(acc), __fmul_rn(sa, sb));
-          }
+          named_bar_sync(1, EPI_THREADS);
         }
-        named_bar_sync(1, EPI_THREADS);
       }
-      tc_fence_before();
-      mbar_arrive(acc_empty);
     }
   epi_done:;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, ncols);
+  if (warp == 1) tmem_dealloc(tmem_base, kCols);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -381,6 +356,7 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   if (Cf && gA != IMQ_PER_TENSOR && gA != IMQ_PER_ROW) return IMQ_ERR_ARG;
   if (Cf && gB != IMQ_PER_TENSOR && gB != IMQ_PER_COL) return IMQ_ERR_ARG;
   if (C && ct == IMQ_I32 && I.acc_bits > 32) return IMQ_ERR_RANGE;
+  if (!C && pl->n_jobs > 1) return IMQ_ERR_ARG;  // the jobs of a tile accumulate in C
   if (I.M == 0 || I.N == 0) return IMQ_OK;
   const size_t esz = ct == IMQ_I64 ? 8 : 4;
   if (I.K_unp == 0) {
@@ -401,17 +377,12 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   memset(&g, 0, sizeof(g));
   g.tiles_m = (int32_t)((I.M_unp + BM - 1) / BM);
   g.tiles_n = (int32_t)((I.N_unp + BN - 1) / BN);
-  g.seq_len = pl->seq_len;
-  g.n_slots = pl->n_slots;
-  for (int i = 0; i < pl->seq_len; ++i) {
-    const imq_group& gr = pl->groups[pl->seq_group[i]];
-    g.seq_kb0[i] = (int32_t)(gr.k_offset / BK);
-    g.seq_nkb[i] = (int32_t)(gr.k_len_padded / BK);
-    g.seq_slot[i] = (int8_t)pl->seq_slot[i];
-    g.seq_rescale[i] = (int8_t)pl->seq_rescale[i];
+  g.n_jobs = pl->n_jobs;
+  for (int j = 0; j < pl->n_jobs; ++j) {
+    g.job_kb0[j] = (int32_t)(pl->job_k0[j] / BK);
+    g.job_nkb[j] = (int32_t)(pl->job_klen[j] / BK);
+    g.job_shift[j] = (int8_t)pl->job_shift[j];
   }
-  g.slot_shift[0] = pl->slot_shift[0];
-  g.slot_shift[1] = pl->slot_shift[1];
   g.bm1 = I.b - 1;
   g.a_outer = I.dir_a == IMQ_DIR_OUTER;
   g.b_outer = I.dir_b == IMQ_DIR_OUTER;
@@ -429,7 +400,7 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   g.dA_per_row = gA == IMQ_PER_ROW;
   g.dB_per_col = gB == IMQ_PER_COL;
   g.C = C;
-  g.c64 = ct == IMQ_I64;
+  g.c64 = C != nullptr && ct == IMQ_I64;
   g.ldc = ldc;
   g.Cf = Cf;
   g.ldcf = ldcf;
@@ -438,18 +409,12 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
 
   const int num_tiles = g.tiles_m * g.tiles_n;
   const int grid = num_tiles < ds->num_sms ? num_tiles : ds->num_sms;
-  if (pl->wide_stage) {
-    const size_t smem = Smem<true>::kBytes;
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_gemm<true><<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
-  } else {
-    const size_t smem = Smem<false>::kBytes;
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_gemm<false><<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
-  }
+  const size_t smem = Smem::kBytes;
+  IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  k_gemm<<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
-static_assert(Smem<true>::kBytes <= 232448, "shared memory budget");
+static_assert(Smem::kBytes <= 232448, "shared memory budget");
 
 }  // namespace imq

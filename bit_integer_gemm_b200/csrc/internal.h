@@ -9,7 +9,7 @@
 
 namespace imq {
 
-constexpr int kMaxSeq = IMQ_MAX_GROUPS;
+constexpr int kMaxJobs = 128;  // accumulation jobs of one output tile
 
 // Per-device state owned by the library: the status word address and small scratch buffers.
 struct DeviceState {
@@ -68,14 +68,12 @@ struct imq_plan {
   int32_t* grpB_n;
   int64_t n_grp_a, n_grp_b;
   imq_group groups[IMQ_MAX_GROUPS];
-  // GEMM schedule over the groups (see gemm.cu)
-  int32_t n_slots;
-  int32_t seq_len;
-  int32_t seq_group[imq::kMaxSeq];
-  int32_t seq_slot[imq::kMaxSeq];
-  int32_t seq_rescale[imq::kMaxSeq];  // left shift applied to the slot before this group, -1: first
-  int32_t slot_shift[2];              // final left shift of each slot
-  int32_t wide_stage;                 // stage the accumulators as int64 in the epilogue
+  // GEMM schedule: each job accumulates one exponent group (or a K-slice of one) in a TMEM slot, and
+  // the epilogue adds (job value) << job_shift into C (see gemm.cu)
+  int32_t n_jobs;
+  int64_t job_k0[imq::kMaxJobs];    // first unpacked inner index (multiple of IMQ_INNER_PAD)
+  int64_t job_klen[imq::kMaxJobs];  // inner length (multiple of IMQ_INNER_PAD)
+  int32_t job_shift[imq::kMaxJobs]; // e * (b - 1)
 };
 
 namespace imq {

@@ -541,43 +541,27 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   if (bound >= ((unsigned __int128)1 << 63)) return fail(IMQ_ERR_UNSUPPORTED);  // C itself may leave int64
   I.acc_bits = bound < two31 ? 32 : 64;
   const int bm1 = b - 1;
-  const int64_t R1 = ((int64_t)1 << bm1) - 1;
-  pl->n_slots = 1;
-  pl->seq_len = 0;
-  pl->wide_stage = 0;
-  pl->slot_shift[0] = pl->slot_shift[1] = 0;
-  if (ng > 0) {
-    if (bound < two31 || ng == 1) {
-      if (bound >= two31 && (unsigned __int128)pl->groups[0].k_len * (unsigned __int128)(R1 * R1) >= two31)
-        return fail(IMQ_ERR_UNSUPPORTED);
-      for (int g = ng - 1; g >= 0; --g) {
-        const int i = pl->seq_len++;
-        pl->seq_group[i] = g;
-        pl->seq_slot[i] = 0;
-        pl->seq_rescale[i] = (g == ng - 1) ? -1 : (pl->groups[g + 1].e - pl->groups[g].e) * bm1;
-      }
-      pl->slot_shift[0] = pl->groups[0].e * bm1;
-    } else {
-      const int e1 = pl->groups[1].e;
-      const int sh1 = e1 * bm1;
-      const bool fits = (sh1 + 31 >= 127) || (bound < (two31 << sh1));
-      if (!fits) return fail(IMQ_ERR_UNSUPPORTED);
-      if ((unsigned __int128)pl->groups[0].k_len * (unsigned __int128)(R1 * R1) >= two31)
-        return fail(IMQ_ERR_UNSUPPORTED);
-      for (int g = ng - 1; g >= 1; --g) {
-        const int i = pl->seq_len++;
-        pl->seq_group[i] = g;
-        pl->seq_slot[i] = 1;
-        pl->seq_rescale[i] = (g == ng - 1) ? -1 : (pl->groups[g + 1].e - pl->groups[g].e) * bm1;
-      }
-      const int i = pl->seq_len++;
-      pl->seq_group[i] = 0;
-      pl->seq_slot[i] = 0;
-      pl->seq_rescale[i] = -1;
-      pl->n_slots = 2;
-      pl->slot_shift[0] = pl->groups[0].e * bm1;
-      pl->slot_shift[1] = sh1;
-      pl->wide_stage = 1;
+  const unsigned __int128 R1 = ((unsigned __int128)1 << bm1) - 1;
+  // One accumulation job per exponent group.  The raw s32 accumulator of group e is bounded both by
+  // k_len * (R-1)^2 and by bound / R^e (R^e times it is a partial sum of the product); a group whose two
+  // bounds both reach 2^31 is split along K into slices of at most (2^31 - 1) / (R-1)^2 indices.
+  pl->n_jobs = 0;
+  for (int g = 0; g < ng; ++g) {
+    const imq_group& gr = pl->groups[g];
+    const int sh = gr.e * bm1;
+    const unsigned __int128 by_len = (unsigned __int128)gr.k_len * R1 * R1;
+    const unsigned __int128 by_bound = sh >= 127 ? 0 : (bound >> sh);
+    int64_t slice = gr.k_len_padded;
+    if (by_len >= two31 && by_bound >= two31) {
+      slice = (int64_t)((two31 - 1) / (R1 * R1)) / IMQ_INNER_PAD * IMQ_INNER_PAD;
+      if (slice < IMQ_INNER_PAD) return fail(IMQ_ERR_UNSUPPORTED);
+    }
+    for (int64_t k0 = 0; k0 < gr.k_len_padded; k0 += slice) {
+      if (pl->n_jobs >= kMaxJobs) return fail(IMQ_ERR_UNSUPPORTED);
+      const int j = pl->n_jobs++;
+      pl->job_k0[j] = gr.k_offset + k0;
+      pl->job_klen[j] = (gr.k_len_padded - k0) < slice ? (gr.k_len_padded - k0) : slice;
+      pl->job_shift[j] = sh;
     }
   }
   I.workspace_bytes = align_up((size_t)(I.M_unp * I.K_unp), 1024) + align_up((size_t)(I.N_unp * I.K_unp), 1024);

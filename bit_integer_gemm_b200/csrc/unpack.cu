@@ -20,7 +20,7 @@
 namespace imq {
 namespace {
 
-template <typename T>
+template <typename T, bool kStaged>
 __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, int64_t nlines, int64_t K,
                                                      int64_t ld, int outer, const int8_t* __restrict__ lvl,
                                                      const int32_t* __restrict__ pos,
@@ -30,8 +30,11 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
   extern __shared__ int32_t line[];
   const int tid = threadIdx.x;
   for (int64_t i = blockIdx.x; i < nlines; i += gridDim.x) {
-    for (int64_t t = tid; t < K; t += 256) line[t] = (int32_t)X[i * ld + t];
-    __syncthreads();
+    const T* xi = X + i * ld;
+    if (kStaged) {
+      for (int64_t t = tid; t < K; t += 256) line[t] = (int32_t)xi[t];
+      __syncthreads();
+    }
     const int L = outer ? (int)lvl[i] : 1;
     const int64_t base = outer ? (int64_t)pos[i] : i;
     for (int l = 0; l < L; ++l) {
@@ -50,7 +53,7 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int k = q * 4 + r;
-            const int32_t d = tt[k] >= 0 ? digit_of(line[tt[k]], l + ll[k], bm1) : 0;
+            const int32_t d = tt[k] >= 0 ? digit_of(kStaged ? line[tt[k]] : (int32_t)xi[tt[k]], l + ll[k], bm1) : 0;
             packed |= ((uint32_t)(uint8_t)(int8_t)d) << (8 * r);
           }
           w[q] = packed;
@@ -124,14 +127,19 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
                       int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st) {
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
   if (line_is_row) {
+    // lines up to 48K entries are staged in shared memory; longer ones are gathered from L2
     const size_t smem = (size_t)(K > 0 ? K : 1) * 4;
-    if (smem > 200 * 1024) return IMQ_ERR_UNSUPPORTED;
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_rows<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    int per_sm = (int)((200 * 1024) / (smem + 1024));
+    const bool staged = smem <= 192 * 1024;
+    int per_sm = staged ? (int)((200 * 1024) / (smem + 1024)) : 8;
     if (per_sm > 8) per_sm = 8;
     if (per_sm < 1) per_sm = 1;
     const int64_t grid = nlines < (int64_t)num_sms * per_sm ? nlines : (int64_t)num_sms * per_sm;
-    k_unpack_rows<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, outer, lvl, pos, tK, lk, K_unp, bm1, out);
+    if (staged) {
+      IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_rows<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      k_unpack_rows<T, true><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, outer, lvl, pos, tK, lk, K_unp, bm1, out);
+    } else {
+      k_unpack_rows<T, false><<<(unsigned)grid, 256, 0, st>>>(X, nlines, K, ld, outer, lvl, pos, tK, lk, K_unp, bm1, out);
+    }
   } else {
     const dim3 grid((unsigned)((nlines + 31) / 32), (unsigned)(K_unp / 128));
     if (K_unp / 128 > 65535) return IMQ_ERR_UNSUPPORTED;

@@ -163,10 +163,9 @@ typedef struct {
  * plan    out: a new plan object.
  * Synchronises the stream once (reads a summary of a few hundred bytes).  Returns any pending device
  * status (e.g. IMQ_ERR_NONFINITE from a preceding quantisation) before planning.
- * IMQ_ERR_UNSUPPORTED: more than IMQ_MAX_GROUPS exponent groups, a line level above 31, an exponent
- * group whose raw int32 accumulation could overflow (k_len*(R-1)^2 >= 2^31), or a bound so large that
- * two TMEM accumulators cannot hold the exact sum (bound / R^e1 >= 2^31 with e1 the smallest
- * non-zero exponent present).
+ * IMQ_ERR_UNSUPPORTED: more than IMQ_MAX_GROUPS exponent groups, more than 128 accumulation jobs
+ * (groups, split along K where a raw int32 accumulator could overflow), or a bound of 2^63 or more
+ * (the product itself may leave int64).
  */
 imq_status imq_plan(const void *A, const void *B, imq_dtype it, int64_t M, int64_t K, int64_t N,
                     int32_t transA, int64_t lda, int32_t transB, int64_t ldb,
@@ -213,17 +212,20 @@ imq_status imq_unpack(const imq_plan_t *plan, const void *A, const void *B,
 
 /*
  * imq_gemm_unpacked -- the low-bit GEMM on already unpacked operands with the fold-back epilogue:
- *   C = sum over exponent groups e of R^e * (A'_e * B'_e), then every OUTER line folded back with its
- *   level weight R^l ("Approach": bit-shift scaling and accumulation reproduce the integer product
- *   exactly).  s8 x s8 -> s32 products run on the tcgen05 tensor cores; partial sums never leave
- *   int32 inside one accumulator (the plan checks the bounds), the fold runs in int32 or int64.
+ *   C = sum over exponent groups e of R^e * (A'_e * B'_e), every OUTER line folded back with its level
+ *   weight R^l ("Approach": bit-shift scaling and accumulation reproduce the integer product
+ *   exactly).  s8 x s8 -> s32 products run on the tcgen05 tensor cores, one int32 tensor-memory
+ *   accumulator per exponent group (the plan splits a group along K if that could overflow); the
+ *   epilogue shifts each group into C.  Every partial sum is bounded by the plan's bound, so int32
+ *   is exact when acc_bits == 32 and int64 otherwise.
  *   Cf[i,j] = (float)C[i,j] * (deltaA[i] * deltaB[j])  (fp32; READING: the page implies dequantised
  *   outputs but gives no formula).
  * deltaA  device fp32: 1 value (gA = IMQ_PER_TENSOR) or M values (IMQ_PER_ROW: one per row of A).
  * deltaB  device fp32: 1 value (IMQ_PER_TENSOR) or N values (IMQ_PER_COL: one per column of B).
  *         Both may be NULL when Cf is NULL.
  * Cint    device or NULL, M x N, leading dim ldc, dtype ct (I32 or I64).  I32 with
- *         plan acc_bits == 64 returns IMQ_ERR_RANGE.
+ *         plan acc_bits == 64 returns IMQ_ERR_RANGE.  When the plan has more than one exponent group
+ *         the groups accumulate in Cint, so it must be given (IMQ_ERR_ARG otherwise).
  * Cf      device or NULL, fp32 M x N, leading dim ldcf.
  * Asynchronous.
  */

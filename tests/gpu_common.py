@@ -57,16 +57,6 @@ def plan_matches(info: dict, pl: oracle.Plan):
     assert info["bound"] == pl.bound
 
 
-def slots_needed_unsupported(pl: oracle.Plan) -> bool:
-    """True when the plan's bound needs more than the two TMEM accumulator slots the GEMM keeps:
-    bound >= 2^31 * R^e1 with e1 the smallest non-zero exponent present, or the e = 0 group alone
-    could overflow int32."""
-    if pl.bound_lt_2_31 or len(pl.groups) == 0:
-        return False
-    R1 = (1 << (pl.b - 1)) - 1
-    if pl.groups[0][2] * R1 * R1 >= 2 ** 31:
-        return True
-    if len(pl.groups) == 1:
-        return False
-    e1 = pl.groups[1][0]
-    return int(round(pl.bound)) >= (2 ** 31) * (2 ** (e1 * (pl.b - 1)))
+def unsupported(pl: oracle.Plan) -> bool:
+    """True when the library must refuse the plan: the bound reaches 2^63 (C may leave int64)."""
+    return int(round(pl.bound)) >= 2 ** 63

@@ -1,0 +1,120 @@
+"""Full-size parity on the five seeded workloads (tiny, q_proj, mlp, attention, wgrad), in the launch
+configuration the benchmark uses: quantiser side outputs feed the plan, imq_unpack then
+imq_gemm_unpacked.  Integer outputs are compared bit-exactly with the oracle -- in full, except the
+three MLP products whose rows are sampled (the oracle's exact product of 512 sampled rows); fp32
+outputs within 1e-6 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_common import assert_f32_close, logical, logical_maxes, plan_matches, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def imq():
+    import bit_integer_gemm_b200 as m
+    assert torch.cuda.is_available(), "a GPU is required"
+    m.lib()
+    m.imq_device_status(clear=True)
+    return m
+
+
+def _quant_both(imq, g):
+    """Quantises A and B on the GPU and with the oracle; checks the quantiser bit-exactly.  Both use
+    int16 unless a value needs int32 (the softmax matrix P: its row maximum is ~1e4 times its 95th
+    percentile)."""
+    ref = [oracle.rtn_quantize(oracle.as_f32(st.data, st.dtype), gran, g.p, g.beta)
+           for st, gran in ((g.A, g.qa), (g.B, g.qb))]
+    wide = max(int(np.abs(r[0]).max()) for r in ref) > 32767
+    out = []
+    for (st, gran), (oi, od, oq) in zip(((g.A, g.qa), (g.B, g.qb)), ref):
+        X = to_device(st)
+        q = imq.imq_rtn_quantize(X, gran, g.p, g.beta, out_dtype=torch.int32 if wide else torch.int16)
+        assert np.array_equal(q.xint.cpu().numpy().astype(np.int64), oi), f"{g.name} {st.name} ints"
+        assert np.array_equal(q.delta.cpu().numpy(), od) and np.array_equal(q.qval.cpu().numpy(), oq)
+        del X
+        out.append((q, oi, od))
+    return out
+
+
+def _check_gemm(imq, g, strategy, qa, qb, A, B, dA, dB, want=None, rows=None, check_unpack=True):
+    """A, B: logical oracle ints.  Returns the GPU plan info."""
+    pl = oracle.plan(A, B, g.b, strategy)
+    plan = imq.imq_plan(qa.xint, qb.xint, g.b, strategy, g.transA, g.transB,
+                        maxes=logical_maxes(imq, qa, qb, g.transA, g.transB))
+    plan_matches(plan.info, pl)
+    Au, Bu = imq.imq_unpack(plan, qa.xint, qb.xint)
+    if check_unpack:
+        oAu, oBu = oracle.unpack(pl, A, B)
+        assert np.array_equal(Au.cpu().numpy(), oAu), f"{g.name} A' bytes"
+        assert np.array_equal(Bu.cpu().numpy(), oBu), f"{g.name} B'^T bytes"
+        del oAu, oBu
+    gA, gB = g.gA, g.gB
+    C, Cf = imq.imq_gemm_unpacked(plan, Au, Bu, qa.delta, gA, qb.delta, gB,
+                                  c_dtype=torch.int32 if pl.acc_bits == 32 else torch.int64)
+    torch.cuda.synchronize()
+    assert imq.imq_device_status() == imq.IMQ_OK
+    got = C.cpu().numpy().astype(np.int64)
+    gotf = Cf.cpu().numpy()
+    if rows is not None:
+        got, gotf = got[rows], gotf[rows]
+        dAs = dA[rows] if gA == oracle.PER_ROW else dA
+    else:
+        dAs = dA
+    if want is None:
+        want = oracle.gemm_exact(A if rows is None else A[rows], B)
+    assert np.array_equal(got, want), f"{g.name} strategy {strategy}: {int((got != want).sum())} wrong"
+    assert_f32_close(gotf, oracle.dequant(want, dAs, gA, dB, gB))
+    info = plan.info
+    plan.destroy()
+    return info
+
+
+def _run(imq, g, strategies=None, rows=None, check_unpack=True):
+    (qa, ia, da), (qb, ib, db) = _quant_both(imq, g)
+    A, B = logical(ia, g.transA), logical(ib, g.transB)
+    want = None
+    infos = {}
+    for st in strategies or g.strategies:
+        if want is None and rows is None:
+            want = oracle.gemm_exact(A, B)
+        if rows is not None and want is None:
+            want = oracle.gemm_exact(A[rows], B)
+        infos[st] = _check_gemm(imq, g, st, qa, qb, A, B, da, db, want=want, rows=rows,
+                                check_unpack=check_unpack)
+    return infos
+
+
+def test_config_tiny(imq):
+    g = workloads.tiny()[0]
+    infos = _run(imq, g, strategies=[0, 1, 2, 3, 4])
+    assert infos[0]["ratio"] > 1.0
+
+
+def test_config_q_proj(imq):
+    g = workloads.q_proj()[0]
+    infos = _run(imq, g, strategies=[0, 1, 2, 3, 4])
+    assert infos[0]["dir_a"] == imq.IMQ_DIR_INNER  # column unpacking of the activations
+    assert infos[0]["ratio"] <= min(i["ratio"] for i in infos.values()) + 1e-12
+
+
+def test_config_mlp(imq):
+    rows = np.sort(np.random.default_rng(0).choice(2048, 512, replace=False))
+    for g in workloads.mlp():
+        _run(imq, g, rows=rows)
+
+
+@pytest.mark.parametrize("head", [0, 7, 19, 31])
+def test_config_attention(imq, head):
+    for g in workloads.attention_head(head):
+        _run(imq, g)
+
+
+def test_config_wgrad(imq):
+    for g in workloads.wgrad():
+        _run(imq, g, check_unpack=(g.b == 8))

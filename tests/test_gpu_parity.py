@@ -12,8 +12,7 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import (assert_f32_close, logical, plan_matches, slots_needed_unsupported,
-                              to_device)
+from tests.gpu_common import assert_f32_close, logical, plan_matches, to_device, unsupported
 
 pytestmark = pytest.mark.gpu
 
@@ -114,7 +113,7 @@ def _run_path(imq, A, B, b, strategy, transA, transB, dtype=torch.int16, check_u
     npdt = np.int16 if dtype == torch.int16 else np.int32
     Ad = torch.from_numpy(A_st.astype(npdt)).cuda()
     Bd = torch.from_numpy(B_st.astype(npdt)).cuda()
-    if slots_needed_unsupported(pl):
+    if unsupported(pl):
         with pytest.raises(imq.ImqError) as e:
             imq.imq_plan(Ad, Bd, b, strategy, transA, transB)
         assert e.value.status == imq.IMQ_ERR_UNSUPPORTED
@@ -153,7 +152,7 @@ def test_path_parity_int32_regime(imq, b, strategy, trans):
     _run_path(imq, A, B, b, strategy, *trans)
 
 
-@pytest.mark.parametrize("b", [3, 4, 5, 8])
+@pytest.mark.parametrize("b", [2, 3, 4, 5, 8])
 @pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4])
 def test_path_parity_int64_regime(imq, b, strategy):
     rng = np.random.default_rng(77 + 10 * b + strategy)
@@ -177,6 +176,16 @@ def test_path_parity_edge_shapes(imq, shape):
     A, B = workloads.random_case(rng, *shape, big=3000, frac=0.1)
     for st in range(5):
         _run_path(imq, A, B, 5, st, False, False)
+
+
+def test_path_group_split_along_k(imq):
+    """K = 140000 at b = 8: the e = 0 group could overflow one int32 accumulator (140000 * 127^2 >= 2^31)
+    and the bound does not rule it out, so the plan splits the group along K into two jobs."""
+    rng = np.random.default_rng(14)
+    A = rng.integers(-32767, 32768, size=(8, 140000)).astype(np.int64)
+    B = rng.integers(-32767, 32768, size=(140000, 16)).astype(np.int64)
+    plan = _run_path(imq, A, B, 8, 0, False, True)
+    assert plan.info["acc_bits"] == 64
 
 
 def test_path_int32_inputs(imq):
