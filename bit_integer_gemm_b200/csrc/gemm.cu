@@ -9,18 +9,22 @@
 //               swizzle, into a 4-stage shared-memory ring (mbarrier complete_tx).
 //   warp 1      MMA issuer (one thread): tcgen05.mma.cta_group::1.kind::i8, M=128 N=256 K=32,
 //               s8 x s8 -> s32 accumulators in tensor memory (TMEM).
-//   warps 2-5   epilogue: tcgen05.ld of the accumulators, fold-back, shift, accumulation into C,
-//               dequantisation.
-// The inner dimension is a sequence of exponent groups whose products carry the weight R^e.  Each group
-// of each tile is one accumulation job; jobs alternate between two 256-column TMEM slots, so the MMAs of
-// job n+1 run while the epilogue drains job n (also across tiles).  The epilogue folds the OUTER lines
-// of a job back with their level weights, shifts by e*(b-1) and adds the result into C (the first job of
-// a tile writes, later ones read-modify-write the tile they own; the last also writes the fp32 copy).
-// Every partial sum is a partial sum of the exact product, so it is bounded by the plan's bound: int32
-// when that is below 2^31, int64 otherwise.  The plan splits a group along K when its raw s32
-// accumulator could overflow.
+//   warps 2-5   epilogue: Horner rescales in TMEM, fold-back, dequantisation, stores.
+// The inner dimension is a sequence of exponent groups whose products carry the weight R^e.  A tile runs
+// them in descending e as steps into one 256-column TMEM slot; between two steps of a chunk the
+// epilogue multiplies the slot by R^(e_prev - e) in place (Horner's rule), at the end of a chunk it
+// drains the slot into C.  The plan proves every slot value stays below 2^31 (one chunk whenever the
+// product fits int32; chunks end only where the bound forces it, and their drains accumulate in C).
+// Two tiles run interleaved, step by step, one per TMEM slot: while the epilogue rescales or drains one
+// tile's slot, the tensor cores work on the other tile.
+// Drain: each epilogue warp owns one TMEM lane quarter = one group of 32 unpacked rows of A; a 32-column
+// chunk is one group of 32 unpacked columns of B.  Column levels of B are folded inside each thread's
+// registers, row levels of A across the lanes with shuffles, and the folded values are transposed
+// through shared memory so that every global access is coalesced along a row of C.
 // Every mbarrier wait is bounded (common.cuh): a stuck pipeline ends the kernel with IMQ_ERR_TIMEOUT.
 #include <string.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -33,15 +37,19 @@ constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK;  // bytes
 constexpr int B_STAGE = BN * BK;
 constexpr int NUM_THREADS = 192;
-constexpr int EPI_THREADS = 128;
+constexpr int EPI_WARPS = 4;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 struct GemmArgs {
   int32_t tiles_m, tiles_n;
-  int32_t n_jobs;
-  int32_t job_kb0[kMaxJobs];
-  int32_t job_nkb[kMaxJobs];
-  int8_t job_shift[kMaxJobs];
+  int32_t n_steps;
+  int32_t step_kb0[kMaxJobs];
+  int32_t step_nkb[kMaxJobs];
+  int8_t step_first[kMaxJobs];   // the step opens a chunk: its first MMA overwrites the slot
+  int8_t step_after[kMaxJobs];   // >= 0: Horner shift of the slot after the step; -1: drain
+  int8_t step_dshift[kMaxJobs];  // shift of the drained value (e of the chunk's last group times b-1)
+  int8_t step_dfirst[kMaxJobs];  // the drain is the tile's first: it writes C without reading it
+  int8_t step_dlast[kMaxJobs];   // the drain is the tile's last: it also writes Cf
   int32_t bm1;
   int32_t a_outer, b_outer;
   const int32_t* srcA;
@@ -67,15 +75,40 @@ struct GemmArgs {
 struct Smem {
   static constexpr size_t kA = 0;
   static constexpr size_t kB = kA + (size_t)STAGES * A_STAGE;
-  static constexpr size_t kStage = kB + (size_t)STAGES * B_STAGE;  // int32 [128][32], XOR-swizzled
-  static constexpr size_t kRsrc = kStage + (size_t)BM * 32 * 4;
-  static constexpr size_t kCsrc = kRsrc + BM * 4;
+  static constexpr size_t kScratch = kB + (size_t)STAGES * B_STAGE;  // per epilogue warp: [32][33] x 8 B
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr size_t kBars = kCsrc + 32 * 4;
-  static constexpr size_t kMisc = kBars + (2 * STAGES + 5) * 8;  // tmem base, abort flag, epilogue flag
+  static constexpr size_t kBars = kScratch + EPI_WARPS * 32 * 33 * 8;
+  static constexpr size_t kMisc = kBars + (2 * STAGES + 5) * 8;  // tmem base, abort flag
   static constexpr size_t kEnd = kMisc + 16;
   static constexpr size_t kBytes = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
+
+// x * 2^k in the two's-complement type T, through the unsigned type (the plan's bounds guarantee the
+// exact result fits T).
+template <typename T>
+__device__ __forceinline__ T shl(T x, int k) {
+  using U = typename std::make_unsigned<T>::type;
+  return (T)((U)x << k);
+}
+
+// Column fold of one 32-column chunk holding 32/L columns of level L: w[s] = sum_l R^l v[s L + l].
+template <int L, typename T>
+__device__ __forceinline__ void fold_cols(const uint32_t (&v)[32], T (&w)[32], int bm1) {
+#pragma unroll
+  for (int s = 0; s < 32 / L; ++s) {
+    T a = 0;
+#pragma unroll
+    for (int l = 0; l < L; ++l) a += shl<T>((T)(int32_t)v[s * L + l], l * bm1);
+    w[s] = a;
+  }
+}
+
+__device__ __forceinline__ int32_t shfl_t(int32_t x, int src) { return __shfl_sync(0xffffffffu, x, src); }
+__device__ __forceinline__ int64_t shfl_t(int64_t x, int src) {
+  const int lo = __shfl_sync(0xffffffffu, (int)(uint32_t)(uint64_t)x, src);
+  const int hi = __shfl_sync(0xffffffffu, (int)(uint32_t)((uint64_t)x >> 32), src);
+  return (int64_t)(((uint64_t)(uint32_t)hi << 32) | (uint32_t)lo);
+}
 
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
   const uint64_t t0 = global_ns();
@@ -84,21 +117,155 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
   return true;
 }
 
+// Drains one TMEM slot (this warp's 32 lanes) of tile (mt, nt) into C: fold, shift, write or add.
+template <typename T>
+__device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, uint32_t acce_bar, int mt, int nt,
+                                           int q, int lane, bool first, bool last, int shift, T* scr) {
+  // the source row lane t holds after the row fold (t < nA)
+  int LA, nA;
+  int64_t my_row;
+  if (g.a_outer) {
+    const int64_t grp = (int64_t)mt * (BM / 32) + q;
+    LA = g.grpA_L[grp];
+    nA = g.grpA_n[grp];
+    my_row = lane < nA ? g.srcA[grp * 32 + (int64_t)lane * LA] : 0;
+  } else {
+    LA = 1;
+    const int64_t r0 = (int64_t)mt * BM + q * 32;
+    const int64_t rem = g.M - r0;
+    nA = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
+    my_row = r0 + lane;
+  }
+  const float my_sa = (last && g.Cf && lane < nA) ? g.dA[g.dA_per_row ? my_row : 0] : 0.0f;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(tbase + c * 32, v);
+    tmem_wait_ld();
+    if (c == BN / 32 - 1) {
+      // the slot is fully read: the MMA warp may reuse it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar);
+    }
+    // columns of this chunk
+    const int64_t gc = (int64_t)nt * (BN / 32) + c;
+    int LB, nB;
+    if (g.b_outer) {
+      LB = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
+      nB = gc < g.n_grp_b ? g.grpB_n[gc] : 0;
+    } else {
+      LB = 1;
+      const int64_t rem = g.N - gc * 32;
+      nB = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
+    }
+    if (nB == 0 || nA == 0) continue;
+    // 1. fold the column levels of B inside the registers (lane = unpacked row)
+    T w[32];
+    switch (LB) {
+      case 1: fold_cols<1>(v, w, g.bm1); break;
+      case 2: fold_cols<2>(v, w, g.bm1); break;
+      case 3: fold_cols<3>(v, w, g.bm1); break;
+      case 4: fold_cols<4>(v, w, g.bm1); break;
+      case 5: fold_cols<5>(v, w, g.bm1); break;
+      case 6: fold_cols<6>(v, w, g.bm1); break;
+      case 7: fold_cols<7>(v, w, g.bm1); break;
+      case 8: fold_cols<8>(v, w, g.bm1); break;
+      default: {
+        // levels 9..31 (three columns at most): fold through the transpose buffer
+#pragma unroll
+        for (int k = 0; k < 32; ++k) scr[lane * 33 + k] = (T)(int32_t)v[k];
+        __syncwarp();
+#pragma unroll
+        for (int s2 = 0; s2 < 3; ++s2) {
+          T a = 0;
+          if (s2 < nB)
+            for (int l = 0; l < LB; ++l) a += shl<T>(scr[lane * 33 + s2 * LB + l], l * g.bm1);
+          w[s2] = a;
+        }
+        __syncwarp();
+      }
+    }
+    // 2. fold the row levels of A across the lanes: lane t gathers lanes t LA + l
+    if (g.a_outer && LA > 1) {
+#pragma unroll
+      for (int s2 = 0; s2 < 32; ++s2) {
+        if (s2 < nB) {
+          T a = 0;
+          for (int l = 0; l < LA; ++l) {
+            const int src = lane * LA + l;
+            a += shl<T>(shfl_t(w[s2], src < 32 ? src : 31), l * g.bm1);
+          }
+          w[s2] = a;
+        }
+      }
+    }
+    // 3. transpose through shared memory: scr[row][column]
+#pragma unroll
+    for (int s2 = 0; s2 < 32; ++s2)
+      if (s2 < nB) scr[lane * 33 + s2] = shl<T>(w[s2], shift);
+    __syncwarp();
+    // 4. lane = output column: coalesced accesses along each row of C
+    int64_t mycol = 0;
+    float my_sb = 0.0f;
+    if (lane < nB) {
+      mycol = g.b_outer ? g.srcB[gc * 32 + (int64_t)lane * LB] : gc * 32 + lane;
+      if (last && g.Cf) my_sb = g.dB[g.dB_per_col ? mycol : 0];
+    }
+    const bool col_ok = lane < nB;
+#pragma unroll 1
+    for (int r0 = 0; r0 < nA; r0 += 8) {
+      T val[8];
+      int64_t row[8];
+      float sa[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        row[u] = shfl_t(my_row, (r0 + u) & 31);
+        sa[u] = __shfl_sync(0xffffffffu, my_sa, (r0 + u) & 31);
+        val[u] = scr[((r0 + u) & 31) * 33 + lane];
+      }
+      if (!first && g.C && col_ok) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (r0 + u < nA) {
+            if (sizeof(T) == 8) val[u] += (T) static_cast<const int64_t*>(g.C)[row[u] * g.ldc + mycol];
+            else val[u] += (T) static_cast<const int32_t*>(g.C)[row[u] * g.ldc + mycol];
+          }
+      }
+      if (col_ok) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (r0 + u < nA) {
+            if (g.C) {
+              if (g.c64) static_cast<int64_t*>(g.C)[row[u] * g.ldc + mycol] = (int64_t)val[u];
+              else static_cast<int32_t*>(g.C)[row[u] * g.ldc + mycol] = (int32_t)val[u];
+            }
+            if (last && g.Cf)
+              g.Cf[row[u] * g.ldcf + mycol] =
+                  __fmul_rn(sizeof(T) == 8 ? __ll2float_rn((long long)val[u]) : __int2float_rn((int)val[u]),
+                            __fmul_rn(sa[u], my_sb));
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <bool kWide>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ GemmArgs g) {
   using L = Smem;
+  using T = typename std::conditional<kWide, int64_t, int32_t>::type;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base + L::kA;
   uint8_t* sB = base + L::kB;
-  int32_t* stg = reinterpret_cast<int32_t*>(base + L::kStage);
-  int32_t* s_rsrc = reinterpret_cast<int32_t*>(base + L::kRsrc);
-  int32_t* s_csrc = reinterpret_cast<int32_t*>(base + L::kCsrc);
+  T* scratch = reinterpret_cast<T*>(base + L::kScratch);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::kBars);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
-  volatile int* epi_ok = reinterpret_cast<volatile int*>(base + L::kMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + STAGES);
@@ -113,7 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(accf0 + 8 * s, 1);
-      mbar_init(acce0 + 8 * s, EPI_THREADS);
+      mbar_init(acce0 + 8 * s, EPI_WARPS);  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -133,6 +300,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = g.tiles_m * g.tiles_n;
+  // this CTA's tiles blockIdx.x + i * gridDim.x, taken in pairs (one per TMEM slot)
+  const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -141,20 +310,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued[STAGES];
       for (int s = 0; s < STAGES; ++s) issued[s] = 2;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
-        for (int j = 0; j < g.n_jobs; ++j) {
-          for (int kb = 0; kb < g.job_nkb[j]; ++kb) {
-            if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
-            const uint32_t fb = full0 + 8 * stage;
-            mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
-            const int32_t x = (g.job_kb0[j] + kb) * BK;
-            tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, x, mt * BM, fb);
-            tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, x, nt * BN, fb);
-            issued[stage] = phase;
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
+      for (int p = 0; p < my_tiles; p += 2) {
+        const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
+        for (int k = 0; k < g.n_steps; ++k) {
+          for (int x = 0; x < npair; ++x) {
+            const int tile = blockIdx.x + (p + x) * gridDim.x;
+            const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
+            for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
+              if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
+              const uint32_t fb = full0 + 8 * stage;
+              mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
+              const int32_t kx = (g.step_kb0[k] + kb) * BK;
+              tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, mt * BM, fb);
+              tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, nt * BN, fb);
+              issued[stage] = phase;
+              if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
           }
         }
@@ -172,33 +345,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_waits[2] = {0, 0};
-      uint32_t job_count = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        for (int j = 0; j < g.n_jobs; ++j, ++job_count) {
-          const uint32_t slot = job_count & 1u;
-          // the epilogue has drained the job this slot held before
-          if (!mbar_wait(acce0 + 8 * slot, (empty_waits[slot] & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns))
-            goto mma_done;
-          ++empty_waits[slot];
-          tc_fence_after();
-          const uint32_t d = tmem_base + slot * BN;
-          for (int kb = 0; kb < g.job_nkb[j]; ++kb) {
-            if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, g.status, g.timeout_ns)) goto mma_done;
+      for (int p = 0; p < my_tiles; p += 2) {
+        const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
+        for (int k = 0; k < g.n_steps; ++k) {
+          for (int slot = 0; slot < npair; ++slot) {
+            // the epilogue has finished the previous event of this slot (a rescale or a drain)
+            if (!mbar_wait(acce0 + 8 * slot, (empty_waits[slot] & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns))
+              goto mma_done;
+            ++empty_waits[slot];
             tc_fence_after();
-            const uint64_t adesc = smem_desc_k_sw128(smem_addr(sA + (size_t)stage * A_STAGE));
-            const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sB + (size_t)stage * B_STAGE));
+            const uint32_t d = tmem_base + (uint32_t)slot * BN;
+            const bool first = g.step_first[k] != 0;
+            for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
+              if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, g.status, g.timeout_ns)) goto mma_done;
+              tc_fence_after();
+              const uint64_t adesc = smem_desc_k_sw128(smem_addr(sA + (size_t)stage * A_STAGE));
+              const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sB + (size_t)stage * B_STAGE));
 #pragma unroll
-            for (int k = 0; k < BK / 32; ++k) {
-              // 32 bytes further along K inside the 128-byte swizzled row: +2 in the address field
-              mma_i8(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb == 0 && k == 0) ? 0u : 1u);
+              for (int kk = 0; kk < BK / 32; ++kk) {
+                // 32 bytes further along K inside the 128-byte swizzled row: +2 in the address field
+                mma_i8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (first && kb == 0 && kk == 0) ? 0u : 1u);
+              }
+              mma_commit(empty0 + 8 * stage);
+              if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
-            mma_commit(empty0 + 8 * stage);
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
-            }
+            mma_commit(accf0 + 8 * slot);
           }
-          mma_commit(accf0 + 8 * slot);
         }
       }
     mma_done:
@@ -209,100 +384,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;   // 0..127
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;     // accumulator row owned by this thread
+    const int q = warp & 3;  // TMEM lane quarter this warp may access = row group of the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    T* scr = scratch + q * 32 * 33;  // this warp's transpose buffer: [row][column], row stride 33
     uint32_t full_waits[2] = {0, 0};
-    uint32_t job_count = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
-      // source rows of this tile
-      int LA, nA;
-      if (g.a_outer) {
-        LA = g.grpA_L[mt];
-        nA = g.grpA_n[mt];
-        if (et < nA) s_rsrc[et] = g.srcA[(int64_t)mt * BM + (int64_t)et * LA];
-      } else {
-        LA = 1;
-        const int64_t rem = g.M - (int64_t)mt * BM;
-        nA = rem < BM ? (int)rem : BM;
-        if (et < nA) s_rsrc[et] = mt * BM + et;
-      }
-      for (int j = 0; j < g.n_jobs; ++j, ++job_count) {
-        const uint32_t slot = job_count & 1u;
-        // one thread waits and all 128 take its answer, so every epilogue thread passes the same named
-        // barriers even when a wait gives up
-        if (et == 0)
-          *epi_ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
-        named_bar_sync(1, EPI_THREADS);
-        const bool ok = *epi_ok != 0;
-        named_bar_sync(1, EPI_THREADS);
-        ++full_waits[slot];
-        if (!ok) goto epi_done;
-        tc_fence_after();
-        const bool first = j == 0, last = j == g.n_jobs - 1;
-        const int64_t mul = (int64_t)1 << g.job_shift[j];
+    for (int p = 0; p < my_tiles; p += 2) {
+      const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
+      for (int k = 0; k < g.n_steps; ++k) {
+        for (int slot = 0; slot < npair; ++slot) {
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++full_waits[slot];
+          if (!ok) goto epi_done;
+          tc_fence_after();
+          const uint32_t tbase = tmem_base + lane_off + (uint32_t)slot * BN;
+          if (g.step_after[k] >= 0) {
+            // Horner step: slot *= R^(e_prev - e), in place.  The plan bounds the result by 2^31, so
+            // a shift of 31 or more only meets zeros.
+            const int sh = g.step_after[k];
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem_base + lane_off + slot * BN + c * 32, v);
-          tmem_wait_ld();
+            for (int c = 0; c < BN / 32; ++c) {
+              uint32_t v[32];
+              tmem_ld32(tbase + c * 32, v);
+              tmem_wait_ld();
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) stg[row * 32 + (jj ^ lane)] = (int32_t)v[jj];
-          if (c == BN / 32 - 1) {
-            // the slot is fully read: let the MMA warp start the job after next in it
+              for (int jj = 0; jj < 32; ++jj) v[jj] = sh < 31 ? (v[jj] << sh) : 0u;
+              tmem_st32(tbase + c * 32, v);
+            }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(acce0 + 8 * slot);
-          }
-          // source columns of this 32-column chunk
-          const int64_t gc = (int64_t)nt * (BN / 32) + c;
-          int LB, nB;
-          if (g.b_outer) {
-            if (gc < g.n_grp_b) {
-              LB = g.grpB_L[gc];
-              nB = g.grpB_n[gc];
-            } else {
-              LB = 1;
-              nB = 0;
-            }
-            if (et < nB) s_csrc[et] = g.srcB[gc * 32 + (int64_t)et * LB];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce0 + 8 * slot);
           } else {
-            LB = 1;
-            const int64_t rem = g.N - gc * 32;
-            nB = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
-            if (et < nB) s_csrc[et] = (int32_t)(gc * 32 + et);
+            const int tile = blockIdx.x + (p + slot) * gridDim.x;
+            drain_slot<T>(g, tbase, acce0 + 8 * slot, tile % g.tiles_m, tile / g.tiles_m, q, lane,
+                          g.step_dfirst[k] != 0, g.step_dlast[k] != 0, g.step_dshift[k], scr);
           }
-          named_bar_sync(1, EPI_THREADS);
-          const int total = nA * nB;
-          for (int o = et; o < total; o += EPI_THREADS) {
-            const int r = o / nB, s = o - r * nB;
-            int64_t acc = 0;
-            for (int la = 0; la < LA; ++la) {
-              const int rr = r * LA + la;
-              for (int lb = 0; lb < LB; ++lb) {
-                const int cc = s * LB + lb;
-                acc += (int64_t)stg[rr * 32 + (cc ^ (rr & 31))] * ((int64_t)1 << ((la + lb) * g.bm1));
-              }
-            }
-            acc *= mul;
-            const int64_t i = s_rsrc[r], col = s_csrc[s];
-            // the same thread owns output (i, col) in every job of this tile
-            if (g.c64) {
-              int64_t* cp = static_cast<int64_t*>(g.C) + i * g.ldc + col;
-              if (!first) acc += *cp;
-              *cp = acc;
-            } else if (g.C) {
-              int32_t* cp = static_cast<int32_t*>(g.C) + i * g.ldc + col;
-              if (!first) acc += *cp;
-              *cp = (int32_t)acc;
-            }
-            if (last && g.Cf) {
-              const float sa = g.dA[g.dA_per_row ? i : 0], sb = g.dB[g.dB_per_col ? col : 0];
-              g.Cf[i * g.ldcf + col] = __fmul_rn(__ll2float_rn(acc), __fmul_rn(sa, sb));
-            }
-          }
-          named_bar_sync(1, EPI_THREADS);
         }
       }
     }
@@ -356,7 +474,7 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   if (Cf && gA != IMQ_PER_TENSOR && gA != IMQ_PER_ROW) return IMQ_ERR_ARG;
   if (Cf && gB != IMQ_PER_TENSOR && gB != IMQ_PER_COL) return IMQ_ERR_ARG;
   if (C && ct == IMQ_I32 && I.acc_bits > 32) return IMQ_ERR_RANGE;
-  if (!C && pl->n_jobs > 1) return IMQ_ERR_ARG;  // the jobs of a tile accumulate in C
+  if (!C && pl->n_chunks > 1) return IMQ_ERR_ARG;  // several chunks of a tile accumulate in C
   if (I.M == 0 || I.N == 0) return IMQ_OK;
   const size_t esz = ct == IMQ_I64 ? 8 : 4;
   if (I.K_unp == 0) {
@@ -377,12 +495,21 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   memset(&g, 0, sizeof(g));
   g.tiles_m = (int32_t)((I.M_unp + BM - 1) / BM);
   g.tiles_n = (int32_t)((I.N_unp + BN - 1) / BN);
-  g.n_jobs = pl->n_jobs;
-  for (int j = 0; j < pl->n_jobs; ++j) {
-    g.job_kb0[j] = (int32_t)(pl->job_k0[j] / BK);
-    g.job_nkb[j] = (int32_t)(pl->job_klen[j] / BK);
-    g.job_shift[j] = (int8_t)pl->job_shift[j];
+  g.n_steps = pl->n_steps;
+  int first_drain = -1, last_drain = -1;
+  for (int k = 0; k < pl->n_steps; ++k) {
+    g.step_kb0[k] = (int32_t)(pl->step_k0[k] / BK);
+    g.step_nkb[k] = (int32_t)(pl->step_klen[k] / BK);
+    g.step_first[k] = (int8_t)pl->step_first[k];
+    g.step_after[k] = (int8_t)pl->step_after[k];
+    g.step_dshift[k] = (int8_t)pl->step_drain_shift[k];
+    if (pl->step_after[k] < 0) {
+      if (first_drain < 0) first_drain = k;
+      last_drain = k;
+    }
   }
+  if (first_drain >= 0) g.step_dfirst[first_drain] = 1;
+  if (last_drain >= 0) g.step_dlast[last_drain] = 1;
   g.bm1 = I.b - 1;
   g.a_outer = I.dir_a == IMQ_DIR_OUTER;
   g.b_outer = I.dir_b == IMQ_DIR_OUTER;
@@ -410,8 +537,14 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   const int num_tiles = g.tiles_m * g.tiles_n;
   const int grid = num_tiles < ds->num_sms ? num_tiles : ds->num_sms;
   const size_t smem = Smem::kBytes;
-  IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_gemm<<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
+  // int64 accumulation in the epilogue whenever the output is int64 or the bound exceeds int32
+  if (g.c64 || I.acc_bits > 32) {
+    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_gemm<true><<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
+  } else {
+    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_gemm<false><<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
+  }
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 

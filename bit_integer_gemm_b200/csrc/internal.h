@@ -68,12 +68,18 @@ struct imq_plan {
   int32_t* grpB_n;
   int64_t n_grp_a, n_grp_b;
   imq_group groups[IMQ_MAX_GROUPS];
-  // GEMM schedule: each job accumulates one exponent group (or a K-slice of one) in a TMEM slot, and
-  // the epilogue adds (job value) << job_shift into C (see gemm.cu)
-  int32_t n_jobs;
-  int64_t job_k0[imq::kMaxJobs];    // first unpacked inner index (multiple of IMQ_INNER_PAD)
-  int64_t job_klen[imq::kMaxJobs];  // inner length (multiple of IMQ_INNER_PAD)
-  int32_t job_shift[imq::kMaxJobs]; // e * (b - 1)
+  // GEMM schedule of one output tile (see gemm.cu): a sequence of steps, each one exponent group (or a
+  // K-slice of one) accumulated into the tile's TMEM slot.  Consecutive steps of a chunk follow Horner's
+  // rule (the slot is multiplied by R^(e_prev - e) between them); at the end of a chunk the slot is
+  // drained into C, shifted by e_last * (b - 1).
+  int32_t n_steps;
+  int64_t step_k0[imq::kMaxJobs];     // first unpacked inner index (multiple of IMQ_INNER_PAD)
+  int64_t step_klen[imq::kMaxJobs];   // inner length (multiple of IMQ_INNER_PAD)
+  int32_t step_first[imq::kMaxJobs];  // 1: first step of its chunk (the MMA overwrites the slot)
+  int32_t step_after[imq::kMaxJobs];  // >= 0: left shift applied to the slot after this step (Horner);
+                                      // -1: the chunk ends here and the slot is drained
+  int32_t step_drain_shift[imq::kMaxJobs];
+  int32_t n_chunks;
 };
 
 namespace imq {

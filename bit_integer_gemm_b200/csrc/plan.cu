@@ -542,27 +542,52 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   I.acc_bits = bound < two31 ? 32 : 64;
   const int bm1 = b - 1;
   const unsigned __int128 R1 = ((unsigned __int128)1 << bm1) - 1;
-  // One accumulation job per exponent group.  The raw s32 accumulator of group e is bounded both by
-  // k_len * (R-1)^2 and by bound / R^e (R^e times it is a partial sum of the product); a group whose two
-  // bounds both reach 2^31 is split along K into slices of at most (2^31 - 1) / (R-1)^2 indices.
-  pl->n_jobs = 0;
-  for (int g = 0; g < ng; ++g) {
+  // Steps of one output tile, groups in descending exponent e.  A chunk accumulates consecutive groups
+  // by Horner's rule in one int32 TMEM slot; after its group of exponent e the slot holds
+  // sum_{e' >= e in chunk} R^(e'-e) C_e', which R^e times is a partial sum of the product, so it stays
+  // below bound / R^e: a group joins the current chunk only when bound / R^e < 2^31.  A group that opens
+  // a chunk needs its raw accumulator below 2^31: by its length (k_len (R-1)^2) or by the bound; when
+  // neither holds it is split along K into slices of (2^31 - 1) / (R-1)^2 indices, each its own chunk.
+  pl->n_steps = 0;
+  pl->n_chunks = 0;
+  auto below = [&](unsigned __int128 x, int sh) { return sh >= 127 ? true : (x >> sh) < two31; };
+  bool open_chunk = false;
+  for (int g = ng - 1; g >= 0; --g) {
     const imq_group& gr = pl->groups[g];
     const int sh = gr.e * bm1;
+    const bool fits_horner = below(bound, sh);
+    if (open_chunk && fits_horner) {
+      // Horner step: the previous step's slot is multiplied by R^(e_prev - e)
+      if (pl->n_steps >= kMaxJobs) return fail(IMQ_ERR_UNSUPPORTED);
+      const int i = pl->n_steps++;
+      pl->step_after[i - 1] = (pl->groups[g + 1].e - gr.e) * bm1;
+      pl->step_k0[i] = gr.k_offset;
+      pl->step_klen[i] = gr.k_len_padded;
+      pl->step_first[i] = 0;
+      pl->step_after[i] = -1;
+      pl->step_drain_shift[i] = sh;
+      // the drain of the chunk now happens after this step
+      continue;
+    }
+    // a new chunk (or several K-slice chunks)
     const unsigned __int128 by_len = (unsigned __int128)gr.k_len * R1 * R1;
-    const unsigned __int128 by_bound = sh >= 127 ? 0 : (bound >> sh);
     int64_t slice = gr.k_len_padded;
-    if (by_len >= two31 && by_bound >= two31) {
+    if (by_len >= two31 && !fits_horner) {
       slice = (int64_t)((two31 - 1) / (R1 * R1)) / IMQ_INNER_PAD * IMQ_INNER_PAD;
       if (slice < IMQ_INNER_PAD) return fail(IMQ_ERR_UNSUPPORTED);
     }
     for (int64_t k0 = 0; k0 < gr.k_len_padded; k0 += slice) {
-      if (pl->n_jobs >= kMaxJobs) return fail(IMQ_ERR_UNSUPPORTED);
-      const int j = pl->n_jobs++;
-      pl->job_k0[j] = gr.k_offset + k0;
-      pl->job_klen[j] = (gr.k_len_padded - k0) < slice ? (gr.k_len_padded - k0) : slice;
-      pl->job_shift[j] = sh;
+      if (pl->n_steps >= kMaxJobs) return fail(IMQ_ERR_UNSUPPORTED);
+      const int i = pl->n_steps++;
+      pl->step_k0[i] = gr.k_offset + k0;
+      pl->step_klen[i] = (gr.k_len_padded - k0) < slice ? (gr.k_len_padded - k0) : slice;
+      pl->step_first[i] = 1;
+      pl->step_after[i] = -1;
+      pl->step_drain_shift[i] = sh;
+      ++pl->n_chunks;
     }
+    // only a chunk whose state bound allows Horner can take further groups
+    open_chunk = fits_horner && slice == gr.k_len_padded;
   }
   I.workspace_bytes = align_up((size_t)(I.M_unp * I.K_unp), 1024) + align_up((size_t)(I.N_unp * I.K_unp), 1024);
 

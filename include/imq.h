@@ -73,7 +73,7 @@ typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2 } imq_dir;
 
 #define IMQ_MAX_GROUPS 64   /* exponent groups e = lA + lB of the inner dimension                         */
 #define IMQ_INNER_PAD 128   /* each exponent group of the unpacked inner dimension is padded to this      */
-#define IMQ_A_GROUP 128     /* OUTER-unpacked rows of A are packed in groups of this many unpacked rows   */
+#define IMQ_A_GROUP 32      /* OUTER-unpacked rows of A are packed in groups of this many unpacked rows   */
 #define IMQ_B_GROUP 32      /* OUTER-unpacked columns of B are packed in groups of this many columns      */
 
 /* ------------------------------------------------------------------------------------------------ */

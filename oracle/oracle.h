@@ -37,7 +37,7 @@
 
 #define OR_MAX_GROUPS 64
 #define OR_INNER_PAD 128
-#define OR_A_GROUP 128
+#define OR_A_GROUP 32
 #define OR_B_GROUP 32
 
 typedef struct {

@@ -375,7 +375,7 @@ def test_layout_follows_documented_order():
             assert want == sorted(want)
             # outer: per group one level L, floor(G/L) sources of that level, lines (src, l) in order
             for src, lvl, lines, G, dirv, outer in (
-                    (mp["srcA"], mp["lvlA"], lv["a_row"], 128, pl.dir_a, oracle.DIR_OUTER),
+                    (mp["srcA"], mp["lvlA"], lv["a_row"], 32, pl.dir_a, oracle.DIR_OUTER),
                     (mp["srcB"], mp["lvlB"], lv["b_col"], 32, pl.dir_b, oracle.DIR_OUTER)):
                 if dirv != outer:
                     assert np.array_equal(src, np.arange(src.size)) and not lvl.any()
