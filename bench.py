@@ -123,7 +123,7 @@ class Path:
         M, K, N = g.M, g.K, g.N
         t = torch
         self.Xint = t.empty((M, K), dtype=t.int16, device=dev)
-        self.Wint = t.empty((K, N), dtype=t.int16, device=dev)
+        self.Wint = t.empty((N, K), dtype=t.int16, device=dev)  # W quantised straight into B^T
         self.dX = t.empty(M, dtype=t.float32, device=dev)
         self.dW = t.empty(N, dtype=t.float32, device=dev)
         self.mx = [t.empty(n, dtype=t.int32, device=dev) for n in (M, K, K, N)]
@@ -138,8 +138,8 @@ class Path:
         imq.imq_rtn_quantize(self.X, imq.IMQ_PER_ROW, g.p, g.beta, Xint=self.Xint, delta=self.dX,
                              want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
         imq.imq_rtn_quantize(self.W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
-                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3])
-        plan = imq.imq_plan(self.Xint, self.Wint, g.b, imq.IMQ_MIX, maxes=self.mx)
+                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True)
+        plan = imq.imq_plan(self.Xint, self.Wint, g.b, imq.IMQ_MIX, transB=True, maxes=self.mx)
         I = plan.info
         if self.ws is None or self.ws.numel() < I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048:
             self.ws = self.torch.empty(I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048,

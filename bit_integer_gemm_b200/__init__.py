@@ -73,7 +73,8 @@ class imq_group(ctypes.Structure):
 # Names and argument types of every entry point of include/imq.h.
 _VP, _I32, _I64, _F64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
 SIGNATURES = {
-    "imq_rtn_quantize": [_VP, _I32, _I64, _I64, _I64, _I32, _F64, _I32, _VP, _I32, _I64, _VP, _VP, _VP, _VP, _VP],
+    "imq_rtn_quantize": [_VP, _I32, _I64, _I64, _I64, _I32, _F64, _I32, _VP, _I32, _I64, _I32, _VP, _VP, _VP, _VP,
+                         _VP],
     "imq_plan": [_VP, _VP, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32, _VP, _VP, _VP, _VP,
                  ctypes.POINTER(_VP), _VP],
     "imq_plan_info_get": [_VP, ctypes.POINTER(imq_plan_info)],
@@ -139,12 +140,13 @@ Quantized = namedtuple("Quantized", "xint delta qval rowmax colmax")
 
 def imq_rtn_quantize(X: torch.Tensor, gran: int, p: float, beta: int, out_dtype=torch.int16,
                      Xint=None, delta=None, qval=None, rowmax=None, colmax=None, want_qval=True,
-                     want_max=True, stream=None) -> Quantized:
-    """RTN quantisation of a stored 2-D matrix (fp32 or bf16) per tensor / stored row / stored column."""
+                     want_max=True, trans_out=False, stream=None) -> Quantized:
+    """RTN quantisation of a stored 2-D matrix (fp32 or bf16) per tensor / stored row / stored column.
+    trans_out writes the quantised matrix transposed (cols x rows)."""
     rows, cols = X.shape
     dev = X.device
     if Xint is None:
-        Xint = torch.empty((rows, cols), dtype=out_dtype, device=dev)
+        Xint = torch.empty((cols, rows) if trans_out else (rows, cols), dtype=out_dtype, device=dev)
     ng = 1 if gran == IMQ_PER_TENSOR else (rows if gran == IMQ_PER_ROW else cols)
     if delta is None:
         delta = torch.empty(ng, dtype=torch.float32, device=dev)
@@ -155,7 +157,8 @@ def imq_rtn_quantize(X: torch.Tensor, gran: int, p: float, beta: int, out_dtype=
     if colmax is None and want_max:
         colmax = torch.empty(cols, dtype=torch.int32, device=dev)
     st = lib().imq_rtn_quantize(_ptr(X), _TORCH_TO_IMQ[X.dtype], rows, cols, _ld(X), gran, float(p), int(beta),
-                                _ptr(Xint), _TORCH_TO_IMQ[Xint.dtype], _ld(Xint), _ptr(delta), _ptr(qval),
+                                _ptr(Xint), _TORCH_TO_IMQ[Xint.dtype], _ld(Xint), int(trans_out), _ptr(delta),
+                                _ptr(qval),
                                 _ptr(rowmax), _ptr(colmax), _stream(stream))
     _check(st, "imq_rtn_quantize")
     return Quantized(Xint, delta, qval, rowmax, colmax)

@@ -38,6 +38,43 @@ imq_status device_state(DeviceState** out) {
   return IMQ_OK;
 }
 
+imq_status partials_buffer(DeviceState* ds, size_t bytes, void** out) {
+  if (bytes > ds->partials_bytes) {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (bytes > ds->partials_bytes) {
+      if (ds->partials) IMQ_CUDA_TRY(cudaFree(ds->partials));
+      ds->partials = nullptr;
+      ds->partials_bytes = 0;
+      const size_t n = (bytes + (1 << 20) - 1) >> 20 << 20;
+      IMQ_CUDA_TRY(cudaMalloc(&ds->partials, n));
+      ds->partials_bytes = n;
+    }
+  }
+  *out = ds->partials;
+  return IMQ_OK;
+}
+
+namespace {
+__global__ void k_reduce_max(const int32_t* __restrict__ part, int64_t nparts, int64_t n, int32_t* __restrict__ out) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    int32_t m = 0;
+    for (int64_t p = 0; p < nparts; ++p) m = max(m, __ldcs(part + p * n + i));
+    out[i] = m;
+  }
+}
+}  // namespace
+
+imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st) {
+  if (n == 0) return IMQ_OK;
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  int64_t grid = (n + 255) / 256;
+  if (grid > ds->num_sms * 4) grid = ds->num_sms * 4;
+  k_reduce_max<<<(unsigned)grid, 256, 0, st>>>(part, nparts, n, out);
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
 }  // namespace imq
 
 using imq::DeviceState;
@@ -45,9 +82,9 @@ using imq::DeviceState;
 extern "C" {
 
 imq_status imq_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld, imq_gran g,
-                            double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq, float* delta,
-                            float* qval, int32_t* rowmax, int32_t* colmax, imq_stream_t stream) {
-  return imq::launch_rtn_quantize(X, xt, rows, cols, ld, g, p, beta, Xint, it, ldq, delta, qval, rowmax,
+                            double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq, int32_t trans_out,
+                            float* delta, float* qval, int32_t* rowmax, int32_t* colmax, imq_stream_t stream) {
+  return imq::launch_rtn_quantize(X, xt, rows, cols, ld, g, p, beta, Xint, it, ldq, trans_out, delta, qval, rowmax,
                                   colmax, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -212,6 +212,17 @@ __device__ __forceinline__ int32_t digit_of(int32_t v, int32_t l, int32_t bm1) {
   return v < 0 ? -d : d;
 }
 
+// Warp-aggregated shared-memory increment: lanes with equal keys add their count once, so a hot bin
+// costs one atomic per warp instead of one per lane.  Every lane of the warp must call it; `active`
+// lanes contribute.
+__device__ __forceinline__ void warp_count(uint32_t* base, uint32_t key, bool active) {
+  const unsigned act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const unsigned peers = __match_any_sync(act, key);
+  const int leader = __ffs(peers) - 1;
+  if ((int)(threadIdx.x & 31) == leader) atomicAdd(base + key, (uint32_t)__popc(peers));
+}
+
 // Number of base-2^(b-1) digits of m (>= 1).
 __device__ __forceinline__ int32_t level_of(uint32_t m, int32_t bm1) {
   if (m == 0) return 1;

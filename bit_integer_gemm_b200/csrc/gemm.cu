@@ -55,6 +55,7 @@ struct GemmArgs {
   const int32_t* srcA;
   const int32_t* grpA_L;
   const int32_t* grpA_n;
+  int64_t n_grp_a;  // row groups of A' (the last tile may hold fewer than BM / 32)
   const int32_t* srcB;
   const int32_t* grpB_L;
   const int32_t* grpB_n;
@@ -126,8 +127,8 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
   int64_t my_row;
   if (g.a_outer) {
     const int64_t grp = (int64_t)mt * (BM / 32) + q;
-    LA = g.grpA_L[grp];
-    nA = g.grpA_n[grp];
+    LA = grp < g.n_grp_a ? g.grpA_L[grp] : 1;
+    nA = grp < g.n_grp_a ? g.grpA_n[grp] : 0;
     my_row = lane < nA ? g.srcA[grp * 32 + (int64_t)lane * LA] : 0;
   } else {
     LA = 1;
@@ -516,6 +517,7 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   g.srcA = pl->srcA;
   g.grpA_L = pl->grpA_L;
   g.grpA_n = pl->grpA_n;
+  g.n_grp_a = pl->n_grp_a;
   g.srcB = pl->srcB;
   g.grpB_L = pl->grpB_L;
   g.grpB_n = pl->grpB_n;

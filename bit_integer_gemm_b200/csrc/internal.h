@@ -14,16 +14,23 @@ constexpr int kMaxJobs = 128;  // accumulation jobs of one output tile
 // Per-device state owned by the library: the status word address and small scratch buffers.
 struct DeviceState {
   int32_t* status = nullptr;   // device address of the status word of this device
-  void* scratch = nullptr;     // per-tensor quantiser scratch (allocated on first use)
+  void* scratch = nullptr;     // per-tensor quantiser state (allocated on first use)
+  void* partials = nullptr;    // per-CTA partial line maxima of the quantiser (grown on demand)
+  size_t partials_bytes = 0;
   int num_sms = 0;
   bool init = false;
 };
 imq_status device_state(DeviceState** out);
+// Returns a device buffer of at least `bytes` for per-CTA partial results (grown on first need; a
+// growth frees the old buffer, which waits for the device).
+imq_status partials_buffer(DeviceState* ds, size_t bytes, void** out);
+// out[i] = max over p < nparts of part[p * n + i] (int32, non-negative); nparts may be 0 (out = 0).
+imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st);
 
 // Percentile + RTN quantisation (rtn.cu).
 imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                imq_gran g, double p, int32_t beta, void* Xint, imq_dtype it,
-                               int64_t ldq, float* delta, float* qval, int32_t* rowmax,
+                               int64_t ldq, int32_t trans_out, float* delta, float* qval, int32_t* rowmax,
                                int32_t* colmax, cudaStream_t stream);
 
 // Line maxima of an integer matrix (plan.cu): logical rows and columns of a stored matrix.

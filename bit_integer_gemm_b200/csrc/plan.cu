@@ -107,31 +107,64 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   unsigned int blmax[4] = {0, 0, 0, 0};
   unsigned __int128 bound = 0;
   for (int v = 0; v < 4; ++v) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + tid; i < a.n[v]; i += stride) {
-      const uint32_t m = (uint32_t)a.mx[v][i];
-      const int L = level_of(m, a.bm1);
-      a.lv[v][i] = (int8_t)L;
-      bsum[v] += (unsigned)L;
-      boor[v] += (L > 1);
-      blmax[v] = max(blmax[v], (unsigned)L);
-      atomicAdd(&hist[v][L], 1u);
+    // whole warps iterate together so the aggregated counters see every lane
+    for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x; i0 < a.n[v]; i0 += stride) {
+      const int64_t i = i0 + tid;
+      const bool in = i < a.n[v];
+      int L = 1;
+      if (in) {
+        const uint32_t m = (uint32_t)a.mx[v][i];
+        L = level_of(m, a.bm1);
+        a.lv[v][i] = (int8_t)L;
+        bsum[v] += (unsigned)L;
+        boor[v] += (L > 1);
+        blmax[v] = max(blmax[v], (unsigned)L);
+        if (v == 1) bound += (unsigned __int128)((unsigned long long)m * (unsigned long long)(uint32_t)a.mx[2][i]);
+      }
+      warp_count(&hist[v][0], (uint32_t)L, in);
       if (v == 1) {
-        const uint32_t mb = (uint32_t)a.mx[2][i];
-        atomicAdd(&joint[L][level_of(mb, a.bm1)], 1u);
-        bound += (unsigned __int128)((unsigned long long)m * (unsigned long long)mb);
+        const int Lb = in ? level_of((uint32_t)a.mx[2][i], a.bm1) : 1;
+        warp_count(&joint[0][0], (uint32_t)(L * kLv + Lb), in);
       }
     }
   }
-  for (int v = 0; v < 4; ++v) {
-    if (bsum[v]) atomicAdd(&ssum[v], bsum[v]);
-    if (boor[v]) atomicAdd(&soor[v], boor[v]);
-    if (blmax[v]) atomicMax(&slmax[v], blmax[v]);
+  // warp reductions first, then one shared atomic per warp, then one global atomic per block
+  unsigned long long blo = (unsigned long long)bound, bhi = (unsigned long long)(bound >> 64);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    for (int v = 0; v < 4; ++v) {
+      bsum[v] += __shfl_xor_sync(0xffffffffu, bsum[v], o);
+      boor[v] += __shfl_xor_sync(0xffffffffu, boor[v], o);
+      blmax[v] = max(blmax[v], __shfl_xor_sync(0xffffffffu, blmax[v], o));
+    }
+    const unsigned long long ol = __shfl_xor_sync(0xffffffffu, blo, o);
+    const unsigned long long oh = __shfl_xor_sync(0xffffffffu, bhi, o);
+    const unsigned long long nl = blo + ol;
+    bhi += oh + (nl < blo ? 1ull : 0ull);
+    blo = nl;
   }
-  if (bound) {
-    const unsigned long long lo = (unsigned long long)bound, hi = (unsigned long long)(bound >> 64);
-    const unsigned long long old = atomicAdd(&a.sum->bound_lo, lo);
-    const unsigned long long carry = (old + lo < old) ? 1ull : 0ull;
-    if (hi + carry) atomicAdd(&a.sum->bound_hi, hi + carry);
+  __shared__ unsigned long long sblo, sbhi;
+  if (tid == 0) {
+    sblo = 0;
+    sbhi = 0;
+  }
+  __syncthreads();
+  if ((tid & 31) == 0) {
+    for (int v = 0; v < 4; ++v) {
+      if (bsum[v]) atomicAdd(&ssum[v], bsum[v]);
+      if (boor[v]) atomicAdd(&soor[v], boor[v]);
+      if (blmax[v]) atomicMax(&slmax[v], blmax[v]);
+    }
+    if (blo || bhi) {
+      const unsigned long long old = atomicAdd(&sblo, blo);
+      atomicAdd(&sbhi, bhi + ((old + blo < old) ? 1ull : 0ull));
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && (sblo || sbhi)) {
+    const unsigned long long old = atomicAdd(&a.sum->bound_lo, sblo);
+    const unsigned long long hi = sbhi + ((old + sblo < old) ? 1ull : 0ull);
+    if (hi) atomicAdd(&a.sum->bound_hi, hi);
   }
   __syncthreads();
   if (tid < 4) {

@@ -8,13 +8,18 @@
 // pattern of a non-negative float orders like an unsigned integer), 8 key bits per pass from the top.
 //
 // Kernels
-//   k_rtn_rows    one CTA per stored row (grid-stride): the row is staged in shared memory once, the
-//                 select passes and the quantisation read it from there (one HBM read, one write).
+//   k_rtn_rows    one warp per stored row: the row is staged in the warp's shared-memory buffer once,
+//                 the select passes and the quantisation read it from there (one HBM read, one write).
 //                 Also used for per-tensor groups with the scale taken from the tensor select.
-//   k_rtn_cols    one CTA per 16 stored columns: histograms per column in shared memory, the column
-//                 slab is streamed once per pass (re-reads hit L2) and once more to quantise.
+//   k_rtn_cols_staged  one CTA per 16 (or 8) stored columns: the column slab is staged in shared
+//                 memory (one HBM read), per-column histograms in shared memory, optional transposed
+//                 output (a K x N weight quantised per output channel straight into N x K).
+//   k_rtn_cols    the same for columns too tall to stage: the slab is streamed once per pass (re-reads
+//                 hit L2) and once more to quantise.
 //   k_tensor_*    per-tensor select: global 256-bin histograms per pass, then k_rtn_rows.
-// Side outputs: max |x_int| per stored row and column, the line statistics the unpack plan needs.
+// Side outputs: max |x_int| per stored row and column, the line statistics the unpack plan needs.  The
+// maxima that cross CTAs are written as per-CTA partials to a library scratch buffer and reduced by a
+// second small kernel (no global atomics).
 #include <math.h>
 
 #include "common.cuh"
@@ -157,120 +162,253 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// per stored row (kSelect) or per tensor (scale from the tensor state)
+// per stored row (kSelect) or per tensor (scale from the tensor state): one warp per row.  Each warp
+// stages its row in its own shared-memory buffer, builds its own 256-bin histograms (warp-aggregated
+// increments) and selects with warp scans, so no block barrier is involved.  Column maxima of the
+// CTA's rows are kept in shared memory and written once per CTA to `part` (reduced afterwards).
 // ------------------------------------------------------------------------------------------------
 template <typename T, bool kSelect, bool kOut16>
 __global__ void __launch_bounds__(kThreads) k_rtn_rows(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
-    void* __restrict__ Xint, int64_t ldq, float* __restrict__ delta, float* __restrict__ qval,
-    int32_t* __restrict__ rowmax, int32_t* __restrict__ colmax, const TensorState* __restrict__ ts,
-    int vec, int32_t* status) {
+    void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
+    int32_t* __restrict__ rowmax, int32_t* __restrict__ part, const TensorState* __restrict__ ts, int vec,
+    int nwarps, int32_t* status) {
   extern __shared__ __align__(16) unsigned char dsm[];
-  T* row = reinterpret_cast<T*>(dsm);
   const int64_t row_bytes = (cols * (int64_t)sizeof(T) + 15) / 16 * 16;
-  uint32_t* cmax = reinterpret_cast<uint32_t*>(dsm + row_bytes);
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t red[kThreads / 32];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ unsigned long long s_k;
-  __shared__ float s_s;
-  __shared__ int s_ok;
-  const int tid = threadIdx.x;
+  uint32_t* cmax = reinterpret_cast<uint32_t*>(dsm);                  // [cols]
+  const int64_t cmax_bytes = part ? (cols * 4 + 15) / 16 * 16 : 0;  // same layout as the host
+  __shared__ uint32_t hist_all[kThreads / 32][256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  T* row = reinterpret_cast<T*>(dsm + cmax_bytes + warp * row_bytes);
+  uint32_t* hist = hist_all[warp];
   constexpr int V = 16 / sizeof(T);
-
-  if (colmax)
-    for (int64_t c = tid; c < cols; c += kThreads) cmax[c] = 0;
-
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const T* xr = X + r * ld;
-    uint32_t mk = 0, bad = 0;
-    if (vec) {
-      const uint4* src = reinterpret_cast<const uint4*>(xr);
-      uint4* dst = reinterpret_cast<uint4*>(row);
-      for (int64_t c = tid; c < cols / V; c += kThreads) {
-        const uint4 w = __ldcs(src + c);
-        dst[c] = w;
-        const T* e = reinterpret_cast<const T*>(&w);
+  if (part)
+    for (int64_t c = tid; c < cols; c += blockDim.x) cmax[c] = 0;
+  __syncthreads();
+  if (warp < nwarps) {
+    for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < rows; r += (int64_t)gridDim.x * nwarps) {
+      const T* xr = X + r * ld;
+      uint32_t mk = 0, bad = 0;
+      if (vec) {
+        const uint4* src = reinterpret_cast<const uint4*>(xr);
+        uint4* dst = reinterpret_cast<uint4*>(row);
+        for (int64_t c = lane; c < cols / V; c += 32) {
+          const uint4 w = __ldcs(src + c);
+          dst[c] = w;
+          const T* e = reinterpret_cast<const T*>(&w);
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
-          const uint32_t k = Key<T>::key(e[j]);
+          for (int j = 0; j < V; ++j) {
+            const uint32_t k = Key<T>::key(e[j]);
+            mk = max(mk, k);
+            bad |= (k >= Key<T>::kInf);
+          }
+        }
+      } else {
+        for (int64_t c = lane; c < cols; c += 32) {
+          const T u = xr[c];
+          row[c] = u;
+          const uint32_t k = Key<T>::key(u);
           mk = max(mk, k);
           bad |= (k >= Key<T>::kInf);
         }
       }
-    } else {
-      for (int64_t c = tid; c < cols; c += kThreads) {
-        const T u = xr[c];
-        row[c] = u;
-        const uint32_t k = Key<T>::key(u);
-        mk = max(mk, k);
-        bad |= (k >= Key<T>::kInf);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+        bad |= __shfl_xor_sync(0xffffffffu, bad, o);
       }
-    }
-    mk = block_max_u32(mk, red);
-    bad = block_max_u32(bad, red);
-
-    if (kSelect) {
-      if (tid == 0) {
-        s_prefix = 0;
-        s_mask = 0;
-        s_k = krank;
-      }
-      for (int pass = 0; pass < num_passes(Key<T>::kBits); ++pass) {
-        hist[tid] = 0;
-        __syncthreads();
-        const uint32_t pre = s_prefix, msk = s_mask;
-        const int sh = pass_shift(Key<T>::kBits, pass);
-        for (int64_t c = tid; c < cols; c += kThreads) {
-          const uint32_t k = Key<T>::key(row[c]);
-          if ((k & msk) == pre) atomicAdd(&hist[(k >> sh) & 0xFFu], 1u);
-        }
-        __syncthreads();
-        if (tid < 32) {
+      __syncwarp();
+      float s;
+      if (kSelect) {
+        uint32_t pre = 0, msk = 0;
+        unsigned long long kk = krank;
+        for (int pass = 0; pass < num_passes(Key<T>::kBits); ++pass) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+          __syncwarp();
+          const int sh = pass_shift(Key<T>::kBits, pass);
+          for (int64_t c0 = 0; c0 < cols; c0 += 32) {
+            const int64_t c = c0 + lane;
+            const uint32_t k = c < cols ? Key<T>::key(row[c]) : 0u;
+            warp_count(hist, (k >> sh) & 0xFFu, c < cols && (k & msk) == pre);
+          }
+          __syncwarp();
           int d;
           unsigned long long below;
-          if (warp_select(hist, 1, s_k, &d, &below)) {
-            s_prefix = pre | ((uint32_t)d << sh);
-            s_mask = msk | (pass_width_mask(Key<T>::kBits, pass) << sh);
-            s_k -= below;
-          }
+          warp_select(hist, 1, kk, &d, &below);
+          d = __shfl_sync(0xffffffffu, d, 0);
+          below = __shfl_sync(0xffffffffu, below, 0);
+          pre |= (uint32_t)d << sh;
+          msk |= pass_width_mask(Key<T>::kBits, pass) << sh;
+          kk -= below;
+          __syncwarp();
         }
-        __syncthreads();
-      }
-    }
-    if (tid == 0) {
-      float s, d;
-      if (kSelect) {
-        const float q = Key<T>::from_key(s_prefix);
-        scale_from_q(q, Key<T>::from_key(mk), beta, &s, &d);
-        delta[r] = d;
-        if (qval) qval[r] = q;
+        const float q = Key<T>::from_key(pre);
+        float dl;
+        scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
+        if (lane == 0) {
+          delta[r] = dl;
+          if (qval) qval[r] = q;
+        }
       } else {
         s = ts->s;
       }
-      if (bad) set_status(status, IMQ_ERR_NONFINITE);
-      s_s = s;
-      s_ok = !bad;
+      if (bad) {
+        if (lane == 0) set_status(status, IMQ_ERR_NONFINITE);
+        continue;
+      }
+      uint32_t rmx = 0;
+      for (int64_t c = lane; c < cols; c += 32) {
+        const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
+                                             status);
+        rmx = max(rmx, a);
+        if (part && a) atomicMax(&cmax[c], a);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) rmx = max(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
+      if (lane == 0 && rowmax) rowmax[r] = (int32_t)rmx;
+      __syncwarp();
+    }
+  }
+  if (part) {
+    __syncthreads();
+    int32_t* mine = part + (int64_t)blockIdx.x * cols;
+    for (int64_t c = tid; c < cols; c += blockDim.x) mine[c] = (int32_t)cmax[c];
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// per stored column, slab staged in shared memory: CW columns x all rows are read from HBM once; the
+// select passes and the quantisation read shared memory.  With trans_out the quantised slab is written
+// transposed (column c of X becomes row c of Xint), with coalesced stores along it.
+// ------------------------------------------------------------------------------------------------
+template <typename T, int CW, bool kOut16>
+__global__ void __launch_bounds__(kThreads) k_rtn_cols_staged(
+    const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
+    void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
+    int32_t* __restrict__ part, int32_t* __restrict__ colmax, int vec, int32_t* status) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  T* S = reinterpret_cast<T*>(dsm);  // [rows][CW]
+  int32_t* prow = part ? part + (int64_t)blockIdx.x * rows : nullptr;  // this CTA's row maxima
+  __shared__ uint32_t hist[256 * CW];  // [bucket][column]
+  __shared__ uint32_t s_prefix[CW], s_mask[CW], s_maxkey[CW], s_cmax[CW];
+  __shared__ unsigned long long s_k[CW];
+  __shared__ float s_s[CW];
+  __shared__ uint32_t s_bad;
+  const int tid = threadIdx.x, cc = tid % CW;
+  const int64_t c0 = (int64_t)blockIdx.x * CW;
+  const int ncol = cols - c0 < CW ? (int)(cols - c0) : CW;
+  if (tid < CW) {
+    s_prefix[tid] = 0;
+    s_mask[tid] = 0;
+    s_maxkey[tid] = 0;
+    s_cmax[tid] = 0;
+    s_k[tid] = krank;
+  }
+  if (tid == 0) s_bad = 0;
+  // stage the slab (columns past the end read as zero)
+  constexpr int V = 16 / sizeof(T);
+  if (vec && ncol == CW) {
+    constexpr int SEG = CW / V;  // 16-byte pieces per row
+    for (int64_t i = tid; i < rows * SEG; i += kThreads) {
+      const int64_t r = i / SEG;
+      const int sg = (int)(i % SEG);
+      reinterpret_cast<uint4*>(S)[i] = __ldcs(reinterpret_cast<const uint4*>(X + r * ld + c0) + sg);
+    }
+  } else {
+    for (int64_t i = tid; i < rows * CW; i += kThreads) {
+      const int64_t r = i / CW;
+      const int k = (int)(i % CW);
+      S[i] = k < ncol ? X[r * ld + c0 + k] : (T)0;
+    }
+  }
+  __syncthreads();
+  // every thread sees one column: i % CW == tid % CW because kThreads is a multiple of CW
+  uint32_t mk = 0, bad = 0;
+  for (int64_t i = tid; i < rows * CW; i += kThreads) {
+    const uint32_t k = Key<T>::key(S[i]);
+    mk = max(mk, k);
+    bad |= (k >= Key<T>::kInf);
+  }
+  if (mk) atomicMax(&s_maxkey[cc], mk);
+  if (bad) atomicOr(&s_bad, 1u);
+  for (int pass = 0; pass < num_passes(Key<T>::kBits); ++pass) {
+    for (int i = tid; i < 256 * CW; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    const uint32_t pre = s_prefix[cc], msk = s_mask[cc];
+    const int sh = pass_shift(Key<T>::kBits, pass);
+    // bins are [bucket][column]: the lanes of a warp mostly hit different columns
+    for (int64_t i = tid; i < rows * CW; i += kThreads) {
+      const uint32_t k = Key<T>::key(S[i]);
+      if ((k & msk) == pre) atomicAdd(&hist[((k >> sh) & 0xFFu) * CW + cc], 1u);
     }
     __syncthreads();
-    const float s = s_s;
-    uint32_t rmx = 0;
-    if (s_ok) {
-      for (int64_t c = tid; c < cols; c += kThreads) {
-        const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint, r * ldq + c, status);
-        rmx = max(rmx, a);
-        if (colmax) cmax[c] = max(cmax[c], a);
+    for (int col = tid >> 5; col < CW; col += kThreads / 32) {
+      int d;
+      unsigned long long below;
+      if (warp_select(hist + col, CW, s_k[col], &d, &below)) {
+        s_prefix[col] = s_prefix[col] | ((uint32_t)d << sh);
+        s_mask[col] = s_mask[col] | (pass_width_mask(Key<T>::kBits, pass) << sh);
+        s_k[col] -= below;
       }
     }
-    rmx = block_max_u32(rmx, red);
-    if (tid == 0 && rowmax) rowmax[r] = (int32_t)rmx;
     __syncthreads();
   }
-  if (colmax) {
-    __syncthreads();
-    for (int64_t c = tid; c < cols; c += kThreads)
-      if (cmax[c]) atomicMax(colmax + c, (int32_t)cmax[c]);
+  if (tid < ncol) {
+    float s, d;
+    const float q = Key<T>::from_key(s_prefix[tid]);
+    scale_from_q(q, Key<T>::from_key(s_maxkey[tid]), beta, &s, &d);
+    delta[c0 + tid] = d;
+    if (qval) qval[c0 + tid] = q;
+    s_s[tid] = s;
   }
+  if (tid == 0 && s_bad) set_status(status, IMQ_ERR_NONFINITE);
+  __syncthreads();
+  if (s_bad) return;
+  if (!trans_out) {
+    uint32_t cmx = 0;
+    const float s = cc < ncol ? s_s[cc] : 0.0f;
+    for (int64_t i0 = 0; i0 < rows * CW; i0 += kThreads) {
+      const int64_t i = i0 + tid;
+      const int64_t r = i / CW;
+      uint32_t a = 0;
+      if (i < rows * CW && cc < ncol) {
+        a = quant_one<kOut16>(Key<T>::value(S[i]), s, Xint, r * ldq + c0 + cc, status);
+        cmx = max(cmx, a);
+      }
+#pragma unroll
+      for (int o = CW / 2; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if (prow && cc == 0 && i < rows * CW) prow[r] = (int32_t)a;
+    }
+    atomicMax(&s_cmax[cc], cmx);
+  } else {
+    // row r of the slab is entry r of output rows c0 .. c0+ncol-1
+    uint32_t cm[CW];
+#pragma unroll
+    for (int k = 0; k < CW; ++k) cm[k] = 0;
+    for (int64_t r = tid; r < rows; r += kThreads) {
+      uint32_t rmx = 0;
+#pragma unroll
+      for (int k = 0; k < CW; ++k) {
+        if (k < ncol) {
+          const uint32_t a =
+              quant_one<kOut16>(Key<T>::value(S[r * CW + k]), s_s[k], Xint, (c0 + k) * ldq + r, status);
+          rmx = max(rmx, a);
+          cm[k] = max(cm[k], a);
+        }
+      }
+      if (prow) prow[r] = (int32_t)rmx;
+    }
+#pragma unroll
+    for (int k = 0; k < CW; ++k) {
+      uint32_t m = cm[k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if ((tid & 31) == 0 && m) atomicMax(&s_cmax[k], m);
+    }
+  }
+  __syncthreads();
+  if (colmax && tid < ncol) colmax[c0 + tid] = (int32_t)s_cmax[tid];
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -279,9 +417,10 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
 template <typename T, bool kOut16>
 __global__ void __launch_bounds__(kThreads) k_rtn_cols(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
-    void* __restrict__ Xint, int64_t ldq, float* __restrict__ delta, float* __restrict__ qval,
-    int32_t* __restrict__ rowmax, int32_t* __restrict__ colmax, int32_t* status) {
+    void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
+    int32_t* __restrict__ part, int32_t* __restrict__ colmax, int32_t* status) {
   constexpr int CW = kColsPerCta;
+  int32_t* prow = part ? part + (int64_t)blockIdx.x * rows : nullptr;  // this CTA's row maxima
   constexpr int RS = kThreads / CW;  // rows per sweep
   __shared__ uint32_t hist[256 * CW];  // [bucket][column]
   __shared__ uint32_t s_prefix[CW], s_mask[CW], s_maxkey[CW], s_cmax[CW];
@@ -305,15 +444,15 @@ __global__ void __launch_bounds__(kThreads) k_rtn_cols(
     const uint32_t pre = s_prefix[cc], msk = s_mask[cc];
     const int sh = pass_shift(Key<T>::kBits, pass);
     uint32_t mk = 0, bad = 0;
-    if (cval) {
-      for (int64_t r = rsub; r < rows; r += RS) {
-        const uint32_t k = Key<T>::key(X[r * ld + c]);
-        if (pass == 0) {
-          mk = max(mk, k);
-          bad |= (k >= Key<T>::kInf);
-        }
-        if ((k & msk) == pre) atomicAdd(&hist[((k >> sh) & 0xFFu) * CW + cc], 1u);
+    for (int64_t r0 = 0; r0 < rows; r0 += RS) {
+      const int64_t r = r0 + rsub;
+      const bool in = cval && r < rows;
+      const uint32_t k = in ? Key<T>::key(X[r * ld + c]) : 0u;
+      if (pass == 0 && in) {
+        mk = max(mk, k);
+        bad |= (k >= Key<T>::kInf);
       }
+      warp_count(hist, ((k >> sh) & 0xFFu) * CW + cc, in && (k & msk) == pre);
     }
     if (pass == 0) {
       if (mk) atomicMax(&s_maxkey[cc], mk);
@@ -350,13 +489,13 @@ __global__ void __launch_bounds__(kThreads) k_rtn_cols(
     const int64_t r = r0 + rsub;
     uint32_t a = 0;
     if (cval && r < rows) {
-      a = quant_one<kOut16>(Key<T>::value(X[r * ld + c]), s, Xint, r * ldq + c, status);
+      a = quant_one<kOut16>(Key<T>::value(X[r * ld + c]), s, Xint, trans_out ? c * ldq + r : r * ldq + c, status);
       cmx = max(cmx, a);
     }
     // max over the CW columns of this row (CW consecutive lanes)
 #pragma unroll
     for (int o = CW / 2; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (rowmax && cc == 0 && r < rows && a) atomicMax(rowmax + r, (int32_t)a);
+    if (prow && cc == 0 && r < rows) prow[r] = (int32_t)a;
   }
   atomicMax(&s_cmax[cc], cmx);
   __syncthreads();
@@ -452,60 +591,112 @@ int64_t nearest_rank(int64_t n, double p) {
   return k;
 }
 
+template <typename T, int CW, bool kOut16>
+imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, unsigned long long k, int32_t beta,
+                           void* Xint, int64_t ldq, int trans_out, float* delta, float* qval, int32_t* rowmax,
+                           int32_t* colmax, DeviceState* ds, cudaStream_t st) {
+  const size_t smem = (size_t)rows * CW * sizeof(T);
+  const bool vec = (ld % (16 / (int64_t)sizeof(T)) == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  const int64_t grid = (cols + CW - 1) / CW;
+  int32_t* part = nullptr;
+  if (rowmax) {
+    void* pb;
+    imq_status e = partials_buffer(ds, (size_t)grid * rows * 4, &pb);
+    if (e != IMQ_OK) return e;
+    part = static_cast<int32_t*>(pb);
+  }
+  auto kern = k_rtn_cols_staged<T, CW, kOut16>;
+  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, part,
+                                               colmax, vec ? 1 : 0, ds->status);
+  if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
+  return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
+}
+
 template <typename T, bool kOut16>
 imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, double p,
-               int32_t beta, void* Xint, int64_t ldq, float* delta, float* qval, int32_t* rowmax,
+               int32_t beta, void* Xint, int64_t ldq, int trans_out, float* delta, float* qval, int32_t* rowmax,
                int32_t* colmax, DeviceState* ds, cudaStream_t st) {
   const int sms = ds->num_sms;
   if (g == IMQ_PER_COL) {
     const unsigned long long k = (unsigned long long)nearest_rank(rows, p);
+    // the slab of 16 (or 8) columns is staged in shared memory when it fits
+    constexpr size_t kSlab = 192 * 1024;
+    if ((size_t)rows * 16 * sizeof(T) <= kSlab)
+      return run_cols_staged<T, 16, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
+                                            colmax, ds, st);
+    if ((size_t)rows * 8 * sizeof(T) <= kSlab)
+      return run_cols_staged<T, 8, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
+                                           colmax, ds, st);
     const int64_t grid = (cols + kColsPerCta - 1) / kColsPerCta;
-    k_rtn_cols<T, kOut16><<<(unsigned)grid, kThreads, 0, st>>>(X, rows, cols, ld, k, beta, Xint, ldq,
-                                                               delta, qval, rowmax, colmax, ds->status);
-    return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+    int32_t* part = nullptr;
+    if (rowmax) {
+      void* pb;
+      imq_status e = partials_buffer(ds, (size_t)grid * rows * 4, &pb);
+      if (e != IMQ_OK) return e;
+      part = static_cast<int32_t*>(pb);
+    }
+    k_rtn_cols<T, kOut16><<<(unsigned)grid, kThreads, 0, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out,
+                                                               delta, qval, part, colmax, ds->status);
+    if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
+    return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
   }
-  // staged rows
+  // one warp per row; the row buffers of the CTA's warps plus its column maxima in shared memory
   const size_t row_bytes = (size_t)((cols * (int64_t)sizeof(T) + 15) / 16 * 16);
-  const size_t smem = row_bytes + (colmax ? (size_t)cols * 4 : 0);
-  if (smem > 200 * 1024) return IMQ_ERR_UNSUPPORTED;
+  const size_t cmax_bytes = colmax ? (size_t)((cols * 4 + 15) / 16 * 16) : 0;
+  constexpr size_t kBudget = 200 * 1024;
+  if (cmax_bytes + row_bytes > kBudget) return IMQ_ERR_UNSUPPORTED;
+  int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
+  if (nwarps > kThreads / 32) nwarps = kThreads / 32;
+  const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
+  int per_sm = (int)(kBudget / (smem + 9 * 1024));
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 4) per_sm = 4;
+  const int64_t blocks = (rows + nwarps - 1) / nwarps;
+  const int64_t grid = blocks < (int64_t)sms * per_sm ? blocks : (int64_t)sms * per_sm;
   const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
                    ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
-  int per_sm = (int)((200 * 1024) / (smem + 2048));
-  if (per_sm > 8) per_sm = 8;
-  if (per_sm < 1) per_sm = 1;
-  const int64_t grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
-  if (g == IMQ_PER_ROW) {
+  int32_t* part = nullptr;
+  if (colmax) {
+    void* pb;
+    imq_status e = partials_buffer(ds, (size_t)grid * cols * 4, &pb);
+    if (e != IMQ_OK) return e;
+    part = static_cast<int32_t*>(pb);
+  }
+  TensorState* ts = nullptr;
+  if (g == IMQ_PER_TENSOR) {
+    if (!ds->scratch) IMQ_CUDA_TRY(cudaMalloc(&ds->scratch, sizeof(TensorState)));
+    ts = static_cast<TensorState*>(ds->scratch);
+    k_tensor_init<<<1, 256, 0, st>>>(ts, (unsigned long long)nearest_rank(rows * cols, p));
+    const int64_t hgrid = rows < (int64_t)sms * 8 ? rows : (int64_t)sms * 8;
+    const int np = num_passes(Key<T>::kBits);
+    for (int pass = 0; pass < np; ++pass) {
+      k_tensor_hist<T><<<(unsigned)hgrid, kThreads, 0, st>>>(X, rows, cols, ld, ts, pass);
+      k_tensor_select<T><<<1, 32, 0, st>>>(ts, pass, pass == np - 1, beta, delta, qval, ds->status);
+    }
+    auto kern = k_rtn_rows<T, false, kOut16>;
+    IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, 0ull, beta, Xint, ldq, trans_out, delta, qval,
+                                                 rowmax, part, ts, vec, nwarps, ds->status);
+  } else {
     auto kern = k_rtn_rows<T, true, kOut16>;
     IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld,
-                                                 (unsigned long long)nearest_rank(cols, p), beta, Xint, ldq,
-                                                 delta, qval, rowmax, colmax, nullptr, vec, ds->status);
-    return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta,
+                                                 Xint, ldq, trans_out, delta, qval, rowmax, part, nullptr, vec, nwarps,
+                                                 ds->status);
   }
-  // per tensor
-  if (!ds->scratch) IMQ_CUDA_TRY(cudaMalloc(&ds->scratch, sizeof(TensorState)));
-  TensorState* ts = static_cast<TensorState*>(ds->scratch);
-  k_tensor_init<<<1, 256, 0, st>>>(ts, (unsigned long long)nearest_rank(rows * cols, p));
-  const int64_t hgrid = rows < (int64_t)sms * 8 ? rows : (int64_t)sms * 8;
-  const int np = num_passes(Key<T>::kBits);
-  for (int pass = 0; pass < np; ++pass) {
-    k_tensor_hist<T><<<(unsigned)hgrid, kThreads, 0, st>>>(X, rows, cols, ld, ts, pass);
-    k_tensor_select<T><<<1, 32, 0, st>>>(ts, pass, pass == np - 1, beta, delta, qval, ds->status);
-  }
-  auto kern = k_rtn_rows<T, false, kOut16>;
-  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, 0ull, beta, Xint, ldq, delta, qval,
-                                               rowmax, colmax, ts, vec, ds->status);
-  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
+  return colmax ? launch_reduce_max(part, grid, cols, colmax, st) : IMQ_OK;
 }
 
 }  // namespace
 
 imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                imq_gran g, double p, int32_t beta, void* Xint, imq_dtype it,
-                               int64_t ldq, float* delta, float* qval, int32_t* rowmax,
+                               int64_t ldq, int32_t trans_out, float* delta, float* qval, int32_t* rowmax,
                                int32_t* colmax, cudaStream_t st) {
-  if (rows < 0 || cols < 0 || ld < cols || ldq < cols || !(p > 0.0 && p <= 1.0) || beta < 1 ||
+  if (trans_out != 0 && trans_out != 1) return IMQ_ERR_ARG;
+  if (rows < 0 || cols < 0 || ld < cols || ldq < (trans_out ? rows : cols) || !(p > 0.0 && p <= 1.0) || beta < 1 ||
       beta > (1 << 24))
     return IMQ_ERR_ARG;
   if (xt != IMQ_F32 && xt != IMQ_BF16) return IMQ_ERR_ARG;
@@ -517,10 +708,11 @@ imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_
   DeviceState* ds;
   imq_status s = device_state(&ds);
   if (s != IMQ_OK) return s;
-  if (rowmax && rows > 0) IMQ_CUDA_TRY(cudaMemsetAsync(rowmax, 0, (size_t)rows * 4, st));
-  if (colmax && cols > 0) IMQ_CUDA_TRY(cudaMemsetAsync(colmax, 0, (size_t)cols * 4, st));
+  // every entry of rowmax / colmax is written by the kernels (directly or by a reduction)
   if (rows == 0 || cols == 0) {
     // every group is empty: q = max = 0, so s = Delta = 1 and there is nothing to quantise
+    if (rowmax && rows > 0) IMQ_CUDA_TRY(cudaMemsetAsync(rowmax, 0, (size_t)rows * 4, st));
+    if (colmax && cols > 0) IMQ_CUDA_TRY(cudaMemsetAsync(colmax, 0, (size_t)cols * 4, st));
     if (ngroups > 0) {
       k_fill_f32<<<1, 256, 0, st>>>(delta, ngroups, 1.0f);
       if (qval) k_fill_f32<<<1, 256, 0, st>>>(qval, ngroups, 0.0f);
@@ -530,12 +722,12 @@ imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_
   const bool o16 = it == IMQ_I16;
   if (xt == IMQ_BF16) {
     const uint16_t* x = static_cast<const uint16_t*>(X);
-    return o16 ? run<uint16_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st)
-               : run<uint16_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st);
+    return o16 ? run<uint16_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st)
+               : run<uint16_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st);
   }
   const uint32_t* x = static_cast<const uint32_t*>(X);
-  return o16 ? run<uint32_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st)
-             : run<uint32_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st);
+  return o16 ? run<uint32_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st)
+             : run<uint32_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st);
 }
 
 }  // namespace imq

@@ -20,45 +20,57 @@
 namespace imq {
 namespace {
 
+// Row gather: a CTA stages a batch of NL source lines in shared memory, then for each 4-byte piece of
+// the inner dimension reads the index maps once and writes the digits of every line of the batch (and
+// every level of an OUTER line).  Lines too long to stage are gathered from global memory (L2).
 template <typename T, bool kStaged>
 __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, int64_t nlines, int64_t K,
-                                                     int64_t ld, int outer, const int8_t* __restrict__ lvl,
+                                                     int64_t ld, int NL, int outer, const int8_t* __restrict__ lvl,
                                                      const int32_t* __restrict__ pos,
                                                      const int32_t* __restrict__ tK,
                                                      const int8_t* __restrict__ lk, int64_t K_unp,
                                                      int bm1, int8_t* __restrict__ out) {
-  extern __shared__ int32_t line[];
+  extern __shared__ __align__(16) unsigned char dsm[];
+  T* lines = reinterpret_cast<T*>(dsm);  // [NL][K]
+  __shared__ int s_L[8];
+  __shared__ int64_t s_base[8];
   const int tid = threadIdx.x;
-  for (int64_t i = blockIdx.x; i < nlines; i += gridDim.x) {
-    const T* xi = X + i * ld;
-    if (kStaged) {
-      for (int64_t t = tid; t < K; t += 256) line[t] = (int32_t)xi[t];
-      __syncthreads();
+  for (int64_t i0 = (int64_t)blockIdx.x * NL; i0 < nlines; i0 += (int64_t)gridDim.x * NL) {
+    const int nb = nlines - i0 < NL ? (int)(nlines - i0) : NL;
+    if (tid < nb) {
+      s_L[tid] = outer ? (int)lvl[i0 + tid] : 1;
+      s_base[tid] = outer ? (int64_t)pos[i0 + tid] : i0 + tid;
     }
-    const int L = outer ? (int)lvl[i] : 1;
-    const int64_t base = outer ? (int64_t)pos[i] : i;
-    for (int l = 0; l < L; ++l) {
-      int8_t* o = out + (base + l) * K_unp;
-      for (int64_t p = (int64_t)tid * 16; p < K_unp; p += 256 * 16) {
-        const int4* tq = reinterpret_cast<const int4*>(tK + p);
-        const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
-        const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
-                                tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
-        const int4 lq = *reinterpret_cast<const int4*>(lk + p);
-        const int8_t* ll = reinterpret_cast<const int8_t*>(&lq);
-        uint32_t w[4];
+    if (kStaged) {
+      for (int b = 0; b < nb; ++b)
+        for (int64_t t = tid; t < K; t += 256) lines[b * K + t] = X[(i0 + b) * ld + t];
+    }
+    __syncthreads();
+    // lane = 4 consecutive inner positions, a warp = 128: index maps read once per batch, 128-byte
+    // coalesced stores, shared-memory gathers at most 2-way bank conflicted
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int64_t p = (int64_t)warp * 128 + lane * 4; p < K_unp; p += 8 * 128) {
+      const int4 t4 = *reinterpret_cast<const int4*>(tK + p);
+      const uint32_t l4 = *reinterpret_cast<const uint32_t*>(lk + p);
+      const int32_t tt[4] = {t4.x, t4.y, t4.z, t4.w};
+      int ll[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+      for (int r = 0; r < 4; ++r) ll[r] = (int)(int8_t)(l4 >> (8 * r));
+      for (int b = 0; b < nb; ++b) {
+        int32_t v[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int32_t t = tt[r] >= 0 ? tt[r] : 0;
+          v[r] = tt[r] < 0 ? 0 : (kStaged ? (int32_t)lines[b * K + t] : (int32_t)X[(i0 + b) * ld + t]);
+        }
+        const int L = s_L[b];
+        for (int l = 0; l < L; ++l) {
           uint32_t packed = 0;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int k = q * 4 + r;
-            const int32_t d = tt[k] >= 0 ? digit_of(kStaged ? line[tt[k]] : (int32_t)xi[tt[k]], l + ll[k], bm1) : 0;
-            packed |= ((uint32_t)(uint8_t)(int8_t)d) << (8 * r);
-          }
-          w[q] = packed;
+          for (int r = 0; r < 4; ++r)
+            packed |= ((uint32_t)(uint8_t)(int8_t)digit_of(v[r], l + ll[r], bm1)) << (8 * r);
+          *reinterpret_cast<uint32_t*>(out + (s_base[b] + l) * K_unp + p) = packed;
         }
-        *reinterpret_cast<int4*>(o + p) = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
       }
     }
     __syncthreads();
@@ -127,18 +139,25 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
                       int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st) {
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
   if (line_is_row) {
-    // lines up to 48K entries are staged in shared memory; longer ones are gathered from L2
-    const size_t smem = (size_t)(K > 0 ? K : 1) * 4;
-    const bool staged = smem <= 192 * 1024;
-    int per_sm = staged ? (int)((200 * 1024) / (smem + 1024)) : 8;
-    if (per_sm > 8) per_sm = 8;
-    if (per_sm < 1) per_sm = 1;
-    const int64_t grid = nlines < (int64_t)num_sms * per_sm ? nlines : (int64_t)num_sms * per_sm;
+    // batches of up to 8 lines (64 KB of shared memory per CTA at most); lines longer than that are
+    // gathered from global memory
+    const size_t line_bytes = (size_t)(K > 0 ? K : 1) * sizeof(T);
+    int NL = (int)((64 * 1024) / line_bytes);
+    if (NL > 8) NL = 8;
+    const bool staged = NL >= 1;
+    if (!staged) NL = 8;
+    const size_t smem = staged ? (size_t)NL * line_bytes : 0;
+    const int per_sm = staged ? (int)((200 * 1024) / (smem + 2048)) : 8;
+    const int64_t batches = (nlines + NL - 1) / NL;
+    int64_t grid = (int64_t)num_sms * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
+    if (grid > batches) grid = batches;
     if (staged) {
       IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_rows<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      k_unpack_rows<T, true><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, outer, lvl, pos, tK, lk, K_unp, bm1, out);
+      k_unpack_rows<T, true><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, NL, outer, lvl, pos, tK, lk, K_unp,
+                                                                bm1, out);
     } else {
-      k_unpack_rows<T, false><<<(unsigned)grid, 256, 0, st>>>(X, nlines, K, ld, outer, lvl, pos, tK, lk, K_unp, bm1, out);
+      k_unpack_rows<T, false><<<(unsigned)grid, 256, 0, st>>>(X, nlines, K, ld, NL, outer, lvl, pos, tK, lk, K_unp,
+                                                              bm1, out);
     }
   } else {
     const dim3 grid((unsigned)((nlines + 31) / 32), (unsigned)(K_unp / 128));

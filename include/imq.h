@@ -91,17 +91,20 @@ typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2 } imq_dir;
  *   Delta_g = q_g / (float)beta            fp32, the dequantisation step (x ~= Delta * x_int)
  *
  * X       device, rows x cols, row-major with leading dimension ld (>= cols), dtype xt (F32 or BF16).
- * Xint    device, rows x cols, leading dimension ldq (>= cols), dtype it (I16 or I32).
+ * Xint    device, dtype it (I16 or I32).  trans_out = 0: rows x cols like X, leading dimension ldq
+ *         (>= cols).  trans_out = 1: the transpose, cols x rows, leading dimension ldq (>= rows) -- a
+ *         weight W stored K x N is quantised per output channel straight into the N x K layout that
+ *         imq_plan takes as B with transB = 1.
  * delta   device, fp32, 1 / rows / cols entries for PER_TENSOR / PER_ROW / PER_COL.
  * qval    device or NULL, fp32, same length as delta: the selected percentile values q_g.
- * rowmax  device or NULL, int32[rows]: max |Xint| of each stored row.
- * colmax  device or NULL, int32[cols]: max |Xint| of each stored column.
+ * rowmax  device or NULL, int32[rows]: max |x_int| over each row of X (whatever trans_out is).
+ * colmax  device or NULL, int32[cols]: max |x_int| over each column of X.
  * Errors: IMQ_ERR_ARG at once; IMQ_ERR_NONFINITE / IMQ_ERR_RANGE through the device status word.
  * Scratch: PER_TENSOR uses a small per-device buffer the library allocates once on first use.
  */
 imq_status imq_rtn_quantize(const void *X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                             imq_gran g, double p, int32_t beta,
-                            void *Xint, imq_dtype it, int64_t ldq,
+                            void *Xint, imq_dtype it, int64_t ldq, int32_t trans_out,
                             float *delta, float *qval, int32_t *rowmax, int32_t *colmax,
                             imq_stream_t stream);
 

@@ -60,6 +60,36 @@ def test_quantize_parity(imq, dtype, gran, shape, p, beta):
         assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0))
 
 
+@pytest.mark.parametrize("gran", [oracle.PER_TENSOR, oracle.PER_ROW, oracle.PER_COL])
+@pytest.mark.parametrize("shape", [(5, 3), (300, 130), (4096, 96), (1000, 17)])
+def test_quantize_transposed_output(imq, gran, shape):
+    rng = np.random.default_rng(zlib.crc32(repr(("T", gran, shape)).encode()))
+    x = _matrix(rng, shape)
+    bits = workloads.f32_to_bf16_bits(x)
+    want_i, want_d, _ = oracle.rtn_quantize(oracle.bf16_bits_to_f32(bits), gran, 0.95, 15)
+    X = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    r = imq.imq_rtn_quantize(X, gran, 0.95, 15, trans_out=True)
+    assert tuple(r.xint.shape) == (shape[1], shape[0])
+    assert np.array_equal(r.xint.cpu().numpy().astype(np.int64), want_i.T)
+    assert np.array_equal(r.delta.cpu().numpy(), want_d)
+    assert np.array_equal(r.rowmax.cpu().numpy(), np.abs(want_i).max(axis=1))
+    assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0))
+
+
+def test_quantize_tall_columns(imq):
+    """Columns too tall for the staged kernel (11008 rows: 8-column slabs) and taller (streaming)."""
+    rng = np.random.default_rng(15)
+    for rows in (11008, 20000):
+        x = _matrix(rng, (rows, 40))
+        bits = workloads.f32_to_bf16_bits(x)
+        want_i, want_d, _ = oracle.rtn_quantize(oracle.bf16_bits_to_f32(bits), oracle.PER_COL, 0.95, 31)
+        X = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+        r = imq.imq_rtn_quantize(X, oracle.PER_COL, 0.95, 31, out_dtype=torch.int32)
+        assert np.array_equal(r.xint.cpu().numpy().astype(np.int64), want_i)
+        assert np.array_equal(r.delta.cpu().numpy(), want_d)
+        assert np.array_equal(r.rowmax.cpu().numpy(), np.abs(want_i).max(axis=1))
+
+
 def test_quantize_strided_input(imq):
     rng = np.random.default_rng(5)
     x = _matrix(rng, (70, 300))
