@@ -55,10 +55,27 @@ imq_status partials_buffer(DeviceState* ds, size_t bytes, void** out) {
 }
 
 namespace {
-__global__ void k_reduce_max(const int32_t* __restrict__ part, int64_t nparts, int64_t n, int32_t* __restrict__ out) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    int32_t m = 0;
-    for (int64_t p = 0; p < nparts; ++p) m = max(m, __ldcs(part + p * n + i));
+// Block of 32 x 8 threads: x = 32 consecutive entries (coalesced), y = a slice of the partials; the
+// eight slices are combined in shared memory.
+__global__ void __launch_bounds__(256) k_reduce_max(const int32_t* __restrict__ part, int64_t nparts, int64_t n,
+                                                    int32_t* __restrict__ out) {
+  __shared__ int32_t red[8][33];
+  const int64_t i = (int64_t)blockIdx.x * 32 + threadIdx.x;
+  int32_t m = 0;
+  if (i < n) {
+    int64_t p = threadIdx.y;
+#pragma unroll 4
+    for (; p + 24 < nparts; p += 32) {
+      const int32_t a = __ldcs(part + p * n + i), b = __ldcs(part + (p + 8) * n + i);
+      const int32_t c = __ldcs(part + (p + 16) * n + i), d = __ldcs(part + (p + 24) * n + i);
+      m = max(max(m, a), max(b, max(c, d)));
+    }
+    for (; p < nparts; p += 8) m = max(m, __ldcs(part + p * n + i));
+  }
+  red[threadIdx.y][threadIdx.x] = m;
+  __syncthreads();
+  if (threadIdx.y == 0 && i < n) {
+    for (int y = 1; y < 8; ++y) m = max(m, red[y][threadIdx.x]);
     out[i] = m;
   }
 }
@@ -69,9 +86,8 @@ imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int
   DeviceState* ds;
   imq_status s = device_state(&ds);
   if (s != IMQ_OK) return s;
-  int64_t grid = (n + 255) / 256;
-  if (grid > ds->num_sms * 4) grid = ds->num_sms * 4;
-  k_reduce_max<<<(unsigned)grid, 256, 0, st>>>(part, nparts, n, out);
+  (void)ds;
+  k_reduce_max<<<(unsigned)((n + 31) / 32), dim3(32, 8), 0, st>>>(part, nparts, n, out);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 

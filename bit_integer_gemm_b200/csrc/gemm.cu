@@ -76,9 +76,11 @@ struct GemmArgs {
 struct Smem {
   static constexpr size_t kA = 0;
   static constexpr size_t kB = kA + (size_t)STAGES * A_STAGE;
-  static constexpr size_t kScratch = kB + (size_t)STAGES * B_STAGE;  // per epilogue warp: [32][33] x 8 B
+  // per epilogue warp: a 32 x 32 transpose buffer of up to 8-byte values, XOR-swizzled
+  static constexpr size_t kScratch = kB + (size_t)STAGES * B_STAGE;
+  static constexpr size_t kRows = kScratch + EPI_WARPS * 32 * 32 * 8;  // per epilogue warp: WarpRows
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr size_t kBars = kScratch + EPI_WARPS * 32 * 33 * 8;
+  static constexpr size_t kBars = kRows + EPI_WARPS * 256;
   static constexpr size_t kMisc = kBars + (2 * STAGES + 5) * 8;  // tmem base, abort flag
   static constexpr size_t kEnd = kMisc + 16;
   static constexpr size_t kBytes = kEnd + 1024;  // slack for 1024-byte alignment of the base
@@ -118,70 +120,118 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
   return true;
 }
 
-// Drains one TMEM slot (this warp's 32 lanes) of tile (mt, nt) into C: fold, shift, write or add.
-template <typename T>
-__device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, uint32_t acce_bar, int mt, int nt,
-                                           int q, int lane, bool first, bool last, int shift, T* scr) {
-  // the source row lane t holds after the row fold (t < nA)
+// Per-warp drain metadata of one tile, fetched before the accumulator is ready: row offsets and row
+// scales in shared memory (read as broadcasts), column indices and column scales in registers.
+struct DrainMeta {
   int LA, nA;
+  int LB[BN / 32], nB[BN / 32];
+  int32_t col[BN / 32];  // this lane's output column in each chunk (lane < nB)
+  float sb[BN / 32];     // its dequantisation scale
+};
+
+struct WarpRows {       // shared memory, per epilogue warp
+  int32_t row[32];      // the output row lane t holds after the row fold
+  float sa[32];         // its dequantisation scale
+};
+
+// Transpose buffer index: row r, column c, XOR-swizzled so that both a row sweep and a column sweep of
+// the warp hit 32 different banks.
+__device__ __forceinline__ int sw(int r, int c) { return r * 32 + (c ^ r); }
+
+__device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt, int q, int lane, bool last,
+                                              DrainMeta& m, WarpRows* wr) {
   int64_t my_row;
   if (g.a_outer) {
     const int64_t grp = (int64_t)mt * (BM / 32) + q;
-    LA = grp < g.n_grp_a ? g.grpA_L[grp] : 1;
-    nA = grp < g.n_grp_a ? g.grpA_n[grp] : 0;
-    my_row = lane < nA ? g.srcA[grp * 32 + (int64_t)lane * LA] : 0;
+    m.LA = grp < g.n_grp_a ? g.grpA_L[grp] : 1;
+    m.nA = grp < g.n_grp_a ? g.grpA_n[grp] : 0;
+    my_row = lane < m.nA ? g.srcA[grp * 32 + (int64_t)lane * m.LA] : 0;
   } else {
-    LA = 1;
+    m.LA = 1;
     const int64_t r0 = (int64_t)mt * BM + q * 32;
     const int64_t rem = g.M - r0;
-    nA = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
-    my_row = r0 + lane;
+    m.nA = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
+    my_row = lane < m.nA ? r0 + lane : 0;
   }
-  const float my_sa = (last && g.Cf && lane < nA) ? g.dA[g.dA_per_row ? my_row : 0] : 0.0f;
+  wr->row[lane] = (int32_t)my_row;
+  wr->sa[lane] = (last && g.Cf && lane < m.nA) ? g.dA[g.dA_per_row ? my_row : 0] : 0.0f;
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    const int64_t gc = (int64_t)nt * (BN / 32) + c;
+    if (g.b_outer) {
+      m.LB[c] = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
+      m.nB[c] = gc < g.n_grp_b ? g.grpB_n[gc] : 0;
+    } else {
+      m.LB[c] = 1;
+      const int64_t rem = g.N - gc * 32;
+      m.nB[c] = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    const int64_t gc = (int64_t)nt * (BN / 32) + c;
+    m.col[c] = 0;
+    if (lane < m.nB[c]) m.col[c] = g.b_outer ? g.srcB[gc * 32 + (int64_t)lane * m.LB[c]] : (int32_t)(gc * 32 + lane);
+  }
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) m.sb[c] = (last && g.Cf && lane < m.nB[c]) ? g.dB[g.dB_per_col ? m.col[c] : 0] : 0.0f;
+  __syncwarp();
+}
+
+// Drains one TMEM slot (this warp's 32 lanes) into C: fold, shift, write or add.
+template <typename T>
+__device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, uint32_t acce_bar, int lane, bool first,
+                                           bool last, int shift, T* scr, const DrainMeta& m, const WarpRows* wr) {
+  uint32_t v[32];
+  tmem_ld32(tbase, v);
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
-    uint32_t v[32];
-    tmem_ld32(tbase + c * 32, v);
     tmem_wait_ld();
-    if (c == BN / 32 - 1) {
+    uint32_t cur[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) cur[k] = v[k];
+    if (c + 1 < BN / 32) {
+      tmem_ld32(tbase + (c + 1) * 32, v);  // the next chunk streams in while this one is folded
+    } else {
       // the slot is fully read: the MMA warp may reuse it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce_bar);
     }
-    // columns of this chunk
-    const int64_t gc = (int64_t)nt * (BN / 32) + c;
-    int LB, nB;
-    if (g.b_outer) {
-      LB = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
-      nB = gc < g.n_grp_b ? g.grpB_n[gc] : 0;
-    } else {
-      LB = 1;
-      const int64_t rem = g.N - gc * 32;
-      nB = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
-    }
+    // dynamic indexing of the unrolled metadata arrays is avoided by a uniform select
+    int LB = 1, nB = 0, mycol = 0;
+    float sb = 0.0f;
+#pragma unroll
+    for (int k = 0; k < BN / 32; ++k)
+      if (k == c) {
+        LB = m.LB[k];
+        nB = m.nB[k];
+        mycol = m.col[k];
+        sb = m.sb[k];
+      }
+    const int nA = m.nA, LA = m.LA;
     if (nB == 0 || nA == 0) continue;
     // 1. fold the column levels of B inside the registers (lane = unpacked row)
     T w[32];
     switch (LB) {
-      case 1: fold_cols<1>(v, w, g.bm1); break;
-      case 2: fold_cols<2>(v, w, g.bm1); break;
-      case 3: fold_cols<3>(v, w, g.bm1); break;
-      case 4: fold_cols<4>(v, w, g.bm1); break;
-      case 5: fold_cols<5>(v, w, g.bm1); break;
-      case 6: fold_cols<6>(v, w, g.bm1); break;
-      case 7: fold_cols<7>(v, w, g.bm1); break;
-      case 8: fold_cols<8>(v, w, g.bm1); break;
+      case 1: fold_cols<1>(cur, w, g.bm1); break;
+      case 2: fold_cols<2>(cur, w, g.bm1); break;
+      case 3: fold_cols<3>(cur, w, g.bm1); break;
+      case 4: fold_cols<4>(cur, w, g.bm1); break;
+      case 5: fold_cols<5>(cur, w, g.bm1); break;
+      case 6: fold_cols<6>(cur, w, g.bm1); break;
+      case 7: fold_cols<7>(cur, w, g.bm1); break;
+      case 8: fold_cols<8>(cur, w, g.bm1); break;
       default: {
         // levels 9..31 (three columns at most): fold through the transpose buffer
 #pragma unroll
-        for (int k = 0; k < 32; ++k) scr[lane * 33 + k] = (T)(int32_t)v[k];
+        for (int k = 0; k < 32; ++k) scr[sw(lane, k)] = (T)(int32_t)cur[k];
         __syncwarp();
 #pragma unroll
         for (int s2 = 0; s2 < 3; ++s2) {
           T a = 0;
           if (s2 < nB)
-            for (int l = 0; l < LB; ++l) a += shl<T>(scr[lane * 33 + s2 * LB + l], l * g.bm1);
+            for (int l = 0; l < LB; ++l) a += shl<T>(scr[sw(lane, s2 * LB + l)], l * g.bm1);
           w[s2] = a;
         }
         __syncwarp();
@@ -204,49 +254,29 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
     // 3. transpose through shared memory: scr[row][column]
 #pragma unroll
     for (int s2 = 0; s2 < 32; ++s2)
-      if (s2 < nB) scr[lane * 33 + s2] = shl<T>(w[s2], shift);
+      if (s2 < nB) scr[sw(lane, s2)] = shl<T>(w[s2], shift);
     __syncwarp();
     // 4. lane = output column: coalesced accesses along each row of C
-    int64_t mycol = 0;
-    float my_sb = 0.0f;
     if (lane < nB) {
-      mycol = g.b_outer ? g.srcB[gc * 32 + (int64_t)lane * LB] : gc * 32 + lane;
-      if (last && g.Cf) my_sb = g.dB[g.dB_per_col ? mycol : 0];
-    }
-    const bool col_ok = lane < nB;
-#pragma unroll 1
-    for (int r0 = 0; r0 < nA; r0 += 8) {
-      T val[8];
-      int64_t row[8];
-      float sa[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        row[u] = shfl_t(my_row, (r0 + u) & 31);
-        sa[u] = __shfl_sync(0xffffffffu, my_sa, (r0 + u) & 31);
-        val[u] = scr[((r0 + u) & 31) * 33 + lane];
-      }
-      if (!first && g.C && col_ok) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (r0 + u < nA) {
-            if (sizeof(T) == 8) val[u] += (T) static_cast<const int64_t*>(g.C)[row[u] * g.ldc + mycol];
-            else val[u] += (T) static_cast<const int32_t*>(g.C)[row[u] * g.ldc + mycol];
-          }
-      }
-      if (col_ok) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (r0 + u < nA) {
-            if (g.C) {
-              if (g.c64) static_cast<int64_t*>(g.C)[row[u] * g.ldc + mycol] = (int64_t)val[u];
-              else static_cast<int32_t*>(g.C)[row[u] * g.ldc + mycol] = (int32_t)val[u];
-            }
-            if (last && g.Cf)
-              g.Cf[row[u] * g.ldcf + mycol] =
-                  __fmul_rn(sizeof(T) == 8 ? __ll2float_rn((long long)val[u]) : __int2float_rn((int)val[u]),
-                            __fmul_rn(sa[u], my_sb));
+#pragma unroll 4
+      for (int r = 0; r < nA; ++r) {
+        T val = scr[sw(r, lane)];
+        const int64_t row = wr->row[r];
+        if (g.C) {
+          if (g.c64) {
+            int64_t* cp = static_cast<int64_t*>(g.C) + row * g.ldc + mycol;
+            if (!first) val += (T)*cp;
+            *cp = (int64_t)val;
+          } else {
+            int32_t* cp = static_cast<int32_t*>(g.C) + row * g.ldc + mycol;
+            if (!first) val += (T)*cp;
+            *cp = (int32_t)val;
           }
         }
+        if (last && g.Cf)
+          g.Cf[row * g.ldcf + mycol] =
+              __fmul_rn(sizeof(T) == 8 ? __ll2float_rn((long long)val) : __int2float_rn((int)val),
+                        __fmul_rn(wr->sa[r], sb));
       }
     }
     __syncwarp();
@@ -264,6 +294,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sA = base + L::kA;
   uint8_t* sB = base + L::kB;
   T* scratch = reinterpret_cast<T*>(base + L::kScratch);
+  WarpRows* wrows = reinterpret_cast<WarpRows*>(base + L::kRows);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::kBars);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
@@ -387,12 +418,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access = row group of the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    T* scr = scratch + q * 32 * 33;  // this warp's transpose buffer: [row][column], row stride 33
+    T* scr = scratch + q * 32 * 32;  // this warp's transpose buffer (XOR-swizzled rows of 32)
     uint32_t full_waits[2] = {0, 0};
     for (int p = 0; p < my_tiles; p += 2) {
       const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
       for (int k = 0; k < g.n_steps; ++k) {
         for (int slot = 0; slot < npair; ++slot) {
+          DrainMeta meta;
+          const bool drain = g.step_after[k] < 0;
+          if (drain) {
+            // metadata of the tile first: its loads overlap the wait for the accumulator
+            const int tile = blockIdx.x + (p + slot) * gridDim.x;
+            drain_prepare(g, tile % g.tiles_m, tile / g.tiles_m, q, lane, g.step_dlast[k] != 0, meta, wrows + q);
+          }
           int ok = 1;
           if (lane == 0) ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -418,9 +456,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(acce0 + 8 * slot);
           } else {
-            const int tile = blockIdx.x + (p + slot) * gridDim.x;
-            drain_slot<T>(g, tbase, acce0 + 8 * slot, tile % g.tiles_m, tile / g.tiles_m, q, lane,
-                          g.step_dfirst[k] != 0, g.step_dlast[k] != 0, g.step_dshift[k], scr);
+            drain_slot<T>(g, tbase, acce0 + 8 * slot, lane, g.step_dfirst[k] != 0, g.step_dlast[k] != 0,
+                          g.step_dshift[k], scr, meta, wrows + q);
           }
         }
       }

@@ -237,6 +237,20 @@ __global__ void __launch_bounds__(1024) k_inner_map(const InnerSeg* __restrict__
   }
 }
 
+// blk16[c] = t0 when the 16 inner positions of block c are t0..t0+15 (t0 % 16 == 0) with one (lA, lB)
+// pair, else -1.
+__global__ void k_inner_blocks(const int32_t* __restrict__ tK, const int8_t* __restrict__ lAk,
+                               const int8_t* __restrict__ lBk, int64_t nblk, int32_t* __restrict__ blk16) {
+  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < nblk; c += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t* t = tK + c * 16;
+    const int32_t t0 = t[0];
+    bool ok = t0 >= 0 && (t0 & 15) == 0;
+    for (int k = 1; k < 16 && ok; ++k)
+      ok = t[k] == t0 + k && lAk[c * 16 + k] == lAk[c * 16] && lBk[c * 16 + k] == lBk[c * 16];
+    blk16[c] = ok ? t0 : -1;
+  }
+}
+
 struct OuterClass {
   int32_t L;
   int32_t per;      // source lines per group
@@ -629,6 +643,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   const size_t o_tK = off2; off2 = align_up(off2 + (size_t)I.K_unp * 4, 256);
   const size_t o_lAk = off2; off2 = align_up(off2 + (size_t)I.K_unp, 256);
   const size_t o_lBk = off2; off2 = align_up(off2 + (size_t)I.K_unp, 256);
+  const size_t o_blk = off2; off2 = align_up(off2 + (size_t)(I.K_unp / 16) * 4, 256);
   size_t o_posA = 0, o_srcA = 0, o_gLA = 0, o_gNA = 0, o_posB = 0, o_srcB = 0, o_gLB = 0, o_gNB = 0;
   if (a_outer) {
     o_posA = off2; off2 = align_up(off2 + (size_t)M * 4, 256);
@@ -651,6 +666,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   pl->tK = reinterpret_cast<int32_t*>(b2 + o_tK);
   pl->lAk = reinterpret_cast<int8_t*>(b2 + o_lAk);
   pl->lBk = reinterpret_cast<int8_t*>(b2 + o_lBk);
+  pl->blk16 = reinterpret_cast<int32_t*>(b2 + o_blk);
   if (a_outer) {
     pl->posA = reinterpret_cast<int32_t*>(b2 + o_posA);
     pl->srcA = reinterpret_cast<int32_t*>(b2 + o_srcA);
@@ -678,8 +694,11 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
         cudaMemcpyAsync(dcls, hcls, sizeof(OuterClass) * (ncls > 0 ? ncls : 1), cudaMemcpyHostToDevice, st) != cudaSuccess)
       return fail(IMQ_ERR_CUDA);
   }
-  if (nseg > 0)
+  if (nseg > 0) {
     k_inner_map<<<nseg, 1024, 0, st>>>(dsegs, pl->lv_a_col, pl->lv_b_row, a_inner, b_inner, K, pl->tK, pl->lAk, pl->lBk);
+    const int64_t nblk = I.K_unp / 16;
+    k_inner_blocks<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(pl->tK, pl->lAk, pl->lBk, nblk, pl->blk16);
+  }
   if (a_outer && cls_a1 > cls_a0)
     k_outer_map<<<cls_a1 - cls_a0, 1024, 0, st>>>(dcls + cls_a0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
                                                   pl->grpA_L, pl->grpA_n);

@@ -162,6 +162,69 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
 }
 
 // ------------------------------------------------------------------------------------------------
+// warp-level routines over one group of n values held contiguously in shared memory (16-byte aligned)
+// ------------------------------------------------------------------------------------------------
+// Exact nearest-rank select: the k-th smallest key (1-based) by 8-bit radix passes on a warp-private
+// 256-bin histogram.  Returns the key; every lane gets it.
+template <typename T>
+__device__ uint32_t warp_select_key(const T* a, int n, unsigned long long k, uint32_t* hist) {
+  constexpr int V = 16 / sizeof(T);
+  const int lane = threadIdx.x & 31;
+  uint32_t pre = 0, msk = 0;
+  for (int pass = 0; pass < num_passes(Key<T>::kBits); ++pass) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+    __syncwarp();
+    const int sh = pass_shift(Key<T>::kBits, pass);
+    const int nv = n / V;
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 w = reinterpret_cast<const uint4*>(a)[i];
+      const T* e = reinterpret_cast<const T*>(&w);
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const uint32_t key = Key<T>::key(e[j]);
+        if ((key & msk) == pre) atomicAdd(&hist[(key >> sh) & 0xFFu], 1u);
+      }
+    }
+    for (int i = nv * V + lane; i < n; i += 32) {
+      const uint32_t key = Key<T>::key(a[i]);
+      if ((key & msk) == pre) atomicAdd(&hist[(key >> sh) & 0xFFu], 1u);
+    }
+    __syncwarp();
+    int d;
+    unsigned long long below;
+    warp_select(hist, 1, k, &d, &below);
+    d = __shfl_sync(0xffffffffu, d, 0);
+    below = __shfl_sync(0xffffffffu, below, 0);
+    pre |= (uint32_t)d << sh;
+    msk |= pass_width_mask(Key<T>::kBits, pass) << sh;
+    k -= below;
+    __syncwarp();
+  }
+  return pre;
+}
+
+// Largest key of the group and whether any key is non-finite (every lane gets both).
+template <typename T>
+__device__ void warp_key_stats(const T* a, int n, uint32_t* mk_out, uint32_t* bad_out) {
+  constexpr int V = 16 / sizeof(T);
+  const int lane = threadIdx.x & 31;
+  uint32_t mk = 0;
+  const int nv = n / V;
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 w = reinterpret_cast<const uint4*>(a)[i];
+    const T* e = reinterpret_cast<const T*>(&w);
+#pragma unroll
+    for (int j = 0; j < V; ++j) mk = max(mk, Key<T>::key(e[j]));
+  }
+  for (int i = nv * V + lane; i < n; i += 32) mk = max(mk, Key<T>::key(a[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+  *mk_out = mk;
+  *bad_out = mk >= Key<T>::kInf;
+}
+
+// ------------------------------------------------------------------------------------------------
 // per stored row (kSelect) or per tensor (scale from the tensor state): one warp per row.  Each warp
 // stages its row in its own shared-memory buffer, builds its own 256-bin histograms (warp-aggregated
 // increments) and selects with warp scans, so no block barrier is involved.  Column maxima of the
@@ -186,64 +249,22 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
     for (int64_t c = tid; c < cols; c += blockDim.x) cmax[c] = 0;
   __syncthreads();
   if (warp < nwarps) {
+    const int n = (int)cols;
     for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < rows; r += (int64_t)gridDim.x * nwarps) {
       const T* xr = X + r * ld;
-      uint32_t mk = 0, bad = 0;
       if (vec) {
         const uint4* src = reinterpret_cast<const uint4*>(xr);
         uint4* dst = reinterpret_cast<uint4*>(row);
-        for (int64_t c = lane; c < cols / V; c += 32) {
-          const uint4 w = __ldcs(src + c);
-          dst[c] = w;
-          const T* e = reinterpret_cast<const T*>(&w);
-#pragma unroll
-          for (int j = 0; j < V; ++j) {
-            const uint32_t k = Key<T>::key(e[j]);
-            mk = max(mk, k);
-            bad |= (k >= Key<T>::kInf);
-          }
-        }
+        for (int c = lane; c < n / V; c += 32) dst[c] = __ldcs(src + c);
       } else {
-        for (int64_t c = lane; c < cols; c += 32) {
-          const T u = xr[c];
-          row[c] = u;
-          const uint32_t k = Key<T>::key(u);
-          mk = max(mk, k);
-          bad |= (k >= Key<T>::kInf);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mk = max(mk, __shfl_xor_sync(0xffffffffu, mk, o));
-        bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+        for (int c = lane; c < n; c += 32) row[c] = xr[c];
       }
       __syncwarp();
+      uint32_t mk, bad;
+      warp_key_stats(row, n, &mk, &bad);
       float s;
       if (kSelect) {
-        uint32_t pre = 0, msk = 0;
-        unsigned long long kk = krank;
-        for (int pass = 0; pass < num_passes(Key<T>::kBits); ++pass) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
-          __syncwarp();
-          const int sh = pass_shift(Key<T>::kBits, pass);
-          for (int64_t c0 = 0; c0 < cols; c0 += 32) {
-            const int64_t c = c0 + lane;
-            const uint32_t k = c < cols ? Key<T>::key(row[c]) : 0u;
-            warp_count(hist, (k >> sh) & 0xFFu, c < cols && (k & msk) == pre);
-          }
-          __syncwarp();
-          int d;
-          unsigned long long below;
-          warp_select(hist, 1, kk, &d, &below);
-          d = __shfl_sync(0xffffffffu, d, 0);
-          below = __shfl_sync(0xffffffffu, below, 0);
-          pre |= (uint32_t)d << sh;
-          msk |= pass_width_mask(Key<T>::kBits, pass) << sh;
-          kk -= below;
-          __syncwarp();
-        }
-        const float q = Key<T>::from_key(pre);
+        const float q = Key<T>::from_key(warp_select_key(row, n, krank, hist));
         float dl;
         scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
         if (lane == 0) {
@@ -258,7 +279,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
         continue;
       }
       uint32_t rmx = 0;
-      for (int64_t c = lane; c < cols; c += 32) {
+      for (int c = lane; c < n; c += 32) {
         const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
                                              status);
         rmx = max(rmx, a);
@@ -278,137 +299,76 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
 }
 
 // ------------------------------------------------------------------------------------------------
-// per stored column, slab staged in shared memory: CW columns x all rows are read from HBM once; the
-// select passes and the quantisation read shared memory.  With trans_out the quantised slab is written
-// transposed (column c of X becomes row c of Xint), with coalesced stores along it.
+// per stored column, slab staged in shared memory: CW columns x all rows are read from HBM once and
+// stored transposed (each column contiguous); then one warp per column runs the same select and
+// quantisation as a row.  With trans_out the quantised column is written as one contiguous output row
+// (a K x N weight quantised per output channel straight into N x K).  Row maxima of the CTA's columns
+// go to `part` (reduced afterwards); column maxima are written directly.
 // ------------------------------------------------------------------------------------------------
 template <typename T, int CW, bool kOut16>
-__global__ void __launch_bounds__(kThreads) k_rtn_cols_staged(
+__global__ void __launch_bounds__(CW * 32) k_rtn_cols_staged(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
     void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
     int32_t* __restrict__ part, int32_t* __restrict__ colmax, int vec, int32_t* status) {
   extern __shared__ __align__(16) unsigned char dsm[];
-  T* S = reinterpret_cast<T*>(dsm);  // [rows][CW]
-  int32_t* prow = part ? part + (int64_t)blockIdx.x * rows : nullptr;  // this CTA's row maxima
-  __shared__ uint32_t hist[256 * CW];  // [bucket][column]
-  __shared__ uint32_t s_prefix[CW], s_mask[CW], s_maxkey[CW], s_cmax[CW];
-  __shared__ unsigned long long s_k[CW];
-  __shared__ float s_s[CW];
-  __shared__ uint32_t s_bad;
-  const int tid = threadIdx.x, cc = tid % CW;
+  const int n = (int)rows;
+  const int colstride = (n + 7) / 8 * 8;  // elements; keeps every column 16-byte aligned
+  T* S = reinterpret_cast<T*>(dsm);       // [CW][colstride]
+  uint32_t* rmax = reinterpret_cast<uint32_t*>(dsm + (size_t)CW * colstride * sizeof(T));  // [rows]
+  __shared__ uint32_t hist_all[CW][256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t c0 = (int64_t)blockIdx.x * CW;
   const int ncol = cols - c0 < CW ? (int)(cols - c0) : CW;
-  if (tid < CW) {
-    s_prefix[tid] = 0;
-    s_mask[tid] = 0;
-    s_maxkey[tid] = 0;
-    s_cmax[tid] = 0;
-    s_k[tid] = krank;
-  }
-  if (tid == 0) s_bad = 0;
-  // stage the slab (columns past the end read as zero)
+  for (int r = tid; r < n; r += CW * 32) rmax[r] = 0;
+  // stage: 16-byte loads along the rows, transposed stores into the columns
   constexpr int V = 16 / sizeof(T);
-  if (vec && ncol == CW) {
-    constexpr int SEG = CW / V;  // 16-byte pieces per row
-    for (int64_t i = tid; i < rows * SEG; i += kThreads) {
-      const int64_t r = i / SEG;
-      const int sg = (int)(i % SEG);
-      reinterpret_cast<uint4*>(S)[i] = __ldcs(reinterpret_cast<const uint4*>(X + r * ld + c0) + sg);
+  constexpr int SEG = CW / V;  // 16-byte pieces per slab row (0 when a slab row is narrower)
+  if (SEG > 0 && vec && ncol == CW) {
+    for (int i = tid; i < n * SEG; i += CW * 32) {
+      const int r = i / SEG, sg = i % SEG;
+      const uint4 w = __ldcs(reinterpret_cast<const uint4*>(X + r * ld + c0) + sg);
+      const T* e = reinterpret_cast<const T*>(&w);
+#pragma unroll
+      for (int j = 0; j < V; ++j) S[(sg * V + j) * colstride + r] = e[j];
     }
   } else {
-    for (int64_t i = tid; i < rows * CW; i += kThreads) {
-      const int64_t r = i / CW;
-      const int k = (int)(i % CW);
-      S[i] = k < ncol ? X[r * ld + c0 + k] : (T)0;
+    for (int i = tid; i < n * CW; i += CW * 32) {
+      const int r = i / CW, k = i % CW;
+      S[k * colstride + r] = k < ncol ? X[r * ld + c0 + k] : (T)0;
     }
   }
   __syncthreads();
-  // every thread sees one column: i % CW == tid % CW because kThreads is a multiple of CW
-  uint32_t mk = 0, bad = 0;
-  for (int64_t i = tid; i < rows * CW; i += kThreads) {
-    const uint32_t k = Key<T>::key(S[i]);
-    mk = max(mk, k);
-    bad |= (k >= Key<T>::kInf);
-  }
-  if (mk) atomicMax(&s_maxkey[cc], mk);
-  if (bad) atomicOr(&s_bad, 1u);
-  for (int pass = 0; pass < num_passes(Key<T>::kBits); ++pass) {
-    for (int i = tid; i < 256 * CW; i += kThreads) hist[i] = 0;
-    __syncthreads();
-    const uint32_t pre = s_prefix[cc], msk = s_mask[cc];
-    const int sh = pass_shift(Key<T>::kBits, pass);
-    // bins are [bucket][column]: the lanes of a warp mostly hit different columns
-    for (int64_t i = tid; i < rows * CW; i += kThreads) {
-      const uint32_t k = Key<T>::key(S[i]);
-      if ((k & msk) == pre) atomicAdd(&hist[((k >> sh) & 0xFFu) * CW + cc], 1u);
+  if (warp < ncol) {
+    const T* col = S + warp * colstride;
+    const int64_t c = c0 + warp;
+    uint32_t mk, bad;
+    warp_key_stats(col, n, &mk, &bad);
+    const float q = Key<T>::from_key(warp_select_key(col, n, krank, hist_all[warp]));
+    float s, dl;
+    scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
+    if (lane == 0) {
+      delta[c] = dl;
+      if (qval) qval[c] = q;
+      if (bad) set_status(status, IMQ_ERR_NONFINITE);
     }
-    __syncthreads();
-    for (int col = tid >> 5; col < CW; col += kThreads / 32) {
-      int d;
-      unsigned long long below;
-      if (warp_select(hist + col, CW, s_k[col], &d, &below)) {
-        s_prefix[col] = s_prefix[col] | ((uint32_t)d << sh);
-        s_mask[col] = s_mask[col] | (pass_width_mask(Key<T>::kBits, pass) << sh);
-        s_k[col] -= below;
-      }
-    }
-    __syncthreads();
-  }
-  if (tid < ncol) {
-    float s, d;
-    const float q = Key<T>::from_key(s_prefix[tid]);
-    scale_from_q(q, Key<T>::from_key(s_maxkey[tid]), beta, &s, &d);
-    delta[c0 + tid] = d;
-    if (qval) qval[c0 + tid] = q;
-    s_s[tid] = s;
-  }
-  if (tid == 0 && s_bad) set_status(status, IMQ_ERR_NONFINITE);
-  __syncthreads();
-  if (s_bad) return;
-  if (!trans_out) {
     uint32_t cmx = 0;
-    const float s = cc < ncol ? s_s[cc] : 0.0f;
-    for (int64_t i0 = 0; i0 < rows * CW; i0 += kThreads) {
-      const int64_t i = i0 + tid;
-      const int64_t r = i / CW;
-      uint32_t a = 0;
-      if (i < rows * CW && cc < ncol) {
-        a = quant_one<kOut16>(Key<T>::value(S[i]), s, Xint, r * ldq + c0 + cc, status);
+    if (!bad) {
+      for (int r = lane; r < n; r += 32) {
+        const uint32_t a = quant_one<kOut16>(Key<T>::value(col[r]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
+                                             status);
         cmx = max(cmx, a);
+        if (part && a) atomicMax(&rmax[r], a);
       }
-#pragma unroll
-      for (int o = CW / 2; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
-      if (prow && cc == 0 && i < rows * CW) prow[r] = (int32_t)a;
-    }
-    atomicMax(&s_cmax[cc], cmx);
-  } else {
-    // row r of the slab is entry r of output rows c0 .. c0+ncol-1
-    uint32_t cm[CW];
-#pragma unroll
-    for (int k = 0; k < CW; ++k) cm[k] = 0;
-    for (int64_t r = tid; r < rows; r += kThreads) {
-      uint32_t rmx = 0;
-#pragma unroll
-      for (int k = 0; k < CW; ++k) {
-        if (k < ncol) {
-          const uint32_t a =
-              quant_one<kOut16>(Key<T>::value(S[r * CW + k]), s_s[k], Xint, (c0 + k) * ldq + r, status);
-          rmx = max(rmx, a);
-          cm[k] = max(cm[k], a);
-        }
-      }
-      if (prow) prow[r] = (int32_t)rmx;
     }
 #pragma unroll
-    for (int k = 0; k < CW; ++k) {
-      uint32_t m = cm[k];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if ((tid & 31) == 0 && m) atomicMax(&s_cmax[k], m);
-    }
+    for (int o = 16; o > 0; o >>= 1) cmx = max(cmx, __shfl_xor_sync(0xffffffffu, cmx, o));
+    if (lane == 0 && colmax) colmax[c] = (int32_t)cmx;
   }
-  __syncthreads();
-  if (colmax && tid < ncol) colmax[c0 + tid] = (int32_t)s_cmax[tid];
+  if (part) {
+    __syncthreads();
+    int32_t* mine = part + (int64_t)blockIdx.x * rows;
+    for (int r = tid; r < n; r += CW * 32) mine[r] = (int32_t)rmax[r];
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -595,7 +555,8 @@ template <typename T, int CW, bool kOut16>
 imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, unsigned long long k, int32_t beta,
                            void* Xint, int64_t ldq, int trans_out, float* delta, float* qval, int32_t* rowmax,
                            int32_t* colmax, DeviceState* ds, cudaStream_t st) {
-  const size_t smem = (size_t)rows * CW * sizeof(T);
+  const size_t colstride = (size_t)(rows + 7) / 8 * 8;
+  const size_t smem = (size_t)CW * colstride * sizeof(T) + (size_t)rows * 4;
   const bool vec = (ld % (16 / (int64_t)sizeof(T)) == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   const int64_t grid = (cols + CW - 1) / CW;
   int32_t* part = nullptr;
@@ -607,8 +568,8 @@ imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, u
   }
   auto kern = k_rtn_cols_staged<T, CW, kOut16>;
   IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, part,
-                                               colmax, vec ? 1 : 0, ds->status);
+  kern<<<(unsigned)grid, CW * 32, smem, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, part,
+                                              colmax, vec ? 1 : 0, ds->status);
   if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
   return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
 }
@@ -620,13 +581,17 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
   const int sms = ds->num_sms;
   if (g == IMQ_PER_COL) {
     const unsigned long long k = (unsigned long long)nearest_rank(rows, p);
-    // the slab of 16 (or 8) columns is staged in shared memory when it fits
+    // the slab of 16 (or 8) columns is staged in shared memory when it fits (plus the row maxima)
     constexpr size_t kSlab = 192 * 1024;
-    if ((size_t)rows * 16 * sizeof(T) <= kSlab)
+    const size_t colb = (size_t)(rows + 7) / 8 * 8 * sizeof(T);
+    if (16 * colb + (size_t)rows * 4 <= kSlab)
       return run_cols_staged<T, 16, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
                                             colmax, ds, st);
-    if ((size_t)rows * 8 * sizeof(T) <= kSlab)
+    if (8 * colb + (size_t)rows * 4 <= kSlab)
       return run_cols_staged<T, 8, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
+                                           colmax, ds, st);
+    if (4 * colb + (size_t)rows * 4 <= kSlab)
+      return run_cols_staged<T, 4, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
                                            colmax, ds, st);
     const int64_t grid = (cols + kColsPerCta - 1) / kColsPerCta;
     int32_t* part = nullptr;

@@ -7,8 +7,10 @@
 //
 // Both unpacked operands are K-major (the inner index contiguous) because that is what the tcgen05
 // GEMM reads through TMA.  Two kernels cover the two storage orders of a source matrix:
-//   k_unpack_rows  the source line is a stored row (A, or B given as B^T): one CTA stages the line in
-//                  shared memory and streams out all its unpacked lines with 16-byte stores.
+//   k_unpack_rows  the source line is a stored row (A, or B given as B^T): a CTA writes the digit planes
+//                  of a batch of lines to shared memory and streams out their unpacked lines, 16-byte
+//                  copies for the inner blocks the plan marked contiguous (k_unpack_rows_direct gathers
+//                  from global memory when the planes do not fit).
 //   k_unpack_cols  the source line is a stored column (B, or A given as A^T): a CTA transposes a
 //                  128 (inner) x 32 (lines) tile through shared memory, reading 64-byte row segments
 //                  and writing 128-byte segments of unpacked lines.
@@ -20,60 +22,143 @@
 namespace imq {
 namespace {
 
-// Row gather: a CTA stages a batch of NL source lines in shared memory, then for each 4-byte piece of
-// the inner dimension reads the index maps once and writes the digits of every line of the batch (and
-// every level of an OUTER line).  Lines too long to stage are gathered from global memory (L2).
-template <typename T, bool kStaged>
+// Row gather: a CTA takes a batch of NL source lines and writes their digit planes to shared memory,
+// plane[b][l][t] = d_l(line b, entry t) for the P levels the batch needs, one byte each.  Then each
+// lane writes 16 consecutive inner positions of an output line: a block the plan marked contiguous
+// (t0..t0+15, one level) is a 16-byte copy from a plane; any other block is gathered byte by byte.
+template <typename T>
 __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, int64_t nlines, int64_t K,
-                                                     int64_t ld, int NL, int outer, const int8_t* __restrict__ lvl,
-                                                     const int32_t* __restrict__ pos,
-                                                     const int32_t* __restrict__ tK,
-                                                     const int8_t* __restrict__ lk, int64_t K_unp,
-                                                     int bm1, int8_t* __restrict__ out) {
+                                                     int64_t ld, int NL, int P, int outer,
+                                                     const int8_t* __restrict__ lvl, const int32_t* __restrict__ pos,
+                                                     const int32_t* __restrict__ tK, const int8_t* __restrict__ lk,
+                                                     const int32_t* __restrict__ blk16, int64_t K_unp, int bm1,
+                                                     int8_t* __restrict__ out) {
   extern __shared__ __align__(16) unsigned char dsm[];
-  T* lines = reinterpret_cast<T*>(dsm);  // [NL][K]
+  const int64_t Kp = (K + 15) / 16 * 16;  // plane row length, 16-byte aligned
+  int8_t* planes = reinterpret_cast<int8_t*>(dsm);  // [NL][P][Kp]
   __shared__ int s_L[8];
   __shared__ int64_t s_base[8];
   const int tid = threadIdx.x;
+  const int64_t nchunk = K_unp / 16;
+  const bool vec4 = (K % 4 == 0) && (ld % 4 == 0);
   for (int64_t i0 = (int64_t)blockIdx.x * NL; i0 < nlines; i0 += (int64_t)gridDim.x * NL) {
     const int nb = nlines - i0 < NL ? (int)(nlines - i0) : NL;
     if (tid < nb) {
       s_L[tid] = outer ? (int)lvl[i0 + tid] : 1;
       s_base[tid] = outer ? (int64_t)pos[i0 + tid] : i0 + tid;
     }
-    if (kStaged) {
-      for (int b = 0; b < nb; ++b)
-        for (int64_t t = tid; t < K; t += 256) lines[b * K + t] = X[(i0 + b) * ld + t];
-    }
-    __syncthreads();
-    // lane = 4 consecutive inner positions, a warp = 128: index maps read once per batch, 128-byte
-    // coalesced stores, shared-memory gathers at most 2-way bank conflicted
-    const int lane = tid & 31, warp = tid >> 5;
-    for (int64_t p = (int64_t)warp * 128 + lane * 4; p < K_unp; p += 8 * 128) {
-      const int4 t4 = *reinterpret_cast<const int4*>(tK + p);
-      const uint32_t l4 = *reinterpret_cast<const uint32_t*>(lk + p);
-      const int32_t tt[4] = {t4.x, t4.y, t4.z, t4.w};
-      int ll[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) ll[r] = (int)(int8_t)(l4 >> (8 * r));
-      for (int b = 0; b < nb; ++b) {
+    // digit planes: 4 entries per thread and iteration, one 4-byte store per plane
+    for (int b = 0; b < nb; ++b) {
+      const T* xr = X + (i0 + b) * ld;
+      int8_t* pb = planes + (int64_t)b * P * Kp;
+      for (int64_t t = (int64_t)tid * 4; t < Kp; t += 256 * 4) {
         int32_t v[4];
+        if (vec4 && t + 3 < K) {
+          if (sizeof(T) == 2) {
+            const uint2 w = *reinterpret_cast<const uint2*>(xr + t);
+            v[0] = (int16_t)(w.x & 0xFFFFu); v[1] = (int16_t)(w.x >> 16);
+            v[2] = (int16_t)(w.y & 0xFFFFu); v[3] = (int16_t)(w.y >> 16);
+          } else {
+            const int4 w = *reinterpret_cast<const int4*>(xr + t);
+            v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) v[r] = t + r < K ? (int32_t)xr[t + r] : 0;
+        }
+        uint32_t a[4], sg[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const int32_t t = tt[r] >= 0 ? tt[r] : 0;
-          v[r] = tt[r] < 0 ? 0 : (kStaged ? (int32_t)lines[b * K + t] : (int32_t)X[(i0 + b) * ld + t]);
+          sg[r] = v[r] < 0 ? 0xFFFFFFFFu : 0u;
+          a[r] = v[r] < 0 ? (uint32_t)(-(int64_t)v[r]) : (uint32_t)v[r];
         }
-        const int L = s_L[b];
-        for (int l = 0; l < L; ++l) {
+        const uint32_t mask = (1u << bm1) - 1u;
+        for (int l = 0; l < P; ++l) {
+          const int sh = l * bm1;
           uint32_t packed = 0;
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
-            packed |= ((uint32_t)(uint8_t)(int8_t)digit_of(v[r], l + ll[r], bm1)) << (8 * r);
-          *reinterpret_cast<uint32_t*>(out + (s_base[b] + l) * K_unp + p) = packed;
+          for (int r = 0; r < 4; ++r) {
+            const uint32_t d = sh < 31 ? ((a[r] >> sh) & mask) : 0u;
+            packed |= (((d ^ sg[r]) - sg[r]) & 0xFFu) << (8 * r);
+          }
+          *reinterpret_cast<uint32_t*>(pb + (int64_t)l * Kp + t) = packed;
         }
       }
     }
     __syncthreads();
+    for (int64_t c = tid; c < nchunk; c += 256) {
+      const int32_t t0 = blk16[c];
+      const int64_t p = c * 16;
+      if (t0 >= 0) {
+        const int lk0 = lk[p];
+        for (int b = 0; b < nb; ++b) {
+          const int L = s_L[b];
+          for (int l = 0; l < L; ++l) {
+            const uint4 w = *reinterpret_cast<const uint4*>(planes + ((int64_t)b * P + l + lk0) * Kp + t0);
+            *reinterpret_cast<uint4*>(out + (s_base[b] + l) * K_unp + p) = w;
+          }
+        }
+      } else {
+        const int4* tq = reinterpret_cast<const int4*>(tK + p);
+        const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
+        const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
+                                tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
+        const int4 lq = *reinterpret_cast<const int4*>(lk + p);
+        const int8_t* ll = reinterpret_cast<const int8_t*>(&lq);
+        for (int b = 0; b < nb; ++b) {
+          const int L = s_L[b];
+          for (int l = 0; l < L; ++l) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t packed = 0;
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int k = q * 4 + r;
+                const uint32_t byte =
+                    tt[k] >= 0 ? (uint8_t)planes[((int64_t)b * P + l + ll[k]) * Kp + tt[k]] : 0u;
+                packed |= byte << (8 * r);
+              }
+              w[q] = packed;
+            }
+            *reinterpret_cast<uint4*>(out + (s_base[b] + l) * K_unp + p) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Row gather for lines too long for shared-memory planes: digits are computed from the source line in
+// global memory (L2); lane = 4 consecutive inner positions, 128-byte coalesced stores per warp.
+template <typename T>
+__global__ void __launch_bounds__(256) k_unpack_rows_direct(const T* __restrict__ X, int64_t nlines, int64_t ld,
+                                                            int outer, const int8_t* __restrict__ lvl,
+                                                            const int32_t* __restrict__ pos,
+                                                            const int32_t* __restrict__ tK,
+                                                            const int8_t* __restrict__ lk, int64_t K_unp, int bm1,
+                                                            int8_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t i = blockIdx.x; i < nlines; i += gridDim.x) {
+    const T* xr = X + i * ld;
+    const int L = outer ? (int)lvl[i] : 1;
+    const int64_t base = outer ? (int64_t)pos[i] : i;
+    for (int64_t p = (int64_t)warp * 128 + lane * 4; p < K_unp; p += 8 * 128) {
+      const int4 t4 = *reinterpret_cast<const int4*>(tK + p);
+      const uint32_t l4 = *reinterpret_cast<const uint32_t*>(lk + p);
+      const int32_t tt[4] = {t4.x, t4.y, t4.z, t4.w};
+      int32_t v[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) v[r] = tt[r] >= 0 ? (int32_t)xr[tt[r]] : 0;
+      for (int l = 0; l < L; ++l) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          packed |= ((uint32_t)(uint8_t)(int8_t)digit_of(v[r], l + (int)(int8_t)(l4 >> (8 * r)), bm1)) << (8 * r);
+        *reinterpret_cast<uint32_t*>(out + (base + l) * K_unp + p) = packed;
+      }
+    }
   }
 }
 
@@ -134,31 +219,33 @@ __global__ void k_zero_unused(const int32_t* __restrict__ grpL, const int32_t* _
 }
 
 template <typename T>
-imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool line_is_row, int outer,
+imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool line_is_row, int outer, int P,
                       const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
-                      int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st) {
+                      const int32_t* blk16, int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st) {
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
   if (line_is_row) {
-    // batches of up to 8 lines (64 KB of shared memory per CTA at most); lines longer than that are
-    // gathered from global memory
-    const size_t line_bytes = (size_t)(K > 0 ? K : 1) * sizeof(T);
-    int NL = (int)((64 * 1024) / line_bytes);
+    // P planes per line: the levels an output line can ask for (line level + inner level)
+    const int64_t Kp = (K + 15) / 16 * 16;
+    int NL = (int)((96 * 1024) / ((int64_t)P * Kp));
     if (NL > 8) NL = 8;
-    const bool staged = NL >= 1;
-    if (!staged) NL = 8;
-    const size_t smem = staged ? (size_t)NL * line_bytes : 0;
-    const int per_sm = staged ? (int)((200 * 1024) / (smem + 2048)) : 8;
-    const int64_t batches = (nlines + NL - 1) / NL;
-    int64_t grid = (int64_t)num_sms * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
-    if (grid > batches) grid = batches;
-    if (staged) {
-      IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_rows<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      k_unpack_rows<T, true><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, NL, outer, lvl, pos, tK, lk, K_unp,
-                                                                bm1, out);
-    } else {
-      k_unpack_rows<T, false><<<(unsigned)grid, 256, 0, st>>>(X, nlines, K, ld, NL, outer, lvl, pos, tK, lk, K_unp,
-                                                              bm1, out);
+    if (NL < 1) {
+      if ((int64_t)P * Kp > 200 * 1024) {
+        // planes do not fit: compute the digits straight from global memory
+        const int64_t grid = nlines < (int64_t)num_sms * 8 ? nlines : (int64_t)num_sms * 8;
+        k_unpack_rows_direct<T><<<(unsigned)grid, 256, 0, st>>>(X, nlines, ld, outer, lvl, pos, tK, lk, K_unp, bm1,
+                                                                 out);
+        return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+      }
+      NL = 1;
     }
+    const size_t smem = (size_t)NL * P * Kp;
+    const int per_sm = (int)((200 * 1024) / (smem + 2048)) < 1 ? 1 : (int)((200 * 1024) / (smem + 2048));
+    const int64_t batches = (nlines + NL - 1) / NL;
+    int64_t grid = (int64_t)num_sms * (per_sm > 8 ? 8 : per_sm);
+    if (grid > batches) grid = batches;
+    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_rows<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_unpack_rows<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, NL, P, outer, lvl, pos, tK, lk, blk16,
+                                                        K_unp, bm1, out);
   } else {
     const dim3 grid((unsigned)((nlines + 31) / 32), (unsigned)(K_unp / 128));
     if (K_unp / 128 > 65535) return IMQ_ERR_UNSUPPORTED;
@@ -174,12 +261,15 @@ imq_status unpack_typed(const imq_plan_t* pl, const T* A, const T* B, int8_t* Au
   const int bm1 = I.b - 1;
   const int a_outer = I.dir_a == IMQ_DIR_OUTER, b_outer = I.dir_b == IMQ_DIR_OUTER;
   // A' lines are the logical rows of A: stored rows unless A is given transposed
-  imq_status s = unpack_one<T>(A, I.M, I.K, pl->lda, !pl->transA, a_outer, pl->lv_a_row, pl->posA, pl->tK,
-                               pl->lAk, I.K_unp, bm1, Au, num_sms, st);
+  // planes an output line may read: OUTER lines their own levels, INNER ones the inner levels
+  const int pa = a_outer ? I.lmax_a_row : (I.dir_a == IMQ_DIR_INNER ? I.lmax_a_col : 1);
+  const int pb = b_outer ? I.lmax_b_col : (I.dir_b == IMQ_DIR_INNER ? I.lmax_b_row : 1);
+  imq_status s = unpack_one<T>(A, I.M, I.K, pl->lda, !pl->transA, a_outer, pa, pl->lv_a_row, pl->posA, pl->tK,
+                               pl->lAk, pl->blk16, I.K_unp, bm1, Au, num_sms, st);
   if (s != IMQ_OK) return s;
   // B'^T lines are the logical columns of B: stored rows only when B is given transposed
-  s = unpack_one<T>(B, I.N, I.K, pl->ldb, pl->transB != 0, b_outer, pl->lv_b_col, pl->posB, pl->tK, pl->lBk,
-                    I.K_unp, bm1, Bu, num_sms, st);
+  s = unpack_one<T>(B, I.N, I.K, pl->ldb, pl->transB != 0, b_outer, pb, pl->lv_b_col, pl->posB, pl->tK, pl->lBk,
+                    pl->blk16, I.K_unp, bm1, Bu, num_sms, st);
   if (s != IMQ_OK) return s;
   if (I.K_unp > 0) {
     if (a_outer && pl->n_grp_a > 0)
