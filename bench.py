@@ -48,6 +48,21 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of `values` over all ranks (the slowest rank decides a step's time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def throughput(ops_per_step: float, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput in TOPS: every rank runs `steps` steps of `ops_per_step` operations."""
+    return ops_per_step * world * steps / (total_ms * 1e-3) / 1e12
+
+
 def _workload():
     g = workloads.q_proj()[0]
     return g
@@ -239,15 +254,12 @@ def run_ours(args):
     barrier()
     e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_start, e_end))
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist if world > 1 else None, dev)
 
     I = path.info
     ops = 2.0 * g.M * g.N * g.K
-    value = ops * world * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = ops * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = throughput(ops, world, args.steps, total_ms)
+    e2e_value = throughput(ops, world, args.steps, e2e_ms)
     bf16_burst, bf16_sus, hbm, src = _peaks()
     int8_peak = 2.0 * bf16_burst  # dense int8 = 2 x dense bf16 on B200 (nominal 4.5 vs 2.25 PFLOP/s)
     exec_ops = 2.0 * I["M_unp"] * I["N_unp"] * I["K_unp"]
