@@ -20,7 +20,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -82,47 +81,79 @@ def _config(g, extra=None):
 # clocks during the timed region
 # ------------------------------------------------------------------------------------------------
 class Clocks:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, read (never set) every few milliseconds on a host
+    thread through NVML while the timed region runs, so that even a short region gets samples.  The
+    GPU is found by its UUID, since NVML numbers GPUs without regard to CUDA_VISIBLE_DEVICES."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device, period_s: float = 0.004):
+        self.device = device
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.handle = None
+        self.error = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            u = str(torch.cuda.get_device_properties(self.device).uuid)
+            for cand in (u, "GPU-" + u):
+                try:
+                    return nv.nvmlDeviceGetHandleByUUID(cand)
+                except Exception:
+                    pass
+        except Exception:
+            pass
+        if nv.nvmlDeviceGetCount() == 1:
+            return nv.nvmlDeviceGetHandleByIndex(0)
+        raise RuntimeError("GPU not identified in NVML")
+
+    def _run(self, nv):
+        import time as _t
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, rs))
+            except Exception as e:  # keep what was read so far
+                self.error = str(e)
+                return
+            _t.sleep(self.period)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            self.handle = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._run, args=(nv,), daemon=True)
+            self._thread.start()
+        except Exception as e:
+            self.error = str(e)
+            self._thread = None
         return self
 
     def __exit__(self, *a):
-        self.samples = []
-        if self.proc is None:
-            return
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out = ""
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) >= 9:
-                self.samples.append(f)
+        if getattr(self, "_thread", None) is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
 
     def summary(self):
-        if not getattr(self, "samples", None):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for s in self.samples for k in range(4) if s[5 + k] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "error": self.error}
+        sm = [s for s, _ in self.samples]
+        seen = 0
+        for _, r in self.samples:
+            seen |= int(r)
+        reasons = sorted(name for bit, name in self.REASONS.items() if seen & bit)
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "NVML"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -219,7 +250,7 @@ def run_ours(args):
     gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
-    with Clocks(dev.index) as clk:
+    with Clocks(dev) as clk:
         for k in range(args.steps):
             flush.zero_()
             starts[k].record()
@@ -376,7 +407,7 @@ def _traffic_from_profiles():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")

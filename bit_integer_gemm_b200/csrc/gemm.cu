@@ -121,13 +121,21 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
 }
 
 // Per-warp drain metadata of one tile, fetched before the accumulator is ready: row offsets and row
-// scales in shared memory (read as broadcasts), column indices and column scales in registers.
+// scales in shared memory, column indices and column scales in registers.  In the store phase of a
+// chunk with nB output columns, lane t writes column s = t % nB of the rows r0 = t / nB, r0 + per, ...
+// (per = 32 / nB rows at a time), so that all lanes store even when nB < 32.
 struct DrainMeta {
   int LA, nA;
-  int LB[BN / 32], nB[BN / 32];
-  int32_t col[BN / 32];  // this lane's output column in each chunk (lane < nB)
+  int32_t pk[BN / 32];   // per chunk: nB | LB << 6 | s << 12 | r0 << 18 | per << 24 (r0 = 63: idle lane)
+  int32_t col[BN / 32];  // the output column of this lane's s in each chunk
   float sb[BN / 32];     // its dequantisation scale
 };
+
+__device__ __forceinline__ int pk_nB(int32_t pk) { return pk & 63; }
+__device__ __forceinline__ int pk_LB(int32_t pk) { return (pk >> 6) & 63; }
+__device__ __forceinline__ int pk_s(int32_t pk) { return (pk >> 12) & 63; }
+__device__ __forceinline__ int pk_r0(int32_t pk) { return (pk >> 18) & 63; }
+__device__ __forceinline__ int pk_per(int32_t pk) { return (pk >> 24) & 63; }
 
 struct WarpRows {       // shared memory, per epilogue warp
   int32_t row[32];      // the output row lane t holds after the row fold
@@ -158,23 +166,28 @@ __device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt,
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) {
     const int64_t gc = (int64_t)nt * (BN / 32) + c;
+    int LB = 1, nB = 0;
     if (g.b_outer) {
-      m.LB[c] = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
-      m.nB[c] = gc < g.n_grp_b ? g.grpB_n[gc] : 0;
+      LB = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
+      nB = gc < g.n_grp_b ? g.grpB_n[gc] : 0;
     } else {
-      m.LB[c] = 1;
       const int64_t rem = g.N - gc * 32;
-      m.nB[c] = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
+      nB = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
     }
-  }
-#pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    const int64_t gc = (int64_t)nt * (BN / 32) + c;
+    int s = 0, r0 = 63, per = 1;
+    if (nB > 0) {
+      per = 32 / nB;
+      s = lane % nB;
+      r0 = lane / nB;
+      if (r0 >= per) r0 = 63;
+    }
+    m.pk[c] = nB | (LB << 6) | (s << 12) | (r0 << 18) | (per << 24);
     m.col[c] = 0;
-    if (lane < m.nB[c]) m.col[c] = g.b_outer ? g.srcB[gc * 32 + (int64_t)lane * m.LB[c]] : (int32_t)(gc * 32 + lane);
+    if (r0 != 63) m.col[c] = g.b_outer ? g.srcB[gc * 32 + (int64_t)s * LB] : (int32_t)(gc * 32 + s);
   }
 #pragma unroll
-  for (int c = 0; c < BN / 32; ++c) m.sb[c] = (last && g.Cf && lane < m.nB[c]) ? g.dB[g.dB_per_col ? m.col[c] : 0] : 0.0f;
+  for (int c = 0; c < BN / 32; ++c)
+    m.sb[c] = (last && g.Cf && pk_r0(m.pk[c]) != 63) ? g.dB[g.dB_per_col ? m.col[c] : 0] : 0.0f;
   __syncwarp();
 }
 
@@ -199,16 +212,16 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
       if (lane == 0) mbar_arrive(acce_bar);
     }
     // dynamic indexing of the unrolled metadata arrays is avoided by a uniform select
-    int LB = 1, nB = 0, mycol = 0;
+    int32_t pk = 0, mycol = 0;
     float sb = 0.0f;
 #pragma unroll
     for (int k = 0; k < BN / 32; ++k)
       if (k == c) {
-        LB = m.LB[k];
-        nB = m.nB[k];
+        pk = m.pk[k];
         mycol = m.col[k];
         sb = m.sb[k];
       }
+    const int LB = pk_LB(pk), nB = pk_nB(pk);
     const int nA = m.nA, LA = m.LA;
     if (nB == 0 || nA == 0) continue;
     // 1. fold the column levels of B inside the registers (lane = unpacked row)
@@ -256,11 +269,13 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
     for (int s2 = 0; s2 < 32; ++s2)
       if (s2 < nB) scr[sw(lane, s2)] = shl<T>(w[s2], shift);
     __syncwarp();
-    // 4. lane = output column: coalesced accesses along each row of C
-    if (lane < nB) {
+    // 4. lane (r0, s) stores column s of rows r0, r0 + per, ...: each row of C takes nB neighbouring
+    //    lanes, and all 32 / nB rows of a pass go out in one instruction
+    {
+      const int s = pk_s(pk), per = pk_per(pk);
 #pragma unroll 4
-      for (int r = 0; r < nA; ++r) {
-        T val = scr[sw(r, lane)];
+      for (int r = pk_r0(pk); r < nA; r += per) {
+        T val = scr[sw(r, s)];
         const int64_t row = wr->row[r];
         if (g.C) {
           if (g.c64) {
