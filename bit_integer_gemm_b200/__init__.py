@@ -32,6 +32,7 @@ IMQ_MIX, IMQ_ROW_ROW, IMQ_ROW_COL, IMQ_COL_ROW, IMQ_COL_COL = 0, 1, 2, 3, 4
 # directions
 IMQ_DIR_NONE, IMQ_DIR_OUTER, IMQ_DIR_INNER = 0, 1, 2
 IMQ_MAX_GROUPS = 64
+IMQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _TORCH_TO_IMQ = {torch.float32: IMQ_F32, torch.bfloat16: IMQ_BF16, torch.int16: IMQ_I16,
                  torch.int32: IMQ_I32, torch.int64: IMQ_I64}
@@ -75,6 +76,8 @@ _VP, _I32, _I64, _F64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ct
 SIGNATURES = {
     "imq_rtn_quantize": [_VP, _I32, _I64, _I64, _I64, _I32, _F64, _I32, _VP, _I32, _I64, _I32, _VP, _VP, _VP, _VP,
                          _VP],
+    "imq_rtn_quantize_rows_noalloc": [_VP, _I32, _I64, _I64, _I64, _F64, _I32, _VP, _I32, _I64, _VP, _VP, _VP,
+                                      _VP, _VP],
     "imq_plan": [_VP, _VP, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32, _VP, _VP, _VP, _VP,
                  ctypes.POINTER(_VP), _VP],
     "imq_plan_info_get": [_VP, ctypes.POINTER(imq_plan_info)],
@@ -161,6 +164,31 @@ def imq_rtn_quantize(X: torch.Tensor, gran: int, p: float, beta: int, out_dtype=
                                 _ptr(qval),
                                 _ptr(rowmax), _ptr(colmax), _stream(stream))
     _check(st, "imq_rtn_quantize")
+    return Quantized(Xint, delta, qval, rowmax, colmax)
+
+
+def imq_rtn_quantize_rows_noalloc(X: torch.Tensor, p: float, beta: int, out_dtype=torch.int16, Xint=None,
+                                  delta=None, qval=None, rowmax=None, colmax=None, want_qval=True,
+                                  want_max=True, stream=None) -> Quantized:
+    """Per-row RTN quantisation like imq_rtn_quantize(X, IMQ_PER_ROW, ...), with the library's scratch
+    in a fixed device array instead of allocated memory (outputs not given are allocated here by torch).
+    Calls whose executions overlap on one device race on that array."""
+    rows, cols = X.shape
+    dev = X.device
+    if Xint is None:
+        Xint = torch.empty((rows, cols), dtype=out_dtype, device=dev)
+    if delta is None:
+        delta = torch.empty(rows, dtype=torch.float32, device=dev)
+    if qval is None and want_qval:
+        qval = torch.empty(rows, dtype=torch.float32, device=dev)
+    if rowmax is None and want_max:
+        rowmax = torch.empty(rows, dtype=torch.int32, device=dev)
+    if colmax is None and want_max:
+        colmax = torch.empty(cols, dtype=torch.int32, device=dev)
+    st = lib().imq_rtn_quantize_rows_noalloc(_ptr(X), _TORCH_TO_IMQ[X.dtype], rows, cols, _ld(X), float(p),
+                                             int(beta), _ptr(Xint), _TORCH_TO_IMQ[Xint.dtype], _ld(Xint),
+                                             _ptr(delta), _ptr(qval), _ptr(rowmax), _ptr(colmax), _stream(stream))
+    _check(st, "imq_rtn_quantize_rows_noalloc")
     return Quantized(Xint, delta, qval, rowmax, colmax)
 
 

@@ -104,6 +104,14 @@ imq_status imq_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t c
                                   colmax, reinterpret_cast<cudaStream_t>(stream));
 }
 
+imq_status imq_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                         double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq,
+                                         float* delta, float* qval, int32_t* rowmax, int32_t* colmax,
+                                         imq_stream_t stream) {
+  return imq::launch_rtn_quantize_rows_noalloc(X, xt, rows, cols, ld, p, beta, Xint, it, ldq, delta, qval, rowmax,
+                                               colmax, reinterpret_cast<cudaStream_t>(stream));
+}
+
 imq_status imq_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
                     int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b, imq_strategy strategy,
                     const int32_t* a_rowmax, const int32_t* a_colmax, const int32_t* b_rowmax,

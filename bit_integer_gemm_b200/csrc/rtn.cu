@@ -22,6 +22,9 @@
 // second small kernel (no global atomics).
 #include <math.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -693,6 +696,115 @@ imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_
   const uint32_t* x = static_cast<const uint32_t*>(X);
   return o16 ? run<uint32_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st)
              : run<uint32_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free per-row quantiser (imq_rtn_quantize_rows_noalloc).
+//
+// Callers whose own allocator has reserved the free device memory, or that must not stall their other
+// streams behind the device-wide wait of a cudaFree, cannot use the grown partials buffer above.  For
+// them the per-CTA column maxima of k_rtn_rows go to one fixed array in this module's device image,
+// mapped by the CUDA runtime when the module loads.  Its device address is looked up once per device,
+// on the first call with that device current.  Every call on a device shares the array, so calls whose
+// executions overlap race on it.  Nothing in it has to start at zero: each CTA writes its whole slice
+// of partial maxima before k_reduce_max reads them.
+// ------------------------------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoallocBytes = IMQ_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocBytes / sizeof(int32_t)];
+std::atomic<int32_t*> g_noalloc_ptr[64];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (looked up on the first call there).
+imq_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return IMQ_ERR_UNSUPPORTED;
+  int32_t* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!ptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    ptr = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (!ptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return IMQ_ERR_CUDA;
+      ptr = static_cast<int32_t*>(p);
+      g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+    }
+  }
+  *out = ptr;
+  return IMQ_OK;
+}
+
+// The per-row branch of run() with the partials taken from the scratch array: same launch shape, same
+// kernel, so the results are those of imq_rtn_quantize with g = IMQ_PER_ROW, trans_out = 0.
+template <typename T, bool kOut16>
+imq_status run_rows_noalloc(const T* X, int64_t rows, int64_t cols, int64_t ld, double p, int32_t beta,
+                            void* Xint, int64_t ldq, float* delta, float* qval, int32_t* rowmax, int32_t* colmax,
+                            DeviceState* ds, cudaStream_t st) {
+  const int sms = ds->num_sms;
+  const size_t row_bytes = (size_t)((cols * (int64_t)sizeof(T) + 15) / 16 * 16);
+  const size_t cmax_bytes = colmax ? (size_t)((cols * 4 + 15) / 16 * 16) : 0;
+  constexpr size_t kBudget = 200 * 1024;
+  if (cmax_bytes + row_bytes > kBudget) return IMQ_ERR_UNSUPPORTED;
+  int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
+  if (nwarps > kThreads / 32) nwarps = kThreads / 32;
+  const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
+  int per_sm = (int)(kBudget / (smem + 9 * 1024));
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 4) per_sm = 4;
+  const int64_t blocks = (rows + nwarps - 1) / nwarps;
+  const int64_t grid = blocks < (int64_t)sms * per_sm ? blocks : (int64_t)sms * per_sm;
+  const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  int32_t* part = nullptr;
+  if (colmax) {
+    // checked before anything is launched: the kernel writes grid x cols partials
+    if ((uint64_t)grid * (uint64_t)cols * sizeof(int32_t) > kNoallocBytes) return IMQ_ERR_UNSUPPORTED;
+    imq_status e = noalloc_scratch(&part);
+    if (e != IMQ_OK) return e;
+  }
+  auto kern = k_rtn_rows<T, true, kOut16>;
+  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta,
+                                               Xint, ldq, 0, delta, qval, rowmax, part, nullptr, vec, nwarps,
+                                               ds->status);
+  if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
+  return colmax ? launch_reduce_max(part, grid, cols, colmax, st) : IMQ_OK;
+}
+}  // namespace
+
+imq_status launch_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                                            double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq,
+                                            float* delta, float* qval, int32_t* rowmax, int32_t* colmax,
+                                            cudaStream_t st) {
+  if (rows < 0 || cols < 0 || ld < cols || ldq < cols || !(p > 0.0 && p <= 1.0) || beta < 1 || beta > (1 << 24))
+    return IMQ_ERR_ARG;
+  if (xt != IMQ_F32 && xt != IMQ_BF16) return IMQ_ERR_ARG;
+  if (it != IMQ_I16 && it != IMQ_I32) return IMQ_ERR_ARG;
+  if (!delta && rows > 0) return IMQ_ERR_ARG;
+  if ((!X || !Xint) && rows > 0 && cols > 0) return IMQ_ERR_ARG;
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  if (rows == 0 || cols == 0) {
+    // every row is empty: q = max = 0, so s = Delta = 1 and there is nothing to quantise
+    if (rowmax && rows > 0) IMQ_CUDA_TRY(cudaMemsetAsync(rowmax, 0, (size_t)rows * 4, st));
+    if (colmax && cols > 0) IMQ_CUDA_TRY(cudaMemsetAsync(colmax, 0, (size_t)cols * 4, st));
+    if (rows > 0) {
+      k_fill_f32<<<1, 256, 0, st>>>(delta, rows, 1.0f);
+      if (qval) k_fill_f32<<<1, 256, 0, st>>>(qval, rows, 0.0f);
+    }
+    return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+  }
+  const bool o16 = it == IMQ_I16;
+  if (xt == IMQ_BF16) {
+    const uint16_t* x = static_cast<const uint16_t*>(X);
+    return o16 ? run_rows_noalloc<uint16_t, true>(x, rows, cols, ld, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st)
+               : run_rows_noalloc<uint16_t, false>(x, rows, cols, ld, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st);
+  }
+  const uint32_t* x = static_cast<const uint32_t*>(X);
+  return o16 ? run_rows_noalloc<uint32_t, true>(x, rows, cols, ld, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st)
+             : run_rows_noalloc<uint32_t, false>(x, rows, cols, ld, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st);
 }
 
 }  // namespace imq

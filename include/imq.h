@@ -108,6 +108,39 @@ imq_status imq_rtn_quantize(const void *X, imq_dtype xt, int64_t rows, int64_t c
                             float *delta, float *qval, int32_t *rowmax, int32_t *colmax,
                             imq_stream_t stream);
 
+/*
+ * imq_rtn_quantize_rows_noalloc -- imq_rtn_quantize with g = IMQ_PER_ROW and trans_out = 0 (the
+ * per-token quantisation of an activation), with the same arguments otherwise and the same results,
+ * but it allocates no device memory.  The IM-Unpack page has no counterpart to this call: it is an
+ * interface convenience of this library, not a step of the method.
+ *
+ * Why: imq_rtn_quantize keeps the per-CTA partial column maxima in a library buffer that it grows
+ * with cudaMalloc, freeing the old one with cudaFree, which waits for all work on the device.  Two
+ * kinds of caller cannot take that: a process whose own allocator has reserved the free device
+ * memory up front (a serving engine that owns every byte of HBM, where the library's cudaMalloc
+ * fails), and a caller that must not stall its other streams behind a device-wide cudaFree.  This
+ * call takes its scratch from one fixed array in the library's device image instead, of
+ * IMQ_NOALLOC_SCRATCH_BYTES per device, which the CUDA runtime maps when it loads the module.
+ *
+ * Scratch needed: 4 * cols * G bytes when colmax is requested, where G is the number of CTAs the
+ * per-row kernel uses (at most 4 per SM; fewer for wide rows).  On 148 SMs any cols <= 3542 fits,
+ * and a 2048 x 4096 bf16 activation takes 4 MiB.  None when colmax is NULL.  Nothing in the
+ * scratch has to start at zero: each CTA writes its whole slice before the reduction reads it.
+ * Errors: those of imq_rtn_quantize, plus IMQ_ERR_UNSUPPORTED, returned at once with nothing launched,
+ * when the scratch needed exceeds IMQ_NOALLOC_SCRATCH_BYTES.
+ * Set-up: the first call on a device looks up the device address of the scratch array for that
+ * device (cudaGetSymbolAddress, with that device current); make this first call before any stream
+ * capture.
+ * Concurrency: every call on a device uses the same scratch array, so calls whose executions overlap
+ * (on different streams, or from different host threads without ordering) race on it and may return
+ * wrong column maxima.  Order them on one stream or with events.
+ */
+#define IMQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+imq_status imq_rtn_quantize_rows_noalloc(const void *X, imq_dtype xt, int64_t rows, int64_t cols,
+                                         int64_t ld, double p, int32_t beta, void *Xint, imq_dtype it,
+                                         int64_t ldq, float *delta, float *qval, int32_t *rowmax,
+                                         int32_t *colmax, imq_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------------ */
 /* 2. Unpack plan                                                                                    */
 /* ------------------------------------------------------------------------------------------------ */
