@@ -36,13 +36,26 @@ constexpr int BM = 128, BN = 256, BK = 128;
 constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK;  // bytes
 constexpr int B_STAGE = BN * BK;
-constexpr int NUM_THREADS = 192;
-constexpr int EPI_WARPS = 4;
+constexpr int NCHUNK = BN / 32;   // 32-column chunks of an accumulator slot
 constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+// Epilogue shape per accumulation width: with int32 values two warps share each TMEM lane quarter (each
+// takes every other chunk), with int64 values one warp per quarter (its transpose buffer is twice as
+// large).  Either way the transpose buffers take 32 KB.
+template <bool kWide>
+struct Epi {
+  static constexpr int kWarps = kWide ? 4 : 8;
+  static constexpr int kPerQuarter = kWarps / 4;
+  static constexpr int kChunks = NCHUNK / kPerQuarter;  // chunks of a slot per warp
+  static constexpr int kThreads = 64 + 32 * kWarps;
+  using T = typename std::conditional<kWide, int64_t, int32_t>::type;
+  static_assert(kWarps * 32 * 32 * sizeof(T) == 32768, "transpose buffers");
+};
 
 struct GemmArgs {
   int32_t tiles_m, tiles_n;
   int32_t n_steps;
+  int32_t sched_off;  // slot 1 trails slot 0 by this many steps (see the order below)
   int32_t step_kb0[kMaxJobs];
   int32_t step_nkb[kMaxJobs];
   int8_t step_first[kMaxJobs];   // the step opens a chunk: its first MMA overwrites the slot
@@ -76,14 +89,40 @@ struct GemmArgs {
 struct Smem {
   static constexpr size_t kA = 0;
   static constexpr size_t kB = kA + (size_t)STAGES * A_STAGE;
-  // per epilogue warp: a 32 x 32 transpose buffer of up to 8-byte values, XOR-swizzled
-  static constexpr size_t kScratch = kB + (size_t)STAGES * B_STAGE;
-  static constexpr size_t kRows = kScratch + EPI_WARPS * 32 * 32 * 8;  // per epilogue warp: WarpRows
+  static constexpr size_t kScratch = kB + (size_t)STAGES * B_STAGE;  // epilogue transpose buffers
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr size_t kBars = kRows + EPI_WARPS * 256;
+  static constexpr size_t kBars = kScratch + 32768;
   static constexpr size_t kMisc = kBars + (2 * STAGES + 5) * 8;  // tmem base, abort flag
   static constexpr size_t kEnd = kMisc + 16;
   static constexpr size_t kBytes = kEnd + 1024;  // slack for 1024-byte alignment of the base
+};
+
+// The order in which a CTA runs the steps of its tiles.  Its tiles p = 0, 1, 2, ... alternate between
+// the two TMEM slots (slot p % 2); each slot runs its tiles' steps in sequence, and between two steps of
+// a slot the epilogue works on it (a Horner rescale or a drain) while the tensor cores run the other
+// slot's step.  Slot 1 trails slot 0 by `off` steps, so that a drain (the long epilogue event) overlaps
+// a long step of the other slot instead of a short one: slot 0's step j0 runs before slot 1's step j1
+// while j0 <= j1 + off.  Producer, MMA issuer and epilogue walk the same order.
+struct Order {
+  int len0, len1, off, n_steps;
+  int j0, j1;
+  __device__ Order(int my_tiles, int n_steps_, int off_)
+      : len0(((my_tiles + 1) / 2) * n_steps_), len1((my_tiles / 2) * n_steps_), off(off_), n_steps(n_steps_),
+        j0(0), j1(0) {}
+  __device__ int total() const { return len0 + len1; }
+  // next (slot, local tile p, step k)
+  __device__ void next(int& slot, int& p, int& k) {
+    int j;
+    if (j1 >= len1 || (j0 < len0 && j0 <= j1 + off)) {
+      slot = 0;
+      j = j0++;
+    } else {
+      slot = 1;
+      j = j1++;
+    }
+    p = 2 * (j / n_steps) + slot;
+    k = j % n_steps;
+  }
 };
 
 // x * 2^k in the two's-complement type T, through the unsigned type (the plan's bounds guarantee the
@@ -94,25 +133,6 @@ __device__ __forceinline__ T shl(T x, int k) {
   return (T)((U)x << k);
 }
 
-// Column fold of one 32-column chunk holding 32/L columns of level L: w[s] = sum_l R^l v[s L + l].
-template <int L, typename T>
-__device__ __forceinline__ void fold_cols(const uint32_t (&v)[32], T (&w)[32], int bm1) {
-#pragma unroll
-  for (int s = 0; s < 32 / L; ++s) {
-    T a = 0;
-#pragma unroll
-    for (int l = 0; l < L; ++l) a += shl<T>((T)(int32_t)v[s * L + l], l * bm1);
-    w[s] = a;
-  }
-}
-
-__device__ __forceinline__ int32_t shfl_t(int32_t x, int src) { return __shfl_sync(0xffffffffu, x, src); }
-__device__ __forceinline__ int64_t shfl_t(int64_t x, int src) {
-  const int lo = __shfl_sync(0xffffffffu, (int)(uint32_t)(uint64_t)x, src);
-  const int hi = __shfl_sync(0xffffffffu, (int)(uint32_t)((uint64_t)x >> 32), src);
-  return (int64_t)(((uint64_t)(uint32_t)hi << 32) | (uint32_t)lo);
-}
-
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity))
@@ -120,15 +140,53 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64
   return true;
 }
 
-// Per-warp drain metadata of one tile, fetched before the accumulator is ready: row offsets and row
-// scales in shared memory, column indices and column scales in registers.  In the store phase of a
+// Transpose buffer index: row r, column c, XOR-swizzled so that both a row sweep and a column sweep of
+// the warp hit 32 different banks.
+__device__ __forceinline__ int sw(int r, int c) { return r * 32 + (c ^ r); }
+
+// Column fold of one 32-column chunk holding 32/L columns of level L, shifted, into the transpose
+// buffer: row `lane`, column s = sum_l R^l v[s L + l] * 2^shift.
+template <int L, typename T>
+__device__ __forceinline__ void fold_store(const uint32_t (&v)[32], T* scr, int lane, int bm1, int shift) {
+#pragma unroll
+  for (int s = 0; s < 32 / L; ++s) {
+    T a = 0;
+#pragma unroll
+    for (int l = 0; l < L; ++l) a += shl<T>((T)(int32_t)v[s * L + l], l * bm1);
+    scr[sw(lane, s)] = shl<T>(a, shift);
+  }
+}
+
+// The same for levels 9..31 (three columns at most), through the buffer to avoid dynamic register
+// indexing.  Each lane reads back only its own row.
+template <typename T>
+__device__ __forceinline__ void fold_store_deep(const uint32_t (&v)[32], T* scr, int lane, int LB, int nB, int bm1,
+                                                int shift) {
+#pragma unroll
+  for (int k = 0; k < 32; ++k) scr[sw(lane, k)] = (T)(int32_t)v[k];
+  T w0 = 0, w1 = 0, w2 = 0;
+  for (int l = 0; l < LB; ++l) {
+    w0 += shl<T>(scr[sw(lane, l)], l * bm1);
+    if (nB > 1) w1 += shl<T>(scr[sw(lane, LB + l)], l * bm1);
+    if (nB > 2) w2 += shl<T>(scr[sw(lane, 2 * LB + l)], l * bm1);
+  }
+  scr[sw(lane, 0)] = shl<T>(w0, shift);
+  scr[sw(lane, 1)] = shl<T>(w1, shift);
+  scr[sw(lane, 2)] = shl<T>(w2, shift);
+}
+
+// Per-warp drain metadata of one tile, fetched before the accumulator is ready.  Lane t holds output
+// row t of the warp's row group (its index in C and its dequantisation scale).  In the store phase of a
 // chunk with nB output columns, lane t writes column s = t % nB of the rows r0 = t / nB, r0 + per, ...
-// (per = 32 / nB rows at a time), so that all lanes store even when nB < 32.
+// (per = 32 / nB rows at a time), so that all lanes store even when nB < 32.  NC = chunks of this warp.
+template <int NC>
 struct DrainMeta {
   int LA, nA;
-  int32_t pk[BN / 32];   // per chunk: nB | LB << 6 | s << 12 | r0 << 18 | per << 24 (r0 = 63: idle lane)
-  int32_t col[BN / 32];  // the output column of this lane's s in each chunk
-  float sb[BN / 32];     // its dequantisation scale
+  int32_t my_row;
+  float my_sa;
+  int32_t pk[NC];   // per chunk: nB | LB << 6 | s << 12 | r0 << 18 | per << 24 (r0 = 63: idle lane)
+  int32_t col[NC];  // the output column of this lane's s in each chunk
+  float sb[NC];     // its dequantisation scale
 };
 
 __device__ __forceinline__ int pk_nB(int32_t pk) { return pk & 63; }
@@ -137,17 +195,10 @@ __device__ __forceinline__ int pk_s(int32_t pk) { return (pk >> 12) & 63; }
 __device__ __forceinline__ int pk_r0(int32_t pk) { return (pk >> 18) & 63; }
 __device__ __forceinline__ int pk_per(int32_t pk) { return (pk >> 24) & 63; }
 
-struct WarpRows {       // shared memory, per epilogue warp
-  int32_t row[32];      // the output row lane t holds after the row fold
-  float sa[32];         // its dequantisation scale
-};
-
-// Transpose buffer index: row r, column c, XOR-swizzled so that both a row sweep and a column sweep of
-// the warp hit 32 different banks.
-__device__ __forceinline__ int sw(int r, int c) { return r * 32 + (c ^ r); }
-
-__device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt, int q, int lane, bool last,
-                                              DrainMeta& m, WarpRows* wr) {
+// Chunks of warp h (of PQ warps on the quarter): h, h + PQ, h + 2 PQ, ...
+template <int NC, int PQ>
+__device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt, int q, int h, int lane, bool last,
+                                              DrainMeta<NC>& m) {
   int64_t my_row;
   if (g.a_outer) {
     const int64_t grp = (int64_t)mt * (BM / 32) + q;
@@ -161,11 +212,11 @@ __device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt,
     m.nA = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
     my_row = lane < m.nA ? r0 + lane : 0;
   }
-  wr->row[lane] = (int32_t)my_row;
-  wr->sa[lane] = (last && g.Cf && lane < m.nA) ? g.dA[g.dA_per_row ? my_row : 0] : 0.0f;
+  m.my_row = (int32_t)my_row;
+  m.my_sa = (last && g.Cf && lane < m.nA) ? g.dA[g.dA_per_row ? my_row : 0] : 0.0f;
 #pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    const int64_t gc = (int64_t)nt * (BN / 32) + c;
+  for (int i = 0; i < NC; ++i) {
+    const int64_t gc = (int64_t)nt * NCHUNK + h + PQ * i;
     int LB = 1, nB = 0;
     if (g.b_outer) {
       LB = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
@@ -181,117 +232,97 @@ __device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt,
       r0 = lane / nB;
       if (r0 >= per) r0 = 63;
     }
-    m.pk[c] = nB | (LB << 6) | (s << 12) | (r0 << 18) | (per << 24);
-    m.col[c] = 0;
-    if (r0 != 63) m.col[c] = g.b_outer ? g.srcB[gc * 32 + (int64_t)s * LB] : (int32_t)(gc * 32 + s);
+    m.pk[i] = nB | (LB << 6) | (s << 12) | (r0 << 18) | (per << 24);
+    m.col[i] = 0;
+    if (r0 != 63) m.col[i] = g.b_outer ? g.srcB[gc * 32 + (int64_t)s * LB] : (int32_t)(gc * 32 + s);
   }
 #pragma unroll
-  for (int c = 0; c < BN / 32; ++c)
-    m.sb[c] = (last && g.Cf && pk_r0(m.pk[c]) != 63) ? g.dB[g.dB_per_col ? m.col[c] : 0] : 0.0f;
-  __syncwarp();
+  for (int i = 0; i < NC; ++i)
+    m.sb[i] = (last && g.Cf && pk_r0(m.pk[i]) != 63) ? g.dB[g.dB_per_col ? m.col[i] : 0] : 0.0f;
 }
 
-// Drains one TMEM slot (this warp's 32 lanes) into C: fold, shift, write or add.
-template <typename T>
-__device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, uint32_t acce_bar, int lane, bool first,
-                                           bool last, int shift, T* scr, const DrainMeta& m, const WarpRows* wr) {
+// Drains this warp's chunks of one TMEM slot (its 32 lanes) into C: fold, shift, write or add.
+template <typename T, int NC, int PQ>
+__device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, uint32_t acce_bar, int lane, int h,
+                                           bool first, bool last, int shift, T* scr, const DrainMeta<NC>& m) {
   uint32_t v[32];
-  tmem_ld32(tbase, v);
+  tmem_ld32(tbase + h * 32, v);
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int i = 0; i < NC; ++i) {
     tmem_wait_ld();
-    uint32_t cur[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) cur[k] = v[k];
-    if (c + 1 < BN / 32) {
-      tmem_ld32(tbase + (c + 1) * 32, v);  // the next chunk streams in while this one is folded
-    } else {
-      // the slot is fully read: the MMA warp may reuse it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar);
-    }
     // dynamic indexing of the unrolled metadata arrays is avoided by a uniform select
     int32_t pk = 0, mycol = 0;
     float sb = 0.0f;
 #pragma unroll
-    for (int k = 0; k < BN / 32; ++k)
-      if (k == c) {
+    for (int k = 0; k < NC; ++k)
+      if (k == i) {
         pk = m.pk[k];
         mycol = m.col[k];
         sb = m.sb[k];
       }
     const int LB = pk_LB(pk), nB = pk_nB(pk);
     const int nA = m.nA, LA = m.LA;
-    if (nB == 0 || nA == 0) continue;
-    // 1. fold the column levels of B inside the registers (lane = unpacked row)
-    T w[32];
-    switch (LB) {
-      case 1: fold_cols<1>(cur, w, g.bm1); break;
-      case 2: fold_cols<2>(cur, w, g.bm1); break;
-      case 3: fold_cols<3>(cur, w, g.bm1); break;
-      case 4: fold_cols<4>(cur, w, g.bm1); break;
-      case 5: fold_cols<5>(cur, w, g.bm1); break;
-      case 6: fold_cols<6>(cur, w, g.bm1); break;
-      case 7: fold_cols<7>(cur, w, g.bm1); break;
-      case 8: fold_cols<8>(cur, w, g.bm1); break;
-      default: {
-        // levels 9..31 (three columns at most): fold through the transpose buffer
-#pragma unroll
-        for (int k = 0; k < 32; ++k) scr[sw(lane, k)] = (T)(int32_t)cur[k];
-        __syncwarp();
-#pragma unroll
-        for (int s2 = 0; s2 < 3; ++s2) {
-          T a = 0;
-          if (s2 < nB)
-            for (int l = 0; l < LB; ++l) a += shl<T>(scr[sw(lane, s2 * LB + l)], l * g.bm1);
-          w[s2] = a;
-        }
-        __syncwarp();
+    const bool work = nB > 0 && nA > 0;
+    // 1. fold the column levels of B inside the registers (row = lane = unpacked row) into the buffer
+    if (work) {
+      switch (LB) {
+        case 1: fold_store<1, T>(v, scr, lane, g.bm1, shift); break;
+        case 2: fold_store<2, T>(v, scr, lane, g.bm1, shift); break;
+        case 3: fold_store<3, T>(v, scr, lane, g.bm1, shift); break;
+        case 4: fold_store<4, T>(v, scr, lane, g.bm1, shift); break;
+        case 5: fold_store<5, T>(v, scr, lane, g.bm1, shift); break;
+        case 6: fold_store<6, T>(v, scr, lane, g.bm1, shift); break;
+        case 7: fold_store<7, T>(v, scr, lane, g.bm1, shift); break;
+        case 8: fold_store<8, T>(v, scr, lane, g.bm1, shift); break;
+        default: fold_store_deep<T>(v, scr, lane, LB, nB, g.bm1, shift);
       }
     }
-    // 2. fold the row levels of A across the lanes: lane t gathers lanes t LA + l
-    if (g.a_outer && LA > 1) {
-#pragma unroll
-      for (int s2 = 0; s2 < 32; ++s2) {
-        if (s2 < nB) {
-          T a = 0;
-          for (int l = 0; l < LA; ++l) {
-            const int src = lane * LA + l;
-            a += shl<T>(shfl_t(w[s2], src < 32 ? src : 31), l * g.bm1);
-          }
-          w[s2] = a;
-        }
-      }
+    // 2. the registers are free: this warp's next chunk streams in while this one is stored; after the
+    //    last chunk the slot is released to the MMA warp
+    if (i + 1 < NC) {
+      tmem_ld32(tbase + (h + PQ * (i + 1)) * 32, v);
+    } else {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar);
     }
-    // 3. transpose through shared memory: scr[row][column]
-#pragma unroll
-    for (int s2 = 0; s2 < 32; ++s2)
-      if (s2 < nB) scr[sw(lane, s2)] = shl<T>(w[s2], shift);
     __syncwarp();
-    // 4. lane (r0, s) stores column s of rows r0, r0 + per, ...: each row of C takes nB neighbouring
-    //    lanes, and all 32 / nB rows of a pass go out in one instruction
-    {
-      const int s = pk_s(pk), per = pk_per(pk);
-#pragma unroll 4
-      for (int r = pk_r0(pk); r < nA; r += per) {
-        T val = scr[sw(r, s)];
-        const int64_t row = wr->row[r];
-        if (g.C) {
-          if (g.c64) {
-            int64_t* cp = static_cast<int64_t*>(g.C) + row * g.ldc + mycol;
-            if (!first) val += (T)*cp;
-            *cp = (int64_t)val;
+    // 3. lane (r0, s) stores column s of output rows r0, r0 + per, ...; the row levels of A (OUTER
+    //    unpacking) are folded here, from LA consecutive rows of the buffer.  The trip count is uniform
+    //    so that every lane takes part in the shuffles of the row metadata.
+    if (work) {
+      const int s = pk_s(pk), per = pk_per(pk), r0 = pk_r0(pk);
+      const int iters = (nA + per - 1) / per;
+#pragma unroll 2
+      for (int it = 0; it < iters; ++it) {
+        const int t = r0 + it * per;
+        const int src = t < 32 ? t : 0;
+        const int64_t row = __shfl_sync(0xffffffffu, m.my_row, src);
+        const float sa = __shfl_sync(0xffffffffu, m.my_sa, src);
+        if (t < nA) {
+          T val;
+          if (LA == 1) {
+            val = scr[sw(t, s)];
           } else {
-            int32_t* cp = static_cast<int32_t*>(g.C) + row * g.ldc + mycol;
-            if (!first) val += (T)*cp;
-            *cp = (int32_t)val;
+            val = 0;
+            for (int l = 0; l < LA; ++l) val += shl<T>(scr[sw(t * LA + l, s)], l * g.bm1);
           }
+          if (g.C) {
+            if (g.c64) {
+              int64_t* cp = static_cast<int64_t*>(g.C) + row * g.ldc + mycol;
+              if (!first) val += (T)*cp;
+              *cp = (int64_t)val;
+            } else {
+              int32_t* cp = static_cast<int32_t*>(g.C) + row * g.ldc + mycol;
+              if (!first) val += (T)*cp;
+              *cp = (int32_t)val;
+            }
+          }
+          if (last && g.Cf)
+            g.Cf[row * g.ldcf + mycol] =
+                __fmul_rn(sizeof(T) == 8 ? __ll2float_rn((long long)val) : __int2float_rn((int)val),
+                          __fmul_rn(sa, sb));
         }
-        if (last && g.Cf)
-          g.Cf[row * g.ldcf + mycol] =
-              __fmul_rn(sizeof(T) == 8 ? __ll2float_rn((long long)val) : __int2float_rn((int)val),
-                        __fmul_rn(wr->sa[r], sb));
       }
     }
     __syncwarp();
@@ -299,17 +330,17 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
 }
 
 template <bool kWide>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ GemmArgs g) {
   using L = Smem;
-  using T = typename std::conditional<kWide, int64_t, int32_t>::type;
+  using E = Epi<kWide>;
+  using T = typename E::T;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base + L::kA;
   uint8_t* sB = base + L::kB;
   T* scratch = reinterpret_cast<T*>(base + L::kScratch);
-  WarpRows* wrows = reinterpret_cast<WarpRows*>(base + L::kRows);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::kBars);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
@@ -327,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(accf0 + 8 * s, 1);
-      mbar_init(acce0 + 8 * s, EPI_WARPS);  // one arrival per epilogue warp
+      mbar_init(acce0 + 8 * s, E::kWarps);  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -347,7 +378,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = g.tiles_m * g.tiles_n;
-  // this CTA's tiles blockIdx.x + i * gridDim.x, taken in pairs (one per TMEM slot)
+  // this CTA's tiles blockIdx.x + p * gridDim.x, p = 0 .. my_tiles - 1
   const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
   if (warp == 0) {
@@ -357,25 +388,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued[STAGES];
       for (int s = 0; s < STAGES; ++s) issued[s] = 2;
-      for (int p = 0; p < my_tiles; p += 2) {
-        const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
-        for (int k = 0; k < g.n_steps; ++k) {
-          for (int x = 0; x < npair; ++x) {
-            const int tile = blockIdx.x + (p + x) * gridDim.x;
-            const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
-            for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
-              if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
-              const uint32_t fb = full0 + 8 * stage;
-              mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
-              const int32_t kx = (g.step_kb0[k] + kb) * BK;
-              tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, mt * BM, fb);
-              tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, nt * BN, fb);
-              issued[stage] = phase;
-              if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
-              }
-            }
+      Order ord(my_tiles, g.n_steps, g.sched_off);
+      for (int e = 0; e < ord.total(); ++e) {
+        int slot, p, k;
+        ord.next(slot, p, k);
+        const int tile = blockIdx.x + p * gridDim.x;
+        const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
+        for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
+          const int32_t kx = (g.step_kb0[k] + kb) * BK;
+          tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, mt * BM, fb);
+          tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, nt * BN, fb);
+          issued[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
       }
@@ -392,36 +421,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_waits[2] = {0, 0};
-      for (int p = 0; p < my_tiles; p += 2) {
-        const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
-        for (int k = 0; k < g.n_steps; ++k) {
-          for (int slot = 0; slot < npair; ++slot) {
-            // the epilogue has finished the previous event of this slot (a rescale or a drain)
-            if (!mbar_wait(acce0 + 8 * slot, (empty_waits[slot] & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns))
-              goto mma_done;
-            ++empty_waits[slot];
-            tc_fence_after();
-            const uint32_t d = tmem_base + (uint32_t)slot * BN;
-            const bool first = g.step_first[k] != 0;
-            for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
-              if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, g.status, g.timeout_ns)) goto mma_done;
-              tc_fence_after();
-              const uint64_t adesc = smem_desc_k_sw128(smem_addr(sA + (size_t)stage * A_STAGE));
-              const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sB + (size_t)stage * B_STAGE));
+      Order ord(my_tiles, g.n_steps, g.sched_off);
+      for (int e = 0; e < ord.total(); ++e) {
+        int slot, p, k;
+        ord.next(slot, p, k);
+        (void)p;
+        // the epilogue has finished the previous event of this slot (a rescale or a drain)
+        if (!mbar_wait(acce0 + 8 * slot, (empty_waits[slot] & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns))
+          goto mma_done;
+        ++empty_waits[slot];
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)slot * BN;
+        const bool first = g.step_first[k] != 0;
+        for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, g.status, g.timeout_ns)) goto mma_done;
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_k_sw128(smem_addr(sA + (size_t)stage * A_STAGE));
+          const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sB + (size_t)stage * B_STAGE));
 #pragma unroll
-              for (int kk = 0; kk < BK / 32; ++kk) {
-                // 32 bytes further along K inside the 128-byte swizzled row: +2 in the address field
-                mma_i8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (first && kb == 0 && kk == 0) ? 0u : 1u);
-              }
-              mma_commit(empty0 + 8 * stage);
-              if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
-              }
-            }
-            mma_commit(accf0 + 8 * slot);
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // 32 bytes further along K inside the 128-byte swizzled row: +2 in the address field
+            mma_i8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (first && kb == 0 && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
+        mma_commit(accf0 + 8 * slot);
       }
     mma_done:
       // every issued MMA must complete before TMEM is released
@@ -431,50 +459,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access = row group of the tile
+    constexpr int PQ = E::kPerQuarter, NC = E::kChunks;
+    const int ew = warp - 2;       // epilogue warp 0 .. kWarps-1
+    const int q = warp & 3;        // TMEM lane quarter this warp may access = row group of the tile
+    const int h = ew / 4;          // which of the quarter's warps: chunks h, h + PQ, ...
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    T* scr = scratch + q * 32 * 32;  // this warp's transpose buffer (XOR-swizzled rows of 32)
+    T* scr = scratch + ew * 32 * 32;  // this warp's transpose buffer (XOR-swizzled rows of 32)
     uint32_t full_waits[2] = {0, 0};
-    for (int p = 0; p < my_tiles; p += 2) {
-      const int npair = my_tiles - p < 2 ? my_tiles - p : 2;
-      for (int k = 0; k < g.n_steps; ++k) {
-        for (int slot = 0; slot < npair; ++slot) {
-          DrainMeta meta;
-          const bool drain = g.step_after[k] < 0;
-          if (drain) {
-            // metadata of the tile first: its loads overlap the wait for the accumulator
-            const int tile = blockIdx.x + (p + slot) * gridDim.x;
-            drain_prepare(g, tile % g.tiles_m, tile / g.tiles_m, q, lane, g.step_dlast[k] != 0, meta, wrows + q);
-          }
-          int ok = 1;
-          if (lane == 0) ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          ++full_waits[slot];
-          if (!ok) goto epi_done;
-          tc_fence_after();
-          const uint32_t tbase = tmem_base + lane_off + (uint32_t)slot * BN;
-          if (g.step_after[k] >= 0) {
-            // Horner step: slot *= R^(e_prev - e), in place.  The plan bounds the result by 2^31, so
-            // a shift of 31 or more only meets zeros.
-            const int sh = g.step_after[k];
+    Order ord(my_tiles, g.n_steps, g.sched_off);
+    for (int e = 0; e < ord.total(); ++e) {
+      int slot, p, k;
+      ord.next(slot, p, k);
+      DrainMeta<NC> meta;
+      const bool drain = g.step_after[k] < 0;
+      if (drain) {
+        // metadata of the tile first: its loads overlap the wait for the accumulator
+        const int tile = blockIdx.x + p * gridDim.x;
+        drain_prepare<NC, PQ>(g, tile % g.tiles_m, tile / g.tiles_m, q, h, lane, g.step_dlast[k] != 0, meta);
+      }
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++full_waits[slot];
+      if (!ok) goto epi_done;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_off + (uint32_t)slot * BN;
+      if (!drain) {
+        // Horner step: slot *= R^(e_prev - e), in place.  The plan bounds the result by 2^31, so
+        // a shift of 31 or more only meets zeros.
+        const int sh = g.step_after[k];
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-              uint32_t v[32];
-              tmem_ld32(tbase + c * 32, v);
-              tmem_wait_ld();
+        for (int i = 0; i < NC; ++i) {
+          uint32_t v[32];
+          const uint32_t ta = tbase + (h + PQ * i) * 32;
+          tmem_ld32(ta, v);
+          tmem_wait_ld();
 #pragma unroll
-              for (int jj = 0; jj < 32; ++jj) v[jj] = sh < 31 ? (v[jj] << sh) : 0u;
-              tmem_st32(tbase + c * 32, v);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acce0 + 8 * slot);
-          } else {
-            drain_slot<T>(g, tbase, acce0 + 8 * slot, lane, g.step_dfirst[k] != 0, g.step_dlast[k] != 0,
-                          g.step_dshift[k], scr, meta, wrows + q);
-          }
+          for (int jj = 0; jj < 32; ++jj) v[jj] = sh < 31 ? (v[jj] << sh) : 0u;
+          tmem_st32(ta, v);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acce0 + 8 * slot);
+      } else {
+        drain_slot<T, NC, PQ>(g, tbase, acce0 + 8 * slot, lane, h, g.step_dfirst[k] != 0, g.step_dlast[k] != 0,
+                              g.step_dshift[k], scr, meta);
       }
     }
   epi_done:;
@@ -512,6 +542,35 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t k, int64_t rows, uint32_t
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Makespan, in SM cycles, of the step order of a CTA with `tiles` tiles when slot 1 trails by `off` steps:
+// a step occupies the tensor cores for 512 cycles per 128-deep k-block (M=128, N=256, K=32 in 128
+// cycles), and the epilogue event after it (done in step order) takes `rescale` or `drain` cycles.  A
+// slot's next step waits for the slot's previous event.  Used only to pick `off`.
+double simulate_order(const GemmArgs& g, int tiles, int off, double rescale, double drain) {
+  const int n = g.n_steps;
+  const int len0 = ((tiles + 1) / 2) * n, len1 = (tiles / 2) * n;
+  double mma_free = 0.0, epi_free = 0.0, slot_ready[2] = {0.0, 0.0};
+  int j0 = 0, j1 = 0;
+  for (int e = 0; e < len0 + len1; ++e) {
+    int slot, j;
+    if (j1 >= len1 || (j0 < len0 && j0 <= j1 + off)) {
+      slot = 0;
+      j = j0++;
+    } else {
+      slot = 1;
+      j = j1++;
+    }
+    const int k = j % n;
+    const double start = mma_free > slot_ready[slot] ? mma_free : slot_ready[slot];
+    const double end = start + 512.0 * g.step_nkb[k];
+    mma_free = end;
+    const double ev_start = epi_free > end ? epi_free : end;
+    epi_free = ev_start + (g.step_after[k] >= 0 ? rescale : drain);
+    slot_ready[slot] = epi_free;
+  }
+  return mma_free > epi_free ? mma_free : epi_free;
 }
 
 }  // namespace
@@ -592,12 +651,29 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   const int grid = num_tiles < ds->num_sms ? num_tiles : ds->num_sms;
   const size_t smem = Smem::kBytes;
   // int64 accumulation in the epilogue whenever the output is int64 or the bound exceeds int32
-  if (g.c64 || I.acc_bits > 32) {
+  const bool wide = g.c64 || I.acc_bits > 32;
+  // the trailing offset of slot 1 with the shortest modelled makespan for the busiest CTA; the event
+  // costs are rough per-tile figures of the epilogue (a rescale is one TMEM read and write of the slot,
+  // a drain also folds and stores it, half as fast with int64 values and half the warps)
+  {
+    const int tiles = (num_tiles + grid - 1) / grid;
+    const double rescale = wide ? 3000.0 : 1500.0, drain = wide ? 28000.0 : 14000.0;
+    double best = simulate_order(g, tiles, 0, rescale, drain);
+    g.sched_off = 0;
+    for (int off = 1; off < g.n_steps && off <= 16; ++off) {
+      const double t = simulate_order(g, tiles, off, rescale, drain);
+      if (t < best) {
+        best = t;
+        g.sched_off = off;
+      }
+    }
+  }
+  if (wide) {
     IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_gemm<true><<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
+    k_gemm<true><<<grid, Epi<true>::kThreads, smem, st>>>(tmA, tmB, g);
   } else {
     IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_gemm<false><<<grid, NUM_THREADS, smem, st>>>(tmA, tmB, g);
+    k_gemm<false><<<grid, Epi<false>::kThreads, smem, st>>>(tmA, tmB, g);
   }
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
