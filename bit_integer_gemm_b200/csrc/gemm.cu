@@ -32,11 +32,8 @@
 namespace imq {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128;
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK;  // bytes
-constexpr int B_STAGE = BN * BK;
-constexpr int NCHUNK = BN / 32;   // 32-column chunks of an accumulator slot
+constexpr int BM = 128, BN = 256, BK = 128;  // per CTA: 128 accumulator rows x 256 columns
+constexpr int NCHUNK = BN / 32;              // 32-column chunks of an accumulator slot
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 // Epilogue shape per accumulation width: with int32 values two warps share each TMEM lane quarter (each
@@ -86,15 +83,25 @@ struct GemmArgs {
   uint64_t timeout_ns;
 };
 
-struct Smem {
+// Tile geometry.  One CTA: a 128 x 256 tile, A 128 rows and B 256 rows (of B'^T) per k-block, 4
+// stages.  CTA pair (cta_group::2): a 256 x 256 tile, each CTA loading its own 128 rows of A and its
+// 128 of the 256 rows of B, so that a k-block costs each SM 32 KB instead of 48 KB; 6 stages.
+template <bool kPair>
+struct Geo {
+  static constexpr int kTM = kPair ? 2 * BM : BM;  // rows of A' per tile
+  static constexpr int kBRows = kPair ? BN / 2 : BN;
+  static constexpr int kStages = kPair ? 6 : 4;
+  static constexpr int kAStage = BM * BK;  // bytes
+  static constexpr int kBStage = kBRows * BK;
   static constexpr size_t kA = 0;
-  static constexpr size_t kB = kA + (size_t)STAGES * A_STAGE;
-  static constexpr size_t kScratch = kB + (size_t)STAGES * B_STAGE;  // epilogue transpose buffers
+  static constexpr size_t kB = kA + (size_t)kStages * kAStage;
+  static constexpr size_t kScratch = kB + (size_t)kStages * kBStage;  // epilogue transpose buffers
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
   static constexpr size_t kBars = kScratch + 32768;
-  static constexpr size_t kMisc = kBars + (2 * STAGES + 5) * 8;  // tmem base, abort flag
+  static constexpr size_t kMisc = kBars + (2 * kStages + 5) * 8;  // tmem base, abort flag
   static constexpr size_t kEnd = kMisc + 16;
   static constexpr size_t kBytes = kEnd + 1024;  // slack for 1024-byte alignment of the base
+  static_assert(kBytes <= 232448, "shared memory budget");
 };
 
 // The order in which a CTA runs the steps of its tiles.  Its tiles p = 0, 1, 2, ... alternate between
@@ -195,19 +202,20 @@ __device__ __forceinline__ int pk_s(int32_t pk) { return (pk >> 12) & 63; }
 __device__ __forceinline__ int pk_r0(int32_t pk) { return (pk >> 18) & 63; }
 __device__ __forceinline__ int pk_per(int32_t pk) { return (pk >> 24) & 63; }
 
-// Chunks of warp h (of PQ warps on the quarter): h, h + PQ, h + 2 PQ, ...
+// Chunks of warp h (of PQ warps on the quarter): h, h + PQ, h + 2 PQ, ...  row0: the first row of A'
+// in this CTA's accumulator.
 template <int NC, int PQ>
-__device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt, int q, int h, int lane, bool last,
-                                              DrainMeta<NC>& m) {
+__device__ __forceinline__ void drain_prepare(const GemmArgs& g, int64_t row0, int nt, int q, int h, int lane,
+                                              bool last, DrainMeta<NC>& m) {
   int64_t my_row;
   if (g.a_outer) {
-    const int64_t grp = (int64_t)mt * (BM / 32) + q;
+    const int64_t grp = row0 / 32 + q;
     m.LA = grp < g.n_grp_a ? g.grpA_L[grp] : 1;
     m.nA = grp < g.n_grp_a ? g.grpA_n[grp] : 0;
     my_row = lane < m.nA ? g.srcA[grp * 32 + (int64_t)lane * m.LA] : 0;
   } else {
     m.LA = 1;
-    const int64_t r0 = (int64_t)mt * BM + q * 32;
+    const int64_t r0 = row0 + q * 32;
     const int64_t rem = g.M - r0;
     m.nA = rem <= 0 ? 0 : (rem < 32 ? (int)rem : 32);
     my_row = lane < m.nA ? r0 + lane : 0;
@@ -242,7 +250,17 @@ __device__ __forceinline__ void drain_prepare(const GemmArgs& g, int mt, int nt,
 }
 
 // Drains this warp's chunks of one TMEM slot (its 32 lanes) into C: fold, shift, write or add.
-template <typename T, int NC, int PQ>
+// Releases a slot to the MMA issuer: a local arrive, or for a CTA pair an arrive on the leading CTA's
+// barrier (acce_bar is then its shared::cluster address).
+template <bool kPair>
+__device__ __forceinline__ void release_slot(uint32_t acce_bar) {
+  if constexpr (kPair)
+    mbar_arrive_cluster(acce_bar);
+  else
+    mbar_arrive(acce_bar);
+}
+
+template <typename T, int NC, int PQ, bool kPair>
 __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, uint32_t acce_bar, int lane, int h,
                                            bool first, bool last, int shift, T* scr, const DrainMeta<NC>& m) {
   uint32_t v[32];
@@ -284,7 +302,7 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
     } else {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar);
+      if (lane == 0) release_slot<kPair>(acce_bar);
     }
     __syncwarp();
     // 3. lane (r0, s) stores column s of output rows r0, r0 + per, ...; the row levels of A (OUTER
@@ -329,13 +347,15 @@ __device__ __forceinline__ void drain_slot(const GemmArgs& g, uint32_t tbase, ui
   }
 }
 
-template <bool kWide>
+template <bool kWide, bool kPair>
 __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ GemmArgs g) {
-  using L = Smem;
+  using L = Geo<kPair>;
   using E = Epi<kWide>;
   using T = typename E::T;
+  constexpr int STAGES = L::kStages;
+  constexpr int A_STAGE = L::kAStage, B_STAGE = L::kBStage;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base + L::kA;
@@ -350,6 +370,8 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
   const uint32_t accf0 = smem_addr(bars + 2 * STAGES), acce0 = smem_addr(bars + 2 * STAGES + 2);
   const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 4);
   constexpr uint32_t kCols = 2 * BN;  // two accumulator slots
+  // CTA pair: rank 0 leads (issues the MMAs, owns the barriers both CTAs' loads and epilogues signal)
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -358,7 +380,7 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(accf0 + 8 * s, 1);
-      mbar_init(acce0 + 8 * s, E::kWarps);  // one arrival per epilogue warp
+      mbar_init(acce0 + 8 * s, E::kWarps * (kPair ? 2 : 1));  // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -370,16 +392,27 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_holder), kCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_addr(tmem_holder), kCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(tmem_holder), kCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // the peer's barriers must be initialised before any load or arrive reaches them
+  if constexpr (kPair)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = g.tiles_m * g.tiles_n;
-  // this CTA's tiles blockIdx.x + p * gridDim.x, p = 0 .. my_tiles - 1
-  const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  // the tiles of this CTA (or pair): unit + p * units, p = 0 .. my_tiles - 1
+  const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int my_tiles = (num_tiles - unit + units - 1) / units;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -392,15 +425,24 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
       for (int e = 0; e < ord.total(); ++e) {
         int slot, p, k;
         ord.next(slot, p, k);
-        const int tile = blockIdx.x + p * gridDim.x;
+        const int tile = unit + p * units;
         const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
+        const int32_t ya = mt * L::kTM + (int32_t)rank * BM, yb = nt * BN + (int32_t)rank * L::kBRows;
         for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
           const int32_t kx = (g.step_kb0[k] + kb) * BK;
-          tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, mt * BM, fb);
-          tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, nt * BN, fb);
+          if constexpr (kPair) {
+            // both CTAs' bytes complete the leader's barrier, which expects them all
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_STAGE + B_STAGE));
+            const uint32_t lfb = mapa_shared(fb, 0);
+            tma_load_2d_pair(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, ya, lfb);
+            tma_load_2d_pair(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, yb, lfb);
+          } else {
+            mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
+            tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, ya, fb);
+            tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, yb, fb);
+          }
           issued[stage] = phase;
           if (++stage == STAGES) {
             stage = 0;
@@ -409,15 +451,17 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
         }
       }
     producer_done:
-      // every issued copy must land before the CTA may exit
-      for (int s = 0; s < STAGES; ++s)
-        if (issued[s] != 2) drain_wait(full0 + 8 * s, issued[s], g.timeout_ns);
+      // every issued copy must land before the CTA may exit.  In a pair the leader's full barriers
+      // complete only with both CTAs' bytes, so the leader's wait covers the peer's copies as well.
+      if (!kPair || rank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s] != 2) drain_wait(full0 + 8 * s, issued[s], g.timeout_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_i8(BM, BN);
+    // ------------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_i8(L::kTM, BN);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_waits[2] = {0, 0};
@@ -426,7 +470,7 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
         int slot, p, k;
         ord.next(slot, p, k);
         (void)p;
-        // the epilogue has finished the previous event of this slot (a rescale or a drain)
+        // the epilogue (of both CTAs) has finished the previous event of this slot
         if (!mbar_wait(acce0 + 8 * slot, (empty_waits[slot] & 1u) ^ 1u, abort_flag, g.status, g.timeout_ns))
           goto mma_done;
         ++empty_waits[slot];
@@ -441,19 +485,33 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             // 32 bytes further along K inside the 128-byte swizzled row: +2 in the address field
-            mma_i8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (first && kb == 0 && kk == 0) ? 0u : 1u);
+            const uint32_t acc = (first && kb == 0 && kk == 0) ? 0u : 1u;
+            if constexpr (kPair)
+              mma_i8_pair(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
+            else
+              mma_i8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, acc);
           }
-          mma_commit(empty0 + 8 * stage);
+          // the stage is free again in both CTAs once these MMAs have read it
+          if constexpr (kPair)
+            mma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+          else
+            mma_commit(empty0 + 8 * stage);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        mma_commit(accf0 + 8 * slot);
+        if constexpr (kPair)
+          mma_commit_pair_mc(accf0 + 8 * slot, 0x3);
+        else
+          mma_commit(accf0 + 8 * slot);
       }
     mma_done:
-      // every issued MMA must complete before TMEM is released
-      mma_commit(drain_bar);
+      // every issued MMA must complete before tensor memory is released
+      if constexpr (kPair)
+        mma_commit_pair(drain_bar);
+      else
+        mma_commit(drain_bar);
       drain_wait(drain_bar, 0, g.timeout_ns);
     }
     __syncwarp();
@@ -465,6 +523,9 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
     const int h = ew / 4;          // which of the quarter's warps: chunks h, h + PQ, ...
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     T* scr = scratch + ew * 32 * 32;  // this warp's transpose buffer (XOR-swizzled rows of 32)
+    // where a released slot is signalled: this CTA's barrier, or the leader's for a pair
+    const uint32_t rel0 = kPair ? mapa_shared(acce0, 0) : acce0;
+    const uint32_t rel1 = kPair ? mapa_shared(acce0 + 8, 0) : acce0 + 8;
     uint32_t full_waits[2] = {0, 0};
     Order ord(my_tiles, g.n_steps, g.sched_off);
     for (int e = 0; e < ord.total(); ++e) {
@@ -474,8 +535,9 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
       const bool drain = g.step_after[k] < 0;
       if (drain) {
         // metadata of the tile first: its loads overlap the wait for the accumulator
-        const int tile = blockIdx.x + p * gridDim.x;
-        drain_prepare<NC, PQ>(g, tile % g.tiles_m, tile / g.tiles_m, q, h, lane, g.step_dlast[k] != 0, meta);
+        const int tile = unit + p * units;
+        const int64_t row0 = (int64_t)(tile % g.tiles_m) * L::kTM + (int64_t)rank * BM;
+        drain_prepare<NC, PQ>(g, row0, tile / g.tiles_m, q, h, lane, g.step_dlast[k] != 0, meta);
       }
       int ok = 1;
       if (lane == 0) ok = mbar_wait(accf0 + 8 * slot, full_waits[slot] & 1u, abort_flag, g.status, g.timeout_ns) ? 1 : 0;
@@ -484,6 +546,7 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
       if (!ok) goto epi_done;
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_off + (uint32_t)slot * BN;
+      const uint32_t rel = slot ? rel1 : rel0;
       if (!drain) {
         // Horner step: slot *= R^(e_prev - e), in place.  The plan bounds the result by 2^31, so
         // a shift of 31 or more only meets zeros.
@@ -501,18 +564,27 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acce0 + 8 * slot);
+        if (lane == 0) release_slot<kPair>(rel);
       } else {
-        drain_slot<T, NC, PQ>(g, tbase, acce0 + 8 * slot, lane, h, g.step_dfirst[k] != 0, g.step_dlast[k] != 0,
-                              g.step_dshift[k], scr, meta);
+        drain_slot<T, NC, PQ, kPair>(g, tbase, rel, lane, h, g.step_dfirst[k] != 0, g.step_dlast[k] != 0,
+                                     g.step_dshift[k], scr, meta);
       }
     }
   epi_done:;
   }
   tc_fence_before();
-  __syncthreads();
+  // neither CTA of a pair leaves (or releases tensor memory) while the other may still reach it
+  if constexpr (kPair)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kCols);
+  if (warp == 1) {
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, kCols);
+    else
+      tmem_dealloc(tmem_base, kCols);
+  }
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -573,6 +645,29 @@ double simulate_order(const GemmArgs& g, int tiles, int off, double rescale, dou
   return mma_free > epi_free ? mma_free : epi_free;
 }
 
+template <bool kWide, bool kPair>
+imq_status launch_k_gemm(int grid, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
+                         cudaStream_t st) {
+  auto kern = k_gemm<kWide, kPair>;
+  const size_t smem = Geo<kPair>::kBytes;
+  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)Epi<kWide>::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kPair ? 1 : 0;  // single CTAs launch without a cluster
+  IMQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, tmA, tmB, g));
+  return IMQ_OK;
+}
+
 }  // namespace
 
 imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu, const float* dA, imq_gran gA,
@@ -600,12 +695,17 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   imq_status s = device_state(&ds);
   if (s != IMQ_OK) return s;
 
+  // a CTA pair per 256 x 256 tile whenever A' has more than one 128-row block
+  const bool pair = I.M_unp > BM && ds->num_sms >= 2;
+  const int tm = pair ? Geo<true>::kTM : Geo<false>::kTM;
   CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, Au, I.K_unp, I.M_unp, BM) || !make_map(&tmB, Bu, I.K_unp, I.N_unp, BN)) return IMQ_ERR_CUDA;
+  if (!make_map(&tmA, Au, I.K_unp, I.M_unp, BM) ||
+      !make_map(&tmB, Bu, I.K_unp, I.N_unp, pair ? Geo<true>::kBRows : Geo<false>::kBRows))
+    return IMQ_ERR_CUDA;
 
   GemmArgs g;
   memset(&g, 0, sizeof(g));
-  g.tiles_m = (int32_t)((I.M_unp + BM - 1) / BM);
+  g.tiles_m = (int32_t)((I.M_unp + tm - 1) / tm);
   g.tiles_n = (int32_t)((I.N_unp + BN - 1) / BN);
   g.n_steps = pl->n_steps;
   int first_drain = -1, last_drain = -1;
@@ -648,15 +748,17 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   g.timeout_ns = kTimeoutNs;
 
   const int num_tiles = g.tiles_m * g.tiles_n;
-  const int grid = num_tiles < ds->num_sms ? num_tiles : ds->num_sms;
-  const size_t smem = Smem::kBytes;
+  // one CTA per SM (a pair per two SMs), never more CTAs (pairs) than tiles
+  const int max_units = pair ? ds->num_sms / 2 : ds->num_sms;
+  const int units = num_tiles < max_units ? num_tiles : max_units;
+  const int grid = pair ? 2 * units : units;
   // int64 accumulation in the epilogue whenever the output is int64 or the bound exceeds int32
   const bool wide = g.c64 || I.acc_bits > 32;
   // the trailing offset of slot 1 with the shortest modelled makespan for the busiest CTA; the event
   // costs are rough per-tile figures of the epilogue (a rescale is one TMEM read and write of the slot,
   // a drain also folds and stores it, half as fast with int64 values and half the warps)
   {
-    const int tiles = (num_tiles + grid - 1) / grid;
+    const int tiles = (num_tiles + units - 1) / units;
     const double rescale = wide ? 3000.0 : 1500.0, drain = wide ? 28000.0 : 14000.0;
     double best = simulate_order(g, tiles, 0, rescale, drain);
     g.sched_off = 0;
@@ -668,16 +770,8 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
       }
     }
   }
-  if (wide) {
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_gemm<true><<<grid, Epi<true>::kThreads, smem, st>>>(tmA, tmB, g);
-  } else {
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_gemm<false><<<grid, Epi<false>::kThreads, smem, st>>>(tmA, tmB, g);
-  }
-  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+  if (wide) return pair ? launch_k_gemm<true, true>(grid, tmA, tmB, g, st) : launch_k_gemm<true, false>(grid, tmA, tmB, g, st);
+  return pair ? launch_k_gemm<false, true>(grid, tmA, tmB, g, st) : launch_k_gemm<false, false>(grid, tmA, tmB, g, st);
 }
-
-static_assert(Smem::kBytes <= 232448, "shared memory budget");
 
 }  // namespace imq
