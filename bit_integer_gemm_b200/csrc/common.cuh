@@ -64,10 +64,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier that may live in another CTA of the cluster, releasing this thread's prior
-// memory operations at cluster scope.
+// Arrive on an mbarrier that may live in another CTA of the cluster.  The default (CTA-scope release)
+// semantics: the arrive is used after tcgen05.wait + tcgen05.fence::before_thread_sync to hand tensor
+// memory back to the MMA issuer, which orders the tcgen05 reads; a cluster-scope release would also
+// wait for every prior global store of the thread to become visible, which that hand-over never needs.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Every thread of every CTA of the cluster arrives, then waits for all the others.

@@ -551,15 +551,18 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
         // Horner step: slot *= R^(e_prev - e), in place.  The plan bounds the result by 2^31, so
         // a shift of 31 or more only meets zeros.
         const int sh = g.step_after[k];
-#pragma unroll 1
-        for (int i = 0; i < NC; ++i) {
-          uint32_t v[32];
-          const uint32_t ta = tbase + (h + PQ * i) * 32;
-          tmem_ld32(ta, v);
-          tmem_wait_ld();
+        // two register buffers: the next chunk's load is in flight while this one is shifted and stored
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tbase + h * 32, v0);
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) v[jj] = sh < 31 ? (v[jj] << sh) : 0u;
-          tmem_st32(ta, v);
+        for (int i = 0; i < NC; ++i) {
+          uint32_t(&cur)[32] = (i & 1) ? v1 : v0;
+          uint32_t(&nxt)[32] = (i & 1) ? v0 : v1;
+          tmem_wait_ld();
+          if (i + 1 < NC) tmem_ld32(tbase + (h + PQ * (i + 1)) * 32, nxt);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) cur[jj] = sh < 31 ? (cur[jj] << sh) : 0u;
+          tmem_st32(tbase + (h + PQ * i) * 32, cur);
         }
         tmem_wait_st();
         tc_fence_before();
