@@ -30,6 +30,14 @@ imq_status device_state(DeviceState** out) {
       void* p = nullptr;
       IMQ_CUDA_TRY(cudaGetSymbolAddress(&p, g_status));
       IMQ_CUDA_TRY(cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev));
+      cudaMemPoolProps props;
+      memset(&props, 0, sizeof(props));
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      IMQ_CUDA_TRY(cudaMemPoolCreate(&d.pool, &props));
+      uint64_t keep = UINT64_MAX;
+      IMQ_CUDA_TRY(cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep));
       d.status = static_cast<int32_t*>(p);
       d.init = true;
     }

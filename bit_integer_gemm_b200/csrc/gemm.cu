@@ -32,8 +32,10 @@
 namespace imq {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128;  // per CTA: 128 accumulator rows x 256 columns
-constexpr int NCHUNK = BN / 32;              // 32-column chunks of an accumulator slot
+// Per CTA: 128 accumulator rows x up to BN columns.  The tile width bn (a multiple of 32, at most BN)
+// is chosen per launch so that the tiles spread evenly over the SMs; each TMEM slot spans BN columns.
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int NCHUNK = BN / 32;  // 32-column chunks of a full-width slot
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 // Epilogue shape per accumulation width: with int32 values two warps share each TMEM lane quarter (each
@@ -51,6 +53,8 @@ struct Epi {
 
 struct GemmArgs {
   int32_t tiles_m, tiles_n;
+  int32_t bn;      // tile width (columns of C' per tile), a multiple of 32 in [32, BN]
+  int32_t nchunk;  // bn / 32
   int32_t n_steps;
   int32_t sched_off;  // slot 1 trails slot 0 by this many steps (see the order below)
   int32_t step_kb0[kMaxJobs];
@@ -89,7 +93,7 @@ struct GemmArgs {
 template <bool kPair>
 struct Geo {
   static constexpr int kTM = kPair ? 2 * BM : BM;  // rows of A' per tile
-  static constexpr int kBRows = kPair ? BN / 2 : BN;
+  static constexpr int kBRows = kPair ? BN / 2 : BN;  // B stage rows at the full tile width
   static constexpr int kStages = kPair ? 6 : 4;
   static constexpr int kAStage = BM * BK;  // bytes
   static constexpr int kBStage = kBRows * BK;
@@ -224,9 +228,12 @@ __device__ __forceinline__ void drain_prepare(const GemmArgs& g, int64_t row0, i
   m.my_sa = (last && g.Cf && lane < m.nA) ? g.dA[g.dA_per_row ? my_row : 0] : 0.0f;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
-    const int64_t gc = (int64_t)nt * NCHUNK + h + PQ * i;
+    const int c = h + PQ * i;
+    const int64_t gc = (int64_t)nt * g.nchunk + c;
     int LB = 1, nB = 0;
-    if (g.b_outer) {
+    if (c >= g.nchunk) {
+      // beyond this launch's tile width: nothing to store
+    } else if (g.b_outer) {
       LB = gc < g.n_grp_b ? g.grpB_L[gc] : 1;
       nB = gc < g.n_grp_b ? g.grpB_n[gc] : 0;
     } else {
@@ -417,6 +424,9 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // rows of B'^T this CTA loads per k-block (half the tile width for a pair) and their bytes
+      const int32_t b_rows = kPair ? g.bn / 2 : g.bn;
+      const uint32_t b_bytes = (uint32_t)b_rows * BK;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued[STAGES];
@@ -427,19 +437,19 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
         ord.next(slot, p, k);
         const int tile = unit + p * units;
         const int mt = tile % g.tiles_m, nt = tile / g.tiles_m;
-        const int32_t ya = mt * L::kTM + (int32_t)rank * BM, yb = nt * BN + (int32_t)rank * L::kBRows;
+        const int32_t ya = mt * L::kTM + (int32_t)rank * BM, yb = nt * g.bn + (int32_t)rank * b_rows;
         for (int kb = 0; kb < g.step_nkb[k]; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, g.status, g.timeout_ns)) goto producer_done;
           const uint32_t fb = full0 + 8 * stage;
           const int32_t kx = (g.step_kb0[k] + kb) * BK;
           if constexpr (kPair) {
             // both CTAs' bytes complete the leader's barrier, which expects them all
-            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_STAGE + B_STAGE));
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * (A_STAGE + b_bytes));
             const uint32_t lfb = mapa_shared(fb, 0);
             tma_load_2d_pair(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, ya, lfb);
             tma_load_2d_pair(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, yb, lfb);
           } else {
-            mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
+            mbar_arrive_expect_tx(fb, A_STAGE + b_bytes);
             tma_load_2d(smem_addr(sA + (size_t)stage * A_STAGE), &tmA, kx, ya, fb);
             tma_load_2d(smem_addr(sB + (size_t)stage * B_STAGE), &tmB, kx, yb, fb);
           }
@@ -461,7 +471,7 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_i8(L::kTM, BN);
+      const uint32_t idesc = idesc_i8(L::kTM, (uint32_t)g.bn);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t empty_waits[2] = {0, 0};
@@ -620,8 +630,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t k, int64_t rows, uint32_t
 }
 
 // Makespan, in SM cycles, of the step order of a CTA with `tiles` tiles when slot 1 trails by `off` steps:
-// a step occupies the tensor cores for 512 cycles per 128-deep k-block (M=128, N=256, K=32 in 128
-// cycles), and the epilogue event after it (done in step order) takes `rescale` or `drain` cycles.  A
+// a step occupies the tensor cores for 2 bn cycles per 128-deep k-block (M=128, N=256, K=32 in 128
+// cycles per SM), and the epilogue event after it (done in step order) takes `rescale` or `drain` cycles.  A
 // slot's next step waits for the slot's previous event.  Used only to pick `off`.
 double simulate_order(const GemmArgs& g, int tiles, int off, double rescale, double drain) {
   const int n = g.n_steps;
@@ -639,7 +649,7 @@ double simulate_order(const GemmArgs& g, int tiles, int off, double rescale, dou
     }
     const int k = j % n;
     const double start = mma_free > slot_ready[slot] ? mma_free : slot_ready[slot];
-    const double end = start + 512.0 * g.step_nkb[k];
+    const double end = start + 2.0 * g.bn * g.step_nkb[k];
     mma_free = end;
     const double ev_start = epi_free > end ? epi_free : end;
     epi_free = ev_start + (g.step_after[k] >= 0 ? rescale : drain);
@@ -702,14 +712,33 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   const bool pair = I.M_unp > BM && ds->num_sms >= 2;
   const int tm = pair ? Geo<true>::kTM : Geo<false>::kTM;
   CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, Au, I.K_unp, I.M_unp, BM) ||
-      !make_map(&tmB, Bu, I.K_unp, I.N_unp, pair ? Geo<true>::kBRows : Geo<false>::kBRows))
-    return IMQ_ERR_CUDA;
-
   GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.tiles_m = (int32_t)((I.M_unp + tm - 1) / tm);
-  g.tiles_n = (int32_t)((I.N_unp + BN - 1) / BN);
+  // tile width: the fewest columns per SM over the busiest unit, ceil(tiles / units) * bn (a tile's
+  // tensor-core time is proportional to bn), plus a per-tile cost worth 96 columns (operand re-reads,
+  // the epilogue's fixed work, the pipeline's start and end) so that narrower tiles are taken only
+  // where they add parallelism (fewer tiles than units) or save a whole wave
+  {
+    const int max_units = pair ? ds->num_sms / 2 : ds->num_sms;
+    double best = 0.0;
+    for (int bn = BN; bn >= 128; bn -= 32) {
+      const int64_t tn = (I.N_unp + bn - 1) / bn;
+      const int64_t tiles = tn * g.tiles_m;
+      const int64_t units = tiles < max_units ? tiles : max_units;
+      const int64_t waves = (tiles + units - 1) / units;
+      const double cost = (double)waves * (bn + 96);
+      if (bn == BN || cost < best) {
+        best = cost;
+        g.bn = bn;
+      }
+    }
+  }
+  g.nchunk = g.bn / 32;
+  g.tiles_n = (int32_t)((I.N_unp + g.bn - 1) / g.bn);
+  if (!make_map(&tmA, Au, I.K_unp, I.M_unp, BM) ||
+      !make_map(&tmB, Bu, I.K_unp, I.N_unp, (uint32_t)(pair ? g.bn / 2 : g.bn)))
+    return IMQ_ERR_CUDA;
   g.n_steps = pl->n_steps;
   int first_drain = -1, last_drain = -1;
   for (int k = 0; k < pl->n_steps; ++k) {

@@ -18,6 +18,9 @@ struct DeviceState {
   void* partials = nullptr;    // per-CTA partial line maxima of the quantiser (grown on demand)
   size_t partials_bytes = 0;
   int num_sms = 0;
+  // stream-ordered pool for plan memory; it keeps what plans free (no trim at synchronisation), so a
+  // new plan reuses memory instead of mapping fresh pages
+  cudaMemPool_t pool = nullptr;
   bool init = false;
 };
 imq_status device_state(DeviceState** out);

@@ -86,6 +86,7 @@ struct LevelArgs {
   int64_t n[4];
   int32_t bm1;
   Summary* sum;
+  const int32_t* status;  // the device status word, copied into the summary by block 0
 };
 
 __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
@@ -94,6 +95,8 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   __shared__ unsigned long long ssum[4], soor[4];
   __shared__ unsigned int slmax[4];
   const int tid = threadIdx.x;
+  // every kernel before this one in stream order has finished: its errors are in the status word
+  if (blockIdx.x == 0 && tid == 0) a.sum->status = *a.status;
   for (int i = tid; i < 4 * kLv; i += 256) (&hist[0][0])[i] = 0;
   for (int i = tid; i < kLv * kLv; i += 256) (&joint[0][0])[i] = 0;
   if (tid < 4) {
@@ -258,13 +261,25 @@ struct OuterClass {
   int64_t count;    // lines of this level
 };
 
-__global__ void __launch_bounds__(1024) k_outer_map(const OuterClass* __restrict__ cls, const int8_t* __restrict__ lv,
-                                                    int64_t n, int G, int32_t* __restrict__ pos,
-                                                    int32_t* __restrict__ src, int32_t* __restrict__ grpL,
-                                                    int32_t* __restrict__ grpN) {
+// The OUTER layout of one matrix: classes of lines of equal level, each a run of groups of G unpacked
+// lines.  One CTA per class.
+struct OuterJob {
+  const OuterClass* cls;
+  int ncls;
+  const int8_t* lv;
+  int64_t n;
+  int G;
+  int32_t* pos;
+  int32_t* src;
+  int32_t* grpL;
+  int32_t* grpN;
+};
+
+__device__ void outer_map_class(const OuterClass c, const int8_t* __restrict__ lv, int64_t n, int G,
+                                int32_t* __restrict__ pos, int32_t* __restrict__ src, int32_t* __restrict__ grpL,
+                                int32_t* __restrict__ grpN) {
   __shared__ int warp_tot[32];
   __shared__ int total;
-  const OuterClass c = cls[blockIdx.x];
   const int64_t ngrp = (c.count + c.per - 1) / c.per;
   for (int64_t g = threadIdx.x; g < ngrp; g += blockDim.x) {
     grpL[c.grp0 + g] = c.L;
@@ -287,11 +302,38 @@ __global__ void __launch_bounds__(1024) k_outer_map(const OuterClass* __restrict
   }
 }
 
+// Both matrices' classes in one launch: blocks [0, a.ncls) take A's, the rest B's.
+__global__ void __launch_bounds__(1024) k_outer_map(OuterJob a, OuterJob b) {
+  const bool is_a = (int)blockIdx.x < a.ncls;
+  const OuterJob& j = is_a ? a : b;
+  const int ci = is_a ? (int)blockIdx.x : (int)blockIdx.x - a.ncls;
+  outer_map_class(j.cls[ci], j.lv, j.n, j.G, j.pos, j.src, j.grpL, j.grpN);
+}
+
+// Stage-2 initial values in one launch: every unpacked inner position starts as padding (source -1,
+// inner levels 0) and every OUTER unpacked line as unused (source -1).
+__global__ void k_plan_init(int32_t* __restrict__ tK, int8_t* __restrict__ lAk, int8_t* __restrict__ lBk,
+                            int64_t K_unp, int32_t* __restrict__ srcA, int64_t M_unp, int32_t* __restrict__ srcB,
+                            int64_t N_unp) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < K_unp; i += stride) {
+    tK[i] = -1;
+    lAk[i] = 0;
+    lBk[i] = 0;
+  }
+  if (srcA)
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < M_unp; i += stride) srcA[i] = -1;
+  if (srcB)
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N_unp; i += stride) srcB[i] = -1;
+}
+
 // ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
 struct Pinned {
   Summary* sum = nullptr;
+  void* tables = nullptr;          // staging of the segment and class tables for their upload
+  cudaEvent_t tables_done = nullptr;  // recorded after the last upload from `tables`
   std::mutex mu;
 };
 Pinned g_pinned[64];
@@ -336,11 +378,15 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   IMQ_CUDA_TRY(cudaGetDevice(&dev));
   Pinned& pin = g_pinned[dev & 63];
   std::lock_guard<std::mutex> lock(pin.mu);
+  const size_t tables_bytes = sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv;
+  // staging: the segment table padded to 256 bytes, then the class table (the device layout)
+  const size_t staging_bytes = align_up(sizeof(InnerSeg) * kLv * kLv, 256) + sizeof(OuterClass) * 2 * kLv;
   if (!pin.sum) IMQ_CUDA_TRY(cudaMallocHost(&pin.sum, sizeof(Summary)));
+  if (!pin.tables) IMQ_CUDA_TRY(cudaMallocHost(&pin.tables, staging_bytes));
+  if (!pin.tables_done) IMQ_CUDA_TRY(cudaEventCreateWithFlags(&pin.tables_done, cudaEventDisableTiming));
 
   imq_plan_t* pl = new imq_plan_t;
   memset(pl, 0, sizeof(*pl));
-  const size_t tables_bytes = sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv;
   pl->host_tables = malloc(tables_bytes);
   if (!pl->host_tables) {
     delete pl;
@@ -377,7 +423,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   off = align_up(off + sizeof(OuterClass) * 2 * kLv, 256);
   const size_t stage1 = off;
   char* blk1 = nullptr;
-  if (cudaMallocAsync((void**)&blk1, stage1, st) != cudaSuccess) {
+  if (cudaMallocFromPoolAsync((void**)&blk1, stage1, ds->pool, st) != cudaSuccess) {
     free(pl->host_tables);
     delete pl;
     return IMQ_ERR_CUDA;
@@ -405,11 +451,13 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   };
 
   const bool have_max = a_rowmax && a_colmax && b_rowmax && b_colmax;
+  const int32_t* lmx[4] = {mx[0], mx[1], mx[2], mx[3]};  // the maxima the levels are computed from
   if (have_max) {
-    const int32_t* given[4] = {a_rowmax, a_colmax, b_rowmax, b_colmax};
-    for (int v = 0; v < 4; ++v)
-      if (nvec[v] && cudaMemcpyAsync(mx[v], given[v], (size_t)nvec[v] * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-        return fail(IMQ_ERR_CUDA);
+    // the caller's maxima are read in place (only the level kernel below reads them)
+    lmx[0] = a_rowmax;
+    lmx[1] = a_colmax;
+    lmx[2] = b_rowmax;
+    lmx[3] = b_colmax;
   } else {
     // A stored M x K (or K x M when transposed); B stored K x N (or N x K)
     imq_status e = transA ? launch_line_max(A, it, K, M, lda, mx[1], mx[0], st)
@@ -428,9 +476,10 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   if (cudaMemsetAsync(dsum, 0, sizeof(Summary), st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
   LevelArgs la;
   for (int v = 0; v < 4; ++v) {
-    la.mx[v] = mx[v];
+    la.mx[v] = lmx[v];
     la.n[v] = nvec[v];
   }
+  la.status = ds->status;
   la.lv[0] = pl->lv_a_row;
   la.lv[1] = pl->lv_a_col;
   la.lv[2] = pl->lv_b_row;
@@ -445,8 +494,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     k_levels<<<(unsigned)grid, 256, 0, st>>>(la);
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
-  if (cudaMemcpyAsync(&dsum->status, ds->status, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(pin.sum, dsum, sizeof(Summary), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+  if (cudaMemcpyAsync(pin.sum, dsum, sizeof(Summary), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return fail(IMQ_ERR_CUDA);
   const Summary S = *pin.sum;
@@ -658,7 +706,8 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     o_gNB = off2; off2 = align_up(off2 + (size_t)pl->n_grp_b * 4, 256);
   }
   char* b2 = nullptr;
-  if (cudaMallocAsync((void**)&b2, off2 > 0 ? off2 : 256, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  if (cudaMallocFromPoolAsync((void**)&b2, off2 > 0 ? off2 : 256, ds->pool, st) != cudaSuccess)
+    return fail(IMQ_ERR_CUDA);
   pl->dev_block2 = b2;
   pl->dev_bytes = stage1 + off2;
   InnerSeg* dsegs = reinterpret_cast<InnerSeg*>(blk1 + o_segs);
@@ -679,19 +728,24 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     pl->grpB_L = reinterpret_cast<int32_t*>(b2 + o_gLB);
     pl->grpB_n = reinterpret_cast<int32_t*>(b2 + o_gNB);
   }
-  if (I.K_unp) {
-    if (cudaMemsetAsync(pl->tK, 0xFF, (size_t)I.K_unp * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(pl->lAk, 0, (size_t)I.K_unp, st) != cudaSuccess ||
-        cudaMemsetAsync(pl->lBk, 0, (size_t)I.K_unp, st) != cudaSuccess)
-      return fail(IMQ_ERR_CUDA);
+  {
+    const int64_t most = I.K_unp > I.M_unp ? (I.K_unp > I.N_unp ? I.K_unp : I.N_unp) : (I.M_unp > I.N_unp ? I.M_unp : I.N_unp);
+    int64_t grid = (most + 255) / 256;
+    if (grid > ds->num_sms * 4) grid = ds->num_sms * 4;
+    if (grid < 1) grid = 1;
+    k_plan_init<<<(unsigned)grid, 256, 0, st>>>(pl->tK, pl->lAk, pl->lBk, I.K_unp, a_outer ? pl->srcA : nullptr,
+                                               I.M_unp, b_outer ? pl->srcB : nullptr, I.N_unp);
   }
-  if (a_outer && I.M_unp && cudaMemsetAsync(pl->srcA, 0xFF, (size_t)I.M_unp * 4, st) != cudaSuccess)
-    return fail(IMQ_ERR_CUDA);
-  if (b_outer && I.N_unp && cudaMemsetAsync(pl->srcB, 0xFF, (size_t)I.N_unp * 4, st) != cudaSuccess)
-    return fail(IMQ_ERR_CUDA);
   if (nseg > 0 || ncls > 0) {
-    if (cudaMemcpyAsync(dsegs, hsegs, sizeof(InnerSeg) * (nseg > 0 ? nseg : 1), cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dcls, hcls, sizeof(OuterClass) * (ncls > 0 ? ncls : 1), cudaMemcpyHostToDevice, st) != cudaSuccess)
+    // one upload from pinned staging (an asynchronous copy; pageable memory would be staged by the
+    // driver first); the staging is reused once the previous plan's upload has completed
+    if (cudaEventSynchronize(pin.tables_done) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+    char* stg = static_cast<char*>(pin.tables);
+    const size_t segb = sizeof(InnerSeg) * (nseg > 0 ? nseg : 1), clsb = sizeof(OuterClass) * (ncls > 0 ? ncls : 1);
+    memcpy(stg, hsegs, segb);
+    memcpy(stg + (o_cls - o_segs), hcls, clsb);
+    if (cudaMemcpyAsync(dsegs, stg, (o_cls - o_segs) + clsb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaEventRecord(pin.tables_done, st) != cudaSuccess)
       return fail(IMQ_ERR_CUDA);
   }
   if (nseg > 0) {
@@ -699,12 +753,13 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     const int64_t nblk = I.K_unp / 16;
     k_inner_blocks<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(pl->tK, pl->lAk, pl->lBk, nblk, pl->blk16);
   }
-  if (a_outer && cls_a1 > cls_a0)
-    k_outer_map<<<cls_a1 - cls_a0, 1024, 0, st>>>(dcls + cls_a0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
-                                                  pl->grpA_L, pl->grpA_n);
-  if (b_outer && cls_b1 > cls_b0)
-    k_outer_map<<<cls_b1 - cls_b0, 1024, 0, st>>>(dcls + cls_b0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
-                                                  pl->grpB_L, pl->grpB_n);
+  {
+    OuterJob ja = {dcls + cls_a0, a_outer ? cls_a1 - cls_a0 : 0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
+                   pl->grpA_L, pl->grpA_n};
+    OuterJob jb = {dcls + cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
+                   pl->grpB_L, pl->grpB_n};
+    if (ja.ncls + jb.ncls > 0) k_outer_map<<<ja.ncls + jb.ncls, 1024, 0, st>>>(ja, jb);
+  }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
   *out = pl;
   return IMQ_OK;

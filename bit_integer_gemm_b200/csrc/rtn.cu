@@ -227,6 +227,107 @@ __device__ void warp_key_stats(const T* a, int n, uint32_t* mk_out, uint32_t* ba
   *bad_out = mk >= Key<T>::kInf;
 }
 
+// Exact nearest-rank select for bf16 keys, without atomics: the k-th smallest 15-bit key is built
+// from the top bit down, bit b being set when fewer than k keys lie below (answer | 2^b).  Two keys are
+// counted per 32-bit word: with both sign bits forced to 1, (0x8000 + key) - t keeps bit 15 of its half
+// exactly when key >= t and never borrows from the other half.  Each half-word counter sees at most
+// n / 64 + 4 keys (n <= 100 000 here: a group fits the shared-memory stage), far below 2^16.
+__device__ uint32_t warp_select_key_bf16(const uint16_t* a, int n, unsigned long long k) {
+  const int lane = threadIdx.x & 31;
+  const int nv = n / 8;
+  uint32_t ans = 0;
+  for (int b = 14; b >= 0; --b) {
+    const uint32_t t = ans | (1u << b);
+    const uint32_t t2 = t | (t << 16);
+    uint32_t acc = 0;
+#pragma unroll 4
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 w = reinterpret_cast<const uint4*>(a)[i];
+      acc += (((w.x | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      acc += (((w.y | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      acc += (((w.z | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      acc += (((w.w | 0x80008000u) - t2) >> 15) & 0x00010001u;
+    }
+    uint32_t ge = (acc & 0xFFFFu) + (acc >> 16);
+    for (int i = nv * 8 + lane; i < n; i += 32) ge += (a[i] & 0x7FFFu) >= t ? 1u : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ge += __shfl_xor_sync(0xffffffffu, ge, o);
+    const unsigned long long below = (unsigned long long)n - ge;
+    if (below < k) ans = t;
+  }
+  return ans;
+}
+
+// The k-th smallest key of a group in shared memory: bisection for bf16, radix passes for f32.
+template <typename T>
+__device__ __forceinline__ uint32_t select_key(const T* a, int n, unsigned long long k, uint32_t* hist) {
+  if constexpr (sizeof(T) == 2)
+    return warp_select_key_bf16(a, n, k);
+  else
+    return warp_select_key(a, n, k, hist);
+}
+
+// x * s rounded to the nearest integer, ties to even: the arithmetic of quant_one, without the store.
+template <bool kOut16>
+__device__ __forceinline__ int32_t quant_val(float x, float s, int32_t* status) {
+  const float y = __fmul_rn(x, s);
+  int32_t v = 0;
+  if (fabsf(y) < 2147483648.0f) {
+    v = __float2int_rn(y);
+  } else {
+    set_status(status, IMQ_ERR_RANGE);
+  }
+  if (kOut16 && (v > 32767 || v < -32767)) {
+    set_status(status, IMQ_ERR_RANGE);
+    v = 0;
+  }
+  return v;
+}
+
+// Quantises 8 consecutive entries of a 16-byte aligned group in shared memory and stores them with
+// 16-byte stores at out[idx .. idx+7] (idx a multiple of 8, out 16-byte aligned); a[j] = |value j|.
+template <typename T, bool kOut16>
+__device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t idx, int32_t* status,
+                                       uint32_t (&a)[8]) {
+  // the 8 entries as 32-bit words (bf16: two per word, low half first), kept in registers
+  uint32_t wd[8];
+  {
+    const uint4 w0 = reinterpret_cast<const uint4*>(src)[0];
+    wd[0] = w0.x; wd[1] = w0.y; wd[2] = w0.z; wd[3] = w0.w;
+    if (sizeof(T) == 4) {
+      const uint4 w1 = reinterpret_cast<const uint4*>(src)[1];
+      wd[4] = w1.x; wd[5] = w1.y; wd[6] = w1.z; wd[7] = w1.w;
+    }
+  }
+  int32_t v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const T e = sizeof(T) == 2 ? (T)((wd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) : (T)wd[j];
+    v[j] = quant_val<kOut16>(Key<T>::value(e), s, status);
+    a[j] = v[j] < 0 ? (uint32_t)(-(int64_t)v[j]) : (uint32_t)v[j];
+  }
+  if (kOut16) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) pk[j] = ((uint32_t)v[2 * j] & 0xFFFFu) | ((uint32_t)v[2 * j + 1] << 16);
+    *reinterpret_cast<uint4*>(static_cast<int16_t*>(out) + idx) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  } else {
+    int32_t* o = static_cast<int32_t*>(out) + idx;
+    reinterpret_cast<int4*>(o)[0] = make_int4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<int4*>(o)[1] = make_int4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+// Raises m[0..7] (16-byte aligned shared memory) to a[j] where a[j] is larger: a plain read first, so
+// that the atomic is only paid where the maximum actually grows.
+__device__ __forceinline__ void max8_shared(uint32_t* m, const uint32_t (&a)[8]) {
+  const uint4 m0 = reinterpret_cast<const uint4*>(m)[0], m1 = reinterpret_cast<const uint4*>(m)[1];
+  const uint32_t mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (a[j] > mm[j]) atomicMax(&m[j], a[j]);
+}
+
 // ------------------------------------------------------------------------------------------------
 // per stored row (kSelect) or per tensor (scale from the tensor state): one warp per row.  Each warp
 // stages its row in its own shared-memory buffer, builds its own 256-bin histograms (warp-aggregated
@@ -253,6 +354,8 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
   __syncthreads();
   if (warp < nwarps) {
     const int n = (int)cols;
+    // vectorised quantisation: whole 8-entry groups, contiguous and 16-byte aligned output rows
+    const bool vq = !trans_out && n % 8 == 0 && ldq % 8 == 0 && (reinterpret_cast<uintptr_t>(Xint) & 15) == 0;
     for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < rows; r += (int64_t)gridDim.x * nwarps) {
       const T* xr = X + r * ld;
       if (vec) {
@@ -267,7 +370,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
       warp_key_stats(row, n, &mk, &bad);
       float s;
       if (kSelect) {
-        const float q = Key<T>::from_key(warp_select_key(row, n, krank, hist));
+        const float q = Key<T>::from_key(select_key(row, n, krank, hist));
         float dl;
         scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
         if (lane == 0) {
@@ -282,11 +385,22 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
         continue;
       }
       uint32_t rmx = 0;
-      for (int c = lane; c < n; c += 32) {
-        const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
-                                             status);
-        rmx = max(rmx, a);
-        if (part && a) atomicMax(&cmax[c], a);
+      if (vq) {
+        // 8 consecutive entries per lane and step: 16-byte shared loads and global stores
+        for (int g = lane; g < n / 8; g += 32) {
+          uint32_t a[8];
+          quant8<T, kOut16>(row + g * 8, s, Xint, r * ldq + g * 8, status, a);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) rmx = max(rmx, a[j]);
+          if (part) max8_shared(cmax + g * 8, a);
+        }
+      } else {
+        for (int c = lane; c < n; c += 32) {
+          const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint,
+                                               trans_out ? c * ldq + r : r * ldq + c, status);
+          rmx = max(rmx, a);
+          if (part && a > cmax[c]) atomicMax(&cmax[c], a);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) rmx = max(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
@@ -326,9 +440,10 @@ __global__ void __launch_bounds__(CW * 32) k_rtn_cols_staged(
   // stage: 16-byte loads along the rows, transposed stores into the columns
   constexpr int V = 16 / sizeof(T);
   constexpr int SEG = CW / V;  // 16-byte pieces per slab row (0 when a slab row is narrower)
+  constexpr int SEGD = SEG > 0 ? SEG : 1;  // divisor of the branch below, which SEG = 0 never takes
   if (SEG > 0 && vec && ncol == CW) {
     for (int i = tid; i < n * SEG; i += CW * 32) {
-      const int r = i / SEG, sg = i % SEG;
+      const int r = i / SEGD, sg = i % SEGD;
       const uint4 w = __ldcs(reinterpret_cast<const uint4*>(X + r * ld + c0) + sg);
       const T* e = reinterpret_cast<const T*>(&w);
 #pragma unroll
@@ -346,7 +461,7 @@ __global__ void __launch_bounds__(CW * 32) k_rtn_cols_staged(
     const int64_t c = c0 + warp;
     uint32_t mk, bad;
     warp_key_stats(col, n, &mk, &bad);
-    const float q = Key<T>::from_key(warp_select_key(col, n, krank, hist_all[warp]));
+    const float q = Key<T>::from_key(select_key(col, n, krank, hist_all[warp]));
     float s, dl;
     scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
     if (lane == 0) {
@@ -355,12 +470,22 @@ __global__ void __launch_bounds__(CW * 32) k_rtn_cols_staged(
       if (bad) set_status(status, IMQ_ERR_NONFINITE);
     }
     uint32_t cmx = 0;
-    if (!bad) {
+    // vectorised quantisation when the column is written as one contiguous, aligned output row
+    const bool vq = trans_out && n % 8 == 0 && ldq % 8 == 0 && (reinterpret_cast<uintptr_t>(Xint) & 15) == 0;
+    if (!bad && vq) {
+      for (int g = lane; g < n / 8; g += 32) {
+        uint32_t a[8];
+        quant8<T, kOut16>(col + g * 8, s, Xint, c * ldq + g * 8, status, a);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cmx = max(cmx, a[j]);
+        if (part) max8_shared(rmax + g * 8, a);
+      }
+    } else if (!bad) {
       for (int r = lane; r < n; r += 32) {
         const uint32_t a = quant_one<kOut16>(Key<T>::value(col[r]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
                                              status);
         cmx = max(cmx, a);
-        if (part && a) atomicMax(&rmax[r], a);
+        if (part && a > rmax[r]) atomicMax(&rmax[r], a);
       }
     }
 #pragma unroll

@@ -40,48 +40,71 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
   __shared__ int64_t s_base[8];
   const int tid = threadIdx.x;
   const int64_t nchunk = K_unp / 16;
-  const bool vec4 = (K % 4 == 0) && (ld % 4 == 0);
+  constexpr int kU = sizeof(T) == 2 ? 8 : 4;  // octets in flight per thread
+  // whole-octet 16-byte loads: every line start and octet 16-byte aligned
+  const bool vec8 = (K % 8 == 0) && (ld % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   for (int64_t i0 = (int64_t)blockIdx.x * NL; i0 < nlines; i0 += (int64_t)gridDim.x * NL) {
     const int nb = nlines - i0 < NL ? (int)(nlines - i0) : NL;
     if (tid < nb) {
       s_L[tid] = outer ? (int)lvl[i0 + tid] : 1;
       s_base[tid] = outer ? (int64_t)pos[i0 + tid] : i0 + tid;
     }
-    // digit planes: 4 entries per thread and iteration, one 4-byte store per plane
-    for (int b = 0; b < nb; ++b) {
-      const T* xr = X + (i0 + b) * ld;
-      int8_t* pb = planes + (int64_t)b * P * Kp;
-      for (int64_t t = (int64_t)tid * 4; t < Kp; t += 256 * 4) {
-        int32_t v[4];
-        if (vec4 && t + 3 < K) {
+    // digit planes: a thread takes octets (8 consecutive entries of one line) and has kU of them in
+    // flight before it computes any digit, so that the line loads overlap
+    const int64_t q_line = Kp / 8;  // octets per line (Kp is a multiple of 16)
+    const int64_t nq = (int64_t)nb * q_line;
+    for (int64_t f0 = 0; f0 < nq; f0 += 256 * kU) {
+      int32_t v[kU][8];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t f = f0 + (int64_t)u * 256 + tid;
+        const int32_t b = (int32_t)f / (int32_t)q_line;  // nb * q_line < 2^31 (nb <= 8, lines < 2^31 bytes)
+        const int64_t t = (f - (int64_t)b * q_line) * 8;
+        const T* xr = X + (i0 + b) * ld + t;
+        if (f < nq && vec8 && t + 8 <= K) {
           if (sizeof(T) == 2) {
-            const uint2 w = *reinterpret_cast<const uint2*>(xr + t);
-            v[0] = (int16_t)(w.x & 0xFFFFu); v[1] = (int16_t)(w.x >> 16);
-            v[2] = (int16_t)(w.y & 0xFFFFu); v[3] = (int16_t)(w.y >> 16);
+            const uint4 w = *reinterpret_cast<const uint4*>(xr);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              v[u][2 * r] = (int16_t)(ww[r] & 0xFFFFu);
+              v[u][2 * r + 1] = (int16_t)(ww[r] >> 16);
+            }
           } else {
-            const int4 w = *reinterpret_cast<const int4*>(xr + t);
-            v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+            const int4 w0 = *reinterpret_cast<const int4*>(xr), w1 = *reinterpret_cast<const int4*>(xr + 4);
+            v[u][0] = w0.x; v[u][1] = w0.y; v[u][2] = w0.z; v[u][3] = w0.w;
+            v[u][4] = w1.x; v[u][5] = w1.y; v[u][6] = w1.z; v[u][7] = w1.w;
           }
         } else {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) v[r] = t + r < K ? (int32_t)xr[t + r] : 0;
+          for (int r = 0; r < 8; ++r) v[u][r] = (f < nq && t + r < K) ? (int32_t)xr[r] : 0;
         }
-        uint32_t a[4], sg[4];
+      }
+      const uint32_t mask = (1u << bm1) - 1u;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          sg[r] = v[r] < 0 ? 0xFFFFFFFFu : 0u;
-          a[r] = v[r] < 0 ? (uint32_t)(-(int64_t)v[r]) : (uint32_t)v[r];
+      for (int u = 0; u < kU; ++u) {
+        const int64_t f = f0 + (int64_t)u * 256 + tid;
+        if (f >= nq) continue;
+        const int32_t b = (int32_t)f / (int32_t)q_line;
+        const int64_t t = (f - (int64_t)b * q_line) * 8;
+        int8_t* pb = planes + (int64_t)b * P * Kp + t;
+        uint32_t a[8], sg[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          sg[r] = v[u][r] < 0 ? 0xFFFFFFFFu : 0u;
+          a[r] = v[u][r] < 0 ? (uint32_t)(-(int64_t)v[u][r]) : (uint32_t)v[u][r];
         }
-        const uint32_t mask = (1u << bm1) - 1u;
         for (int l = 0; l < P; ++l) {
           const int sh = l * bm1;
-          uint32_t packed = 0;
+          uint32_t lo = 0, hi = 0;
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const uint32_t d = sh < 31 ? ((a[r] >> sh) & mask) : 0u;
-            packed |= (((d ^ sg[r]) - sg[r]) & 0xFFu) << (8 * r);
+            const uint32_t d0 = sh < 31 ? ((a[r] >> sh) & mask) : 0u;
+            const uint32_t d1 = sh < 31 ? ((a[r + 4] >> sh) & mask) : 0u;
+            lo |= (((d0 ^ sg[r]) - sg[r]) & 0xFFu) << (8 * r);
+            hi |= (((d1 ^ sg[r + 4]) - sg[r + 4]) & 0xFFu) << (8 * r);
           }
-          *reinterpret_cast<uint32_t*>(pb + (int64_t)l * Kp + t) = packed;
+          *reinterpret_cast<uint2*>(pb + (int64_t)l * Kp) = make_uint2(lo, hi);
         }
       }
     }
