@@ -153,6 +153,192 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
   }
 }
 
+// Digit planes of one int16 line, SIMD within a register: a word holds two entries; their magnitudes
+// come from a branch-free absolute value per 16-bit half, a plane's digits from one mask and shift per
+// word (masking first keeps the upper half's bits out of the lower half), four digits are gathered into the bytes of one word with a byte permute, and the negative
+// entries' digits are negated byte-wise as (0x80808080 - d) ^ 0x80808080 (a digit is at most 127, so
+// no byte borrows).  Digits of level l with l * bm1 >= 16 are zero for int16 magnitudes.  The line is
+// 16-byte aligned and K a multiple of 8; entries K .. Kp-1 of the planes are written as zeros.
+__device__ __forceinline__ void digit_planes_i16(const int16_t* __restrict__ xr, int64_t K, int64_t Kp, int P,
+                                                 int bm1, int8_t* __restrict__ planes, int lane) {
+  const uint32_t mask = (1u << bm1) - 1u;
+  const int64_t nq = Kp / 8;
+  constexpr int kU = 8;
+  for (int64_t q0 = 0; q0 < nq; q0 += 32 * kU) {
+    uint4 w[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t t = (q0 + u * 32 + lane) * 8;
+      w[u] = t + 8 <= K ? *reinterpret_cast<const uint4*>(xr + t) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t t = (q0 + u * 32 + lane) * 8;
+      if (t >= Kp) continue;
+      const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+      uint32_t A[4], S[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t sgn = (ww[r] >> 15) & 0x00010001u;  // 1 in each negative half
+        S[r] = sgn * 0xFFFFu;                              // 0xFFFF in each negative half
+        A[r] = (ww[r] ^ S[r]) + sgn;                       // |entry| per half (no carry between halves)
+      }
+      const uint32_t Mlo = __byte_perm(S[0], S[1], 0x6420), Mhi = __byte_perm(S[2], S[3], 0x6420);
+      for (int l = 0; l < P; ++l) {
+        const int sh = l * bm1;
+        uint32_t lo = 0, hi = 0;
+        if (sh < 16) {
+          // the digit's bits of both halves (clipped to 16 bits), then shifted down within each half
+          const uint32_t m2 = ((mask << sh) & 0xFFFFu) * 0x00010001u;
+          const uint32_t d0 = (A[0] & m2) >> sh, d1 = (A[1] & m2) >> sh;
+          const uint32_t d2 = (A[2] & m2) >> sh, d3 = (A[3] & m2) >> sh;
+          const uint32_t plo = __byte_perm(d0, d1, 0x6420), phi = __byte_perm(d2, d3, 0x6420);
+          const uint32_t nlo = (0x80808080u - plo) ^ 0x80808080u, nhi = (0x80808080u - phi) ^ 0x80808080u;
+          lo = (plo & ~Mlo) | (nlo & Mlo);
+          hi = (phi & ~Mhi) | (nhi & Mhi);
+        }
+        *reinterpret_cast<uint2*>(planes + (int64_t)l * Kp + t) = make_uint2(lo, hi);
+      }
+    }
+  }
+}
+
+// Row gather, one warp per source line: the warp loads its line (every load of a lane in flight before
+// any digit is computed), writes the line's P digit planes to its own shared memory,
+// plane[l][t] = d_l(entry t), and streams out the line's unpacked lines: a 16-byte block the plan marked
+// contiguous (t0..t0+15, one level) is one 16-byte copy from a plane, any other block is gathered byte by
+// byte.  Warps work independently (no CTA barrier), so one warp's loads overlap another's stores.
+// The per-chunk plan metadata (block start and first inner level), the same for every line, is copied
+// to shared memory once per CTA when it fits (meta_smem), so that the output loop reads it at shared-
+// memory latency.
+constexpr int64_t kMetaMaxChunks = 4096;
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_unpack_lines(const T* __restrict__ X, int64_t nlines, int64_t K,
+                                                      int64_t ld, int P, int nwarps, int outer,
+                                                      const int8_t* __restrict__ lvl, const int32_t* __restrict__ pos,
+                                                      const int32_t* __restrict__ tK, const int8_t* __restrict__ lk,
+                                                      const int32_t* __restrict__ blk16, int64_t K_unp, int bm1,
+                                                      int meta_smem, int8_t* __restrict__ out) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t Kp = (K + 15) / 16 * 16;  // plane row length, 16-byte aligned
+  const int64_t nchunk = K_unp / 16;
+  // [planes of nwarps lines][block starts, int32 x nchunk][first inner levels, int8 x nchunk]
+  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)nwarps * P * Kp);
+  int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);
+  if (meta_smem) {
+    for (int64_t c = threadIdx.x; c < nchunk; c += blockDim.x) {
+      s_blk[c] = blk16[c];
+      s_lk0[c] = lk[c * 16];
+    }
+    __syncthreads();
+  }
+  if (warp >= nwarps) return;
+  int8_t* planes = reinterpret_cast<int8_t*>(dsm) + (int64_t)warp * P * Kp;  // [P][Kp]
+  constexpr int kU = sizeof(T) == 2 ? 8 : 4;  // octets in flight per lane
+  const bool vec8 = (K % 8 == 0) && (ld % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  const int64_t nq = Kp / 8;  // octets per line
+  const uint32_t mask = (1u << bm1) - 1u;
+  for (int64_t line = (int64_t)blockIdx.x * nwarps + warp; line < nlines; line += (int64_t)gridDim.x * nwarps) {
+    const T* xr = X + line * ld;
+    const int L = outer ? (int)lvl[line] : 1;
+    const int64_t base = outer ? (int64_t)pos[line] : line;
+    // 1. digit planes of the line
+    bool planes_done = false;
+    if constexpr (sizeof(T) == 2) {
+      if (vec8) {
+        digit_planes_i16(reinterpret_cast<const int16_t*>(xr), K, Kp, P, bm1, planes, lane);
+        planes_done = true;
+      }
+    }
+    for (int64_t q0 = 0; q0 < (planes_done ? 0 : nq); q0 += 32 * kU) {
+      int32_t v[kU][8];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t t = (q0 + u * 32 + lane) * 8;
+        if (t + 8 <= K && vec8) {
+          if (sizeof(T) == 2) {
+            const uint4 w = *reinterpret_cast<const uint4*>(xr + t);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              v[u][2 * r] = (int16_t)(ww[r] & 0xFFFFu);
+              v[u][2 * r + 1] = (int16_t)(ww[r] >> 16);
+            }
+          } else {
+            const int4 w0 = *reinterpret_cast<const int4*>(xr + t), w1 = *reinterpret_cast<const int4*>(xr + t + 4);
+            v[u][0] = w0.x; v[u][1] = w0.y; v[u][2] = w0.z; v[u][3] = w0.w;
+            v[u][4] = w1.x; v[u][5] = w1.y; v[u][6] = w1.z; v[u][7] = w1.w;
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) v[u][r] = (t < Kp && t + r < K) ? (int32_t)xr[t + r] : 0;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t t = (q0 + u * 32 + lane) * 8;
+        if (t >= Kp) continue;
+        uint32_t a[8], sg[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          sg[r] = v[u][r] < 0 ? 0xFFFFFFFFu : 0u;
+          a[r] = v[u][r] < 0 ? (uint32_t)(-(int64_t)v[u][r]) : (uint32_t)v[u][r];
+        }
+        for (int l = 0; l < P; ++l) {
+          const int sh = l * bm1;
+          uint32_t lo = 0, hi = 0;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const uint32_t d0 = sh < 31 ? ((a[r] >> sh) & mask) : 0u;
+            const uint32_t d1 = sh < 31 ? ((a[r + 4] >> sh) & mask) : 0u;
+            lo |= (((d0 ^ sg[r]) - sg[r]) & 0xFFu) << (8 * r);
+            hi |= (((d1 ^ sg[r + 4]) - sg[r + 4]) & 0xFFu) << (8 * r);
+          }
+          *reinterpret_cast<uint2*>(planes + (int64_t)l * Kp + t) = make_uint2(lo, hi);
+        }
+      }
+    }
+    __syncwarp();
+    // 2. the L unpacked lines, 16 inner positions per lane and step (512 contiguous bytes per warp)
+    for (int64_t c = lane; c < nchunk; c += 32) {
+      const int32_t t0 = meta_smem ? s_blk[c] : blk16[c];
+      const int64_t p = c * 16;
+      if (t0 >= 0) {
+        const int lk0 = meta_smem ? s_lk0[c] : lk[p];
+        for (int l = 0; l < L; ++l) {
+          const uint4 w = *reinterpret_cast<const uint4*>(planes + (int64_t)(l + lk0) * Kp + t0);
+          *reinterpret_cast<uint4*>(out + (base + l) * K_unp + p) = w;
+        }
+      } else {
+        const int4* tq = reinterpret_cast<const int4*>(tK + p);
+        const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
+        const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
+                                tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
+        const int4 lq = *reinterpret_cast<const int4*>(lk + p);
+        const int8_t* ll = reinterpret_cast<const int8_t*>(&lq);
+        for (int l = 0; l < L; ++l) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t packed = 0;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int k = q * 4 + r;
+              const uint32_t byte = tt[k] >= 0 ? (uint8_t)planes[(int64_t)(l + ll[k]) * Kp + tt[k]] : 0u;
+              packed |= byte << (8 * r);
+            }
+            w[q] = packed;
+          }
+          *reinterpret_cast<uint4*>(out + (base + l) * K_unp + p) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
 // Row gather for lines too long for shared-memory planes: digits are computed from the source line in
 // global memory (L2); lane = 4 consecutive inner positions, 128-byte coalesced stores per warp.
 template <typename T>
@@ -249,6 +435,26 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
   if (line_is_row) {
     // P planes per line: the levels an output line can ask for (line level + inner level)
     const int64_t Kp = (K + 15) / 16 * 16;
+    // one warp per line, each with its own planes, while 8 warps' planes fit in 96 KB (two CTAs per
+    // SM), else fewer warps per CTA down to one
+    {
+      const int64_t per_warp = (int64_t)P * Kp;
+      int nw = (int)((96 * 1024) / per_warp);
+      if (nw > 8) nw = 8;
+      if (nw >= 1) {
+        const int64_t nchunk = K_unp / 16;
+        const int meta_smem = nchunk <= kMetaMaxChunks ? 1 : 0;
+        const size_t smem = (size_t)nw * per_warp + (meta_smem ? (size_t)nchunk * 5 : 0);
+        const int per_sm = (int)((200 * 1024) / (smem + 1024)) < 1 ? 1 : (int)((200 * 1024) / (smem + 1024));
+        const int64_t ctas = (nlines + nw - 1) / nw;
+        int64_t grid = (int64_t)num_sms * (per_sm > 8 ? 8 : per_sm);
+        if (grid > ctas) grid = ctas;
+        IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_lines<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        k_unpack_lines<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, P, nw, outer, lvl, pos, tK, lk, blk16,
+                                                             K_unp, bm1, meta_smem, out);
+        return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+      }
+    }
     int NL = (int)((96 * 1024) / ((int64_t)P * Kp));
     if (NL > 8) NL = 8;
     if (NL < 1) {
