@@ -394,12 +394,25 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _gemm_source_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    for name in ("gemm.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "bit_integer_gemm_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _traffic_from_profiles():
-    """DRAM bytes per GEMM launch from the committed ncu summary of the current kernel, if present."""
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when the GEMM's source has
+    changed since those counters were taken (the summary records the hash of the source it measured)."""
     path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     try:
         with open(path) as f:
-            return json.load(f).get("bytes_per_launch")
+            rec = json.load(f)
+        if rec.get("source_sha1") != _gemm_source_sha1():
+            return None
+        return rec.get("bytes_per_launch")
     except Exception:
         return None
 
