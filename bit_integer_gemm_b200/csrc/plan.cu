@@ -12,8 +12,9 @@
 //                  histograms, the joint histogram of (level of A column t, level of B row t), and the
 //                  exact 128-bit bound sum_t max|A[:,t]| * max|B[t,:]|
 //   -- the summary (a few KB) is read back; the host fixes directions, groups and sizes --
-//   k_inner_map    one CTA per (lA, lB) segment: stream compaction of the inner indices t it holds
-//   k_outer_map    one CTA per level class: stable compaction of the lines of that level into groups
+//   k_plan_maps    one launch: one CTA per exponent group of the inner dimension (stream compaction of
+//                  the inner indices of each of its (lA, lB) segments, padding, 16-position blocks) and
+//                  one CTA per OUTER level class (stable compaction of the lines of that level into groups)
 #include <string.h>
 
 #include <mutex>
@@ -212,39 +213,52 @@ struct InnerSeg {
   int64_t off;
 };
 
-__global__ void __launch_bounds__(1024) k_inner_map(const InnerSeg* __restrict__ segs, const int8_t* __restrict__ lva,
-                                                    const int8_t* __restrict__ lvb, int a_inner, int b_inner,
-                                                    int64_t K, int32_t* __restrict__ tK,
-                                                    int8_t* __restrict__ lAk, int8_t* __restrict__ lBk) {
+// One exponent group of the unpacked inner dimension: positions [k0, k0 + kpad), filled by segments
+// seg0 .. seg0 + nseg - 1 in order and padded (source -1) up to kpad, a multiple of IMQ_INNER_PAD.
+struct InnerGroup {
+  int64_t k0, kpad;
+  int32_t seg0, nseg;
+};
+
+// The inner map of one exponent group (one CTA of 1024 threads): each segment's inner indices t (with
+// line levels la > seg.la and lb > seg.lb) in increasing order, then the padding, then blk16 for the
+// group's 16-position blocks: blk16[c] = t0 when block c holds t0..t0+15 (t0 % 16 == 0) with one
+// (lA, lB) pair, else -1.
+__device__ void inner_map_group(const InnerGroup grp, const InnerSeg* __restrict__ segs,
+                                const int8_t* __restrict__ lva, const int8_t* __restrict__ lvb, int a_inner,
+                                int b_inner, int64_t K, int32_t* __restrict__ tK, int8_t* __restrict__ lAk,
+                                int8_t* __restrict__ lBk, int32_t* __restrict__ blk16) {
   __shared__ int warp_tot[32];
   __shared__ int total;
-  const InnerSeg sg = segs[blockIdx.x];
-  int64_t base = sg.off;
-  for (int64_t t0 = 0; t0 < K; t0 += 1024) {
-    const int64_t t = t0 + threadIdx.x;
-    int pred = 0;
-    if (t < K) {
-      const int la = a_inner ? lva[t] : 1;
-      const int lb = b_inner ? lvb[t] : 1;
-      pred = (la > sg.la) && (lb > sg.lb);
+  int64_t base = grp.k0;
+  for (int si = 0; si < grp.nseg; ++si) {
+    const InnerSeg sg = segs[grp.seg0 + si];
+    for (int64_t t0 = 0; t0 < K; t0 += 1024) {
+      const int64_t t = t0 + threadIdx.x;
+      int pred = 0;
+      if (t < K) {
+        const int la = a_inner ? lva[t] : 1;
+        const int lb = b_inner ? lvb[t] : 1;
+        pred = (la > sg.la) && (lb > sg.lb);
+      }
+      const int r = block_rank(pred, warp_tot, &total);
+      if (pred) {
+        tK[base + r] = (int32_t)t;
+        lAk[base + r] = (int8_t)sg.la;
+        lBk[base + r] = (int8_t)sg.lb;
+      }
+      __syncthreads();
+      base += total;
+      __syncthreads();
     }
-    const int r = block_rank(pred, warp_tot, &total);
-    if (pred) {
-      tK[base + r] = (int32_t)t;
-      lAk[base + r] = (int8_t)sg.la;
-      lBk[base + r] = (int8_t)sg.lb;
-    }
-    __syncthreads();
-    base += total;
-    __syncthreads();
   }
-}
-
-// blk16[c] = t0 when the 16 inner positions of block c are t0..t0+15 (t0 % 16 == 0) with one (lA, lB)
-// pair, else -1.
-__global__ void k_inner_blocks(const int32_t* __restrict__ tK, const int8_t* __restrict__ lAk,
-                               const int8_t* __restrict__ lBk, int64_t nblk, int32_t* __restrict__ blk16) {
-  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < nblk; c += (int64_t)gridDim.x * blockDim.x) {
+  for (int64_t q = base + threadIdx.x; q < grp.k0 + grp.kpad; q += blockDim.x) {
+    tK[q] = -1;
+    lAk[q] = 0;
+    lBk[q] = 0;
+  }
+  __syncthreads();  // the block's writes above are visible to all its threads after this
+  for (int64_t c = grp.k0 / 16 + threadIdx.x; c < (grp.k0 + grp.kpad) / 16; c += blockDim.x) {
     const int32_t* t = tK + c * 16;
     const int32_t t0 = t[0];
     bool ok = t0 >= 0 && (t0 & 15) == 0;
@@ -282,8 +296,10 @@ __device__ void outer_map_class(const OuterClass c, const int8_t* __restrict__ l
   __shared__ int total;
   const int64_t ngrp = (c.count + c.per - 1) / c.per;
   for (int64_t g = threadIdx.x; g < ngrp; g += blockDim.x) {
+    const int32_t ng = (int32_t)(g < ngrp - 1 ? c.per : c.count - (ngrp - 1) * c.per);
     grpL[c.grp0 + g] = c.L;
-    grpN[c.grp0 + g] = (int32_t)(g < ngrp - 1 ? c.per : c.count - (ngrp - 1) * c.per);
+    grpN[c.grp0 + g] = ng;
+    for (int u = ng * c.L; u < G; ++u) src[(c.grp0 + g) * G + u] = -1;  // unused unpacked lines
   }
   int64_t rank0 = 0;
   for (int64_t i0 = 0; i0 < n; i0 += 1024) {
@@ -302,29 +318,34 @@ __device__ void outer_map_class(const OuterClass c, const int8_t* __restrict__ l
   }
 }
 
-// Both matrices' classes in one launch: blocks [0, a.ncls) take A's, the rest B's.
-__global__ void __launch_bounds__(1024) k_outer_map(OuterJob a, OuterJob b) {
-  const bool is_a = (int)blockIdx.x < a.ncls;
-  const OuterJob& j = is_a ? a : b;
-  const int ci = is_a ? (int)blockIdx.x : (int)blockIdx.x - a.ncls;
-  outer_map_class(j.cls[ci], j.lv, j.n, j.G, j.pos, j.src, j.grpL, j.grpN);
-}
+// Stage 2 of a plan in one launch: blocks [0, ngrp) build the inner map of one exponent group each, the
+// next a.ncls blocks one OUTER class of A each, the rest one OUTER class of B each.
+struct MapsArgs {
+  const InnerGroup* grps;
+  int ngrp;
+  const InnerSeg* segs;
+  const int8_t* lva;
+  const int8_t* lvb;
+  int a_inner, b_inner;
+  int64_t K;
+  int32_t* tK;
+  int8_t* lAk;
+  int8_t* lBk;
+  int32_t* blk16;
+  OuterJob a, b;
+};
 
-// Stage-2 initial values in one launch: every unpacked inner position starts as padding (source -1,
-// inner levels 0) and every OUTER unpacked line as unused (source -1).
-__global__ void k_plan_init(int32_t* __restrict__ tK, int8_t* __restrict__ lAk, int8_t* __restrict__ lBk,
-                            int64_t K_unp, int32_t* __restrict__ srcA, int64_t M_unp, int32_t* __restrict__ srcB,
-                            int64_t N_unp) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < K_unp; i += stride) {
-    tK[i] = -1;
-    lAk[i] = 0;
-    lBk[i] = 0;
+__global__ void __launch_bounds__(1024) k_plan_maps(MapsArgs m) {
+  const int bx = (int)blockIdx.x;
+  if (bx < m.ngrp) {
+    inner_map_group(m.grps[bx], m.segs, m.lva, m.lvb, m.a_inner, m.b_inner, m.K, m.tK, m.lAk, m.lBk, m.blk16);
+    return;
   }
-  if (srcA)
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < M_unp; i += stride) srcA[i] = -1;
-  if (srcB)
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N_unp; i += stride) srcB[i] = -1;
+  const int ob = bx - m.ngrp;
+  const bool is_a = ob < m.a.ncls;
+  const OuterJob& j = is_a ? m.a : m.b;
+  const int ci = is_a ? ob : ob - m.a.ncls;
+  outer_map_class(j.cls[ci], j.lv, j.n, j.G, j.pos, j.src, j.grpL, j.grpN);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -378,9 +399,11 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   IMQ_CUDA_TRY(cudaGetDevice(&dev));
   Pinned& pin = g_pinned[dev & 63];
   std::lock_guard<std::mutex> lock(pin.mu);
-  const size_t tables_bytes = sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv;
-  // staging: the segment table padded to 256 bytes, then the class table (the device layout)
-  const size_t staging_bytes = align_up(sizeof(InnerSeg) * kLv * kLv, 256) + sizeof(OuterClass) * 2 * kLv;
+  const size_t tables_bytes =
+      sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
+  // staging in the device layout: segments, classes and groups, each padded to 256 bytes
+  const size_t staging_bytes = align_up(sizeof(InnerSeg) * kLv * kLv, 256) +
+                               align_up(sizeof(OuterClass) * 2 * kLv, 256) + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
   if (!pin.sum) IMQ_CUDA_TRY(cudaMallocHost(&pin.sum, sizeof(Summary)));
   if (!pin.tables) IMQ_CUDA_TRY(cudaMallocHost(&pin.tables, staging_bytes));
   if (!pin.tables_done) IMQ_CUDA_TRY(cudaEventCreateWithFlags(&pin.tables_done, cudaEventDisableTiming));
@@ -394,6 +417,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   }
   InnerSeg* hsegs = static_cast<InnerSeg*>(pl->host_tables);
   OuterClass* hcls = reinterpret_cast<OuterClass*>(hsegs + kLv * kLv);
+  InnerGroup* hgrps = reinterpret_cast<InnerGroup*>(hcls + 2 * kLv);
   pl->device = dev;
   pl->A = A;
   pl->B = B;
@@ -421,6 +445,8 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   off = align_up(off + sizeof(InnerSeg) * kLv * kLv, 256);
   const size_t o_cls = off;
   off = align_up(off + sizeof(OuterClass) * 2 * kLv, 256);
+  const size_t o_grps = off;
+  off = align_up(off + sizeof(InnerGroup) * IMQ_MAX_GROUPS, 256);
   const size_t stage1 = off;
   char* blk1 = nullptr;
   if (cudaMallocFromPoolAsync((void**)&blk1, stage1, ds->pool, st) != cudaSuccess) {
@@ -562,6 +588,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   int ng = 0;
   for (int e = 0; e <= maxla + maxlb - 2; ++e) {
     int64_t glen = 0;
+    const int seg_first = nseg;
     for (int sa = 0; sa < maxla; ++sa) {
       const int sb = e - sa;
       if (sb < 0 || sb >= maxlb) continue;
@@ -579,6 +606,10 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     pl->groups[ng].k_offset = koff;
     pl->groups[ng].k_len = glen;
     pl->groups[ng].k_len_padded = (glen + IMQ_INNER_PAD - 1) / IMQ_INNER_PAD * IMQ_INNER_PAD;
+    hgrps[ng].k0 = koff;
+    hgrps[ng].kpad = pl->groups[ng].k_len_padded;
+    hgrps[ng].seg0 = seg_first;
+    hgrps[ng].nseg = nseg - seg_first;
     koff += pl->groups[ng].k_len_padded;
     keff += glen;
     ++ng;
@@ -728,37 +759,37 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     pl->grpB_L = reinterpret_cast<int32_t*>(b2 + o_gLB);
     pl->grpB_n = reinterpret_cast<int32_t*>(b2 + o_gNB);
   }
-  {
-    const int64_t most = I.K_unp > I.M_unp ? (I.K_unp > I.N_unp ? I.K_unp : I.N_unp) : (I.M_unp > I.N_unp ? I.M_unp : I.N_unp);
-    int64_t grid = (most + 255) / 256;
-    if (grid > ds->num_sms * 4) grid = ds->num_sms * 4;
-    if (grid < 1) grid = 1;
-    k_plan_init<<<(unsigned)grid, 256, 0, st>>>(pl->tK, pl->lAk, pl->lBk, I.K_unp, a_outer ? pl->srcA : nullptr,
-                                               I.M_unp, b_outer ? pl->srcB : nullptr, I.N_unp);
-  }
-  if (nseg > 0 || ncls > 0) {
+  if (ng > 0 || ncls > 0) {
     // one upload from pinned staging (an asynchronous copy; pageable memory would be staged by the
     // driver first); the staging is reused once the previous plan's upload has completed
     if (cudaEventSynchronize(pin.tables_done) != cudaSuccess) return fail(IMQ_ERR_CUDA);
     char* stg = static_cast<char*>(pin.tables);
-    const size_t segb = sizeof(InnerSeg) * (nseg > 0 ? nseg : 1), clsb = sizeof(OuterClass) * (ncls > 0 ? ncls : 1);
-    memcpy(stg, hsegs, segb);
-    memcpy(stg + (o_cls - o_segs), hcls, clsb);
-    if (cudaMemcpyAsync(dsegs, stg, (o_cls - o_segs) + clsb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+    memcpy(stg, hsegs, sizeof(InnerSeg) * (size_t)nseg);
+    memcpy(stg + (o_cls - o_segs), hcls, sizeof(OuterClass) * (size_t)ncls);
+    memcpy(stg + (o_grps - o_segs), hgrps, sizeof(InnerGroup) * (size_t)ng);
+    if (cudaMemcpyAsync(dsegs, stg, (o_grps - o_segs) + sizeof(InnerGroup) * (size_t)ng, cudaMemcpyHostToDevice,
+                        st) != cudaSuccess ||
         cudaEventRecord(pin.tables_done, st) != cudaSuccess)
       return fail(IMQ_ERR_CUDA);
-  }
-  if (nseg > 0) {
-    k_inner_map<<<nseg, 1024, 0, st>>>(dsegs, pl->lv_a_col, pl->lv_b_row, a_inner, b_inner, K, pl->tK, pl->lAk, pl->lBk);
-    const int64_t nblk = I.K_unp / 16;
-    k_inner_blocks<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(pl->tK, pl->lAk, pl->lBk, nblk, pl->blk16);
-  }
-  {
-    OuterJob ja = {dcls + cls_a0, a_outer ? cls_a1 - cls_a0 : 0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
-                   pl->grpA_L, pl->grpA_n};
-    OuterJob jb = {dcls + cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
-                   pl->grpB_L, pl->grpB_n};
-    if (ja.ncls + jb.ncls > 0) k_outer_map<<<ja.ncls + jb.ncls, 1024, 0, st>>>(ja, jb);
+    MapsArgs m;
+    m.grps = reinterpret_cast<const InnerGroup*>(blk1 + o_grps);
+    m.ngrp = ng;
+    m.segs = dsegs;
+    m.lva = pl->lv_a_col;
+    m.lvb = pl->lv_b_row;
+    m.a_inner = a_inner;
+    m.b_inner = b_inner;
+    m.K = K;
+    m.tK = pl->tK;
+    m.lAk = pl->lAk;
+    m.lBk = pl->lBk;
+    m.blk16 = pl->blk16;
+    m.a = {dcls + cls_a0, a_outer ? cls_a1 - cls_a0 : 0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
+           pl->grpA_L, pl->grpA_n};
+    m.b = {dcls + cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
+           pl->grpB_L, pl->grpB_n};
+    const int blocks = ng + m.a.ncls + m.b.ncls;
+    if (blocks > 0) k_plan_maps<<<blocks, 1024, 0, st>>>(m);
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
   *out = pl;

@@ -239,15 +239,17 @@ __device__ uint32_t warp_select_key_bf16(const uint16_t* a, int n, unsigned long
   for (int b = 14; b >= 0; --b) {
     const uint32_t t = ans | (1u << b);
     const uint32_t t2 = t | (t << 16);
-    uint32_t acc = 0;
+    // four independent counters, so that consecutive words do not wait on one another's add
+    uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
 #pragma unroll 4
     for (int i = lane; i < nv; i += 32) {
       const uint4 w = reinterpret_cast<const uint4*>(a)[i];
-      acc += (((w.x | 0x80008000u) - t2) >> 15) & 0x00010001u;
-      acc += (((w.y | 0x80008000u) - t2) >> 15) & 0x00010001u;
-      acc += (((w.z | 0x80008000u) - t2) >> 15) & 0x00010001u;
-      acc += (((w.w | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      c0 += (((w.x | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      c1 += (((w.y | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      c2 += (((w.z | 0x80008000u) - t2) >> 15) & 0x00010001u;
+      c3 += (((w.w | 0x80008000u) - t2) >> 15) & 0x00010001u;
     }
+    const uint32_t acc = (c0 + c1) + (c2 + c3);
     uint32_t ge = (acc & 0xFFFFu) + (acc >> 16);
     for (int i = nv * 8 + lane; i < n; i += 32) ge += (a[i] & 0x7FFFu) >= t ? 1u : 0u;
 #pragma unroll
