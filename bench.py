@@ -7,7 +7,7 @@ W 4096x4096 bf16 per-output-channel RTN, p = 0.95, beta = 15, b = 5, Mix): perce
 plan, unpack, tcgen05 int8 GEMM with fold-back and dequantisation.  `value` is the effective TOPS of
 the original-shape product, 2*M*N*K / step time, with inputs resident in HBM; `e2e` is the same through
 the C ABI with the inputs copied from pinned host memory and C (int32) plus Cf (fp32) copied back inside
-the timed region.  Between timed steps L2 is flushed by writing 256 MB.  The dominant kernel (the GEMM)
+the timed region, the copies pipelined against the compute on their own streams.  Between timed steps L2 is flushed by writing 256 MB.  The dominant kernel (the GEMM)
 is timed with CUDA events on its stream for the roofline.  With --gpus N > 1 every rank runs its own
 replica (the path has no data exchange); time is the max over ranks.
 
@@ -179,11 +179,17 @@ class Path:
         self.info = None
         self.launches = 0
 
-    def step(self, gemm_events=None):
+    def step(self, gemm_events=None, X=None, W=None, C=None, Cf=None):
+        """One pass of the path on the current stream; X, W in and C, Cf out default to the Path's own
+        buffers (the end-to-end loop passes double-buffered ones)."""
         imq, g = self.imq, self.g
-        imq.imq_rtn_quantize(self.X, imq.IMQ_PER_ROW, g.p, g.beta, Xint=self.Xint, delta=self.dX,
+        X = self.X if X is None else X
+        W = self.W if W is None else W
+        C = self.C if C is None else C
+        Cf = self.Cf if Cf is None else Cf
+        imq.imq_rtn_quantize(X, imq.IMQ_PER_ROW, g.p, g.beta, Xint=self.Xint, delta=self.dX,
                              want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
-        imq.imq_rtn_quantize(self.W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
+        imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
                              want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True)
         plan = imq.imq_plan(self.Xint, self.Wint, g.b, imq.IMQ_MIX, transB=True, maxes=self.mx)
         I = plan.info
@@ -198,8 +204,7 @@ class Path:
         imq.imq_unpack(plan, self.Xint, self.Wint, A_unp=Au, B_unp_t=Bu)
         if gemm_events is not None:
             gemm_events[0].record()
-        imq.imq_gemm_unpacked(plan, Au, Bu, self.dX, imq.IMQ_PER_ROW, self.dW, imq.IMQ_PER_COL, C=self.C,
-                              Cf=self.Cf)
+        imq.imq_gemm_unpacked(plan, Au, Bu, self.dX, imq.IMQ_PER_ROW, self.dW, imq.IMQ_PER_COL, C=C, Cf=Cf)
         if gemm_events is not None:
             gemm_events[1].record()
         self.info = I
@@ -264,26 +269,49 @@ def run_ours(args):
     launches = path.launches * args.steps
 
     # ---- end to end through the C ABI with host buffers ----
+    # Every step copies its X and W from pinned host memory and reads C and Cf back.  The copies run on
+    # their own streams, double-buffered, so that step k+1's upload and step k-1's download overlap
+    # step k's compute; the time is from the first upload's start to the last download's end.
     Xp = Xh.pin_memory()
     Wp = Wh.pin_memory()
-    Cp = torch.empty((g.M, g.N), dtype=torch.int32).pin_memory()
-    Cfp = torch.empty((g.M, g.N), dtype=torch.float32).pin_memory()
-    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    Cp = [torch.empty((g.M, g.N), dtype=torch.int32).pin_memory() for _ in range(2)]
+    Cfp = [torch.empty((g.M, g.N), dtype=torch.float32).pin_memory() for _ in range(2)]
+    Xd = [X, torch.empty_like(X)]
+    Wd = [W, torch.empty_like(W)]
+    Cd = [path.C, torch.empty_like(path.C)]
+    Cfd = [path.Cf, torch.empty_like(path.Cf)]
+    s_comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done = [ev() for _ in range(args.steps)]
+    comp_done = [ev() for _ in range(args.steps)]
+    out_done = [ev() for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    t_start.record(s_in)
     for k in range(args.steps):
-        flush.zero_()
-        e_start[k].record()
-        X.copy_(Xp, non_blocking=True)
-        W.copy_(Wp, non_blocking=True)
-        path.step()
-        Cp.copy_(path.C, non_blocking=True)
-        Cfp.copy_(path.Cf, non_blocking=True)
-        e_end[k].record()
+        b = k % 2
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(comp_done[k - 2])  # step k-2 has read this input slot
+            Xd[b].copy_(Xp, non_blocking=True)
+            Wd[b].copy_(Wp, non_blocking=True)
+            in_done[k].record(s_in)
+        s_comp.wait_event(in_done[k])
+        if k >= 2:
+            s_comp.wait_event(out_done[k - 2])  # step k-2's result has been read from this slot
+        path.step(X=Xd[b], W=Wd[b], C=Cd[b], Cf=Cfd[b])
+        comp_done[k].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[k])
+            Cp[b].copy_(Cd[b], non_blocking=True)
+            Cfp[b].copy_(Cfd[b], non_blocking=True)
+            out_done[k].record(s_out)
+    t_end.record(s_out)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_start, e_end))
+    e2e_ms = t_start.elapsed_time(t_end)
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist if world > 1 else None, dev)
 
@@ -310,7 +338,11 @@ def run_ours(args):
                      "kernel": "k_gemm (tcgen05 kind::i8)", "peak_source": f"{src} bf16 burst x2",
                      "gemm_ms": round(gemm_avg_ms, 4), "exec_ops_per_launch": exec_ops},
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": 2 * (g.M * g.K + g.K * g.N),
-                "d2h_bytes_per_step": 8 * g.M * g.N},
+                "d2h_bytes_per_step": 8 * g.M * g.N,
+                "how": "every step uploads X, W from pinned host memory and reads C, Cf back; uploads, "
+                       "compute and downloads on three streams, double-buffered, timed from the first "
+                       "upload to the last download; no L2 flush (inputs arrive from the host each step, "
+                       "per-step working set about 270 MB > L2)"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }

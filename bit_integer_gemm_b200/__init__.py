@@ -121,7 +121,8 @@ def _check(status: int, what: str):
 
 def _stream(stream) -> int:
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        # torch's current stream on the current device, without building a Stream object
+        return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
