@@ -46,21 +46,6 @@ imq_status device_state(DeviceState** out) {
   return IMQ_OK;
 }
 
-imq_status partials_buffer(DeviceState* ds, size_t bytes, void** out) {
-  if (bytes > ds->partials_bytes) {
-    std::lock_guard<std::mutex> lock(g_dev_mu);
-    if (bytes > ds->partials_bytes) {
-      if (ds->partials) IMQ_CUDA_TRY(cudaFree(ds->partials));
-      ds->partials = nullptr;
-      ds->partials_bytes = 0;
-      const size_t n = (bytes + (1 << 20) - 1) >> 20 << 20;
-      IMQ_CUDA_TRY(cudaMalloc(&ds->partials, n));
-      ds->partials_bytes = n;
-    }
-  }
-  *out = ds->partials;
-  return IMQ_OK;
-}
 
 namespace {
 // Block of 32 x 8 threads: x = 32 consecutive entries (coalesced), y = a slice of the partials; the

@@ -11,22 +11,16 @@ namespace imq {
 
 constexpr int kMaxJobs = 128;  // accumulation jobs of one output tile
 
-// Per-device state owned by the library: the status word address and small scratch buffers.
+// Per-device state owned by the library: the status word address, the SM count and the memory pool.
 struct DeviceState {
   int32_t* status = nullptr;   // device address of the status word of this device
-  void* scratch = nullptr;     // per-tensor quantiser state (allocated on first use)
-  void* partials = nullptr;    // per-CTA partial line maxima of the quantiser (grown on demand)
-  size_t partials_bytes = 0;
   int num_sms = 0;
-  // stream-ordered pool for plan memory; it keeps what plans free (no trim at synchronisation), so a
-  // new plan reuses memory instead of mapping fresh pages
+  // stream-ordered pool for plan memory and the quantiser's per-call scratch; it keeps what is freed
+  // (no trim at synchronisation), so later calls reuse memory instead of mapping fresh pages
   cudaMemPool_t pool = nullptr;
   bool init = false;
 };
 imq_status device_state(DeviceState** out);
-// Returns a device buffer of at least `bytes` for per-CTA partial results (grown on first need; a
-// growth frees the old buffer, which waits for the device).
-imq_status partials_buffer(DeviceState* ds, size_t bytes, void** out);
 // out[i] = max over p < nparts of part[p * n + i] (int32, non-negative); nparts may be 0 (out = 0).
 imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st);
 

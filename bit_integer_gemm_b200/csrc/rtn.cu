@@ -18,8 +18,8 @@
 //                 hit L2) and once more to quantise.
 //   k_tensor_*    per-tensor select: global 256-bin histograms per pass, then k_rtn_rows.
 // Side outputs: max |x_int| per stored row and column, the line statistics the unpack plan needs.  The
-// maxima that cross CTAs are written as per-CTA partials to a library scratch buffer and reduced by a
-// second small kernel (no global atomics).
+// maxima that cross CTAs are written as per-CTA partials to per-call scratch (stream-ordered, from the
+// library's pool) and reduced by a second small kernel (no global atomics).
 #include <math.h>
 
 #include <atomic>
@@ -673,6 +673,21 @@ __global__ void k_fill_f32(float* p, int64_t n, float v) {
     p[i] = v;
 }
 
+// Per-call scratch from the library's stream-ordered pool, allocated and freed on the call's stream:
+// the free is ordered after every kernel of the call that uses it, and calls on different streams never
+// share it, so they may run concurrently.
+struct StreamScratch {
+  void* p = nullptr;
+  cudaStream_t st = nullptr;
+  imq_status alloc(DeviceState* ds, size_t bytes, cudaStream_t s) {
+    st = s;
+    return cudaMallocFromPoolAsync(&p, bytes > 0 ? bytes : 16, ds->pool, s) == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+  }
+  ~StreamScratch() {
+    if (p) cudaFreeAsync(p, st);
+  }
+};
+
 int64_t nearest_rank(int64_t n, double p) {
   if (n <= 0) return 1;
   int64_t k = (int64_t)ceil(p * (double)n);
@@ -690,11 +705,10 @@ imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, u
   const bool vec = (ld % (16 / (int64_t)sizeof(T)) == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   const int64_t grid = (cols + CW - 1) / CW;
   int32_t* part = nullptr;
+  StreamScratch sp;
   if (rowmax) {
-    void* pb;
-    imq_status e = partials_buffer(ds, (size_t)grid * rows * 4, &pb);
-    if (e != IMQ_OK) return e;
-    part = static_cast<int32_t*>(pb);
+    if (sp.alloc(ds, (size_t)grid * rows * 4, st) != IMQ_OK) return IMQ_ERR_CUDA;
+    part = static_cast<int32_t*>(sp.p);
   }
   auto kern = k_rtn_cols_staged<T, CW, kOut16>;
   IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -725,11 +739,10 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
                                            colmax, ds, st);
     const int64_t grid = (cols + kColsPerCta - 1) / kColsPerCta;
     int32_t* part = nullptr;
+    StreamScratch sp;
     if (rowmax) {
-      void* pb;
-      imq_status e = partials_buffer(ds, (size_t)grid * rows * 4, &pb);
-      if (e != IMQ_OK) return e;
-      part = static_cast<int32_t*>(pb);
+      if (sp.alloc(ds, (size_t)grid * rows * 4, st) != IMQ_OK) return IMQ_ERR_CUDA;
+      part = static_cast<int32_t*>(sp.p);
     }
     k_rtn_cols<T, kOut16><<<(unsigned)grid, kThreads, 0, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out,
                                                                delta, qval, part, colmax, ds->status);
@@ -752,16 +765,15 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
   const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
                    ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   int32_t* part = nullptr;
+  StreamScratch sp, sts;
   if (colmax) {
-    void* pb;
-    imq_status e = partials_buffer(ds, (size_t)grid * cols * 4, &pb);
-    if (e != IMQ_OK) return e;
-    part = static_cast<int32_t*>(pb);
+    if (sp.alloc(ds, (size_t)grid * cols * 4, st) != IMQ_OK) return IMQ_ERR_CUDA;
+    part = static_cast<int32_t*>(sp.p);
   }
   TensorState* ts = nullptr;
   if (g == IMQ_PER_TENSOR) {
-    if (!ds->scratch) IMQ_CUDA_TRY(cudaMalloc(&ds->scratch, sizeof(TensorState)));
-    ts = static_cast<TensorState*>(ds->scratch);
+    if (sts.alloc(ds, sizeof(TensorState), st) != IMQ_OK) return IMQ_ERR_CUDA;
+    ts = static_cast<TensorState*>(sts.p);
     k_tensor_init<<<1, 256, 0, st>>>(ts, (unsigned long long)nearest_rank(rows * cols, p));
     const int64_t hgrid = rows < (int64_t)sms * 8 ? rows : (int64_t)sms * 8;
     const int np = num_passes(Key<T>::kBits);
@@ -828,9 +840,8 @@ imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_
 // ------------------------------------------------------------------------------------------------
 // Allocation-free per-row quantiser (imq_rtn_quantize_rows_noalloc).
 //
-// Callers whose own allocator has reserved the free device memory, or that must not stall their other
-// streams behind the device-wide wait of a cudaFree, cannot use the grown partials buffer above.  For
-// them the per-CTA column maxima of k_rtn_rows go to one fixed array in this module's device image,
+// Callers whose own allocator has reserved the free device memory cannot let the library's pool grow
+// for the per-call scratch above.  For them the per-CTA column maxima of k_rtn_rows go to one fixed array in this module's device image,
 // mapped by the CUDA runtime when the module loads.  Its device address is looked up once per device,
 // on the first call with that device current.  Every call on a device shares the array, so calls whose
 // executions overlap race on it.  Nothing in it has to start at zero: each CTA writes its whole slice

@@ -100,7 +100,9 @@ typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2 } imq_dir;
  * rowmax  device or NULL, int32[rows]: max |x_int| over each row of X (whatever trans_out is).
  * colmax  device or NULL, int32[cols]: max |x_int| over each column of X.
  * Errors: IMQ_ERR_ARG at once; IMQ_ERR_NONFINITE / IMQ_ERR_RANGE through the device status word.
- * Scratch: PER_TENSOR uses a small per-device buffer the library allocates once on first use.
+ * Scratch: the per-CTA partial line maxima (and, for PER_TENSOR, the select state) come from a
+ *         library-owned stream-ordered memory pool, allocated and freed on `stream`; calls on
+ *         different streams therefore never share scratch and may run concurrently.
  */
 imq_status imq_rtn_quantize(const void *X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                             imq_gran g, double p, int32_t beta,
@@ -114,12 +116,11 @@ imq_status imq_rtn_quantize(const void *X, imq_dtype xt, int64_t rows, int64_t c
  * but it allocates no device memory.  The IM-Unpack page has no counterpart to this call: it is an
  * interface convenience of this library, not a step of the method.
  *
- * Why: imq_rtn_quantize keeps the per-CTA partial column maxima in a library buffer that it grows
- * with cudaMalloc, freeing the old one with cudaFree, which waits for all work on the device.  Two
- * kinds of caller cannot take that: a process whose own allocator has reserved the free device
- * memory up front (a serving engine that owns every byte of HBM, where the library's cudaMalloc
- * fails), and a caller that must not stall its other streams behind a device-wide cudaFree.  This
- * call takes its scratch from one fixed array in the library's device image instead, of
+ * Why: imq_rtn_quantize takes its per-CTA partial column maxima from a library-owned memory pool,
+ * which maps more device memory whenever it has to grow.  A process whose own allocator has reserved
+ * the free device memory up front (a serving engine that owns every byte of HBM) cannot let a
+ * library grow a pool: the allocation fails there, or it takes memory the process had planned for.
+ * This call takes its scratch from one fixed array in the library's device image instead, of
  * IMQ_NOALLOC_SCRATCH_BYTES per device, which the CUDA runtime maps when it loads the module.
  *
  * Scratch needed: 4 * cols * G bytes when colmax is requested, where G is the number of CTAs the
