@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
 // go to `part` (reduced afterwards); column maxima are written directly.
 // ------------------------------------------------------------------------------------------------
 template <typename T, int CW, bool kOut16>
-__global__ void __launch_bounds__(CW * 32) k_rtn_cols_staged(
+__global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
     void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
     int32_t* __restrict__ part, int32_t* __restrict__ colmax, int vec, int32_t* status) {
