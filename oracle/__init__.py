@@ -28,7 +28,7 @@ _SO = os.path.join(_HERE, "liboracle.so")
 _SRCS = ["percentile.c", "rtn.c", "digits.c", "plan.c", "unpack.c", "gemm.c", "dequant.c"]
 
 PER_TENSOR, PER_ROW, PER_COL = 0, 1, 2
-MIX, ROW_ROW, ROW_COL, COL_ROW, COL_COL = 0, 1, 2, 3, 4
+MIX, ROW_ROW, ROW_COL, COL_ROW, COL_COL, MIX_JOINT = 0, 1, 2, 3, 4, 5
 DIR_NONE, DIR_OUTER, DIR_INNER = 0, 1, 2
 OK, ERR_ARG, ERR_NONFINITE, ERR_RANGE = 0, 1, 2, 3
 MAX_GROUPS = 64

@@ -30,6 +30,9 @@
 #define OR_ROW_COL 2
 #define OR_COL_ROW 3
 #define OR_COL_COL 4
+/* Joint Mix: the (A, B) direction pair of least exact unpacked cost M_eff * N_eff * K_eff over the four
+ * pairs (a reading of the page's per-matrix choice; see oracle_plan). */
+#define OR_MIX_JOINT 5
 
 #define OR_DIR_NONE 0
 #define OR_DIR_OUTER 1

@@ -29,7 +29,7 @@ static int64_t iabs64(int64_t v) { return v < 0 ? -v : v; }
 int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N, int b,
                 int strategy, int32_t *LrA, int32_t *LcA, int32_t *LrB, int32_t *LcB,
                 oracle_plan_t *out) {
-  if (b < 2 || b > 8 || M < 0 || K < 0 || N < 0 || strategy < 0 || strategy > 4) return OR_ERR_ARG;
+  if (b < 2 || b > 8 || M < 0 || K < 0 || N < 0 || strategy < 0 || strategy > 5) return OR_ERR_ARG;
   memset(out, 0, sizeof(*out));
   out->b = b;
   out->strategy = strategy;
@@ -66,7 +66,7 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
 
   /* direction of each matrix */
   int da, db;
-  if (strategy == OR_MIX) {
+  if (strategy == OR_MIX || strategy == OR_MIX_JOINT) {
     if (out->oor_lines[0] == 0 && out->oor_lines[1] == 0) {
       da = OR_DIR_NONE;
     } else {
@@ -92,6 +92,30 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
   } else {
     da = (strategy == OR_ROW_ROW || strategy == OR_ROW_COL) ? OR_DIR_OUTER : OR_DIR_INNER;
     db = (strategy == OR_ROW_ROW || strategy == OR_COL_ROW) ? OR_DIR_INNER : OR_DIR_OUTER;
+  }
+  if (strategy == OR_MIX_JOINT) {
+    /* Joint Mix: starting from the per-matrix Mix choice above, take the direction pair whose exact
+     * unpacked size M_eff * N_eff * K_eff is strictly smaller, trying the pairs in the order
+     * row/row, row/col, col/row, col/col (A's direction / B's).  A matrix without out-of-range entries
+     * stays not unpacked (its size factors are 1 either way). */
+    const int pa[4] = {OR_DIR_OUTER, OR_DIR_OUTER, OR_DIR_INNER, OR_DIR_INNER};
+    const int pb[4] = {OR_DIR_INNER, OR_DIR_OUTER, OR_DIR_INNER, OR_DIR_OUTER};
+    unsigned __int128 best = 0;
+    for (int c = -1; c < 4; ++c) {
+      const int ca = c < 0 ? da : (da == OR_DIR_NONE ? OR_DIR_NONE : pa[c]);
+      const int cb = c < 0 ? db : (db == OR_DIR_NONE ? OR_DIR_NONE : pb[c]);
+      unsigned __int128 me = 0, ne = 0, ke = 0;
+      for (int64_t i = 0; i < M; ++i) me += (ca == OR_DIR_OUTER) ? (unsigned)LrA[i] : 1u;
+      for (int64_t j = 0; j < N; ++j) ne += (cb == OR_DIR_OUTER) ? (unsigned)LcB[j] : 1u;
+      for (int64_t t = 0; t < K; ++t)
+        ke += (unsigned __int128)((ca == OR_DIR_INNER) ? LcA[t] : 1) * (unsigned)((cb == OR_DIR_INNER) ? LrB[t] : 1);
+      const unsigned __int128 cost = me * ne * ke;
+      if (c < 0 || cost < best) {
+        best = cost;
+        da = ca;
+        db = cb;
+      }
+    }
   }
   out->dir_a = da;
   out->dir_b = db;

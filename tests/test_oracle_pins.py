@@ -308,6 +308,69 @@ def test_mix_choice_bruteforce():
         assert pl.dir_b == choose(lbr, lbc, False)
 
 
+def _pair_cost(lar, lac, lbr, lbc, da, db):
+    """Exact unpacked size M_eff * N_eff * K_eff of one direction pair, from the line levels."""
+    M, N = lar.size, lbc.size
+    me = int(lar.sum()) if da == oracle.DIR_OUTER else M
+    ne = int(lbc.sum()) if db == oracle.DIR_OUTER else N
+    la = lac if da == oracle.DIR_INNER else np.ones_like(lac)
+    lb = lbr if db == oracle.DIR_INNER else np.ones_like(lbr)
+    return me * ne * int((la.astype(np.int64) * lb.astype(np.int64)).sum())
+
+
+def test_joint_mix_is_the_cheapest_pair_bruteforce():
+    """Joint Mix (a reading of the per-matrix choice that weighs both matrices together): the pair of
+    least exact unpacked size, strict improvements over the per-matrix Mix choice taken in the order
+    row/row, row/col, col/row, col/col.  Costs re-derived from numpy levels."""
+    rng = np.random.default_rng(27)
+    pairs = [(oracle.DIR_OUTER, oracle.DIR_INNER), (oracle.DIR_OUTER, oracle.DIR_OUTER),
+             (oracle.DIR_INNER, oracle.DIR_INNER), (oracle.DIR_INNER, oracle.DIR_OUTER)]
+    differs = 0
+    for _ in range(400):
+        M, K, N = (int(x) for x in rng.integers(1, 10, size=3))
+        b = int(rng.integers(2, 9))
+        A, B = workloads.random_case(rng, M, K, N, big=int(rng.choice([50, 5000])), frac=0.15)
+        LA, LB = _levels_numpy(A, b), _levels_numpy(B, b)
+        lar, lac, lbr, lbc = LA.max(1), LA.max(0), LB.max(1), LB.max(0)
+        mix = oracle.plan(A, B, b, oracle.MIX)
+        joint = oracle.plan(A, B, b, oracle.MIX_JOINT)
+        da, db = mix.dir_a, mix.dir_b
+        best = _pair_cost(lar, lac, lbr, lbc, da, db)
+        for pa, pb in pairs:
+            ca = oracle.DIR_NONE if mix.dir_a == oracle.DIR_NONE else pa
+            cb = oracle.DIR_NONE if mix.dir_b == oracle.DIR_NONE else pb
+            c = _pair_cost(lar, lac, lbr, lbc, ca, cb)
+            if c < best:
+                best, da, db = c, ca, cb
+        assert (joint.dir_a, joint.dir_b) == (da, db)
+        assert joint.ratio <= mix.ratio
+        differs += (joint.dir_a, joint.dir_b) != (mix.dir_a, mix.dir_b)
+        # the exact product whatever the directions
+        Au, Bu = oracle.unpack(joint, A, B)
+        assert np.array_equal(oracle.unpacked_gemm(joint, Au, Bu), A @ B)
+    assert differs > 0  # the two rules do part ways on some inputs
+
+
+def test_joint_mix_worked_case():
+    """Closed form, b = 5 (R = 16): 300 needs 3 digits.  A 3x4 with 300 at (0,0), B 4x1 with 300 at
+    (0,0), all else 1.  Levels: A rows 3,1,1 and columns 3,1,1,1; B rows 3,1,1,1 and column 3.
+    Per-matrix Mix: A's column side 6*3 = 18 < row side 5*4 = 20, B's row side 6*1 < column side 3*4,
+    so col/row with size 3*1*(3*3+1+1+1) = 36.  Row/row costs 5*1*6 = 30, row/col 5*3*4 = 60 and
+    col/col 3*3*6 = 54, so Joint Mix takes row/row: ratio 30/12 = 2.5 against Mix's 36/12 = 3."""
+    A = np.ones((3, 4), dtype=np.int64)
+    B = np.ones((4, 1), dtype=np.int64)
+    A[0, 0] = 300
+    B[0, 0] = 300
+    mix = oracle.plan(A, B, 5, oracle.MIX)
+    joint = oracle.plan(A, B, 5, oracle.MIX_JOINT)
+    assert (mix.dir_a, mix.dir_b) == (oracle.DIR_INNER, oracle.DIR_INNER)
+    assert mix.ratio == pytest.approx(3.0)
+    assert (joint.dir_a, joint.dir_b) == (oracle.DIR_OUTER, oracle.DIR_INNER)
+    assert joint.ratio == pytest.approx(2.5)
+    Au, Bu = oracle.unpack(joint, A, B)
+    assert np.array_equal(oracle.unpacked_gemm(joint, Au, Bu), A @ B)
+
+
 def test_mix_beats_fixed_on_channel_outliers():
     """The measured-effects table reports Mix below every fixed strategy on linear layers, where
     heavy hitters sit in channels; a channel-structured case reproduces that ordering."""
