@@ -545,7 +545,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   I.oor_lines_b_col = (int64_t)S.oor[3];
 
   int da, db;
-  if (strategy == IMQ_MIX) {
+  if (strategy == IMQ_MIX || strategy == IMQ_MIX_JOINT) {
     if (S.oor[0] == 0 && S.oor[1] == 0) {
       da = IMQ_DIR_NONE;
     } else {
@@ -565,6 +565,35 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   } else {
     da = (strategy == IMQ_ROW_ROW || strategy == IMQ_ROW_COL) ? IMQ_DIR_OUTER : IMQ_DIR_INNER;
     db = (strategy == IMQ_ROW_ROW || strategy == IMQ_COL_ROW) ? IMQ_DIR_INNER : IMQ_DIR_OUTER;
+  }
+  if (strategy == IMQ_MIX_JOINT) {
+    // the exact unpacked size M_eff * N_eff * K_eff of a direction pair, from the summary: level sums
+    // for the outer dimensions, the joint histogram of (A column level, B row level) for K_eff
+    unsigned __int128 kk_both = 0;
+    for (int x = 1; x < kLv; ++x)
+      for (int y = 1; y < kLv; ++y) kk_both += (unsigned __int128)((unsigned)(x * y)) * S.joint[x][y];
+    auto size_of = [&](int ca, int cb) {
+      const unsigned __int128 me = ca == IMQ_DIR_OUTER ? (unsigned __int128)S.sum[0] : (unsigned __int128)M;
+      const unsigned __int128 ne = cb == IMQ_DIR_OUTER ? (unsigned __int128)S.sum[3] : (unsigned __int128)N;
+      unsigned __int128 ke = (unsigned __int128)K;
+      if (ca == IMQ_DIR_INNER && cb == IMQ_DIR_INNER) ke = kk_both;
+      else if (ca == IMQ_DIR_INNER) ke = S.sum[1];
+      else if (cb == IMQ_DIR_INNER) ke = S.sum[2];
+      return me * ne * ke;
+    };
+    const int pa[4] = {IMQ_DIR_OUTER, IMQ_DIR_OUTER, IMQ_DIR_INNER, IMQ_DIR_INNER};
+    const int pb[4] = {IMQ_DIR_INNER, IMQ_DIR_OUTER, IMQ_DIR_INNER, IMQ_DIR_OUTER};
+    unsigned __int128 best = size_of(da, db);
+    const bool a_none = da == IMQ_DIR_NONE, b_none = db == IMQ_DIR_NONE;
+    for (int c = 0; c < 4; ++c) {
+      const int ca = a_none ? IMQ_DIR_NONE : pa[c], cb = b_none ? IMQ_DIR_NONE : pb[c];
+      const unsigned __int128 cost = size_of(ca, cb);
+      if (cost < best) {
+        best = cost;
+        da = ca;
+        db = cb;
+      }
+    }
   }
   I.dir_a = da;
   I.dir_b = db;

@@ -66,7 +66,14 @@ typedef enum { IMQ_PER_TENSOR = 0, IMQ_PER_ROW = 1, IMQ_PER_COL = 2 } imq_gran;
  * "row" of B = an inner index (INNER), "col" of B = an output column (OUTER).
  * READING: the page never says whether its GEMM is A*B or A*B^T; the directions are therefore named
  * by axis (OUTER/INNER) in imq_plan_info. */
-typedef enum { IMQ_MIX = 0, IMQ_ROW_ROW = 1, IMQ_ROW_COL = 2, IMQ_COL_ROW = 3, IMQ_COL_COL = 4 } imq_strategy;
+typedef enum {
+  IMQ_MIX = 0, IMQ_ROW_ROW = 1, IMQ_ROW_COL = 2, IMQ_COL_ROW = 3, IMQ_COL_COL = 4,
+  /* Joint Mix (READING of the per-matrix choice that weighs both matrices together): the direction pair
+   * of least exact unpacked size M_eff * N_eff * K_eff (the unpack ratio's numerator) over the four
+   * pairs, starting from the Mix choice and taking strict improvements in the order row/row, row/col,
+   * col/row, col/col; a matrix without out-of-range entries stays not unpacked. */
+  IMQ_MIX_JOINT = 5
+} imq_strategy;
 
 /* Direction a matrix is unpacked in.  NONE: the matrix has no out-of-range entry (Mix only). */
 typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2 } imq_dir;

@@ -92,15 +92,17 @@ def _run(imq, g, strategies=None, rows=None, check_unpack=True):
 
 def test_config_tiny(imq):
     g = workloads.tiny()[0]
-    infos = _run(imq, g, strategies=[0, 1, 2, 3, 4])
+    infos = _run(imq, g, strategies=[0, 1, 2, 3, 4, 5])
     assert infos[0]["ratio"] > 1.0
+    assert infos[5]["ratio"] <= min(i["ratio"] for i in infos.values()) + 1e-12
 
 
 def test_config_q_proj(imq):
     g = workloads.q_proj()[0]
-    infos = _run(imq, g, strategies=[0, 1, 2, 3, 4])
+    infos = _run(imq, g, strategies=[0, 1, 2, 3, 4, 5])
     assert infos[0]["dir_a"] == imq.IMQ_DIR_INNER  # column unpacking of the activations
     assert infos[0]["ratio"] <= min(i["ratio"] for i in infos.values()) + 1e-12
+    assert infos[5]["ratio"] <= infos[0]["ratio"]  # joint Mix is never worse than Mix
 
 
 def test_config_mlp(imq):
@@ -113,6 +115,15 @@ def test_config_mlp(imq):
 def test_config_attention(imq, head):
     for g in workloads.attention_head(head):
         _run(imq, g)
+
+
+@pytest.mark.parametrize("head", [0, 19])
+def test_config_attention_joint_mix(imq, head):
+    """P.V with its diagonal-ish peaks is where per-matrix choices are weakest; joint Mix is checked
+    there against the oracle and is never worse than Mix."""
+    for g in workloads.attention_head(head):
+        infos = _run(imq, g, strategies=[0, 5])
+        assert infos[5]["ratio"] <= infos[0]["ratio"]
 
 
 def test_config_wgrad(imq):

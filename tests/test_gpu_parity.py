@@ -174,7 +174,7 @@ def _run_path(imq, A, B, b, strategy, transA, transB, dtype=torch.int16, check_u
 
 
 @pytest.mark.parametrize("b", [2, 3, 5, 8])
-@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4, 5])
 @pytest.mark.parametrize("trans", [(False, False), (True, False), (False, True), (True, True)])
 def test_path_parity_int32_regime(imq, b, strategy, trans):
     rng = np.random.default_rng(1000 * b + 10 * strategy + 2 * trans[0] + trans[1])
@@ -183,13 +183,36 @@ def test_path_parity_int32_regime(imq, b, strategy, trans):
 
 
 @pytest.mark.parametrize("b", [2, 3, 4, 5, 8])
-@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4, 5])
 def test_path_parity_int64_regime(imq, b, strategy):
     rng = np.random.default_rng(77 + 10 * b + strategy)
     A, B = workloads.random_case(rng, 200, 384, 300, big=3000, frac=0.05)
     plan = _run_path(imq, A, B, b, strategy, False, True)
     if plan is not None:
         assert plan.info["acc_bits"] == 64
+
+
+def test_joint_mix_parity_where_it_differs_from_mix(imq):
+    """Joint Mix on inputs where it picks another direction pair than per-matrix Mix: the closed-form
+    worked case of the oracle pins, and random cases found by the oracle."""
+    A = np.ones((3, 4), dtype=np.int64)
+    B = np.ones((4, 1), dtype=np.int64)
+    A[0, 0] = 300
+    B[0, 0] = 300
+    plan = _run_path(imq, A, B, 5, imq.IMQ_MIX_JOINT, False, False)
+    assert (plan.info["dir_a"], plan.info["dir_b"]) == (imq.IMQ_DIR_OUTER, imq.IMQ_DIR_INNER)
+    rng = np.random.default_rng(4242)
+    found = 0
+    while found < 6:
+        M, K, N = (int(x) for x in rng.integers(1, 40, size=3))
+        b = int(rng.integers(2, 8))
+        A, B = workloads.random_case(rng, M, K, N, big=int(rng.choice([50, 5000])), frac=0.15)
+        mix, joint = oracle.plan(A, B, b, oracle.MIX), oracle.plan(A, B, b, oracle.MIX_JOINT)
+        if (mix.dir_a, mix.dir_b) == (joint.dir_a, joint.dir_b):
+            continue
+        found += 1
+        for transB in (False, True):
+            _run_path(imq, A, B, b, imq.IMQ_MIX_JOINT, False, transB)
 
 
 def test_path_parity_no_outliers_is_plain_int8(imq):
