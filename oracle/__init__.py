@@ -85,6 +85,7 @@ def _lib():
         lib.oracle_percentile_abs.argtypes = [vp, i64, f64]
         lib.oracle_percentile_abs.restype = ctypes.c_float
         lib.oracle_rtn_quantize.argtypes = [vp, i64, i64, i32, f64, i32, vp, vp, vp]
+        lib.oracle_rtn_quantize_ex.argtypes = [vp, i64, i64, i32, f64, i32, i32, vp, vp, vp]
         lib.oracle_level.argtypes = [i64, i32]
         lib.oracle_level.restype = i32
         lib.oracle_digit.argtypes = [i64, i32, i32]
@@ -130,16 +131,17 @@ def percentile_abs(v: np.ndarray, p: float) -> np.float32:
     return np.float32(_lib().oracle_percentile_abs(_ptr(v), v.size, float(p)))
 
 
-def rtn_quantize(x: np.ndarray, gran: int, p: float, beta: int):
-    """x: 2-D float32.  Returns (xint int64, delta float32, qval float32); raises OracleError."""
+def rtn_quantize(x: np.ndarray, gran: int, p: float, beta: int, clip: bool = False):
+    """x: 2-D float32.  Returns (xint int64, delta float32, qval float32); raises OracleError.  clip:
+    the clipping comparison variant (scaled values clamped to [-beta, beta] before rounding)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     rows, cols = x.shape
     ng = 1 if gran == PER_TENSOR else (rows if gran == PER_ROW else cols)
     xint = np.zeros((rows, cols), dtype=np.int64)
     delta = np.zeros(ng, dtype=np.float32)
     qval = np.zeros(ng, dtype=np.float32)
-    st = _lib().oracle_rtn_quantize(_ptr(x), rows, cols, gran, float(p), int(beta), _ptr(xint),
-                                    _ptr(delta), _ptr(qval))
+    st = _lib().oracle_rtn_quantize_ex(_ptr(x), rows, cols, gran, float(p), int(beta), int(bool(clip)),
+                                       _ptr(xint), _ptr(delta), _ptr(qval))
     if st != OK:
         raise OracleError(st, "rtn_quantize")
     return xint, delta, qval

@@ -66,6 +66,9 @@ float oracle_percentile_abs(const float *v, int64_t n, double p);
 /* rtn.c */
 int oracle_rtn_quantize(const float *x, int64_t rows, int64_t cols, int gran, double p, int beta,
                         int64_t *xint, float *delta, float *qval);
+/* The same with clip != 0: the clipping comparison variant (scaled values clamped to [-beta, beta]). */
+int oracle_rtn_quantize_ex(const float *x, int64_t rows, int64_t cols, int gran, double p, int beta, int clip,
+                           int64_t *xint, float *delta, float *qval);
 /* digits.c */
 int oracle_level(int64_t v, int b);
 int64_t oracle_digit(int64_t v, int l, int b);

@@ -118,6 +118,46 @@ def test_rtn_rank_k_maps_to_beta_and_sign_symmetry():
         assert np.array_equal(xneg, -xint) and np.array_equal(dneg, delta)
 
 
+def test_rtn_clip_exhaustive_bf16_against_exact_rounding():
+    """Clipping variant (the measured-effects table's 99.5% row): the exactly rounded fp32 product,
+    clamped to [-beta, beta] (clamping before or after rounding agree since beta is an integer)."""
+    bits = _all_finite_bf16()
+    x = oracle.bf16_bits_to_f32(bits).reshape(1, -1)
+    for beta in (15, 255):
+        xint, delta, q = oracle.rtn_quantize(x, oracle.PER_TENSOR, 0.995, beta, clip=True)
+        s = np.float32(beta) / np.float32(q[0])
+        prod32 = (x.astype(np.float64) * np.float64(s)).astype(np.float32)
+        want = np.array([max(-beta, min(beta, _rne_int(Fraction(float(v))))) for v in prod32.ravel()],
+                        dtype=np.int64)
+        assert np.array_equal(xint.ravel(), want)
+        # the scale is the unclipped one: clipping only changes the heavy hitters
+        _, d0, q0 = oracle.rtn_quantize(x, oracle.PER_TENSOR, 0.995, beta)
+        assert d0[0] == delta[0] and q0[0] == q[0]
+
+
+def test_rtn_variants_error_ordering():
+    """The comparison the measured-effects table draws, on heavy-hitter data with an exact float64
+    reference product: keeping heavy hitters (the method, p = 95 %, beta = 15) loses far less than
+    clipping them at the 99.5 % point, and the unpacked product of the method is the exact product
+    of its integers (so its only error is the rounding of RTN)."""
+    g = workloads.q_proj()[0]
+    X = oracle.as_f32(g.A.data[:96], "bf16")
+    W = oracle.as_f32(g.B.data[:, :80], "bf16")
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+
+    def err(p, beta, clip):
+        xa, da, _ = oracle.rtn_quantize(X, oracle.PER_ROW, p, beta, clip=clip)
+        wb, db, _ = oracle.rtn_quantize(W, oracle.PER_COL, p, beta, clip=clip)
+        Cf = oracle.dequant(oracle.gemm_exact(xa, wb), da, oracle.PER_ROW, db, oracle.PER_COL)
+        return np.linalg.norm(Cf - ref) / np.linalg.norm(ref)
+
+    e_method = err(0.95, 15, False)
+    e_clip = err(0.995, 15, True)
+    e_wide = err(1.0, 255, False)
+    assert e_method < 0.1 * e_clip, (e_method, e_clip)
+    assert e_method < 0.2 and e_wide < 0.2
+
+
 def test_rtn_granularities_agree_with_per_group_calls():
     rng = np.random.default_rng(14)
     X = rng.standard_normal((9, 13)).astype(np.float32)
