@@ -33,6 +33,7 @@ IMQ_MIX, IMQ_ROW_ROW, IMQ_ROW_COL, IMQ_COL_ROW, IMQ_COL_COL, IMQ_MIX_JOINT = 0, 
 IMQ_DIR_NONE, IMQ_DIR_OUTER, IMQ_DIR_INNER = 0, 1, 2
 IMQ_MAX_GROUPS = 64
 IMQ_NOALLOC_SCRATCH_BYTES = 8 << 20
+IMQ_RTN_CLIP = 1
 
 _TORCH_TO_IMQ = {torch.float32: IMQ_F32, torch.bfloat16: IMQ_BF16, torch.int16: IMQ_I16,
                  torch.int32: IMQ_I32, torch.int64: IMQ_I64}
@@ -76,6 +77,8 @@ _VP, _I32, _I64, _F64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ct
 SIGNATURES = {
     "imq_rtn_quantize": [_VP, _I32, _I64, _I64, _I64, _I32, _F64, _I32, _VP, _I32, _I64, _I32, _VP, _VP, _VP, _VP,
                          _VP],
+    "imq_rtn_quantize_ex": [_VP, _I32, _I64, _I64, _I64, _I32, _F64, _I32, _VP, _I32, _I64, _I32, _VP, _VP, _VP,
+                            _VP, ctypes.c_uint32, _VP],
     "imq_rtn_quantize_rows_noalloc": [_VP, _I32, _I64, _I64, _I64, _F64, _I32, _VP, _I32, _I64, _VP, _VP, _VP,
                                       _VP, _VP],
     "imq_plan": [_VP, _VP, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32, _VP, _VP, _VP, _VP,
@@ -144,9 +147,10 @@ Quantized = namedtuple("Quantized", "xint delta qval rowmax colmax")
 
 def imq_rtn_quantize(X: torch.Tensor, gran: int, p: float, beta: int, out_dtype=torch.int16,
                      Xint=None, delta=None, qval=None, rowmax=None, colmax=None, want_qval=True,
-                     want_max=True, trans_out=False, stream=None) -> Quantized:
+                     want_max=True, trans_out=False, clip=False, stream=None) -> Quantized:
     """RTN quantisation of a stored 2-D matrix (fp32 or bf16) per tensor / stored row / stored column.
-    trans_out writes the quantised matrix transposed (cols x rows)."""
+    trans_out writes the quantised matrix transposed (cols x rows); clip selects the clipping
+    comparison variant (imq_rtn_quantize_ex with IMQ_RTN_CLIP)."""
     rows, cols = X.shape
     dev = X.device
     if Xint is None:
@@ -160,11 +164,15 @@ def imq_rtn_quantize(X: torch.Tensor, gran: int, p: float, beta: int, out_dtype=
         rowmax = torch.empty(rows, dtype=torch.int32, device=dev)
     if colmax is None and want_max:
         colmax = torch.empty(cols, dtype=torch.int32, device=dev)
-    st = lib().imq_rtn_quantize(_ptr(X), _TORCH_TO_IMQ[X.dtype], rows, cols, _ld(X), gran, float(p), int(beta),
-                                _ptr(Xint), _TORCH_TO_IMQ[Xint.dtype], _ld(Xint), int(trans_out), _ptr(delta),
-                                _ptr(qval),
-                                _ptr(rowmax), _ptr(colmax), _stream(stream))
-    _check(st, "imq_rtn_quantize")
+    args = (_ptr(X), _TORCH_TO_IMQ[X.dtype], rows, cols, _ld(X), gran, float(p), int(beta), _ptr(Xint),
+            _TORCH_TO_IMQ[Xint.dtype], _ld(Xint), int(trans_out), _ptr(delta), _ptr(qval), _ptr(rowmax),
+            _ptr(colmax))
+    if clip:
+        st = lib().imq_rtn_quantize_ex(*args, IMQ_RTN_CLIP, _stream(stream))
+        _check(st, "imq_rtn_quantize_ex")
+    else:
+        st = lib().imq_rtn_quantize(*args, _stream(stream))
+        _check(st, "imq_rtn_quantize")
     return Quantized(Xint, delta, qval, rowmax, colmax)
 
 

@@ -94,7 +94,15 @@ imq_status imq_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t c
                             double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq, int32_t trans_out,
                             float* delta, float* qval, int32_t* rowmax, int32_t* colmax, imq_stream_t stream) {
   return imq::launch_rtn_quantize(X, xt, rows, cols, ld, g, p, beta, Xint, it, ldq, trans_out, delta, qval, rowmax,
-                                  colmax, reinterpret_cast<cudaStream_t>(stream));
+                                  colmax, 0u, reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_rtn_quantize_ex(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld, imq_gran g,
+                               double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq, int32_t trans_out,
+                               float* delta, float* qval, int32_t* rowmax, int32_t* colmax, uint32_t flags,
+                               imq_stream_t stream) {
+  return imq::launch_rtn_quantize(X, xt, rows, cols, ld, g, p, beta, Xint, it, ldq, trans_out, delta, qval, rowmax,
+                                  colmax, flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
 imq_status imq_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,

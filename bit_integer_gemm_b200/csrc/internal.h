@@ -28,7 +28,7 @@ imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int
 imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                imq_gran g, double p, int32_t beta, void* Xint, imq_dtype it,
                                int64_t ldq, int32_t trans_out, float* delta, float* qval, int32_t* rowmax,
-                               int32_t* colmax, cudaStream_t stream);
+                               int32_t* colmax, uint32_t flags, cudaStream_t stream);
 // imq_rtn_quantize_rows_noalloc: the per-row quantiser with its scratch in a fixed device array.
 imq_status launch_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                             double p, int32_t beta, void* Xint, imq_dtype it, int64_t ldq,

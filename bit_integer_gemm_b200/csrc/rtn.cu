@@ -129,9 +129,12 @@ __device__ __forceinline__ void scale_from_q(float q, float qmax, int beta, floa
 }
 
 // Quantises one value; returns |v| (0 on a range error, which is recorded).
+// clip > 0: the clipping comparison variant, the scaled value clamped to [-clip, clip] (clip = beta).
 template <bool kOut16>
-__device__ __forceinline__ uint32_t quant_one(float x, float s, void* out, int64_t idx, int32_t* status) {
-  const float y = __fmul_rn(x, s);
+__device__ __forceinline__ uint32_t quant_one(float x, float s, void* out, int64_t idx, int32_t* status,
+                                              int clip) {
+  float y = __fmul_rn(x, s);
+  if (clip) y = fminf(fmaxf(y, -(float)clip), (float)clip);
   int32_t v = 0;
   if (fabsf(y) < 2147483648.0f) {
     v = __float2int_rn(y);
@@ -271,8 +274,9 @@ __device__ __forceinline__ uint32_t select_key(const T* a, int n, unsigned long 
 
 // x * s rounded to the nearest integer, ties to even: the arithmetic of quant_one, without the store.
 template <bool kOut16>
-__device__ __forceinline__ int32_t quant_val(float x, float s, int32_t* status) {
-  const float y = __fmul_rn(x, s);
+__device__ __forceinline__ int32_t quant_val(float x, float s, int32_t* status, int clip) {
+  float y = __fmul_rn(x, s);
+  if (clip) y = fminf(fmaxf(y, -(float)clip), (float)clip);
   int32_t v = 0;
   if (fabsf(y) < 2147483648.0f) {
     v = __float2int_rn(y);
@@ -289,7 +293,7 @@ __device__ __forceinline__ int32_t quant_val(float x, float s, int32_t* status) 
 // Quantises 8 consecutive entries of a 16-byte aligned group in shared memory and stores them with
 // 16-byte stores at out[idx .. idx+7] (idx a multiple of 8, out 16-byte aligned); a[j] = |value j|.
 template <typename T, bool kOut16>
-__device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t idx, int32_t* status,
+__device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t idx, int32_t* status, int clip,
                                        uint32_t (&a)[8]) {
   // the 8 entries as 32-bit words (bf16: two per word, low half first), kept in registers
   uint32_t wd[8];
@@ -305,7 +309,7 @@ __device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const T e = sizeof(T) == 2 ? (T)((wd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) : (T)wd[j];
-    v[j] = quant_val<kOut16>(Key<T>::value(e), s, status);
+    v[j] = quant_val<kOut16>(Key<T>::value(e), s, status, clip);
     a[j] = v[j] < 0 ? (uint32_t)(-(int64_t)v[j]) : (uint32_t)v[j];
   }
   if (kOut16) {
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
     void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
     int32_t* __restrict__ rowmax, int32_t* __restrict__ part, const TensorState* __restrict__ ts, int vec,
-    int nwarps, int32_t* status) {
+    int nwarps, int32_t* status, int clip) {
   extern __shared__ __align__(16) unsigned char dsm[];
   const int64_t row_bytes = (cols * (int64_t)sizeof(T) + 15) / 16 * 16;
   uint32_t* cmax = reinterpret_cast<uint32_t*>(dsm);                  // [cols]
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
         // 8 consecutive entries per lane and step: 16-byte shared loads and global stores
         for (int g = lane; g < n / 8; g += 32) {
           uint32_t a[8];
-          quant8<T, kOut16>(row + g * 8, s, Xint, r * ldq + g * 8, status, a);
+          quant8<T, kOut16>(row + g * 8, s, Xint, r * ldq + g * 8, status, clip, a);
 #pragma unroll
           for (int j = 0; j < 8; ++j) rmx = max(rmx, a[j]);
           if (part) max8_shared(cmax + g * 8, a);
@@ -399,7 +403,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
       } else {
         for (int c = lane; c < n; c += 32) {
           const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint,
-                                               trans_out ? c * ldq + r : r * ldq + c, status);
+                                               trans_out ? c * ldq + r : r * ldq + c, status, clip);
           rmx = max(rmx, a);
           if (part && a > cmax[c]) atomicMax(&cmax[c], a);
         }
@@ -428,7 +432,7 @@ template <typename T, int CW, bool kOut16>
 __global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
     void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
-    int32_t* __restrict__ part, int32_t* __restrict__ colmax, int vec, int32_t* status) {
+    int32_t* __restrict__ part, int32_t* __restrict__ colmax, int vec, int32_t* status, int clip) {
   extern __shared__ __align__(16) unsigned char dsm[];
   const int n = (int)rows;
   const int colstride = (n + 7) / 8 * 8;  // elements; keeps every column 16-byte aligned
@@ -477,7 +481,7 @@ __global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
     if (!bad && vq) {
       for (int g = lane; g < n / 8; g += 32) {
         uint32_t a[8];
-        quant8<T, kOut16>(col + g * 8, s, Xint, c * ldq + g * 8, status, a);
+        quant8<T, kOut16>(col + g * 8, s, Xint, c * ldq + g * 8, status, clip, a);
 #pragma unroll
         for (int j = 0; j < 8; ++j) cmx = max(cmx, a[j]);
         if (part) max8_shared(rmax + g * 8, a);
@@ -485,7 +489,7 @@ __global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
     } else if (!bad) {
       for (int r = lane; r < n; r += 32) {
         const uint32_t a = quant_one<kOut16>(Key<T>::value(col[r]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
-                                             status);
+                                             status, clip);
         cmx = max(cmx, a);
         if (part && a > rmax[r]) atomicMax(&rmax[r], a);
       }
@@ -508,7 +512,7 @@ template <typename T, bool kOut16>
 __global__ void __launch_bounds__(kThreads) k_rtn_cols(
     const T* __restrict__ X, int64_t rows, int64_t cols, int64_t ld, unsigned long long krank, int beta,
     void* __restrict__ Xint, int64_t ldq, int trans_out, float* __restrict__ delta, float* __restrict__ qval,
-    int32_t* __restrict__ part, int32_t* __restrict__ colmax, int32_t* status) {
+    int32_t* __restrict__ part, int32_t* __restrict__ colmax, int32_t* status, int clip) {
   constexpr int CW = kColsPerCta;
   int32_t* prow = part ? part + (int64_t)blockIdx.x * rows : nullptr;  // this CTA's row maxima
   constexpr int RS = kThreads / CW;  // rows per sweep
@@ -579,7 +583,8 @@ __global__ void __launch_bounds__(kThreads) k_rtn_cols(
     const int64_t r = r0 + rsub;
     uint32_t a = 0;
     if (cval && r < rows) {
-      a = quant_one<kOut16>(Key<T>::value(X[r * ld + c]), s, Xint, trans_out ? c * ldq + r : r * ldq + c, status);
+      a = quant_one<kOut16>(Key<T>::value(X[r * ld + c]), s, Xint, trans_out ? c * ldq + r : r * ldq + c, status,
+                            clip);
       cmx = max(cmx, a);
     }
     // max over the CW columns of this row (CW consecutive lanes)
@@ -699,7 +704,7 @@ int64_t nearest_rank(int64_t n, double p) {
 template <typename T, int CW, bool kOut16>
 imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, unsigned long long k, int32_t beta,
                            void* Xint, int64_t ldq, int trans_out, float* delta, float* qval, int32_t* rowmax,
-                           int32_t* colmax, DeviceState* ds, cudaStream_t st) {
+                           int32_t* colmax, int clip, DeviceState* ds, cudaStream_t st) {
   const size_t colstride = (size_t)(rows + 7) / 8 * 8;
   const size_t smem = (size_t)CW * colstride * sizeof(T) + (size_t)rows * 4;
   const bool vec = (ld % (16 / (int64_t)sizeof(T)) == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
@@ -713,7 +718,7 @@ imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, u
   auto kern = k_rtn_cols_staged<T, CW, kOut16>;
   IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   kern<<<(unsigned)grid, CW * 32, smem, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, part,
-                                              colmax, vec ? 1 : 0, ds->status);
+                                              colmax, vec ? 1 : 0, ds->status, clip);
   if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
   return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
 }
@@ -721,7 +726,7 @@ imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, u
 template <typename T, bool kOut16>
 imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, double p,
                int32_t beta, void* Xint, int64_t ldq, int trans_out, float* delta, float* qval, int32_t* rowmax,
-               int32_t* colmax, DeviceState* ds, cudaStream_t st) {
+               int32_t* colmax, int clip, DeviceState* ds, cudaStream_t st) {
   const int sms = ds->num_sms;
   if (g == IMQ_PER_COL) {
     const unsigned long long k = (unsigned long long)nearest_rank(rows, p);
@@ -730,13 +735,13 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
     const size_t colb = (size_t)(rows + 7) / 8 * 8 * sizeof(T);
     if (16 * colb + (size_t)rows * 4 <= kSlab)
       return run_cols_staged<T, 16, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
-                                            colmax, ds, st);
+                                            colmax, clip, ds, st);
     if (8 * colb + (size_t)rows * 4 <= kSlab)
       return run_cols_staged<T, 8, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
-                                           colmax, ds, st);
+                                           colmax, clip, ds, st);
     if (4 * colb + (size_t)rows * 4 <= kSlab)
       return run_cols_staged<T, 4, kOut16>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, rowmax,
-                                           colmax, ds, st);
+                                           colmax, clip, ds, st);
     const int64_t grid = (cols + kColsPerCta - 1) / kColsPerCta;
     int32_t* part = nullptr;
     StreamScratch sp;
@@ -745,7 +750,7 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
       part = static_cast<int32_t*>(sp.p);
     }
     k_rtn_cols<T, kOut16><<<(unsigned)grid, kThreads, 0, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out,
-                                                               delta, qval, part, colmax, ds->status);
+                                                               delta, qval, part, colmax, ds->status, clip);
     if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
     return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
   }
@@ -784,13 +789,13 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
     auto kern = k_rtn_rows<T, false, kOut16>;
     IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, 0ull, beta, Xint, ldq, trans_out, delta, qval,
-                                                 rowmax, part, ts, vec, nwarps, ds->status);
+                                                 rowmax, part, ts, vec, nwarps, ds->status, clip);
   } else {
     auto kern = k_rtn_rows<T, true, kOut16>;
     IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta,
                                                  Xint, ldq, trans_out, delta, qval, rowmax, part, nullptr, vec, nwarps,
-                                                 ds->status);
+                                                 ds->status, clip);
   }
   if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
   return colmax ? launch_reduce_max(part, grid, cols, colmax, st) : IMQ_OK;
@@ -801,8 +806,10 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
 imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
                                imq_gran g, double p, int32_t beta, void* Xint, imq_dtype it,
                                int64_t ldq, int32_t trans_out, float* delta, float* qval, int32_t* rowmax,
-                               int32_t* colmax, cudaStream_t st) {
+                               int32_t* colmax, uint32_t flags, cudaStream_t st) {
   if (trans_out != 0 && trans_out != 1) return IMQ_ERR_ARG;
+  if (flags & ~(uint32_t)IMQ_RTN_CLIP) return IMQ_ERR_ARG;
+  const int clip = (flags & IMQ_RTN_CLIP) ? beta : 0;
   if (rows < 0 || cols < 0 || ld < cols || ldq < (trans_out ? rows : cols) || !(p > 0.0 && p <= 1.0) || beta < 1 ||
       beta > (1 << 24))
     return IMQ_ERR_ARG;
@@ -829,12 +836,12 @@ imq_status launch_rtn_quantize(const void* X, imq_dtype xt, int64_t rows, int64_
   const bool o16 = it == IMQ_I16;
   if (xt == IMQ_BF16) {
     const uint16_t* x = static_cast<const uint16_t*>(X);
-    return o16 ? run<uint16_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st)
-               : run<uint16_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st);
+    return o16 ? run<uint16_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, clip, ds, st)
+               : run<uint16_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, clip, ds, st);
   }
   const uint32_t* x = static_cast<const uint32_t*>(X);
-  return o16 ? run<uint32_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st)
-             : run<uint32_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, ds, st);
+  return o16 ? run<uint32_t, true>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, clip, ds, st)
+             : run<uint32_t, false>(x, rows, cols, ld, g, p, beta, Xint, ldq, trans_out, delta, qval, rowmax, colmax, clip, ds, st);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -905,7 +912,7 @@ imq_status run_rows_noalloc(const T* X, int64_t rows, int64_t cols, int64_t ld, 
   IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta,
                                                Xint, ldq, 0, delta, qval, rowmax, part, nullptr, vec, nwarps,
-                                               ds->status);
+                                               ds->status, 0);
   if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
   return colmax ? launch_reduce_max(part, grid, cols, colmax, st) : IMQ_OK;
 }

@@ -118,6 +118,22 @@ imq_status imq_rtn_quantize(const void *X, imq_dtype xt, int64_t rows, int64_t c
                             imq_stream_t stream);
 
 /*
+ * imq_rtn_quantize_ex -- imq_rtn_quantize with option flags (0 gives imq_rtn_quantize exactly).
+ *   IMQ_RTN_CLIP  the clipping comparison variant of the measured-effects table (its 99.5% row, with
+ *                 p = 0.995): the scaled value x * s_g is clamped to [-beta, beta] before rounding
+ *                 (READING; equal to clamping the rounded value, beta being an integer), so no entry
+ *                 leaves +-beta and nothing is left to unpack when beta <= R - 1.  The scale and Delta
+ *                 are those of the unclipped rule.  The method itself keeps heavy hitters: flags = 0.
+ * Errors: those of imq_rtn_quantize; IMQ_ERR_ARG for an unknown flag.
+ */
+#define IMQ_RTN_CLIP 1u
+imq_status imq_rtn_quantize_ex(const void *X, imq_dtype xt, int64_t rows, int64_t cols, int64_t ld,
+                               imq_gran g, double p, int32_t beta,
+                               void *Xint, imq_dtype it, int64_t ldq, int32_t trans_out,
+                               float *delta, float *qval, int32_t *rowmax, int32_t *colmax,
+                               uint32_t flags, imq_stream_t stream);
+
+/*
  * imq_rtn_quantize_rows_noalloc -- imq_rtn_quantize with g = IMQ_PER_ROW and trans_out = 0 (the
  * per-token quantisation of an activation), with the same arguments otherwise and the same results,
  * but it allocates no device memory.  The IM-Unpack page has no counterpart to this call: it is an

@@ -129,3 +129,37 @@ def test_config_attention_joint_mix(imq, head):
 def test_config_wgrad(imq):
     for g in workloads.wgrad():
         _run(imq, g, check_unpack=(g.b == 8))
+
+
+def test_rtn_variants_quantisation_error_q_proj(imq):
+    """The RTN comparison of the measured-effects table on the q_proj-shaped workload (512 of its 2048
+    rows), through the whole library path, against the float64 product of the unquantised inputs:
+    heavy hitters kept (the method, p = 95 %, beta = 15), clipped at the 99.5 % point (beta = 15) and
+    widened (p = 100 %, beta = 255).  Each variant's Cf also matches the oracle's exact dequantised
+    product."""
+    g = workloads.q_proj()[0]
+    rows = np.arange(0, 2048, 4)
+    Xs = workloads.Stored("X", np.ascontiguousarray(g.A.data[rows]), g.A.dtype)
+    X = to_device(Xs)
+    W = to_device(g.B)
+    Xf, Wf = oracle.as_f32(Xs.data, Xs.dtype), oracle.as_f32(g.B.data, g.B.dtype)
+    ref = Xf.astype(np.float64) @ Wf.astype(np.float64)
+    errs = {}
+    for name, p, beta, clip in (("method", 0.95, 15, False), ("clip", 0.995, 15, True), ("wide", 1.0, 255, False)):
+        qa = imq.imq_rtn_quantize(X, imq.IMQ_PER_ROW, p, beta, clip=clip)
+        qb = imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, p, beta, clip=clip)
+        plan = imq.imq_plan(qa.xint, qb.xint, g.b, imq.IMQ_MIX, maxes=(qa.rowmax, qa.colmax, qb.rowmax, qb.colmax))
+        Au, Bu = imq.imq_unpack(plan, qa.xint, qb.xint)
+        C, Cf = imq.imq_gemm_unpacked(plan, Au, Bu, qa.delta, imq.IMQ_PER_ROW, qb.delta, imq.IMQ_PER_COL)
+        torch.cuda.synchronize()
+        assert imq.imq_device_status() == imq.IMQ_OK
+        xa, da, _ = oracle.rtn_quantize(Xf, oracle.PER_ROW, p, beta, clip=clip)
+        wb, db, _ = oracle.rtn_quantize(Wf, oracle.PER_COL, p, beta, clip=clip)
+        want = oracle.gemm_exact(xa, wb)
+        assert np.array_equal(C.cpu().numpy().astype(np.int64), want), name
+        assert_f32_close(Cf.cpu().numpy(), oracle.dequant(want, da, oracle.PER_ROW, db, oracle.PER_COL))
+        if clip:
+            assert plan.info["ratio"] == 1.0  # nothing leaves +-15 = R - 1 at b = 5
+        errs[name] = float(np.linalg.norm(Cf.cpu().numpy().astype(np.float64) - ref) / np.linalg.norm(ref))
+    assert errs["method"] < 0.1 * errs["clip"], errs
+    assert errs["method"] < 0.1 and errs["wide"] < 0.2, errs

@@ -60,6 +60,39 @@ def test_quantize_parity(imq, dtype, gran, shape, p, beta):
         assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0))
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("gran", [oracle.PER_TENSOR, oracle.PER_ROW, oracle.PER_COL])
+@pytest.mark.parametrize("shape", [(3, 5), (37, 129), (257, 1000), (1000, 64), (20000, 8)])
+@pytest.mark.parametrize("p,beta", [(0.995, 15), (0.9, 255)])
+@pytest.mark.parametrize("trans_out", [False, True])
+def test_quantize_clip_parity(imq, dtype, gran, shape, p, beta, trans_out):
+    """The clipping comparison variant (imq_rtn_quantize_ex, IMQ_RTN_CLIP) on every quantiser path:
+    per tensor, per row, per column staged and streamed (20000-row columns), plain and transposed out."""
+    rng = np.random.default_rng(zlib.crc32(repr(("clip", dtype, gran, shape, p, trans_out)).encode()))
+    x = _matrix(rng, shape)
+    st = workloads.Stored("x", workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x, dtype)
+    want_i, want_d, want_q = oracle.rtn_quantize(oracle.as_f32(st.data, dtype), gran, p, beta, clip=True)
+    assert np.abs(want_i).max() <= beta
+    r = imq.imq_rtn_quantize(to_device(st), gran, p, beta, trans_out=trans_out, clip=True)
+    torch.cuda.synchronize()
+    assert imq.imq_device_status() == imq.IMQ_OK
+    got = r.xint.cpu().numpy().astype(np.int64)
+    assert np.array_equal(got.T if trans_out else got, want_i)
+    assert np.array_equal(r.delta.cpu().numpy().view(np.uint32), want_d.view(np.uint32))
+    assert np.array_equal(r.qval.cpu().numpy().view(np.uint32), want_q.view(np.uint32))
+    assert np.array_equal(r.rowmax.cpu().numpy(), np.abs(want_i).max(axis=1))
+    assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0))
+
+
+def test_quantize_ex_rejects_unknown_flags(imq):
+    X = torch.ones((4, 8), device="cuda")
+    Xint = torch.empty((4, 8), dtype=torch.int16, device="cuda")
+    d = torch.empty(4, device="cuda")
+    st = imq.lib().imq_rtn_quantize_ex(imq._ptr(X), imq.IMQ_F32, 4, 8, 8, imq.IMQ_PER_ROW, 0.95, 15, imq._ptr(Xint),
+                                       imq.IMQ_I16, 8, 0, imq._ptr(d), None, None, None, 2, imq._stream(None))
+    assert st == imq.IMQ_ERR_ARG
+
+
 @pytest.mark.parametrize("gran", [oracle.PER_TENSOR, oracle.PER_ROW, oracle.PER_COL])
 @pytest.mark.parametrize("shape", [(5, 3), (300, 130), (4096, 96), (1000, 17)])
 def test_quantize_transposed_output(imq, gran, shape):
