@@ -12,7 +12,8 @@ is timed with CUDA events on its stream for the roofline.  With --gpus N > 1 eve
 replica (the path has no data exchange); time is the max over ranks.
 
 --impl reference times the CPU oracle (the reference arm of this build) on a bounded sample of the same
-workload on the host cores.
+workload on the host cores.  --workload training_triple times instead the forward, input-gradient and
+weight-gradient GEMMs of one linear layer with per-tensor RTN (one GPU; no end-to-end or CPU arm).
 """
 from __future__ import annotations
 
@@ -213,6 +214,126 @@ class Path:
         outer = int(I["dir_a"] == imq.IMQ_DIR_OUTER) + int(I["dir_b"] == imq.IMQ_DIR_OUTER)
         self.launches = 2 + 1 + (1 if I["K_unp"] > 0 else 0) + outer + 2 + outer + 1
         plan.destroy()
+
+
+class GemmPath:
+    """One pass of the path for one workloads.Gemm (stored operands with their quantisation groups and
+    transposes) on the current device: RTN of A and B, plan with the quantisers' maxima over logical
+    lines, unpack into a workspace, GEMM with fold-back and dequantisation."""
+
+    def __init__(self, imq, torch, g, A, B):
+        self.imq, self.torch, self.g, self.A, self.B = imq, torch, g, A, B
+        t, dev = torch, A.device
+        self.Ai = t.empty(tuple(A.shape), dtype=t.int16, device=dev)
+        self.Bi = t.empty(tuple(B.shape), dtype=t.int16, device=dev)
+        ng = lambda gran, shp: 1 if gran == imq.IMQ_PER_TENSOR else (shp[0] if gran == imq.IMQ_PER_ROW else shp[1])
+        self.dA = t.empty(ng(g.qa, A.shape), dtype=t.float32, device=dev)
+        self.dB = t.empty(ng(g.qb, B.shape), dtype=t.float32, device=dev)
+        self.mA = [t.empty(n, dtype=t.int32, device=dev) for n in A.shape]  # stored rows, stored columns
+        self.mB = [t.empty(n, dtype=t.int32, device=dev) for n in B.shape]
+        self.C = None
+        self.Cf = t.empty((g.M, g.N), dtype=t.float32, device=dev)
+        self.ws = None
+        self.info = None
+
+    def step(self, gemm_events=None):
+        imq, g = self.imq, self.g
+        imq.imq_rtn_quantize(self.A, g.qa, g.p, g.beta, Xint=self.Ai, delta=self.dA, want_qval=False,
+                             rowmax=self.mA[0], colmax=self.mA[1])
+        imq.imq_rtn_quantize(self.B, g.qb, g.p, g.beta, Xint=self.Bi, delta=self.dB, want_qval=False,
+                             rowmax=self.mB[0], colmax=self.mB[1])
+        # maxima over LOGICAL lines: a transposed operand's stored rows are its logical columns
+        a_row, a_col = (self.mA[1], self.mA[0]) if g.transA else (self.mA[0], self.mA[1])
+        b_row, b_col = (self.mB[1], self.mB[0]) if g.transB else (self.mB[0], self.mB[1])
+        plan = imq.imq_plan(self.Ai, self.Bi, g.b, imq.IMQ_MIX, g.transA, g.transB,
+                            maxes=(a_row, a_col, b_row, b_col))
+        I = plan.info
+        need = I["workspace_bytes"]
+        if self.ws is None or self.ws.numel() < need + 1024:
+            self.ws = self.torch.empty(need + 1024, dtype=self.torch.int8, device=self.A.device)
+        if self.C is None or (self.C.dtype == self.torch.int32) != (I["acc_bits"] == 32):
+            self.C = self.torch.empty((g.M, g.N), device=self.A.device,
+                                      dtype=self.torch.int32 if I["acc_bits"] == 32 else self.torch.int64)
+        na = I["M_unp"] * I["K_unp"]
+        a_off = (-self.ws.data_ptr()) % 1024
+        b_off = a_off + (na + 1023) // 1024 * 1024
+        Au = self.ws[a_off:a_off + na].view(I["M_unp"], I["K_unp"])
+        Bu = self.ws[b_off:b_off + I["N_unp"] * I["K_unp"]].view(I["N_unp"], I["K_unp"])
+        imq.imq_unpack(plan, self.Ai, self.Bi, A_unp=Au, B_unp_t=Bu)
+        if gemm_events is not None:
+            gemm_events[0].record()
+        imq.imq_gemm_unpacked(plan, Au, Bu, self.dA, g.gA, self.dB, g.gB, C=self.C, Cf=self.Cf)
+        if gemm_events is not None:
+            gemm_events[1].record()
+        self.info = I
+        plan.destroy()
+
+
+def run_triple(args):
+    """--workload training_triple: one step is the forward, input-gradient and weight-gradient GEMMs of
+    one linear layer (X 16384 x 512, W 512 x 2048, dY 16384 x 2048), each with per-tensor RTN."""
+    import torch
+
+    import bit_integer_gemm_b200 as imq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    imq.lib()
+    gems = workloads.training_triple()
+    dev_of = {}
+    for g in gems:
+        for st in (g.A, g.B):
+            if st.name not in dev_of:
+                dev_of[st.name] = torch.from_numpy(st.data.view(np.int16)).to(dev).view(torch.bfloat16)
+    paths = [GemmPath(imq, torch, g, dev_of[g.A.name], dev_of[g.B.name]) for g in gems]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        for pth in paths:
+            pth.step()
+    torch.cuda.synchronize()
+    if imq.imq_device_status() != imq.IMQ_OK:
+        raise RuntimeError("device status not OK after warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    gev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in paths]
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with Clocks(dev) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record()
+            for pth, ev in zip(paths, gev[k]):
+                pth.step(ev)
+            ends[k].record()
+        torch.cuda.synchronize()
+    total_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    gemm_ms = [sum(a.elapsed_time(b) for a, b in gev[k][i:i + 1]) for k in range(args.steps) for i in range(3)]
+    ops = sum(2.0 * g.M * g.N * g.K for g in gems)
+    value = throughput(ops, 1, args.steps, total_ms)
+    exec_ops = sum(2.0 * p.info["M_unp"] * p.info["N_unp"] * p.info["K_unp"] for p in paths)
+    gemm_total_ms = sum(gemm_ms) / args.steps
+    bf16_burst, _, _, src = _peaks()
+    int8_peak = 2.0 * bf16_burst
+    achieved = exec_ops / (gemm_total_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic (seeded, bf16)",
+        "config": {"workload": "training triple of one linear layer: forward X.W, dgrad dY.W^T, wgrad dY^T.X "
+                               "(X 16384x512, W 512x2048, dY 16384x2048 bf16), per-tensor RTN p=0.95 beta=31, "
+                               "b=5, Mix",
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "gemms": [{"name": g.name, "M": g.M, "K": g.K, "N": g.N, "ratio": round(p.info["ratio"], 4),
+                              "dir_a": p.info["dir_a"], "dir_b": p.info["dir_b"], "M_unp": p.info["M_unp"],
+                              "N_unp": p.info["N_unp"], "K_unp": p.info["K_unp"],
+                              "gemm_ms": round(sum(gemm_ms[i::3]) / args.steps, 4)}
+                             for i, (g, p) in enumerate(zip(gems, paths))]},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(int8_peak, 1), "unit": "TOPS",
+                     "frac": round(achieved / int8_peak, 4), "traffic": None,
+                     "kernel": "k_gemm, the three launches of a step together", "peak_source": f"{src} bf16 burst x2"},
+        "e2e": None,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_ours(args):
@@ -457,11 +578,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--workload", choices=["q_proj", "training_triple"], default="q_proj",
+                    help="q_proj: the headline step (default); training_triple: the three GEMMs of one "
+                         "quantised-training step of a linear layer (one GPU, no end-to-end or CPU arms)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "training_triple":
+        run_triple(args)
     else:
         run_ours(args)
 

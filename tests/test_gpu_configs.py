@@ -131,6 +131,15 @@ def test_config_wgrad(imq):
         _run(imq, g, check_unpack=(g.b == 8))
 
 
+@pytest.mark.parametrize("b", [4, 5])
+def test_config_training_triple(imq, b):
+    """Forward, input gradient and weight gradient of one linear layer, each with per-tensor RTN, through
+    the library with the stored matrices of one training step (transposes instead of copies)."""
+    for g in workloads.training_triple(b):
+        infos = _run(imq, g, check_unpack=(g.name != "train_dgrad"))
+        assert infos[0]["M"] == g.M and infos[0]["N"] == g.N and infos[0]["K"] == g.K
+
+
 def test_rtn_variants_quantisation_error_q_proj(imq):
     """The RTN comparison of the measured-effects table on the q_proj-shaped workload (512 of its 2048
     rows), through the whole library path, against the float64 product of the unquantised inputs:

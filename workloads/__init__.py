@@ -197,7 +197,23 @@ def wgrad() -> list:
     return gem
 
 
-CONFIGS = {"tiny": tiny, "q_proj": q_proj, "mlp": mlp, "attention": attention, "wgrad": wgrad}
+def training_triple(b: int = 5) -> list:
+    """The three GEMMs of one quantised-training step of a linear layer Y = X W (X 16384 x 512, W 512 x
+    2048, the weight-gradient layer's shapes): forward X.W, input gradient dY.W^T (W as stored, transB)
+    and weight gradient dY^T.X (dY as stored, transA), each operand quantised per tensor with p = 0.95,
+    beta = 31.  dY and X are the weight-gradient workload's (seed 4); W, which that workload lacks, is
+    drawn like the projection weights (N(0, 0.02), 0.05 % of entries x30) from seed 5."""
+    w = wgrad()[0]
+    dY, X = w.A, w.B
+    rng = np.random.default_rng(5)
+    W = _bf("W", _scatter_scale(rng, _normal(rng, (512, 2048), 0.02), 0.0005, 30))
+    mk = lambda n, a, bb, ta, tb: Gemm(n, a, bb, ta, tb, PER_TENSOR, PER_TENSOR, 0.95, 31, b, [MIX])
+    return [mk("train_forward", X, W, False, False), mk("train_dgrad", dY, W, False, True),
+            mk("train_wgrad", dY, X, True, False)]
+
+
+CONFIGS = {"tiny": tiny, "q_proj": q_proj, "mlp": mlp, "attention": attention, "wgrad": wgrad,
+           "training_triple": training_triple}
 
 
 def random_case(rng, M, K, N, big=5000, frac=0.1):
