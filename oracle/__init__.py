@@ -28,8 +28,8 @@ _SO = os.path.join(_HERE, "liboracle.so")
 _SRCS = ["percentile.c", "rtn.c", "digits.c", "plan.c", "unpack.c", "gemm.c", "dequant.c"]
 
 PER_TENSOR, PER_ROW, PER_COL = 0, 1, 2
-MIX, ROW_ROW, ROW_COL, COL_ROW, COL_COL, MIX_JOINT = 0, 1, 2, 3, 4, 5
-DIR_NONE, DIR_OUTER, DIR_INNER = 0, 1, 2
+MIX, ROW_ROW, ROW_COL, COL_ROW, COL_COL, MIX_JOINT, HYBRID = 0, 1, 2, 3, 4, 5, 6
+DIR_NONE, DIR_OUTER, DIR_INNER, DIR_BOTH = 0, 1, 2, 3
 OK, ERR_ARG, ERR_NONFINITE, ERR_RANGE = 0, 1, 2, 3
 MAX_GROUPS = 64
 
@@ -95,7 +95,7 @@ def _lib():
         lib.oracle_plan.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp,
                                     ctypes.POINTER(_Plan)]
         lib.oracle_plan_maps.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 11
-        lib.oracle_unpack.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 11
+        lib.oracle_unpack.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 13
         lib.oracle_gemm_i64.argtypes = [vp, vp, i64, i64, i64, vp, i32]
         lib.oracle_gemm_i64.restype = None
         lib.oracle_unpacked_gemm.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 7
@@ -189,7 +189,10 @@ class Plan:
     lmax: tuple
     suml: tuple
     oor_lines: tuple
-    levels: dict = field(default_factory=dict)  # a_row, a_col, b_row, b_col (int32)
+    # a_row, a_col, b_row, b_col (int32): line levels; under HYBRID the levels each line carries in the
+    # unpacked GEMM (1 for a row of A or column of B that is not unpacked OUTER, the inner levels taken
+    # over the lines that are not)
+    levels: dict = field(default_factory=dict)
     maps: dict = field(default_factory=dict)    # tK, lAk, lBk, srcA, lvlA, srcB, lvlB (int32)
     _raw: object = None
 
@@ -240,6 +243,7 @@ def unpack(pl: Plan, A: np.ndarray, B: np.ndarray):
     mp = pl.maps
     st = _lib().oracle_unpack(ctypes.byref(pl._raw), *[_ptr(mp[k]) for k in
                               ("tK", "lAk", "lBk", "srcA", "lvlA", "srcB", "lvlB")],
+                              _ptr(pl.levels["a_row"]), _ptr(pl.levels["b_col"]),
                               _ptr(A), _ptr(B), _ptr(Au), _ptr(Bu))
     if st != OK:
         raise OracleError(st, "unpack")

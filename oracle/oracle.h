@@ -33,10 +33,14 @@
 /* Joint Mix: the (A, B) direction pair of least exact unpacked cost M_eff * N_eff * K_eff over the four
  * pairs (a reading of the page's per-matrix choice; see oracle_plan). */
 #define OR_MIX_JOINT 5
+/* Hybrid ("unpack both"): per matrix, the outer lines with at least tau out-of-range entries unpacked
+ * OUTER and the rest INNER, tau of least unpacked size (a reading; see oracle_plan). */
+#define OR_HYBRID 6
 
 #define OR_DIR_NONE 0
 #define OR_DIR_OUTER 1
 #define OR_DIR_INNER 2
+#define OR_DIR_BOTH 3 /* OR_DIR_OUTER | OR_DIR_INNER: the hybrid's two parts */
 
 #define OR_MAX_GROUPS 64
 #define OR_INNER_PAD 128
@@ -83,8 +87,8 @@ int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t 
 /* unpack.c */
 int oracle_unpack(const oracle_plan_t *pl, const int32_t *tK, const int32_t *lAk,
                   const int32_t *lBk, const int32_t *srcA, const int32_t *lvlA,
-                  const int32_t *srcB, const int32_t *lvlB, const int64_t *A, const int64_t *B,
-                  int8_t *Aunp, int8_t *Bunp_t);
+                  const int32_t *srcB, const int32_t *lvlB, const int32_t *LrA, const int32_t *LcB,
+                  const int64_t *A, const int64_t *B, int8_t *Aunp, int8_t *Bunp_t);
 /* gemm.c */
 void oracle_gemm_i64(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N,
                      int64_t *C, int nthreads);

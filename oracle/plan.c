@@ -15,6 +15,12 @@
  *   Mix: per matrix the smaller factor; tie -> fewer lines holding outliers; tie -> row unpacking;
  *        a matrix without any out-of-range entry is not unpacked.
  *   unpack ratio = M_eff * N_eff * K_eff / (M * N * K): executed multiply-adds over original ones.
+ *   Hybrid ("unpack both", for matrices whose heavy hitters sit in some rows AND some columns): per
+ *        matrix, the outer lines (rows of A, columns of B) holding at least tau out-of-range entries are
+ *        unpacked OUTER with all their digits, the remaining lines INNER, the inner levels taken over
+ *        those remaining lines only; tau is the threshold of least M_eff * K_eff (A) or N_eff * K_eff (B),
+ *        the smallest such tau on a tie; the direction is then OUTER, INNER or both (OR_DIR_BOTH).  The
+ *        level vectors the plan returns are then the levels each line carries in the unpacked GEMM.
  *   layout: inner pairs (t, lA, lB) ordered by e = lA + lB, then lA, then t, each exponent group padded
  *   with zeros to OR_INNER_PAD; OUTER lines sorted by level (stable), floor(G / L) source lines per
  *   group of G unpacked lines (G = OR_A_GROUP for rows of A, OR_B_GROUP for columns of B), the L lines
@@ -26,10 +32,69 @@
 
 static int64_t iabs64(int64_t v) { return v < 0 ? -v : v; }
 
+/* The hybrid choice for one matrix seen as n_out outer lines of n_in inner entries, entry (o, t) at
+ * X[o * s_out + t * s_in].  On entry Lo holds the outer lines' levels; on exit Lo and Li hold the levels
+ * each line carries: Lo[o] unchanged for a line unpacked OUTER (its out-of-range count >= tau), else 1;
+ * Li[t] the largest level of entry t over the lines that are not (1 when there is none). */
+static int hybrid_choose(const int64_t *X, int64_t n_out, int64_t n_in, int64_t s_out, int64_t s_in, int b,
+                         int32_t *Lo, int32_t *Li) {
+  int8_t *lev = malloc((size_t)(n_out * n_in > 0 ? n_out * n_in : 1));
+  int64_t *cnt = calloc((size_t)(n_out > 0 ? n_out : 1), sizeof(int64_t));
+  char *present = calloc((size_t)(n_in + 2), 1);
+  if (!lev || !cnt || !present) {
+    free(lev);
+    free(cnt);
+    free(present);
+    return OR_ERR_ARG;
+  }
+  int64_t cmax = 0;
+  for (int64_t o = 0; o < n_out; ++o) {
+    for (int64_t t = 0; t < n_in; ++t) {
+      lev[o * n_in + t] = (int8_t)oracle_level(X[o * s_out + t * s_in], b);
+      if (lev[o * n_in + t] > 1) cnt[o] += 1;
+    }
+    present[cnt[o]] = 1;
+    if (cnt[o] > cmax) cmax = cnt[o];
+  }
+  /* every threshold at which the set of OUTER lines changes, and one above all counts (no OUTER line) */
+  int64_t best_tau = 1;
+  unsigned __int128 best = 0;
+  int first = 1;
+  for (int64_t tau = 1; tau <= cmax + 1; ++tau) {
+    if (!(tau == cmax + 1 || present[tau])) continue;
+    unsigned __int128 me = 0, ke = 0;
+    for (int64_t o = 0; o < n_out; ++o) me += (unsigned)(cnt[o] >= tau ? Lo[o] : 1);
+    for (int64_t t = 0; t < n_in; ++t) {
+      int li = 1;
+      for (int64_t o = 0; o < n_out; ++o)
+        if (cnt[o] < tau && lev[o * n_in + t] > li) li = lev[o * n_in + t];
+      ke += (unsigned)li;
+    }
+    const unsigned __int128 cost = me * ke;
+    if (first || cost < best) {
+      best = cost;
+      best_tau = tau;
+      first = 0;
+    }
+  }
+  for (int64_t t = 0; t < n_in; ++t) {
+    int li = 1;
+    for (int64_t o = 0; o < n_out; ++o)
+      if (cnt[o] < best_tau && lev[o * n_in + t] > li) li = lev[o * n_in + t];
+    Li[t] = li;
+  }
+  for (int64_t o = 0; o < n_out; ++o)
+    if (cnt[o] < best_tau) Lo[o] = 1;
+  free(lev);
+  free(cnt);
+  free(present);
+  return OR_OK;
+}
+
 int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N, int b,
                 int strategy, int32_t *LrA, int32_t *LcA, int32_t *LrB, int32_t *LcB,
                 oracle_plan_t *out) {
-  if (b < 2 || b > 8 || M < 0 || K < 0 || N < 0 || strategy < 0 || strategy > 5) return OR_ERR_ARG;
+  if (b < 2 || b > 8 || M < 0 || K < 0 || N < 0 || strategy < 0 || strategy > 6) return OR_ERR_ARG;
   memset(out, 0, sizeof(*out));
   out->b = b;
   out->strategy = strategy;
@@ -53,6 +118,11 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
       if (l > LrB[t]) LrB[t] = l;
       if (l > LcB[j]) LcB[j] = l;
     }
+  if (strategy == OR_HYBRID) {
+    /* A: rows outer, columns inner; B: columns outer (entry (j, t) at B[t * N + j]), rows inner */
+    if (hybrid_choose(A, M, K, K, 1, b, LrA, LcA) != OR_OK) return OR_ERR_ARG;
+    if (hybrid_choose(B, N, K, 1, N, b, LcB, LrB) != OR_OK) return OR_ERR_ARG;
+  }
   const int32_t *vecs[4] = {LrA, LcA, LrB, LcB};
   const int64_t lens[4] = {M, K, K, N};
   for (int v = 0; v < 4; ++v) {
@@ -89,6 +159,10 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
       else if (out->oor_lines[2] > out->oor_lines[3]) db = OR_DIR_OUTER;
       else db = OR_DIR_INNER;
     }
+  } else if (strategy == OR_HYBRID) {
+    /* the levels above are already those of the hybrid choice */
+    da = (out->oor_lines[0] ? OR_DIR_OUTER : 0) | (out->oor_lines[1] ? OR_DIR_INNER : 0);
+    db = (out->oor_lines[3] ? OR_DIR_OUTER : 0) | (out->oor_lines[2] ? OR_DIR_INNER : 0);
   } else {
     da = (strategy == OR_ROW_ROW || strategy == OR_ROW_COL) ? OR_DIR_OUTER : OR_DIR_INNER;
     db = (strategy == OR_ROW_ROW || strategy == OR_COL_ROW) ? OR_DIR_INNER : OR_DIR_OUTER;
@@ -122,15 +196,15 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
 
   /* levels each index carries in the unpacked GEMM */
   out->M_eff = 0;
-  for (int64_t i = 0; i < M; ++i) out->M_eff += (da == OR_DIR_OUTER) ? LrA[i] : 1;
+  for (int64_t i = 0; i < M; ++i) out->M_eff += (da & OR_DIR_OUTER) ? LrA[i] : 1;
   out->N_eff = 0;
-  for (int64_t j = 0; j < N; ++j) out->N_eff += (db == OR_DIR_OUTER) ? LcB[j] : 1;
-  int maxla = (da == OR_DIR_INNER) ? out->lmax[1] : 1;
-  int maxlb = (db == OR_DIR_INNER) ? out->lmax[2] : 1;
+  for (int64_t j = 0; j < N; ++j) out->N_eff += (db & OR_DIR_OUTER) ? LcB[j] : 1;
+  int maxla = (da & OR_DIR_INNER) ? out->lmax[1] : 1;
+  int maxlb = (db & OR_DIR_INNER) ? out->lmax[2] : 1;
   out->K_eff = 0;
   for (int64_t t = 0; t < K; ++t) {
-    int64_t la = (da == OR_DIR_INNER) ? LcA[t] : 1;
-    int64_t lb = (db == OR_DIR_INNER) ? LrB[t] : 1;
+    int64_t la = (da & OR_DIR_INNER) ? LcA[t] : 1;
+    int64_t lb = (db & OR_DIR_INNER) ? LrB[t] : 1;
     out->K_eff += la * lb;
   }
   if (M > 0 && N > 0 && K > 0)
@@ -148,8 +222,8 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
       int lb = e - la;
       if (lb < 0 || lb >= maxlb) continue;
       for (int64_t t = 0; t < K; ++t) {
-        int64_t a = (da == OR_DIR_INNER) ? LcA[t] : 1;
-        int64_t bb = (db == OR_DIR_INNER) ? LrB[t] : 1;
+        int64_t a = (da & OR_DIR_INNER) ? LcA[t] : 1;
+        int64_t bb = (db & OR_DIR_INNER) ? LrB[t] : 1;
         if (a > la && bb > lb) len += 1;
       }
     }
@@ -167,7 +241,7 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
   out->K_unp = off;
 
   /* outer sizes: groups of lines of equal level */
-  if (da == OR_DIR_OUTER) {
+  if (da & OR_DIR_OUTER) {
     int64_t groups = 0;
     for (int L = 1; L <= out->lmax[0]; ++L) {
       int64_t cnt = 0;
@@ -179,7 +253,7 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
   } else {
     out->M_unp = M;
   }
-  if (db == OR_DIR_OUTER) {
+  if (db & OR_DIR_OUTER) {
     int64_t groups = 0;
     for (int L = 1; L <= out->lmax[3]; ++L) {
       int64_t cnt = 0;
@@ -215,8 +289,8 @@ int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t 
                      int32_t *lBk, int32_t *srcA, int32_t *lvlA, int32_t *srcB, int32_t *lvlB) {
   const int da = pl->dir_a, db = pl->dir_b;
   const int64_t M = pl->M, K = pl->K, N = pl->N;
-  int maxla = (da == OR_DIR_INNER) ? pl->lmax[1] : 1;
-  int maxlb = (db == OR_DIR_INNER) ? pl->lmax[2] : 1;
+  int maxla = (da & OR_DIR_INNER) ? pl->lmax[1] : 1;
+  int maxlb = (db & OR_DIR_INNER) ? pl->lmax[2] : 1;
 
   for (int64_t p = 0; p < pl->K_unp; ++p) { tK[p] = -1; lAk[p] = 0; lBk[p] = 0; }
   for (int g = 0; g < pl->n_groups; ++g) {
@@ -226,8 +300,8 @@ int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t 
       int lb = e - la;
       if (lb < 0 || lb >= maxlb) continue;
       for (int64_t t = 0; t < K; ++t) {
-        int64_t a = (da == OR_DIR_INNER) ? LcA[t] : 1;
-        int64_t bb = (db == OR_DIR_INNER) ? LrB[t] : 1;
+        int64_t a = (da & OR_DIR_INNER) ? LcA[t] : 1;
+        int64_t bb = (db & OR_DIR_INNER) ? LrB[t] : 1;
         if (a > la && bb > lb) {
           tK[p] = (int32_t)t;
           lAk[p] = la;
@@ -240,7 +314,7 @@ int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t 
   }
 
   for (int64_t u = 0; u < pl->M_unp; ++u) { srcA[u] = -1; lvlA[u] = 0; }
-  if (da == OR_DIR_OUTER) {
+  if (da & OR_DIR_OUTER) {
     int64_t grp = 0;
     for (int L = 1; L <= pl->lmax[0]; ++L) {
       int64_t per = OR_A_GROUP / L, rank = 0;
@@ -257,7 +331,7 @@ int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t 
   }
 
   for (int64_t w = 0; w < pl->N_unp; ++w) { srcB[w] = -1; lvlB[w] = 0; }
-  if (db == OR_DIR_OUTER) {
+  if (db & OR_DIR_OUTER) {
     int64_t grp = 0;
     for (int L = 1; L <= pl->lmax[3]; ++L) {
       int64_t per = OR_B_GROUP / L, rank = 0;

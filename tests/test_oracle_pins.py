@@ -233,7 +233,7 @@ def test_unpacked_equals_direct_random_tiny():
         if case < 100:
             assert np.array_equal(direct, oracle.gemm_i64(A, B))
         R = 1 << (b - 1)
-        for st in range(5):
+        for st in range(7):
             pl = oracle.plan(A, B, b, st)
             Au, Bu = oracle.unpack(pl, A, B)
             assert np.abs(Au.astype(np.int64)).max(initial=0) <= R - 1
@@ -411,6 +411,94 @@ def test_joint_mix_worked_case():
     assert np.array_equal(oracle.unpacked_gemm(joint, Au, Bu), A @ B)
 
 
+def _hybrid_expected(X, b, outer_axis):
+    """Brute force of the hybrid choice for one matrix, from numpy levels: every threshold tau from 1 to
+    (largest out-of-range count) + 1, the lines with count >= tau OUTER with their own level, the inner
+    levels the maxima over the other lines; least size, smallest tau on a tie.  Returns the (outer,
+    inner) level vectors each line carries and the size."""
+    L = _levels_numpy(X, b)
+    if outer_axis == 1:
+        L = L.T  # outer lines as rows
+    cnt = (L > 1).sum(axis=1)
+    lo_true = L.max(axis=1, initial=1)
+    best = None
+    for tau in range(1, int(cnt.max(initial=0)) + 2):
+        S = cnt >= tau
+        lo = np.where(S, lo_true, 1)
+        li = L[~S].max(axis=0, initial=1) if L.shape[1] else np.zeros(0, np.int64)
+        size = int(lo.sum()) * int(li.sum())
+        if best is None or size < best[0]:
+            best = (size, lo, li)
+    return best[1], best[2], best[0]
+
+
+def test_hybrid_choice_bruteforce():
+    """Hybrid ("unpack both", a reading: the outer lines dense with out-of-range entries unpacked OUTER,
+    the rest INNER): the levels each line carries equal a brute force over every threshold, the
+    per-matrix size is never above the smaller of the pure row and pure column sizes (which are its
+    thresholds 1 and max + 1), and the unpacked product is exact."""
+    rng = np.random.default_rng(29)
+    wins = 0
+    for case in range(300):
+        M, K, N = (int(x) for x in rng.integers(1, 14, size=3))
+        b = int(rng.integers(2, 9))
+        if case % 2:
+            A, B = workloads.rows_and_cols_case(rng, M, K, N, big=int(rng.choice([100, 5000])),
+                                                dense_rows=int(rng.integers(0, 3)), dense_cols=int(rng.integers(0, 3)))
+        else:
+            A, B = workloads.random_case(rng, M, K, N, big=int(rng.choice([50, 5000])), frac=0.15)
+        pl = oracle.plan(A, B, b, oracle.HYBRID)
+        lar, lac, size_a = _hybrid_expected(A, b, 0)
+        lbc, lbr, size_b = _hybrid_expected(B, b, 1)
+        assert np.array_equal(pl.levels["a_row"], lar) and np.array_equal(pl.levels["a_col"], lac)
+        assert np.array_equal(pl.levels["b_row"], lbr) and np.array_equal(pl.levels["b_col"], lbc)
+        assert pl.dir_a == (oracle.DIR_OUTER if (lar > 1).any() else 0) | (oracle.DIR_INNER if (lac > 1).any() else 0)
+        assert pl.dir_b == (oracle.DIR_OUTER if (lbc > 1).any() else 0) | (oracle.DIR_INNER if (lbr > 1).any() else 0)
+        LA, LB = _levels_numpy(A, b), _levels_numpy(B, b)
+        assert size_a <= min(int(LA.max(1).sum()) * K, M * int(LA.max(0).sum()))
+        assert size_b <= min(int(LB.max(0).sum()) * K, N * int(LB.max(1).sum()))
+        wins += size_a < min(int(LA.max(1).sum()) * K, M * int(LA.max(0).sum()))
+        Au, Bu = oracle.unpack(pl, A, B)
+        assert np.abs(Au.astype(np.int64)).max(initial=0) <= (1 << (b - 1)) - 1
+        assert np.array_equal(oracle.unpacked_gemm(pl, Au, Bu), A @ B), case
+    assert wins > 0  # the hybrid is strictly smaller than both pure directions on some inputs
+
+
+def test_hybrid_worked_case():
+    """Closed form, b = 5 (R = 16, 100 has 2 digits).  A 64 x 64 of ones with row 0 all 100 and
+    columns 5 and 9 equal to 100 in rows 10..29.  Row unpacking doubles the 21 rows holding outliers:
+    85 x 64.  Column unpacking doubles every column (row 0 reaches all of them): 64 x 128.  The hybrid
+    unpacks row 0 (64 outliers) OUTER and columns 5 and 9 INNER over the other rows (2 outliers each,
+    below any threshold from 3 to 64): 65 x 66, the smallest threshold of that size being 3.  B is 64 x 8
+    of ones (nothing to unpack).  Ratios: Mix 85/64, hybrid 65 * 66 / 64^2."""
+    A = np.ones((64, 64), np.int64)
+    A[0, :] = 100
+    A[10:30, 5] = 100
+    A[10:30, 9] = 100
+    B = np.ones((64, 8), np.int64)
+    mix = oracle.plan(A, B, 5, oracle.MIX)
+    hyb = oracle.plan(A, B, 5, oracle.HYBRID)
+    assert (mix.dir_a, mix.M_eff, mix.K_eff) == (oracle.DIR_OUTER, 85, 64)
+    assert (hyb.dir_a, hyb.dir_b, hyb.M_eff, hyb.K_eff, hyb.N_eff) == (oracle.DIR_BOTH, oracle.DIR_NONE, 65, 66, 8)
+    assert hyb.ratio == pytest.approx(65 * 66 / 64 ** 2, rel=1e-15)
+    want_rows = np.ones(64, np.int32)
+    want_rows[0] = 2
+    want_cols = np.ones(64, np.int32)
+    want_cols[[5, 9]] = 2
+    assert np.array_equal(hyb.levels["a_row"], want_rows) and np.array_equal(hyb.levels["a_col"], want_cols)
+    Au, Bu = oracle.unpack(hyb, A, B)
+    # row 0's two lines hold its digits (4 and 6: 100 = 6 * 16 + 4) in the level-0 segment only
+    r0 = np.flatnonzero(hyb.maps["srcA"] == 0)
+    lvl0 = hyb.maps["tK"] >= 0
+    hi = lvl0 & (hyb.maps["lAk"] > 0)
+    assert np.all(Au[r0[0], lvl0 & ~hi] == 4) and np.all(Au[r0[1], lvl0 & ~hi] == 6)
+    assert not Au[r0][:, hi].any()
+    # rows 10..29 carry the digits of columns 5 and 9 in the inner segments
+    r10 = int(np.flatnonzero(hyb.maps["srcA"] == 10)[0])
+    assert sorted(Au[r10, hi].tolist()) == [6, 6]
+    assert np.array_equal(oracle.unpacked_gemm(hyb, Au, Bu), A @ B)
+
+
 def test_mix_beats_fixed_on_channel_outliers():
     """The measured-effects table reports Mix below every fixed strategy on linear layers, where
     heavy hitters sit in channels; a channel-structured case reproduces that ordering."""
@@ -459,11 +547,13 @@ def test_layout_follows_documented_order():
         M, K, N = (int(x) for x in rng.integers(1, 40, size=3))
         b = int(rng.integers(2, 9))
         A, B = workloads.random_case(rng, M, K, N, big=4000, frac=0.2)
-        for st in range(5):
+        if _ % 3 == 0:
+            A, B = workloads.rows_and_cols_case(rng, M, K, N, big=4000, dense_rows=2, dense_cols=2)
+        for st in range(7):
             pl = oracle.plan(A, B, b, st)
             mp, lv = pl.maps, pl.levels
-            la = lv["a_col"] if pl.dir_a == oracle.DIR_INNER else np.ones(K, np.int32)
-            lb = lv["b_row"] if pl.dir_b == oracle.DIR_INNER else np.ones(K, np.int32)
+            la = lv["a_col"] if pl.dir_a & oracle.DIR_INNER else np.ones(K, np.int32)
+            lb = lv["b_row"] if pl.dir_b & oracle.DIR_INNER else np.ones(K, np.int32)
             # inner: groups ascending in e, offsets multiples of 128, inside a group (lA, t) ascending
             want = []
             for e, off, ln, padded in pl.groups:
@@ -480,7 +570,7 @@ def test_layout_follows_documented_order():
             for src, lvl, lines, G, dirv, outer in (
                     (mp["srcA"], mp["lvlA"], lv["a_row"], 32, pl.dir_a, oracle.DIR_OUTER),
                     (mp["srcB"], mp["lvlB"], lv["b_col"], 32, pl.dir_b, oracle.DIR_OUTER)):
-                if dirv != outer:
+                if not dirv & outer:
                     assert np.array_equal(src, np.arange(src.size)) and not lvl.any()
                     continue
                 assert src.size % G == 0

@@ -216,6 +216,24 @@ CONFIGS = {"tiny": tiny, "q_proj": q_proj, "mlp": mlp, "attention": attention, "
            "training_triple": training_triple}
 
 
+def rows_and_cols_case(rng, M, K, N, big=5000, dense_rows=1, dense_cols=1, scatter=0.02):
+    """Small random integer operands whose heavy hitters sit in a few whole rows AND a few whole columns
+    of each matrix (plus a scattered fraction): entries in [-20, 20], heavy ones up to +-big.  A has
+    `dense_rows` heavy rows and `dense_cols` heavy columns (in a random half of the rows); B likewise."""
+    out = []
+    for rows, cols in ((M, K), (K, N)):
+        X = rng.integers(-20, 21, size=(rows, cols)).astype(np.int64)
+        for r in rng.choice(rows, size=min(dense_rows, rows), replace=False):
+            X[r, :] = rng.integers(-big, big + 1, size=cols)
+        for c in rng.choice(cols, size=min(dense_cols, cols), replace=False):
+            sel = rng.random(rows) < 0.5
+            X[sel, c] = rng.integers(-big, big + 1, size=int(sel.sum()))
+        mask = rng.random(X.shape) < scatter
+        X[mask] = rng.integers(-big, big + 1, size=int(mask.sum()))
+        out.append(X)
+    return out[0], out[1]
+
+
 def random_case(rng, M, K, N, big=5000, frac=0.1):
     """Small random integer GEMM operands with heavy hitters: entries mostly in [-20, 20], a fraction
     `frac` of them up to +-big.  Used for brute-force checks."""
