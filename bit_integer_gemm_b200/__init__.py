@@ -28,9 +28,9 @@ IMQ_F32, IMQ_BF16, IMQ_I16, IMQ_I32, IMQ_I64 = 0, 1, 2, 3, 4
 # quantisation groups
 IMQ_PER_TENSOR, IMQ_PER_ROW, IMQ_PER_COL = 0, 1, 2
 # strategies
-IMQ_MIX, IMQ_ROW_ROW, IMQ_ROW_COL, IMQ_COL_ROW, IMQ_COL_COL, IMQ_MIX_JOINT = 0, 1, 2, 3, 4, 5
+IMQ_MIX, IMQ_ROW_ROW, IMQ_ROW_COL, IMQ_COL_ROW, IMQ_COL_COL, IMQ_MIX_JOINT, IMQ_HYBRID = 0, 1, 2, 3, 4, 5, 6
 # directions
-IMQ_DIR_NONE, IMQ_DIR_OUTER, IMQ_DIR_INNER = 0, 1, 2
+IMQ_DIR_NONE, IMQ_DIR_OUTER, IMQ_DIR_INNER, IMQ_DIR_BOTH = 0, 1, 2, 3
 IMQ_MAX_GROUPS = 64
 IMQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 IMQ_RTN_CLIP = 1

@@ -122,7 +122,7 @@ imq_status imq_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64
   if (it != IMQ_I16 && it != IMQ_I32) return IMQ_ERR_ARG;
   if (M < 0 || K < 0 || N < 0 || b < 2 || b > 8) return IMQ_ERR_ARG;
   if (M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return IMQ_ERR_UNSUPPORTED;
-  if ((int)strategy < 0 || (int)strategy > (int)IMQ_MIX_JOINT) return IMQ_ERR_ARG;
+  if ((int)strategy < 0 || (int)strategy > (int)IMQ_HYBRID) return IMQ_ERR_ARG;
   if (transA != 0 && transA != 1) return IMQ_ERR_ARG;
   if (transB != 0 && transB != 1) return IMQ_ERR_ARG;
   if (lda < (transA ? M : K) || ldb < (transB ? K : N)) return IMQ_ERR_ARG;

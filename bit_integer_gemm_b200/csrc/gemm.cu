@@ -755,8 +755,8 @@ imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu,
   if (first_drain >= 0) g.step_dfirst[first_drain] = 1;
   if (last_drain >= 0) g.step_dlast[last_drain] = 1;
   g.bm1 = I.b - 1;
-  g.a_outer = I.dir_a == IMQ_DIR_OUTER;
-  g.b_outer = I.dir_b == IMQ_DIR_OUTER;
+  g.a_outer = (I.dir_a & IMQ_DIR_OUTER) != 0;
+  g.b_outer = (I.dir_b & IMQ_DIR_OUTER) != 0;
   g.srcA = pl->srcA;
   g.grpA_L = pl->grpA_L;
   g.grpA_n = pl->grpA_n;

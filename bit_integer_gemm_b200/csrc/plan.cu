@@ -8,6 +8,7 @@
 //
 // Device work, in stream order:
 //   k_line_max     max |v| of every logical line, unless the caller passes the quantiser's side outputs
+//   k_hyb_*        (hybrid strategy only) the carried level of every line, decided on the device
 //   k_levels       int8 level of every line plus a summary: level sums, lines with level > 1, level
 //                  histograms, the joint histogram of (level of A column t, level of B row t), and the
 //                  exact 128-bit bound sum_t max|A[:,t]| * max|B[t,:]|
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(256) k_line_max(const T* __restrict__ X, int64
 // ------------------------------------------------------------------------------------------------
 struct LevelArgs {
   const int32_t* mx[4];
+  const int8_t* lvin[4];  // when not null, the levels themselves (the hybrid's carried levels)
   int8_t* lv[4];
   int64_t n[4];
   int32_t bm1;
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
       int L = 1;
       if (in) {
         const uint32_t m = (uint32_t)a.mx[v][i];
-        L = level_of(m, a.bm1);
+        L = a.lvin[v] ? (int)a.lvin[v][i] : level_of(m, a.bm1);
         a.lv[v][i] = (int8_t)L;
         bsum[v] += (unsigned)L;
         boor[v] += (L > 1);
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
       }
       warp_count(&hist[v][0], (uint32_t)L, in);
       if (v == 1) {
-        const int Lb = in ? level_of((uint32_t)a.mx[2][i], a.bm1) : 1;
+        const int Lb = !in ? 1 : (a.lvin[2] ? (int)a.lvin[2][i] : level_of((uint32_t)a.mx[2][i], a.bm1));
         warp_count(&joint[0][0], (uint32_t)(L * kLv + Lb), in);
       }
     }
@@ -180,6 +182,227 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
     if ((&hist[0][0])[i]) atomicAdd(&a.sum->hist[0][0] + i, (&hist[0][0])[i]);
   for (int i = tid; i < kLv * kLv; i += 256)
     if ((&joint[0][0])[i]) atomicAdd(&a.sum->joint[0][0] + i, (&joint[0][0])[i]);
+}
+
+// ------------------------------------------------------------------------------------------------
+// hybrid choice ("unpack both"): per matrix, the outer lines holding at least tau out-of-range entries
+// are unpacked OUTER, the others INNER, tau of least unpacked size (smallest on a tie).
+//   k_hyb_count   out-of-range entries of every outer line, cnt[o]
+//   k_hyb_minc    mex[t][l] = least cnt[o] over the lines o whose entry t has level l
+//   k_hyb_hist    suffix minima over l (then mex[t][l] = least count of a line reaching level >= l at t),
+//                 H[c] = #(t, l >= 2) with mex[t][l] = c, G[c] = sum of (level - 1) over lines of count c
+//   k_hyb_choose  one CTA per matrix: with S(tau) = {o : cnt[o] >= tau},
+//                 size(tau) = (n_out + sum_{c >= tau} G[c]) * (n_in + sum_{c < tau} H[c]),
+//                 since the inner level of t over the lines outside S(tau) is 1 + #{l >= 2 : mex[t][l] < tau}
+//   k_hyb_apply   the carried levels: lo[o] = level of o if cnt[o] >= tau else 1;
+//                 li[t] = largest l with mex[t][l] < tau, else 1
+// ------------------------------------------------------------------------------------------------
+constexpr int kHybL = 33;                 // levels 0..32 (level_of of a 32-bit magnitude is at most 32)
+constexpr int32_t kHybInf = 0x7F7F7F7F;   // mex before any entry (a memset byte pattern above any count)
+
+struct HybMat {
+  const void* X;        // the stored matrix, int16 or int32
+  int64_t rows, cols, ld;
+  int outer_is_row;     // outer lines are the stored rows (else the stored columns)
+  int64_t n_out, n_in;
+  const int32_t* omax;  // max |v| of every outer line
+  int32_t* cnt;         // [n_out]
+  int32_t* mex;         // [n_in][kHybL]
+  unsigned long long* H;  // [n_in + 2]
+  unsigned long long* G;  // [n_in + 2]
+  int32_t* tau;         // [1]
+  int8_t* lo;           // [n_out] carried levels of the outer lines
+  int8_t* li;           // [n_in] carried levels of the inner indices
+};
+
+struct HybArgs {
+  HybMat m[2];
+  int32_t bm1;
+};
+
+// Tiles of 32 stored rows x 256 stored columns, one column per thread (blockIdx.z = matrix).
+template <typename T>
+__global__ void __launch_bounds__(256) k_hyb_count(HybArgs a) {
+  const HybMat& m = a.m[blockIdx.z];
+  if ((int64_t)blockIdx.x * 256 >= m.cols) return;
+  const T* X = static_cast<const T*>(m.X);
+  const uint32_t lim = (1u << a.bm1) - 1u;
+  const int64_t c = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r0 = (int64_t)blockIdx.y * 32; r0 < m.rows; r0 += (int64_t)gridDim.y * 32) {
+    const int64_t r1 = r0 + 32 < m.rows ? r0 + 32 : m.rows;
+    int colcnt = 0;
+    for (int64_t r = r0; r < r1; ++r) {
+      bool oor = false;
+      if (c < m.cols) {
+        const int64_t v = X[r * m.ld + c];
+        oor = (uint64_t)(v < 0 ? -v : v) > lim;
+      }
+      if (m.outer_is_row) {
+        const unsigned ball = __ballot_sync(0xffffffffu, oor);
+        if (lane == 0 && ball) atomicAdd(m.cnt + r, __popc(ball));
+      } else {
+        colcnt += oor;
+      }
+    }
+    if (!m.outer_is_row && colcnt) atomicAdd(m.cnt + c, colcnt);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_hyb_minc(HybArgs a) {
+  const HybMat& m = a.m[blockIdx.z];
+  if ((int64_t)blockIdx.x * 256 >= m.cols) return;
+  const T* X = static_cast<const T*>(m.X);
+  const uint32_t lim = (1u << a.bm1) - 1u;
+  const int64_t c = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (c >= m.cols) return;
+  const int32_t ccol = m.outer_is_row ? 0 : m.cnt[c];
+  for (int64_t r0 = (int64_t)blockIdx.y * 32; r0 < m.rows; r0 += (int64_t)gridDim.y * 32) {
+    const int64_t r1 = r0 + 32 < m.rows ? r0 + 32 : m.rows;
+    for (int64_t r = r0; r < r1; ++r) {
+      const int64_t v = X[r * m.ld + c];
+      const uint32_t mag = (uint32_t)(v < 0 ? -v : v);
+      if (mag > lim) {
+        const int64_t t = m.outer_is_row ? c : r;
+        const int32_t cn = m.outer_is_row ? m.cnt[r] : ccol;
+        atomicMin(m.mex + t * kHybL + level_of(mag, a.bm1), cn);
+      }
+    }
+  }
+}
+
+// blockIdx.y = matrix; grid-stride over the inner indices, then over the outer lines.
+__global__ void __launch_bounds__(256) k_hyb_hist(HybArgs a) {
+  const HybMat& m = a.m[blockIdx.y];
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < m.n_in; t += stride) {
+    int32_t run = kHybInf;
+    for (int l = kHybL - 1; l >= 2; --l) {
+      int32_t* p = m.mex + t * kHybL + l;
+      run = min(run, *p);
+      *p = run;
+      if (run != kHybInf) atomicAdd(m.H + run, 1ull);
+    }
+  }
+  for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < m.n_out; o += stride) {
+    const int32_t c = m.cnt[o];
+    if (c > 0) atomicAdd(m.G + c, (unsigned long long)(level_of((uint32_t)m.omax[o], a.bm1) - 1));
+  }
+}
+
+// Inclusive block scan (1024 threads) of v; *total gets the block sum.
+__device__ __forceinline__ unsigned long long block_scan_ull(unsigned long long v, unsigned long long* warp_tot,
+                                                             unsigned long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    warp_tot[lane] = w;
+    if (lane == 31) *total = w;
+  }
+  __syncthreads();
+  const unsigned long long r = v + (warp > 0 ? warp_tot[warp - 1] : 0ull);
+  __syncthreads();
+  return r;
+}
+
+// One CTA of 1024 threads per matrix (blockIdx.x): tau from 1 to n_in + 1 (beyond the largest count
+// every tau has S empty, the same size as the first such tau, so the smallest-tau rule is unaffected).
+__global__ void __launch_bounds__(1024) k_hyb_choose(HybArgs a) {
+  const HybMat& m = a.m[blockIdx.x];
+  __shared__ unsigned long long warp_tot[32];
+  __shared__ unsigned long long tot;
+  __shared__ unsigned long long best_hi[32], best_lo[32];
+  __shared__ int64_t best_tau[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nt = m.n_in + 1;  // thresholds 1 .. n_in + 1; H and G are indexed 0 .. n_in + 1
+  // total of G
+  unsigned long long gsum = 0;
+  for (int64_t c = threadIdx.x; c <= nt; c += blockDim.x) gsum += m.G[c];
+  (void)block_scan_ull(gsum, warp_tot, &tot);
+  const unsigned long long gtot = tot;
+  __syncthreads();
+  unsigned long long hcarry = 0, gcarry = 0;  // sums over c < tau0
+  unsigned __int128 best = ~(unsigned __int128)0;
+  int64_t btau = 1;
+  for (int64_t tau0 = 1; tau0 <= nt; tau0 += blockDim.x) {
+    const int64_t tau = tau0 + threadIdx.x;
+    const bool in = tau <= nt;
+    // element c = tau - 1 joins the sums below tau
+    const unsigned long long h = in ? m.H[tau - 1] : 0ull, g = in ? m.G[tau - 1] : 0ull;
+    const unsigned long long hs = block_scan_ull(h, warp_tot, &tot);
+    const unsigned long long htot = tot;
+    const unsigned long long gs = block_scan_ull(g, warp_tot, &tot);
+    const unsigned long long gtot_chunk = tot;
+    if (in) {
+      const unsigned __int128 mo = (unsigned __int128)m.n_out + (gtot - (gcarry + gs));
+      const unsigned __int128 ki = (unsigned __int128)m.n_in + (hcarry + hs);
+      const unsigned __int128 cost = mo * ki;
+      if (cost < best) {  // taus ascend per thread: the first strict minimum is the smallest tau
+        best = cost;
+        btau = tau;
+      }
+    }
+    hcarry += htot;
+    gcarry += gtot_chunk;
+  }
+  // (cost, tau) lexicographic minimum over the block
+  unsigned long long bh = (unsigned long long)(best >> 64), bl = (unsigned long long)best;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long oh = __shfl_xor_sync(0xffffffffu, bh, o), ol = __shfl_xor_sync(0xffffffffu, bl, o);
+    const int64_t ot = __shfl_xor_sync(0xffffffffu, btau, o);
+    if (oh < bh || (oh == bh && (ol < bl || (ol == bl && ot < btau)))) {
+      bh = oh;
+      bl = ol;
+      btau = ot;
+    }
+  }
+  if (lane == 0) {
+    best_hi[warp] = bh;
+    best_lo[warp] = bl;
+    best_tau[warp] = btau;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+      if (best_hi[w] < bh || (best_hi[w] == bh && (best_lo[w] < bl || (best_lo[w] == bl && best_tau[w] < btau)))) {
+        bh = best_hi[w];
+        bl = best_lo[w];
+        btau = best_tau[w];
+      }
+    *m.tau = (int32_t)btau;
+  }
+}
+
+// blockIdx.y = matrix.
+__global__ void __launch_bounds__(256) k_hyb_apply(HybArgs a) {
+  const HybMat& m = a.m[blockIdx.y];
+  const int32_t tau = *m.tau;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < m.n_out; o += stride)
+    m.lo[o] = (int8_t)(m.cnt[o] >= tau ? level_of((uint32_t)m.omax[o], a.bm1) : 1);
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < m.n_in; t += stride) {
+    int l = 1;
+    for (int k = kHybL - 1; k >= 2; --k)
+      if (m.mex[t * kHybL + k] < tau) {
+        l = k;
+        break;
+      }
+    m.li[t] = (int8_t)l;
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -447,6 +670,29 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   off = align_up(off + sizeof(OuterClass) * 2 * kLv, 256);
   const size_t o_grps = off;
   off = align_up(off + sizeof(InnerGroup) * IMQ_MAX_GROUPS, 256);
+  // hybrid scratch: per matrix (A: M outer lines, B: N outer lines; K inner indices each) the counts and
+  // the two histograms (zeroed together), then the least-count tables (filled with kHybInf), then the
+  // threshold and the carried levels
+  const bool hybrid = strategy == IMQ_HYBRID;
+  const int64_t hyb_out[2] = {M, N};
+  size_t o_hcnt[2] = {0, 0}, o_hH[2] = {0, 0}, o_hG[2] = {0, 0}, o_hmex[2] = {0, 0}, o_htau[2] = {0, 0};
+  size_t o_hlo[2] = {0, 0}, o_hli[2] = {0, 0}, o_hzero = 0, o_hinf = 0, o_hend = 0;
+  if (hybrid) {
+    o_hzero = off;
+    for (int h = 0; h < 2; ++h) {
+      o_hcnt[h] = off; off = align_up(off + (size_t)hyb_out[h] * 4, 256);
+      o_hH[h] = off; off = align_up(off + (size_t)(K + 2) * 8, 256);
+      o_hG[h] = off; off = align_up(off + (size_t)(K + 2) * 8, 256);
+    }
+    o_hinf = off;
+    for (int h = 0; h < 2; ++h) { o_hmex[h] = off; off = align_up(off + (size_t)K * kHybL * 4, 256); }
+    o_hend = off;
+    for (int h = 0; h < 2; ++h) {
+      o_htau[h] = off; off = align_up(off + 4, 256);
+      o_hlo[h] = off; off = align_up(off + (size_t)hyb_out[h], 256);
+      o_hli[h] = off; off = align_up(off + (size_t)K, 256);
+    }
+  }
   const size_t stage1 = off;
   char* blk1 = nullptr;
   if (cudaMallocFromPoolAsync((void**)&blk1, stage1, ds->pool, st) != cudaSuccess) {
@@ -503,7 +749,61 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   LevelArgs la;
   for (int v = 0; v < 4; ++v) {
     la.mx[v] = lmx[v];
+    la.lvin[v] = nullptr;
     la.n[v] = nvec[v];
+  }
+  if (hybrid) {
+    // A: outer lines = its rows (stored rows unless transposed); B: outer lines = its columns (stored
+    // columns unless transposed); the inner indices are the other stored axis
+    HybArgs ha;
+    ha.bm1 = b - 1;
+    for (int h = 0; h < 2; ++h) {
+      HybMat& m = ha.m[h];
+      const int32_t tr = h == 0 ? transA : transB;
+      m.X = h == 0 ? A : B;
+      m.ld = h == 0 ? lda : ldb;
+      m.n_out = hyb_out[h];
+      m.n_in = K;
+      m.outer_is_row = h == 0 ? !tr : tr;
+      m.rows = m.outer_is_row ? m.n_out : K;
+      m.cols = m.outer_is_row ? K : m.n_out;
+      m.omax = h == 0 ? lmx[0] : lmx[3];
+      m.cnt = reinterpret_cast<int32_t*>(blk1 + o_hcnt[h]);
+      m.mex = reinterpret_cast<int32_t*>(blk1 + o_hmex[h]);
+      m.H = reinterpret_cast<unsigned long long*>(blk1 + o_hH[h]);
+      m.G = reinterpret_cast<unsigned long long*>(blk1 + o_hG[h]);
+      m.tau = reinterpret_cast<int32_t*>(blk1 + o_htau[h]);
+      m.lo = reinterpret_cast<int8_t*>(blk1 + o_hlo[h]);
+      m.li = reinterpret_cast<int8_t*>(blk1 + o_hli[h]);
+    }
+    if (cudaMemsetAsync(blk1 + o_hzero, 0, o_hinf - o_hzero, st) != cudaSuccess ||
+        cudaMemsetAsync(blk1 + o_hinf, 0x7F, o_hend - o_hinf, st) != cudaSuccess)
+      return fail(IMQ_ERR_CUDA);
+    int64_t maxc = 1, maxr = 1, maxn = 1;
+    for (int h = 0; h < 2; ++h) {
+      maxc = ha.m[h].cols > maxc ? ha.m[h].cols : maxc;
+      maxr = ha.m[h].rows > maxr ? ha.m[h].rows : maxr;
+      maxn = ha.m[h].n_out > maxn ? ha.m[h].n_out : maxn;
+    }
+    maxn = K > maxn ? K : maxn;
+    const dim3 gscan((unsigned)((maxc + 255) / 256), (unsigned)((maxr + 31) / 32 < 1024 ? (maxr + 31) / 32 : 1024), 2);
+    const int64_t gl = (maxn + 255) / 256 < (int64_t)ds->num_sms * 4 ? (maxn + 255) / 256 : (int64_t)ds->num_sms * 4;
+    const dim3 glines((unsigned)gl, 2);
+    if (it == IMQ_I16) {
+      k_hyb_count<int16_t><<<gscan, 256, 0, st>>>(ha);
+      k_hyb_minc<int16_t><<<gscan, 256, 0, st>>>(ha);
+    } else {
+      k_hyb_count<int32_t><<<gscan, 256, 0, st>>>(ha);
+      k_hyb_minc<int32_t><<<gscan, 256, 0, st>>>(ha);
+    }
+    k_hyb_hist<<<glines, 256, 0, st>>>(ha);
+    k_hyb_choose<<<2, 1024, 0, st>>>(ha);
+    k_hyb_apply<<<glines, 256, 0, st>>>(ha);
+    if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
+    la.lvin[0] = ha.m[0].lo;
+    la.lvin[1] = ha.m[0].li;
+    la.lvin[2] = ha.m[1].li;
+    la.lvin[3] = ha.m[1].lo;
   }
   la.status = ds->status;
   la.lv[0] = pl->lv_a_row;
@@ -562,6 +862,10 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
       else if (S.oor[2] != S.oor[3]) db = S.oor[2] < S.oor[3] ? IMQ_DIR_INNER : IMQ_DIR_OUTER;
       else db = IMQ_DIR_INNER;
     }
+  } else if (strategy == IMQ_HYBRID) {
+    // the summary already holds the carried levels of the hybrid choice
+    da = (S.oor[0] ? IMQ_DIR_OUTER : 0) | (S.oor[1] ? IMQ_DIR_INNER : 0);
+    db = (S.oor[3] ? IMQ_DIR_OUTER : 0) | (S.oor[2] ? IMQ_DIR_INNER : 0);
   } else {
     da = (strategy == IMQ_ROW_ROW || strategy == IMQ_ROW_COL) ? IMQ_DIR_OUTER : IMQ_DIR_INNER;
     db = (strategy == IMQ_ROW_ROW || strategy == IMQ_COL_ROW) ? IMQ_DIR_INNER : IMQ_DIR_OUTER;
@@ -597,8 +901,8 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   }
   I.dir_a = da;
   I.dir_b = db;
-  const bool a_outer = da == IMQ_DIR_OUTER, a_inner = da == IMQ_DIR_INNER;
-  const bool b_outer = db == IMQ_DIR_OUTER, b_inner = db == IMQ_DIR_INNER;
+  const bool a_outer = (da & IMQ_DIR_OUTER) != 0, a_inner = (da & IMQ_DIR_INNER) != 0;
+  const bool b_outer = (db & IMQ_DIR_OUTER) != 0, b_inner = (db & IMQ_DIR_INNER) != 0;
 
   // inner segments from the joint level histogram
   const int maxla = a_inner ? (int)lmax[1] : 1;

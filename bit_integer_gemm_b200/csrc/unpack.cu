@@ -5,6 +5,10 @@
 // unpacking.  Entry p of unpacked line u is digit (line level + inner level of p) of the source entry
 // (source line of u, inner index tK[p]); the layout is the one documented in include/imq.h.
 //
+// A line of a source unpacked OUTER with level L > 1 under the hybrid strategy holds all the digits of
+// its entries, so it is zero at inner positions of level lk > 0 (the other sources, single lines, hold
+// the digits of every inner level); for the pure strategies one of L > 1, lk > 0 never holds.
+//
 // Both unpacked operands are K-major (the inner index contiguous) because that is what the tcgen05
 // GEMM reads through TMA.  Two kernels cover the two storage orders of a source matrix:
 //   k_unpack_rows  the source line is a stored row (A, or B given as B^T): a CTA writes the digit planes
@@ -116,8 +120,10 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
         const int lk0 = lk[p];
         for (int b = 0; b < nb; ++b) {
           const int L = s_L[b];
+          const bool zero = L > 1 && lk0 > 0;
           for (int l = 0; l < L; ++l) {
-            const uint4 w = *reinterpret_cast<const uint4*>(planes + ((int64_t)b * P + l + lk0) * Kp + t0);
+            const uint4 w = zero ? make_uint4(0u, 0u, 0u, 0u)
+                                 : *reinterpret_cast<const uint4*>(planes + ((int64_t)b * P + l + lk0) * Kp + t0);
             *reinterpret_cast<uint4*>(out + (s_base[b] + l) * K_unp + p) = w;
           }
         }
@@ -138,8 +144,9 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
 #pragma unroll
               for (int r = 0; r < 4; ++r) {
                 const int k = q * 4 + r;
-                const uint32_t byte =
-                    tt[k] >= 0 ? (uint8_t)planes[((int64_t)b * P + l + ll[k]) * Kp + tt[k]] : 0u;
+                const uint32_t byte = (tt[k] >= 0 && (L == 1 || ll[k] == 0))
+                                          ? (uint8_t)planes[((int64_t)b * P + l + ll[k]) * Kp + tt[k]]
+                                          : 0u;
                 packed |= byte << (8 * r);
               }
               w[q] = packed;
@@ -307,8 +314,10 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* __restrict__ X, i
       const int64_t p = c * 16;
       if (t0 >= 0) {
         const int lk0 = meta_smem ? s_lk0[c] : lk[p];
+        const bool zero = L > 1 && lk0 > 0;
         for (int l = 0; l < L; ++l) {
-          const uint4 w = *reinterpret_cast<const uint4*>(planes + (int64_t)(l + lk0) * Kp + t0);
+          const uint4 w = zero ? make_uint4(0u, 0u, 0u, 0u)
+                               : *reinterpret_cast<const uint4*>(planes + (int64_t)(l + lk0) * Kp + t0);
           *reinterpret_cast<uint4*>(out + (base + l) * K_unp + p) = w;
         }
       } else {
@@ -326,7 +335,9 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* __restrict__ X, i
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
               const int k = q * 4 + r;
-              const uint32_t byte = tt[k] >= 0 ? (uint8_t)planes[(int64_t)(l + ll[k]) * Kp + tt[k]] : 0u;
+              const uint32_t byte = (tt[k] >= 0 && (L == 1 || ll[k] == 0))
+                                        ? (uint8_t)planes[(int64_t)(l + ll[k]) * Kp + tt[k]]
+                                        : 0u;
               packed |= byte << (8 * r);
             }
             w[q] = packed;
@@ -363,8 +374,11 @@ __global__ void __launch_bounds__(256) k_unpack_rows_direct(const T* __restrict_
       for (int l = 0; l < L; ++l) {
         uint32_t packed = 0;
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-          packed |= ((uint32_t)(uint8_t)(int8_t)digit_of(v[r], l + (int)(int8_t)(l4 >> (8 * r)), bm1)) << (8 * r);
+        for (int r = 0; r < 4; ++r) {
+          const int lkr = (int)(int8_t)(l4 >> (8 * r));
+          const int32_t d = (L > 1 && lkr > 0) ? 0 : digit_of(v[r], l + lkr, bm1);
+          packed |= ((uint32_t)(uint8_t)(int8_t)d) << (8 * r);
+        }
         *reinterpret_cast<uint32_t*>(out + (base + l) * K_unp + p) = packed;
       }
     }
@@ -407,7 +421,7 @@ __global__ void __launch_bounds__(256) k_unpack_cols(const T* __restrict__ X, in
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int pp = lane * 4 + r;
-        const int32_t d = s_t[pp] >= 0 ? digit_of(S[jj][pp], l + s_l[pp], bm1) : 0;
+        const int32_t d = (s_t[pp] >= 0 && (L == 1 || s_l[pp] == 0)) ? digit_of(S[jj][pp], l + s_l[pp], bm1) : 0;
         packed |= ((uint32_t)(uint8_t)(int8_t)d) << (8 * r);
       }
       *reinterpret_cast<uint32_t*>(out + (base + l) * K_unp + p0 + lane * 4) = packed;
@@ -488,11 +502,15 @@ imq_status unpack_typed(const imq_plan_t* pl, const T* A, const T* B, int8_t* Au
                         cudaStream_t st) {
   const imq_plan_info& I = pl->info;
   const int bm1 = I.b - 1;
-  const int a_outer = I.dir_a == IMQ_DIR_OUTER, b_outer = I.dir_b == IMQ_DIR_OUTER;
+  const int a_outer = (I.dir_a & IMQ_DIR_OUTER) != 0, b_outer = (I.dir_b & IMQ_DIR_OUTER) != 0;
+  const int a_inner = (I.dir_a & IMQ_DIR_INNER) != 0, b_inner = (I.dir_b & IMQ_DIR_INNER) != 0;
   // A' lines are the logical rows of A: stored rows unless A is given transposed
-  // planes an output line may read: OUTER lines their own levels, INNER ones the inner levels
-  const int pa = a_outer ? I.lmax_a_row : (I.dir_a == IMQ_DIR_INNER ? I.lmax_a_col : 1);
-  const int pb = b_outer ? I.lmax_b_col : (I.dir_b == IMQ_DIR_INNER ? I.lmax_b_row : 1);
+  // planes an output line may read: OUTER lines their own levels, INNER ones the inner levels (the
+  // hybrid's OUTER lines read only inner level 0, its single lines only the inner levels)
+  const int pa_o = a_outer ? I.lmax_a_row : 1, pa_i = a_inner ? I.lmax_a_col : 1;
+  const int pb_o = b_outer ? I.lmax_b_col : 1, pb_i = b_inner ? I.lmax_b_row : 1;
+  const int pa = pa_o > pa_i ? pa_o : pa_i;
+  const int pb = pb_o > pb_i ? pb_o : pb_i;
   imq_status s = unpack_one<T>(A, I.M, I.K, pl->lda, !pl->transA, a_outer, pa, pl->lv_a_row, pl->posA, pl->tK,
                                pl->lAk, pl->blk16, I.K_unp, bm1, Au, num_sms, st);
   if (s != IMQ_OK) return s;

@@ -72,11 +72,21 @@ typedef enum {
    * of least exact unpacked size M_eff * N_eff * K_eff (the unpack ratio's numerator) over the four
    * pairs, starting from the Mix choice and taking strict improvements in the order row/row, row/col,
    * col/row, col/col; a matrix without out-of-range entries stays not unpacked. */
-  IMQ_MIX_JOINT = 5
+  IMQ_MIX_JOINT = 5,
+  /* Hybrid, "unpack both" (READING of the per-matrix choice for matrices whose heavy hitters sit in
+   * some rows AND some columns, which pure row or column unpacking both handle badly): per matrix, the
+   * outer lines (rows of A, columns of B) holding at least tau out-of-range entries are unpacked OUTER
+   * with all their digits, the other lines INNER, the inner levels taken over those other lines only;
+   * tau is the threshold of least M_eff * K_eff (A) or N_eff * K_eff (B) -- thresholds 1 and max + 1
+   * are pure row and pure column unpacking, so the size is never above the smaller of the two -- the
+   * smallest such tau on a tie.  The plan reads A and B twice more (out-of-range counts per line, then
+   * the least count per inner index and level) and decides on the device. */
+  IMQ_HYBRID = 6
 } imq_strategy;
 
-/* Direction a matrix is unpacked in.  NONE: the matrix has no out-of-range entry (Mix only). */
-typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2 } imq_dir;
+/* Direction a matrix is unpacked in, a bit set.  NONE: the matrix has no out-of-range entry (Mix and
+ * the hybrid).  BOTH = OUTER | INNER: the hybrid unpacks some outer lines OUTER and the rest INNER. */
+typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2, IMQ_DIR_BOTH = 3 } imq_dir;
 
 #define IMQ_MAX_GROUPS 64   /* exponent groups e = lA + lB of the inner dimension                         */
 #define IMQ_INNER_PAD 128   /* each exponent group of the unpacked inner dimension is padded to this      */
@@ -211,10 +221,13 @@ typedef struct {
  *   Mix (READING of "chosen per matrix via outlier counts"): per matrix, the direction with the
  *   smaller factor; on a tie the one with fewer lines holding outliers; then row unpacking.  A matrix
  *   without any out-of-range entry is not unpacked (IMQ_DIR_NONE).
+ *   IMQ_HYBRID: see imq_strategy.  The plan's levels (imq_plan_levels, the lmax / sum_l / oor_lines
+ *   fields) are then the levels each line carries in the unpacked GEMM: 1 for an outer line that is
+ *   not unpacked OUTER, and inner levels taken over those lines only.
  *
  * A       device, logical M x K.  transA = 0: stored M x K with leading dim lda; transA = 1: stored
  *         K x M (A^T row-major) with leading dim lda.   dtype it (I16 or I32), as written by
- *         imq_rtn_quantize.
+ *         imq_rtn_quantize; I32 entries must differ from -2^31 (the quantiser never writes it).
  * B       device, logical K x N.  transB = 0: stored K x N; transB = 1: stored N x K (B^T row-major).
  * a_rowmax, a_colmax, b_rowmax, b_colmax
  *         device or NULL, int32 max |v| per logical line (A rows: M, A cols: K, B rows: K, B cols: N),
@@ -263,6 +276,9 @@ imq_status imq_plan_destroy(imq_plan_t *plan);
  *   OUTER rows of A: source rows sorted by level L (stable), floor(IMQ_A_GROUP / L) source rows per
  *   group of IMQ_A_GROUP unpacked rows, lines (source, level) consecutive, unused rows zero.
  *   OUTER columns of B: the same with IMQ_B_GROUP.
+ *   IMQ_DIR_BOTH (hybrid): a source row of A unpacked OUTER (level above 1) has all its digits on its
+ *   own lines and zeros at the inner pairs with lA > 0; the other rows are single lines with the
+ *   digits of every pair; likewise for the columns of B with lB > 0.
  * A_unp   device int8, M_unp x K_unp row-major (K contiguous), written in full.
  * B_unp_t device int8, N_unp x K_unp row-major (K contiguous, i.e. B'^T), written in full.
  * A, B must be the matrices (same pointers and layouts) the plan was made from.  Asynchronous.

@@ -207,7 +207,7 @@ def _run_path(imq, A, B, b, strategy, transA, transB, dtype=torch.int16, check_u
 
 
 @pytest.mark.parametrize("b", [2, 3, 5, 8])
-@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4, 5, 6])
 @pytest.mark.parametrize("trans", [(False, False), (True, False), (False, True), (True, True)])
 def test_path_parity_int32_regime(imq, b, strategy, trans):
     rng = np.random.default_rng(1000 * b + 10 * strategy + 2 * trans[0] + trans[1])
@@ -216,7 +216,7 @@ def test_path_parity_int32_regime(imq, b, strategy, trans):
 
 
 @pytest.mark.parametrize("b", [2, 3, 4, 5, 8])
-@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("strategy", [0, 1, 2, 3, 4, 5, 6])
 def test_path_parity_int64_regime(imq, b, strategy):
     rng = np.random.default_rng(77 + 10 * b + strategy)
     A, B = workloads.random_case(rng, 200, 384, 300, big=3000, frac=0.05)
@@ -248,6 +248,43 @@ def test_joint_mix_parity_where_it_differs_from_mix(imq):
             _run_path(imq, A, B, b, imq.IMQ_MIX_JOINT, False, transB)
 
 
+@pytest.mark.parametrize("b", [3, 5])
+@pytest.mark.parametrize("trans", [(False, False), (True, False), (False, True), (True, True)])
+def test_hybrid_parity_rows_and_columns(imq, b, trans):
+    """Hybrid (unpack both) on operands whose heavy hitters sit in a few whole rows and a few whole
+    columns, sizes spanning several tiles with ragged edges: the device's choice, levels, layout bytes
+    and the exact product equal the oracle's, and both matrices are unpacked in both directions."""
+    rng = np.random.default_rng(500 + 10 * b + 2 * trans[0] + trans[1])
+    A, B = workloads.rows_and_cols_case(rng, 300, 520, 270, big=3000, dense_rows=3, dense_cols=4, scatter=0.002)
+    plan = _run_path(imq, A, B, b, imq.IMQ_HYBRID, *trans)
+    assert (plan.info["dir_a"], plan.info["dir_b"]) == (imq.IMQ_DIR_BOTH, imq.IMQ_DIR_BOTH)
+    mix = oracle.plan(A, B, b, oracle.MIX)
+    assert plan.info["ratio"] < mix.ratio
+
+
+def test_hybrid_parity_worked_case_and_random(imq):
+    """The oracle pins' worked case (one dense row and two outlier columns; the hybrid takes the row
+    OUTER and the columns INNER), then random small cases of both input kinds, int16 and int32."""
+    A = np.ones((64, 64), np.int64)
+    A[0, :] = 100
+    A[10:30, 5] = 100
+    A[10:30, 9] = 100
+    B = np.ones((64, 8), np.int64)
+    plan = _run_path(imq, A, B, 5, imq.IMQ_HYBRID, False, False)
+    assert (plan.info["dir_a"], plan.info["M_eff"], plan.info["K_eff"]) == (imq.IMQ_DIR_BOTH, 65, 66)
+    rng = np.random.default_rng(4343)
+    for case in range(24):
+        M, K, N = (int(x) for x in rng.integers(1, 90, size=3))
+        b = int(rng.integers(2, 9))
+        if case % 2:
+            A, B = workloads.rows_and_cols_case(rng, M, K, N, big=int(rng.choice([100, 5000])),
+                                                dense_rows=int(rng.integers(0, 3)), dense_cols=int(rng.integers(0, 3)))
+        else:
+            A, B = workloads.random_case(rng, M, K, N, big=int(rng.choice([50, 5000])), frac=0.1)
+        _run_path(imq, A, B, b, imq.IMQ_HYBRID, bool(case % 3 == 1), bool(case % 4 >= 2),
+                  dtype=torch.int32 if case % 5 == 0 else torch.int16)
+
+
 def test_path_parity_no_outliers_is_plain_int8(imq):
     rng = np.random.default_rng(3)
     A = rng.integers(-127, 128, size=(256 + 17, 1024 + 40)).astype(np.int64)
@@ -260,7 +297,7 @@ def test_path_parity_no_outliers_is_plain_int8(imq):
 def test_path_parity_edge_shapes(imq, shape):
     rng = np.random.default_rng(sum(shape))
     A, B = workloads.random_case(rng, *shape, big=3000, frac=0.1)
-    for st in range(5):
+    for st in range(7):
         _run_path(imq, A, B, 5, st, False, False)
 
 
