@@ -13,7 +13,9 @@ replica (the path has no data exchange); time is the max over ranks.
 
 --impl reference times the CPU oracle (the reference arm of this build) on a bounded sample of the same
 workload on the host cores.  --workload training_triple times instead the forward, input-gradient and
-weight-gradient GEMMs of one linear layer with per-tensor RTN (one GPU; no end-to-end or CPU arm).
+weight-gradient GEMMs of one linear layer with per-tensor RTN, and --workload heavy_tokens activations
+whose heavy hitters sit in channels and tokens (one GPU; no end-to-end or CPU arm).  --strategy picks
+the unpack strategy (mix by default).
 """
 from __future__ import annotations
 
@@ -68,10 +70,11 @@ def _workload():
     return g
 
 
-def _config(g, extra=None):
+def _config(g, extra=None, strategy="mix"):
+    name = workloads.STRATEGY_NAMES[STRATEGIES[strategy]]
     c = {"workload": f"q_proj-shaped X {g.M}x{g.K} bf16 per-token RTN x W {g.K}x{g.N} bf16 "
-                     f"per-channel RTN, p={g.p}, beta={g.beta}, b={g.b}, Mix",
-         "M": g.M, "K": g.K, "N": g.N, "b": g.b, "beta": g.beta, "p": g.p, "strategy": "mix",
+                     f"per-channel RTN, p={g.p}, beta={g.beta}, b={g.b}, {name[0].upper() + name[1:]}",
+         "M": g.M, "K": g.K, "N": g.N, "b": g.b, "beta": g.beta, "p": g.p, "strategy": strategy,
          "l2": "flushed between timed steps (256 MB write)"}
     if extra:
         c.update(extra)
@@ -163,8 +166,9 @@ class Clocks:
 class Path:
     """Preallocated buffers and one step of the path on the current device."""
 
-    def __init__(self, imq, torch, g, X, W):
+    def __init__(self, imq, torch, g, X, W, strategy=0):
         self.imq, self.torch, self.g = imq, torch, g
+        self.strategy = strategy
         dev = X.device
         self.X, self.W = X, W
         M, K, N = g.M, g.K, g.N
@@ -192,7 +196,7 @@ class Path:
                              want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
         imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
                              want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True)
-        plan = imq.imq_plan(self.Xint, self.Wint, g.b, imq.IMQ_MIX, transB=True, maxes=self.mx)
+        plan = imq.imq_plan(self.Xint, self.Wint, g.b, self.strategy, transB=True, maxes=self.mx)
         I = plan.info
         if self.ws is None or self.ws.numel() < I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048:
             self.ws = self.torch.empty(I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048,
@@ -209,10 +213,14 @@ class Path:
         if gemm_events is not None:
             gemm_events[1].record()
         self.info = I
-        # kernels of this library launched by the step: 2 quantisers, levels, inner map, one outer map
-        # per OUTER operand, 2 unpack kernels, one zeroing kernel per OUTER operand, the GEMM
-        outer = int(I["dir_a"] == imq.IMQ_DIR_OUTER) + int(I["dir_b"] == imq.IMQ_DIR_OUTER)
-        self.launches = 2 + 1 + (1 if I["K_unp"] > 0 else 0) + outer + 2 + outer + 1
+        # kernels of this library launched by the step (the launch list of the same step shows them):
+        # 2 quantisers, each followed by the reduction of its per-CTA line maxima; the level kernel; the
+        # maps kernel; 2 unpack kernels; one zeroing kernel per OUTER operand; the GEMM
+        outer = int(bool(I["dir_a"] & imq.IMQ_DIR_OUTER)) + int(bool(I["dir_b"] & imq.IMQ_DIR_OUTER))
+        self.launches = 4 + 1 + (1 if I["K_unp"] > 0 else 0) + 2 + outer + 1
+        if self.strategy == imq.IMQ_HYBRID:
+            self.launches += 4  # the hybrid's count (both operands' outer lines are stored rows), histogram,
+            # choice and level kernels
         plan.destroy()
 
 
@@ -221,8 +229,9 @@ class GemmPath:
     transposes) on the current device: RTN of A and B, plan with the quantisers' maxima over logical
     lines, unpack into a workspace, GEMM with fold-back and dequantisation."""
 
-    def __init__(self, imq, torch, g, A, B):
+    def __init__(self, imq, torch, g, A, B, strategy=0):
         self.imq, self.torch, self.g, self.A, self.B = imq, torch, g, A, B
+        self.strategy = strategy
         t, dev = torch, A.device
         self.Ai = t.empty(tuple(A.shape), dtype=t.int16, device=dev)
         self.Bi = t.empty(tuple(B.shape), dtype=t.int16, device=dev)
@@ -245,7 +254,7 @@ class GemmPath:
         # maxima over LOGICAL lines: a transposed operand's stored rows are its logical columns
         a_row, a_col = (self.mA[1], self.mA[0]) if g.transA else (self.mA[0], self.mA[1])
         b_row, b_col = (self.mB[1], self.mB[0]) if g.transB else (self.mB[0], self.mB[1])
-        plan = imq.imq_plan(self.Ai, self.Bi, g.b, imq.IMQ_MIX, g.transA, g.transB,
+        plan = imq.imq_plan(self.Ai, self.Bi, g.b, self.strategy, g.transA, g.transB,
                             maxes=(a_row, a_col, b_row, b_col))
         I = plan.info
         need = I["workspace_bytes"]
@@ -266,25 +275,54 @@ class GemmPath:
         if gemm_events is not None:
             gemm_events[1].record()
         self.info = I
+        # kernels of this library launched by the step: per quantiser its kernel and the reduction of its
+        # per-CTA line maxima, plus for a per-tensor bf16 group the init and two histogram + select passes;
+        # the level and maps kernels (and those of the hybrid choice); 2 unpack kernels; one zeroing
+        # kernel per OUTER operand; the GEMM
+        quant = lambda gran: 7 if gran == imq.IMQ_PER_TENSOR else 2
+        outer = int(bool(I["dir_a"] & imq.IMQ_DIR_OUTER)) + int(bool(I["dir_b"] & imq.IMQ_DIR_OUTER))
+        hybrid = 0
+        if self.strategy == imq.IMQ_HYBRID:
+            # histogram, choice and levels, plus one count kernel for operands whose outer lines are
+            # stored rows and two for operands whose outer lines are stored columns
+            rows_outer = [not g.transA, g.transB]
+            hybrid = 3 + (1 if any(rows_outer) else 0) + (2 if not all(rows_outer) else 0)
+        self.launches = (quant(g.qa) + quant(g.qb) + 1 + (1 if I["K_unp"] > 0 else 0) + hybrid + 2 + outer + 1)
         plan.destroy()
 
 
-def run_triple(args):
-    """--workload training_triple: one step is the forward, input-gradient and weight-gradient GEMMs of
-    one linear layer (X 16384 x 512, W 512 x 2048, dY 16384 x 2048), each with per-tensor RTN."""
+STRATEGIES = {"mix": workloads.MIX, "row_row": workloads.ROW_ROW, "row_col": workloads.ROW_COL,
+              "col_row": workloads.COL_ROW, "col_col": workloads.COL_COL, "joint": workloads.MIX_JOINT,
+              "hybrid": workloads.HYBRID}
+
+GEMM_WORKLOADS = {
+    "training_triple": (workloads.training_triple,
+                        "training triple of one linear layer: forward X.W, dgrad dY.W^T, wgrad dY^T.X (X 16384x512, "
+                        "W 512x2048, dY 16384x2048 bf16), per-tensor RTN p=0.95 beta=31, b=5"),
+    "heavy_tokens": (workloads.heavy_tokens,
+                     "X 2048x4096 bf16 with 6 heavy channels and 4 heavy tokens, per-tensor RTN, x W 4096x4096 "
+                     "bf16 per-channel RTN, p=0.95, beta=15, b=8"),
+}
+
+
+def run_gemms(args):
+    """--workload training_triple | heavy_tokens: one step is the whole path (RTN of both operands, plan,
+    unpack, GEMM) for each GEMM of the workload, with the strategy --strategy names."""
     import torch
 
     import bit_integer_gemm_b200 as imq
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     imq.lib()
-    gems = workloads.training_triple()
+    make, desc = GEMM_WORKLOADS[args.workload]
+    strategy = STRATEGIES[args.strategy]
+    gems = make()
     dev_of = {}
     for g in gems:
         for st in (g.A, g.B):
             if st.name not in dev_of:
                 dev_of[st.name] = torch.from_numpy(st.data.view(np.int16)).to(dev).view(torch.bfloat16)
-    paths = [GemmPath(imq, torch, g, dev_of[g.A.name], dev_of[g.B.name]) for g in gems]
+    paths = [GemmPath(imq, torch, g, dev_of[g.A.name], dev_of[g.B.name], strategy) for g in gems]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         for pth in paths:
@@ -306,7 +344,8 @@ def run_triple(args):
             ends[k].record()
         torch.cuda.synchronize()
     total_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
-    gemm_ms = [sum(a.elapsed_time(b) for a, b in gev[k][i:i + 1]) for k in range(args.steps) for i in range(3)]
+    n = len(paths)
+    gemm_ms = [gev[k][i][0].elapsed_time(gev[k][i][1]) for k in range(args.steps) for i in range(n)]
     ops = sum(2.0 * g.M * g.N * g.K for g in gems)
     value = throughput(ops, 1, args.steps, total_ms)
     exec_ops = sum(2.0 * p.info["M_unp"] * p.info["N_unp"] * p.info["K_unp"] for p in paths)
@@ -318,19 +357,19 @@ def run_triple(args):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic (seeded, bf16)",
-        "config": {"workload": "training triple of one linear layer: forward X.W, dgrad dY.W^T, wgrad dY^T.X "
-                               "(X 16384x512, W 512x2048, dY 16384x2048 bf16), per-tensor RTN p=0.95 beta=31, "
-                               "b=5, Mix",
+        "config": {"workload": f"{desc}, {workloads.STRATEGY_NAMES[strategy]}",
+                   "strategy": args.strategy,
                    "l2": "flushed between timed steps (256 MB write)",
                    "gemms": [{"name": g.name, "M": g.M, "K": g.K, "N": g.N, "ratio": round(p.info["ratio"], 4),
                               "dir_a": p.info["dir_a"], "dir_b": p.info["dir_b"], "M_unp": p.info["M_unp"],
                               "N_unp": p.info["N_unp"], "K_unp": p.info["K_unp"],
-                              "gemm_ms": round(sum(gemm_ms[i::3]) / args.steps, 4)}
+                              "gemm_ms": round(sum(gemm_ms[i::n]) / args.steps, 4)}
                              for i, (g, p) in enumerate(zip(gems, paths))]},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(int8_peak, 1), "unit": "TOPS",
                      "frac": round(achieved / int8_peak, 4), "traffic": None,
-                     "kernel": "k_gemm, the three launches of a step together", "peak_source": f"{src} bf16 burst x2"},
+                     "kernel": f"k_gemm, the {n} launch(es) of a step together", "peak_source": f"{src} bf16 burst x2"},
         "e2e": None,
+        "gpu_launches": args.steps * sum(p.launches for p in paths),
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
@@ -357,7 +396,7 @@ def run_ours(args):
     Wh = torch.from_numpy(g.B.data.view(np.int16)).view(torch.bfloat16)
     X = Xh.to(dev)
     W = Wh.to(dev)
-    path = Path(imq, torch, g, X, W)
+    path = Path(imq, torch, g, X, W, STRATEGIES[args.strategy])
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def barrier():
@@ -453,7 +492,8 @@ def run_ours(args):
         "config": _config(g, {"parallelism": f"replicas x{world}", "ratio": round(I["ratio"], 4),
                               "dir_a": I["dir_a"], "dir_b": I["dir_b"], "M_unp": I["M_unp"],
                               "N_unp": I["N_unp"], "K_unp": I["K_unp"], "acc_bits": I["acc_bits"],
-                              "pct_int8_peak_effective": round(100 * value / world / int8_peak, 2)}),
+                              "pct_int8_peak_effective": round(100 * value / world / int8_peak, 2)},
+                          args.strategy),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(achieved / int8_peak, 4), "traffic": traffic,
                      "kernel": "k_gemm (tcgen05 kind::i8)", "peak_source": f"{src} bf16 burst x2",
@@ -540,7 +580,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
-            "data": "synthetic (seeded, bf16)", "config": _config(g, {"parallelism": "host cores"}),
+            "data": "synthetic (seeded, bf16)", "config": _config(g, {"parallelism": "host cores"}, args.strategy),
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -578,16 +618,19 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", choices=["q_proj", "training_triple"], default="q_proj",
+    ap.add_argument("--workload", choices=["q_proj"] + sorted(GEMM_WORKLOADS), default="q_proj",
                     help="q_proj: the headline step (default); training_triple: the three GEMMs of one "
-                         "quantised-training step of a linear layer (one GPU, no end-to-end or CPU arms)")
+                         "quantised-training step of a linear layer; heavy_tokens: activations with heavy "
+                         "channels and heavy tokens (the last two: one GPU, no end-to-end or CPU arms)")
+    ap.add_argument("--strategy", choices=sorted(STRATEGIES), default="mix",
+                    help="unpack strategy of the plans (default mix)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == "training_triple":
-        run_triple(args)
+    elif args.workload in GEMM_WORKLOADS:
+        run_gemms(args)
     else:
         run_ours(args)
 

@@ -187,8 +187,10 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
 // ------------------------------------------------------------------------------------------------
 // hybrid choice ("unpack both"): per matrix, the outer lines holding at least tau out-of-range entries
 // are unpacked OUTER, the others INNER, tau of least unpacked size (smallest on a tie).
-//   k_hyb_count   out-of-range entries of every outer line, cnt[o]
-//   k_hyb_minc    mex[t][l] = least cnt[o] over the lines o whose entry t has level l
+//   k_hyb_rows    outer lines stored as rows: a CTA per row counts its out-of-range entries, cnt[o], and
+//                 takes the count into mex[t][l] = least cnt[o] over the lines o whose entry t has level l
+//   k_hyb_count   outer lines stored as columns: cnt[o] ...
+//   k_hyb_minc    ... then mex, two passes
 //   k_hyb_hist    suffix minima over l (then mex[t][l] = least count of a line reaching level >= l at t),
 //                 H[c] = #(t, l >= 2) with mex[t][l] = c, G[c] = sum of (level - 1) over lines of count c
 //   k_hyb_choose  one CTA per matrix: with S(tau) = {o : cnt[o] >= tau},
@@ -207,10 +209,11 @@ struct HybMat {
   int64_t n_out, n_in;
   const int32_t* omax;  // max |v| of every outer line
   int32_t* cnt;         // [n_out]
-  int32_t* mex;         // [n_in][kHybL]
+  int32_t* mex;         // [kHybL][n_in], level-major so that a warp's inner indices are adjacent
   unsigned long long* H;  // [n_in + 2]
   unsigned long long* G;  // [n_in + 2]
   int32_t* tau;         // [1]
+  int32_t* cmax;        // [1] largest cnt[o] (zeroed with the counts)
   int8_t* lo;           // [n_out] carried levels of the outer lines
   int8_t* li;           // [n_in] carried levels of the inner indices
 };
@@ -220,75 +223,225 @@ struct HybArgs {
   int32_t bm1;
 };
 
-// Tiles of 32 stored rows x 256 stored columns, one column per thread (blockIdx.z = matrix).
+// The matrices whose outer lines are stored columns: tiles of 8 stored rows x (256 kC) stored columns,
+// kC consecutive columns per thread (one 16-byte load per row when the rows are 16-byte aligned, else
+// one column per thread; blockIdx.z = matrix).  k_hyb_count adds each column's out-of-range entries of
+// the tile into cnt; k_hyb_minc then takes the column's count into mex for each of them.
+template <typename T, bool kMin>
+__device__ __forceinline__ void hyb_cols_tile(const HybMat& m, uint32_t lim, int bm1) {
+  constexpr int kV = 16 / sizeof(T);
+  const T* X = static_cast<const T*>(m.X);
+  const bool vec = (m.cols % kV == 0) && (m.ld % kV == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  const int kC = vec ? kV : 1;
+  const int64_t c0 = ((int64_t)blockIdx.x * 256 + threadIdx.x) * kC;
+  if (c0 >= m.cols) return;
+  int32_t cnt[kV];
+#pragma unroll
+  for (int k = 0; k < kV; ++k) cnt[k] = 0;
+  if (kMin) {
+#pragma unroll
+    for (int k = 0; k < kV; ++k) cnt[k] = k < kC ? m.cnt[c0 + k] : 0;
+  }
+  for (int64_t r0 = (int64_t)blockIdx.y * 8; r0 < m.rows; r0 += (int64_t)gridDim.y * 8) {
+    const int64_t r1 = r0 + 8 < m.rows ? r0 + 8 : m.rows;
+    int32_t add[kV];
+#pragma unroll
+    for (int k = 0; k < kV; ++k) add[k] = 0;
+#pragma unroll 8
+    for (int64_t r = r0; r < r1; ++r) {
+      T v[kV];
+      if (vec) {
+        const uint4 w = *reinterpret_cast<const uint4*>(X + r * m.ld + c0);
+        const T* p = reinterpret_cast<const T*>(&w);
+#pragma unroll
+        for (int k = 0; k < kV; ++k) v[k] = p[k];
+      } else {
+        v[0] = X[r * m.ld + c0];
+#pragma unroll
+        for (int k = 1; k < kV; ++k) v[k] = 0;
+      }
+#pragma unroll
+      for (int k = 0; k < kV; ++k) {
+        const int64_t x = v[k];
+        const uint32_t mag = (uint32_t)(x < 0 ? -x : x);
+        if (mag > lim) {
+          if (kMin)
+            atomicMin(m.mex + (int64_t)level_of(mag, bm1) * m.n_in + r, cnt[k]);
+          else
+            add[k] += 1;
+        }
+      }
+    }
+    if (!kMin) {
+#pragma unroll
+      for (int k = 0; k < kV; ++k)
+        if (add[k]) atomicAdd(m.cnt + c0 + k, add[k]);
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_hyb_count(HybArgs a) {
   const HybMat& m = a.m[blockIdx.z];
-  if ((int64_t)blockIdx.x * 256 >= m.cols) return;
-  const T* X = static_cast<const T*>(m.X);
-  const uint32_t lim = (1u << a.bm1) - 1u;
-  const int64_t c = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  const int lane = threadIdx.x & 31;
-  for (int64_t r0 = (int64_t)blockIdx.y * 32; r0 < m.rows; r0 += (int64_t)gridDim.y * 32) {
-    const int64_t r1 = r0 + 32 < m.rows ? r0 + 32 : m.rows;
-    int colcnt = 0;
-    for (int64_t r = r0; r < r1; ++r) {
-      bool oor = false;
-      if (c < m.cols) {
-        const int64_t v = X[r * m.ld + c];
-        oor = (uint64_t)(v < 0 ? -v : v) > lim;
-      }
-      if (m.outer_is_row) {
-        const unsigned ball = __ballot_sync(0xffffffffu, oor);
-        if (lane == 0 && ball) atomicAdd(m.cnt + r, __popc(ball));
-      } else {
-        colcnt += oor;
-      }
-    }
-    if (!m.outer_is_row && colcnt) atomicAdd(m.cnt + c, colcnt);
-  }
+  if (m.outer_is_row) return;
+  hyb_cols_tile<T, false>(m, (1u << a.bm1) - 1u, a.bm1);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_hyb_minc(HybArgs a) {
   const HybMat& m = a.m[blockIdx.z];
-  if ((int64_t)blockIdx.x * 256 >= m.cols) return;
-  const T* X = static_cast<const T*>(m.X);
-  const uint32_t lim = (1u << a.bm1) - 1u;
-  const int64_t c = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (c >= m.cols) return;
-  const int32_t ccol = m.outer_is_row ? 0 : m.cnt[c];
-  for (int64_t r0 = (int64_t)blockIdx.y * 32; r0 < m.rows; r0 += (int64_t)gridDim.y * 32) {
-    const int64_t r1 = r0 + 32 < m.rows ? r0 + 32 : m.rows;
-    for (int64_t r = r0; r < r1; ++r) {
-      const int64_t v = X[r * m.ld + c];
-      const uint32_t mag = (uint32_t)(v < 0 ? -v : v);
-      if (mag > lim) {
-        const int64_t t = m.outer_is_row ? c : r;
-        const int32_t cn = m.outer_is_row ? m.cnt[r] : ccol;
-        atomicMin(m.mex + t * kHybL + level_of(mag, a.bm1), cn);
+  if (m.outer_is_row) return;
+  hyb_cols_tile<T, true>(m, (1u << a.bm1) - 1u, a.bm1);
+}
+
+// Count and least counts in one pass when the outer lines are the stored rows: one warp per row counts
+// the row's out-of-range entries (16-byte loads when the rows are 16-byte aligned), then sweeps the
+// row again (now in L1 / L2) to take the count into mex for each of them.  blockIdx.y = matrix; a
+// matrix whose outer lines are stored columns is skipped here (k_hyb_count / k_hyb_minc serve it).
+// Out-of-range halves of a word of two int16 entries: bit 15 / bit 31 set where |entry| > lim (lim <=
+// 127).  |entry| per half without a carry between halves (as in the unpack kernel), then lim is
+// subtracted by adding 0x7FFF - lim: a half reaches 0x8000 exactly when it exceeds lim, and no half
+// carries out (|entry| <= 0x8000).
+__device__ __forceinline__ uint32_t oor_halves(uint32_t w, uint32_t lim) {
+  const uint32_t sgn = (w >> 15) & 0x00010001u;
+  const uint32_t mag = (w ^ (sgn * 0xFFFFu)) + sgn;
+  return (mag + (0x7FFFu - lim) * 0x00010001u) & 0x80008000u;
+}
+
+// One stored row (an outer line) per CTA of kRowThreads threads: the row's out-of-range entries are
+// counted (16-byte loads, two int16 entries per word at a time) and summed over the CTA, then the row is
+// swept again (now in L1 / L2) to take the count into mex for each of them.
+constexpr int kRowThreads = 128;
+
+template <typename T>
+__device__ __forceinline__ void hyb_row(const HybMat& m, int64_t r, uint32_t lim, int bm1, int* red) {
+  const T* xr = static_cast<const T*>(m.X) + r * m.ld;
+  constexpr int kV = 16 / sizeof(T);  // entries per 16-byte load
+  constexpr int kU = 4;               // 16-byte loads of a thread in flight
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool vec = (m.cols % kV == 0) && (m.ld % kV == 0) && ((reinterpret_cast<uintptr_t>(m.X) & 15) == 0);
+  int c = 0;
+  if (vec) {
+    for (int64_t t0 = (int64_t)tid * kV; t0 < m.cols; t0 += (int64_t)kRowThreads * kV * kU) {
+      uint4 w[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t t = t0 + (int64_t)u * kRowThreads * kV;
+        w[u] = t < m.cols ? *reinterpret_cast<const uint4*>(xr + t) : make_uint4(0u, 0u, 0u, 0u);
       }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if constexpr (sizeof(T) == 2) {
+          c += __popc(oor_halves(w[u].x, lim) | (oor_halves(w[u].y, lim) >> 1)) +
+               __popc(oor_halves(w[u].z, lim) | (oor_halves(w[u].w, lim) >> 1));
+        } else {
+          const int32_t v[4] = {(int32_t)w[u].x, (int32_t)w[u].y, (int32_t)w[u].z, (int32_t)w[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) c += (uint32_t)(v[k] < 0 ? -(int64_t)v[k] : v[k]) > lim;
+        }
+      }
+    }
+  } else {
+    for (int64_t t = tid; t < m.cols; t += kRowThreads) {
+      const int64_t x = xr[t];
+      c += (uint64_t)(x < 0 ? -x : x) > lim;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) red[warp] = c;
+  __syncthreads();
+  c = 0;
+#pragma unroll
+  for (int w = 0; w < kRowThreads / 32; ++w) c += red[w];
+  __syncthreads();  // red is reused by the next row
+  if (tid == 0) m.cnt[r] = c;
+  if (c == 0) return;
+  if (vec && sizeof(T) == 2) {
+    for (int64_t t0 = (int64_t)tid * kV; t0 < m.cols; t0 += (int64_t)kRowThreads * kV * kU) {
+      uint4 w[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t t = t0 + (int64_t)u * kRowThreads * kV;
+        w[u] = t < m.cols ? *reinterpret_cast<const uint4*>(xr + t) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        const int64_t t = t0 + (int64_t)u * kRowThreads * kV;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t hit = oor_halves(ww[q], lim);
+          if (hit == 0) continue;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            if (!(hit & (0x8000u << (16 * hf)))) continue;
+            const int32_t x = (int16_t)(ww[q] >> (16 * hf));
+            const uint32_t mag = (uint32_t)(x < 0 ? -x : x);
+            atomicMin(m.mex + (int64_t)level_of(mag, bm1) * m.n_in + t + 2 * q + hf, c);
+          }
+        }
+      }
+    }
+  } else {
+    for (int64_t t = tid; t < m.cols; t += kRowThreads) {
+      const int64_t x = xr[t];
+      const uint32_t mag = (uint32_t)(x < 0 ? -x : x);
+      if (mag > lim) atomicMin(m.mex + (int64_t)level_of(mag, bm1) * m.n_in + t, c);
     }
   }
 }
 
-// blockIdx.y = matrix; grid-stride over the inner indices, then over the outer lines.
+// The matrices whose outer lines are stored rows: CTAs run over the rows of matrix 0 then matrix 1 (a
+// matrix whose outer lines are stored columns has none here; the column kernels serve it).
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) k_hyb_rows(HybArgs a) {
+  __shared__ int red[kRowThreads / 32];
+  const uint32_t lim = (1u << a.bm1) - 1u;
+  const int64_t n0 = a.m[0].outer_is_row ? a.m[0].rows : 0;
+  const int64_t n1 = a.m[1].outer_is_row ? a.m[1].rows : 0;
+  for (int64_t w = blockIdx.x; w < n0 + n1; w += gridDim.x) {
+    if (w < n0)
+      hyb_row<T>(a.m[0], w, lim, a.bm1, red);
+    else
+      hyb_row<T>(a.m[1], w - n0, lim, a.bm1, red);
+  }
+}
+
+// blockIdx.y = matrix; grid-stride over the inner indices, then over the outer lines.  The levels 2..32
+// of one inner index are loaded together (independent loads), turned into suffix minima in registers and
+// written back (level-major: the loads of a warp are coalesced).
 __global__ void __launch_bounds__(256) k_hyb_hist(HybArgs a) {
   const HybMat& m = a.m[blockIdx.y];
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < m.n_in; t += stride) {
+    int32_t v[kHybL];
+#pragma unroll
+    for (int l = 2; l < kHybL; ++l) v[l] = m.mex[(int64_t)l * m.n_in + t];
     int32_t run = kHybInf;
+#pragma unroll
     for (int l = kHybL - 1; l >= 2; --l) {
-      int32_t* p = m.mex + t * kHybL + l;
-      run = min(run, *p);
-      *p = run;
-      if (run != kHybInf) atomicAdd(m.H + run, 1ull);
+      run = min(run, v[l]);
+      v[l] = run;
+    }
+#pragma unroll
+    for (int l = 2; l < kHybL; ++l) {
+      m.mex[(int64_t)l * m.n_in + t] = v[l];
+      if (v[l] != kHybInf) atomicAdd(m.H + v[l], 1ull);
     }
   }
+  int32_t cm = 0;
   for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < m.n_out; o += stride) {
     const int32_t c = m.cnt[o];
-    if (c > 0) atomicAdd(m.G + c, (unsigned long long)(level_of((uint32_t)m.omax[o], a.bm1) - 1));
+    if (c > 0) {
+      atomicAdd(m.G + c, (unsigned long long)(level_of((uint32_t)m.omax[o], a.bm1) - 1));
+      cm = max(cm, c);
+    }
   }
+  // the largest count, one atomic per warp
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+  if ((threadIdx.x & 31) == 0 && cm > 0) atomicMax(m.cmax, cm);
 }
 
 // Inclusive block scan (1024 threads) of v; *total gets the block sum.
@@ -318,8 +471,9 @@ __device__ __forceinline__ unsigned long long block_scan_ull(unsigned long long 
   return r;
 }
 
-// One CTA of 1024 threads per matrix (blockIdx.x): tau from 1 to n_in + 1 (beyond the largest count
-// every tau has S empty, the same size as the first such tau, so the smallest-tau rule is unaffected).
+// One CTA of 1024 threads per matrix (blockIdx.x): tau from 1 to the largest count + 1, a contiguous
+// run of thresholds per thread.  One block scan of the per-thread sums of H and G gives each thread the
+// sums below its first threshold; the thread then walks its run.
 __global__ void __launch_bounds__(1024) k_hyb_choose(HybArgs a) {
   const HybMat& m = a.m[blockIdx.x];
   __shared__ unsigned long long warp_tot[32];
@@ -327,36 +481,34 @@ __global__ void __launch_bounds__(1024) k_hyb_choose(HybArgs a) {
   __shared__ unsigned long long best_hi[32], best_lo[32];
   __shared__ int64_t best_tau[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t nt = m.n_in + 1;  // thresholds 1 .. n_in + 1; H and G are indexed 0 .. n_in + 1
-  // total of G
-  unsigned long long gsum = 0;
-  for (int64_t c = threadIdx.x; c <= nt; c += blockDim.x) gsum += m.G[c];
-  (void)block_scan_ull(gsum, warp_tot, &tot);
+  // thresholds 1 .. cmax + 1: above the largest count every threshold leaves S empty, and H and G are 0
+  // beyond it (H and G are indexed 0 .. n_in + 1, cmax <= n_in)
+  const int64_t nt = (int64_t)*m.cmax + 1;
+  const int64_t per = (nt + blockDim.x - 1) / blockDim.x;
+  const int64_t tau0 = 1 + (int64_t)threadIdx.x * per;
+  const int64_t tau1 = tau0 + per - 1 < nt ? tau0 + per - 1 : nt;  // this thread's run tau0 .. tau1
+  // element c = tau - 1 joins the sums below tau + 1
+  unsigned long long hs = 0, gs = 0;
+  for (int64_t tau = tau0; tau <= tau1; ++tau) {
+    hs += m.H[tau - 1];
+    gs += m.G[tau - 1];
+  }
+  const unsigned long long hin = block_scan_ull(hs, warp_tot, &tot);
+  const unsigned long long gin = block_scan_ull(gs, warp_tot, &tot);
   const unsigned long long gtot = tot;
-  __syncthreads();
-  unsigned long long hcarry = 0, gcarry = 0;  // sums over c < tau0
+  unsigned long long hbelow = hin - hs, gbelow = gin - gs;  // sums over c < tau0 - 1
   unsigned __int128 best = ~(unsigned __int128)0;
   int64_t btau = 1;
-  for (int64_t tau0 = 1; tau0 <= nt; tau0 += blockDim.x) {
-    const int64_t tau = tau0 + threadIdx.x;
-    const bool in = tau <= nt;
-    // element c = tau - 1 joins the sums below tau
-    const unsigned long long h = in ? m.H[tau - 1] : 0ull, g = in ? m.G[tau - 1] : 0ull;
-    const unsigned long long hs = block_scan_ull(h, warp_tot, &tot);
-    const unsigned long long htot = tot;
-    const unsigned long long gs = block_scan_ull(g, warp_tot, &tot);
-    const unsigned long long gtot_chunk = tot;
-    if (in) {
-      const unsigned __int128 mo = (unsigned __int128)m.n_out + (gtot - (gcarry + gs));
-      const unsigned __int128 ki = (unsigned __int128)m.n_in + (hcarry + hs);
-      const unsigned __int128 cost = mo * ki;
-      if (cost < best) {  // taus ascend per thread: the first strict minimum is the smallest tau
-        best = cost;
-        btau = tau;
-      }
+  for (int64_t tau = tau0; tau <= tau1; ++tau) {
+    hbelow += m.H[tau - 1];
+    gbelow += m.G[tau - 1];
+    const unsigned __int128 mo = (unsigned __int128)m.n_out + (gtot - gbelow);
+    const unsigned __int128 ki = (unsigned __int128)m.n_in + hbelow;
+    const unsigned __int128 cost = mo * ki;
+    if (cost < best) {  // thresholds ascend: the first strict minimum is the smallest tau
+      best = cost;
+      btau = tau;
     }
-    hcarry += htot;
-    gcarry += gtot_chunk;
   }
   // (cost, tau) lexicographic minimum over the block
   unsigned long long bh = (unsigned long long)(best >> 64), bl = (unsigned long long)best;
@@ -395,12 +547,10 @@ __global__ void __launch_bounds__(256) k_hyb_apply(HybArgs a) {
   for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < m.n_out; o += stride)
     m.lo[o] = (int8_t)(m.cnt[o] >= tau ? level_of((uint32_t)m.omax[o], a.bm1) : 1);
   for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < m.n_in; t += stride) {
+    // suffix minima are non-decreasing in l: the levels below tau are 2 .. L
     int l = 1;
-    for (int k = kHybL - 1; k >= 2; --k)
-      if (m.mex[t * kHybL + k] < tau) {
-        l = k;
-        break;
-      }
+#pragma unroll
+    for (int k = 2; k < kHybL; ++k) l += m.mex[(int64_t)k * m.n_in + t] < tau;
     m.li[t] = (int8_t)l;
   }
 }
@@ -676,7 +826,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   const bool hybrid = strategy == IMQ_HYBRID;
   const int64_t hyb_out[2] = {M, N};
   size_t o_hcnt[2] = {0, 0}, o_hH[2] = {0, 0}, o_hG[2] = {0, 0}, o_hmex[2] = {0, 0}, o_htau[2] = {0, 0};
-  size_t o_hlo[2] = {0, 0}, o_hli[2] = {0, 0}, o_hzero = 0, o_hinf = 0, o_hend = 0;
+  size_t o_hlo[2] = {0, 0}, o_hli[2] = {0, 0}, o_hcmax[2] = {0, 0}, o_hzero = 0, o_hinf = 0, o_hend = 0;
   if (hybrid) {
     o_hzero = off;
     for (int h = 0; h < 2; ++h) {
@@ -684,6 +834,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
       o_hH[h] = off; off = align_up(off + (size_t)(K + 2) * 8, 256);
       o_hG[h] = off; off = align_up(off + (size_t)(K + 2) * 8, 256);
     }
+    for (int h = 0; h < 2; ++h) { o_hcmax[h] = off; off = align_up(off + 4, 256); }
     o_hinf = off;
     for (int h = 0; h < 2; ++h) { o_hmex[h] = off; off = align_up(off + (size_t)K * kHybL * 4, 256); }
     o_hend = off;
@@ -773,6 +924,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
       m.H = reinterpret_cast<unsigned long long*>(blk1 + o_hH[h]);
       m.G = reinterpret_cast<unsigned long long*>(blk1 + o_hG[h]);
       m.tau = reinterpret_cast<int32_t*>(blk1 + o_htau[h]);
+      m.cmax = reinterpret_cast<int32_t*>(blk1 + o_hcmax[h]);
       m.lo = reinterpret_cast<int8_t*>(blk1 + o_hlo[h]);
       m.li = reinterpret_cast<int8_t*>(blk1 + o_hli[h]);
     }
@@ -786,15 +938,32 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
       maxn = ha.m[h].n_out > maxn ? ha.m[h].n_out : maxn;
     }
     maxn = K > maxn ? K : maxn;
-    const dim3 gscan((unsigned)((maxc + 255) / 256), (unsigned)((maxr + 31) / 32 < 1024 ? (maxr + 31) / 32 : 1024), 2);
-    const int64_t gl = (maxn + 255) / 256 < (int64_t)ds->num_sms * 4 ? (maxn + 255) / 256 : (int64_t)ds->num_sms * 4;
+    // column kernels: 256 threads x up to 16 / sizeof(entry) columns, 8 rows per tile; the grid covers
+    // the wider of the two matrices at one column per thread (threads past the end return)
+    const dim3 gscan((unsigned)((maxc + 255) / 256), (unsigned)((maxr + 7) / 8 < 4096 ? (maxr + 7) / 8 : 4096), 2);
+    const int64_t gl = (maxn + 255) / 256 < (int64_t)ds->num_sms * 8 ? (maxn + 255) / 256 : (int64_t)ds->num_sms * 8;
     const dim3 glines((unsigned)gl, 2);
+    const bool any_rows = ha.m[0].outer_is_row || ha.m[1].outer_is_row;
+    const bool any_cols = !ha.m[0].outer_is_row || !ha.m[1].outer_is_row;
+    int64_t nrows = 0;
+    for (int h = 0; h < 2; ++h)
+      if (ha.m[h].outer_is_row) nrows += ha.m[h].rows;
+    // one CTA per row, up to 16 resident per SM
+    int64_t gr = nrows < (int64_t)ds->num_sms * 16 ? nrows : (int64_t)ds->num_sms * 16;
+    if (gr < 1) gr = 1;
+    const dim3 growsg((unsigned)gr);
     if (it == IMQ_I16) {
-      k_hyb_count<int16_t><<<gscan, 256, 0, st>>>(ha);
-      k_hyb_minc<int16_t><<<gscan, 256, 0, st>>>(ha);
+      if (any_rows) k_hyb_rows<int16_t><<<growsg, kRowThreads, 0, st>>>(ha);
+      if (any_cols) {
+        k_hyb_count<int16_t><<<gscan, 256, 0, st>>>(ha);
+        k_hyb_minc<int16_t><<<gscan, 256, 0, st>>>(ha);
+      }
     } else {
-      k_hyb_count<int32_t><<<gscan, 256, 0, st>>>(ha);
-      k_hyb_minc<int32_t><<<gscan, 256, 0, st>>>(ha);
+      if (any_rows) k_hyb_rows<int32_t><<<growsg, kRowThreads, 0, st>>>(ha);
+      if (any_cols) {
+        k_hyb_count<int32_t><<<gscan, 256, 0, st>>>(ha);
+        k_hyb_minc<int32_t><<<gscan, 256, 0, st>>>(ha);
+      }
     }
     k_hyb_hist<<<glines, 256, 0, st>>>(ha);
     k_hyb_choose<<<2, 1024, 0, st>>>(ha);

@@ -32,6 +32,18 @@
 
 static int64_t iabs64(int64_t v) { return v < 0 ? -v : v; }
 
+/* Li[t] = the largest level of entry t over the outer lines with fewer than tau out-of-range entries
+ * (1 when there is none); lev is n_out x n_in, row by row. */
+static void inner_levels(const int8_t *lev, const int64_t *cnt, int64_t n_out, int64_t n_in, int64_t tau,
+                         int32_t *Li) {
+  for (int64_t t = 0; t < n_in; ++t) Li[t] = 1;
+  for (int64_t o = 0; o < n_out; ++o) {
+    if (cnt[o] >= tau) continue;
+    for (int64_t t = 0; t < n_in; ++t)
+      if (lev[o * n_in + t] > Li[t]) Li[t] = lev[o * n_in + t];
+  }
+}
+
 /* The hybrid choice for one matrix seen as n_out outer lines of n_in inner entries, entry (o, t) at
  * X[o * s_out + t * s_in].  On entry Lo holds the outer lines' levels; on exit Lo and Li hold the levels
  * each line carries: Lo[o] unchanged for a line unpacked OUTER (its out-of-range count >= tau), else 1;
@@ -64,12 +76,8 @@ static int hybrid_choose(const int64_t *X, int64_t n_out, int64_t n_in, int64_t 
     if (!(tau == cmax + 1 || present[tau])) continue;
     unsigned __int128 me = 0, ke = 0;
     for (int64_t o = 0; o < n_out; ++o) me += (unsigned)(cnt[o] >= tau ? Lo[o] : 1);
-    for (int64_t t = 0; t < n_in; ++t) {
-      int li = 1;
-      for (int64_t o = 0; o < n_out; ++o)
-        if (cnt[o] < tau && lev[o * n_in + t] > li) li = lev[o * n_in + t];
-      ke += (unsigned)li;
-    }
+    inner_levels(lev, cnt, n_out, n_in, tau, Li);
+    for (int64_t t = 0; t < n_in; ++t) ke += (unsigned)Li[t];
     const unsigned __int128 cost = me * ke;
     if (first || cost < best) {
       best = cost;
@@ -77,12 +85,7 @@ static int hybrid_choose(const int64_t *X, int64_t n_out, int64_t n_in, int64_t 
       first = 0;
     }
   }
-  for (int64_t t = 0; t < n_in; ++t) {
-    int li = 1;
-    for (int64_t o = 0; o < n_out; ++o)
-      if (cnt[o] < best_tau && lev[o * n_in + t] > li) li = lev[o * n_in + t];
-    Li[t] = li;
-  }
+  inner_levels(lev, cnt, n_out, n_in, best_tau, Li);
   for (int64_t o = 0; o < n_out; ++o)
     if (cnt[o] < best_tau) Lo[o] = 1;
   free(lev);

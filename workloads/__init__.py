@@ -20,6 +20,9 @@ planted the way the page describes them (a few entries far outside the bulk, con
   wgrad      dY 16384x2048 Student-t(3) drawn as N(0,1)/sqrt(chi2_3/3); X 16384x512 N(0,1) with 4
              columns x50.  bf16.  Seed 4.
 
+Two more are built from the same pieces: the quantised-training triple of one linear layer (seed 5 for
+its weight) and heavy_tokens (seed 6), activations with heavy hitters in some channels AND some tokens.
+
 Matrices are returned as numpy arrays: float32 for 'f32', bfloat16 bit patterns in uint16 for 'bf16'.
 """
 from __future__ import annotations
@@ -29,9 +32,9 @@ from dataclasses import dataclass, field
 import numpy as np
 
 PER_TENSOR, PER_ROW, PER_COL = 0, 1, 2
-MIX, ROW_ROW, ROW_COL, COL_ROW, COL_COL = 0, 1, 2, 3, 4
+MIX, ROW_ROW, ROW_COL, COL_ROW, COL_COL, MIX_JOINT, HYBRID = 0, 1, 2, 3, 4, 5, 6
 STRATEGY_NAMES = {MIX: "mix", ROW_ROW: "row/row", ROW_COL: "row/col", COL_ROW: "col/row",
-                  COL_COL: "col/col"}
+                  COL_COL: "col/col", MIX_JOINT: "joint mix", HYBRID: "hybrid"}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -212,8 +215,27 @@ def training_triple(b: int = 5) -> list:
             mk("train_wgrad", dY, X, True, False)]
 
 
+def heavy_tokens(b: int = 8) -> list:
+    """Activations whose heavy hitters sit in a few channels AND a few tokens, the structure that pure
+    row or pure column unpacking both handle badly (the page prints no such workload; this is a
+    stand-in for it): X 2048 x 4096 N(0,1) with 6 channels x60 (as q_proj) and 4 tokens x60 outside
+    those channels, quantised per tensor; W 4096 x 4096 N(0, 0.02^2) per output channel, no planted
+    heavy hitters.  p = 0.95, beta = 15 and b = 8: the b-bit bound 127 is 8.5 beta, so only the planted
+    heavy hitters leave it.  bf16.  Seed 6."""
+    rng = np.random.default_rng(6)
+    X = _normal(rng, (2048, 4096))
+    ch = rng.choice(4096, 6, replace=False)
+    X[:, ch] *= np.float32(60)
+    rows = rng.choice(2048, 4, replace=False)
+    other = np.setdiff1d(np.arange(4096), ch)
+    X[np.ix_(rows, other)] *= np.float32(60)
+    W = _normal(rng, (4096, 4096), 0.02)
+    return [Gemm("heavy_tokens", _bf("X", X), _bf("W", W), False, False, PER_TENSOR, PER_COL, 0.95, 15, b,
+                 [MIX, HYBRID])]
+
+
 CONFIGS = {"tiny": tiny, "q_proj": q_proj, "mlp": mlp, "attention": attention, "wgrad": wgrad,
-           "training_triple": training_triple}
+           "training_triple": training_triple, "heavy_tokens": heavy_tokens}
 
 
 def rows_and_cols_case(rng, M, K, N, big=5000, dense_rows=1, dense_cols=1, scatter=0.02):
