@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libimq.so")
 
 # status codes
 IMQ_OK, IMQ_ERR_ARG, IMQ_ERR_NONFINITE, IMQ_ERR_RANGE = 0, 1, 2, 3
-IMQ_ERR_BUFFER, IMQ_ERR_TIMEOUT, IMQ_ERR_CUDA, IMQ_ERR_UNSUPPORTED = 4, 5, 6, 7
+IMQ_ERR_BUFFER, IMQ_ERR_TIMEOUT, IMQ_ERR_CUDA, IMQ_ERR_UNSUPPORTED, IMQ_ERR_PLAN = 4, 5, 6, 7, 8
 # dtypes
 IMQ_F32, IMQ_BF16, IMQ_I16, IMQ_I32, IMQ_I64 = 0, 1, 2, 3, 4
 # quantisation groups
@@ -88,6 +88,7 @@ SIGNATURES = {
     "imq_plan_groups": [_VP, ctypes.POINTER(imq_group), _I32, ctypes.POINTER(_I32)],
     "imq_plan_destroy": [_VP],
     "imq_unpack": [_VP, _VP, _VP, _VP, _VP, _VP],
+    "imq_rtn_quantize_unpack": [_VP, _VP, _I32, _I64, _F64, _I32, _VP, _VP, _VP],
     "imq_gemm_unpacked": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP],
     "imq_unpacked_gemm": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP, _SZ, _VP],
     "imq_device_status": [_VP, _I32],
@@ -270,6 +271,23 @@ def imq_unpack(plan: Plan, A: torch.Tensor, B: torch.Tensor, A_unp=None, B_unp_t
     _check(lib().imq_unpack(plan.handle, _ptr(A), _ptr(B), _ptr(A_unp), _ptr(B_unp_t), _stream(stream)),
            "imq_unpack")
     return A_unp, B_unp_t
+
+
+def imq_rtn_quantize_unpack(plan: Plan, X: torch.Tensor, p: float, beta: int, A_unp=None, deltaA=None,
+                            stream=None):
+    """Per-row RTN of X (M x K, float32 or bfloat16, row-major) fused with its unpacking into the plan's
+    A' layout.  Returns (A_unp, deltaA).  IMQ_ERR_PLAN in the device status word when an entry exceeds
+    the plan's column maxima (see include/imq.h)."""
+    I = plan.info
+    if X.dim() != 2 or X.stride(1) != 1 or tuple(X.shape) != (I["M"], I["K"]):
+        raise ValueError("X must be a row-major M x K matrix of the plan's shape")
+    if A_unp is None:
+        A_unp = torch.empty((I["M_unp"], I["K_unp"]), dtype=torch.int8, device=X.device)
+    if deltaA is None:
+        deltaA = torch.empty(I["M"], dtype=torch.float32, device=X.device)
+    _check(lib().imq_rtn_quantize_unpack(plan.handle, _ptr(X), _TORCH_TO_IMQ[X.dtype], _ld(X), float(p), int(beta),
+                                         _ptr(A_unp), _ptr(deltaA), _stream(stream)), "imq_rtn_quantize_unpack")
+    return A_unp, deltaA
 
 
 def _outputs(I, dev, C, c_dtype, Cf, want_int, want_f32):

@@ -184,6 +184,12 @@ imq_status imq_unpack(const imq_plan_t* plan, const void* A, const void* B, int8
   return imq::launch_unpack(plan, A, B, A_unp, B_unp_t, reinterpret_cast<cudaStream_t>(stream));
 }
 
+imq_status imq_rtn_quantize_unpack(const imq_plan_t* plan, const void* X, imq_dtype xt, int64_t ld, double p,
+                                   int32_t beta, int8_t* A_unp, float* deltaA, imq_stream_t stream) {
+  return imq::launch_rtn_quantize_unpack(plan, X, xt, ld, p, beta, A_unp, deltaA,
+                                         reinterpret_cast<cudaStream_t>(stream));
+}
+
 imq_status imq_gemm_unpacked(const imq_plan_t* plan, const int8_t* A_unp, const int8_t* B_unp_t, const float* deltaA,
                              imq_gran gA, const float* deltaB, imq_gran gB, void* Cint, imq_dtype ct, int64_t ldc,
                              float* Cf, int64_t ldcf, imq_stream_t stream) {
@@ -235,6 +241,7 @@ const char* imq_status_str(imq_status s) {
     case IMQ_ERR_TIMEOUT: return "bounded wait timed out in a kernel";
     case IMQ_ERR_CUDA: return "CUDA runtime error";
     case IMQ_ERR_UNSUPPORTED: return "unsupported input";
+    case IMQ_ERR_PLAN: return "input not covered by the plan";
   }
   return "unknown status";
 }

@@ -301,6 +301,33 @@ __device__ __forceinline__ void warp_count(uint32_t* base, uint32_t key, bool ac
   if ((int)(threadIdx.x & 31) == leader) atomicAdd(base + key, (uint32_t)__popc(peers));
 }
 
+// Digit l (base 2^bm1, sign-magnitude) of 16 int16 entries held as 8 words (two entries per word, low
+// half first), as 16 bytes in entry order.  |entry| per half without a carry between halves; the
+// digit's bits are masked, then shifted down within each half; a byte permute gathers the four digits of
+// two words; negative entries' digits are negated byte-wise as (0x80808080 - d) ^ 0x80808080 (a digit
+// is at most 127, so no byte borrows).  Digits with l * bm1 >= 16 are zero for int16 magnitudes.
+__device__ __forceinline__ uint4 digits16_i16(const uint32_t (&w)[8], int l, int bm1) {
+  const int sh = l * bm1;
+  if (sh >= 16) return make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t m2 = ((((1u << bm1) - 1u) << sh) & 0xFFFFu) * 0x00010001u;
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t d[2], S[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t ww = w[2 * q + h];
+      const uint32_t sgn = (ww >> 15) & 0x00010001u;
+      S[h] = sgn * 0xFFFFu;
+      d[h] = (((ww ^ S[h]) + sgn) & m2) >> sh;
+    }
+    const uint32_t pd = __byte_perm(d[0], d[1], 0x6420), neg = __byte_perm(S[0], S[1], 0x6420);
+    const uint32_t nd = (0x80808080u - pd) ^ 0x80808080u;
+    o[q] = (pd & ~neg) | (nd & neg);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Number of base-2^(b-1) digits of m (>= 1).
 __device__ __forceinline__ int32_t level_of(uint32_t m, int32_t bm1) {
   if (m == 0) return 1;

@@ -94,6 +94,9 @@ struct imq_plan {
 };
 
 namespace imq {
+// Fused per-row RTN of X and unpack into the plan's A' layout (rtn.cu).
+imq_status launch_rtn_quantize_unpack(const imq_plan_t* pl, const void* X, imq_dtype xt, int64_t ld, double p,
+                                      int32_t beta, int8_t* A_unp, float* delta, cudaStream_t stream);
 imq_status launch_unpack(const imq_plan_t* pl, const void* A, const void* B, int8_t* Au, int8_t* Bu,
                          cudaStream_t stream);
 imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu, const float* dA,

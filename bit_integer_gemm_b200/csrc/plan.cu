@@ -876,11 +876,14 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   const bool have_max = a_rowmax && a_colmax && b_rowmax && b_colmax;
   const int32_t* lmx[4] = {mx[0], mx[1], mx[2], mx[3]};  // the maxima the levels are computed from
   if (have_max) {
-    // the caller's maxima are read in place (only the level kernel below reads them)
+    // the caller's maxima are read in place by the kernels below; A's column maxima are also kept in
+    // the plan (the fused quantise-and-unpack path checks new activations against them)
     lmx[0] = a_rowmax;
     lmx[1] = a_colmax;
     lmx[2] = b_rowmax;
     lmx[3] = b_colmax;
+    if (K > 0 && cudaMemcpyAsync(mx[1], a_colmax, (size_t)K * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return fail(IMQ_ERR_CUDA);
   } else {
     // A stored M x K (or K x M when transposed); B stored K x N (or N x K)
     imq_status e = transA ? launch_line_max(A, it, K, M, lda, mx[1], mx[0], st)

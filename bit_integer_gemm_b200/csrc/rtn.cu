@@ -952,4 +952,186 @@ imq_status launch_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t
              : run_rows_noalloc<uint32_t, false>(x, rows, cols, ld, p, beta, Xint, ldq, delta, qval, rowmax, colmax, ds, st);
 }
 
+// ------------------------------------------------------------------------------------------------
+// Fused per-row RTN and unpack (imq_rtn_quantize_unpack).  One warp per row of X: the row is staged in
+// shared memory, its percentile selected and its values quantised (as in k_rtn_rows) into an int16 row
+// that never leaves shared memory; the warp then writes the row's unpacked line in the plan's layout (a
+// 16-position block the plan marked contiguous is one digit plane of 16 consecutive entries, computed
+// from two 16-byte reads; any other block is gathered entry by entry).  Each quantised entry is checked
+// against the plan's maximum |A[:, t]|: one above it may need a digit the layout does not hold, or break
+// the plan's accumulator bound, and sets IMQ_ERR_PLAN.
+// ------------------------------------------------------------------------------------------------
+namespace {
+struct FusedArgs {
+  int64_t rows, cols, ld;  // X, row-major
+  int64_t K_unp;
+  const int32_t* tK;
+  const int8_t* lAk;
+  const int32_t* blk16;
+  const int32_t* amax;  // [cols] max |A[:, t]| of the plan
+  int32_t bm1;
+  unsigned long long krank;
+  int32_t beta;
+  float* delta;
+  int8_t* out;
+  int32_t* status;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restrict__ X, FusedArgs f, int nwarps) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  const int64_t row_bytes = (f.cols * (int64_t)sizeof(T) + 15) / 16 * 16;
+  const int64_t q_bytes = (f.cols * 2 + 31) / 32 * 32;
+  __shared__ uint32_t hist_all[kThreads / 32][256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (warp >= nwarps) return;
+  T* row = reinterpret_cast<T*>(dsm + (int64_t)warp * (row_bytes + q_bytes));
+  int16_t* qv = reinterpret_cast<int16_t*>(dsm + (int64_t)warp * (row_bytes + q_bytes) + row_bytes);
+  uint32_t* hist = hist_all[warp];
+  constexpr int V = 16 / sizeof(T);
+  const int n = (int)f.cols;
+  const bool vec = (f.cols % V == 0) && (f.ld % V == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  const int64_t nchunk = f.K_unp / 16;
+  for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < f.rows; r += (int64_t)gridDim.x * nwarps) {
+    const T* xr = X + r * f.ld;
+    if (vec) {
+      const uint4* src = reinterpret_cast<const uint4*>(xr);
+      uint4* dst = reinterpret_cast<uint4*>(row);
+      for (int c = lane; c < n / V; c += 32) dst[c] = __ldcs(src + c);
+    } else {
+      for (int c = lane; c < n; c += 32) row[c] = xr[c];
+    }
+    __syncwarp();
+    uint32_t mk, bad;
+    warp_key_stats(row, n, &mk, &bad);
+    const float q = Key<T>::from_key(select_key(row, n, f.krank, hist));
+    float s, dl;
+    scale_from_q(q, Key<T>::from_key(mk), f.beta, &s, &dl);
+    if (lane == 0) f.delta[r] = dl;
+    if (bad) {
+      if (lane == 0) set_status(f.status, IMQ_ERR_NONFINITE);
+      continue;
+    }
+    // quantise into the int16 row, 8 entries per lane and step where the row allows, checking coverage
+    bool over = false;
+    const int n8 = (n % 8 == 0) ? n / 8 : 0;
+    for (int g = lane; g < n8; g += 32) {
+      const int4 m0 = *reinterpret_cast<const int4*>(f.amax + g * 8);
+      const int4 m1 = *reinterpret_cast<const int4*>(f.amax + g * 8 + 4);
+      const int32_t mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+      int32_t v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[j] = quant_val<true>(Key<T>::value(row[g * 8 + j]), s, f.status, 0);
+        over |= (v[j] < 0 ? -v[j] : v[j]) > mm[j];
+      }
+      uint32_t pk[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) pk[j] = ((uint32_t)v[2 * j] & 0xFFFFu) | ((uint32_t)v[2 * j + 1] << 16);
+      *reinterpret_cast<uint4*>(qv + g * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+    for (int c = n8 * 8 + lane; c < n; c += 32) {
+      const int32_t v = quant_val<true>(Key<T>::value(row[c]), s, f.status, 0);
+      over |= (v < 0 ? -v : v) > f.amax[c];
+      qv[c] = (int16_t)v;
+    }
+    if (over) set_status(f.status, IMQ_ERR_PLAN);
+    __syncwarp();
+    // the unpacked line of row r, 16 inner positions per lane and step
+    int8_t* orow = f.out + r * f.K_unp;
+    for (int64_t c = lane; c < nchunk; c += 32) {
+      const int32_t t0 = f.blk16[c];
+      const int64_t p = c * 16;
+      uint4 o;
+      if (t0 >= 0) {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(qv + t0), w1 = *reinterpret_cast<const uint4*>(qv + t0 + 8);
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        o = digits16_i16(w, f.lAk[p], f.bm1);
+      } else {
+        const int4* tq = reinterpret_cast<const int4*>(f.tK + p);
+        const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
+        const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
+                                tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
+        const int4 lq = *reinterpret_cast<const int4*>(f.lAk + p);
+        const int8_t* ll = reinterpret_cast<const int8_t*>(&lq);
+        uint32_t w[4];
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          uint32_t packed = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = qd * 4 + k;
+            const int32_t d = tt[e] >= 0 ? digit_of((int32_t)qv[tt[e]], ll[e], f.bm1) : 0;
+            packed |= ((uint32_t)(uint8_t)(int8_t)d) << (8 * k);
+          }
+          w[qd] = packed;
+        }
+        o = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      *reinterpret_cast<uint4*>(orow + p) = o;
+    }
+    __syncwarp();
+  }
+}
+
+template <typename T>
+imq_status run_rtn_unpack(const T* X, const FusedArgs& f, DeviceState* ds, cudaStream_t st) {
+  const int64_t row_bytes = (f.cols * (int64_t)sizeof(T) + 15) / 16 * 16;
+  const int64_t q_bytes = (f.cols * 2 + 31) / 32 * 32;
+  const int64_t per_warp = row_bytes + q_bytes;
+  constexpr size_t kBudget = 200 * 1024;
+  if ((size_t)per_warp > kBudget) return IMQ_ERR_UNSUPPORTED;
+  int nwarps = (int)(kBudget / 2 / per_warp);  // two CTAs per SM where the rows allow
+  if (nwarps < 1) nwarps = 1;
+  if (nwarps > kThreads / 32) nwarps = kThreads / 32;
+  const size_t smem = (size_t)nwarps * per_warp;
+  int per_sm = (int)(kBudget / (smem + 9 * 1024));
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 4) per_sm = 4;
+  const int64_t blocks = (f.rows + nwarps - 1) / nwarps;
+  const int64_t grid = blocks < (int64_t)ds->num_sms * per_sm ? blocks : (int64_t)ds->num_sms * per_sm;
+  IMQ_CUDA_TRY(cudaFuncSetAttribute(k_rtn_unpack_rows<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  k_rtn_unpack_rows<T><<<(unsigned)grid, kThreads, smem, st>>>(X, f, nwarps);
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+}  // namespace
+
+imq_status launch_rtn_quantize_unpack(const imq_plan_t* pl, const void* X, imq_dtype xt, int64_t ld, double p,
+                                      int32_t beta, int8_t* A_unp, float* delta, cudaStream_t st) {
+  if (!pl) return IMQ_ERR_ARG;
+  const imq_plan_info& I = pl->info;
+  if (I.dir_a & IMQ_DIR_OUTER) return IMQ_ERR_ARG;  // A's lines would depend on the new values
+  if (xt != IMQ_F32 && xt != IMQ_BF16) return IMQ_ERR_ARG;
+  if (ld < I.K || !(p > 0.0 && p <= 1.0) || beta < 1 || beta > (1 << 24)) return IMQ_ERR_ARG;
+  if (I.M > 0 && !delta) return IMQ_ERR_ARG;
+  if (I.M > 0 && I.K > 0 && (!X || !A_unp)) return IMQ_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(A_unp) & 15) != 0) return IMQ_ERR_ARG;
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  if (I.M == 0) return IMQ_OK;
+  if (I.K == 0) {
+    // empty rows: q = max = 0, so Delta = 1, and A' has no columns
+    k_fill_f32<<<1, 256, 0, st>>>(delta, I.M, 1.0f);
+    return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+  }
+  FusedArgs f;
+  f.rows = I.M;
+  f.cols = I.K;
+  f.ld = ld;
+  f.K_unp = I.K_unp;
+  f.tK = pl->tK;
+  f.lAk = pl->lAk;
+  f.blk16 = pl->blk16;
+  f.amax = pl->max_a_col;
+  f.bm1 = I.b - 1;
+  f.krank = (unsigned long long)nearest_rank(I.K, p);
+  f.beta = beta;
+  f.delta = delta;
+  f.out = A_unp;
+  f.status = ds->status;
+  if (xt == IMQ_BF16) return run_rtn_unpack<uint16_t>(static_cast<const uint16_t*>(X), f, ds, st);
+  return run_rtn_unpack<uint32_t>(static_cast<const uint32_t*>(X), f, ds, st);
+}
+
 }  // namespace imq

@@ -53,7 +53,8 @@ typedef enum {
   IMQ_ERR_BUFFER = 4,      /* workspace smaller than imq_plan_info.workspace_bytes                      */
   IMQ_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out                                    */
   IMQ_ERR_CUDA = 6,        /* a CUDA runtime call failed                                                 */
-  IMQ_ERR_UNSUPPORTED = 7  /* legal input outside what the kernels implement (see imq_plan)             */
+  IMQ_ERR_UNSUPPORTED = 7, /* legal input outside what the kernels implement (see imq_plan)             */
+  IMQ_ERR_PLAN = 8         /* imq_rtn_quantize_unpack: a quantised entry above the plan's max |A[:, t]| */
 } imq_status;
 
 typedef enum { IMQ_F32 = 0, IMQ_BF16 = 1, IMQ_I16 = 2, IMQ_I32 = 3, IMQ_I64 = 4 } imq_dtype;
@@ -285,6 +286,34 @@ imq_status imq_plan_destroy(imq_plan_t *plan);
  */
 imq_status imq_unpack(const imq_plan_t *plan, const void *A, const void *B,
                       int8_t *A_unp, int8_t *B_unp_t, imq_stream_t stream);
+
+/*
+ * imq_rtn_quantize_unpack -- per-row RTN of X fused with its unpacking into the A' layout of an existing
+ * plan, for inference with a weight that is quantised, planned and unpacked once (B'^T kept by the
+ * caller) while the activations change ("Approach" and "Key results": quantised linear layers at
+ * inference; the page does not describe caching, this is the library's way of not re-unpacking a
+ * static weight).  The integer activations are never written to memory: one warp per row stages the
+ * row, selects its percentile, quantises it (exactly as imq_rtn_quantize with IMQ_PER_ROW and I16
+ * output) in shared memory and writes the row's unpacked line.
+ *   Coverage: the plan stays valid for X when every quantised entry satisfies |x_int[i,t]| <= the
+ *   maximum |A[:, t]| the plan was made from (its a_colmax, or the column maxima of its A): the
+ *   levels, the inner layout and the accumulator bound then all hold and imq_gemm_unpacked with the
+ *   kept B'^T gives X_int * B exactly.  A larger entry sets IMQ_ERR_PLAN in the device status word;
+ *   the caller then plans again.  To cover later batches, plan with widened column maxima (any values
+ *   >= the true ones; the plan's levels and bound follow the maxima it is given).
+ * plan    a plan whose A is INNER or not unpacked (imq_plan_info.dir_a of IMQ_DIR_INNER or
+ *         IMQ_DIR_NONE; OUTER rows would depend on the new values): IMQ_ERR_ARG otherwise.  Its M x K
+ *         is X's shape.
+ * X       device, M x K row-major with leading dimension ld (>= K), dtype xt (F32 or BF16).
+ * A_unp   device int8, M_unp (= M) x K_unp, 16-byte aligned, written in full.
+ * deltaA  device fp32[M]: the dequantisation step of every row.
+ * Errors: IMQ_ERR_ARG at once; IMQ_ERR_NONFINITE, IMQ_ERR_RANGE (an entry above 32767), IMQ_ERR_PLAN
+ *         through the device status word.  IMQ_ERR_UNSUPPORTED when a row (input and int16 copy) does
+ *         not fit in shared memory (K above about 33 000 for BF16).  Asynchronous; allocates nothing.
+ */
+imq_status imq_rtn_quantize_unpack(const imq_plan_t *plan, const void *X, imq_dtype xt, int64_t ld,
+                                   double p, int32_t beta, int8_t *A_unp, float *deltaA,
+                                   imq_stream_t stream);
 
 /*
  * imq_gemm_unpacked -- the low-bit GEMM on already unpacked operands with the fold-back epilogue:

@@ -588,3 +588,26 @@ def test_layout_follows_documented_order():
                         assert lines[s[k * L]] == L
                         seen.append((L, int(s[k * L])))
                 assert seen == sorted(seen) and len(seen) == lines.size
+
+
+def test_cached_plan_is_exact_for_covered_inputs():
+    """A plan made from one A serves any other A' whose entries stay within the first one's column
+    maxima, |A'[i,t]| <= max_i |A[i,t]| (what the fused quantise-and-unpack path checks against a plan
+    kept with an unpacked weight): the levels, the inner layout and the bound all still hold, so the
+    unpacked product with the kept B' is exact.  Random inputs, A not unpacked OUTER (A's rows are then
+    single lines whose layout does not depend on the new values)."""
+    rng = np.random.default_rng(31)
+    checked = 0
+    for case in range(400):
+        M, K, N = (int(x) for x in rng.integers(1, 12, size=3))
+        b = int(rng.integers(2, 9))
+        A, B = workloads.random_case(rng, M, K, N, big=int(rng.choice([60, 3000])), frac=0.15)
+        pl = oracle.plan(A, B, b, oracle.COL_ROW if case % 2 else oracle.MIX)
+        if pl.dir_a & oracle.DIR_OUTER:
+            continue
+        cmax = np.abs(A).max(axis=0)
+        A2 = rng.integers(-cmax, cmax + 1, size=(M, K)).astype(np.int64)  # within the column maxima
+        Au, Bu = oracle.unpack(pl, A2, B)
+        assert np.array_equal(oracle.unpacked_gemm(pl, Au, Bu), A2 @ B), case
+        checked += 1
+    assert checked > 150
