@@ -977,21 +977,42 @@ struct FusedArgs {
   int32_t* status;
 };
 
+// Bytes of shared memory one warp of k_rtn_unpack_rows uses: the staged row and, for fp32 input, a
+// separate int16 row (a bf16 row is quantised in place: each lane reads its 8 entries before writing
+// their 8 int16 values at the same address).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restrict__ X, FusedArgs f, int nwarps) {
+__host__ __device__ constexpr int64_t fused_warp_bytes(int64_t cols) {
+  return (cols * (int64_t)sizeof(T) + 15) / 16 * 16 + (sizeof(T) == 2 ? 0 : (cols * 2 + 31) / 32 * 32);
+}
+constexpr int64_t kFusedMetaMaxChunks = 4096;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restrict__ X, FusedArgs f, int nwarps,
+                                                              int meta_smem) {
   extern __shared__ __align__(16) unsigned char dsm[];
   const int64_t row_bytes = (f.cols * (int64_t)sizeof(T) + 15) / 16 * 16;
-  const int64_t q_bytes = (f.cols * 2 + 31) / 32 * 32;
+  const int64_t wbytes = fused_warp_bytes<T>(f.cols);
   __shared__ uint32_t hist_all[kThreads / 32][256];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t nchunk = f.K_unp / 16;
+  // [rows of nwarps warps][block starts, int32 x nchunk][first inner levels, int8 x nchunk]
+  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)nwarps * wbytes);
+  int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);
+  if (meta_smem) {
+    for (int64_t c = tid; c < nchunk; c += blockDim.x) {
+      s_blk[c] = f.blk16[c];
+      s_lk0[c] = f.lAk[c * 16];
+    }
+    __syncthreads();
+  }
   if (warp >= nwarps) return;
-  T* row = reinterpret_cast<T*>(dsm + (int64_t)warp * (row_bytes + q_bytes));
-  int16_t* qv = reinterpret_cast<int16_t*>(dsm + (int64_t)warp * (row_bytes + q_bytes) + row_bytes);
+  T* row = reinterpret_cast<T*>(dsm + (int64_t)warp * wbytes);
+  int16_t* qv = sizeof(T) == 2 ? reinterpret_cast<int16_t*>(row)
+                               : reinterpret_cast<int16_t*>(dsm + (int64_t)warp * wbytes + row_bytes);
   uint32_t* hist = hist_all[warp];
   constexpr int V = 16 / sizeof(T);
   const int n = (int)f.cols;
   const bool vec = (f.cols % V == 0) && (f.ld % V == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
-  const int64_t nchunk = f.K_unp / 16;
   for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < f.rows; r += (int64_t)gridDim.x * nwarps) {
     const T* xr = X + r * f.ld;
     if (vec) {
@@ -1016,13 +1037,23 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
     bool over = false;
     const int n8 = (n % 8 == 0) ? n / 8 : 0;
     for (int g = lane; g < n8; g += 32) {
+      uint32_t wd[8];
+      {
+        const uint4 w0 = reinterpret_cast<const uint4*>(row + g * 8)[0];
+        wd[0] = w0.x; wd[1] = w0.y; wd[2] = w0.z; wd[3] = w0.w;
+        if (sizeof(T) == 4) {
+          const uint4 w1 = reinterpret_cast<const uint4*>(row + g * 8)[1];
+          wd[4] = w1.x; wd[5] = w1.y; wd[6] = w1.z; wd[7] = w1.w;
+        }
+      }
       const int4 m0 = *reinterpret_cast<const int4*>(f.amax + g * 8);
       const int4 m1 = *reinterpret_cast<const int4*>(f.amax + g * 8 + 4);
       const int32_t mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
       int32_t v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        v[j] = quant_val<true>(Key<T>::value(row[g * 8 + j]), s, f.status, 0);
+        const T e = sizeof(T) == 2 ? (T)((wd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) : (T)wd[j];
+        v[j] = quant_val<true>(Key<T>::value(e), s, f.status, 0);
         over |= (v[j] < 0 ? -v[j] : v[j]) > mm[j];
       }
       uint32_t pk[4];
@@ -1040,13 +1071,13 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
     // the unpacked line of row r, 16 inner positions per lane and step
     int8_t* orow = f.out + r * f.K_unp;
     for (int64_t c = lane; c < nchunk; c += 32) {
-      const int32_t t0 = f.blk16[c];
+      const int32_t t0 = meta_smem ? s_blk[c] : f.blk16[c];
       const int64_t p = c * 16;
       uint4 o;
       if (t0 >= 0) {
         const uint4 w0 = *reinterpret_cast<const uint4*>(qv + t0), w1 = *reinterpret_cast<const uint4*>(qv + t0 + 8);
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        o = digits16_i16(w, f.lAk[p], f.bm1);
+        o = digits16_i16(w, meta_smem ? s_lk0[c] : f.lAk[p], f.bm1);
       } else {
         const int4* tq = reinterpret_cast<const int4*>(f.tK + p);
         const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
@@ -1076,22 +1107,25 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
 
 template <typename T>
 imq_status run_rtn_unpack(const T* X, const FusedArgs& f, DeviceState* ds, cudaStream_t st) {
-  const int64_t row_bytes = (f.cols * (int64_t)sizeof(T) + 15) / 16 * 16;
-  const int64_t q_bytes = (f.cols * 2 + 31) / 32 * 32;
-  const int64_t per_warp = row_bytes + q_bytes;
+  const int64_t per_warp = fused_warp_bytes<T>(f.cols);
+  const int64_t nchunk = f.K_unp / 16;
+  const int meta_smem = nchunk <= kFusedMetaMaxChunks ? 1 : 0;
+  const size_t meta = meta_smem ? (size_t)nchunk * 5 : 0;
   constexpr size_t kBudget = 200 * 1024;
-  if ((size_t)per_warp > kBudget) return IMQ_ERR_UNSUPPORTED;
-  int nwarps = (int)(kBudget / 2 / per_warp);  // two CTAs per SM where the rows allow
-  if (nwarps < 1) nwarps = 1;
+  if ((size_t)per_warp + meta > kBudget) return IMQ_ERR_UNSUPPORTED;
+  // eight warps per CTA while their rows fit in about a third of the budget (several CTAs per SM)
+  int nwarps = (int)((kBudget / 3 - meta) / per_warp);
+  if (nwarps < 1) nwarps = (int)((kBudget - meta) / per_warp) >= 1 ? 1 : 0;
+  if (nwarps < 1) return IMQ_ERR_UNSUPPORTED;
   if (nwarps > kThreads / 32) nwarps = kThreads / 32;
-  const size_t smem = (size_t)nwarps * per_warp;
+  const size_t smem = (size_t)nwarps * per_warp + meta;
   int per_sm = (int)(kBudget / (smem + 9 * 1024));
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 4) per_sm = 4;
   const int64_t blocks = (f.rows + nwarps - 1) / nwarps;
   const int64_t grid = blocks < (int64_t)ds->num_sms * per_sm ? blocks : (int64_t)ds->num_sms * per_sm;
   IMQ_CUDA_TRY(cudaFuncSetAttribute(k_rtn_unpack_rows<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_rtn_unpack_rows<T><<<(unsigned)grid, kThreads, smem, st>>>(X, f, nwarps);
+  k_rtn_unpack_rows<T><<<(unsigned)grid, kThreads, smem, st>>>(X, f, nwarps, meta_smem);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 }  // namespace
