@@ -186,6 +186,22 @@ class Path:
         self.info = None
         self.launches = 0
 
+    def _workspace(self, I):
+        """A' and B'^T views of one workspace (1024-byte aligned), rebuilt only when the plan's sizes
+        change."""
+        key = (I["M_unp"], I["N_unp"], I["K_unp"])
+        if getattr(self, "_ws_key", None) != key:
+            need = I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048
+            if self.ws is None or self.ws.numel() < need:
+                self.ws = self.torch.empty(need, dtype=self.torch.int8, device=self.X.device)
+            na = I["M_unp"] * I["K_unp"]
+            a_off = (-self.ws.data_ptr()) % 1024
+            b_off = a_off + (na + 1023) // 1024 * 1024
+            self._views = (self.ws[a_off:a_off + na].view(I["M_unp"], I["K_unp"]),
+                           self.ws[b_off:b_off + I["N_unp"] * I["K_unp"]].view(I["N_unp"], I["K_unp"]))
+            self._ws_key = key
+        return self._views
+
     def prepare_cache(self):
         """Cached-weight mode, before any timing: W quantised per output channel, the plan made with
         the activations' column maxima widened to the largest value of the same level (R^L - 1, so later
@@ -238,14 +254,7 @@ class Path:
                              want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True)
         plan = imq.imq_plan(self.Xint, self.Wint, g.b, self.strategy, transB=True, maxes=self.mx)
         I = plan.info
-        if self.ws is None or self.ws.numel() < I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048:
-            self.ws = self.torch.empty(I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048,
-                                       dtype=self.torch.int8, device=self.X.device)
-        na = I["M_unp"] * I["K_unp"]
-        a_off = (-self.ws.data_ptr()) % 1024
-        b_off = a_off + (na + 1023) // 1024 * 1024
-        Au = self.ws[a_off:a_off + na].view(I["M_unp"], I["K_unp"])
-        Bu = self.ws[b_off:b_off + I["N_unp"] * I["K_unp"]].view(I["N_unp"], I["K_unp"])
+        Au, Bu = self._workspace(I)
         imq.imq_unpack(plan, self.Xint, self.Wint, A_unp=Au, B_unp_t=Bu)
         if gemm_events is not None:
             gemm_events[0].record()

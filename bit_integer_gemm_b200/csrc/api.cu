@@ -2,7 +2,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -48,27 +50,43 @@ imq_status device_state(DeviceState** out) {
 
 
 namespace {
-// Block of 32 x 8 threads: x = 32 consecutive entries (coalesced), y = a slice of the partials; the
-// eight slices are combined in shared memory.
-__global__ void __launch_bounds__(256) k_reduce_max(const int32_t* __restrict__ part, int64_t nparts, int64_t n,
-                                                    int32_t* __restrict__ out) {
-  __shared__ int32_t red[8][33];
+std::mutex g_smem_mu;
+std::map<std::pair<int, const void*>, size_t> g_smem_set;  // (device, kernel) -> limit already set
+}  // namespace
+
+cudaError_t ensure_smem(const void* fn, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  size_t& have = g_smem_set[{dev, fn}];
+  if (have >= bytes && have > 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
+
+namespace {
+// Block of 32 x 32 threads: x = 32 consecutive entries (coalesced), y = one of 32 slices of the partials
+// (four loads of a thread in flight); the slices are combined in shared memory.
+__global__ void __launch_bounds__(1024) k_reduce_max(const int32_t* __restrict__ part, int64_t nparts, int64_t n,
+                                                     int32_t* __restrict__ out) {
+  __shared__ int32_t red[32][33];
   const int64_t i = (int64_t)blockIdx.x * 32 + threadIdx.x;
   int32_t m = 0;
   if (i < n) {
     int64_t p = threadIdx.y;
-#pragma unroll 4
-    for (; p + 24 < nparts; p += 32) {
-      const int32_t a = __ldcs(part + p * n + i), b = __ldcs(part + (p + 8) * n + i);
-      const int32_t c = __ldcs(part + (p + 16) * n + i), d = __ldcs(part + (p + 24) * n + i);
+    for (; p + 96 < nparts; p += 128) {
+      const int32_t a = __ldcs(part + p * n + i), b = __ldcs(part + (p + 32) * n + i);
+      const int32_t c = __ldcs(part + (p + 64) * n + i), d = __ldcs(part + (p + 96) * n + i);
       m = max(max(m, a), max(b, max(c, d)));
     }
-    for (; p < nparts; p += 8) m = max(m, __ldcs(part + p * n + i));
+    for (; p < nparts; p += 32) m = max(m, __ldcs(part + p * n + i));
   }
   red[threadIdx.y][threadIdx.x] = m;
   __syncthreads();
   if (threadIdx.y == 0 && i < n) {
-    for (int y = 1; y < 8; ++y) m = max(m, red[y][threadIdx.x]);
+    for (int y = 1; y < 32; ++y) m = max(m, red[y][threadIdx.x]);
     out[i] = m;
   }
 }
@@ -80,7 +98,7 @@ imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int
   imq_status s = device_state(&ds);
   if (s != IMQ_OK) return s;
   (void)ds;
-  k_reduce_max<<<(unsigned)((n + 31) / 32), dim3(32, 8), 0, st>>>(part, nparts, n, out);
+  k_reduce_max<<<(unsigned)((n + 31) / 32), dim3(32, 32), 0, st>>>(part, nparts, n, out);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 

@@ -663,7 +663,7 @@ imq_status launch_k_gemm(int grid, const CUtensorMap& tmA, const CUtensorMap& tm
                          cudaStream_t st) {
   auto kern = k_gemm<kWide, kPair>;
   const size_t smem = Geo<kPair>::kBytes;
-  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)grid);

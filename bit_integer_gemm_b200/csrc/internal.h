@@ -21,6 +21,10 @@ struct DeviceState {
   bool init = false;
 };
 imq_status device_state(DeviceState** out);
+// Raises the dynamic shared-memory limit of kernel `fn` on the current device to at least `bytes`.  The
+// attribute call costs microseconds of host time, so it is made only when no earlier call on this device
+// already set a limit at least as large.
+cudaError_t ensure_smem(const void* fn, size_t bytes);
 // out[i] = max over p < nparts of part[p * n + i] (int32, non-negative); nparts may be 0 (out = 0).
 imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st);
 

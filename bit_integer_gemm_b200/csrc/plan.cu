@@ -18,6 +18,7 @@
 //                  one CTA per OUTER level class (stable compaction of the lines of that level into groups)
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -36,7 +37,15 @@ struct Summary {
   unsigned int joint[kLv][kLv];
   unsigned long long bound_lo, bound_hi;
   int32_t status;  // copy of the device status word taken in stream order
-  int32_t pad_;
+  uint32_t done;   // blocks of k_levels that have added their part
+};
+
+// The summary as the host receives it: pinned host memory that k_levels' last block writes directly (a
+// mapped pointer), then `seq`, which the host waits for.  No copy is enqueued and the stream is not
+// synchronised: the host sees the summary as soon as it exists.
+struct HostSummary {
+  Summary s;
+  uint32_t seq;
 };
 
 // ------------------------------------------------------------------------------------------------
@@ -90,6 +99,8 @@ struct LevelArgs {
   int32_t bm1;
   Summary* sum;
   const int32_t* status;  // the device status word, copied into the summary by block 0
+  HostSummary* hsum;      // device address of the mapped host copy
+  uint32_t seq;           // written to hsum->seq once hsum->s is complete
 };
 
 __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
@@ -182,6 +193,23 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
     if ((&hist[0][0])[i]) atomicAdd(&a.sum->hist[0][0] + i, (&hist[0][0])[i]);
   for (int i = tid; i < kLv * kLv; i += 256)
     if ((&joint[0][0])[i]) atomicAdd(&a.sum->joint[0][0] + i, (&joint[0][0])[i]);
+  // the last block to finish copies the completed summary to the host, then publishes `seq`
+  __shared__ bool last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(&a.sum->done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const volatile uint32_t* src = reinterpret_cast<const volatile uint32_t*>(a.sum);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(&a.hsum->s);
+  for (int i = tid; i < (int)(sizeof(Summary) / 4); i += blockDim.x) dst[i] = src[i];
+  __threadfence_system();
+  __syncthreads();
+  if (tid == 0) {
+    *reinterpret_cast<volatile uint32_t*>(&a.hsum->seq) = a.seq;
+    __threadfence_system();
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -651,7 +679,7 @@ struct OuterClass {
 // The OUTER layout of one matrix: classes of lines of equal level, each a run of groups of G unpacked
 // lines.  One CTA per class.
 struct OuterJob {
-  const OuterClass* cls;
+  int cls0;  // first class of this matrix in the class table
   int ncls;
   const int8_t* lv;
   int64_t n;
@@ -691,12 +719,24 @@ __device__ void outer_map_class(const OuterClass c, const int8_t* __restrict__ l
   }
 }
 
+// The segment, class and group tables of a plan.  They travel inside the launch's parameters when the
+// segments fit (the usual case: a separate upload would cost a copy and an event on the host); the
+// parameter block is read in place (__grid_constant__).
+constexpr int kParamSegs = 48;
+struct MapsTables {
+  InnerSeg segs[kParamSegs];
+  OuterClass cls[2 * kLv];
+  InnerGroup grps[IMQ_MAX_GROUPS];
+};
+
 // Stage 2 of a plan in one launch: blocks [0, ngrp) build the inner map of one exponent group each, the
 // next a.ncls blocks one OUTER class of A each, the rest one OUTER class of B each.
 struct MapsArgs {
+  int inline_tables;       // 1: the tables are `t` below, 0: the device copies at grps / segs / cls
   const InnerGroup* grps;
   int ngrp;
   const InnerSeg* segs;
+  const OuterClass* cls;
   const int8_t* lva;
   const int8_t* lvb;
   int a_inner, b_inner;
@@ -706,26 +746,34 @@ struct MapsArgs {
   int8_t* lBk;
   int32_t* blk16;
   OuterJob a, b;
+  MapsTables t;
 };
+// kernel parameters above 4 KB need CUDA 12.1 or later; the limit there is 32 764 bytes
+static_assert(sizeof(MapsArgs) <= 32764, "plan tables exceed the kernel parameter limit");
 
-__global__ void __launch_bounds__(1024) k_plan_maps(MapsArgs m) {
+__global__ void __launch_bounds__(1024) k_plan_maps(const __grid_constant__ MapsArgs m) {
+  const InnerSeg* segs = m.inline_tables ? m.t.segs : m.segs;
+  const OuterClass* cls = m.inline_tables ? m.t.cls : m.cls;
+  const InnerGroup* grps = m.inline_tables ? m.t.grps : m.grps;
   const int bx = (int)blockIdx.x;
   if (bx < m.ngrp) {
-    inner_map_group(m.grps[bx], m.segs, m.lva, m.lvb, m.a_inner, m.b_inner, m.K, m.tK, m.lAk, m.lBk, m.blk16);
+    inner_map_group(grps[bx], segs, m.lva, m.lvb, m.a_inner, m.b_inner, m.K, m.tK, m.lAk, m.lBk, m.blk16);
     return;
   }
   const int ob = bx - m.ngrp;
   const bool is_a = ob < m.a.ncls;
   const OuterJob& j = is_a ? m.a : m.b;
   const int ci = is_a ? ob : ob - m.a.ncls;
-  outer_map_class(j.cls[ci], j.lv, j.n, j.G, j.pos, j.src, j.grpL, j.grpN);
+  outer_map_class(cls[j.cls0 + ci], j.lv, j.n, j.G, j.pos, j.src, j.grpL, j.grpN);
 }
 
 // ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
 struct Pinned {
-  Summary* sum = nullptr;
+  HostSummary* sum = nullptr;   // mapped pinned memory
+  HostSummary* sum_dev = nullptr;  // its device address
+  uint32_t seq = 0;
   void* tables = nullptr;          // staging of the segment and class tables for their upload
   cudaEvent_t tables_done = nullptr;  // recorded after the last upload from `tables`
   std::mutex mu;
@@ -748,11 +796,11 @@ imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t co
   const size_t smem = smem_cols ? (size_t)cols * 4 : 0;
   const int64_t grid = rows < (int64_t)ds->num_sms * 4 ? rows : (int64_t)ds->num_sms * 4;
   if (it == IMQ_I16) {
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_line_max<int16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_line_max<int16_t>), smem));
     k_line_max<int16_t><<<(unsigned)grid, 256, smem, st>>>(static_cast<const int16_t*>(X), rows, cols, ld,
                                                            rowmax, colmax, smem_cols);
   } else {
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_line_max<int32_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_line_max<int32_t>), smem));
     k_line_max<int32_t><<<(unsigned)grid, 256, smem, st>>>(static_cast<const int32_t*>(X), rows, cols, ld,
                                                            rowmax, colmax, smem_cols);
   }
@@ -777,7 +825,11 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   // staging in the device layout: segments, classes and groups, each padded to 256 bytes
   const size_t staging_bytes = align_up(sizeof(InnerSeg) * kLv * kLv, 256) +
                                align_up(sizeof(OuterClass) * 2 * kLv, 256) + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
-  if (!pin.sum) IMQ_CUDA_TRY(cudaMallocHost(&pin.sum, sizeof(Summary)));
+  if (!pin.sum) {
+    IMQ_CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&pin.sum), sizeof(HostSummary), cudaHostAllocMapped));
+    IMQ_CUDA_TRY(cudaHostGetDevicePointer(reinterpret_cast<void**>(&pin.sum_dev), pin.sum, 0));
+    pin.sum->seq = 0;
+  }
   if (!pin.tables) IMQ_CUDA_TRY(cudaMallocHost(&pin.tables, staging_bytes));
   if (!pin.tables_done) IMQ_CUDA_TRY(cudaEventCreateWithFlags(&pin.tables_done, cudaEventDisableTiming));
 
@@ -984,6 +1036,8 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   la.lv[3] = pl->lv_b_col;
   la.bm1 = b - 1;
   la.sum = dsum;
+  la.hsum = pin.sum_dev;
+  la.seq = ++pin.seq;
   {
     const int64_t nmax = (M > K ? M : K) > N ? (M > K ? M : K) : N;
     int64_t grid = (nmax + 255) / 256;
@@ -992,10 +1046,31 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     k_levels<<<(unsigned)grid, 256, 0, st>>>(la);
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
-  if (cudaMemcpyAsync(pin.sum, dsum, sizeof(Summary), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return fail(IMQ_ERR_CUDA);
-  const Summary S = *pin.sum;
+  // wait for the summary: spin on its sequence number, asking the stream every few thousand polls
+  // whether it is still running (an error there is returned; a finished stream without the number, which
+  // a launch failure could leave, falls back to a plain copy of the device summary)
+  {
+    const volatile uint32_t* seqp = &pin.sum->seq;
+    bool have = false;
+    for (uint64_t it = 1;; ++it) {
+      if (*seqp == la.seq) {
+        have = true;
+        break;
+      }
+      if ((it & 4095) == 0) {
+        const cudaError_t q = cudaStreamQuery(st);
+        if (q == cudaSuccess) {
+          have = *seqp == la.seq;
+          break;
+        }
+        if (q != cudaErrorNotReady) return fail(IMQ_ERR_CUDA);
+      }
+    }
+    std::atomic_thread_fence(std::memory_order_acquire);
+    if (!have && (cudaMemcpy(&pin.sum->s, dsum, sizeof(Summary), cudaMemcpyDeviceToHost) != cudaSuccess))
+      return fail(IMQ_ERR_CUDA);
+  }
+  const Summary S = pin.sum->s;
   // a pending kernel error (e.g. a non-finite quantiser input) is reported before planning
   if (S.status != IMQ_OK) return fail((imq_status)S.status);
 
@@ -1265,19 +1340,27 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     pl->grpB_n = reinterpret_cast<int32_t*>(b2 + o_gNB);
   }
   if (ng > 0 || ncls > 0) {
-    // one upload from pinned staging (an asynchronous copy; pageable memory would be staged by the
-    // driver first); the staging is reused once the previous plan's upload has completed
-    if (cudaEventSynchronize(pin.tables_done) != cudaSuccess) return fail(IMQ_ERR_CUDA);
-    char* stg = static_cast<char*>(pin.tables);
-    memcpy(stg, hsegs, sizeof(InnerSeg) * (size_t)nseg);
-    memcpy(stg + (o_cls - o_segs), hcls, sizeof(OuterClass) * (size_t)ncls);
-    memcpy(stg + (o_grps - o_segs), hgrps, sizeof(InnerGroup) * (size_t)ng);
-    if (cudaMemcpyAsync(dsegs, stg, (o_grps - o_segs) + sizeof(InnerGroup) * (size_t)ng, cudaMemcpyHostToDevice,
-                        st) != cudaSuccess ||
-        cudaEventRecord(pin.tables_done, st) != cudaSuccess)
-      return fail(IMQ_ERR_CUDA);
     MapsArgs m;
+    m.inline_tables = nseg <= kParamSegs ? 1 : 0;
+    if (m.inline_tables) {
+      memcpy(m.t.segs, hsegs, sizeof(InnerSeg) * (size_t)nseg);
+      memcpy(m.t.cls, hcls, sizeof(OuterClass) * (size_t)ncls);
+      memcpy(m.t.grps, hgrps, sizeof(InnerGroup) * (size_t)ng);
+    } else {
+      // one upload from pinned staging (an asynchronous copy; pageable memory would be staged by the
+      // driver first); the staging is reused once the previous plan's upload has completed
+      if (cudaEventSynchronize(pin.tables_done) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+      char* stg = static_cast<char*>(pin.tables);
+      memcpy(stg, hsegs, sizeof(InnerSeg) * (size_t)nseg);
+      memcpy(stg + (o_cls - o_segs), hcls, sizeof(OuterClass) * (size_t)ncls);
+      memcpy(stg + (o_grps - o_segs), hgrps, sizeof(InnerGroup) * (size_t)ng);
+      if (cudaMemcpyAsync(dsegs, stg, (o_grps - o_segs) + sizeof(InnerGroup) * (size_t)ng, cudaMemcpyHostToDevice,
+                          st) != cudaSuccess ||
+          cudaEventRecord(pin.tables_done, st) != cudaSuccess)
+        return fail(IMQ_ERR_CUDA);
+    }
     m.grps = reinterpret_cast<const InnerGroup*>(blk1 + o_grps);
+    m.cls = dcls;
     m.ngrp = ng;
     m.segs = dsegs;
     m.lva = pl->lv_a_col;
@@ -1289,9 +1372,9 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     m.lAk = pl->lAk;
     m.lBk = pl->lBk;
     m.blk16 = pl->blk16;
-    m.a = {dcls + cls_a0, a_outer ? cls_a1 - cls_a0 : 0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
+    m.a = {cls_a0, a_outer ? cls_a1 - cls_a0 : 0, pl->lv_a_row, M, IMQ_A_GROUP, pl->posA, pl->srcA,
            pl->grpA_L, pl->grpA_n};
-    m.b = {dcls + cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
+    m.b = {cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
            pl->grpB_L, pl->grpB_n};
     const int blocks = ng + m.a.ncls + m.b.ncls;
     if (blocks > 0) k_plan_maps<<<blocks, 1024, 0, st>>>(m);

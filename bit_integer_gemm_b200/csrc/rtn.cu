@@ -716,7 +716,7 @@ imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, u
     part = static_cast<int32_t*>(sp.p);
   }
   auto kern = k_rtn_cols_staged<T, CW, kOut16>;
-  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   kern<<<(unsigned)grid, CW * 32, smem, st>>>(X, rows, cols, ld, k, beta, Xint, ldq, trans_out, delta, qval, part,
                                               colmax, vec ? 1 : 0, ds->status, clip);
   if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
@@ -787,12 +787,12 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
       k_tensor_select<T><<<1, 32, 0, st>>>(ts, pass, pass == np - 1, beta, delta, qval, ds->status);
     }
     auto kern = k_rtn_rows<T, false, kOut16>;
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, 0ull, beta, Xint, ldq, trans_out, delta, qval,
                                                  rowmax, part, ts, vec, nwarps, ds->status, clip);
   } else {
     auto kern = k_rtn_rows<T, true, kOut16>;
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta,
                                                  Xint, ldq, trans_out, delta, qval, rowmax, part, nullptr, vec, nwarps,
                                                  ds->status, clip);
@@ -909,7 +909,7 @@ imq_status run_rows_noalloc(const T* X, int64_t rows, int64_t cols, int64_t ld, 
     if (e != IMQ_OK) return e;
   }
   auto kern = k_rtn_rows<T, true, kOut16>;
-  IMQ_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   kern<<<(unsigned)grid, kThreads, smem, st>>>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta,
                                                Xint, ldq, 0, delta, qval, rowmax, part, nullptr, vec, nwarps,
                                                ds->status, 0);
@@ -1124,7 +1124,7 @@ imq_status run_rtn_unpack(const T* X, const FusedArgs& f, DeviceState* ds, cudaS
   if (per_sm > 4) per_sm = 4;
   const int64_t blocks = (f.rows + nwarps - 1) / nwarps;
   const int64_t grid = blocks < (int64_t)ds->num_sms * per_sm ? blocks : (int64_t)ds->num_sms * per_sm;
-  IMQ_CUDA_TRY(cudaFuncSetAttribute(k_rtn_unpack_rows<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_rtn_unpack_rows<T>), smem));
   k_rtn_unpack_rows<T><<<(unsigned)grid, kThreads, smem, st>>>(X, f, nwarps, meta_smem);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }

@@ -463,7 +463,7 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
         const int64_t ctas = (nlines + nw - 1) / nw;
         int64_t grid = (int64_t)num_sms * (per_sm > 8 ? 8 : per_sm);
         if (grid > ctas) grid = ctas;
-        IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_lines<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
         k_unpack_lines<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, P, nw, outer, lvl, pos, tK, lk, blk16,
                                                              K_unp, bm1, meta_smem, out);
         return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
@@ -486,7 +486,7 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
     const int64_t batches = (nlines + NL - 1) / NL;
     int64_t grid = (int64_t)num_sms * (per_sm > 8 ? 8 : per_sm);
     if (grid > batches) grid = batches;
-    IMQ_CUDA_TRY(cudaFuncSetAttribute(k_unpack_rows<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_rows<T>), smem));
     k_unpack_rows<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, NL, P, outer, lvl, pos, tK, lk, blk16,
                                                         K_unp, bm1, out);
   } else {
