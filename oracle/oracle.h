@@ -46,7 +46,6 @@
 #define OR_INNER_PAD 128
 #define OR_A_GROUP 32
 #define OR_B_GROUP 32
-#define OR_B_WINDOW 1024 /* OUTER columns of B: every window of this many sources starts a new group */
 
 typedef struct {
   int32_t b, strategy, dir_a, dir_b;

@@ -22,13 +22,9 @@
  *        the smallest such tau on a tie; the direction is then OUTER, INNER or both (OR_DIR_BOTH).  The
  *        level vectors the plan returns are then the levels each line carries in the unpacked GEMM.
  *   layout: inner pairs (t, lA, lB) ordered by e = lA + lB, then lA, then t, each exponent group padded
- *   with zeros to OR_INNER_PAD.  OUTER rows of A: sorted by level (stable), floor(G / L) source rows per
- *   group of G = OR_A_GROUP unpacked rows, the L rows of one source consecutive, unused rows empty.
- *   OUTER columns of B: in index order, the L lines of one source consecutive, packed into groups of
- *   OR_B_GROUP lines; a source starts the next group when its lines do not fit in what is left of the
- *   current one, and the first source of every window of OR_B_WINDOW consecutive sources starts a new
- *   group; unused lines (at the end of a group) empty.  (Adjacent columns of C then come from one
- *   group, which the GEMM writes with contiguous stores.)
+ *   with zeros to OR_INNER_PAD; OUTER lines sorted by level (stable), floor(G / L) source lines per
+ *   group of G unpacked lines (G = OR_A_GROUP for rows of A, OR_B_GROUP for columns of B), the L lines
+ *   of one source consecutive, unused lines empty.
  */
 #include <stdlib.h>
 #include <string.h>
@@ -261,13 +257,12 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
     out->M_unp = M;
   }
   if (db & OR_DIR_OUTER) {
-    int64_t groups = 0, used = 0;
-    for (int64_t j = 0; j < N; ++j) {
-      if (j == 0 || j % OR_B_WINDOW == 0 || used + LcB[j] > OR_B_GROUP) {
-        groups += 1;
-        used = 0;
-      }
-      used += LcB[j];
+    int64_t groups = 0;
+    for (int L = 1; L <= out->lmax[3]; ++L) {
+      int64_t cnt = 0;
+      for (int64_t j = 0; j < N; ++j) cnt += (LcB[j] == L);
+      int64_t per = OR_B_GROUP / L;
+      groups += (cnt + per - 1) / per;
     }
     out->N_unp = groups * OR_B_GROUP;
   } else {
@@ -340,17 +335,16 @@ int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t 
 
   for (int64_t w = 0; w < pl->N_unp; ++w) { srcB[w] = -1; lvlB[w] = 0; }
   if (db & OR_DIR_OUTER) {
-    int64_t grp = -1, used = 0;
-    for (int64_t j = 0; j < N; ++j) {
-      if (j == 0 || j % OR_B_WINDOW == 0 || used + LcB[j] > OR_B_GROUP) {
-        grp += 1;
-        used = 0;
+    int64_t grp = 0;
+    for (int L = 1; L <= pl->lmax[3]; ++L) {
+      int64_t per = OR_B_GROUP / L, rank = 0;
+      for (int64_t j = 0; j < N; ++j) {
+        if (LcB[j] != L) continue;
+        int64_t base = (grp + rank / per) * OR_B_GROUP + (rank % per) * L;
+        for (int l = 0; l < L; ++l) { srcB[base + l] = (int32_t)j; lvlB[base + l] = l; }
+        rank += 1;
       }
-      for (int l = 0; l < LcB[j]; ++l) {
-        srcB[grp * OR_B_GROUP + used + l] = (int32_t)j;
-        lvlB[grp * OR_B_GROUP + used + l] = l;
-      }
-      used += LcB[j];
+      grp += (rank + per - 1) / per;
     }
   } else {
     for (int64_t j = 0; j < N; ++j) srcB[j] = (int32_t)j;

@@ -566,30 +566,10 @@ def test_layout_follows_documented_order():
                 assert np.all(mp["tK"][off + ln:off + padded] == -1)
                 want.append(e)
             assert want == sorted(want)
-            # outer columns of B: sources in index order, greedy groups of 32 lines, a new group at every
-            # window of 1024 sources (only one window at these sizes); unused lines at the group ends
-            if pl.dir_b & oracle.DIR_OUTER:
-                src, lvl, lines = mp["srcB"], mp["lvlB"], lv["b_col"]
-                want_src, want_lvl, used = [], [], 32
-                for j in range(N):
-                    L = int(lines[j])
-                    if j % 1024 == 0 or used + L > 32:
-                        pad = (-len(want_src)) % 32
-                        want_src += [-1] * pad
-                        want_lvl += [0] * pad
-                        used = 0
-                    want_src += [j] * L
-                    want_lvl += list(range(L))
-                    used += L
-                pad = (-len(want_src)) % 32
-                want_src += [-1] * pad
-                want_lvl += [0] * pad
-                assert src.tolist() == want_src and lvl.tolist() == want_lvl
-            else:
-                assert np.array_equal(mp["srcB"], np.arange(N)) and not mp["lvlB"].any()
-            # outer rows of A: per group one level L, floor(G/L) sources of that level, lines (src, l) in order
+            # outer: per group one level L, floor(G/L) sources of that level, lines (src, l) in order
             for src, lvl, lines, G, dirv, outer in (
-                    (mp["srcA"], mp["lvlA"], lv["a_row"], 32, pl.dir_a, oracle.DIR_OUTER),):
+                    (mp["srcA"], mp["lvlA"], lv["a_row"], 32, pl.dir_a, oracle.DIR_OUTER),
+                    (mp["srcB"], mp["lvlB"], lv["b_col"], 32, pl.dir_b, oracle.DIR_OUTER)):
                 if not dirv & outer:
                     assert np.array_equal(src, np.arange(src.size)) and not lvl.any()
                     continue
@@ -631,31 +611,3 @@ def test_cached_plan_is_exact_for_covered_inputs():
         assert np.array_equal(oracle.unpacked_gemm(pl, Au, Bu), A2 @ B), case
         checked += 1
     assert checked > 150
-
-
-def test_outer_columns_of_b_restart_groups_at_windows():
-    """OUTER columns of B across several windows of 1024 sources: every window's first source starts a
-    group (the group before it may end partly empty), within a window the greedy rule holds, and the
-    unpacked product stays exact."""
-    rng = np.random.default_rng(32)
-    M, K, N, b = 3, 4, 2600, 5
-    A = rng.integers(-15, 16, size=(M, K)).astype(np.int64)
-    B = rng.integers(-15, 16, size=(K, N)).astype(np.int64)
-    B[0, rng.random(N) < 0.6] = 300   # most columns get 3 levels, the rest 1
-    pl = oracle.plan(A, B, b, oracle.ROW_COL)
-    assert pl.dir_b == oracle.DIR_OUTER
-    src = pl.maps["srcB"]
-    starts = {}
-    for w in range(src.size):
-        if src[w] >= 0 and (w == 0 or src[w - 1] != src[w]):
-            starts[int(src[w])] = w
-    for j in (0, 1024, 2048):
-        assert starts[j] % 32 == 0
-    # within a window a group is only closed when the next source does not fit
-    for j in range(1, N):
-        if j % 1024 and starts[j] % 32 == 0:
-            g0 = starts[j] - 32
-            used = int((src[g0:g0 + 32] >= 0).sum())
-            assert used + int(pl.levels["b_col"][j]) > 32
-    Au, Bu = oracle.unpack(pl, A, B)
-    assert np.array_equal(oracle.unpacked_gemm(pl, Au, Bu), A @ B)
