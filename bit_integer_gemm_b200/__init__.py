@@ -92,6 +92,7 @@ SIGNATURES = {
     "imq_gemm_unpacked": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP],
     "imq_unpacked_gemm": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP, _SZ, _VP],
     "imq_device_status": [_VP, _I32],
+    "imq_check_bounded_wait": [ctypes.c_uint64, _VP],
     "imq_status_str": [_I32],
 }
 
@@ -288,6 +289,11 @@ def imq_rtn_quantize_unpack(plan: Plan, X: torch.Tensor, p: float, beta: int, A_
     _check(lib().imq_rtn_quantize_unpack(plan.handle, _ptr(X), _TORCH_TO_IMQ[X.dtype], _ld(X), float(p), int(beta),
                                          _ptr(A_unp), _ptr(deltaA), _stream(stream)), "imq_rtn_quantize_unpack")
     return A_unp, deltaA
+
+
+def imq_check_bounded_wait(timeout_ns: int, stream=None):
+    """Diagnostic: a kernel whose bounded wait runs out after timeout_ns and records IMQ_ERR_TIMEOUT."""
+    _check(lib().imq_check_bounded_wait(int(timeout_ns), _stream(stream)), "imq_check_bounded_wait")
 
 
 def _outputs(I, dev, C, c_dtype, Cf, want_int, want_f32):

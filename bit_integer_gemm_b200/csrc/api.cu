@@ -90,6 +90,21 @@ __global__ void __launch_bounds__(1024) k_reduce_max(const int32_t* __restrict__
     out[i] = m;
   }
 }
+
+// One mbarrier that nothing arrives at, waited on by the library's bounded wait: the wait gives up after
+// timeout_ns, raises the abort flag and records IMQ_ERR_TIMEOUT, and the kernel returns.
+__global__ void k_check_bounded_wait(int32_t* status, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_addr(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(smem_addr(&bar), 0, &abort_flag, status, timeout_ns);
+  __syncthreads();
+}
 }  // namespace
 
 imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st) {
@@ -232,6 +247,15 @@ imq_status imq_unpacked_gemm(const imq_plan_t* plan, const void* A, const void* 
   imq_status s = imq_unpack(plan, A, B, Au, Bu, stream);
   if (s != IMQ_OK) return s;
   return imq_gemm_unpacked(plan, Au, Bu, deltaA, gA, deltaB, gB, Cint, ct, ldc, Cf, ldcf, stream);
+}
+
+imq_status imq_check_bounded_wait(uint64_t timeout_ns, imq_stream_t stream) {
+  if (timeout_ns < 1000ull || timeout_ns > 1000000000ull) return IMQ_ERR_ARG;
+  DeviceState* ds;
+  imq_status s = imq::device_state(&ds);
+  if (s != IMQ_OK) return s;
+  imq::k_check_bounded_wait<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ds->status, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
 imq_status imq_device_status(imq_stream_t stream, int32_t clear) {

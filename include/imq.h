@@ -355,6 +355,13 @@ imq_status imq_unpacked_gemm(const imq_plan_t *plan, const void *A, const void *
  * non-zero, resets it to IMQ_OK. */
 imq_status imq_device_status(imq_stream_t stream, int32_t clear);
 
+/* Diagnostic, no counterpart on the page: launches one kernel whose bounded wait (the one every wait of
+ * the GEMM goes through) waits on an mbarrier that nothing arrives at, so it gives up after timeout_ns
+ * (1 us .. 1 s, else IMQ_ERR_ARG) and records IMQ_ERR_TIMEOUT in the device status word.  It shows that
+ * a stalled wait ends the kernel with a status the host reads and leaves the context usable.
+ * Asynchronous. */
+imq_status imq_check_bounded_wait(uint64_t timeout_ns, imq_stream_t stream);
+
 /* Static, never NULL. */
 const char *imq_status_str(imq_status s);
 
