@@ -33,6 +33,12 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kColsPerCta = 16;
+// Per-warp select scratch in 32-bit words: the 256-bin histogram of the fp32 radix passes, or the
+// one-bin-per-key histogram of the sampled bf16 select (keys lo .. lo + kSelWords - 1).
+constexpr int kSelWords = 384;
+// bf16 groups with at least this many entries take the sampled select; smaller ones bisect directly.
+constexpr int kSampledMin = 1024;
+constexpr int kSampleSize = 128;  // 4 keys per lane
 
 struct TensorState {
   unsigned long long krem;  // rank still to be found (1-based) inside the current prefix
@@ -117,7 +123,9 @@ __device__ bool warp_select(const uint32_t* hist, int stride, unsigned long long
   return lane == 0;
 }
 
-__device__ __forceinline__ void scale_from_q(float q, float qmax, int beta, float* s, float* d) {
+// Scale and step from the selected q; q == 0 falls back to the group maximum qmax.  Returns the q the
+// scale was derived from (reported as qval).
+__device__ __forceinline__ float scale_from_q(float q, float qmax, int beta, float* s, float* d) {
   if (q == 0.0f) q = qmax;
   if (q == 0.0f) {
     *s = 1.0f;
@@ -126,6 +134,7 @@ __device__ __forceinline__ void scale_from_q(float q, float qmax, int beta, floa
     *s = __fdiv_rn((float)beta, q);
     *d = __fdiv_rn(q, (float)beta);
   }
+  return q;
 }
 
 // Quantises one value; returns |v| (0 on a range error, which is recorded).
@@ -165,6 +174,26 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
   uint32_t r = 0;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = max(r, red[w]);
   return r;
+}
+
+// Copies n16 16-byte pieces from global memory (streaming loads) to shared memory, lane-strided over
+// one warp, with kBatch loads in flight per lane before their stores: a store waits for its load, so a
+// plain copy loop would keep a single load per lane in flight and pay one memory latency per piece.
+template <int kBatch>
+__device__ __forceinline__ void warp_copy16(const uint4* __restrict__ src, uint4* dst, int n16, int lane) {
+  for (int c0 = lane; c0 < n16; c0 += 32 * kBatch) {
+    uint4 buf[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < n16) buf[j] = __ldcs(src + c);
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < n16) dst[c] = buf[j];
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -263,13 +292,192 @@ __device__ uint32_t warp_select_key_bf16(const uint16_t* a, int n, unsigned long
   return ans;
 }
 
-// The k-th smallest key of a group in shared memory: bisection for bf16, radix passes for f32.
+// Per 16-bit half of two packed keys (sign bits of w forced to 1, t2 = t * 0x10001, t <= 0x7FFF): 1 in
+// bit 0 (low half) and bit 16 (high half) where the key is >= t.  (0x8000 + key) - t lies in [1, 0xFFFF]
+// for keys and t below 2^15, so bit 15 of each half is set exactly when key >= t and no half borrows.
+__device__ __forceinline__ uint32_t ge_pair(uint32_t w_signed, uint32_t t2) {
+  return ((w_signed - t2) >> 15) & 0x00010001u;
+}
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Largest bf16 key of a group and whether any key is non-finite, two keys per 32-bit word.
+__device__ void warp_key_stats_bf16(const uint16_t* a, int n, uint32_t* mk_out, uint32_t* bad_out) {
+  const int lane = threadIdx.x & 31;
+  const int nv = n / 8;
+  uint32_t m0 = 0, m1 = 0;
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 w = reinterpret_cast<const uint4*>(a)[i];
+    m0 = max_u16x2(m0, max_u16x2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu));
+    m1 = max_u16x2(m1, max_u16x2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+  }
+  m0 = max_u16x2(m0, m1);
+  uint32_t mk = max(m0 & 0xFFFFu, m0 >> 16);
+  for (int i = nv * 8 + lane; i < n; i += 32) mk = max(mk, (uint32_t)(a[i] & 0x7FFFu));
+  mk = __reduce_max_sync(0xffffffffu, mk);
+  *mk_out = mk;
+  *bad_out = mk >= Key<uint16_t>::kInf;
+}
+
+// Exact nearest-rank select for bf16 keys by sampling (the SampleSelect scheme of Ribizel and Anzt,
+// "Parallel selection on GPUs", 2019, on one warp), which also returns the group's largest key:
+//   1. kSampleSize keys at evenly spaced positions; lo = the sample order statistic whose rank lies
+//      2.5 binomial standard deviations (+1.5) below the target rank k * S / n (bisection on the key
+//      value over the sample, which the lanes hold in registers);
+//   2. one pass over the group counts the keys below lo, histograms the keys in [lo, lo + kSelWords - 1]
+//      into the warp's scratch (one bin per key value) and takes the largest key;
+//   3. if the bracket holds (fewer than k keys below lo, at least k up to the histogram's top) the answer
+//      is the bin where the running count reaches k; otherwise the group is bisected in full.
+// The sample only steers the work: every answer is the exact k-th smallest key.
+__device__ uint32_t warp_select_key_bf16_sampled(const uint16_t* a, int n, unsigned long long k, uint32_t* hist,
+                                                  uint32_t* mk_out) {
+  const int lane = threadIdx.x & 31;
+  constexpr unsigned kFull = 0xffffffffu;
+  // ---- 1. sample: keys j and j + 32 of sample slice m in word m (positions at the slice midpoints)
+  uint32_t sw[kSampleSize / 64];
+#pragma unroll
+  for (int m = 0; m < kSampleSize / 64; ++m) {
+    const int j0 = 64 * m + lane, j1 = j0 + 32;
+    // (2j + 1) n < 2^31 for the groups staged here (n below 2^21)
+    const uint32_t k0 = a[((2u * j0 + 1u) * (uint32_t)n) / (2u * kSampleSize)] & 0x7FFFu;
+    const uint32_t k1 = a[((2u * j1 + 1u) * (uint32_t)n) / (2u * kSampleSize)] & 0x7FFFu;
+    sw[m] = k0 | (k1 << 16);
+  }
+#pragma unroll
+  for (int j = 0; j < kSelWords / 32; ++j) hist[j * 32 + lane] = 0;
+  uint32_t smn = 0xFFFFFFFFu, smx = 0;
+#pragma unroll
+  for (int m = 0; m < kSampleSize / 64; ++m) {
+    smn = min_u16x2(smn, sw[m]);
+    smx = max_u16x2(smx, sw[m]);
+    sw[m] |= 0x80008000u;
+  }
+  smn = __reduce_min_sync(kFull, min(smn & 0xFFFFu, smn >> 16));
+  smx = __reduce_max_sync(kFull, max(smx & 0xFFFFu, smx >> 16));
+  const float pk = (float)((double)k / (double)n);
+  const int r_lo = (int)floorf(pk * (float)kSampleSize - 2.5f * sqrtf((float)kSampleSize * pk * (1.0f - pk)) - 1.5f);
+  uint32_t lo = 0;
+  if (r_lo >= 1) {
+    // the r_lo-th smallest sample key: answer in [l, h], #{sample < mid} decides the half
+    uint32_t l = smn, h = smx;
+    while (l < h) {
+      const uint32_t mid = (l + h + 1) >> 1, t2 = mid * 0x10001u;
+      uint32_t g = 0;
+#pragma unroll
+      for (int m = 0; m < kSampleSize / 64; ++m) g += ge_pair(sw[m], t2);
+      const uint32_t below = kSampleSize - __reduce_add_sync(kFull, (g & 0xFFFFu) + (g >> 16));
+      if (below < (uint32_t)r_lo) l = mid; else h = mid - 1;
+    }
+    lo = l;
+  }
+  const uint32_t hi = min(lo + (uint32_t)kSelWords - 1u, 0x7FFFu);
+  __syncwarp();
+  // ---- 2. count below lo, histogram [lo, hi], largest key
+  const uint32_t lo2 = lo * 0x10001u, hi2 = (hi | 0x8000u) * 0x10001u;
+  const int nv = n / 8;
+  uint32_t ge = 0, mx2 = 0;
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 w4 = reinterpret_cast<const uint4*>(a)[i];
+    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t kk = ws[q] & 0x7FFF7FFFu;
+      const uint32_t gl = ((kk | 0x80008000u) - lo2) & 0x80008000u;  // bit 15 / 31: key >= lo
+      const uint32_t c = gl & (hi2 - kk);                               // bit 15 / 31: lo <= key <= hi
+      ge += gl >> 15;
+      mx2 = max_u16x2(mx2, kk);
+      if (c & 0x8000u) atomicAdd(&hist[(kk & 0xFFFFu) - lo], 1u);
+      if (c & 0x80000000u) atomicAdd(&hist[(kk >> 16) - lo], 1u);
+    }
+  }
+  uint32_t mk = max(mx2 & 0xFFFFu, mx2 >> 16);
+  uint32_t ge_tail = 0;
+  for (int i = nv * 8 + lane; i < n; i += 32) {
+    const uint32_t key = a[i] & 0x7FFFu;
+    mk = max(mk, key);
+    ge_tail += key >= lo ? 1u : 0u;
+    if (key >= lo && key <= hi) atomicAdd(&hist[key - lo], 1u);
+  }
+  mk = __reduce_max_sync(kFull, mk);
+  *mk_out = mk;
+  const uint32_t n_ge = __reduce_add_sync(kFull, (ge & 0xFFFFu) + (ge >> 16) + ge_tail);
+  const unsigned long long below = (unsigned long long)n - n_ge;
+  __syncwarp();
+  // ---- 3. running count over the bins: lane owns bins [12 lane, 12 lane + 12)
+  constexpr int kPer = kSelWords / 32;
+  uint32_t c[kPer], own = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    c[j] = hist[lane * kPer + j];
+    own += c[j];
+  }
+  uint32_t incl = own;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t total = __shfl_sync(kFull, incl, 31);
+  __syncwarp();
+  if (!(below < k && k <= below + total)) return warp_select_key_bf16(a, n, k);
+  const uint32_t r = (uint32_t)(k - below);
+  const unsigned ball = __ballot_sync(kFull, incl - own < r && r <= incl);
+  const int src = __ffs(ball) - 1;
+  uint32_t bin = 0;
+  if (lane == src) {
+    uint32_t cum = incl - own;
+    bin = lane * kPer + kPer - 1;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (cum + c[j] >= r) {
+        bin = lane * kPer + j;
+        break;
+      }
+      cum += c[j];
+    }
+  }
+  return lo + __shfl_sync(kFull, bin, src);
+}
+
+// Largest key (mk) and the k-th smallest key of a group in shared memory: sampled select for bf16
+// groups of kSampledMin entries and more (which returns the largest key as well), a key-statistics pass
+// and bisection for smaller bf16 groups, radix passes for f32.  `scratch` is the warp's kSelWords words.
+// bad: the group holds a non-finite value.
 template <typename T>
-__device__ __forceinline__ uint32_t select_key(const T* a, int n, unsigned long long k, uint32_t* hist) {
+__device__ __forceinline__ uint32_t stats_and_select(const T* a, int n, unsigned long long k, uint32_t* scratch,
+                                                     uint32_t* mk, uint32_t* bad) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t key;
+    if (n >= kSampledMin) {
+      key = warp_select_key_bf16_sampled(a, n, k, scratch, mk);
+    } else {
+      warp_key_stats_bf16(a, n, mk, bad);
+      key = warp_select_key_bf16(a, n, k);
+    }
+    *bad = *mk >= Key<T>::kInf;
+    return key;
+  } else {
+    warp_key_stats(a, n, mk, bad);
+    return warp_select_key(a, n, k, scratch);
+  }
+}
+
+// Largest key of a group and whether any key is non-finite (groups that are not selected on).
+template <typename T>
+__device__ __forceinline__ void key_stats(const T* a, int n, uint32_t* mk_out, uint32_t* bad_out) {
   if constexpr (sizeof(T) == 2)
-    return warp_select_key_bf16(a, n, k);
+    warp_key_stats_bf16(a, n, mk_out, bad_out);
   else
-    return warp_select_key(a, n, k, hist);
+    warp_key_stats(a, n, mk_out, bad_out);
 }
 
 // x * s rounded to the nearest integer, ties to even: the arithmetic of quant_one, without the store.
@@ -292,8 +500,11 @@ __device__ __forceinline__ int32_t quant_val(float x, float s, int32_t* status, 
 
 // Quantises 8 consecutive entries of a 16-byte aligned group in shared memory and stores them with
 // 16-byte stores at out[idx .. idx+7] (idx a multiple of 8, out 16-byte aligned); a[j] = |value j|.
+// The conversion saturates (a NaN never gets here: its group is refused first), so an entry out of the
+// output's range shows in a[j] as a magnitude above 32767 (int16) or of at least 2^31 - 1 (int32: no
+// float below 2^31 rounds to 2^31 - 1); range_error() on the group's largest a[j] reports it.
 template <typename T, bool kOut16>
-__device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t idx, int32_t* status, int clip,
+__device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t idx, int clip,
                                        uint32_t (&a)[8]) {
   // the 8 entries as 32-bit words (bf16: two per word, low half first), kept in registers
   uint32_t wd[8];
@@ -309,8 +520,10 @@ __device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const T e = sizeof(T) == 2 ? (T)((wd[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) : (T)wd[j];
-    v[j] = quant_val<kOut16>(Key<T>::value(e), s, status, clip);
-    a[j] = v[j] < 0 ? (uint32_t)(-(int64_t)v[j]) : (uint32_t)v[j];
+    float y = __fmul_rn(Key<T>::value(e), s);
+    if (clip) y = fminf(fmaxf(y, -(float)clip), (float)clip);
+    v[j] = __float2int_rn(y);
+    a[j] = v[j] < 0 ? 0u - (uint32_t)v[j] : (uint32_t)v[j];
   }
   if (kOut16) {
     uint32_t pk[4];
@@ -322,6 +535,51 @@ __device__ __forceinline__ void quant8(const T* src, float s, void* out, int64_t
     reinterpret_cast<int4*>(o)[0] = make_int4(v[0], v[1], v[2], v[3]);
     reinterpret_cast<int4*>(o)[1] = make_int4(v[4], v[5], v[6], v[7]);
   }
+}
+
+// True when a quantised magnitude from quant8 lies outside the output type's range.
+template <bool kOut16>
+__device__ __forceinline__ bool range_error(uint32_t amax) {
+  return kOut16 ? amax > 32767u : amax >= 0x7FFFFFFFu;
+}
+
+// Quantises a bf16 group held in shared memory (n a multiple of 8, 16-byte aligned) into int16 at
+// out[0 .. n) (16-byte aligned), 8 entries per lane and step, and overwrites each staged entry with its
+// |x_int| (16 bits) so that line maxima across the group can be folded afterwards without atomics.
+__device__ __forceinline__ void quant_bf16_inplace(uint16_t* grp, int n, float s, int clip, int16_t* out) {
+  const int lane = threadIdx.x & 31;
+  for (int g = lane; g < n / 8; g += 32) {
+    const uint4 w = reinterpret_cast<const uint4*>(grp)[g];
+    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+    uint32_t pv[4], pa[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float y0 = __fmul_rn(__uint_as_float(wd[q] << 16), s);
+      float y1 = __fmul_rn(__uint_as_float(wd[q] & 0xFFFF0000u), s);
+      if (clip) {
+        y0 = fminf(fmaxf(y0, -(float)clip), (float)clip);
+        y1 = fminf(fmaxf(y1, -(float)clip), (float)clip);
+      }
+      const int32_t v0 = __float2int_rn(y0), v1 = __float2int_rn(y1);
+      const uint32_t a0 = v0 < 0 ? 0u - (uint32_t)v0 : (uint32_t)v0, a1 = v1 < 0 ? 0u - (uint32_t)v1 : (uint32_t)v1;
+      pv[q] = __byte_perm((uint32_t)v0, (uint32_t)v1, 0x5410);
+      pa[q] = __byte_perm(a0, a1, 0x5410);
+    }
+    *reinterpret_cast<uint4*>(out + g * 8) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+    reinterpret_cast<uint4*>(grp)[g] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+  }
+}
+
+// Largest |x_int| of a group from its largest |x| (xmax): a correctly rounded multiply and rint are
+// monotone and odd, so the group's largest quantised magnitude is rint(fl(xmax * s)) (clamped with the
+// clipping variant).  Sets *range when it lies outside the output type (int16: above 32767, int32: at or
+// above 2^31).
+template <bool kOut16>
+__device__ __forceinline__ uint32_t group_max_int(float xmax, float s, int clip, bool* range) {
+  float y = __fmul_rn(xmax, s);
+  if (clip) y = fminf(y, (float)clip);
+  *range = kOut16 ? !(y < 32767.5f) : !(y < 2147483648.0f);
+  return *range ? 0u : (uint32_t)__float2int_rn(y);
 }
 
 // Raises m[0..7] (16-byte aligned shared memory) to a[j] where a[j] is larger: a plain read first, so
@@ -350,7 +608,8 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
   const int64_t row_bytes = (cols * (int64_t)sizeof(T) + 15) / 16 * 16;
   uint32_t* cmax = reinterpret_cast<uint32_t*>(dsm);                  // [cols]
   const int64_t cmax_bytes = part ? (cols * 4 + 15) / 16 * 16 : 0;  // same layout as the host
-  __shared__ uint32_t hist_all[kThreads / 32][256];
+  __shared__ uint32_t hist_all[kThreads / 32][kSelWords];
+  __shared__ int s_done[kThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   T* row = reinterpret_cast<T*>(dsm + cmax_bytes + warp * row_bytes);
   uint32_t* hist = hist_all[warp];
@@ -358,60 +617,99 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
   if (part)
     for (int64_t c = tid; c < cols; c += blockDim.x) cmax[c] = 0;
   __syncthreads();
-  if (warp < nwarps) {
-    const int n = (int)cols;
-    // vectorised quantisation: whole 8-entry groups, contiguous and 16-byte aligned output rows
-    const bool vq = !trans_out && n % 8 == 0 && ldq % 8 == 0 && (reinterpret_cast<uintptr_t>(Xint) & 15) == 0;
-    for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < rows; r += (int64_t)gridDim.x * nwarps) {
+  const int n = (int)cols;
+  // vectorised quantisation: whole 8-entry groups, contiguous and 16-byte aligned output rows
+  const bool vq = !trans_out && n % 8 == 0 && ldq % 8 == 0 && (reinterpret_cast<uintptr_t>(Xint) & 15) == 0;
+  // bf16 in, int16 out: rows quantised in place (|x_int| kept in the staged row), and the CTA folds
+  // each round of nwarps rows into its column maxima, every thread owning whole 8-column groups
+  const bool inplace = sizeof(T) == 2 && kOut16 && vq;
+  // rows are dealt to the CTAs in turn (row r to CTA r mod gridDim.x), so that every SM gets the same
+  // number of rows to within one per CTA; round j of a CTA takes its rows j*nwarps .. j*nwarps+nwarps-1
+  for (int64_t j0 = 0; j0 * gridDim.x + blockIdx.x < rows; j0 += nwarps) {
+    const int64_t r = (j0 + warp) * gridDim.x + blockIdx.x;
+    int done = 0;
+    if (warp < nwarps && r < rows) {
       const T* xr = X + r * ld;
       if (vec) {
-        const uint4* src = reinterpret_cast<const uint4*>(xr);
-        uint4* dst = reinterpret_cast<uint4*>(row);
-        for (int c = lane; c < n / V; c += 32) dst[c] = __ldcs(src + c);
+        warp_copy16<8>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), n / V, lane);
       } else {
         for (int c = lane; c < n; c += 32) row[c] = xr[c];
       }
       __syncwarp();
       uint32_t mk, bad;
-      warp_key_stats(row, n, &mk, &bad);
       float s;
       if (kSelect) {
-        const float q = Key<T>::from_key(select_key(row, n, krank, hist));
+        const float q = Key<T>::from_key(stats_and_select(row, n, krank, hist, &mk, &bad));
         float dl;
-        scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
+        const float qu = scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
         if (lane == 0) {
           delta[r] = dl;
-          if (qval) qval[r] = q;
+          if (qval) qval[r] = qu;
         }
       } else {
+        key_stats(row, n, &mk, &bad);
         s = ts->s;
       }
+      __syncwarp();
       if (bad) {
         if (lane == 0) set_status(status, IMQ_ERR_NONFINITE);
-        continue;
-      }
-      uint32_t rmx = 0;
-      if (vq) {
-        // 8 consecutive entries per lane and step: 16-byte shared loads and global stores
-        for (int g = lane; g < n / 8; g += 32) {
-          uint32_t a[8];
-          quant8<T, kOut16>(row + g * 8, s, Xint, r * ldq + g * 8, status, clip, a);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) rmx = max(rmx, a[j]);
-          if (part) max8_shared(cmax + g * 8, a);
+      } else if (inplace) {
+        quant_bf16_inplace(reinterpret_cast<uint16_t*>(row), n, s, clip, static_cast<int16_t*>(Xint) + r * ldq);
+        bool range;
+        const uint32_t rmx = group_max_int<kOut16>(Key<T>::from_key(mk), s, clip, &range);
+        if (lane == 0) {
+          if (range) set_status(status, IMQ_ERR_RANGE);
+          if (rowmax) rowmax[r] = (int32_t)rmx;
         }
+        done = 1;
       } else {
-        for (int c = lane; c < n; c += 32) {
-          const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint,
-                                               trans_out ? c * ldq + r : r * ldq + c, status, clip);
-          rmx = max(rmx, a);
-          if (part && a > cmax[c]) atomicMax(&cmax[c], a);
-        }
-      }
+        uint32_t rmx = 0;
+        if (vq) {
+          // 8 consecutive entries per lane and step: 16-byte shared loads and global stores
+          for (int g = lane; g < n / 8; g += 32) {
+            uint32_t a[8];
+            quant8<T, kOut16>(row + g * 8, s, Xint, r * ldq + g * 8, clip, a);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) rmx = max(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
-      if (lane == 0 && rowmax) rowmax[r] = (int32_t)rmx;
+            for (int j = 0; j < 8; ++j) rmx = max(rmx, a[j]);
+            if (part) max8_shared(cmax + g * 8, a);
+          }
+        } else {
+          for (int c = lane; c < n; c += 32) {
+            const uint32_t a = quant_one<kOut16>(Key<T>::value(row[c]), s, Xint,
+                                                 trans_out ? c * ldq + r : r * ldq + c, status, clip);
+            rmx = max(rmx, a);
+            if (part && a > cmax[c]) atomicMax(&cmax[c], a);
+          }
+        }
+        rmx = __reduce_max_sync(0xffffffffu, rmx);
+        if (lane == 0 && vq && range_error<kOut16>(rmx)) set_status(status, IMQ_ERR_RANGE);
+        if (lane == 0 && rowmax) rowmax[r] = (int32_t)rmx;
+      }
       __syncwarp();
+    }
+    if (inplace && part) {
+      if (lane == 0) s_done[warp] = done;
+      __syncthreads();
+      for (int g = tid; g < n / 8; g += blockDim.x) {
+        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+        for (int w = 0; w < nwarps; ++w) {
+          if (!s_done[w]) continue;
+          const uint4 a = reinterpret_cast<const uint4*>(dsm + cmax_bytes + w * row_bytes)[g];
+          m0 = max_u16x2(m0, a.x);
+          m1 = max_u16x2(m1, a.y);
+          m2 = max_u16x2(m2, a.z);
+          m3 = max_u16x2(m3, a.w);
+        }
+        uint4* cm = reinterpret_cast<uint4*>(cmax) + 2 * g;
+        uint4 c0 = cm[0], c1 = cm[1];
+        c0.x = max(c0.x, m0 & 0xFFFFu); c0.y = max(c0.y, m0 >> 16);
+        c0.z = max(c0.z, m1 & 0xFFFFu); c0.w = max(c0.w, m1 >> 16);
+        c1.x = max(c1.x, m2 & 0xFFFFu); c1.y = max(c1.y, m2 >> 16);
+        c1.z = max(c1.z, m3 & 0xFFFFu); c1.w = max(c1.w, m3 >> 16);
+        cm[0] = c0;
+        cm[1] = c1;
+      }
+      __syncthreads();
     }
   }
   if (part) {
@@ -438,7 +736,7 @@ __global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
   const int colstride = (n + 7) / 8 * 8;  // elements; keeps every column 16-byte aligned
   T* S = reinterpret_cast<T*>(dsm);       // [CW][colstride]
   uint32_t* rmax = reinterpret_cast<uint32_t*>(dsm + (size_t)CW * colstride * sizeof(T));  // [rows]
-  __shared__ uint32_t hist_all[CW][256];
+  __shared__ uint32_t hist_all[CW][kSelWords];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t c0 = (int64_t)blockIdx.x * CW;
   const int ncol = cols - c0 < CW ? (int)(cols - c0) : CW;
@@ -448,12 +746,25 @@ __global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
   constexpr int SEG = CW / V;  // 16-byte pieces per slab row (0 when a slab row is narrower)
   constexpr int SEGD = SEG > 0 ? SEG : 1;  // divisor of the branch below, which SEG = 0 never takes
   if (SEG > 0 && vec && ncol == CW) {
-    for (int i = tid; i < n * SEG; i += CW * 32) {
-      const int r = i / SEGD, sg = i % SEGD;
-      const uint4 w = __ldcs(reinterpret_cast<const uint4*>(X + r * ld + c0) + sg);
-      const T* e = reinterpret_cast<const T*>(&w);
+    // kB loads in flight per thread before their transposed stores (see warp_copy16)
+    constexpr int kB = 8;
+    for (int i0 = tid; i0 < n * SEG; i0 += CW * 32 * kB) {
+      uint4 buf[kB];
 #pragma unroll
-      for (int j = 0; j < V; ++j) S[(sg * V + j) * colstride + r] = e[j];
+      for (int b = 0; b < kB; ++b) {
+        const int i = i0 + b * CW * 32;
+        if (i < n * SEG) buf[b] = __ldcs(reinterpret_cast<const uint4*>(X + (i / SEGD) * ld + c0) + i % SEGD);
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int i = i0 + b * CW * 32;
+        if (i < n * SEG) {
+          const int r = i / SEGD, sg = i % SEGD;
+          const T* e = reinterpret_cast<const T*>(&buf[b]);
+#pragma unroll
+          for (int j = 0; j < V; ++j) S[(sg * V + j) * colstride + r] = e[j];
+        }
+      }
     }
   } else {
     for (int i = tid; i < n * CW; i += CW * 32) {
@@ -462,46 +773,82 @@ __global__ void __launch_bounds__(CW * 32, 1) k_rtn_cols_staged(
     }
   }
   __syncthreads();
+  // vectorised quantisation when the column is written as one contiguous, aligned output row
+  const bool vq = trans_out && n % 8 == 0 && ldq % 8 == 0 && (reinterpret_cast<uintptr_t>(Xint) & 15) == 0;
+  // bf16 in, int16 out: columns quantised in place (|x_int| kept in the staged column) and the row maxima
+  // folded afterwards over the CTA's columns, every thread owning whole 8-row groups
+  const bool inplace = sizeof(T) == 2 && kOut16 && vq;
+  __shared__ int s_done[CW];
   if (warp < ncol) {
-    const T* col = S + warp * colstride;
+    T* col = S + warp * colstride;
     const int64_t c = c0 + warp;
     uint32_t mk, bad;
-    warp_key_stats(col, n, &mk, &bad);
-    const float q = Key<T>::from_key(select_key(col, n, krank, hist_all[warp]));
+    const float q = Key<T>::from_key(stats_and_select(col, n, krank, hist_all[warp], &mk, &bad));
     float s, dl;
-    scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
+    const float qu = scale_from_q(q, Key<T>::from_key(mk), beta, &s, &dl);
     if (lane == 0) {
       delta[c] = dl;
-      if (qval) qval[c] = q;
+      if (qval) qval[c] = qu;
       if (bad) set_status(status, IMQ_ERR_NONFINITE);
     }
-    uint32_t cmx = 0;
-    // vectorised quantisation when the column is written as one contiguous, aligned output row
-    const bool vq = trans_out && n % 8 == 0 && ldq % 8 == 0 && (reinterpret_cast<uintptr_t>(Xint) & 15) == 0;
-    if (!bad && vq) {
-      for (int g = lane; g < n / 8; g += 32) {
-        uint32_t a[8];
-        quant8<T, kOut16>(col + g * 8, s, Xint, c * ldq + g * 8, status, clip, a);
+    __syncwarp();
+    if (inplace) {
+      uint32_t cmx = 0;
+      if (!bad) {
+        quant_bf16_inplace(reinterpret_cast<uint16_t*>(col), n, s, clip, static_cast<int16_t*>(Xint) + c * ldq);
+        bool range;
+        cmx = group_max_int<kOut16>(Key<T>::from_key(mk), s, clip, &range);
+        if (lane == 0 && range) set_status(status, IMQ_ERR_RANGE);
+      }
+      if (lane == 0) {
+        s_done[warp] = bad ? 0 : 1;
+        if (colmax) colmax[c] = (int32_t)cmx;
+      }
+    } else {
+      uint32_t cmx = 0;
+      if (!bad && vq) {
+        for (int g = lane; g < n / 8; g += 32) {
+          uint32_t a[8];
+          quant8<T, kOut16>(col + g * 8, s, Xint, c * ldq + g * 8, clip, a);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) cmx = max(cmx, a[j]);
-        if (part) max8_shared(rmax + g * 8, a);
+          for (int j = 0; j < 8; ++j) cmx = max(cmx, a[j]);
+          if (part) max8_shared(rmax + g * 8, a);
+        }
+      } else if (!bad) {
+        for (int r = lane; r < n; r += 32) {
+          const uint32_t a = quant_one<kOut16>(Key<T>::value(col[r]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
+                                               status, clip);
+          cmx = max(cmx, a);
+          if (part && a > rmax[r]) atomicMax(&rmax[r], a);
+        }
       }
-    } else if (!bad) {
-      for (int r = lane; r < n; r += 32) {
-        const uint32_t a = quant_one<kOut16>(Key<T>::value(col[r]), s, Xint, trans_out ? c * ldq + r : r * ldq + c,
-                                             status, clip);
-        cmx = max(cmx, a);
-        if (part && a > rmax[r]) atomicMax(&rmax[r], a);
-      }
+      cmx = __reduce_max_sync(0xffffffffu, cmx);
+      if (lane == 0 && !bad && vq && range_error<kOut16>(cmx)) set_status(status, IMQ_ERR_RANGE);
+      if (lane == 0 && colmax) colmax[c] = (int32_t)cmx;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cmx = max(cmx, __shfl_xor_sync(0xffffffffu, cmx, o));
-    if (lane == 0 && colmax) colmax[c] = (int32_t)cmx;
   }
   if (part) {
     __syncthreads();
     int32_t* mine = part + (int64_t)blockIdx.x * rows;
-    for (int r = tid; r < n; r += CW * 32) mine[r] = (int32_t)rmax[r];
+    if (inplace) {
+      // row maxima of this CTA's columns: 8 rows per thread and step, 16-byte reads of each column
+      for (int g = tid; g < n / 8; g += CW * 32) {
+        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+        for (int w = 0; w < ncol; ++w) {
+          if (!s_done[w]) continue;
+          const uint4 a = *reinterpret_cast<const uint4*>(S + w * colstride + g * 8);
+          m0 = max_u16x2(m0, a.x);
+          m1 = max_u16x2(m1, a.y);
+          m2 = max_u16x2(m2, a.z);
+          m3 = max_u16x2(m3, a.w);
+        }
+        int4* o = reinterpret_cast<int4*>(mine + g * 8);
+        o[0] = make_int4((int)(m0 & 0xFFFFu), (int)(m0 >> 16), (int)(m1 & 0xFFFFu), (int)(m1 >> 16));
+        o[1] = make_int4((int)(m2 & 0xFFFFu), (int)(m2 >> 16), (int)(m3 & 0xFFFFu), (int)(m3 >> 16));
+      }
+    } else {
+      for (int r = tid; r < n; r += CW * 32) mine[r] = (int32_t)rmax[r];
+    }
   }
 }
 
@@ -569,9 +916,9 @@ __global__ void __launch_bounds__(kThreads) k_rtn_cols(
     const int64_t cg = (int64_t)blockIdx.x * CW + tid;
     float s, d;
     const float q = Key<T>::from_key(s_prefix[tid]);
-    scale_from_q(q, Key<T>::from_key(s_maxkey[tid]), beta, &s, &d);
+    const float qu = scale_from_q(q, Key<T>::from_key(s_maxkey[tid]), beta, &s, &d);
     delta[cg] = d;
-    if (qval) qval[cg] = q;
+    if (qval) qval[cg] = qu;
     s_s[tid] = s;
   }
   if (tid == 0 && s_bad) set_status(status, IMQ_ERR_NONFINITE);
@@ -659,12 +1006,12 @@ __global__ void k_tensor_select(TensorState* ts, int pass, int last, int beta, f
     if (last) {
       const float q = Key<T>::from_key(ts->prefix);
       float s, dl;
-      scale_from_q(q, Key<T>::from_key(ts->maxkey), beta, &s, &dl);
+      const float qu = scale_from_q(q, Key<T>::from_key(ts->maxkey), beta, &s, &dl);
       ts->s = s;
       ts->delta = dl;
       ts->q = q;
       delta[0] = dl;
-      if (qval) qval[0] = q;
+      if (qval) qval[0] = qu;
       if (ts->nonfinite) {
         set_status(status, IMQ_ERR_NONFINITE);
         ts->s = 0.0f;
@@ -762,11 +1109,11 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
   int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
   if (nwarps > kThreads / 32) nwarps = kThreads / 32;
   const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
-  int per_sm = (int)(kBudget / (smem + 9 * 1024));
+  int per_sm = (int)(kBudget / (smem + kThreads / 32 * kSelWords * 4 + 1024));
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 4) per_sm = 4;
-  const int64_t blocks = (rows + nwarps - 1) / nwarps;
-  const int64_t grid = blocks < (int64_t)sms * per_sm ? blocks : (int64_t)sms * per_sm;
+  // one CTA per row up to every resident slot: rows are dealt to the CTAs in turn
+  const int64_t grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
   const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
                    ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   int32_t* part = nullptr;
@@ -894,11 +1241,11 @@ imq_status run_rows_noalloc(const T* X, int64_t rows, int64_t cols, int64_t ld, 
   int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
   if (nwarps > kThreads / 32) nwarps = kThreads / 32;
   const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
-  int per_sm = (int)(kBudget / (smem + 9 * 1024));
+  int per_sm = (int)(kBudget / (smem + kThreads / 32 * kSelWords * 4 + 1024));
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 4) per_sm = 4;
-  const int64_t blocks = (rows + nwarps - 1) / nwarps;
-  const int64_t grid = blocks < (int64_t)sms * per_sm ? blocks : (int64_t)sms * per_sm;
+  // one CTA per row up to every resident slot: rows are dealt to the CTAs in turn
+  const int64_t grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
   const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
                    ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   int32_t* part = nullptr;
@@ -992,7 +1339,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
   extern __shared__ __align__(16) unsigned char dsm[];
   const int64_t row_bytes = (f.cols * (int64_t)sizeof(T) + 15) / 16 * 16;
   const int64_t wbytes = fused_warp_bytes<T>(f.cols);
-  __shared__ uint32_t hist_all[kThreads / 32][256];
+  __shared__ uint32_t hist_all[kThreads / 32][kSelWords];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t nchunk = f.K_unp / 16;
   // [rows of nwarps warps][block starts, int32 x nchunk][first inner levels, int8 x nchunk]
@@ -1013,19 +1360,18 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
   constexpr int V = 16 / sizeof(T);
   const int n = (int)f.cols;
   const bool vec = (f.cols % V == 0) && (f.ld % V == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
-  for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < f.rows; r += (int64_t)gridDim.x * nwarps) {
+  // rows dealt to the CTAs in turn (row r to CTA r mod gridDim.x): every SM gets the same number of rows
+  // to within one per CTA
+  for (int64_t r = (int64_t)warp * gridDim.x + blockIdx.x; r < f.rows; r += (int64_t)gridDim.x * nwarps) {
     const T* xr = X + r * f.ld;
     if (vec) {
-      const uint4* src = reinterpret_cast<const uint4*>(xr);
-      uint4* dst = reinterpret_cast<uint4*>(row);
-      for (int c = lane; c < n / V; c += 32) dst[c] = __ldcs(src + c);
+      warp_copy16<8>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), n / V, lane);
     } else {
       for (int c = lane; c < n; c += 32) row[c] = xr[c];
     }
     __syncwarp();
     uint32_t mk, bad;
-    warp_key_stats(row, n, &mk, &bad);
-    const float q = Key<T>::from_key(select_key(row, n, f.krank, hist));
+    const float q = Key<T>::from_key(stats_and_select(row, n, f.krank, hist, &mk, &bad));
     float s, dl;
     scale_from_q(q, Key<T>::from_key(mk), f.beta, &s, &dl);
     if (lane == 0) f.delta[r] = dl;
@@ -1119,11 +1465,11 @@ imq_status run_rtn_unpack(const T* X, const FusedArgs& f, DeviceState* ds, cudaS
   if (nwarps < 1) return IMQ_ERR_UNSUPPORTED;
   if (nwarps > kThreads / 32) nwarps = kThreads / 32;
   const size_t smem = (size_t)nwarps * per_warp + meta;
-  int per_sm = (int)(kBudget / (smem + 9 * 1024));
+  int per_sm = (int)(kBudget / (smem + kThreads / 32 * kSelWords * 4 + 1024));
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 4) per_sm = 4;
-  const int64_t blocks = (f.rows + nwarps - 1) / nwarps;
-  const int64_t grid = blocks < (int64_t)ds->num_sms * per_sm ? blocks : (int64_t)ds->num_sms * per_sm;
+  // one CTA per row up to every resident slot: rows are dealt to the CTAs in turn
+  const int64_t grid = f.rows < (int64_t)ds->num_sms * per_sm ? f.rows : (int64_t)ds->num_sms * per_sm;
   IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_rtn_unpack_rows<T>), smem));
   k_rtn_unpack_rows<T><<<(unsigned)grid, kThreads, smem, st>>>(X, f, nwarps, meta_smem);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;

@@ -114,7 +114,8 @@ typedef enum { IMQ_DIR_NONE = 0, IMQ_DIR_OUTER = 1, IMQ_DIR_INNER = 2, IMQ_DIR_B
  *         weight W stored K x N is quantised per output channel straight into the N x K layout that
  *         imq_plan takes as B with transB = 1.
  * delta   device, fp32, 1 / rows / cols entries for PER_TENSOR / PER_ROW / PER_COL.
- * qval    device or NULL, fp32, same length as delta: the selected percentile values q_g.
+ * qval    device or NULL, fp32, same length as delta: the q each scale was derived from -- the
+ *         selected percentile q_g, or the group's maximum where q_g is 0 (0 when that is 0 too).
  * rowmax  device or NULL, int32[rows]: max |x_int| over each row of X (whatever trans_out is).
  * colmax  device or NULL, int32[cols]: max |x_int| over each column of X.
  * Errors: IMQ_ERR_ARG at once; IMQ_ERR_NONFINITE / IMQ_ERR_RANGE through the device status word.
@@ -159,7 +160,7 @@ imq_status imq_rtn_quantize_ex(const void *X, imq_dtype xt, int64_t rows, int64_
  *
  * Scratch needed: 4 * cols * G bytes when colmax is requested, where G is the number of CTAs the
  * per-row kernel uses (at most 4 per SM; fewer for wide rows).  On 148 SMs any cols <= 3542 fits,
- * and a 2048 x 4096 bf16 activation takes 4 MiB.  None when colmax is NULL.  Nothing in the
+ * and a 2048 x 4096 bf16 activation takes 4.6 MiB (296 CTAs).  None when colmax is NULL.  Nothing in the
  * scratch has to start at zero: each CTA writes its whole slice before the reduction reads it.
  * Errors: those of imq_rtn_quantize, plus IMQ_ERR_UNSUPPORTED, returned at once with nothing launched,
  * when the scratch needed exceeds IMQ_NOALLOC_SCRATCH_BYTES.

@@ -60,6 +60,59 @@ def test_quantize_parity(imq, dtype, gran, shape, p, beta):
         assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0))
 
 
+def _select_patterns(rng, n):
+    """bf16 groups of n entries built against a select that brackets the rank from an evenly spaced
+    sample: sorted groups, ties, a period equal to the sample spacing (the sample then sees only the
+    large entries and the bracket misses), heavy tails, signed zeros and subnormals."""
+    spaced = ((2 * np.arange(256) + 1) * n) // 512
+    rows = []
+    rows.append(rng.standard_normal(n))
+    rows.append(np.sort(np.abs(rng.standard_normal(n))))
+    rows.append(-np.sort(np.abs(rng.standard_normal(n)))[::-1])
+    rows.append(np.full(n, 0.5))
+    rows.append(rng.integers(0, 3, n) * 0.25 * rng.choice([-1.0, 1.0], n))
+    r = rng.standard_normal(n) * 0.01
+    r[spaced] = 10.0
+    rows.append(r)
+    r = rng.standard_normal(n)
+    r[: n // 2] = 0.0
+    rows.append(rng.permutation(r))
+    rows.append(np.clip(rng.standard_cauchy(n), -1e3, 1e3))
+    r = rng.choice([1e-40, -1e-40, 0.0, -0.0, 3e-39], n)
+    normal = rng.random(n) < 0.6
+    r[normal] = rng.standard_normal(int(normal.sum())) * 1e-30
+    rows.append(r)
+    rows.append(np.zeros(n))
+    r = rng.standard_normal(n) * 1e-3
+    r[rng.integers(n)] = 2.0
+    rows.append(r)
+    r = rng.standard_normal(n)
+    r[rng.choice(n, n // 20, replace=False)] *= 60.0  # 5 % heavy hitters: the rank sits at their edge
+    rows.append(r)
+    return np.stack(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("n", [1024, 1031, 4096, 11008])
+@pytest.mark.parametrize("p", [0.95, 0.5, 1.0, 0.999, 1e-4])
+def test_quantize_select_adversarial_groups(imq, n, p):
+    """The sampled bf16 select (groups of 1024 and more) against the oracle's full sort, per row and per
+    column (the transposed matrix: the staged column kernel), including the groups that defeat it."""
+    rng = np.random.default_rng(zlib.crc32(repr(("sel", n, p)).encode()))
+    x = _select_patterns(rng, n)
+    for gran, mat in ((oracle.PER_ROW, x), (oracle.PER_COL, np.ascontiguousarray(x.T))):
+        bits = workloads.f32_to_bf16_bits(mat)
+        want_i, want_d, want_q = oracle.rtn_quantize(oracle.bf16_bits_to_f32(bits), gran, p, 15)
+        X = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+        r = imq.imq_rtn_quantize(X, gran, p, 15, out_dtype=torch.int32)
+        torch.cuda.synchronize()
+        assert imq.imq_device_status() == imq.IMQ_OK
+        assert np.array_equal(r.qval.cpu().numpy().view(np.uint32), want_q.view(np.uint32)), gran
+        assert np.array_equal(r.delta.cpu().numpy().view(np.uint32), want_d.view(np.uint32)), gran
+        assert np.array_equal(r.xint.cpu().numpy().astype(np.int64), want_i), gran
+        assert np.array_equal(r.rowmax.cpu().numpy(), np.abs(want_i).max(axis=1)), gran
+        assert np.array_equal(r.colmax.cpu().numpy(), np.abs(want_i).max(axis=0)), gran
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("gran", [oracle.PER_TENSOR, oracle.PER_ROW, oracle.PER_COL])
 @pytest.mark.parametrize("shape", [(3, 5), (37, 129), (257, 1000), (1000, 64), (20000, 8)])

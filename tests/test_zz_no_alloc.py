@@ -47,8 +47,8 @@ def _scratch_needed(rows, cols, itemsize, sms):
         return None
     nwarps = min((budget - cmax) // row_bytes, 8)
     smem = cmax + nwarps * row_bytes
-    per_sm = min(max(budget // (smem + 9 * 1024), 1), 4)
-    grid = min((rows + nwarps - 1) // nwarps, sms * per_sm)
+    per_sm = min(max(budget // (smem + 8 * 384 * 4 + 1024), 1), 4)
+    grid = min(rows, sms * per_sm)
     return grid * cols * 4
 
 
