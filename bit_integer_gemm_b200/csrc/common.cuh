@@ -301,31 +301,50 @@ __device__ __forceinline__ void warp_count(uint32_t* base, uint32_t key, bool ac
   if ((int)(threadIdx.x & 31) == leader) atomicAdd(base + key, (uint32_t)__popc(peers));
 }
 
-// Digit l (base 2^bm1, sign-magnitude) of 16 int16 entries held as 8 words (two entries per word, low
-// half first), as 16 bytes in entry order.  |entry| per half without a carry between halves; the
-// digit's bits are masked, then shifted down within each half; a byte permute gathers the four digits of
-// two words; negative entries' digits are negated byte-wise as (0x80808080 - d) ^ 0x80808080 (a digit
-// is at most 127, so no byte borrows).  Digits with l * bm1 >= 16 are zero for int16 magnitudes.
-__device__ __forceinline__ uint4 digits16_i16(const uint32_t (&w)[8], int l, int bm1) {
+// Magnitudes and signs of 16 int16 entries held as 8 words (two entries per word, low half first):
+// |entry| per half without a carry between halves, and per 4 entries a byte mask (0xFF where the entry
+// is negative) in entry order.
+struct Mag16 {
+  uint32_t a[8];
+  uint32_t neg[4];
+};
+__device__ __forceinline__ Mag16 mag16_i16(const uint32_t (&w)[8]) {
+  Mag16 m;
+  uint32_t S[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const uint32_t sgn = (w[h] >> 15) & 0x00010001u;  // 1 in each negative half
+    S[h] = sgn * 0xFFFFu;                              // 0xFFFF in each negative half
+    m.a[h] = (w[h] ^ S[h]) + sgn;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) m.neg[q] = __byte_perm(S[2 * q], S[2 * q + 1], 0x6420);
+  return m;
+}
+
+// Digit l (base 2^bm1, sign-magnitude) of the 16 entries of m, as 16 bytes in entry order: the digit's
+// bits are masked, then shifted down within each half; a byte permute gathers the four digits of two
+// words; negative entries' digits are negated byte-wise as (0x80808080 - d) ^ 0x80808080 (a digit is at
+// most 127, so no byte borrows).  Digits with l * bm1 >= 16 are zero for int16 magnitudes.
+__device__ __forceinline__ uint4 digits16_from(const Mag16& m, int l, int bm1) {
   const int sh = l * bm1;
   if (sh >= 16) return make_uint4(0u, 0u, 0u, 0u);
   const uint32_t m2 = ((((1u << bm1) - 1u) << sh) & 0xFFFFu) * 0x00010001u;
   uint32_t o[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint32_t d[2], S[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t ww = w[2 * q + h];
-      const uint32_t sgn = (ww >> 15) & 0x00010001u;
-      S[h] = sgn * 0xFFFFu;
-      d[h] = (((ww ^ S[h]) + sgn) & m2) >> sh;
-    }
-    const uint32_t pd = __byte_perm(d[0], d[1], 0x6420), neg = __byte_perm(S[0], S[1], 0x6420);
+    const uint32_t d0 = (m.a[2 * q] & m2) >> sh, d1 = (m.a[2 * q + 1] & m2) >> sh;
+    const uint32_t pd = __byte_perm(d0, d1, 0x6420);
     const uint32_t nd = (0x80808080u - pd) ^ 0x80808080u;
-    o[q] = (pd & ~neg) | (nd & neg);
+    o[q] = (pd & ~m.neg[q]) | (nd & m.neg[q]);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Digit l of 16 int16 entries held as 8 words, as 16 bytes in entry order.
+__device__ __forceinline__ uint4 digits16_i16(const uint32_t (&w)[8], int l, int bm1) {
+  if (l * bm1 >= 16) return make_uint4(0u, 0u, 0u, 0u);
+  return digits16_from(mag16_i16(w), l, bm1);
 }
 
 // Number of base-2^(b-1) digits of m (>= 1).

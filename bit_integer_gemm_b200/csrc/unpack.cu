@@ -10,7 +10,12 @@
 // the digits of every inner level); for the pure strategies one of L > 1, lk > 0 never holds.
 //
 // Both unpacked operands are K-major (the inner index contiguous) because that is what the tcgen05
-// GEMM reads through TMA.  Two kernels cover the two storage orders of a source matrix:
+// GEMM reads through TMA.  The kernels cover the two storage orders of a source matrix:
+//   k_unpack_lines16  int16 source lines that are stored rows (A, or B given as B^T): one warp per line
+//                  with the line staged, digits computed per 16-position block for every output level;
+//                  it also zeroes the unused lines of OUTER groups.
+//   k_unpack_lines / k_unpack_rows  the same for int32 sources (and lines too long to stage): digit
+//                  planes in shared memory, 16-byte copies out of them.
 //   k_unpack_rows  the source line is a stored row (A, or B given as B^T): a CTA writes the digit planes
 //                  of a batch of lines to shared memory and streams out their unpacked lines, 16-byte
 //                  copies for the inner blocks the plan marked contiguous (k_unpack_rows_direct gathers
@@ -25,6 +30,25 @@
 
 namespace imq {
 namespace {
+
+// Copies n16 16-byte pieces from global to shared memory over one warp, kBatch loads in flight per lane
+// before their stores (a store waits for its load).
+template <int kBatch>
+__device__ __forceinline__ void warp_copy16_global(const uint4* __restrict__ src, uint4* dst, int n16, int lane) {
+  for (int c0 = lane; c0 < n16; c0 += 32 * kBatch) {
+    uint4 buf[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < n16) buf[j] = src[c];
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int c = c0 + 32 * j;
+      if (c < n16) dst[c] = buf[j];
+    }
+  }
+}
 
 // Row gather: a CTA takes a batch of NL source lines and writes their digit planes to shared memory,
 // plane[b][l][t] = d_l(line b, entry t) for the P levels the batch needs, one byte each.  Then each
@@ -350,6 +374,189 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* __restrict__ X, i
   }
 }
 
+// Digit kL (base 2^kBm1, sign-magnitude) of the 16 entries of m as 16 bytes in entry order, with the
+// level and base fixed at compile time (digits16_from with its masks and shifts folded).
+template <int kBm1, int kL>
+__device__ __forceinline__ uint4 digits16_fixed(const Mag16& m) {
+  constexpr int sh = kL * kBm1;
+  if constexpr (sh >= 16) {
+    return make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    constexpr uint32_t m2 = ((((1u << kBm1) - 1u) << sh) & 0xFFFFu) * 0x00010001u;
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t pd = __byte_perm((m.a[2 * q] & m2) >> sh, (m.a[2 * q + 1] & m2) >> sh, 0x6420);
+      const uint32_t nd = (0x80808080u - pd) ^ 0x80808080u;
+      o[q] = (pd & ~m.neg[q]) | (nd & m.neg[q]);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take the unrolled path
+
+// Row gather for int16 sources, one warp per source line (base 2^kBm1 fixed at compile time).  The warp
+// stages its line in its own shared memory (16-byte loads, all of a lane's in flight) and writes the
+// line's L unpacked lines, 16 inner positions per lane and step: a block the plan marked contiguous
+// (t0..t0+15, t0 % 16 == 0, one inner level lk0) takes the magnitudes and signs of its 16 entries once
+// and emits the digit (l + lk0) for every output line l from them; any other block is gathered entry by
+// entry.  The per-block plan metadata is staged in shared memory once per CTA.  Lines are dealt to the
+// CTAs in turn (line i to CTA i mod gridDim.x).  After its lines, each CTA zeroes the unused lines of the
+// OUTER groups dealt to it (group g to CTA g mod gridDim.x), lines n*L .. G-1 of a group of n sources of
+// level L, which no source line writes.
+template <int kBm1>
+__global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* __restrict__ X, int64_t nlines, int64_t K,
+                                                           int64_t ld, int nwarps, int outer,
+                                                           const int8_t* __restrict__ lvl,
+                                                           const int32_t* __restrict__ pos,
+                                                           const int32_t* __restrict__ tK,
+                                                           const int8_t* __restrict__ lk,
+                                                           const int32_t* __restrict__ blk16, int64_t K_unp,
+                                                           int8_t* __restrict__ out,
+                                                           const int32_t* __restrict__ grpL,
+                                                           const int32_t* __restrict__ grpN, int64_t ngrp, int G) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t Kr = (K + 15) / 16 * 16;  // staged line length in entries (32-byte multiple)
+  const int nchunk = (int)(K_unp / 16);
+  // [lines of nwarps warps, int16 x Kr][block starts, int32 x nchunk][first inner levels, int8 x nchunk]
+  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)nwarps * Kr * 2);
+  int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);
+  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
+    s_blk[c] = blk16[c];
+    s_lk0[c] = lk[(int64_t)c * 16];
+  }
+  __syncthreads();
+  if (warp < nwarps) {
+    int16_t* row = reinterpret_cast<int16_t*>(dsm) + (int64_t)warp * Kr;
+    const bool vec8 = (K % 8 == 0) && (ld % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+    for (int64_t line = (int64_t)warp * gridDim.x + blockIdx.x; line < nlines;
+         line += (int64_t)gridDim.x * nwarps) {
+      const int16_t* xr = X + line * ld;
+      if (vec8) {
+        warp_copy16_global<4>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), (int)(K / 8), lane);
+      } else {
+        for (int64_t t = lane; t < K; t += 32) row[t] = xr[t];
+      }
+      __syncwarp();
+      const int L = outer ? (int)lvl[line] : 1;
+      int8_t* o0 = out + (outer ? (int64_t)pos[line] : line) * K_unp;
+      if (L <= kFastLevels) {
+        int8_t* ol[kFastLevels];
+#pragma unroll
+        for (int l = 0; l < kFastLevels; ++l) ol[l] = o0 + (int64_t)l * K_unp;
+        for (int c = lane; c < nchunk; c += 32) {
+          const int t0 = s_blk[c];
+          const int p = c * 16;
+          uint4 d[kFastLevels];
+          if (t0 >= 0) {
+            const int lk0 = s_lk0[c];
+            if (L > 1 && lk0 > 0) {
+#pragma unroll
+              for (int l = 0; l < kFastLevels; ++l) d[l] = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+              const uint4 w0 = *reinterpret_cast<const uint4*>(row + t0);
+              const uint4 w1 = *reinterpret_cast<const uint4*>(row + t0 + 8);
+              const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              const Mag16 m = mag16_i16(w);
+              if (L == 1) {
+                d[0] = digits16_from(m, lk0, kBm1);
+              } else {
+                d[0] = digits16_fixed<kBm1, 0>(m);
+                d[1] = digits16_fixed<kBm1, 1>(m);
+                if (L > 2) d[2] = digits16_fixed<kBm1, 2>(m);
+                if (L > 3) d[3] = digits16_fixed<kBm1, 3>(m);
+              }
+            }
+          } else {
+            // gathered entry by entry (block boundaries of segments and padding; rare)
+#pragma unroll
+            for (int l = 0; l < kFastLevels; ++l) {
+              uint32_t wv[4] = {0u, 0u, 0u, 0u};
+              if (l < L) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const int4 tq = reinterpret_cast<const int4*>(tK + p)[q];
+                  const uint32_t lq = reinterpret_cast<const uint32_t*>(lk + p)[q];
+                  const int32_t tt[4] = {tq.x, tq.y, tq.z, tq.w};
+#pragma unroll
+                  for (int r = 0; r < 4; ++r) {
+                    const int lr = (int)(int8_t)(lq >> (8 * r));
+                    const int32_t dg =
+                        (tt[r] >= 0 && (L == 1 || lr == 0)) ? digit_of((int32_t)row[tt[r]], l + lr, kBm1) : 0;
+                    wv[q] |= ((uint32_t)(uint8_t)(int8_t)dg) << (8 * r);
+                  }
+                }
+              }
+              d[l] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+          }
+#pragma unroll
+          for (int l = 0; l < kFastLevels; ++l)
+            if (l < L) *reinterpret_cast<uint4*>(ol[l] + p) = d[l];
+        }
+      } else {
+        // lines of more levels (small b): one output line at a time
+        for (int c = lane; c < nchunk; c += 32) {
+          const int t0 = s_blk[c];
+          const int p = c * 16;
+          const int lk0 = t0 >= 0 ? s_lk0[c] : 0;
+          for (int l = 0; l < L; ++l) {
+            uint4 dv;
+            if (t0 >= 0) {
+              if (lk0 > 0) {
+                dv = make_uint4(0u, 0u, 0u, 0u);
+              } else {
+                const uint4 w0 = *reinterpret_cast<const uint4*>(row + t0);
+                const uint4 w1 = *reinterpret_cast<const uint4*>(row + t0 + 8);
+                const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                dv = digits16_i16(w, l, kBm1);
+              }
+            } else {
+              uint32_t wv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const int32_t t = tK[p + k];
+                const int lr = lk[p + k];
+                const int32_t dg = (t >= 0 && lr == 0) ? digit_of((int32_t)row[t], l, kBm1) : 0;
+                wv[k >> 2] |= ((uint32_t)(uint8_t)(int8_t)dg) << (8 * (k & 3));
+              }
+              dv = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            *reinterpret_cast<uint4*>(o0 + (int64_t)l * K_unp + p) = dv;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+  // unused lines of the OUTER groups dealt to this CTA
+  for (int64_t g = blockIdx.x; g < ngrp; g += gridDim.x) {
+    const int64_t first = g * G + (int64_t)grpN[g] * grpL[g];
+    const int64_t n16 = ((g + 1) * G - first) * K_unp / 16;
+    uint4* o = reinterpret_cast<uint4*>(out + first * K_unp);
+    for (int64_t k = threadIdx.x; k < n16; k += blockDim.x) o[k] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <int kBm1>
+imq_status launch_lines16(const int16_t* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
+                          const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
+                          const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL, const int32_t* grpN,
+                          int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st) {
+  auto kern = k_unpack_lines16<kBm1>;
+  IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
+  int per_sm = 0;
+  IMQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem));
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = (int64_t)num_sms * per_sm;
+  if (grid > nlines) grid = nlines;
+  kern<<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN,
+                                          ngrp, G);
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
 // Row gather for lines too long for shared-memory planes: digits are computed from the source line in
 // global memory (L2); lane = 4 consecutive inner positions, 128-byte coalesced stores per warp.
 template <typename T>
@@ -441,11 +648,49 @@ __global__ void k_zero_unused(const int32_t* __restrict__ grpL, const int32_t* _
   }
 }
 
+// The unused lines of an operand's OUTER groups (zeroed by the int16 row kernel itself, else by
+// k_zero_unused after the operand's unpack).
+struct ZeroJob {
+  const int32_t* grpL = nullptr;
+  const int32_t* grpN = nullptr;
+  int64_t ngrp = 0;
+  int G = 0;
+};
+
+// One operand.  *zeroed is set when the launch also zeroed the operand's unused OUTER lines.
 template <typename T>
 imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool line_is_row, int outer, int P,
                       const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
-                      const int32_t* blk16, int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st) {
+                      const int32_t* blk16, int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st,
+                      const ZeroJob& zj, bool* zeroed) {
+  *zeroed = false;
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
+  if constexpr (sizeof(T) == 2) {
+    // int16 rows: one warp per line with the line staged (8 warps while their lines fit in 64 KB, so that
+    // three CTAs share an SM; fewer for longer lines), the block metadata staged once per CTA
+    const int64_t Kr = (K + 15) / 16 * 16;
+    const int64_t nchunk = K_unp / 16;
+    int nw = (int)((64 * 1024) / (Kr * 2));
+    if (nw < 1) nw = (int)((192 * 1024) / (Kr * 2)) >= 1 ? 1 : 0;
+    if (nw > 8) nw = 8;
+    const size_t smem = (size_t)nw * Kr * 2 + (size_t)nchunk * 5;
+    if (line_is_row && nw >= 1 && nchunk <= kMetaMaxChunks && smem <= 200 * 1024 && bm1 >= 1 && bm1 <= 7) {
+      const int16_t* X16 = reinterpret_cast<const int16_t*>(X);
+      const int64_t ng = outer ? zj.ngrp : 0;
+      imq_status s;
+      switch (bm1) {
+        case 1: s = launch_lines16<1>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+        case 2: s = launch_lines16<2>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+        case 3: s = launch_lines16<3>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+        case 4: s = launch_lines16<4>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+        case 5: s = launch_lines16<5>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+        case 6: s = launch_lines16<6>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+        default: s = launch_lines16<7>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
+      }
+      *zeroed = s == IMQ_OK;
+      return s;
+    }
+  }
   if (line_is_row) {
     // P planes per line: the levels an output line can ask for (line level + inner level)
     const int64_t Kp = (K + 15) / 16 * 16;
@@ -511,18 +756,22 @@ imq_status unpack_typed(const imq_plan_t* pl, const T* A, const T* B, int8_t* Au
   const int pb_o = b_outer ? I.lmax_b_col : 1, pb_i = b_inner ? I.lmax_b_row : 1;
   const int pa = pa_o > pa_i ? pa_o : pa_i;
   const int pb = pb_o > pb_i ? pb_o : pb_i;
+  ZeroJob za, zb;
+  if (a_outer) za = ZeroJob{pl->grpA_L, pl->grpA_n, pl->n_grp_a, IMQ_A_GROUP};
+  if (b_outer) zb = ZeroJob{pl->grpB_L, pl->grpB_n, pl->n_grp_b, IMQ_B_GROUP};
+  bool za_done = false, zb_done = false;
   imq_status s = unpack_one<T>(A, I.M, I.K, pl->lda, !pl->transA, a_outer, pa, pl->lv_a_row, pl->posA, pl->tK,
-                               pl->lAk, pl->blk16, I.K_unp, bm1, Au, num_sms, st);
+                               pl->lAk, pl->blk16, I.K_unp, bm1, Au, num_sms, st, za, &za_done);
   if (s != IMQ_OK) return s;
   // B'^T lines are the logical columns of B: stored rows only when B is given transposed
   s = unpack_one<T>(B, I.N, I.K, pl->ldb, pl->transB != 0, b_outer, pb, pl->lv_b_col, pl->posB, pl->tK, pl->lBk,
-                    pl->blk16, I.K_unp, bm1, Bu, num_sms, st);
+                    pl->blk16, I.K_unp, bm1, Bu, num_sms, st, zb, &zb_done);
   if (s != IMQ_OK) return s;
   if (I.K_unp > 0) {
-    if (a_outer && pl->n_grp_a > 0)
+    if (a_outer && pl->n_grp_a > 0 && !za_done)
       k_zero_unused<<<(unsigned)(pl->n_grp_a < 4096 ? pl->n_grp_a : 4096), 256, 0, st>>>(
           pl->grpA_L, pl->grpA_n, pl->n_grp_a, IMQ_A_GROUP, I.K_unp, Au);
-    if (b_outer && pl->n_grp_b > 0)
+    if (b_outer && pl->n_grp_b > 0 && !zb_done)
       k_zero_unused<<<(unsigned)(pl->n_grp_b < 4096 ? pl->n_grp_b : 4096), 256, 0, st>>>(
           pl->grpB_L, pl->grpB_n, pl->n_grp_b, IMQ_B_GROUP, I.K_unp, Bu);
   }
