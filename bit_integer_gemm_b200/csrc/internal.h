@@ -25,6 +25,9 @@ imq_status device_state(DeviceState** out);
 // attribute call costs microseconds of host time, so it is made only when no earlier call on this device
 // already set a limit at least as large.
 cudaError_t ensure_smem(const void* fn, size_t bytes);
+// Resident blocks per SM of kernel fn at this block size and dynamic shared memory (the occupancy
+// query, cached per device, kernel and configuration).
+cudaError_t blocks_per_sm(const void* fn, int threads, size_t smem, int* out);
 // out[i] = max over p < nparts of part[p * n + i] (int32, non-negative); nparts may be 0 (out = 0).
 imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st);
 

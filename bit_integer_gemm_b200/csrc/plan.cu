@@ -97,6 +97,7 @@ struct LevelArgs {
   int8_t* lv[4];
   int64_t n[4];
   int32_t bm1;
+  int32_t* keep_a_col;     // when set, A's column maxima mx[1] are copied here (kept in the plan)
   Summary* sum;
   const int32_t* status;  // the device status word, copied into the summary by block 0
   HostSummary* hsum;      // device address of the mapped host copy
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
       int L = 1;
       if (in) {
         const uint32_t m = (uint32_t)a.mx[v][i];
+        if (v == 1 && a.keep_a_col) a.keep_a_col[i] = (int32_t)m;
         L = a.lvin[v] ? (int)a.lvin[v][i] : level_of(m, a.bm1);
         a.lv[v][i] = (int8_t)L;
         bsum[v] += (unsigned)L;
@@ -206,10 +208,8 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   for (int i = tid; i < (int)(sizeof(Summary) / 4); i += blockDim.x) dst[i] = src[i];
   __threadfence_system();
   __syncthreads();
-  if (tid == 0) {
-    *reinterpret_cast<volatile uint32_t*>(&a.hsum->seq) = a.seq;
-    __threadfence_system();
-  }
+  // the fence above orders the summary before `seq`; nothing after it needs to wait for the write
+  if (tid == 0) *reinterpret_cast<volatile uint32_t*>(&a.hsum->seq) = a.seq;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -722,11 +722,15 @@ __device__ void outer_map_class(const OuterClass c, const int8_t* __restrict__ l
 // The segment, class and group tables of a plan.  They travel inside the launch's parameters when the
 // segments fit (the usual case: a separate upload would cost a copy and an event on the host); the
 // parameter block is read in place (__grid_constant__).
-constexpr int kParamSegs = 48;
+// Tables passed inline in the maps kernel's parameters when they fit (about 1.3 KB, so the launch stays
+// within the classic 4 KB parameter space); larger plans upload them to device memory instead.
+constexpr int kParamSegs = 24;
+constexpr int kParamCls = 24;
+constexpr int kParamGrps = 16;
 struct MapsTables {
   InnerSeg segs[kParamSegs];
-  OuterClass cls[2 * kLv];
-  InnerGroup grps[IMQ_MAX_GROUPS];
+  OuterClass cls[kParamCls];
+  InnerGroup grps[kParamGrps];
 };
 
 // Stage 2 of a plan in one launch: blocks [0, ngrp) build the inner map of one exponent group each, the
@@ -934,8 +938,6 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     lmx[1] = a_colmax;
     lmx[2] = b_rowmax;
     lmx[3] = b_colmax;
-    if (K > 0 && cudaMemcpyAsync(mx[1], a_colmax, (size_t)K * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-      return fail(IMQ_ERR_CUDA);
   } else {
     // A stored M x K (or K x M when transposed); B stored K x N (or N x K)
     imq_status e = transA ? launch_line_max(A, it, K, M, lda, mx[1], mx[0], st)
@@ -953,6 +955,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   }
   if (cudaMemsetAsync(dsum, 0, sizeof(Summary), st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
   LevelArgs la;
+  la.keep_a_col = have_max ? mx[1] : nullptr;  // k_levels copies the caller's A column maxima there
   for (int v = 0; v < 4; ++v) {
     la.mx[v] = lmx[v];
     la.lvin[v] = nullptr;
@@ -1120,9 +1123,10 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   if (strategy == IMQ_MIX_JOINT) {
     // the exact unpacked size M_eff * N_eff * K_eff of a direction pair, from the summary: level sums
     // for the outer dimensions, the joint histogram of (A column level, B row level) for K_eff
+    // joint[x][y] is zero above the largest levels, so the sums stop there
     unsigned __int128 kk_both = 0;
-    for (int x = 1; x < kLv; ++x)
-      for (int y = 1; y < kLv; ++y) kk_both += (unsigned __int128)((unsigned)(x * y)) * S.joint[x][y];
+    for (int x = 1; x <= (int)lmax[1]; ++x)
+      for (int y = 1; y <= (int)lmax[2]; ++y) kk_both += (unsigned __int128)((unsigned)(x * y)) * S.joint[x][y];
     auto size_of = [&](int ca, int cb) {
       const unsigned __int128 me = ca == IMQ_DIR_OUTER ? (unsigned __int128)S.sum[0] : (unsigned __int128)M;
       const unsigned __int128 ne = cb == IMQ_DIR_OUTER ? (unsigned __int128)S.sum[3] : (unsigned __int128)N;
@@ -1154,10 +1158,12 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   // inner segments from the joint level histogram
   const int maxla = a_inner ? (int)lmax[1] : 1;
   const int maxlb = b_inner ? (int)lmax[2] : 1;
+  // inner indices whose (A column, B row) levels exceed (sa, sb); joint[x][y] is zero above the largest
+  // levels, so the sum stops there
   auto seg_len = [&](int sa, int sb) {
     int64_t n = 0;
-    for (int x = 1; x < kLv; ++x)
-      for (int y = 1; y < kLv; ++y) {
+    for (int x = 1; x <= (int)lmax[1]; ++x)
+      for (int y = 1; y <= (int)lmax[2]; ++y) {
         const int ea = a_inner ? x : 1, eb = b_inner ? y : 1;
         if (ea > sa && eb > sb) n += S.joint[x][y];
       }
@@ -1341,7 +1347,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   }
   if (ng > 0 || ncls > 0) {
     MapsArgs m;
-    m.inline_tables = nseg <= kParamSegs ? 1 : 0;
+    m.inline_tables = (nseg <= kParamSegs && ncls <= kParamCls && ng <= kParamGrps) ? 1 : 0;
     if (m.inline_tables) {
       memcpy(m.t.segs, hsegs, sizeof(InnerSeg) * (size_t)nseg);
       memcpy(m.t.cls, hcls, sizeof(OuterClass) * (size_t)ncls);

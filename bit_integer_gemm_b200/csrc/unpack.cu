@@ -548,7 +548,7 @@ imq_status launch_lines16(const int16_t* X, int64_t nlines, int64_t K, int64_t l
   auto kern = k_unpack_lines16<kBm1>;
   IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   int per_sm = 0;
-  IMQ_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem));
+  IMQ_CUDA_TRY(blocks_per_sm(reinterpret_cast<const void*>(kern), 256, smem, &per_sm));
   if (per_sm < 1) per_sm = 1;
   int64_t grid = (int64_t)num_sms * per_sm;
   if (grid > nlines) grid = nlines;
