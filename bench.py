@@ -185,6 +185,11 @@ class Path:
         self.ws = None
         self.info = None
         self.launches = 0
+        # the two quantisers are independent: W's runs on a second stream, joined before the plan, so that
+        # the row quantiser of X fills the SMs the column quantiser leaves idle in its last wave
+        self.aux = t.cuda.Stream(device=dev)
+        self.ev_fork = t.cuda.Event()
+        self.ev_join = t.cuda.Event()
 
     def _workspace(self, I):
         """A' and B'^T views of one workspace (1024-byte aligned), rebuilt only when the plan's sizes
@@ -248,10 +253,15 @@ class Path:
                 gemm_events[1].record()
             self.launches = 2
             return
+        main = self.torch.cuda.current_stream()
+        self.ev_fork.record(main)
+        self.aux.wait_event(self.ev_fork)
+        imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
+                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True, stream=self.aux)
         imq.imq_rtn_quantize(X, imq.IMQ_PER_ROW, g.p, g.beta, Xint=self.Xint, delta=self.dX,
                              want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
-        imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
-                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True)
+        self.ev_join.record(self.aux)
+        main.wait_event(self.ev_join)
         plan = imq.imq_plan(self.Xint, self.Wint, g.b, self.strategy, transB=True, maxes=self.mx)
         I = plan.info
         Au, Bu = self._workspace(I)
