@@ -191,22 +191,6 @@ class Path:
         self.ev_fork = t.cuda.Event()
         self.ev_join = t.cuda.Event()
 
-    def _workspace(self, I):
-        """A' and B'^T views of one workspace (1024-byte aligned), rebuilt only when the plan's sizes
-        change."""
-        key = (I["M_unp"], I["N_unp"], I["K_unp"])
-        if getattr(self, "_ws_key", None) != key:
-            need = I["M_unp"] * I["K_unp"] + I["N_unp"] * I["K_unp"] + 2048
-            if self.ws is None or self.ws.numel() < need:
-                self.ws = self.torch.empty(need, dtype=self.torch.int8, device=self.X.device)
-            na = I["M_unp"] * I["K_unp"]
-            a_off = (-self.ws.data_ptr()) % 1024
-            b_off = a_off + (na + 1023) // 1024 * 1024
-            self._views = (self.ws[a_off:a_off + na].view(I["M_unp"], I["K_unp"]),
-                           self.ws[b_off:b_off + I["N_unp"] * I["K_unp"]].view(I["N_unp"], I["K_unp"]))
-            self._ws_key = key
-        return self._views
-
     def prepare_cache(self):
         """Cached-weight mode, before any timing: W quantised per output channel, the plan made with
         the activations' column maxima widened to the largest value of the same level (R^L - 1, so later
@@ -262,10 +246,15 @@ class Path:
                              want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
         self.ev_join.record(self.aux)
         main.wait_event(self.ev_join)
-        plan = imq.imq_plan(self.Xint, self.Wint, g.b, self.strategy, transB=True, maxes=self.mx)
+        # plan and unpack in one host call (the unpack queued right behind the plan's last kernel)
+        plan, Au, Bu = imq.imq_plan_unpack(self.Xint, self.Wint, g.b, self.strategy, transB=True, maxes=self.mx,
+                                           workspace=self.ws)
         I = plan.info
-        Au, Bu = self._workspace(I)
-        imq.imq_unpack(plan, self.Xint, self.Wint, A_unp=Au, B_unp_t=Bu)
+        if Au is None:
+            # first step, or a plan larger than the workspace: size it, then unpack
+            self.ws = imq.workspace_for(plan, self.X.device)
+            Au, Bu = imq.workspace_views(plan, self.ws)
+            imq.imq_unpack(plan, self.Xint, self.Wint, A_unp=Au, B_unp_t=Bu)
         if gemm_events is not None:
             gemm_events[0].record()
         imq.imq_gemm_unpacked(plan, Au, Bu, self.dX, imq.IMQ_PER_ROW, self.dW, imq.IMQ_PER_COL, C=C, Cf=Cf)

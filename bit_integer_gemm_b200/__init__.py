@@ -83,6 +83,8 @@ SIGNATURES = {
                                       _VP, _VP],
     "imq_plan": [_VP, _VP, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32, _VP, _VP, _VP, _VP,
                  ctypes.POINTER(_VP), _VP],
+    "imq_plan_unpack": [_VP, _VP, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32, _VP, _VP, _VP,
+                        _VP, _VP, _SZ, ctypes.POINTER(_VP), _VP],
     "imq_plan_info_get": [_VP, ctypes.POINTER(imq_plan_info)],
     "imq_plan_levels": [_VP, _VP, _VP, _VP, _VP],
     "imq_plan_groups": [_VP, ctypes.POINTER(imq_group), _I32, ctypes.POINTER(_I32)],
@@ -212,9 +214,15 @@ class Plan:
     def __init__(self, handle, A, B):
         self.handle = handle
         self._keep = (A, B)  # the plan refers to A and B
-        inf = imq_plan_info()
-        _check(lib().imq_plan_info_get(handle, ctypes.byref(inf)), "imq_plan_info_get")
-        self.info = inf.as_dict()
+        self.raw = imq_plan_info()  # the C struct; `info` is built from it on first use
+        _check(lib().imq_plan_info_get(handle, ctypes.byref(self.raw)), "imq_plan_info_get")
+        self._info = None
+
+    @property
+    def info(self) -> dict:
+        if self._info is None:
+            self._info = self.raw.as_dict()
+        return self._info
 
     def levels(self):
         I = self.info
@@ -257,6 +265,55 @@ def imq_plan(A: torch.Tensor, B: torch.Tensor, b: int, strategy: int = IMQ_MIX, 
                         _ld(B), int(b), int(strategy), *[_ptr(m) for m in mx], ctypes.byref(h), _stream(stream))
     _check(st, "imq_plan")
     return Plan(h, A, B)
+
+
+_VIEWS = {}  # (workspace address, bytes, M_unp, N_unp, K_unp) -> (workspace, A' view, B'^T view)
+
+
+def workspace_views(plan: Plan, workspace: torch.Tensor):
+    """A' and B'^T views of a workspace in the layout of imq_plan_unpack and imq_unpacked_gemm (kept per
+    workspace and plan shape, so that a loop over equal-shaped plans builds them once)."""
+    r = plan.raw
+    key = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), r.M_unp, r.N_unp, r.K_unp)
+    hit = _VIEWS.get(key)
+    if hit is not None and hit[0] is workspace:
+        return hit[1], hit[2]
+    off = (-workspace.data_ptr()) % 1024
+    w8 = workspace.view(torch.int8) if workspace.dtype != torch.int8 else workspace
+    na = r.M_unp * r.K_unp
+    b_off = off + (na + 1023) // 1024 * 1024
+    views = (w8[off:off + na].view(r.M_unp, r.K_unp), w8[b_off:b_off + r.N_unp * r.K_unp].view(r.N_unp, r.K_unp))
+    if len(_VIEWS) >= 4:  # the views keep their workspace alive: hold only a few
+        _VIEWS.clear()
+    _VIEWS[key] = (workspace,) + views
+    return views
+
+
+def imq_plan_unpack(A: torch.Tensor, B: torch.Tensor, b: int, strategy: int = IMQ_MIX, transA: bool = False,
+                    transB: bool = False, maxes=None, workspace=None, stream=None):
+    """imq_plan followed, in the same host call, by imq_unpack into `workspace` (a 1-D uint8/int8 device
+    tensor).  Returns (plan, A_unp, B_unp_t) with the operands as views of the workspace, or (plan, None,
+    None) when the workspace is smaller than the plan needs (nothing unpacked; workspace_for(plan) gives
+    one that fits)."""
+    M = A.shape[1] if transA else A.shape[0]
+    K = A.shape[0] if transA else A.shape[1]
+    N = B.shape[0] if transB else B.shape[1]
+    if A.dtype != B.dtype:
+        raise ValueError("A and B must have the same integer dtype")
+    mx = [None] * 4 if maxes is None else list(maxes)
+    wp, wn = (None, 0) if workspace is None else _aligned(workspace)
+    h = ctypes.c_void_p()
+    st = lib().imq_plan_unpack(_ptr(A), _ptr(B), _TORCH_TO_IMQ[A.dtype], M, K, N, int(transA), _ld(A), int(transB),
+                               _ld(B), int(b), int(strategy), *[_ptr(m) for m in mx], wp, wn, ctypes.byref(h),
+                               _stream(stream))
+    if st == IMQ_ERR_BUFFER and h.value:
+        return Plan(h, A, B), None, None
+    _check(st, "imq_plan_unpack")
+    plan = Plan(h, A, B)
+    if workspace is None:
+        return plan, None, None
+    Au, Bu = workspace_views(plan, workspace)
+    return plan, Au, Bu
 
 
 # ------------------------------------------------------------------------------------------------
@@ -309,12 +366,14 @@ def _outputs(I, dev, C, c_dtype, Cf, want_int, want_f32):
 def imq_gemm_unpacked(plan: Plan, A_unp, B_unp_t, deltaA=None, gA=IMQ_PER_TENSOR, deltaB=None,
                       gB=IMQ_PER_TENSOR, C=None, c_dtype=None, Cf=None, want_int=True, want_f32=True,
                       stream=None):
-    I = plan.info
-    C, Cf = _outputs(I, A_unp.device, C, c_dtype, Cf, want_int, want_f32 and deltaA is not None)
+    want_f32 = want_f32 and deltaA is not None
+    if (C is None and want_int) or (Cf is None and want_f32):
+        C, Cf = _outputs(plan.info, A_unp.device, C, c_dtype, Cf, want_int, want_f32)
+    n = plan.raw.N
     st = lib().imq_gemm_unpacked(plan.handle, _ptr(A_unp), _ptr(B_unp_t), _ptr(deltaA), gA, _ptr(deltaB), gB,
                                  _ptr(C), _TORCH_TO_IMQ[C.dtype] if C is not None else IMQ_I32,
-                                 _ld(C) if C is not None else I["N"], _ptr(Cf),
-                                 _ld(Cf) if Cf is not None else I["N"], _stream(stream))
+                                 _ld(C) if C is not None else n, _ptr(Cf),
+                                 _ld(Cf) if Cf is not None else n, _stream(stream))
     _check(st, "imq_gemm_unpacked")
     return C, Cf
 

@@ -268,6 +268,22 @@ imq_status imq_unpacked_gemm(const imq_plan_t* plan, const void* A, const void* 
   return imq_gemm_unpacked(plan, Au, Bu, deltaA, gA, deltaB, gB, Cint, ct, ldc, Cf, ldcf, stream);
 }
 
+imq_status imq_plan_unpack(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                           int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
+                           imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                           const int32_t* b_rowmax, const int32_t* b_colmax, void* workspace,
+                           size_t workspace_bytes, imq_plan_t** plan, imq_stream_t stream) {
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 1023)) return IMQ_ERR_ARG;
+  imq_status s = imq_plan(A, B, it, M, K, N, transA, lda, transB, ldb, b, strategy, a_rowmax, a_colmax, b_rowmax,
+                          b_colmax, plan, stream);
+  if (s != IMQ_OK) return s;
+  const imq_plan_info& I = (*plan)->info;
+  if (I.workspace_bytes > 0 && (!workspace || workspace_bytes < I.workspace_bytes)) return IMQ_ERR_BUFFER;
+  int8_t* Au = static_cast<int8_t*>(workspace);
+  const size_t a_bytes = ((size_t)(I.M_unp * I.K_unp) + 1023) / 1024 * 1024;
+  return imq_unpack(*plan, A, B, Au, Au ? Au + a_bytes : nullptr, stream);
+}
+
 imq_status imq_check_bounded_wait(uint64_t timeout_ns, imq_stream_t stream) {
   if (timeout_ns < 1000ull || timeout_ns > 1000000000ull) return IMQ_ERR_ARG;
   DeviceState* ds;

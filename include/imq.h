@@ -349,6 +349,24 @@ imq_status imq_unpacked_gemm(const imq_plan_t *plan, const void *A, const void *
                              void *Cint, imq_dtype ct, int64_t ldc, float *Cf, int64_t ldcf,
                              void *workspace, size_t workspace_bytes, imq_stream_t stream);
 
+/*
+ * imq_plan_unpack -- imq_plan followed, in the same host call, by imq_unpack into the caller's workspace
+ * (the plan and unpack steps of "Approach" without a return to the caller in between: the unpack is
+ * queued right behind the plan's last kernel).  Arguments as imq_plan, plus:
+ * workspace  device, 1024-byte aligned, workspace_bytes long; A' = workspace[0 .. M_unp*K_unp) and
+ *            B'^T from the next 1024-byte boundary (the layout imq_unpacked_gemm uses), so the caller
+ *            passes those two pointers to imq_gemm_unpacked.
+ * Errors: those of imq_plan and imq_unpack.  IMQ_ERR_BUFFER when workspace_bytes is below the plan's
+ *         workspace_bytes (or workspace is NULL): *plan is then a valid plan (destroy it as usual) and
+ *         nothing was unpacked; the caller may allocate imq_plan_info.workspace_bytes and call
+ *         imq_unpack.  IMQ_ERR_ARG for a misaligned workspace.  Synchronises like imq_plan.
+ */
+imq_status imq_plan_unpack(const void *A, const void *B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                           int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
+                           imq_strategy strategy, const int32_t *a_rowmax, const int32_t *a_colmax,
+                           const int32_t *b_rowmax, const int32_t *b_colmax, void *workspace,
+                           size_t workspace_bytes, imq_plan_t **plan, imq_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------------ */
 /* Status                                                                                            */
 /* ------------------------------------------------------------------------------------------------ */

@@ -418,3 +418,43 @@ def test_repeatable(imq):
     C1, _ = imq.imq_unpacked_gemm(plan, Ad, Bd, want_f32=False)
     C2, _ = imq.imq_unpacked_gemm(plan, Ad, Bd, want_f32=False)
     assert torch.equal(C1, C2)
+
+
+@pytest.mark.parametrize("strategy", [0, 1, 4, 6])
+@pytest.mark.parametrize("transB", [False, True])
+def test_plan_unpack_matches_plan_then_unpack(imq, strategy, transB):
+    """imq_plan_unpack: the same plan and the same unpacked bytes as imq_plan followed by imq_unpack, and
+    the exact product through imq_gemm_unpacked on its workspace views."""
+    rng = np.random.default_rng(31 + strategy)
+    A, B = workloads.rows_and_cols_case(rng, 200, 300, 150, big=3000, dense_rows=2, dense_cols=2)
+    Ad = torch.from_numpy(A.astype(np.int16)).cuda()
+    Bd = torch.from_numpy(np.ascontiguousarray(B.T if transB else B).astype(np.int16)).cuda()
+    ref = imq.imq_plan(Ad, Bd, 5, strategy, transB=transB)
+    rAu, rBu = imq.imq_unpack(ref, Ad, Bd)
+    ws = imq.workspace_for(ref)
+    plan, Au, Bu = imq.imq_plan_unpack(Ad, Bd, 5, strategy, transB=transB, workspace=ws)
+    assert plan.info == ref.info
+    assert torch.equal(Au, rAu) and torch.equal(Bu, rBu)
+    C, _ = imq.imq_gemm_unpacked(plan, Au, Bu, want_f32=False, c_dtype=torch.int64)
+    torch.cuda.synchronize()
+    assert imq.imq_device_status() == imq.IMQ_OK
+    assert np.array_equal(C.cpu().numpy(), oracle.gemm_i64(A, B))
+
+
+def test_plan_unpack_small_workspace(imq):
+    """A workspace below the plan's size: a valid plan, nothing written, IMQ_ERR_BUFFER turned into
+    (plan, None, None); without a workspace the same."""
+    rng = np.random.default_rng(41)
+    A, B = workloads.random_case(rng, 64, 96, 80, big=3000, frac=0.05)
+    Ad = torch.from_numpy(A.astype(np.int16)).cuda()
+    Bd = torch.from_numpy(B.astype(np.int16)).cuda()
+    small = torch.full((4096,), 7, dtype=torch.uint8, device="cuda")
+    plan, Au, Bu = imq.imq_plan_unpack(Ad, Bd, 4, 0, workspace=small)
+    assert Au is None and Bu is None and plan.info["workspace_bytes"] > 4096 - 1024
+    torch.cuda.synchronize()
+    assert bool((small == 7).all())
+    plan2, Au2, _ = imq.imq_plan_unpack(Ad, Bd, 4, 0)
+    assert Au2 is None and plan2.info == plan.info
+    Au, Bu = imq.imq_unpack(plan, Ad, Bd)
+    C, _ = imq.imq_gemm_unpacked(plan, Au, Bu, want_f32=False, c_dtype=torch.int64)
+    assert np.array_equal(C.cpu().numpy(), oracle.gemm_i64(A, B))
