@@ -185,8 +185,8 @@ class Path:
         self.ws = None
         self.info = None
         self.launches = 0
-        # the two quantisers are independent: W's runs on a second stream, joined before the plan, so that
-        # the row quantiser of X fills the SMs the column quantiser leaves idle in its last wave
+        # the two quantisers are independent: X's (the shorter) runs on a second stream, joined before the
+        # plan, so that it fills the SMs that W's column quantiser leaves idle in its last wave
         self.aux = t.cuda.Stream(device=dev)
         self.ev_fork = t.cuda.Event()
         self.ev_join = t.cuda.Event()
@@ -240,10 +240,10 @@ class Path:
         main = self.torch.cuda.current_stream()
         self.ev_fork.record(main)
         self.aux.wait_event(self.ev_fork)
-        imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
-                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True, stream=self.aux)
         imq.imq_rtn_quantize(X, imq.IMQ_PER_ROW, g.p, g.beta, Xint=self.Xint, delta=self.dX,
-                             want_qval=False, rowmax=self.mx[0], colmax=self.mx[1])
+                             want_qval=False, rowmax=self.mx[0], colmax=self.mx[1], stream=self.aux)
+        imq.imq_rtn_quantize(W, imq.IMQ_PER_COL, g.p, g.beta, Xint=self.Wint, delta=self.dW,
+                             want_qval=False, rowmax=self.mx[2], colmax=self.mx[3], trans_out=True)
         self.ev_join.record(self.aux)
         main.wait_event(self.ev_join)
         # plan and unpack in one host call (the unpack queued right behind the plan's last kernel)

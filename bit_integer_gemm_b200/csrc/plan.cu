@@ -16,6 +16,7 @@
 //   k_plan_maps    one launch: one CTA per exponent group of the inner dimension (stream compaction of
 //                  the inner indices of each of its (lA, lB) segments, padding, 16-position blocks) and
 //                  one CTA per OUTER level class (stable compaction of the lines of that level into groups)
+#include <stddef.h>
 #include <string.h>
 
 #include <atomic>
@@ -47,6 +48,19 @@ struct HostSummary {
   Summary s;
   uint32_t seq;
 };
+
+// Copies a summary to the mapped host copy with the threads of one block: everything but the rows of
+// the joint histogram above max(1, largest A column level), which are zero and which the host never
+// reads, so that few words cross to host memory.
+__device__ void summary_to_host(const Summary* src, Summary* dst, unsigned lmax_a_col) {
+  const unsigned rows = (lmax_a_col > 1 ? lmax_a_col : 1) + 1;
+  const int head = (int)((offsetof(Summary, joint) + sizeof(unsigned int) * kLv * rows) / 4);
+  const int tail0 = (int)(offsetof(Summary, bound_lo) / 4), n = (int)(sizeof(Summary) / 4);
+  const volatile uint32_t* s = reinterpret_cast<const volatile uint32_t*>(src);
+  uint32_t* d = reinterpret_cast<uint32_t*>(dst);
+  for (int i = threadIdx.x; i < head; i += blockDim.x) d[i] = s[i];
+  for (int i = tail0 + threadIdx.x; i < n; i += blockDim.x) d[i] = s[i];
+}
 
 // ------------------------------------------------------------------------------------------------
 // line maxima of a stored integer matrix
@@ -203,9 +217,7 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   __syncthreads();
   if (!last) return;
   __threadfence();
-  const volatile uint32_t* src = reinterpret_cast<const volatile uint32_t*>(a.sum);
-  uint32_t* dst = reinterpret_cast<uint32_t*>(&a.hsum->s);
-  for (int i = tid; i < (int)(sizeof(Summary) / 4); i += blockDim.x) dst[i] = src[i];
+  summary_to_host(a.sum, &a.hsum->s, *reinterpret_cast<volatile unsigned int*>(&a.sum->lmax[1]));
   __threadfence_system();
   __syncthreads();
   // the fence above orders the summary before `seq`; nothing after it needs to wait for the write
