@@ -263,13 +263,22 @@ class Path:
         self.info = I
         # kernels of this library launched by the step (the launch list of the same step shows them):
         # 2 quantisers, each followed by the reduction of its per-CTA line maxima; the level kernel; the
-        # maps kernel; 2 unpack kernels; one zeroing kernel per OUTER operand; the GEMM
-        outer = int(bool(I["dir_a"] & imq.IMQ_DIR_OUTER)) + int(bool(I["dir_b"] & imq.IMQ_DIR_OUTER))
-        self.launches = 4 + 1 + (1 if I["K_unp"] > 0 else 0) + 2 + outer + 1
+        # maps kernel; 2 unpack kernels (int16 rows: they also zero the unused OUTER lines); the GEMM
+        self.launches = 4 + 1 + (1 if I["K_unp"] > 0 else 0) + 2 + 1
         if self.strategy == imq.IMQ_HYBRID:
             self.launches += 4  # the hybrid's count (both operands' outer lines are stored rows), histogram,
             # choice and level kernels
         plan.destroy()
+
+
+def _rows_unpack(line_is_row, K, K_unp):
+    """True when the library unpacks int16 lines with its staged-row kernel (the condition of its launcher:
+    stored rows, the line and the block metadata within shared memory)."""
+    Kr = (K + 15) // 16 * 16
+    nw = min(8, (64 * 1024) // (Kr * 2))
+    if nw < 1:
+        nw = 1 if (192 * 1024) // (Kr * 2) >= 1 else 0
+    return bool(line_is_row) and nw >= 1 and K_unp // 16 <= 4096 and nw * Kr * 2 + (K_unp // 16) * 5 <= 200 * 1024
 
 
 class GemmPath:
@@ -325,10 +334,13 @@ class GemmPath:
         self.info = I
         # kernels of this library launched by the step: per quantiser its kernel and the reduction of its
         # per-CTA line maxima, plus for a per-tensor bf16 group the init and two histogram + select passes;
-        # the level and maps kernels (and those of the hybrid choice); 2 unpack kernels; one zeroing
-        # kernel per OUTER operand; the GEMM
+        # the level and maps kernels (and those of the hybrid choice); 2 unpack kernels; the zeroing
+        # launches counted above; the GEMM
         quant = lambda gran: 7 if gran == imq.IMQ_PER_TENSOR else 2
-        outer = int(bool(I["dir_a"] & imq.IMQ_DIR_OUTER)) + int(bool(I["dir_b"] & imq.IMQ_DIR_OUTER))
+        # a zeroing launch per OUTER operand unless its int16 lines are stored rows, which the row unpack
+        # kernel stages and zeroes itself
+        outer = (int(bool(I["dir_a"] & imq.IMQ_DIR_OUTER) and not _rows_unpack(not g.transA, I["K"], I["K_unp"])) +
+                 int(bool(I["dir_b"] & imq.IMQ_DIR_OUTER) and not _rows_unpack(g.transB, I["K"], I["K_unp"])))
         hybrid = 0
         if self.strategy == imq.IMQ_HYBRID:
             # histogram, choice and levels, plus one count kernel for operands whose outer lines are
