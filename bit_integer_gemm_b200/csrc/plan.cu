@@ -36,7 +36,7 @@ struct Summary {
   unsigned int lmax[4];
   unsigned int hist[4][kLv];
   unsigned int joint[kLv][kLv];
-  unsigned long long bound_lo, bound_hi;
+  unsigned long long bound_lo, bound_hi;  // sums of the bound's products' low / high 32-bit halves
   int32_t status;  // copy of the device status word taken in stream order
   uint32_t done;   // blocks of k_levels that have added their part
 };
@@ -137,32 +137,48 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   unsigned long long bsum[4] = {0, 0, 0, 0}, boor[4] = {0, 0, 0, 0};
   unsigned int blmax[4] = {0, 0, 0, 0};
-  unsigned __int128 bound = 0;
-  for (int v = 0; v < 4; ++v) {
-    // whole warps iterate together so the aggregated counters see every lane
-    for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x; i0 < a.n[v]; i0 += stride) {
-      const int64_t i = i0 + tid;
-      const bool in = i < a.n[v];
+  // the bound sum_t max|A[:,t]| * max|B[t,:]| as two 64-bit sums, of the products' low 32-bit halves and
+  // of their high halves (products < 2^62 and at most 2^31 lines: neither sum can overflow, so blocks add
+  // them without carries and the host joins them as hi * 2^32 + lo)
+  unsigned long long blo = 0, bhi = 0;
+  const int64_t nmax = max(max(a.n[0], a.n[1]), max(a.n[2], a.n[3]));
+  // whole warps iterate together so the aggregated counters see every lane; the entries of all four
+  // vectors are loaded before any is used, so that their loads are in flight together
+  for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x; i0 < nmax; i0 += stride) {
+    const int64_t i = i0 + tid;
+    bool in[4];
+    uint32_t m[4];
+    int lvi[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      in[v] = i < a.n[v];
+      m[v] = in[v] ? (uint32_t)a.mx[v][i] : 0u;
+      lvi[v] = (in[v] && a.lvin[v]) ? (int)a.lvin[v][i] : -1;
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
       int L = 1;
-      if (in) {
-        const uint32_t m = (uint32_t)a.mx[v][i];
-        if (v == 1 && a.keep_a_col) a.keep_a_col[i] = (int32_t)m;
-        L = a.lvin[v] ? (int)a.lvin[v][i] : level_of(m, a.bm1);
+      if (in[v]) {
+        if (v == 1 && a.keep_a_col) a.keep_a_col[i] = (int32_t)m[v];
+        L = lvi[v] >= 0 ? lvi[v] : level_of(m[v], a.bm1);
         a.lv[v][i] = (int8_t)L;
         bsum[v] += (unsigned)L;
         boor[v] += (L > 1);
         blmax[v] = max(blmax[v], (unsigned)L);
-        if (v == 1) bound += (unsigned __int128)((unsigned long long)m * (unsigned long long)(uint32_t)a.mx[2][i]);
+        if (v == 1) {
+          const unsigned long long prod = (unsigned long long)m[1] * (unsigned long long)m[2];
+          blo += prod & 0xFFFFFFFFull;
+          bhi += prod >> 32;
+        }
       }
-      warp_count(&hist[v][0], (uint32_t)L, in);
+      warp_count(&hist[v][0], (uint32_t)L, in[v]);
       if (v == 1) {
-        const int Lb = !in ? 1 : (a.lvin[2] ? (int)a.lvin[2][i] : level_of((uint32_t)a.mx[2][i], a.bm1));
-        warp_count(&joint[0][0], (uint32_t)(L * kLv + Lb), in);
+        const int Lb = !in[1] ? 1 : (lvi[2] >= 0 ? lvi[2] : level_of(m[2], a.bm1));
+        warp_count(&joint[0][0], (uint32_t)(L * kLv + Lb), in[1]);
       }
     }
   }
   // warp reductions first, then one shared atomic per warp, then one global atomic per block
-  unsigned long long blo = (unsigned long long)bound, bhi = (unsigned long long)(bound >> 64);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     for (int v = 0; v < 4; ++v) {
@@ -170,11 +186,8 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
       boor[v] += __shfl_xor_sync(0xffffffffu, boor[v], o);
       blmax[v] = max(blmax[v], __shfl_xor_sync(0xffffffffu, blmax[v], o));
     }
-    const unsigned long long ol = __shfl_xor_sync(0xffffffffu, blo, o);
-    const unsigned long long oh = __shfl_xor_sync(0xffffffffu, bhi, o);
-    const unsigned long long nl = blo + ol;
-    bhi += oh + (nl < blo ? 1ull : 0ull);
-    blo = nl;
+    blo += __shfl_xor_sync(0xffffffffu, blo, o);
+    bhi += __shfl_xor_sync(0xffffffffu, bhi, o);
   }
   __shared__ unsigned long long sblo, sbhi;
   if (tid == 0) {
@@ -188,16 +201,13 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
       if (boor[v]) atomicAdd(&soor[v], boor[v]);
       if (blmax[v]) atomicMax(&slmax[v], blmax[v]);
     }
-    if (blo || bhi) {
-      const unsigned long long old = atomicAdd(&sblo, blo);
-      atomicAdd(&sbhi, bhi + ((old + blo < old) ? 1ull : 0ull));
-    }
+    if (blo) atomicAdd(&sblo, blo);
+    if (bhi) atomicAdd(&sbhi, bhi);
   }
   __syncthreads();
-  if (tid == 0 && (sblo || sbhi)) {
-    const unsigned long long old = atomicAdd(&a.sum->bound_lo, sblo);
-    const unsigned long long hi = sbhi + ((old + sblo < old) ? 1ull : 0ull);
-    if (hi) atomicAdd(&a.sum->bound_hi, hi);
+  if (tid == 0) {
+    if (sblo) atomicAdd(&a.sum->bound_lo, sblo);
+    if (sbhi) atomicAdd(&a.sum->bound_hi, sbhi);
   }
   __syncthreads();
   if (tid < 4) {
@@ -1259,7 +1269,8 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
                 : 1.0;
 
   // bound and accumulator schedule
-  const unsigned __int128 bound = ((unsigned __int128)S.bound_hi << 64) | S.bound_lo;
+  // k_levels sums the products' low and high 32-bit halves separately
+  const unsigned __int128 bound = ((unsigned __int128)S.bound_hi << 32) + S.bound_lo;
   I.bound = (double)bound;
   const unsigned __int128 two31 = (unsigned __int128)1 << 31;
   if (bound >= ((unsigned __int128)1 << 63)) return fail(IMQ_ERR_UNSUPPORTED);  // C itself may leave int64
