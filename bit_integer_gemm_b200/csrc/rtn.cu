@@ -4,16 +4,21 @@
 // summary), "Problem" / "Approach" and the measured-effects rows on beta and p.  The scale of a group
 // maps its nearest-rank p-quantile q of |x| to beta; entries are rounded to the nearest integer
 // (ties to even) after one fp32 multiply and are NOT clipped, so heavy hitters stay far outside
-// +-beta.  q is found exactly by a radix select on the order-preserving bit keys of |x| (the IEEE bit
-// pattern of a non-negative float orders like an unsigned integer), 8 key bits per pass from the top.
+// +-beta.  q is found exactly on the order-preserving bit keys of |x| (the IEEE bit pattern of a
+// non-negative float orders like an unsigned integer): bf16 groups of 1024 entries or more by a sample
+// select (a sample brackets the rank, one pass counts below the bracket and histograms inside it),
+// smaller bf16 groups by bisection on the key, fp32 groups by radix passes of 8 key bits.
 //
 // Kernels
 //   k_rtn_rows    one warp per stored row: the row is staged in the warp's shared-memory buffer once,
-//                 the select passes and the quantisation read it from there (one HBM read, one write).
-//                 Also used for per-tensor groups with the scale taken from the tensor select.
-//   k_rtn_cols_staged  one CTA per 16 (or 8) stored columns: the column slab is staged in shared
-//                 memory (one HBM read), per-column histograms in shared memory, optional transposed
-//                 output (a K x N weight quantised per output channel straight into N x K).
+//                 the select and the quantisation read it from there (one HBM read, one write); rows
+//                 are dealt to the CTAs in turn.  bf16 to int16: quantised in place, the CTA folds the
+//                 column maxima of each round of rows without atomics.  Also used for per-tensor
+//                 groups with the scale taken from the tensor select.
+//   k_rtn_cols_staged  one CTA per 16 (or 8, 4) stored columns: the column slab is staged in shared
+//                 memory (one HBM read), one warp per column, optional transposed output (a K x N
+//                 weight quantised per output channel straight into N x K); bf16 to int16 quantised in
+//                 place with the row maxima folded over the CTA's columns.
 //   k_rtn_cols    the same for columns too tall to stage: the slab is streamed once per pass (re-reads
 //                 hit L2) and once more to quantise.
 //   k_tensor_*    per-tensor select: global 256-bin histograms per pass, then k_rtn_rows.
