@@ -587,16 +587,17 @@ def run_ours(args):
 # ------------------------------------------------------------------------------------------------
 # the oracle on the host (cpu_baseline and the reference arm)
 # ------------------------------------------------------------------------------------------------
-def _oracle_sample(g, rows: int, qW=None):
+def _oracle_sample(g, rows: int, qW=None, nthreads: int = 0):
     """Definition tier of the oracle on `rows` rows of X: RTN of those rows (per token), RTN of W (per
-    channel; once, passed in when already done), the direct int64 product and the dequantisation."""
+    channel; once, passed in when already done), the direct int64 product (on `nthreads` host threads,
+    0 = all) and the dequantisation."""
     import oracle
     t0 = time.perf_counter()
     if qW is None:
         qW = oracle.rtn_quantize(oracle.as_f32(g.B.data, "bf16"), oracle.PER_COL, g.p, g.beta)
     xs = oracle.as_f32(g.A.data[:rows], "bf16")
     xi, dx, _ = oracle.rtn_quantize(xs, oracle.PER_ROW, g.p, g.beta)
-    C = oracle.gemm_i64(xi, qW[0])
+    C = oracle.gemm_i64(xi, qW[0], nthreads)
     oracle.dequant(C, dx, oracle.PER_ROW, qW[1], oracle.PER_COL)
     return time.perf_counter() - t0, qW
 
@@ -620,9 +621,15 @@ def cpu_baseline(g, target_s=15.0):
     t_rows, _ = _oracle_sample(g, rows, qW)
     t = t_w + t_rows
     ops = 2.0 * rows * g.N * g.K
+    # the same per-row work on one host thread, on the probe's rows (W's RTN already done)
+    t_one, _ = _oracle_sample(g, probe_rows, qW, nthreads=1)
+    one = 2.0 * probe_rows * g.N * g.K / t_one / 1e12
     return {"value": round(ops / t / 1e12, 6), "unit": UNIT, "cores": _cores(), "kind": "oracle",
             "sample": f"{rows} of {g.M} rows of X: RTN of those rows + RTN of all of W + int64 product + "
-                      f"dequant; {t:.1f} s on the host", "seconds": round(t, 2)}
+                      f"dequant; {t:.1f} s on the host", "seconds": round(t, 2),
+            "single_thread": {"value": round(one, 6), "unit": UNIT,
+                              "sample": f"{probe_rows} rows of X (RTN + int64 product + dequant, W quantised "
+                                        f"before), one host thread, {t_one:.2f} s"}}
 
 
 def run_reference(args):
