@@ -27,9 +27,9 @@ imq_status device_state(DeviceState** out) {
   IMQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return IMQ_ERR_UNSUPPORTED;
   DeviceState& d = g_dev[dev];
-  if (!d.init) {
+  if (!d.init.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_dev_mu);
-    if (!d.init) {
+    if (!d.init.load(std::memory_order_relaxed)) {
       void* p = nullptr;
       IMQ_CUDA_TRY(cudaGetSymbolAddress(&p, g_status));
       IMQ_CUDA_TRY(cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev));
@@ -42,7 +42,7 @@ imq_status device_state(DeviceState** out) {
       uint64_t keep = UINT64_MAX;
       IMQ_CUDA_TRY(cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep));
       d.status = static_cast<int32_t*>(p);
-      d.init = true;
+      d.init.store(true, std::memory_order_release);
     }
   }
   *out = &d;

@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -18,7 +20,8 @@ struct DeviceState {
   // stream-ordered pool for plan memory and the quantiser's per-call scratch; it keeps what is freed
   // (no trim at synchronisation), so later calls reuse memory instead of mapping fresh pages
   cudaMemPool_t pool = nullptr;
-  bool init = false;
+  // set (release) after every field above; read with acquire before any of them is used
+  std::atomic<bool> init{false};
 };
 imq_status device_state(DeviceState** out);
 // Raises the dynamic shared-memory limit of kernel `fn` on the current device to at least `bytes`.  The

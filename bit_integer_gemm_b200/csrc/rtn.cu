@@ -1045,6 +1045,32 @@ struct StreamScratch {
   }
 };
 
+// Launch shape of the per-row kernel k_rtn_rows: one warp per row, the row buffers of the CTA's warps
+// plus (when column maxima are wanted) its column maxima in shared memory, as many CTAs as fit on an SM
+// (at most 4), and one CTA per row up to every resident slot (rows are dealt to the CTAs in turn).
+// Returns false when one row and the column maxima do not fit the shared-memory budget.
+struct RowsShape {
+  int64_t grid;
+  int nwarps;
+  size_t smem;
+};
+bool rows_launch_shape(int64_t rows, int64_t cols, size_t elem, bool want_colmax, int sms, RowsShape* out) {
+  const size_t row_bytes = (size_t)((cols * (int64_t)elem + 15) / 16 * 16);
+  const size_t cmax_bytes = want_colmax ? (size_t)((cols * 4 + 15) / 16 * 16) : 0;
+  constexpr size_t kBudget = 200 * 1024;
+  if (cmax_bytes + row_bytes > kBudget) return false;
+  int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
+  if (nwarps > kThreads / 32) nwarps = kThreads / 32;
+  const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
+  int per_sm = (int)(kBudget / (smem + kThreads / 32 * kSelWords * 4 + 1024));
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 4) per_sm = 4;
+  out->grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
+  out->nwarps = nwarps;
+  out->smem = smem;
+  return true;
+}
+
 int64_t nearest_rank(int64_t n, double p) {
   if (n <= 0) return 1;
   int64_t k = (int64_t)ceil(p * (double)n);
@@ -1106,19 +1132,11 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
     if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
     return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
   }
-  // one warp per row; the row buffers of the CTA's warps plus its column maxima in shared memory
-  const size_t row_bytes = (size_t)((cols * (int64_t)sizeof(T) + 15) / 16 * 16);
-  const size_t cmax_bytes = colmax ? (size_t)((cols * 4 + 15) / 16 * 16) : 0;
-  constexpr size_t kBudget = 200 * 1024;
-  if (cmax_bytes + row_bytes > kBudget) return IMQ_ERR_UNSUPPORTED;
-  int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
-  if (nwarps > kThreads / 32) nwarps = kThreads / 32;
-  const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
-  int per_sm = (int)(kBudget / (smem + kThreads / 32 * kSelWords * 4 + 1024));
-  if (per_sm < 1) per_sm = 1;
-  if (per_sm > 4) per_sm = 4;
-  // one CTA per row up to every resident slot: rows are dealt to the CTAs in turn
-  const int64_t grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
+  RowsShape sh;
+  if (!rows_launch_shape(rows, cols, sizeof(T), colmax != nullptr, sms, &sh)) return IMQ_ERR_UNSUPPORTED;
+  const int64_t grid = sh.grid;
+  const int nwarps = sh.nwarps;
+  const size_t smem = sh.smem;
   const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
                    ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   int32_t* part = nullptr;
@@ -1212,13 +1230,18 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocBytes / sizeo
 std::atomic<int32_t*> g_noalloc_ptr[64];
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device (looked up on the first call there).
-imq_status noalloc_scratch(int32_t** out) {
+// Device address of the scratch array on the current device (looked up on the first call there).  The
+// look-up may load the module, which a stream capture in progress would not record: a first call on a
+// device made while `st` is capturing is refused with IMQ_ERR_UNSUPPORTED before anything else happens.
+imq_status noalloc_scratch(int32_t** out, cudaStream_t st) {
   int dev = 0;
   IMQ_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return IMQ_ERR_UNSUPPORTED;
   int32_t* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
   if (!ptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    IMQ_CUDA_TRY(cudaStreamIsCapturing(st, &cs));
+    if (cs != cudaStreamCaptureStatusNone) return IMQ_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     ptr = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
     if (!ptr) {
@@ -1238,26 +1261,19 @@ template <typename T, bool kOut16>
 imq_status run_rows_noalloc(const T* X, int64_t rows, int64_t cols, int64_t ld, double p, int32_t beta,
                             void* Xint, int64_t ldq, float* delta, float* qval, int32_t* rowmax, int32_t* colmax,
                             DeviceState* ds, cudaStream_t st) {
-  const int sms = ds->num_sms;
-  const size_t row_bytes = (size_t)((cols * (int64_t)sizeof(T) + 15) / 16 * 16);
-  const size_t cmax_bytes = colmax ? (size_t)((cols * 4 + 15) / 16 * 16) : 0;
-  constexpr size_t kBudget = 200 * 1024;
-  if (cmax_bytes + row_bytes > kBudget) return IMQ_ERR_UNSUPPORTED;
-  int nwarps = (int)((kBudget - cmax_bytes) / row_bytes);
-  if (nwarps > kThreads / 32) nwarps = kThreads / 32;
-  const size_t smem = cmax_bytes + (size_t)nwarps * row_bytes;
-  int per_sm = (int)(kBudget / (smem + kThreads / 32 * kSelWords * 4 + 1024));
-  if (per_sm < 1) per_sm = 1;
-  if (per_sm > 4) per_sm = 4;
-  // one CTA per row up to every resident slot: rows are dealt to the CTAs in turn
-  const int64_t grid = rows < (int64_t)sms * per_sm ? rows : (int64_t)sms * per_sm;
+  // the launch shape of the allocating per-row path, from the same helper
+  RowsShape sh;
+  if (!rows_launch_shape(rows, cols, sizeof(T), colmax != nullptr, ds->num_sms, &sh)) return IMQ_ERR_UNSUPPORTED;
+  const int64_t grid = sh.grid;
+  const int nwarps = sh.nwarps;
+  const size_t smem = sh.smem;
   const bool vec = (cols % (16 / (int64_t)sizeof(T)) == 0) && (ld % (16 / (int64_t)sizeof(T)) == 0) &&
                    ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
   int32_t* part = nullptr;
   if (colmax) {
     // checked before anything is launched: the kernel writes grid x cols partials
     if ((uint64_t)grid * (uint64_t)cols * sizeof(int32_t) > kNoallocBytes) return IMQ_ERR_UNSUPPORTED;
-    imq_status e = noalloc_scratch(&part);
+    imq_status e = noalloc_scratch(&part, st);
     if (e != IMQ_OK) return e;
   }
   auto kern = k_rtn_rows<T, true, kOut16>;

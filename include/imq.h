@@ -166,7 +166,7 @@ imq_status imq_rtn_quantize_ex(const void *X, imq_dtype xt, int64_t rows, int64_
  * when the scratch needed exceeds IMQ_NOALLOC_SCRATCH_BYTES.
  * Set-up: the first call on a device looks up the device address of the scratch array for that
  * device (cudaGetSymbolAddress, with that device current); make this first call before any stream
- * capture.
+ * capture.  A first call on a device whose stream is capturing returns IMQ_ERR_UNSUPPORTED at once.
  * Concurrency: every call on a device uses the same scratch array, so calls whose executions overlap
  * (on different streams, or from different host threads without ordering) race on it and may return
  * wrong column maxima.  Order them on one stream or with events.

@@ -38,18 +38,34 @@ def _same(a, b):
             assert torch.equal(x, y), name
 
 
-def _scratch_needed(rows, cols, itemsize, sms):
-    """Bytes of partial column maxima the per-row kernel writes (its launch shape, restated)."""
-    row_bytes = (cols * itemsize + 15) // 16 * 16
-    cmax = (cols * 4 + 15) // 16 * 16
-    budget = 200 * 1024
-    if cmax + row_bytes > budget:
-        return None
-    nwarps = min((budget - cmax) // row_bytes, 8)
-    smem = cmax + nwarps * row_bytes
-    per_sm = min(max(budget // (smem + 8 * 384 * 4 + 1024), 1), 4)
-    grid = min(rows, sms * per_sm)
-    return grid * cols * 4
+def _rejected(imq, rows, cols, dtype="bf16"):
+    """True when the allocation-free call refuses this shape (IMQ_ERR_UNSUPPORTED: its scratch would
+    exceed the fixed array).  A refused call launches nothing, so the output keeps its fill."""
+    x = torch.zeros((rows, cols), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device="cuda")
+    xint = torch.full((rows, cols), 12345, dtype=torch.int16, device="cuda")
+    try:
+        imq.imq_rtn_quantize_rows_noalloc(x, 0.95, 15, Xint=xint)
+    except imq.ImqError as e:
+        assert e.status == imq.IMQ_ERR_UNSUPPORTED, e
+        torch.cuda.synchronize()
+        assert bool((xint == 12345).all()), "a refused call wrote its output"
+        return True
+    torch.cuda.synchronize()
+    return False
+
+
+def _widest_accepted(imq, rows, hi):
+    """The widest bf16 row length (a multiple of 8, below hi) the call accepts for `rows` rows, found by
+    bisection through the entry point itself (no launch constants restated here)."""
+    lo = 8
+    assert not _rejected(imq, rows, lo)
+    while hi - lo > 8:
+        mid = (lo + hi) // 16 * 8
+        if _rejected(imq, rows, mid):
+            hi = mid
+        else:
+            lo = mid
+    return lo
 
 
 PAIRS = [
@@ -90,11 +106,9 @@ def test_empty(imq, rows, cols):
 
 
 def test_scratch_above_the_maximum_is_rejected_before_any_launch(imq):
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
     rows, cols = 1024, 16384
-    need = _scratch_needed(rows, cols, 2, sms)
-    if need is None or need <= imq.IMQ_NOALLOC_SCRATCH_BYTES:
-        pytest.skip(f"this device needs only {need} bytes for the rejected shape")
+    if not _rejected(imq, rows, cols):
+        pytest.skip("this device's launch shape fits the widest test row in the fixed array")
     x = _input(7, rows, cols, "bf16")
     xint = torch.full((rows, cols), 12345, dtype=torch.int16, device="cuda")
     with pytest.raises(imq.ImqError) as e:
@@ -109,15 +123,13 @@ def test_scratch_above_the_maximum_is_rejected_before_any_launch(imq):
 
 
 def test_shape_near_the_maximum(imq):
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    rows, cols = 1000, 16384
-
-    def fits(c):
-        need = _scratch_needed(rows, c, 2, sms)
-        return need is not None and need <= imq.IMQ_NOALLOC_SCRATCH_BYTES
-
-    while not fits(cols):
-        cols -= 8
+    """The widest accepted row length for 1000 rows runs and matches the allocating entry point; 8 more
+    columns are refused."""
+    rows = 1000
+    if not _rejected(imq, rows, 16384):
+        pytest.skip("this device's launch shape fits the widest test row in the fixed array")
+    cols = _widest_accepted(imq, rows, 16384)
+    assert _rejected(imq, rows, cols + 8)
     x = _input(8, rows, cols, "bf16")
     _same(imq.imq_rtn_quantize_rows_noalloc(x, 0.95, 15, out_dtype=torch.int32),
           imq.imq_rtn_quantize(x, imq.IMQ_PER_ROW, 0.95, 15, out_dtype=torch.int32))
@@ -125,22 +137,44 @@ def test_shape_near_the_maximum(imq):
     assert imq.imq_device_status(clear=True) == imq.IMQ_OK
 
 
+# Run in a fresh process: no allocating call of the library may come first there, so the library's
+# memory pool holds nothing that a pool allocation could reuse unseen.  The first call loads the
+# kernels; then two passes over two shapes (the second needing more scratch than the first) must leave
+# the device's free memory unchanged.
+_FRESH = r"""
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import bit_integer_gemm_b200 as imq
+imq.lib()
+bufs = []
+for i, (r, c) in enumerate([(512, 1024), (2048, 8192)]):
+    rng = np.random.default_rng(10 + i)
+    x = torch.from_numpy(rng.standard_normal((r, c)).astype(np.float32)).cuda().to(torch.bfloat16)
+    bufs.append(dict(X=x, Xint=torch.empty((r, c), dtype=torch.int16, device="cuda"),
+                     delta=torch.empty(r, device="cuda"), qval=torch.empty(r, device="cuda"),
+                     rowmax=torch.empty(r, dtype=torch.int32, device="cuda"),
+                     colmax=torch.empty(c, dtype=torch.int32, device="cuda")))
+imq.imq_rtn_quantize_rows_noalloc(p=0.95, beta=15, **bufs[0])
+torch.cuda.synchronize()
+free0 = torch.cuda.mem_get_info()[0]
+for b in bufs + bufs:
+    imq.imq_rtn_quantize_rows_noalloc(p=0.95, beta=15, **b)
+torch.cuda.synchronize()
+free1 = torch.cuda.mem_get_info()[0]
+assert imq.imq_device_status(clear=True) == imq.IMQ_OK
+print("FREE", free0, free1)
+"""
+
+
 def test_no_device_memory_is_allocated(imq):
-    # outputs preallocated; a first pass loads every kernel the second pass launches
-    shapes = [(512, 1024), (2048, 8192)]
-    bufs = []
-    for i, (r, c) in enumerate(shapes):
-        x = _input(10 + i, r, c, "bf16")
-        bufs.append(dict(X=x, Xint=torch.empty((r, c), dtype=torch.int16, device="cuda"),
-                         delta=torch.empty(r, device="cuda"), qval=torch.empty(r, device="cuda"),
-                         rowmax=torch.empty(r, dtype=torch.int32, device="cuda"),
-                         colmax=torch.empty(c, dtype=torch.int32, device="cuda")))
-    imq.imq_rtn_quantize_rows_noalloc(p=0.95, beta=15, **bufs[0])
-    torch.cuda.synchronize()
-    free0 = torch.cuda.mem_get_info()[0]
-    # the second shape needs more scratch than the first: the allocating entry point would grow its buffer
-    for b in bufs + bufs:
-        imq.imq_rtn_quantize_rows_noalloc(p=0.95, beta=15, **b)
-    torch.cuda.synchronize()
-    assert torch.cuda.mem_get_info()[0] == free0
-    assert imq.imq_device_status(clear=True) == imq.IMQ_OK
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", _FRESH, root], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = [ln for ln in out.stdout.splitlines() if ln.startswith("FREE")][-1]
+    free0, free1 = (int(v) for v in line.split()[1:])
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
