@@ -88,11 +88,13 @@ SIGNATURES = {
     "imq_plan_info_get": [_VP, ctypes.POINTER(imq_plan_info)],
     "imq_plan_levels": [_VP, _VP, _VP, _VP, _VP],
     "imq_plan_groups": [_VP, ctypes.POINTER(imq_group), _I32, ctypes.POINTER(_I32)],
+    "imq_plan_maps": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP],
     "imq_plan_destroy": [_VP],
     "imq_unpack": [_VP, _VP, _VP, _VP, _VP, _VP],
     "imq_rtn_quantize_unpack": [_VP, _VP, _I32, _I64, _F64, _I32, _VP, _VP, _VP],
     "imq_gemm_unpacked": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP],
     "imq_unpacked_gemm": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP, _SZ, _VP],
+    "imq_level_cover": [_VP, _I64, _I32, _I32, _VP, _VP],
     "imq_device_status": [_VP, _I32],
     "imq_check_bounded_wait": [ctypes.c_uint64, _VP],
     "imq_status_str": [_I32],
@@ -232,6 +234,20 @@ class Plan:
                "imq_plan_levels")
         return dict(zip(("a_row", "a_col", "b_row", "b_col"), out))
 
+    def maps(self):
+        """The plan's index maps of the unpacked operands (imq_plan_maps), as numpy arrays: tK, lAk, lBk
+        (K_unp), srcA, lvlA (M_unp), srcB, lvlB (N_unp)."""
+        import numpy as np
+        I = self.info
+        out = {"tK": np.zeros(I["K_unp"], np.int32), "lAk": np.zeros(I["K_unp"], np.int8),
+               "lBk": np.zeros(I["K_unp"], np.int8), "srcA": np.zeros(I["M_unp"], np.int32),
+               "lvlA": np.zeros(I["M_unp"], np.int8), "srcB": np.zeros(I["N_unp"], np.int32),
+               "lvlB": np.zeros(I["N_unp"], np.int8)}
+        _check(lib().imq_plan_maps(self.handle, *[out[k].ctypes.data_as(ctypes.c_void_p) for k in
+                                                  ("tK", "lAk", "lBk", "srcA", "lvlA", "srcB", "lvlB")]),
+               "imq_plan_maps")
+        return out
+
     def groups(self):
         arr = (imq_group * IMQ_MAX_GROUPS)()
         n = ctypes.c_int32(0)
@@ -346,6 +362,15 @@ def imq_rtn_quantize_unpack(plan: Plan, X: torch.Tensor, p: float, beta: int, A_
     _check(lib().imq_rtn_quantize_unpack(plan.handle, _ptr(X), _TORCH_TO_IMQ[X.dtype], _ld(X), float(p), int(beta),
                                          _ptr(A_unp), _ptr(deltaA), _stream(stream)), "imq_rtn_quantize_unpack")
     return A_unp, deltaA
+
+
+def imq_level_cover(maxima: torch.Tensor, b: int, cap: int = 32767, out=None, stream=None) -> torch.Tensor:
+    """min(R^L - 1, cap) for every line maximum (L its number of base-R digits), int32 on the device."""
+    if out is None:
+        out = torch.empty_like(maxima)
+    _check(lib().imq_level_cover(_ptr(maxima), maxima.numel(), int(b), int(cap), _ptr(out), _stream(stream)),
+           "imq_level_cover")
+    return out
 
 
 def imq_check_bounded_wait(timeout_ns: int, stream=None):

@@ -204,6 +204,67 @@ imq_status imq_plan_levels(const imq_plan_t* plan, int8_t* a_row, int8_t* a_col,
   return e == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
+namespace {
+// Host copy of one OUTER map: the source line of every unpacked line (device srcX) and its level, which
+// follows from the group's level L: the L lines of one source are consecutive inside a group of G.
+imq_status outer_map_to_host(const int32_t* d_src, const int32_t* d_grpL, int64_t n_unp, int64_t n_grp, int G,
+                             int32_t* src, int8_t* lvl) {
+  int32_t* s = src;
+  int32_t* tmp = nullptr;
+  if (!s) {
+    tmp = static_cast<int32_t*>(malloc((size_t)(n_unp > 0 ? n_unp : 1) * 4));
+    if (!tmp) return IMQ_ERR_CUDA;
+    s = tmp;
+  }
+  int32_t* gl = static_cast<int32_t*>(malloc((size_t)(n_grp > 0 ? n_grp : 1) * 4));
+  cudaError_t e = gl ? cudaSuccess : cudaErrorMemoryAllocation;
+  if (e == cudaSuccess && n_unp) e = cudaMemcpy(s, d_src, (size_t)n_unp * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && n_grp) e = cudaMemcpy(gl, d_grpL, (size_t)n_grp * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && lvl)
+    for (int64_t u = 0; u < n_unp; ++u) lvl[u] = s[u] < 0 ? 0 : (int8_t)((u % G) % gl[u / G]);
+  free(gl);
+  free(tmp);
+  return e == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+}  // namespace
+
+imq_status imq_plan_maps(const imq_plan_t* plan, int32_t* tK, int8_t* lAk, int8_t* lBk, int32_t* srcA, int8_t* lvlA,
+                         int32_t* srcB, int8_t* lvlB) {
+  if (!plan) return IMQ_ERR_ARG;
+  const imq_plan_info& I = plan->info;
+  int dev = 0;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  IMQ_CUDA_TRY(cudaSetDevice(plan->device));
+  imq_status s = IMQ_OK;
+  cudaError_t e = cudaDeviceSynchronize();  // the maps kernel runs on the caller's stream
+  if (e == cudaSuccess && tK && I.K_unp) e = cudaMemcpy(tK, plan->tK, (size_t)I.K_unp * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && lAk && I.K_unp) e = cudaMemcpy(lAk, plan->lAk, (size_t)I.K_unp, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && lBk && I.K_unp) e = cudaMemcpy(lBk, plan->lBk, (size_t)I.K_unp, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) s = IMQ_ERR_CUDA;
+  if (s == IMQ_OK) {
+    if (I.dir_a & IMQ_DIR_OUTER) {
+      s = outer_map_to_host(plan->srcA, plan->grpA_L, I.M_unp, plan->n_grp_a, IMQ_A_GROUP, srcA, lvlA);
+    } else {
+      for (int64_t u = 0; u < I.M_unp; ++u) {
+        if (srcA) srcA[u] = (int32_t)u;
+        if (lvlA) lvlA[u] = 0;
+      }
+    }
+  }
+  if (s == IMQ_OK) {
+    if (I.dir_b & IMQ_DIR_OUTER) {
+      s = outer_map_to_host(plan->srcB, plan->grpB_L, I.N_unp, plan->n_grp_b, IMQ_B_GROUP, srcB, lvlB);
+    } else {
+      for (int64_t w = 0; w < I.N_unp; ++w) {
+        if (srcB) srcB[w] = (int32_t)w;
+        if (lvlB) lvlB[w] = 0;
+      }
+    }
+  }
+  cudaSetDevice(dev);
+  return s;
+}
+
 imq_status imq_plan_groups(const imq_plan_t* plan, imq_group* groups, int32_t max_groups, int32_t* n_out) {
   if (!plan || !n_out || (max_groups > 0 && !groups)) return IMQ_ERR_ARG;
   const int n = plan->info.n_groups;
@@ -282,6 +343,12 @@ imq_status imq_plan_unpack(const void* A, const void* B, imq_dtype it, int64_t M
   int8_t* Au = static_cast<int8_t*>(workspace);
   const size_t a_bytes = ((size_t)(I.M_unp * I.K_unp) + 1023) / 1024 * 1024;
   return imq_unpack(*plan, A, B, Au, Au ? Au + a_bytes : nullptr, stream);
+}
+
+imq_status imq_level_cover(const int32_t* maxima, int64_t n, int32_t b, int32_t cap, int32_t* out,
+                           imq_stream_t stream) {
+  if (n < 0 || b < 2 || b > 8 || cap < 0 || (n > 0 && (!maxima || !out))) return IMQ_ERR_ARG;
+  return imq::launch_level_cover(maxima, n, b, cap, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 imq_status imq_check_bounded_wait(uint64_t timeout_ns, imq_stream_t stream) {

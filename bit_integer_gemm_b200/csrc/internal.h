@@ -45,6 +45,9 @@ imq_status launch_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t
                                             float* delta, float* qval, int32_t* rowmax, int32_t* colmax,
                                             cudaStream_t stream);
 
+// imq_level_cover (plan.cu).
+imq_status launch_level_cover(const int32_t* maxima, int64_t n, int32_t b, int32_t cap, int32_t* out,
+                              cudaStream_t stream);
 // Line maxima of an integer matrix (plan.cu): logical rows and columns of a stored matrix.
 imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t cols, int64_t ld,
                            int32_t* rowmax, int32_t* colmax, cudaStream_t stream);

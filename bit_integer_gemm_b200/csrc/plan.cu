@@ -810,6 +810,31 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
+namespace {
+// out[i] = min(R^L - 1, cap) with L the level of m[i] (R = 2^bm1): the largest magnitude with as many
+// base-R digits as m[i].
+__global__ void __launch_bounds__(256) k_level_cover(const int32_t* __restrict__ m, int64_t n, int32_t bm1,
+                                                     int32_t cap, int32_t* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int L = level_of((uint32_t)m[i], bm1);
+    const int64_t top = (int64_t)L * bm1 >= 31 ? (int64_t)INT32_MAX : ((int64_t)1 << (L * bm1)) - 1;
+    out[i] = (int32_t)(top < cap ? top : cap);
+  }
+}
+}  // namespace
+
+imq_status launch_level_cover(const int32_t* maxima, int64_t n, int32_t b, int32_t cap, int32_t* out,
+                              cudaStream_t st) {
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  if (n == 0) return IMQ_OK;
+  int64_t grid = (n + 255) / 256;
+  if (grid > (int64_t)ds->num_sms * 4) grid = (int64_t)ds->num_sms * 4;
+  k_level_cover<<<(unsigned)grid, 256, 0, st>>>(maxima, n, b - 1, cap, out);
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
 imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t cols, int64_t ld,
                            int32_t* rowmax, int32_t* colmax, cudaStream_t st) {
   DeviceState* ds;

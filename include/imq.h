@@ -261,6 +261,18 @@ imq_status imq_plan_levels(const imq_plan_t *plan, int8_t *a_row, int8_t *a_col,
 imq_status imq_plan_groups(const imq_plan_t *plan, imq_group *groups, int32_t max_groups,
                            int32_t *n_out);
 
+/* Copies the plan's index maps of the unpacked operands to HOST buffers (the layout described under
+ * imq_unpack), so that a caller can name every byte of A' and B'^T:
+ *   tK[K_unp]    source inner index t of unpacked inner position p, -1 on padding
+ *   lAk[K_unp]   digit level lA of A at position p;  lBk[K_unp]: digit level lB of B (0 on padding)
+ *   srcA[M_unp]  source row of A of unpacked row u, -1 on an unused row;  lvlA[M_unp]: its level l
+ *   srcB[N_unp]  source column of B of unpacked row w of B'^T, -1 unused;  lvlB[N_unp]: its level m
+ * Byte (u, p) of A' is then digit lvlA[u] + lAk[p] of A[srcA[u], tK[p]] (zero where srcA or tK is -1,
+ * and, for a row unpacked both ways by the hybrid, at lAk[p] > 0); likewise for B'^T.  Any pointer
+ * may be NULL.  Synchronous; a diagnostic query, not part of the hot path. */
+imq_status imq_plan_maps(const imq_plan_t *plan, int32_t *tK, int8_t *lAk, int8_t *lBk, int32_t *srcA,
+                         int8_t *lvlA, int32_t *srcB, int8_t *lvlB);
+
 /* Frees the plan and its device arrays.  Call only after work that uses it has finished. */
 imq_status imq_plan_destroy(imq_plan_t *plan);
 
@@ -315,6 +327,18 @@ imq_status imq_unpack(const imq_plan_t *plan, const void *A, const void *B,
 imq_status imq_rtn_quantize_unpack(const imq_plan_t *plan, const void *X, imq_dtype xt, int64_t ld,
                                    double p, int32_t beta, int8_t *A_unp, float *deltaA,
                                    imq_stream_t stream);
+
+/*
+ * imq_level_cover -- out[i] = min(R^L - 1, cap), L the level of maxima[i] (its number of base-R digits,
+ * R = 2^(b-1)): the largest magnitude with as many digits.  For a plan kept with an unpacked weight
+ * (imq_rtn_quantize_unpack): planned with A's column maxima raised this way, the plan covers every later
+ * activation whose entries need no more digits than the one it was made from, since levels, layout and
+ * the bound only depend on the maxima the plan is given ("Approach": the digit count decides how many
+ * lines an entry takes).  maxima, out: device int32[n] (they may alias).  cap >= 0 (32767 for int16
+ * activations).  Asynchronous.
+ */
+imq_status imq_level_cover(const int32_t *maxima, int64_t n, int32_t b, int32_t cap, int32_t *out,
+                           imq_stream_t stream);
 
 /*
  * imq_gemm_unpacked -- the low-bit GEMM on already unpacked operands with the fold-back epilogue:

@@ -63,13 +63,11 @@ class _Plan(ctypes.Structure):
         ("b", ctypes.c_int32), ("strategy", ctypes.c_int32),
         ("dir_a", ctypes.c_int32), ("dir_b", ctypes.c_int32),
         ("M", ctypes.c_int64), ("K", ctypes.c_int64), ("N", ctypes.c_int64),
-        ("M_unp", ctypes.c_int64), ("N_unp", ctypes.c_int64), ("K_unp", ctypes.c_int64),
         ("M_eff", ctypes.c_int64), ("N_eff", ctypes.c_int64), ("K_eff", ctypes.c_int64),
         ("ratio", ctypes.c_double), ("bound", ctypes.c_double),
         ("bound_lt_2_31", ctypes.c_int32), ("n_groups", ctypes.c_int32),
         ("lmax", ctypes.c_int32 * 4), ("suml", ctypes.c_int64 * 4), ("oor_lines", ctypes.c_int64 * 4),
-        ("group_e", ctypes.c_int32 * MAX_GROUPS), ("group_off", ctypes.c_int64 * MAX_GROUPS),
-        ("group_len", ctypes.c_int64 * MAX_GROUPS), ("group_padded", ctypes.c_int64 * MAX_GROUPS),
+        ("group_e", ctypes.c_int32 * MAX_GROUPS), ("group_len", ctypes.c_int64 * MAX_GROUPS),
     ]
 
 
@@ -94,8 +92,8 @@ def _lib():
         lib.oracle_digits_array.restype = None
         lib.oracle_plan.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp,
                                     ctypes.POINTER(_Plan)]
-        lib.oracle_plan_maps.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 11
-        lib.oracle_unpack.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 13
+        lib.oracle_unpack_lines.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 7
+        lib.oracle_unpack.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 9
         lib.oracle_gemm_i64.argtypes = [vp, vp, i64, i64, i64, vp, i32]
         lib.oracle_gemm_i64.restype = None
         lib.oracle_unpacked_gemm.argtypes = [ctypes.POINTER(_Plan)] + [vp] * 7
@@ -169,6 +167,8 @@ def digits_array(v: np.ndarray, b: int, nl: int):
 
 @dataclass
 class Plan:
+    """The oracle's plan: directions, level statistics, unpacked sizes and the unpacked lines and inner
+    triples, with no memory layout (see oracle/plan.c)."""
     b: int
     strategy: int
     dir_a: int
@@ -176,16 +176,13 @@ class Plan:
     M: int
     K: int
     N: int
-    M_unp: int
-    N_unp: int
-    K_unp: int
     M_eff: int
     N_eff: int
     K_eff: int
     ratio: float
     bound: float
     bound_lt_2_31: bool
-    groups: list  # [(e, offset, len, padded)]
+    groups: list  # [(e, number of inner triples with lA + lB = e)], e ascending
     lmax: tuple
     suml: tuple
     oor_lines: tuple
@@ -193,7 +190,9 @@ class Plan:
     # unpacked GEMM (1 for a row of A or column of B that is not unpacked OUTER, the inner levels taken
     # over the lines that are not)
     levels: dict = field(default_factory=dict)
-    maps: dict = field(default_factory=dict)    # tK, lAk, lBk, srcA, lvlA, srcB, lvlB (int32)
+    # a_lines (M_eff x 2: row i, level l), b_lines (N_eff x 2: column j, level m), pairs (K_eff x 3:
+    # t, lA, lB), each in lexicographic order (int32)
+    lines: dict = field(default_factory=dict)
     _raw: object = None
 
     @property
@@ -216,51 +215,48 @@ def plan(A: np.ndarray, B: np.ndarray, b: int, strategy: int) -> Plan:
                          _ptr(lv["a_col"]), _ptr(lv["b_row"]), _ptr(lv["b_col"]), ctypes.byref(raw))
     if st != OK:
         raise OracleError(st, "plan")
-    mp = {"tK": np.zeros(raw.K_unp, np.int32), "lAk": np.zeros(raw.K_unp, np.int32),
-          "lBk": np.zeros(raw.K_unp, np.int32), "srcA": np.zeros(raw.M_unp, np.int32),
-          "lvlA": np.zeros(raw.M_unp, np.int32), "srcB": np.zeros(raw.N_unp, np.int32),
-          "lvlB": np.zeros(raw.N_unp, np.int32)}
-    st = lib.oracle_plan_maps(ctypes.byref(raw), _ptr(lv["a_row"]), _ptr(lv["a_col"]),
-                              _ptr(lv["b_row"]), _ptr(lv["b_col"]), *[_ptr(mp[k]) for k in
-                              ("tK", "lAk", "lBk", "srcA", "lvlA", "srcB", "lvlB")])
+    ln = {"a_lines": np.zeros((raw.M_eff, 2), np.int32), "b_lines": np.zeros((raw.N_eff, 2), np.int32),
+          "pairs": np.zeros((raw.K_eff, 3), np.int32)}
+    st = lib.oracle_unpack_lines(ctypes.byref(raw), _ptr(lv["a_row"]), _ptr(lv["a_col"]), _ptr(lv["b_row"]),
+                                 _ptr(lv["b_col"]), _ptr(ln["a_lines"]), _ptr(ln["b_lines"]), _ptr(ln["pairs"]))
     if st != OK:
-        raise OracleError(st, "plan_maps")
-    groups = [(raw.group_e[g], raw.group_off[g], raw.group_len[g], raw.group_padded[g])
-              for g in range(raw.n_groups)]
+        raise OracleError(st, "unpack_lines")
+    groups = [(raw.group_e[g], raw.group_len[g]) for g in range(raw.n_groups)]
     return Plan(b=raw.b, strategy=raw.strategy, dir_a=raw.dir_a, dir_b=raw.dir_b, M=raw.M, K=raw.K,
-                N=raw.N, M_unp=raw.M_unp, N_unp=raw.N_unp, K_unp=raw.K_unp, M_eff=raw.M_eff,
-                N_eff=raw.N_eff, K_eff=raw.K_eff, ratio=raw.ratio, bound=raw.bound,
+                N=raw.N, M_eff=raw.M_eff, N_eff=raw.N_eff, K_eff=raw.K_eff, ratio=raw.ratio, bound=raw.bound,
                 bound_lt_2_31=bool(raw.bound_lt_2_31), groups=groups, lmax=tuple(raw.lmax),
-                suml=tuple(raw.suml), oor_lines=tuple(raw.oor_lines), levels=lv, maps=mp, _raw=raw)
+                suml=tuple(raw.suml), oor_lines=tuple(raw.oor_lines), levels=lv, lines=ln, _raw=raw)
 
 
 def unpack(pl: Plan, A: np.ndarray, B: np.ndarray):
-    """Returns (A' int8 M_unp x K_unp, B'^T int8 N_unp x K_unp) in the library's layout."""
+    """Returns (A' int8 M_eff x K_eff, B'^T int8 N_eff x K_eff): entry (u, p) of A' is the digit of A for
+    unpacked line pl.lines['a_lines'][u] and inner triple pl.lines['pairs'][p]; likewise B'^T."""
     A = np.ascontiguousarray(A, dtype=np.int64)
     B = np.ascontiguousarray(B, dtype=np.int64)
-    Au = np.zeros((pl.M_unp, pl.K_unp), np.int8)
-    Bu = np.zeros((pl.N_unp, pl.K_unp), np.int8)
-    mp = pl.maps
-    st = _lib().oracle_unpack(ctypes.byref(pl._raw), *[_ptr(mp[k]) for k in
-                              ("tK", "lAk", "lBk", "srcA", "lvlA", "srcB", "lvlB")],
-                              _ptr(pl.levels["a_row"]), _ptr(pl.levels["b_col"]),
-                              _ptr(A), _ptr(B), _ptr(Au), _ptr(Bu))
+    Aq = np.zeros((pl.M_eff, pl.K_eff), np.int8)
+    Bq = np.zeros((pl.N_eff, pl.K_eff), np.int8)
+    ln = pl.lines
+    st = _lib().oracle_unpack(ctypes.byref(pl._raw), _ptr(pl.levels["a_row"]), _ptr(pl.levels["b_col"]),
+                              _ptr(ln["a_lines"]), _ptr(ln["b_lines"]), _ptr(ln["pairs"]), _ptr(A), _ptr(B),
+                              _ptr(Aq), _ptr(Bq))
     if st != OK:
         raise OracleError(st, "unpack")
-    return Au, Bu
+    return Aq, Bq
 
 
-def unpacked_gemm(pl: Plan, Au: np.ndarray, Bu: np.ndarray) -> np.ndarray:
-    """The integer product rebuilt from the unpacked operands (groups weighted by R^e, lines folded)."""
-    Au = np.ascontiguousarray(Au, dtype=np.int8)
-    Bu = np.ascontiguousarray(Bu, dtype=np.int8)
+def unpacked_gemm(pl: Plan, Aq: np.ndarray, Bq: np.ndarray, return_macs: bool = False):
+    """The integer product rebuilt from the unpacked operands (each inner triple weighted by R^(lA+lB),
+    each pair of lines by R^(l+m)); with return_macs also the multiply-adds the loop executed."""
+    Aq = np.ascontiguousarray(Aq, dtype=np.int8)
+    Bq = np.ascontiguousarray(Bq, dtype=np.int8)
     C = np.zeros((pl.M, pl.N), np.int64)
-    mp = pl.maps
-    st = _lib().oracle_unpacked_gemm(ctypes.byref(pl._raw), _ptr(mp["srcA"]), _ptr(mp["lvlA"]),
-                                     _ptr(mp["srcB"]), _ptr(mp["lvlB"]), _ptr(Au), _ptr(Bu), _ptr(C))
+    macs = ctypes.c_int64(0)
+    ln = pl.lines
+    st = _lib().oracle_unpacked_gemm(ctypes.byref(pl._raw), _ptr(ln["a_lines"]), _ptr(ln["b_lines"]),
+                                     _ptr(ln["pairs"]), _ptr(Aq), _ptr(Bq), _ptr(C), ctypes.byref(macs))
     if st != OK:
         raise OracleError(st, "unpacked_gemm")
-    return C
+    return (C, int(macs.value)) if return_macs else C
 
 
 # ----------------------------------------------------------------------------------------------

@@ -27,28 +27,33 @@ void oracle_gemm_i64(const int64_t *A, const int64_t *B, int64_t M, int64_t K, i
   }
 }
 
-/* C (M x N, overwritten) from the unpacked operands: for every pair of used lines (u, w),
- *   acc = sum over exponent groups g of R^e_g * sum_{p in g} A'[u,p] * B'^T[w,p]
- * and acc * R^(lvlA[u] + lvlB[w]) is added to C[srcA[u], srcB[w]]. */
-int oracle_unpacked_gemm(const oracle_plan_t *pl, const int32_t *srcA, const int32_t *lvlA,
-                         const int32_t *srcB, const int32_t *lvlB, const int8_t *Aunp,
-                         const int8_t *Bunp_t, int64_t *C) {
-  const int64_t N = pl->N, Ku = pl->K_unp;
+/* C (M x N, overwritten) from the unpacked operands ("Approach": bit-shift scaling and accumulation):
+ * for every unpacked line (i, l) of A and (j, m) of B,
+ *   C[i, j] += R^(l + m) * sum over inner triples (t, lA, lB) of R^(lA + lB) * A'[(i,l),p] * B'[p,(j,m)]
+ * with R = 2^(b-1).  *macs (when not NULL) gets the number of multiply-adds of unpacked entries the
+ * loop executed, the count the unpack ratio describes. */
+int oracle_unpacked_gemm(const oracle_plan_t *pl, const int32_t *a_lines, const int32_t *b_lines,
+                         const int32_t *pairs, const int8_t *Aq, const int8_t *Bq, int64_t *C,
+                         int64_t *macs) {
+  const int64_t N = pl->N, Ke = pl->K_eff;
   const int sh = pl->b - 1;
+  int64_t count = 0;
   memset(C, 0, (size_t)(pl->M * N) * sizeof(int64_t));
-  for (int64_t u = 0; u < pl->M_unp; ++u) {
-    if (srcA[u] < 0) continue;
-    for (int64_t w = 0; w < pl->N_unp; ++w) {
-      if (srcB[w] < 0) continue;
+  for (int64_t u = 0; u < pl->M_eff; ++u) {
+    const int64_t i = a_lines[2 * u];
+    const int l = a_lines[2 * u + 1];
+    for (int64_t w = 0; w < pl->N_eff; ++w) {
+      const int64_t j = b_lines[2 * w];
+      const int m = b_lines[2 * w + 1];
       int64_t acc = 0;
-      for (int g = 0; g < pl->n_groups; ++g) {
-        int64_t part = 0;
-        for (int64_t p = pl->group_off[g]; p < pl->group_off[g] + pl->group_padded[g]; ++p)
-          part += (int64_t)Aunp[u * Ku + p] * (int64_t)Bunp_t[w * Ku + p];
-        acc += part * ((int64_t)1 << (pl->group_e[g] * sh));
+      for (int64_t p = 0; p < Ke; ++p) {
+        const int e = pairs[3 * p + 1] + pairs[3 * p + 2];
+        acc += (int64_t)Aq[u * Ke + p] * (int64_t)Bq[w * Ke + p] * ((int64_t)1 << (e * sh));
       }
-      C[(int64_t)srcA[u] * N + srcB[w]] += acc * ((int64_t)1 << ((lvlA[u] + lvlB[w]) * sh));
+      count += Ke;
+      C[i * N + j] += acc * ((int64_t)1 << ((l + m) * sh));
     }
   }
+  if (macs) *macs = count;
   return OR_OK;
 }

@@ -42,27 +42,25 @@
 #define OR_DIR_INNER 2
 #define OR_DIR_BOTH 3 /* OR_DIR_OUTER | OR_DIR_INNER: the hybrid's two parts */
 
+/* Exponents e = lA + lB of the inner pairs: at most 2 * 31 + 1 distinct values (levels are at most 32). */
 #define OR_MAX_GROUPS 64
-#define OR_INNER_PAD 128
-#define OR_A_GROUP 32
-#define OR_B_GROUP 32
 
+/* The plan: sizes and counts only.  The unpacked operands are stated without any memory layout: an
+ * unpacked line of A is a pair (source row i, level l), an unpacked line of B a pair (source column j,
+ * level m), an unpacked inner index a triple (t, lA, lB); see oracle_unpack_lines. */
 typedef struct {
   int32_t b, strategy, dir_a, dir_b;
   int64_t M, K, N;
-  int64_t M_unp, N_unp, K_unp;
-  int64_t M_eff, N_eff, K_eff;
+  int64_t M_eff, N_eff, K_eff;  /* numbers of unpacked lines of A, of B, and of inner triples     */
   double ratio;
   double bound;            /* sum_t max_i|A_it| * max_j|B_tj|, rounded to double          */
   int32_t bound_lt_2_31;   /* exact comparison of the bound with 2^31                     */
-  int32_t n_groups;
+  int32_t n_groups;        /* distinct exponents e = lA + lB among the inner triples      */
   int32_t lmax[4];         /* A rows, A cols, B rows, B cols                              */
   int64_t suml[4];
   int64_t oor_lines[4];
-  int32_t group_e[OR_MAX_GROUPS];
-  int64_t group_off[OR_MAX_GROUPS];
-  int64_t group_len[OR_MAX_GROUPS];
-  int64_t group_padded[OR_MAX_GROUPS];
+  int32_t group_e[OR_MAX_GROUPS];    /* the exponents, ascending                         */
+  int64_t group_len[OR_MAX_GROUPS];  /* inner triples with that exponent                 */
 } oracle_plan_t;
 
 /* percentile.c */
@@ -81,20 +79,19 @@ void oracle_digits_array(const int64_t *v, int64_t n, int b, int nl, int64_t *ou
 int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N, int b,
                 int strategy, int32_t *LrA, int32_t *LcA, int32_t *LrB, int32_t *LcB,
                 oracle_plan_t *out);
-int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcA,
-                     const int32_t *LrB, const int32_t *LcB, int32_t *tK, int32_t *lAk,
-                     int32_t *lBk, int32_t *srcA, int32_t *lvlA, int32_t *srcB, int32_t *lvlB);
+int oracle_unpack_lines(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcA,
+                        const int32_t *LrB, const int32_t *LcB, int32_t *a_lines, int32_t *b_lines,
+                        int32_t *pairs);
 /* unpack.c */
-int oracle_unpack(const oracle_plan_t *pl, const int32_t *tK, const int32_t *lAk,
-                  const int32_t *lBk, const int32_t *srcA, const int32_t *lvlA,
-                  const int32_t *srcB, const int32_t *lvlB, const int32_t *LrA, const int32_t *LcB,
-                  const int64_t *A, const int64_t *B, int8_t *Aunp, int8_t *Bunp_t);
+int oracle_unpack(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcB,
+                  const int32_t *a_lines, const int32_t *b_lines, const int32_t *pairs,
+                  const int64_t *A, const int64_t *B, int8_t *Aq, int8_t *Bq);
 /* gemm.c */
 void oracle_gemm_i64(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_t N,
                      int64_t *C, int nthreads);
-int oracle_unpacked_gemm(const oracle_plan_t *pl, const int32_t *srcA, const int32_t *lvlA,
-                         const int32_t *srcB, const int32_t *lvlB, const int8_t *Aunp,
-                         const int8_t *Bunp_t, int64_t *C);
+int oracle_unpacked_gemm(const oracle_plan_t *pl, const int32_t *a_lines, const int32_t *b_lines,
+                         const int32_t *pairs, const int8_t *Aq, const int8_t *Bq, int64_t *C,
+                         int64_t *macs);
 /* dequant.c */
 void oracle_dequant(const int64_t *C, int64_t M, int64_t N, const float *dA, int gA,
                     const float *dB, int gB, double *Cf);

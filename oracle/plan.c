@@ -21,10 +21,12 @@
  *        those remaining lines only; tau is the threshold of least M_eff * K_eff (A) or N_eff * K_eff (B),
  *        the smallest such tau on a tie; the direction is then OUTER, INNER or both (OR_DIR_BOTH).  The
  *        level vectors the plan returns are then the levels each line carries in the unpacked GEMM.
- *   layout: inner pairs (t, lA, lB) ordered by e = lA + lB, then lA, then t, each exponent group padded
- *   with zeros to OR_INNER_PAD; OUTER lines sorted by level (stable), floor(G / L) source lines per
- *   group of G unpacked lines (G = OR_A_GROUP for rows of A, OR_B_GROUP for columns of B), the L lines
- *   of one source consecutive, unused lines empty.
+ *   the unpacked operands have no memory layout here: an unpacked line of A is a pair (row i, level l),
+ *   l < the level row i carries when A is unpacked OUTER (else l = 0 only); an unpacked line of B is a
+ *   pair (column j, level m) likewise; an unpacked inner index is a triple (t, lA, lB), lA < the level
+ *   of A's column t when A is unpacked INNER (else 0 only), lB < the level of B's row t when B is
+ *   unpacked INNER (else 0 only).  oracle_unpack_lines lists them in lexicographic order, which is a
+ *   naming, not a layout: every check against a kernel matches entries by these pairs and triples.
  */
 #include <stdlib.h>
 #include <string.h>
@@ -216,58 +218,23 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
   else
     out->ratio = 1.0;
 
-  /* exponent groups of the inner dimension */
-  int64_t off = 0;
+  /* exponents of the inner triples: e = lA + lB, with the number of triples carrying each */
   int ng = 0;
   for (int e = 0; e <= maxla + maxlb - 2; ++e) {
     int64_t len = 0;
-    for (int la = 0; la < maxla; ++la) {
-      int lb = e - la;
-      if (lb < 0 || lb >= maxlb) continue;
-      for (int64_t t = 0; t < K; ++t) {
-        int64_t a = (da & OR_DIR_INNER) ? LcA[t] : 1;
-        int64_t bb = (db & OR_DIR_INNER) ? LrB[t] : 1;
-        if (a > la && bb > lb) len += 1;
-      }
+    for (int64_t t = 0; t < K; ++t) {
+      const int64_t a = (da & OR_DIR_INNER) ? LcA[t] : 1;
+      const int64_t bb = (db & OR_DIR_INNER) ? LrB[t] : 1;
+      for (int la = 0; la < a; ++la)
+        if (e - la >= 0 && e - la < bb) len += 1;
     }
     if (len == 0) continue;
     if (ng >= OR_MAX_GROUPS) return OR_ERR_ARG;
-    int64_t padded = (len + OR_INNER_PAD - 1) / OR_INNER_PAD * OR_INNER_PAD;
     out->group_e[ng] = e;
-    out->group_off[ng] = off;
     out->group_len[ng] = len;
-    out->group_padded[ng] = padded;
-    off += padded;
     ng += 1;
   }
   out->n_groups = ng;
-  out->K_unp = off;
-
-  /* outer sizes: groups of lines of equal level */
-  if (da & OR_DIR_OUTER) {
-    int64_t groups = 0;
-    for (int L = 1; L <= out->lmax[0]; ++L) {
-      int64_t cnt = 0;
-      for (int64_t i = 0; i < M; ++i) cnt += (LrA[i] == L);
-      int64_t per = OR_A_GROUP / L;
-      groups += (cnt + per - 1) / per;
-    }
-    out->M_unp = groups * OR_A_GROUP;
-  } else {
-    out->M_unp = M;
-  }
-  if (db & OR_DIR_OUTER) {
-    int64_t groups = 0;
-    for (int L = 1; L <= out->lmax[3]; ++L) {
-      int64_t cnt = 0;
-      for (int64_t j = 0; j < N; ++j) cnt += (LcB[j] == L);
-      int64_t per = OR_B_GROUP / L;
-      groups += (cnt + per - 1) / per;
-    }
-    out->N_unp = groups * OR_B_GROUP;
-  } else {
-    out->N_unp = N;
-  }
 
   /* bound on |C| and on every partial sum of the fold-back */
   __int128 bound = 0;
@@ -284,70 +251,45 @@ int oracle_plan(const int64_t *A, const int64_t *B, int64_t M, int64_t K, int64_
   return OR_OK;
 }
 
-/* Fills the index maps of the layout described at the top of this file.
- * tK/lAk/lBk: K_unp entries (tK = -1 on padding).  srcA/lvlA: M_unp entries (srcA = -1 on unused
- * lines).  srcB/lvlB: N_unp entries. */
-int oracle_plan_maps(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcA,
-                     const int32_t *LrB, const int32_t *LcB, int32_t *tK, int32_t *lAk,
-                     int32_t *lBk, int32_t *srcA, int32_t *lvlA, int32_t *srcB, int32_t *lvlB) {
+/* The unpacked lines and inner triples of a plan, in lexicographic order (see the top of this file):
+ * a_lines[2u], a_lines[2u+1] = (i, l) for u < M_eff; b_lines[2w], b_lines[2w+1] = (j, m) for w < N_eff;
+ * pairs[3p .. 3p+2] = (t, lA, lB) for p < K_eff.  The level vectors are those oracle_plan returned. */
+int oracle_unpack_lines(const oracle_plan_t *pl, const int32_t *LrA, const int32_t *LcA,
+                        const int32_t *LrB, const int32_t *LcB, int32_t *a_lines, int32_t *b_lines,
+                        int32_t *pairs) {
   const int da = pl->dir_a, db = pl->dir_b;
-  const int64_t M = pl->M, K = pl->K, N = pl->N;
-  int maxla = (da & OR_DIR_INNER) ? pl->lmax[1] : 1;
-  int maxlb = (db & OR_DIR_INNER) ? pl->lmax[2] : 1;
-
-  for (int64_t p = 0; p < pl->K_unp; ++p) { tK[p] = -1; lAk[p] = 0; lBk[p] = 0; }
-  for (int g = 0; g < pl->n_groups; ++g) {
-    int e = pl->group_e[g];
-    int64_t p = pl->group_off[g];
-    for (int la = 0; la < maxla; ++la) {
-      int lb = e - la;
-      if (lb < 0 || lb >= maxlb) continue;
-      for (int64_t t = 0; t < K; ++t) {
-        int64_t a = (da & OR_DIR_INNER) ? LcA[t] : 1;
-        int64_t bb = (db & OR_DIR_INNER) ? LrB[t] : 1;
-        if (a > la && bb > lb) {
-          tK[p] = (int32_t)t;
-          lAk[p] = la;
-          lBk[p] = lb;
-          p += 1;
-        }
-      }
+  int64_t u = 0;
+  for (int64_t i = 0; i < pl->M; ++i) {
+    const int L = (da & OR_DIR_OUTER) ? LrA[i] : 1;
+    for (int l = 0; l < L; ++l) {
+      a_lines[2 * u] = (int32_t)i;
+      a_lines[2 * u + 1] = l;
+      u += 1;
     }
-    if (p != pl->group_off[g] + pl->group_len[g]) return OR_ERR_ARG;
   }
-
-  for (int64_t u = 0; u < pl->M_unp; ++u) { srcA[u] = -1; lvlA[u] = 0; }
-  if (da & OR_DIR_OUTER) {
-    int64_t grp = 0;
-    for (int L = 1; L <= pl->lmax[0]; ++L) {
-      int64_t per = OR_A_GROUP / L, rank = 0;
-      for (int64_t i = 0; i < M; ++i) {
-        if (LrA[i] != L) continue;
-        int64_t base = (grp + rank / per) * OR_A_GROUP + (rank % per) * L;
-        for (int l = 0; l < L; ++l) { srcA[base + l] = (int32_t)i; lvlA[base + l] = l; }
-        rank += 1;
-      }
-      grp += (rank + per - 1) / per;
+  if (u != pl->M_eff) return OR_ERR_ARG;
+  int64_t w = 0;
+  for (int64_t j = 0; j < pl->N; ++j) {
+    const int L = (db & OR_DIR_OUTER) ? LcB[j] : 1;
+    for (int m = 0; m < L; ++m) {
+      b_lines[2 * w] = (int32_t)j;
+      b_lines[2 * w + 1] = m;
+      w += 1;
     }
-  } else {
-    for (int64_t i = 0; i < M; ++i) srcA[i] = (int32_t)i;
   }
-
-  for (int64_t w = 0; w < pl->N_unp; ++w) { srcB[w] = -1; lvlB[w] = 0; }
-  if (db & OR_DIR_OUTER) {
-    int64_t grp = 0;
-    for (int L = 1; L <= pl->lmax[3]; ++L) {
-      int64_t per = OR_B_GROUP / L, rank = 0;
-      for (int64_t j = 0; j < N; ++j) {
-        if (LcB[j] != L) continue;
-        int64_t base = (grp + rank / per) * OR_B_GROUP + (rank % per) * L;
-        for (int l = 0; l < L; ++l) { srcB[base + l] = (int32_t)j; lvlB[base + l] = l; }
-        rank += 1;
+  if (w != pl->N_eff) return OR_ERR_ARG;
+  int64_t p = 0;
+  for (int64_t t = 0; t < pl->K; ++t) {
+    const int la = (da & OR_DIR_INNER) ? LcA[t] : 1;
+    const int lb = (db & OR_DIR_INNER) ? LrB[t] : 1;
+    for (int x = 0; x < la; ++x)
+      for (int y = 0; y < lb; ++y) {
+        pairs[3 * p] = (int32_t)t;
+        pairs[3 * p + 1] = x;
+        pairs[3 * p + 2] = y;
+        p += 1;
       }
-      grp += (rank + per - 1) / per;
-    }
-  } else {
-    for (int64_t j = 0; j < N; ++j) srcB[j] = (int32_t)j;
   }
+  if (p != pl->K_eff) return OR_ERR_ARG;
   return OR_OK;
 }

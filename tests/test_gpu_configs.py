@@ -1,8 +1,8 @@
 """Full-size parity on the five seeded workloads (tiny, q_proj, mlp, attention, wgrad), in the launch
 configuration the benchmark uses: quantiser side outputs feed the plan, imq_unpack then
-imq_gemm_unpacked.  Integer outputs are compared bit-exactly with the oracle -- in full, except the
-three MLP products whose rows are sampled (the oracle's exact product of 512 sampled rows); fp32
-outputs within 1e-6 relative.
+imq_gemm_unpacked.  Integer outputs are compared bit-exactly with the oracle in full -- every quantised
+entry, the plan, every unpacked byte (matched to the oracle's digit through the library's index maps)
+and every entry of C; fp32 outputs within 1e-6 relative.
 """
 import numpy as np
 import pytest
@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import assert_f32_close, logical, logical_maxes, plan_matches, to_device
+from tests.gpu_common import assert_f32_close, check_unpacked, logical, logical_maxes, plan_matches, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -47,13 +47,10 @@ def _check_gemm(imq, g, strategy, qa, qb, A, B, dA, dB, want=None, rows=None, ch
     pl = oracle.plan(A, B, g.b, strategy)
     plan = imq.imq_plan(qa.xint, qb.xint, g.b, strategy, g.transA, g.transB,
                         maxes=logical_maxes(imq, qa, qb, g.transA, g.transB))
-    plan_matches(plan.info, pl)
+    plan_matches(plan.info, pl, plan.groups())
     Au, Bu = imq.imq_unpack(plan, qa.xint, qb.xint)
     if check_unpack:
-        oAu, oBu = oracle.unpack(pl, A, B)
-        assert np.array_equal(Au.cpu().numpy(), oAu), f"{g.name} A' bytes"
-        assert np.array_equal(Bu.cpu().numpy(), oBu), f"{g.name} B'^T bytes"
-        del oAu, oBu
+        check_unpacked(plan, pl, Au.cpu().numpy(), Bu.cpu().numpy(), A, B)
     gA, gB = g.gA, g.gB
     C, Cf = imq.imq_gemm_unpacked(plan, Au, Bu, qa.delta, gA, qb.delta, gB,
                                   c_dtype=torch.int32 if pl.acc_bits == 32 else torch.int64)
@@ -106,13 +103,12 @@ def test_config_q_proj(imq):
     assert infos[5]["ratio"] <= infos[0]["ratio"]  # joint Mix is never worse than Mix
 
 
-def test_config_mlp(imq):
-    rows = np.sort(np.random.default_rng(0).choice(2048, 512, replace=False))
-    for g in workloads.mlp():
-        _run(imq, g, rows=rows)
+@pytest.mark.parametrize("which", [0, 1, 2], ids=["gate", "up", "down"])
+def test_config_mlp(imq, which):
+    _run(imq, workloads.mlp()[which])
 
 
-@pytest.mark.parametrize("head", [0, 7, 19, 31])
+@pytest.mark.parametrize("head", list(range(32)))
 def test_config_attention(imq, head):
     for g in workloads.attention_head(head):
         _run(imq, g)
@@ -137,9 +133,12 @@ def test_config_heavy_tokens_hybrid(imq):
     assert infos[0]["ratio"] > 1.9 and infos[6]["ratio"] < 1.01
 
 
-def test_config_wgrad(imq):
-    for g in workloads.wgrad():
-        _run(imq, g, check_unpack=(g.b == 8))
+@pytest.mark.parametrize("b", [3, 4, 5, 8])
+def test_config_wgrad(imq, b):
+    """The weight-gradient sweep: every unpack width and all five strategies, every byte and every
+    output entry."""
+    g = [w for w in workloads.wgrad() if w.b == b][0]
+    _run(imq, g)
 
 
 @pytest.mark.parametrize("b", [4, 5])
@@ -147,7 +146,7 @@ def test_config_training_triple(imq, b):
     """Forward, input gradient and weight gradient of one linear layer, each with per-tensor RTN, through
     the library with the stored matrices of one training step (transposes instead of copies)."""
     for g in workloads.training_triple(b):
-        infos = _run(imq, g, check_unpack=(g.name != "train_dgrad"))
+        infos = _run(imq, g)
         assert infos[0]["M"] == g.M and infos[0]["N"] == g.N and infos[0]["K"] == g.K
 
 

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import assert_f32_close, to_device
+from tests.gpu_common import assert_f32_close, check_unpacked, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -64,8 +64,7 @@ def test_fused_matches_separate_path_and_oracle(imq, dtype, shape, b):
     xi, dx, _ = oracle.rtn_quantize(oracle.as_f32(Xs.data, dtype), oracle.PER_ROW, p, beta)
     wi, dw, _ = oracle.rtn_quantize(oracle.as_f32(Ws.data, "bf16"), oracle.PER_COL, p, beta)
     pl = oracle.plan(xi, wi, b, oracle.COL_ROW)
-    oAu, _ = oracle.unpack(pl, xi, wi)
-    assert np.array_equal(Af.cpu().numpy(), oAu)
+    check_unpacked(plan, pl, Af.cpu().numpy(), Bu.cpu().numpy(), xi, wi)
     assert np.array_equal(dAf.cpu().numpy(), dx)
     # the GEMM with the kept B'^T
     C, Cf = imq.imq_gemm_unpacked(plan, Af, Bu, dAf, imq.IMQ_PER_ROW, qw.delta, imq.IMQ_PER_COL)

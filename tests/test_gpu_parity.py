@@ -12,7 +12,8 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_common import assert_f32_close, logical, plan_matches, to_device, unsupported
+from tests.gpu_common import (assert_f32_close, check_layout, check_unpacked, logical, plan_matches, to_device,
+                               unsupported)
 
 pytestmark = pytest.mark.gpu
 
@@ -235,16 +236,14 @@ def _run_path(imq, A, B, b, strategy, transA, transB, dtype=torch.int16, check_u
         assert e.value.status == imq.IMQ_ERR_UNSUPPORTED
         return None
     plan = imq.imq_plan(Ad, Bd, b, strategy, transA, transB)
-    plan_matches(plan.info, pl)
+    plan_matches(plan.info, pl, plan.groups())
     lv = plan.levels()
     for k in ("a_row", "a_col", "b_row", "b_col"):
         assert np.array_equal(lv[k].astype(np.int32), pl.levels[k]), k
-    assert plan.groups() == [tuple(g) for g in pl.groups]
     Au, Bu = imq.imq_unpack(plan, Ad, Bd)
     if check_unpack:
-        oAu, oBu = oracle.unpack(pl, A, B)
-        assert np.array_equal(Au.cpu().numpy(), oAu), "A' bytes"
-        assert np.array_equal(Bu.cpu().numpy(), oBu), "B'^T bytes"
+        mp = check_unpacked(plan, pl, Au.cpu().numpy(), Bu.cpu().numpy(), A, B)
+        check_layout(plan, mp)
     rng = np.random.default_rng(M * 7 + N)
     dA = rng.uniform(1e-3, 1.0, M).astype(np.float32)
     dB = rng.uniform(1e-3, 1.0, N).astype(np.float32)

@@ -285,22 +285,25 @@ def test_ratio_closed_forms():
     B8 = rng.integers(-127, 128, size=(70, 17)).astype(np.int64)
     pl = oracle.plan(A8, B8, 8, oracle.MIX)
     assert (pl.dir_a, pl.dir_b, pl.ratio) == (oracle.DIR_NONE, oracle.DIR_NONE, 1.0)
-    assert pl.K_unp == 128 and pl.M_unp == 33 and pl.N_unp == 17
+    assert (pl.M_eff, pl.N_eff, pl.K_eff) == (33, 17, 70)
     Au, Bu = oracle.unpack(pl, A8, B8)
-    assert np.array_equal(Au[:, :70], A8.astype(np.int8)) and not Au[:, 70:].any()
-    assert np.array_equal(Bu[:, :70], B8.T.astype(np.int8))
+    assert np.array_equal(Au, A8.astype(np.int8))
+    assert np.array_equal(Bu, B8.T.astype(np.int8))
 
 
 def test_ratio_equals_counted_macs():
+    """The ratio (computed from the line levels) equals the multiply-adds the naive unpacked loop
+    counts while it rebuilds the product, over the original M N K."""
     rng = np.random.default_rng(24)
     for _ in range(200):
         M, K, N = (int(x) for x in rng.integers(1, 12, size=3))
         b = int(rng.integers(2, 9))
         A, B = workloads.random_case(rng, M, K, N, big=3000, frac=0.2)
-        for st in range(5):
+        for st in range(7):
             pl = oracle.plan(A, B, b, st)
-            mp = pl.maps
-            macs = int((mp["srcA"] >= 0).sum()) * int((mp["srcB"] >= 0).sum()) * int((mp["tK"] >= 0).sum())
+            Au, Bu = oracle.unpack(pl, A, B)
+            C, macs = oracle.unpacked_gemm(pl, Au, Bu, return_macs=True)
+            assert np.array_equal(C, A @ B)
             assert macs == pl.M_eff * pl.N_eff * pl.K_eff
             assert pl.ratio == pytest.approx(macs / (M * N * K), rel=1e-12)
 
@@ -487,15 +490,18 @@ def test_hybrid_worked_case():
     want_cols[[5, 9]] = 2
     assert np.array_equal(hyb.levels["a_row"], want_rows) and np.array_equal(hyb.levels["a_col"], want_cols)
     Au, Bu = oracle.unpack(hyb, A, B)
-    # row 0's two lines hold its digits (4 and 6: 100 = 6 * 16 + 4) in the level-0 segment only
-    r0 = np.flatnonzero(hyb.maps["srcA"] == 0)
-    lvl0 = hyb.maps["tK"] >= 0
-    hi = lvl0 & (hyb.maps["lAk"] > 0)
-    assert np.all(Au[r0[0], lvl0 & ~hi] == 4) and np.all(Au[r0[1], lvl0 & ~hi] == 6)
-    assert not Au[r0][:, hi].any()
-    # rows 10..29 carry the digits of columns 5 and 9 in the inner segments
-    r10 = int(np.flatnonzero(hyb.maps["srcA"] == 10)[0])
-    assert sorted(Au[r10, hi].tolist()) == [6, 6]
+    # row 0's two lines (0, 0) and (0, 1) hold its digits (4 and 6: 100 = 6 * 16 + 4) at the triples
+    # with lA = 0 only
+    al, pr = hyb.lines["a_lines"], hyb.lines["pairs"]
+    assert al[:3].tolist() == [[0, 0], [0, 1], [1, 0]]
+    lo = pr[:, 1] == 0
+    hi = ~lo
+    assert int(hi.sum()) == 2 and sorted(pr[hi, 0].tolist()) == [5, 9]
+    assert np.all(Au[0, lo] == 4) and np.all(Au[1, lo] == 6)
+    assert not Au[:2][:, hi].any()
+    # row 10 (line 11) carries the high digits of columns 5 and 9 at their lA = 1 triples
+    assert al[11].tolist() == [10, 0]
+    assert sorted(Au[11, hi].tolist()) == [6, 6]
     assert np.array_equal(oracle.unpacked_gemm(hyb, Au, Bu), A @ B)
 
 
@@ -539,55 +545,38 @@ def test_dequant_exact_rational_bound():
 
 
 # ------------------------------------------------------------------------------------------------
-# the unpacked layout (a READING: the page fixes no operand order) is the documented one
+# the unpacked lines and inner triples ("Approach": a row or column with out-of-bound entries becomes
+# several in-bound ones) -- re-derived from numpy levels, independent of the oracle's C code
 # ------------------------------------------------------------------------------------------------
-def test_layout_follows_documented_order():
+def test_unpacked_lines_and_triples_from_levels():
+    """Line (i, l) of A for every l below the level row i carries when A is unpacked OUTER (l = 0 only
+    otherwise); likewise (j, m) for B; triple (t, lA, lB) for lA below A's column level when A is INNER
+    and lB below B's row level when B is INNER.  The exponent counts are those of the triples."""
     rng = np.random.default_rng(28)
-    for _ in range(150):
-        M, K, N = (int(x) for x in rng.integers(1, 40, size=3))
+    for case in range(150):
+        M, K, N = (int(x) for x in rng.integers(1, 30, size=3))
         b = int(rng.integers(2, 9))
         A, B = workloads.random_case(rng, M, K, N, big=4000, frac=0.2)
-        if _ % 3 == 0:
+        if case % 3 == 0:
             A, B = workloads.rows_and_cols_case(rng, M, K, N, big=4000, dense_rows=2, dense_cols=2)
-        for st in range(7):
+        LA, LB = _levels_numpy(A, b), _levels_numpy(B, b)
+        for st in range(6):  # the hybrid's carried levels are pinned by its own brute force above
             pl = oracle.plan(A, B, b, st)
-            mp, lv = pl.maps, pl.levels
-            la = lv["a_col"] if pl.dir_a & oracle.DIR_INNER else np.ones(K, np.int32)
-            lb = lv["b_row"] if pl.dir_b & oracle.DIR_INNER else np.ones(K, np.int32)
-            # inner: groups ascending in e, offsets multiples of 128, inside a group (lA, t) ascending
-            want = []
-            for e, off, ln, padded in pl.groups:
-                assert off % 128 == 0 and padded % 128 == 0 and padded - ln < 128
-                pairs = sorted((lA, t) for t in range(K) for lA in range(la[t]) for lB in [e - lA]
-                               if 0 <= lB < lb[t])
-                got = list(zip(mp["lAk"][off:off + ln].tolist(), mp["tK"][off:off + ln].tolist()))
-                assert got == pairs
-                assert np.all(mp["lAk"][off:off + ln] + mp["lBk"][off:off + ln] == e)
-                assert np.all(mp["tK"][off + ln:off + padded] == -1)
-                want.append(e)
-            assert want == sorted(want)
-            # outer: per group one level L, floor(G/L) sources of that level, lines (src, l) in order
-            for src, lvl, lines, G, dirv, outer in (
-                    (mp["srcA"], mp["lvlA"], lv["a_row"], 32, pl.dir_a, oracle.DIR_OUTER),
-                    (mp["srcB"], mp["lvlB"], lv["b_col"], 32, pl.dir_b, oracle.DIR_OUTER)):
-                if not dirv & outer:
-                    assert np.array_equal(src, np.arange(src.size)) and not lvl.any()
-                    continue
-                assert src.size % G == 0
-                seen = []
-                for g0 in range(0, src.size, G):
-                    s, l = src[g0:g0 + G], lvl[g0:g0 + G]
-                    used = s >= 0
-                    n = int(used.sum())
-                    assert used[:n].all() and not used[n:].any()
-                    L = int(lines[s[0]])
-                    assert n % L == 0 and n // L <= G // L
-                    for k in range(n // L):
-                        assert np.all(s[k * L:(k + 1) * L] == s[k * L])
-                        assert np.array_equal(l[k * L:(k + 1) * L], np.arange(L))
-                        assert lines[s[k * L]] == L
-                        seen.append((L, int(s[k * L])))
-                assert seen == sorted(seen) and len(seen) == lines.size
+            la_row = LA.max(1) if pl.dir_a & oracle.DIR_OUTER else np.ones(M, np.int64)
+            la_col = LA.max(0) if pl.dir_a & oracle.DIR_INNER else np.ones(K, np.int64)
+            lb_row = LB.max(1) if pl.dir_b & oracle.DIR_INNER else np.ones(K, np.int64)
+            lb_col = LB.max(0) if pl.dir_b & oracle.DIR_OUTER else np.ones(N, np.int64)
+            a_lines = [[i, l] for i in range(M) for l in range(la_row[i])]
+            b_lines = [[j, m] for j in range(N) for m in range(lb_col[j])]
+            pairs = [[t, x, y] for t in range(K) for x in range(la_col[t]) for y in range(lb_row[t])]
+            assert pl.lines["a_lines"].tolist() == a_lines
+            assert pl.lines["b_lines"].tolist() == b_lines
+            assert pl.lines["pairs"].tolist() == pairs
+            assert (pl.M_eff, pl.N_eff, pl.K_eff) == (len(a_lines), len(b_lines), len(pairs))
+            es = {}
+            for _, x, y in pairs:
+                es[x + y] = es.get(x + y, 0) + 1
+            assert pl.groups == sorted(es.items())
 
 
 def test_cached_plan_is_exact_for_covered_inputs():
