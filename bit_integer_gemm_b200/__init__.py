@@ -95,6 +95,14 @@ SIGNATURES = {
     "imq_gemm_unpacked": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP],
     "imq_unpacked_gemm": [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _VP, _I32, _I64, _VP, _I64, _VP, _SZ, _VP],
     "imq_level_cover": [_VP, _I64, _I32, _I32, _VP, _VP],
+    "imq_plan_batched": [_I32, _VP, _I64, _VP, _I64, _I32, _I64, _I64, _I64, _I32, _I64, _I32, _I64, _I32, _I32,
+                         _VP, _VP, _VP, _VP, _VP, _VP],
+    "imq_batch_workspace": [_I32, _VP, _VP, _VP],
+    "imq_unpack_batched": [_I32, _VP, _VP, _I64, _VP, _I64, _VP, _SZ, _VP],
+    "imq_gemm_unpacked_batched": [_I32, _VP, _VP, _SZ, _VP, _I64, _I32, _VP, _I64, _I32, _VP, _I64, _I32, _I64, _VP,
+                                  _I64, _I64, _VP],
+    "imq_unpacked_gemm_batched": [_I32, _VP, _VP, _I64, _VP, _I64, _VP, _I64, _I32, _VP, _I64, _I32, _VP, _I64, _I32,
+                                  _I64, _VP, _I64, _I64, _VP, _SZ, _VP],
     "imq_device_status": [_VP, _I32],
     "imq_check_bounded_wait": [ctypes.c_uint64, _VP],
     "imq_status_str": [_I32],
@@ -213,9 +221,10 @@ def imq_rtn_quantize_rows_noalloc(X: torch.Tensor, p: float, beta: int, out_dtyp
 class Plan:
     """Owns an imq_plan_t handle; `info` is the imq_plan_info summary as a dict."""
 
-    def __init__(self, handle, A, B):
+    def __init__(self, handle, A, B, transA=False, transB=False):
         self.handle = handle
         self._keep = (A, B)  # the plan refers to A and B
+        self._transA, self._transB = bool(transA), bool(transB)
         self.raw = imq_plan_info()  # the C struct; `info` is built from it on first use
         _check(lib().imq_plan_info_get(handle, ctypes.byref(self.raw)), "imq_plan_info_get")
         self._info = None
@@ -432,3 +441,99 @@ def imq_unpacked_gemm(plan: Plan, A, B, deltaA=None, gA=IMQ_PER_TENSOR, deltaB=N
 
 def imq_device_status(clear: bool = False, stream=None) -> int:
     return int(lib().imq_device_status(_stream(stream), int(clear)))
+
+
+# ------------------------------------------------------------------------------------------------
+# 4. batches of equal-shaped GEMMs
+# ------------------------------------------------------------------------------------------------
+class PlanBatch:
+    """The plans of one imq_plan_batched call (a list of Plan, problem h first at index h) and the
+    handle array the batched calls take."""
+
+    def __init__(self, plans, A, B):
+        self.plans = plans
+        self._keep = (A, B)
+        self.handles = (ctypes.c_void_p * len(plans))(*[p.handle for p in plans])
+
+    def __len__(self):
+        return len(self.plans)
+
+    def __getitem__(self, h):
+        return self.plans[h]
+
+    def workspace_layout(self):
+        """(offsets [(A' offset, B'^T offset)] per problem, total bytes) of imq_batch_workspace."""
+        n = len(self.plans)
+        off = (ctypes.c_size_t * (2 * n))()
+        tot = ctypes.c_size_t(0)
+        _check(lib().imq_batch_workspace(n, self.handles, off, ctypes.byref(tot)), "imq_batch_workspace")
+        return [(off[2 * h], off[2 * h + 1]) for h in range(n)], tot.value
+
+    def destroy(self):
+        for p in self.plans:
+            p.destroy()
+
+
+def imq_plan_batched(A: torch.Tensor, B: torch.Tensor, batch: int, M: int, K: int, N: int, b: int,
+                     strategy: int = IMQ_MIX, transA: bool = False, transB: bool = False, strideA=None,
+                     strideB=None, lda=None, ldb=None, maxes=None, stream=None) -> PlanBatch:
+    """Plans `batch` problems of one shape: problem h's A starts strideA elements after problem h-1's
+    (default: its stored rows times lda), likewise B; lda / ldb default to the tensors' row strides."""
+    if A.dtype != B.dtype:
+        raise ValueError("A and B must have the same integer dtype")
+    lda = _ld(A) if lda is None else lda
+    ldb = _ld(B) if ldb is None else ldb
+    strideA = (K if transA else M) * lda if strideA is None else strideA
+    strideB = (N if transB else K) * ldb if strideB is None else strideB
+    mx = [None] * 4 if maxes is None else list(maxes)
+    hs = (ctypes.c_void_p * batch)()
+    st = lib().imq_plan_batched(batch, _ptr(A), strideA, _ptr(B), strideB, _TORCH_TO_IMQ[A.dtype], M, K, N,
+                                int(transA), lda, int(transB), ldb, int(b), int(strategy), *[_ptr(m) for m in mx], hs,
+                                _stream(stream))
+    _check(st, "imq_plan_batched")
+    return PlanBatch([Plan(hs[h], A, B, transA, transB) for h in range(batch)], A, B)
+
+
+def batch_workspace(batch: PlanBatch, device=None) -> torch.Tensor:
+    _, tot = batch.workspace_layout()
+    return torch.empty(max(tot, 1) + 1024, dtype=torch.uint8, device=device or "cuda")
+
+
+def batch_views(batch: PlanBatch, workspace: torch.Tensor):
+    """[(A' view, B'^T view)] per problem in the batch workspace layout."""
+    offs, _ = batch.workspace_layout()
+    base = (-workspace.data_ptr()) % 1024
+    w8 = workspace.view(torch.int8) if workspace.dtype != torch.int8 else workspace
+    out = []
+    for (oa, ob), p in zip(offs, batch.plans):
+        r = p.raw
+        out.append((w8[base + oa:base + oa + r.M_unp * r.K_unp].view(r.M_unp, r.K_unp),
+                    w8[base + ob:base + ob + r.N_unp * r.K_unp].view(r.N_unp, r.K_unp)))
+    return out
+
+
+def imq_unpack_batched(batch: PlanBatch, A: torch.Tensor, B: torch.Tensor, workspace: torch.Tensor, strideA=None,
+                       strideB=None, stream=None):
+    r = batch.plans[0].raw
+    strideA = (r.K if batch.plans[0]._transA else r.M) * _ld(A) if strideA is None else strideA
+    strideB = (r.N if batch.plans[0]._transB else r.K) * _ld(B) if strideB is None else strideB
+    wp, wn = _aligned(workspace)
+    _check(lib().imq_unpack_batched(len(batch), batch.handles, _ptr(A), strideA, _ptr(B), strideB, wp, wn,
+                                    _stream(stream)), "imq_unpack_batched")
+
+
+def imq_gemm_unpacked_batched(batch: PlanBatch, workspace: torch.Tensor, deltaA, strideDA: int, gA: int, deltaB,
+                              strideDB: int, gB: int, C: torch.Tensor, Cf: torch.Tensor, strideC=None, strideCf=None,
+                              stream=None):
+    """C, Cf: (batch, M, N)-shaped (or any tensors with the given batch strides and unit column stride)."""
+    r = batch.plans[0].raw
+    ldc = C.stride(-2) if C is not None else r.N
+    ldcf = Cf.stride(-2) if Cf is not None else r.N
+    strideC = (C.stride(0) if C is not None else 0) if strideC is None else strideC
+    strideCf = (Cf.stride(0) if Cf is not None else 0) if strideCf is None else strideCf
+    wp, wn = _aligned(workspace)
+    st = lib().imq_gemm_unpacked_batched(len(batch), batch.handles, wp, wn, _ptr(deltaA), strideDA, gA, _ptr(deltaB),
+                                         strideDB, gB, _ptr(C), strideC,
+                                         _TORCH_TO_IMQ[C.dtype] if C is not None else IMQ_I32, ldc, _ptr(Cf), strideCf,
+                                         ldcf, _stream(stream))
+    _check(st, "imq_gemm_unpacked_batched")

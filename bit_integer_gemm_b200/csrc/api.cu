@@ -6,6 +6,7 @@
 #include <mutex>
 #include <tuple>
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -83,6 +84,47 @@ cudaError_t blocks_per_sm(const void* fn, int threads, size_t smem, int* out) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, threads, smem);
   if (e == cudaSuccess) cache[key] = *out;
   return e;
+}
+
+namespace {
+constexpr int kStageRing = 8;
+constexpr size_t kStageBytes = 256 * 1024;
+struct Staging {
+  void* buf[kStageRing] = {};
+  cudaEvent_t done[kStageRing] = {};
+  int next = 0;
+  std::mutex mu;
+};
+Staging g_staging[64];
+}  // namespace
+
+imq_status upload_table(const void* host, size_t bytes, void** dev, cudaStream_t st) {
+  *dev = nullptr;
+  if (bytes > kStageBytes) return IMQ_ERR_UNSUPPORTED;
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  int d = 0;
+  IMQ_CUDA_TRY(cudaGetDevice(&d));
+  Staging& sg = g_staging[d & 63];
+  std::lock_guard<std::mutex> lock(sg.mu);
+  const int k = sg.next;
+  sg.next = (k + 1) % kStageRing;
+  if (!sg.buf[k]) {
+    IMQ_CUDA_TRY(cudaMallocHost(&sg.buf[k], kStageBytes));
+    IMQ_CUDA_TRY(cudaEventCreateWithFlags(&sg.done[k], cudaEventDisableTiming));
+  } else {
+    IMQ_CUDA_TRY(cudaEventSynchronize(sg.done[k]));  // the buffer's previous upload has been read
+  }
+  IMQ_CUDA_TRY(cudaMallocFromPoolAsync(dev, bytes > 0 ? bytes : 16, ds->pool, st));
+  memcpy(sg.buf[k], host, bytes);
+  if (cudaMemcpyAsync(*dev, sg.buf[k], bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaEventRecord(sg.done[k], st) != cudaSuccess) {
+    cudaFreeAsync(*dev, st);
+    *dev = nullptr;
+    return IMQ_ERR_CUDA;
+  }
+  return IMQ_OK;
 }
 
 namespace {
@@ -349,6 +391,137 @@ imq_status imq_level_cover(const int32_t* maxima, int64_t n, int32_t b, int32_t 
                            imq_stream_t stream) {
   if (n < 0 || b < 2 || b > 8 || cap < 0 || (n > 0 && (!maxima || !out))) return IMQ_ERR_ARG;
   return imq::launch_level_cover(maxima, n, b, cap, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_plan_batched(int32_t batch, const void* A, int64_t strideA, const void* B, int64_t strideB, imq_dtype it,
+                            int64_t M, int64_t K, int64_t N, int32_t transA, int64_t lda, int32_t transB, int64_t ldb,
+                            int32_t b, imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                            const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** plans,
+                            imq_stream_t stream) {
+  if (!plans || batch < 0) return IMQ_ERR_ARG;
+  for (int32_t h = 0; h < batch; ++h) plans[h] = nullptr;
+  if (batch == 0) return IMQ_OK;
+  if (it != IMQ_I16 && it != IMQ_I32) return IMQ_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || b < 2 || b > 8 || strideA < 0 || strideB < 0) return IMQ_ERR_ARG;
+  if (M > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return IMQ_ERR_UNSUPPORTED;
+  if ((int)strategy < 0 || (int)strategy > (int)IMQ_HYBRID) return IMQ_ERR_ARG;
+  if ((transA != 0 && transA != 1) || (transB != 0 && transB != 1)) return IMQ_ERR_ARG;
+  if (lda < (transA ? M : K) || ldb < (transB ? K : N)) return IMQ_ERR_ARG;
+  if ((M > 0 && K > 0 && !A) || (K > 0 && N > 0 && !B)) return IMQ_ERR_ARG;
+  return imq::build_plans(batch, A, strideA, B, strideB, it, M, K, N, transA, lda, transB, ldb, b, strategy,
+                          a_rowmax, a_colmax, b_rowmax, b_colmax, plans, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+size_t align1k(size_t x) { return (x + 1023) / 1024 * 1024; }
+
+// The batch workspace: for each plan its A' then its B'^T, each from a 1024-byte boundary.
+imq_status batch_layout(int32_t batch, imq_plan_t* const* plans, size_t* offsets, size_t* total) {
+  if (batch < 0 || (batch > 0 && !plans)) return IMQ_ERR_ARG;
+  size_t off = 0;
+  for (int32_t h = 0; h < batch; ++h) {
+    if (!plans[h]) return IMQ_ERR_ARG;
+    const imq_plan_info& I = plans[h]->info;
+    if (offsets) offsets[2 * h] = off;
+    off += align1k((size_t)(I.M_unp * I.K_unp));
+    if (offsets) offsets[2 * h + 1] = off;
+    off += align1k((size_t)(I.N_unp * I.K_unp));
+  }
+  *total = off;
+  return IMQ_OK;
+}
+
+// Same device, same shapes, b, layouts and strategy: the plans of one imq_plan_batched call.
+bool same_batch(int32_t batch, imq_plan_t* const* plans) {
+  const imq_plan_t* p0 = plans[0];
+  for (int32_t h = 1; h < batch; ++h) {
+    const imq_plan_t* p = plans[h];
+    if (p->device != p0->device || p->it != p0->it || p->transA != p0->transA || p->transB != p0->transB ||
+        p->lda != p0->lda || p->ldb != p0->ldb || p->info.M != p0->info.M || p->info.K != p0->info.K ||
+        p->info.N != p0->info.N || p->info.b != p0->info.b)
+      return false;
+  }
+  return true;
+}
+}  // namespace
+
+imq_status imq_batch_workspace(int32_t batch, imq_plan_t* const* plans, size_t* offsets, size_t* total_bytes) {
+  if (!total_bytes) return IMQ_ERR_ARG;
+  return batch_layout(batch, plans, offsets, total_bytes);
+}
+
+imq_status imq_unpack_batched(int32_t batch, imq_plan_t* const* plans, const void* A, int64_t strideA, const void* B,
+                              int64_t strideB, void* workspace, size_t workspace_bytes, imq_stream_t stream) {
+  if (batch == 0) return IMQ_OK;
+  size_t total = 0;
+  std::vector<size_t> off((size_t)batch * 2);
+  imq_status s = batch_layout(batch, plans, off.data(), &total);
+  if (s != IMQ_OK) return s;
+  if (!same_batch(batch, plans)) return IMQ_ERR_ARG;
+  if (workspace_bytes < total) return IMQ_ERR_BUFFER;
+  if (total > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 1023))) return IMQ_ERR_ARG;
+  if (strideA < 0 || strideB < 0) return IMQ_ERR_ARG;
+  const imq_plan_info& I0 = plans[0]->info;
+  if ((I0.M > 0 && I0.K > 0 && !A) || (I0.K > 0 && I0.N > 0 && !B)) return IMQ_ERR_ARG;
+  const size_t esz = plans[0]->it == IMQ_I16 ? 2 : 4;
+  std::vector<const void*> pa((size_t)batch), pb((size_t)batch);
+  std::vector<int8_t*> wa((size_t)batch), wb((size_t)batch);
+  for (int32_t h = 0; h < batch; ++h) {
+    pa[h] = static_cast<const char*>(A) + (size_t)h * strideA * esz;
+    pb[h] = static_cast<const char*>(B) + (size_t)h * strideB * esz;
+    wa[h] = static_cast<int8_t*>(workspace) + off[2 * h];
+    wb[h] = static_cast<int8_t*>(workspace) + off[2 * h + 1];
+  }
+  int dev = 0;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != plans[0]->device) return IMQ_ERR_ARG;
+  return imq::launch_unpack_batch(plans, batch, pa.data(), pb.data(), wa.data(), wb.data(),
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_gemm_unpacked_batched(int32_t batch, imq_plan_t* const* plans, const void* workspace,
+                                     size_t workspace_bytes, const float* deltaA, int64_t strideDA, imq_gran gA,
+                                     const float* deltaB, int64_t strideDB, imq_gran gB, void* Cint, int64_t strideC,
+                                     imq_dtype ct, int64_t ldc, float* Cf, int64_t strideCf, int64_t ldcf,
+                                     imq_stream_t stream) {
+  if (batch == 0) return IMQ_OK;
+  size_t total = 0;
+  std::vector<size_t> off((size_t)batch * 2);
+  imq_status s = batch_layout(batch, plans, off.data(), &total);
+  if (s != IMQ_OK) return s;
+  if (!same_batch(batch, plans)) return IMQ_ERR_ARG;
+  if (workspace_bytes < total) return IMQ_ERR_BUFFER;
+  if (total > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 1023))) return IMQ_ERR_ARG;
+  if (strideDA < 0 || strideDB < 0 || strideC < 0 || strideCf < 0) return IMQ_ERR_ARG;
+  const size_t csz = ct == IMQ_I64 ? 8 : 4;
+  std::vector<imq::GemmSpec> specs((size_t)batch);
+  for (int32_t h = 0; h < batch; ++h) {
+    imq::GemmSpec& g = specs[h];
+    g.plan = plans[h];
+    g.Au = static_cast<const int8_t*>(workspace) + off[2 * h];
+    g.Bu = static_cast<const int8_t*>(workspace) + off[2 * h + 1];
+    g.dA = deltaA ? deltaA + (size_t)h * strideDA : nullptr;
+    g.gA = gA;
+    g.dB = deltaB ? deltaB + (size_t)h * strideDB : nullptr;
+    g.gB = gB;
+    g.C = Cint ? static_cast<char*>(Cint) + (size_t)h * strideC * csz : nullptr;
+    g.ct = ct;
+    g.ldc = ldc;
+    g.Cf = Cf ? Cf + (size_t)h * strideCf : nullptr;
+    g.ldcf = ldcf;
+  }
+  return imq::launch_gemm_multi(specs.data(), batch, reinterpret_cast<cudaStream_t>(stream));
+}
+
+imq_status imq_unpacked_gemm_batched(int32_t batch, imq_plan_t* const* plans, const void* A, int64_t strideA,
+                                     const void* B, int64_t strideB, const float* deltaA, int64_t strideDA,
+                                     imq_gran gA, const float* deltaB, int64_t strideDB, imq_gran gB, void* Cint,
+                                     int64_t strideC, imq_dtype ct, int64_t ldc, float* Cf, int64_t strideCf,
+                                     int64_t ldcf, void* workspace, size_t workspace_bytes, imq_stream_t stream) {
+  imq_status s = imq_unpack_batched(batch, plans, A, strideA, B, strideB, workspace, workspace_bytes, stream);
+  if (s != IMQ_OK) return s;
+  return imq_gemm_unpacked_batched(batch, plans, workspace, workspace_bytes, deltaA, strideDA, gA, deltaB, strideDB,
+                                   gB, Cint, strideC, ct, ldc, Cf, strideCf, ldcf, stream);
 }
 
 imq_status imq_check_bounded_wait(uint64_t timeout_ns, imq_stream_t stream) {

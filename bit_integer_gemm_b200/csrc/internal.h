@@ -31,6 +31,10 @@ cudaError_t ensure_smem(const void* fn, size_t bytes);
 // Resident blocks per SM of kernel fn at this block size and dynamic shared memory (the occupancy
 // query, cached per device, kernel and configuration).
 cudaError_t blocks_per_sm(const void* fn, int threads, size_t smem, int* out);
+// Copies a small host table to new device memory from the library's pool, through pinned staging (a
+// ring of buffers, each reused once its previous upload has completed), in stream order on `st`.  The
+// caller frees *dev with cudaFreeAsync on `st` after the kernels that read it.
+imq_status upload_table(const void* host, size_t bytes, void** dev, cudaStream_t st);
 // out[i] = max over p < nparts of part[p * n + i] (int32, non-negative); nparts may be 0 (out = 0).
 imq_status launch_reduce_max(const int32_t* part, int64_t nparts, int64_t n, int32_t* out, cudaStream_t st);
 
@@ -112,9 +116,34 @@ imq_status launch_rtn_quantize_unpack(const imq_plan_t* pl, const void* X, imq_d
                                       int32_t beta, int8_t* A_unp, float* delta, cudaStream_t stream);
 imq_status launch_unpack(const imq_plan_t* pl, const void* A, const void* B, int8_t* Au, int8_t* Bu,
                          cudaStream_t stream);
+// The unpack of n plans made together (imq_plan_batched): as few launches as their kernels allow.
+imq_status launch_unpack_batch(const imq_plan_t* const* pls, int n, const void* const* A, const void* const* B,
+                               int8_t* const* Au, int8_t* const* Bu, cudaStream_t stream);
+// Plans of `batch` equal-shaped problems with one host round trip (plan.cu).
+imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B, int64_t strideB, imq_dtype it,
+                       int64_t M, int64_t K, int64_t N, int32_t transA, int64_t lda, int32_t transB, int64_t ldb,
+                       int32_t b, imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                       const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out, cudaStream_t st);
 imq_status launch_gemm(const imq_plan_t* pl, const int8_t* Au, const int8_t* Bu, const float* dA,
                        imq_gran gA, const float* dB, imq_gran gB, void* C, imq_dtype ct,
                        int64_t ldc, float* Cf, int64_t ldcf, cudaStream_t stream);
+// One GEMM problem: a plan, its unpacked operands, scales and outputs (the arguments of imq_gemm_unpacked).
+struct GemmSpec {
+  const imq_plan_t* plan;
+  const int8_t* Au;
+  const int8_t* Bu;
+  const float* dA;
+  imq_gran gA;
+  const float* dB;
+  imq_gran gB;
+  void* C;
+  imq_dtype ct;
+  int64_t ldc;
+  float* Cf;
+  int64_t ldcf;
+};
+// The GEMMs of n problems in as few launches as the problem table allows (gemm.cu).
+imq_status launch_gemm_multi(const GemmSpec* specs, int n, cudaStream_t stream);
 }  // namespace imq
 
 #define IMQ_CUDA_TRY(expr)                                    \

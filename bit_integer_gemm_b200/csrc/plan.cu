@@ -21,6 +21,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -797,8 +798,9 @@ __global__ void __launch_bounds__(1024) k_plan_maps(const __grid_constant__ Maps
 // host side
 // ------------------------------------------------------------------------------------------------
 struct Pinned {
-  HostSummary* sum = nullptr;   // mapped pinned memory
-  HostSummary* sum_dev = nullptr;  // its device address
+  HostSummary* sum = nullptr;   // mapped pinned memory: `cap` summary slots, one per plan of a batch
+  HostSummary* sum_dev = nullptr;  // their device address
+  int cap = 0;
   uint32_t seq = 0;
   void* tables = nullptr;          // staging of the segment and class tables for their upload
   cudaEvent_t tables_done = nullptr;  // recorded after the last upload from `tables`
@@ -858,32 +860,77 @@ imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t co
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
-// Builds a plan; see imq_plan in include/imq.h.
-imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
-                      int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
-                      imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
-                      const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out,
-                      cudaStream_t st) {
-  DeviceState* ds;
-  imq_status s = device_state(&ds);
-  if (s != IMQ_OK) return s;
-  int dev;
-  IMQ_CUDA_TRY(cudaGetDevice(&dev));
-  Pinned& pin = g_pinned[dev & 63];
-  std::lock_guard<std::mutex> lock(pin.mu);
-  const size_t tables_bytes =
-      sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
-  // staging in the device layout: segments, classes and groups, each padded to 256 bytes
+// One plan in the making: its arguments and what its first stage leaves for the second.
+struct PlanJob {
+  const void* A;
+  const void* B;
+  imq_dtype it;
+  int64_t M, K, N;
+  int32_t transA;
+  int64_t lda;
+  int32_t transB;
+  int64_t ldb;
+  int32_t b;
+  imq_strategy strategy;
+  const int32_t* a_rowmax;
+  const int32_t* a_colmax;
+  const int32_t* b_rowmax;
+  const int32_t* b_colmax;
+  int slot;  // summary slot of the batch
+  // state after plan_begin
+  imq_plan_t* pl = nullptr;
+  char* blk1 = nullptr;
+  Summary* dsum = nullptr;
+  size_t o_segs = 0, o_cls = 0, o_grps = 0;
+  uint32_t seq = 0;
+};
+
+// Frees a plan that failed before it was returned.
+imq_status plan_fail(imq_plan_t* pl, imq_status e, cudaStream_t st) {
+  if (!pl) return e;
+  if (pl->dev_block) cudaFreeAsync(pl->dev_block, st);
+  if (pl->dev_block2) cudaFreeAsync(pl->dev_block2, st);
+  free(pl->host_tables);
+  delete pl;
+  return e;
+}
+
+// Makes sure the pinned summary slots and table staging of this device exist (nslots slots).
+imq_status pinned_ready(Pinned& pin, int nslots) {
   const size_t staging_bytes = align_up(sizeof(InnerSeg) * kLv * kLv, 256) +
                                align_up(sizeof(OuterClass) * 2 * kLv, 256) + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
-  if (!pin.sum) {
-    IMQ_CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&pin.sum), sizeof(HostSummary), cudaHostAllocMapped));
+  if (pin.cap < nslots) {
+    // every earlier plan has read its summary before returning, so the old slots are idle
+    if (pin.sum) cudaFreeHost(pin.sum);
+    pin.sum = nullptr;
+    pin.cap = 0;
+    const int cap = nslots < 16 ? 16 : nslots;
+    IMQ_CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&pin.sum), sizeof(HostSummary) * (size_t)cap,
+                               cudaHostAllocMapped));
     IMQ_CUDA_TRY(cudaHostGetDevicePointer(reinterpret_cast<void**>(&pin.sum_dev), pin.sum, 0));
-    pin.sum->seq = 0;
+    for (int i = 0; i < cap; ++i) pin.sum[i].seq = 0;
+    pin.cap = cap;
   }
   if (!pin.tables) IMQ_CUDA_TRY(cudaMallocHost(&pin.tables, staging_bytes));
   if (!pin.tables_done) IMQ_CUDA_TRY(cudaEventCreateWithFlags(&pin.tables_done, cudaEventDisableTiming));
+  return IMQ_OK;
+}
 
+// Stage 1 of a plan: line maxima (unless given), the hybrid's choice, the level kernel, which writes the
+// plan's summary into summary slot j.slot.  Nothing is waited for.
+imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaStream_t st) {
+  const void* A = job.A;
+  const void* B = job.B;
+  const imq_dtype it = job.it;
+  const int64_t M = job.M, K = job.K, N = job.N;
+  const int32_t transA = job.transA, transB = job.transB;
+  const int64_t lda = job.lda, ldb = job.ldb;
+  const int32_t b = job.b;
+  const imq_strategy strategy = job.strategy;
+  const int32_t *a_rowmax = job.a_rowmax, *a_colmax = job.a_colmax, *b_rowmax = job.b_rowmax,
+                *b_colmax = job.b_colmax;
+  const size_t tables_bytes =
+      sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
   imq_plan_t* pl = new imq_plan_t;
   memset(pl, 0, sizeof(*pl));
   pl->host_tables = malloc(tables_bytes);
@@ -891,9 +938,6 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     delete pl;
     return IMQ_ERR_CUDA;
   }
-  InnerSeg* hsegs = static_cast<InnerSeg*>(pl->host_tables);
-  OuterClass* hcls = reinterpret_cast<OuterClass*>(hsegs + kLv * kLv);
-  InnerGroup* hgrps = reinterpret_cast<InnerGroup*>(hcls + 2 * kLv);
   pl->device = dev;
   pl->A = A;
   pl->B = B;
@@ -968,13 +1012,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   pl->lv_b_col = reinterpret_cast<int8_t*>(blk1 + o_lv[3]);
   Summary* dsum = reinterpret_cast<Summary*>(blk1 + o_sum);
 
-  auto fail = [&](imq_status e) {
-    cudaFreeAsync(pl->dev_block, st);
-    if (pl->dev_block2) cudaFreeAsync(pl->dev_block2, st);
-    free(pl->host_tables);
-    delete pl;
-    return e;
-  };
+  auto fail = [&](imq_status e) { return plan_fail(pl, e, st); };
 
   const bool have_max = a_rowmax && a_colmax && b_rowmax && b_colmax;
   const int32_t* lmx[4] = {mx[0], mx[1], mx[2], mx[3]};  // the maxima the levels are computed from
@@ -1086,7 +1124,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   la.lv[3] = pl->lv_b_col;
   la.bm1 = b - 1;
   la.sum = dsum;
-  la.hsum = pin.sum_dev;
+  la.hsum = pin.sum_dev + job.slot;
   la.seq = ++pin.seq;
   {
     const int64_t nmax = (M > K ? M : K) > N ? (M > K ? M : K) : N;
@@ -1096,31 +1134,69 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
     k_levels<<<(unsigned)grid, 256, 0, st>>>(la);
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  job.pl = pl;
+  job.blk1 = blk1;
+  job.dsum = dsum;
+  job.o_segs = o_segs;
+  job.o_cls = o_cls;
+  job.o_grps = o_grps;
+  job.seq = la.seq;
+  return IMQ_OK;
+}
+
+// Waits for the summary of a plan whose stage 1 is queued on `st`, and copies it to *out.
+imq_status plan_wait(PlanJob& job, Pinned& pin, cudaStream_t st, Summary* out) {
+  imq_plan_t* pl = job.pl;
+  auto fail = [&](imq_status e) {
+    job.pl = nullptr;
+    return plan_fail(pl, e, st);
+  };
+  HostSummary* hs = pin.sum + job.slot;
+  const Summary* dsum = job.dsum;
   // wait for the summary: spin on its sequence number, asking the stream every few thousand polls
   // whether it is still running (an error there is returned; a finished stream without the number, which
   // a launch failure could leave, falls back to a plain copy of the device summary)
   {
-    const volatile uint32_t* seqp = &pin.sum->seq;
+    const volatile uint32_t* seqp = &hs->seq;
     bool have = false;
     for (uint64_t it = 1;; ++it) {
-      if (*seqp == la.seq) {
+      if (*seqp == job.seq) {
         have = true;
         break;
       }
       if ((it & 4095) == 0) {
         const cudaError_t q = cudaStreamQuery(st);
         if (q == cudaSuccess) {
-          have = *seqp == la.seq;
+          have = *seqp == job.seq;
           break;
         }
         if (q != cudaErrorNotReady) return fail(IMQ_ERR_CUDA);
       }
     }
     std::atomic_thread_fence(std::memory_order_acquire);
-    if (!have && (cudaMemcpy(&pin.sum->s, dsum, sizeof(Summary), cudaMemcpyDeviceToHost) != cudaSuccess))
+    if (!have && (cudaMemcpy(&hs->s, dsum, sizeof(Summary), cudaMemcpyDeviceToHost) != cudaSuccess))
       return fail(IMQ_ERR_CUDA);
   }
-  const Summary S = pin.sum->s;
+  *out = hs->s;
+  return IMQ_OK;
+}
+
+// Stage 2 of a plan: the host decisions from its summary, then the maps kernel.  *out gets the plan.
+imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState* ds, cudaStream_t st,
+                       imq_plan_t** out) {
+  imq_plan_t* pl = job.pl;
+  job.pl = nullptr;
+  auto fail = [&](imq_status e) { return plan_fail(pl, e, st); };
+  const int64_t M = job.M, K = job.K, N = job.N;
+  const int32_t b = job.b;
+  const imq_strategy strategy = job.strategy;
+  const int64_t nvec[4] = {M, K, K, N};
+  imq_plan_info& I = pl->info;
+  InnerSeg* hsegs = static_cast<InnerSeg*>(pl->host_tables);
+  OuterClass* hcls = reinterpret_cast<OuterClass*>(hsegs + kLv * kLv);
+  InnerGroup* hgrps = reinterpret_cast<InnerGroup*>(hcls + 2 * kLv);
+  char* blk1 = job.blk1;
+  const size_t o_segs = job.o_segs, o_cls = job.o_cls, o_grps = job.o_grps;
   // a pending kernel error (e.g. a non-finite quantiser input) is reported before planning
   if (S.status != IMQ_OK) return fail((imq_status)S.status);
 
@@ -1374,7 +1450,7 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   if (cudaMallocFromPoolAsync((void**)&b2, off2 > 0 ? off2 : 256, ds->pool, st) != cudaSuccess)
     return fail(IMQ_ERR_CUDA);
   pl->dev_block2 = b2;
-  pl->dev_bytes = stage1 + off2;
+  pl->dev_bytes += off2;
   InnerSeg* dsegs = reinterpret_cast<InnerSeg*>(blk1 + o_segs);
   OuterClass* dcls = reinterpret_cast<OuterClass*>(blk1 + o_cls);
   pl->tK = reinterpret_cast<int32_t*>(b2 + o_tK);
@@ -1435,6 +1511,88 @@ imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
   *out = pl;
+  return IMQ_OK;
+}
+
+imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B, int64_t strideB, imq_dtype it,
+                       int64_t M, int64_t K, int64_t N, int32_t transA, int64_t lda, int32_t transB, int64_t ldb,
+                       int32_t b, imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                       const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out, cudaStream_t st);
+
+// Builds a plan; see imq_plan in include/imq.h.
+imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
+                      int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
+                      imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                      const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out,
+                      cudaStream_t st) {
+  const int64_t sa = 0, sb = 0;
+  return build_plans(1, A, sa, B, sb, it, M, K, N, transA, lda, transB, ldb, b, strategy, a_rowmax, a_colmax,
+                     b_rowmax, b_colmax, out, st);
+}
+
+// Plans of `batch` equal-shaped problems: problem h reads A + h * strideA, B + h * strideB (elements)
+// and the maxima vectors at h times their lengths.  Every stage 1 is queued first, then the summaries
+// are waited for together, then every stage 2 runs: one host round trip for the whole batch.
+imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B, int64_t strideB, imq_dtype it,
+                       int64_t M, int64_t K, int64_t N, int32_t transA, int64_t lda, int32_t transB, int64_t ldb,
+                       int32_t b, imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
+                       const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out, cudaStream_t st) {
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  int dev;
+  IMQ_CUDA_TRY(cudaGetDevice(&dev));
+  Pinned& pin = g_pinned[dev & 63];
+  std::lock_guard<std::mutex> lock(pin.mu);
+  s = pinned_ready(pin, batch);
+  if (s != IMQ_OK) return s;
+  const size_t esz = it == IMQ_I16 ? 2 : 4;
+  const bool have_max = a_rowmax && a_colmax && b_rowmax && b_colmax;
+  std::vector<PlanJob> jobs((size_t)batch);
+  for (int h = 0; h < batch; ++h) out[h] = nullptr;
+  auto drop = [&](int upto, imq_status e) {
+    // level kernels already queued write into the pinned summary slots: let them finish first
+    cudaStreamSynchronize(st);
+    for (int h = 0; h < upto; ++h)
+      if (jobs[h].pl) plan_fail(jobs[h].pl, e, st);
+    for (int h = 0; h < batch; ++h)
+      if (out[h]) {
+        imq_plan_destroy(out[h]);
+        out[h] = nullptr;
+      }
+    return e;
+  };
+  for (int h = 0; h < batch; ++h) {
+    PlanJob& j = jobs[h];
+    j.A = static_cast<const char*>(A) + (size_t)h * strideA * esz;
+    j.B = static_cast<const char*>(B) + (size_t)h * strideB * esz;
+    j.it = it;
+    j.M = M;
+    j.K = K;
+    j.N = N;
+    j.transA = transA;
+    j.lda = lda;
+    j.transB = transB;
+    j.ldb = ldb;
+    j.b = b;
+    j.strategy = strategy;
+    j.a_rowmax = have_max ? a_rowmax + (size_t)h * M : nullptr;
+    j.a_colmax = have_max ? a_colmax + (size_t)h * K : nullptr;
+    j.b_rowmax = have_max ? b_rowmax + (size_t)h * K : nullptr;
+    j.b_colmax = have_max ? b_colmax + (size_t)h * N : nullptr;
+    j.slot = h;
+    s = plan_begin(j, pin, ds, dev, st);
+    if (s != IMQ_OK) return drop(h, s);
+  }
+  std::vector<Summary> sums((size_t)batch);
+  for (int h = 0; h < batch; ++h) {
+    s = plan_wait(jobs[h], pin, st, &sums[h]);
+    if (s != IMQ_OK) return drop(batch, s);
+  }
+  for (int h = 0; h < batch; ++h) {
+    s = plan_finish(jobs[h], sums[h], pin, ds, st, &out[h]);
+    if (s != IMQ_OK) return drop(batch, s);
+  }
   return IMQ_OK;
 }
 

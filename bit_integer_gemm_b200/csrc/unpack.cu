@@ -25,6 +25,8 @@
 //                  and writing 128-byte segments of unpacked lines.
 // HBM traffic: each source entry is read once (the gathered rows are L2-resident), each unpacked byte
 // is written once.
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -244,14 +246,45 @@ __device__ __forceinline__ void digit_planes_i16(const int16_t* __restrict__ xr,
 // memory latency.
 constexpr int64_t kMetaMaxChunks = 4096;
 
+// What differs between the problems of a batched unpack launch (blockIdx.y = problem): the source, the
+// plan's maps and the destination.  A single-problem launch passes no table and its own arguments.
+struct LineJob {
+  const void* X;
+  int outer;
+  const int8_t* lvl;
+  const int32_t* pos;
+  const int32_t* tK;
+  const int8_t* lk;
+  const int32_t* blk16;
+  int64_t K_unp;
+  int8_t* out;
+  const int32_t* grpL;
+  const int32_t* grpN;
+  int64_t ngrp;
+};
+// The same bound for the int16 staged-line kernel below (its chunk index is an int).
+constexpr int64_t kMetaMaxChunks16 = 32768;
+
 template <typename T>
-__global__ void __launch_bounds__(256) k_unpack_lines(const T* __restrict__ X, int64_t nlines, int64_t K,
+__global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines, int64_t K,
                                                       int64_t ld, int P, int nwarps, int outer,
-                                                      const int8_t* __restrict__ lvl, const int32_t* __restrict__ pos,
-                                                      const int32_t* __restrict__ tK, const int8_t* __restrict__ lk,
-                                                      const int32_t* __restrict__ blk16, int64_t K_unp, int bm1,
-                                                      int meta_smem, int8_t* __restrict__ out) {
+                                                      const int8_t* lvl, const int32_t* pos,
+                                                      const int32_t* tK, const int8_t* lk,
+                                                      const int32_t* blk16, int64_t K_unp, int bm1,
+                                                      int meta_smem, int8_t* out, const LineJob* __restrict__ jobs) {
   extern __shared__ __align__(16) unsigned char dsm[];
+  if (jobs) {
+    const LineJob& jb = jobs[blockIdx.y];
+    X = static_cast<const T*>(jb.X);
+    outer = jb.outer;
+    lvl = jb.lvl;
+    pos = jb.pos;
+    tK = jb.tK;
+    lk = jb.lk;
+    blk16 = jb.blk16;
+    K_unp = jb.K_unp;
+    out = jb.out;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t Kp = (K + 15) / 16 * 16;  // plane row length, 16-byte aligned
   const int64_t nchunk = K_unp / 16;
@@ -406,17 +439,28 @@ constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take th
 // OUTER groups dealt to it (group g to CTA g mod gridDim.x), lines n*L .. G-1 of a group of n sources of
 // level L, which no source line writes.
 template <int kBm1>
-__global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* __restrict__ X, int64_t nlines, int64_t K,
-                                                           int64_t ld, int nwarps, int outer,
-                                                           const int8_t* __restrict__ lvl,
-                                                           const int32_t* __restrict__ pos,
-                                                           const int32_t* __restrict__ tK,
-                                                           const int8_t* __restrict__ lk,
-                                                           const int32_t* __restrict__ blk16, int64_t K_unp,
-                                                           int8_t* __restrict__ out,
-                                                           const int32_t* __restrict__ grpL,
-                                                           const int32_t* __restrict__ grpN, int64_t ngrp, int G) {
+__global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int64_t nlines, int64_t K,
+                                                           int64_t ld, int nwarps, int outer, const int8_t* lvl,
+                                                           const int32_t* pos, const int32_t* tK, const int8_t* lk,
+                                                           const int32_t* blk16, int64_t K_unp, int8_t* out,
+                                                           const int32_t* grpL, const int32_t* grpN, int64_t ngrp,
+                                                           int G, const LineJob* __restrict__ jobs) {
   extern __shared__ __align__(16) unsigned char dsm[];
+  if (jobs) {
+    const LineJob& jb = jobs[blockIdx.y];
+    X = static_cast<const int16_t*>(jb.X);
+    outer = jb.outer;
+    lvl = jb.lvl;
+    pos = jb.pos;
+    tK = jb.tK;
+    lk = jb.lk;
+    blk16 = jb.blk16;
+    K_unp = jb.K_unp;
+    out = jb.out;
+    grpL = jb.grpL;
+    grpN = jb.grpN;
+    ngrp = jb.ngrp;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t Kr = (K + 15) / 16 * 16;  // staged line length in entries (32-byte multiple)
   const int nchunk = (int)(K_unp / 16);
@@ -540,20 +584,23 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* __rest
   }
 }
 
+// nprob > 1: `jobs` (device) holds the per-problem arguments and the ones given here are ignored.
 template <int kBm1>
 imq_status launch_lines16(const int16_t* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
                           const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
                           const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL, const int32_t* grpN,
-                          int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st) {
+                          int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs = nullptr,
+                          int nprob = 1) {
   auto kern = k_unpack_lines16<kBm1>;
   IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   int per_sm = 0;
   IMQ_CUDA_TRY(blocks_per_sm(reinterpret_cast<const void*>(kern), 256, smem, &per_sm));
   if (per_sm < 1) per_sm = 1;
-  int64_t grid = (int64_t)num_sms * per_sm;
+  // every resident slot once over the whole batch
+  int64_t grid = ((int64_t)num_sms * per_sm + nprob - 1) / nprob;
   if (grid > nlines) grid = nlines;
-  kern<<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN,
-                                          ngrp, G);
+  kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16,
+                                                                 K_unp, out, grpL, grpN, ngrp, G, jobs);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
@@ -674,7 +721,8 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
     if (nw < 1) nw = (int)((192 * 1024) / (Kr * 2)) >= 1 ? 1 : 0;
     if (nw > 8) nw = 8;
     const size_t smem = (size_t)nw * Kr * 2 + (size_t)nchunk * 5;
-    if (line_is_row && nw >= 1 && nchunk <= kMetaMaxChunks && smem <= 200 * 1024 && bm1 >= 1 && bm1 <= 7) {
+    // the block metadata (5 bytes per 16 positions) is staged whole; the shared-memory budget bounds it
+    if (line_is_row && nw >= 1 && nchunk <= kMetaMaxChunks16 && smem <= 200 * 1024 && bm1 >= 1 && bm1 <= 7) {
       const int16_t* X16 = reinterpret_cast<const int16_t*>(X);
       const int64_t ng = outer ? zj.ngrp : 0;
       imq_status s;
@@ -710,7 +758,7 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
         if (grid > ctas) grid = ctas;
         IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
         k_unpack_lines<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, P, nw, outer, lvl, pos, tK, lk, blk16,
-                                                             K_unp, bm1, meta_smem, out);
+                                                             K_unp, bm1, meta_smem, out, nullptr);
         return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
       }
     }
@@ -778,6 +826,123 @@ imq_status unpack_typed(const imq_plan_t* pl, const T* A, const T* B, int8_t* Au
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
+
+// One operand side (A when side == 0, else B) of a batch of plans made together (equal shapes, layouts
+// and b): one launch for the whole batch when every problem takes the staged int16 kernel or the digit-
+// plane kernel, else one unpack per problem.
+template <typename T>
+imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* const* src, int8_t* const* dst,
+                             int side, int num_sms, cudaStream_t st) {
+  const imq_plan_t* p0 = pls[0];
+  const imq_plan_info& I0 = p0->info;
+  const int bm1 = I0.b - 1;
+  const int64_t K = I0.K;
+  const int64_t nlines = side == 0 ? I0.M : I0.N;
+  const int64_t ld = side == 0 ? p0->lda : p0->ldb;
+  const bool line_is_row = side == 0 ? !p0->transA : p0->transB != 0;
+  int64_t nchunk = 0;
+  int P = 1;
+  std::vector<LineJob> jobs((size_t)n);
+  for (int h = 0; h < n; ++h) {
+    const imq_plan_t* pl = pls[h];
+    const imq_plan_info& I = pl->info;
+    const int dir = side == 0 ? I.dir_a : I.dir_b;
+    const int outer = (dir & IMQ_DIR_OUTER) != 0, inner = (dir & IMQ_DIR_INNER) != 0;
+    const int po = outer ? (side == 0 ? I.lmax_a_row : I.lmax_b_col) : 1;
+    const int pi = inner ? (side == 0 ? I.lmax_a_col : I.lmax_b_row) : 1;
+    P = P > po ? P : po;
+    P = P > pi ? P : pi;
+    nchunk = nchunk > I.K_unp / 16 ? nchunk : I.K_unp / 16;
+    LineJob& j = jobs[h];
+    j.X = src[h];
+    j.outer = outer;
+    j.lvl = side == 0 ? pl->lv_a_row : pl->lv_b_col;
+    j.pos = side == 0 ? pl->posA : pl->posB;
+    j.tK = pl->tK;
+    j.lk = side == 0 ? pl->lAk : pl->lBk;
+    j.blk16 = pl->blk16;
+    j.K_unp = I.K_unp;
+    j.out = dst[h];
+    j.grpL = outer ? (side == 0 ? pl->grpA_L : pl->grpB_L) : nullptr;
+    j.grpN = outer ? (side == 0 ? pl->grpA_n : pl->grpB_n) : nullptr;
+    j.ngrp = outer ? (side == 0 ? pl->n_grp_a : pl->n_grp_b) : 0;
+    if (I.b != I0.b || I.K != K || I.M != I0.M || I.N != I0.N) return IMQ_ERR_ARG;
+  }
+  if (nlines == 0 || nchunk == 0) return IMQ_OK;
+  void* dj = nullptr;
+  imq_status s = IMQ_OK;
+  if (sizeof(T) == 2 && line_is_row && bm1 >= 1 && bm1 <= 7) {
+    const int64_t Kr = (K + 15) / 16 * 16;
+    int nw = (int)((64 * 1024) / (Kr * 2));
+    if (nw < 1) nw = (int)((192 * 1024) / (Kr * 2)) >= 1 ? 1 : 0;
+    if (nw > 8) nw = 8;
+    const size_t smem = (size_t)nw * Kr * 2 + (size_t)nchunk * 5;
+    if (nw >= 1 && nchunk <= kMetaMaxChunks16 && smem <= 200 * 1024) {
+      s = upload_table(jobs.data(), sizeof(LineJob) * (size_t)n, &dj, st);
+      if (s != IMQ_OK) return s;
+      const int16_t* X0 = static_cast<const int16_t*>(src[0]);
+      const LineJob* J = static_cast<const LineJob*>(dj);
+      const int G = side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP;
+      switch (bm1) {
+        case 1: s = launch_lines16<1>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+        case 2: s = launch_lines16<2>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+        case 3: s = launch_lines16<3>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+        case 4: s = launch_lines16<4>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+        case 5: s = launch_lines16<5>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+        case 6: s = launch_lines16<6>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+        default: s = launch_lines16<7>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
+      }
+      cudaFreeAsync(dj, st);
+      return s;
+    }
+  }
+  if (line_is_row) {
+    const int64_t Kp = (K + 15) / 16 * 16;
+    const int64_t per_warp = (int64_t)P * Kp;
+    int nw = (int)((96 * 1024) / per_warp);
+    if (nw > 8) nw = 8;
+    if (nw >= 1) {
+      const int meta_smem = nchunk <= kMetaMaxChunks ? 1 : 0;
+      const size_t smem = (size_t)nw * per_warp + (meta_smem ? (size_t)nchunk * 5 : 0);
+      const int per_sm = (int)((200 * 1024) / (smem + 1024)) < 1 ? 1 : (int)((200 * 1024) / (smem + 1024));
+      const int64_t ctas = (nlines + nw - 1) / nw;
+      int64_t grid = ((int64_t)num_sms * (per_sm > 8 ? 8 : per_sm) + n - 1) / n;
+      if (grid > ctas) grid = ctas;
+      s = upload_table(jobs.data(), sizeof(LineJob) * (size_t)n, &dj, st);
+      if (s != IMQ_OK) return s;
+      IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
+      k_unpack_lines<T><<<dim3((unsigned)grid, (unsigned)n), 256, smem, st>>>(
+          static_cast<const T*>(src[0]), nlines, K, ld, P, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, bm1,
+          meta_smem, nullptr, static_cast<const LineJob*>(dj));
+      s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+      cudaFreeAsync(dj, st);
+      if (s != IMQ_OK) return s;
+      // this kernel does not zero the unused lines of OUTER groups
+      for (int h = 0; h < n; ++h)
+        if (jobs[h].outer && jobs[h].ngrp > 0)
+          k_zero_unused<<<(unsigned)(jobs[h].ngrp < 4096 ? jobs[h].ngrp : 4096), 256, 0, st>>>(
+              jobs[h].grpL, jobs[h].grpN, jobs[h].ngrp, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP, jobs[h].K_unp,
+              jobs[h].out);
+      return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+    }
+  }
+  // anything else: problem by problem
+  for (int h = 0; h < n; ++h) {
+    const imq_plan_t* pl = pls[h];
+    const LineJob& j = jobs[h];
+    ZeroJob zj;
+    if (j.outer) zj = ZeroJob{j.grpL, j.grpN, j.ngrp, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP};
+    bool zeroed = false;
+    s = unpack_one<T>(static_cast<const T*>(j.X), nlines, K, ld, line_is_row, j.outer, P, j.lvl, j.pos, pl->tK, j.lk,
+                      pl->blk16, j.K_unp, bm1, j.out, num_sms, st, zj, &zeroed);
+    if (s != IMQ_OK) return s;
+    if (j.outer && j.ngrp > 0 && !zeroed && j.K_unp > 0)
+      k_zero_unused<<<(unsigned)(j.ngrp < 4096 ? j.ngrp : 4096), 256, 0, st>>>(j.grpL, j.grpN, j.ngrp, zj.G, j.K_unp,
+                                                                               j.out);
+  }
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
 }  // namespace
 
 imq_status launch_unpack(const imq_plan_t* pl, const void* A, const void* B, int8_t* Au, int8_t* Bu,
@@ -792,4 +957,22 @@ imq_status launch_unpack(const imq_plan_t* pl, const void* A, const void* B, int
                                ds->num_sms, st);
 }
 
+}  // namespace imq
+
+namespace imq {
+imq_status launch_unpack_batch(const imq_plan_t* const* pls, int n, const void* const* A, const void* const* B,
+                               int8_t* const* Au, int8_t* const* Bu, cudaStream_t st) {
+  if (n <= 0) return IMQ_OK;
+  DeviceState* ds;
+  imq_status s = device_state(&ds);
+  if (s != IMQ_OK) return s;
+  if (pls[0]->it == IMQ_I16) {
+    s = unpack_side_batch<int16_t>(pls, n, A, Au, 0, ds->num_sms, st);
+    if (s == IMQ_OK) s = unpack_side_batch<int16_t>(pls, n, B, Bu, 1, ds->num_sms, st);
+  } else {
+    s = unpack_side_batch<int32_t>(pls, n, A, Au, 0, ds->num_sms, st);
+    if (s == IMQ_OK) s = unpack_side_batch<int32_t>(pls, n, B, Bu, 1, ds->num_sms, st);
+  }
+  return s;
+}
 }  // namespace imq

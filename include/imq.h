@@ -392,6 +392,67 @@ imq_status imq_plan_unpack(const void *A, const void *B, imq_dtype it, int64_t M
                            size_t workspace_bytes, imq_plan_t **plan, imq_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------------ */
+/* 4. Batches of equal-shaped GEMMs (attention heads)                                                */
+/* ------------------------------------------------------------------------------------------------ */
+/*
+ * The page singles out the attention GEMMs: its "Key results" quote an unpack ratio of about 3-4x for
+ * attention-output GEMMs at 5 bits, and its "Limitations" name the self-attention matrix, whose outliers
+ * sit on the diagonal, as the case unpacking handles worst.  One attention layer is many small GEMMs of
+ * one shape (one per head), each needing its own plan: the calls below plan, unpack and multiply such a
+ * batch with one host round trip for all the plans, one unpack launch per operand and one GEMM launch
+ * whose tile scheduler runs the tiles of every problem (as few as the problem table allows: 64 problems
+ * per launch).  Problem h reads A + h * strideA and B + h * strideB (in elements of the integer dtype)
+ * with the leading dimensions lda, ldb; every problem is planned separately (its own levels, directions
+ * and layout), exactly as imq_plan would plan it alone.
+ */
+
+/*
+ * imq_plan_batched -- `batch` plans, plans[h] for problem h (HOST array of batch handles, each freed
+ * with imq_plan_destroy).  Arguments as imq_plan; the four line-maxima vectors, when all are given,
+ * hold batch consecutive vectors (problem h's a_rowmax at a_rowmax + h * M, a_colmax at + h * K,
+ * b_rowmax at + h * K, b_colmax at + h * N); when any is NULL each plan computes its own.  Synchronises
+ * once for the whole batch.  On an error no plan is returned (every entry of plans is NULL).
+ */
+imq_status imq_plan_batched(int32_t batch, const void *A, int64_t strideA, const void *B, int64_t strideB,
+                            imq_dtype it, int64_t M, int64_t K, int64_t N, int32_t transA, int64_t lda,
+                            int32_t transB, int64_t ldb, int32_t b, imq_strategy strategy,
+                            const int32_t *a_rowmax, const int32_t *a_colmax, const int32_t *b_rowmax,
+                            const int32_t *b_colmax, imq_plan_t **plans, imq_stream_t stream);
+
+/*
+ * imq_batch_workspace -- the device workspace a batch needs (*total_bytes) and, when offsets (HOST,
+ * 2 * batch entries) is given, where each operand lies in it: problem h's A' at offsets[2h] and its B'^T
+ * at offsets[2h + 1], each from a 1024-byte boundary (the workspace itself 1024-byte aligned).
+ */
+imq_status imq_batch_workspace(int32_t batch, imq_plan_t *const *plans, size_t *offsets, size_t *total_bytes);
+
+/* imq_unpack_batched -- imq_unpack of every problem of a batch planned by one imq_plan_batched call, into
+ * the workspace layout of imq_batch_workspace.  A, B, strides: those the plans were made from.
+ * IMQ_ERR_BUFFER when workspace_bytes is below the batch's need; IMQ_ERR_ARG for plans of different
+ * shapes, layouts or b.  Asynchronous. */
+imq_status imq_unpack_batched(int32_t batch, imq_plan_t *const *plans, const void *A, int64_t strideA,
+                              const void *B, int64_t strideB, void *workspace, size_t workspace_bytes,
+                              imq_stream_t stream);
+
+/* imq_gemm_unpacked_batched -- imq_gemm_unpacked of every problem of the batch from the unpacked operands
+ * in the workspace: problem h uses deltaA + h * strideDA, deltaB + h * strideDB (each NULL when Cf is
+ * NULL), writes C at Cint + h * strideC and Cf at Cf + h * strideCf (strides in elements of C's dtype
+ * and of fp32; leading dimensions ldc, ldcf).  Errors as imq_gemm_unpacked.  Asynchronous. */
+imq_status imq_gemm_unpacked_batched(int32_t batch, imq_plan_t *const *plans, const void *workspace,
+                                     size_t workspace_bytes, const float *deltaA, int64_t strideDA,
+                                     imq_gran gA, const float *deltaB, int64_t strideDB, imq_gran gB,
+                                     void *Cint, int64_t strideC, imq_dtype ct, int64_t ldc, float *Cf,
+                                     int64_t strideCf, int64_t ldcf, imq_stream_t stream);
+
+/* imq_unpacked_gemm_batched -- imq_unpack_batched followed by imq_gemm_unpacked_batched. */
+imq_status imq_unpacked_gemm_batched(int32_t batch, imq_plan_t *const *plans, const void *A, int64_t strideA,
+                                     const void *B, int64_t strideB, const float *deltaA, int64_t strideDA,
+                                     imq_gran gA, const float *deltaB, int64_t strideDB, imq_gran gB,
+                                     void *Cint, int64_t strideC, imq_dtype ct, int64_t ldc, float *Cf,
+                                     int64_t strideCf, int64_t ldcf, void *workspace, size_t workspace_bytes,
+                                     imq_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------------ */
 /* Status                                                                                            */
 /* ------------------------------------------------------------------------------------------------ */
 /* Synchronises the stream, returns the device status word of the current device and, when clear is

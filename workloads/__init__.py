@@ -175,7 +175,7 @@ def attention_head(h: int, seq: int = 2048, dim: int = 128) -> list:
     P = np.exp(logits)
     P /= P.sum(axis=1, keepdims=True)
     V = _normal(rng, (seq, dim))
-    q, k, p, v = _bf("Q", Q), _bf("K", Kt), _bf("P", P.astype(np.float32)), _bf("V", V)
+    q, k, p, v = _bf(f"Q{h}", Q), _bf(f"K{h}", Kt), _bf(f"P{h}", P.astype(np.float32)), _bf(f"V{h}", V)
     return [Gemm(f"attn_qk_h{h}", q, k, False, True, PER_ROW, PER_ROW, 0.95, 15, 5),
             Gemm(f"attn_pv_h{h}", p, v, False, False, PER_ROW, PER_COL, 0.95, 15, 5)]
 
