@@ -134,7 +134,8 @@ struct Geo {
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
   static constexpr size_t kBars = kScratch + 32768;
   static constexpr size_t kMisc = kBars + (2 * kStages + 5) * 8;  // tmem base, abort flag
-  static constexpr size_t kEnd = kMisc + 16;
+  static constexpr size_t kOut = kMisc + 16;  // per epilogue warp: the drain's output fields (a table launch)
+  static constexpr size_t kEnd = kOut + 8 * 64;
   static constexpr size_t kBytes = kEnd + 1024;  // slack for 1024-byte alignment of the base
   static_assert(kBytes <= 232448, "shared memory budget");
 };
@@ -367,8 +368,17 @@ __device__ __forceinline__ void release_slot(uint32_t acce_bar) {
 // Drains this warp's chunks of one TMEM slot (its 32 lanes) into C: fold, shift, then write (first),
 // add (a later drain of the same tile), or add atomically (atomic: several K splits share the tile).
 // `last` (never with atomic): also writes Cf.
+// The problem's output fields, read once per drain into registers (a problem table in global memory could
+// alias the drain's own stores as far as the compiler knows, which would reload them at every store).
+struct DrainOut {
+  void* C;
+  float* Cf;
+  int64_t ldc, ldcf;
+  int32_t c64, bm1;
+};
+
 template <typename T, int NC, int PQ, bool kPair>
-__device__ __forceinline__ void drain_slot(const GemmProb& g, uint32_t tbase, uint32_t acce_bar, int lane, int h,
+__device__ __forceinline__ void drain_slot(const DrainOut& g, uint32_t tbase, uint32_t acce_bar, int lane, int h,
                                            bool first, bool last, bool atomic, int shift, T* scr,
                                            const DrainMeta<NC>& m) {
   uint32_t v[32];
@@ -658,6 +668,7 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1) k_gemm(const __grid_c
     const int h = ew / 4;          // which of the quarter's warps: chunks h, h + PQ, ...
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     T* scr = scratch + ew * 32 * 32;  // this warp's transpose buffer (XOR-swizzled rows of 32)
+    DrainOut* wout = reinterpret_cast<DrainOut*>(base + G::kOut) + ew;
     // where a released slot is signalled: this CTA's barrier, or the leader's for a pair
     const uint32_t rel0 = kPair ? mapa_shared(acce0, 0) : acce0;
     const uint32_t rel1 = kPair ? mapa_shared(acce0 + 8, 0) : acce0 + 8;
@@ -707,8 +718,17 @@ __global__ void __launch_bounds__(Epi<kWide>::kThreads, 1) k_gemm(const __grid_c
         __syncwarp();
         if (lane == 0) release_slot<kPair>(rel);
       } else {
-        drain_slot<T, NC, PQ, kPair>(g, tbase, rel, lane, h, g.pc_dfirst[pc] != 0, last, atomic, g.pc_dshift[pc],
-                                     scr, meta);
+        if constexpr (kMulti) {
+          // from the table into this warp's shared slot, read from there by the stores
+          if (lane == 0) *wout = DrainOut{g.C, g.Cf, g.ldc, g.ldcf, g.c64, g.bm1};
+          __syncwarp();
+          drain_slot<T, NC, PQ, kPair>(*wout, tbase, rel, lane, h, g.pc_dfirst[pc] != 0, last, atomic,
+                                       g.pc_dshift[pc], scr, meta);
+        } else {
+          const DrainOut out{g.C, g.Cf, g.ldc, g.ldcf, g.c64, g.bm1};
+          drain_slot<T, NC, PQ, kPair>(out, tbase, rel, lane, h, g.pc_dfirst[pc] != 0, last, atomic, g.pc_dshift[pc],
+                                       scr, meta);
+        }
       }
     }
   epi_done:;

@@ -725,6 +725,222 @@ __global__ void __launch_bounds__(kThreads) k_rtn_rows(
 }
 
 // ------------------------------------------------------------------------------------------------
+// per stored row, bf16, the row in registers: one CTA of NT threads per row, thread t holding the
+// 16-byte vectors t, t + NT, ... (VPT of them) of every row it processes, so that it also owns the same
+// columns in every row and keeps their maxima in its registers.  The exact nearest-rank select is a
+// two-pass radix select on the 15-bit keys of |x| (the bf16 bit pattern without its sign orders like the
+// magnitude): a 256-bin shared histogram of the high 8 key bits picks the bucket holding rank k, a 128-bin
+// histogram of the low 7 bits of that bucket's keys picks the key.  The row is read from HBM once and
+// written once; the shared memory is two small histograms, so several CTAs share an SM.
+// Requires n % 8 == 0, 16-byte aligned rows (X, ld, Xint, ldq) and no transposed output.
+// ------------------------------------------------------------------------------------------------
+template <int NT>
+__device__ __forceinline__ uint32_t block_reduce_max(uint32_t v, uint32_t* red) {
+  v = __reduce_max_sync(0xffffffffu, v);
+  if constexpr (NT == 32) {
+    return v;
+  } else {
+    const int warp = threadIdx.x >> 5;
+    __syncthreads();  // red is free
+    if ((threadIdx.x & 31) == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t m = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) m = max(m, red[w]);
+    return m;
+  }
+}
+
+template <int NT, int VPT, bool kOut16>
+__global__ void __launch_bounds__(NT) k_rtn_rows_reg(const uint16_t* __restrict__ X, int64_t rows, int n, int64_t ld,
+                                                     unsigned long long krank, int beta, void* __restrict__ Xint,
+                                                     int64_t ldq, float* __restrict__ delta, float* __restrict__ qval,
+                                                     int32_t* __restrict__ rowmax, int32_t* __restrict__ part,
+                                                     int32_t* status, int clip) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t red[NT / 32];
+  __shared__ int s_sel[2];
+  __shared__ unsigned long long s_below;
+  const int tid = threadIdx.x;
+  const int nvec = n / 8;
+  constexpr int CW = kOut16 ? 4 : 8;  // column maxima words per vector: two 16-bit or one 32-bit per entry
+  uint32_t cm[VPT][CW];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int c = 0; c < CW; ++c) cm[j][c] = 0;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint16_t* xr = X + r * ld;
+    uint4 w[VPT];
+    uint32_t kmax = 0, bad = 0;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      w[j] = v < nvec ? __ldcs(reinterpret_cast<const uint4*>(xr) + v) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t k0 = ww[q] & 0x7FFFu, k1 = (ww[q] >> 16) & 0x7FFFu;
+        kmax = max(kmax, max(k0, k1));
+      }
+    }
+    bad = kmax >= 0x7F80u;  // an Inf or NaN among this thread's entries (padding vectors are zeros)
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+    const uint32_t rkmax = block_reduce_max<NT>(kmax, red);  // also orders the zeroing before the counts
+    if (NT == 32) __syncwarp();
+    // pass A: high 8 key bits
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      if (tid + j * NT >= nvec) continue;
+      const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        atomicAdd(&hist[(ww[q] & 0x7FFFu) >> 7], 1u);
+        atomicAdd(&hist[((ww[q] >> 16) & 0x7FFFu) >> 7], 1u);
+      }
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int d;
+      unsigned long long below;
+      if (warp_select(hist, 1, krank, &d, &below)) {
+        s_sel[0] = d;
+        s_below = below;
+      }
+    }
+    __syncthreads();
+    const uint32_t bucket = (uint32_t)s_sel[0];
+    const unsigned long long krem = krank - s_below;
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+    __syncthreads();
+    // pass B: low 7 key bits of the keys in that bucket
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      if (tid + j * NT >= nvec) continue;
+      const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t k0 = ww[q] & 0x7FFFu, k1 = (ww[q] >> 16) & 0x7FFFu;
+        if ((k0 >> 7) == bucket) atomicAdd(&hist[k0 & 127u], 1u);
+        if ((k1 >> 7) == bucket) atomicAdd(&hist[k1 & 127u], 1u);
+      }
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int d;
+      unsigned long long below;
+      if (warp_select(hist, 1, krem, &d, &below)) s_sel[1] = d;
+    }
+    // the bad flag of the whole row, which also publishes s_sel[1]
+    const uint32_t rbad = block_reduce_max<NT>(bad, red);
+    if (NT == 32) __syncwarp();
+    const uint32_t qkey = (bucket << 7) | (uint32_t)s_sel[1];
+    float s, dl;
+    const float qu = scale_from_q(__uint_as_float(qkey << 16), __uint_as_float(rkmax << 16), beta, &s, &dl);
+    if (tid == 0) {
+      delta[r] = dl;
+      if (qval) qval[r] = qu;
+    }
+    if (rbad) {
+      if (tid == 0) set_status(status, IMQ_ERR_NONFINITE);
+    } else {
+      bool range;
+      const uint32_t rmx = group_max_int<kOut16>(__uint_as_float(rkmax << 16), s, clip, &range);
+      if (tid == 0) {
+        if (range) set_status(status, IMQ_ERR_RANGE);
+        if (rowmax) rowmax[r] = (int32_t)rmx;
+      }
+      char* orow = static_cast<char*>(Xint) + r * ldq * (kOut16 ? 2 : 4);
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = tid + j * NT;
+        if (v >= nvec) continue;
+        const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+        int32_t q[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float y0 = __fmul_rn(__uint_as_float(ww[e] << 16), s);
+          float y1 = __fmul_rn(__uint_as_float(ww[e] & 0xFFFF0000u), s);
+          if (clip) {
+            y0 = fminf(fmaxf(y0, -(float)clip), (float)clip);
+            y1 = fminf(fmaxf(y1, -(float)clip), (float)clip);
+          }
+          q[2 * e] = __float2int_rn(y0);
+          q[2 * e + 1] = __float2int_rn(y1);
+        }
+        if constexpr (kOut16) {
+          uint32_t pv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pv[e] = __byte_perm((uint32_t)q[2 * e], (uint32_t)q[2 * e + 1], 0x5410);
+            const uint32_t a0 = (uint32_t)abs(q[2 * e]), a1 = (uint32_t)abs(q[2 * e + 1]);
+            cm[j][e] = max_u16x2(cm[j][e], __byte_perm(a0, a1, 0x5410));
+          }
+          __stcs(reinterpret_cast<uint4*>(orow) + v, make_uint4(pv[0], pv[1], pv[2], pv[3]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) cm[j][e] = max(cm[j][e], q[e] < 0 ? 0u - (uint32_t)q[e] : (uint32_t)q[e]);
+          int4* o = reinterpret_cast<int4*>(orow) + 2 * v;
+          __stcs(o, make_int4(q[0], q[1], q[2], q[3]));
+          __stcs(o + 1, make_int4(q[4], q[5], q[6], q[7]));
+        }
+      }
+    }
+  }
+  if (part) {
+    int32_t* mine = part + (int64_t)blockIdx.x * n;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v >= nvec) continue;
+      int4* o = reinterpret_cast<int4*>(mine + (int64_t)v * 8);
+      if constexpr (kOut16) {
+        o[0] = make_int4((int)(cm[j][0] & 0xFFFFu), (int)(cm[j][0] >> 16), (int)(cm[j][1] & 0xFFFFu),
+                         (int)(cm[j][1] >> 16));
+        o[1] = make_int4((int)(cm[j][2] & 0xFFFFu), (int)(cm[j][2] >> 16), (int)(cm[j][3] & 0xFFFFu),
+                         (int)(cm[j][3] >> 16));
+      } else {
+        o[0] = make_int4((int)cm[j][0], (int)cm[j][1], (int)cm[j][2], (int)cm[j][3]);
+        o[1] = make_int4((int)cm[j][4], (int)cm[j][5], (int)cm[j][6], (int)cm[j][7]);
+      }
+    }
+  }
+}
+
+// bf16 transpose through shared memory: X (rows x cols, leading dimension ld) into Y (cols x rows, dense),
+// 64 x 64 tiles, 16-byte loads and stores (rows and cols multiples of 8, X and ld 16-byte aligned).
+__global__ void __launch_bounds__(256) k_transpose_bf16(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
+                                                        int64_t ld, uint16_t* __restrict__ Y) {
+  __shared__ uint16_t tile[64][64 + 8];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int tid = threadIdx.x;
+  // load: 64 rows x 8 vectors of 8 entries, two per thread
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = tid + k * 256, rr = i >> 3, cv = (i & 7) * 8;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 + rr < rows && c0 + cv < cols) w = __ldcs(reinterpret_cast<const uint4*>(X + (r0 + rr) * ld + c0 + cv));
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      tile[rr][cv + 2 * e] = (uint16_t)(ww[e] & 0xFFFFu);
+      tile[rr][cv + 2 * e + 1] = (uint16_t)(ww[e] >> 16);
+    }
+  }
+  __syncthreads();
+  // store: 64 output rows (columns of X) x 8 vectors of 8 entries (rows of X)
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = tid + k * 256, cc = i >> 3, rv = (i & 7) * 8;
+    if (c0 + cc >= cols || r0 + rv >= rows) continue;
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = (uint32_t)tile[rv + 2 * e][cc] | ((uint32_t)tile[rv + 2 * e + 1][cc] << 16);
+    *reinterpret_cast<uint4*>(Y + (c0 + cc) * rows + r0 + rv) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // per stored column, slab staged in shared memory: CW columns x all rows are read from HBM once and
 // stored transposed (each column contiguous); then one warp per column runs the same select and
 // quantisation as a row.  With trans_out the quantised column is written as one contiguous output row
@@ -1101,11 +1317,82 @@ imq_status run_cols_staged(const T* X, int64_t rows, int64_t cols, int64_t ld, u
   return rowmax ? launch_reduce_max(part, grid, rows, rowmax, st) : IMQ_OK;
 }
 
+// The register-resident per-row kernel for bf16 rows of n entries (n % 8 == 0, n <= 16384, 16-byte
+// aligned rows of X and Xint): NT threads per row and VPT 16-byte vectors per thread.  rowmax / colmax
+// are over the rows and columns of the matrix given here (the caller swaps them for a transposed input).
+template <int NT, int VPT, bool kOut16>
+imq_status launch_rows_reg(const uint16_t* X, int64_t rows, int n, int64_t ld, unsigned long long k, int32_t beta,
+                           void* Xint, int64_t ldq, float* delta, float* qval, int32_t* rowmax, int32_t* colmax,
+                           int clip, DeviceState* ds, cudaStream_t st) {
+  auto kern = k_rtn_rows_reg<NT, VPT, kOut16>;
+  int per_sm = 0;
+  IMQ_CUDA_TRY(blocks_per_sm(reinterpret_cast<const void*>(kern), NT, 0, &per_sm));
+  if (per_sm < 1) per_sm = 1;
+  const int64_t grid = rows < (int64_t)ds->num_sms * per_sm ? rows : (int64_t)ds->num_sms * per_sm;
+  int32_t* part = nullptr;
+  StreamScratch sp;
+  if (colmax) {
+    if (sp.alloc(ds, (size_t)grid * n * 4, st) != IMQ_OK) return IMQ_ERR_CUDA;
+    part = static_cast<int32_t*>(sp.p);
+  }
+  kern<<<(unsigned)grid, NT, 0, st>>>(X, rows, n, ld, k, beta, Xint, ldq, delta, qval, rowmax, part, ds->status, clip);
+  if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
+  return colmax ? launch_reduce_max(part, grid, n, colmax, st) : IMQ_OK;
+}
+
+// True (and *status set) when the register-resident kernel takes this shape; false leaves it to the
+// staged kernels.
+template <bool kOut16>
+bool try_rows_reg(const uint16_t* X, int64_t rows, int64_t n, int64_t ld, unsigned long long k, int32_t beta,
+                  void* Xint, int64_t ldq, float* delta, float* qval, int32_t* rowmax, int32_t* colmax, int clip,
+                  DeviceState* ds, cudaStream_t st, imq_status* status) {
+  if (n % 8 != 0 || n > 16384 || ld % 8 != 0 || ldq % 8 != 0 || (reinterpret_cast<uintptr_t>(X) & 15) ||
+      (reinterpret_cast<uintptr_t>(Xint) & 15))
+    return false;
+  const int nvec = (int)(n / 8), nn = (int)n;
+  if (nvec <= 32)
+    *status = launch_rows_reg<32, 1, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  else if (nvec <= 128)
+    *status = launch_rows_reg<128, 1, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  else if (nvec <= 256)
+    *status = launch_rows_reg<256, 1, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  else if (nvec <= 512)
+    *status = launch_rows_reg<256, 2, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  else if (nvec <= 1024)
+    *status = launch_rows_reg<256, 4, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  else if (nvec <= 1536)
+    *status = launch_rows_reg<256, 6, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  else
+    *status = launch_rows_reg<256, 8, kOut16>(X, rows, nn, ld, k, beta, Xint, ldq, delta, qval, rowmax, colmax, clip, ds, st);
+  return true;
+}
+
 template <typename T, bool kOut16>
 imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, double p,
                int32_t beta, void* Xint, int64_t ldq, int trans_out, float* delta, float* qval, int32_t* rowmax,
                int32_t* colmax, int clip, DeviceState* ds, cudaStream_t st) {
   const int sms = ds->num_sms;
+  if constexpr (sizeof(T) == 2) {
+    // bf16 rows: the register-resident kernel; bf16 columns into the transposed layout: a transpose,
+    // then the same kernel on the rows of the transpose (its row and column maxima swapped)
+    imq_status rs = IMQ_OK;
+    if (g == IMQ_PER_ROW && !trans_out &&
+        try_rows_reg<kOut16>(X, rows, cols, ld, (unsigned long long)nearest_rank(cols, p), beta, Xint, ldq, delta,
+                             qval, rowmax, colmax, clip, ds, st, &rs))
+      return rs;
+    if (g == IMQ_PER_COL && trans_out && rows % 8 == 0 && cols % 8 == 0 && rows <= 16384 && ld % 8 == 0 &&
+        ldq % 8 == 0 && !(reinterpret_cast<uintptr_t>(X) & 15) && !(reinterpret_cast<uintptr_t>(Xint) & 15)) {
+      StreamScratch tp;
+      if (tp.alloc(ds, (size_t)rows * cols * 2, st) != IMQ_OK) return IMQ_ERR_CUDA;
+      uint16_t* Y = static_cast<uint16_t*>(tp.p);
+      const dim3 tg((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+      k_transpose_bf16<<<tg, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(X), rows, cols, ld, Y);
+      if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
+      if (try_rows_reg<kOut16>(Y, cols, rows, rows, (unsigned long long)nearest_rank(rows, p), beta, Xint, ldq, delta,
+                               qval, colmax, rowmax, clip, ds, st, &rs))
+        return rs;
+    }
+  }
   if (g == IMQ_PER_COL) {
     const unsigned long long k = (unsigned long long)nearest_rank(rows, p);
     // the slab of 16 (or 8) columns is staged in shared memory when it fits (plus the row maxima)

@@ -271,7 +271,9 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
                                                       const int8_t* lvl, const int32_t* pos,
                                                       const int32_t* tK, const int8_t* lk,
                                                       const int32_t* blk16, int64_t K_unp, int bm1,
-                                                      int meta_smem, int8_t* out, const LineJob* __restrict__ jobs) {
+                                                      int meta_smem, int8_t* out, const int32_t* grpL,
+                                                      const int32_t* grpN, int64_t ngrp, int G,
+                                                      const LineJob* __restrict__ jobs) {
   extern __shared__ __align__(16) unsigned char dsm[];
   if (jobs) {
     const LineJob& jb = jobs[blockIdx.y];
@@ -284,6 +286,17 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
     blk16 = jb.blk16;
     K_unp = jb.K_unp;
     out = jb.out;
+    grpL = jb.grpL;
+    grpN = jb.grpN;
+    ngrp = jb.ngrp;
+  }
+  // unused lines of the OUTER groups dealt to this CTA (lines n*L .. G-1 of a group of n sources of level
+  // L, which no source line writes), before the lines themselves
+  for (int64_t g = blockIdx.x; g < ngrp; g += gridDim.x) {
+    const int64_t first = g * G + (int64_t)grpN[g] * grpL[g];
+    const int64_t n16 = ((g + 1) * G - first) * K_unp / 16;
+    uint4* o = reinterpret_cast<uint4*>(out + first * K_unp);
+    for (int64_t k = threadIdx.x; k < n16; k += blockDim.x) o[k] = make_uint4(0u, 0u, 0u, 0u);
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t Kp = (K + 15) / 16 * 16;  // plane row length, 16-byte aligned
@@ -427,6 +440,46 @@ __device__ __forceinline__ uint4 digits16_fixed(const Mag16& m) {
   }
 }
 
+// Magnitudes and signs of 16 consecutive int32 entries (shared memory), for their digits of any level.
+struct Mag16w {
+  uint32_t m[16];
+  uint32_t neg;  // bit k: entry k is negative
+};
+__device__ __forceinline__ Mag16w mag16_i32(const int32_t* v16) {
+  Mag16w r;
+  r.neg = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int4 w = reinterpret_cast<const int4*>(v16)[q];
+    const int32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      r.m[4 * q + k] = e[k] < 0 ? (uint32_t)(-(int64_t)e[k]) : (uint32_t)e[k];
+      r.neg |= (uint32_t)(e[k] < 0) << (4 * q + k);
+    }
+  }
+  return r;
+}
+// Digit l (base 2^bm1, sign-magnitude) of the 16 entries as 16 bytes in entry order.
+__device__ __forceinline__ uint4 digits16_i32(const Mag16w& m, int l, int bm1) {
+  const int sh = l * bm1;
+  if (sh >= 31) return make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t mask = (1u << bm1) - 1u;
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t packed = 0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int k = 4 * q + r;
+      const uint32_t d = (m.m[k] >> sh) & mask;
+      packed |= (((m.neg >> k) & 1u) ? ((0u - d) & 0xFFu) : d) << (8 * r);
+    }
+    o[q] = packed;
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take the unrolled path
 
 // Row gather for int16 sources, one warp per source line (base 2^kBm1 fixed at compile time).  The warp
@@ -437,18 +490,19 @@ constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take th
 // entry.  The per-block plan metadata is staged in shared memory once per CTA.  Lines are dealt to the
 // CTAs in turn (line i to CTA i mod gridDim.x).  After its lines, each CTA zeroes the unused lines of the
 // OUTER groups dealt to it (group g to CTA g mod gridDim.x), lines n*L .. G-1 of a group of n sources of
-// level L, which no source line writes.
-template <int kBm1>
-__global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int64_t nlines, int64_t K,
+// level L, which no source line writes.  cta_line: lines too long for a line per warp (more than 8192
+// entries) are staged one at a time per CTA by all its threads, and all its threads write its blocks.
+template <typename T, int kBm1>
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(const T* X, int64_t nlines, int64_t K,
                                                            int64_t ld, int nwarps, int outer, const int8_t* lvl,
                                                            const int32_t* pos, const int32_t* tK, const int8_t* lk,
                                                            const int32_t* blk16, int64_t K_unp, int8_t* out,
                                                            const int32_t* grpL, const int32_t* grpN, int64_t ngrp,
-                                                           int G, const LineJob* __restrict__ jobs) {
+                                                           int G, int cta_line, const LineJob* __restrict__ jobs) {
   extern __shared__ __align__(16) unsigned char dsm[];
   if (jobs) {
     const LineJob& jb = jobs[blockIdx.y];
-    X = static_cast<const int16_t*>(jb.X);
+    X = static_cast<const T*>(jb.X);
     outer = jb.outer;
     lvl = jb.lvl;
     pos = jb.pos;
@@ -464,33 +518,26 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t Kr = (K + 15) / 16 * 16;  // staged line length in entries (32-byte multiple)
   const int nchunk = (int)(K_unp / 16);
-  // [lines of nwarps warps, int16 x Kr][block starts, int32 x nchunk][first inner levels, int8 x nchunk]
-  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)nwarps * Kr * 2);
+  // [lines of nwarps warps (one line in cta_line mode), int16 x Kr][block starts, int32 x nchunk]
+  // [first inner levels, int8 x nchunk]
+  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)(cta_line ? 1 : nwarps) * Kr * (int64_t)sizeof(T));
   int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);
   for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
     s_blk[c] = blk16[c];
     s_lk0[c] = lk[(int64_t)c * 16];
   }
   __syncthreads();
-  if (warp < nwarps) {
-    int16_t* row = reinterpret_cast<int16_t*>(dsm) + (int64_t)warp * Kr;
-    const bool vec8 = (K % 8 == 0) && (ld % 8 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
-    for (int64_t line = (int64_t)warp * gridDim.x + blockIdx.x; line < nlines;
-         line += (int64_t)gridDim.x * nwarps) {
-      const int16_t* xr = X + line * ld;
-      if (vec8) {
-        warp_copy16_global<4>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), (int)(K / 8), lane);
-      } else {
-        for (int64_t t = lane; t < K; t += 32) row[t] = xr[t];
-      }
-      __syncwarp();
+  constexpr int kPer16 = 16 / (int)sizeof(T);  // entries per 16-byte load
+  const bool vec8 = (K % kPer16 == 0) && (ld % kPer16 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  // The unpacked lines of source line `line`, staged in `row`: blocks c_first, c_first + c_step, ...
+  auto emit = [&](int64_t line, const T* row, int c_first, int c_step) {
       const int L = outer ? (int)lvl[line] : 1;
       int8_t* o0 = out + (outer ? (int64_t)pos[line] : line) * K_unp;
       if (L <= kFastLevels) {
         int8_t* ol[kFastLevels];
 #pragma unroll
         for (int l = 0; l < kFastLevels; ++l) ol[l] = o0 + (int64_t)l * K_unp;
-        for (int c = lane; c < nchunk; c += 32) {
+        for (int c = c_first; c < nchunk; c += c_step) {
           const int t0 = s_blk[c];
           const int p = c * 16;
           uint4 d[kFastLevels];
@@ -499,7 +546,7 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
             if (L > 1 && lk0 > 0) {
 #pragma unroll
               for (int l = 0; l < kFastLevels; ++l) d[l] = make_uint4(0u, 0u, 0u, 0u);
-            } else {
+            } else if constexpr (sizeof(T) == 2) {
               const uint4 w0 = *reinterpret_cast<const uint4*>(row + t0);
               const uint4 w1 = *reinterpret_cast<const uint4*>(row + t0 + 8);
               const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -511,6 +558,14 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
                 d[1] = digits16_fixed<kBm1, 1>(m);
                 if (L > 2) d[2] = digits16_fixed<kBm1, 2>(m);
                 if (L > 3) d[3] = digits16_fixed<kBm1, 3>(m);
+              }
+            } else {
+              const Mag16w m = mag16_i32(reinterpret_cast<const int32_t*>(row + t0));
+              if (L == 1) {
+                d[0] = digits16_i32(m, lk0, kBm1);
+              } else {
+#pragma unroll
+                for (int l = 0; l < kFastLevels; ++l) d[l] = l < L ? digits16_i32(m, l, kBm1) : make_uint4(0u, 0u, 0u, 0u);
               }
             }
           } else {
@@ -542,7 +597,7 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
         }
       } else {
         // lines of more levels (small b): one output line at a time
-        for (int c = lane; c < nchunk; c += 32) {
+        for (int c = c_first; c < nchunk; c += c_step) {
           const int t0 = s_blk[c];
           const int p = c * 16;
           const int lk0 = t0 >= 0 ? s_lk0[c] : 0;
@@ -551,11 +606,13 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
             if (t0 >= 0) {
               if (lk0 > 0) {
                 dv = make_uint4(0u, 0u, 0u, 0u);
-              } else {
+              } else if constexpr (sizeof(T) == 2) {
                 const uint4 w0 = *reinterpret_cast<const uint4*>(row + t0);
                 const uint4 w1 = *reinterpret_cast<const uint4*>(row + t0 + 8);
                 const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
                 dv = digits16_i16(w, l, kBm1);
+              } else {
+                dv = digits16_i32(mag16_i32(reinterpret_cast<const int32_t*>(row + t0)), l, kBm1);
               }
             } else {
               uint32_t wv[4] = {0u, 0u, 0u, 0u};
@@ -572,6 +629,36 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
           }
         }
       }
+  };
+  if (cta_line) {
+    // long lines: one line at a time per CTA, staged by all its threads, its blocks spread over all of them
+    T* row = reinterpret_cast<T*>(dsm);
+    for (int64_t line = blockIdx.x; line < nlines; line += gridDim.x) {
+      const T* xr = X + line * ld;
+      __syncthreads();  // the previous line has been read
+      if (vec8) {
+        const uint4* src = reinterpret_cast<const uint4*>(xr);
+        uint4* dst = reinterpret_cast<uint4*>(row);
+        for (int64_t q = threadIdx.x; q < K / kPer16; q += blockDim.x) dst[q] = src[q];
+      } else {
+        for (int64_t t = threadIdx.x; t < K; t += blockDim.x) row[t] = xr[t];
+      }
+      __syncthreads();
+      emit(line, row, (int)threadIdx.x, (int)blockDim.x);
+    }
+  } else if (warp < nwarps) {
+    T* row = reinterpret_cast<T*>(dsm) + (int64_t)warp * Kr;
+    for (int64_t line = (int64_t)warp * gridDim.x + blockIdx.x; line < nlines;
+         line += (int64_t)gridDim.x * nwarps) {
+      const T* xr = X + line * ld;
+      if (vec8) {
+        warp_copy16_global<4>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), (int)(K / kPer16),
+                              lane);
+      } else {
+        for (int64_t t = lane; t < K; t += 32) row[t] = xr[t];
+      }
+      __syncwarp();
+      emit(line, row, lane, 32);
       __syncwarp();
     }
   }
@@ -585,13 +672,13 @@ __global__ void __launch_bounds__(256, 3) k_unpack_lines16(const int16_t* X, int
 }
 
 // nprob > 1: `jobs` (device) holds the per-problem arguments and the ones given here are ignored.
-template <int kBm1>
-imq_status launch_lines16(const int16_t* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
+template <typename T, int kBm1>
+imq_status launch_lines16(const T* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
                           const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
                           const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL, const int32_t* grpN,
                           int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs = nullptr,
                           int nprob = 1) {
-  auto kern = k_unpack_lines16<kBm1>;
+  auto kern = k_unpack_lines16<T, kBm1>;
   IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   int per_sm = 0;
   IMQ_CUDA_TRY(blocks_per_sm(reinterpret_cast<const void*>(kern), 256, smem, &per_sm));
@@ -600,8 +687,42 @@ imq_status launch_lines16(const int16_t* X, int64_t nlines, int64_t K, int64_t l
   int64_t grid = ((int64_t)num_sms * per_sm + nprob - 1) / nprob;
   if (grid > nlines) grid = nlines;
   kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16,
-                                                                 K_unp, out, grpL, grpN, ngrp, G, jobs);
+                                                                 K_unp, out, grpL, grpN, ngrp, G, nw == 0 ? 1 : 0,
+                                                                 jobs);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
+// The staged-line kernel for base 2^bm1 (bm1 in 1..7), the base fixed at compile time.
+template <typename T>
+imq_status launch_staged(int bm1, const T* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
+                         const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
+                         const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL, const int32_t* grpN,
+                         int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs,
+                         int nprob) {
+  switch (bm1) {
+    case 1: return launch_lines16<T, 1>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    case 2: return launch_lines16<T, 2>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    case 3: return launch_lines16<T, 3>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    case 4: return launch_lines16<T, 4>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    case 5: return launch_lines16<T, 5>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    case 6: return launch_lines16<T, 6>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    default: return launch_lines16<T, 7>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+  }
+}
+
+// Launch shape of the staged-line kernel for lines of K entries of T and nchunk 16-position blocks: a
+// line per warp (8 warps while their lines fit in 64 KB, so that three CTAs share an SM), or for lines
+// above 16 KB one line per CTA (nw = 0: all 8 warps stage it and write its blocks).  False when the
+// line and the block metadata (5 bytes per block, staged whole) do not fit the shared-memory budget.
+bool staged_shape(int64_t K, size_t elem, int64_t nchunk, int* nw_out, size_t* smem_out) {
+  const int64_t line_bytes = (K + 15) / 16 * 16 * (int64_t)elem;
+  const bool cta_line = line_bytes > 16 * 1024;
+  int nw = cta_line ? 0 : (int)((64 * 1024) / line_bytes);
+  if (nw > 8) nw = 8;
+  const size_t smem = (size_t)(cta_line ? 1 : nw) * line_bytes + (size_t)nchunk * 5;
+  *nw_out = nw;
+  *smem_out = smem;
+  return nchunk <= kMetaMaxChunks16 && smem <= 200 * 1024;
 }
 
 // Row gather for lines too long for shared-memory planes: digits are computed from the source line in
@@ -712,29 +833,15 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
                       const ZeroJob& zj, bool* zeroed) {
   *zeroed = false;
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
-  if constexpr (sizeof(T) == 2) {
-    // int16 rows: one warp per line with the line staged (8 warps while their lines fit in 64 KB, so that
-    // three CTAs share an SM; fewer for longer lines), the block metadata staged once per CTA
-    const int64_t Kr = (K + 15) / 16 * 16;
+  // rows (int16 or int32): the staged-line kernel, which also zeroes the unused OUTER lines
+  {
     const int64_t nchunk = K_unp / 16;
-    int nw = (int)((64 * 1024) / (Kr * 2));
-    if (nw < 1) nw = (int)((192 * 1024) / (Kr * 2)) >= 1 ? 1 : 0;
-    if (nw > 8) nw = 8;
-    const size_t smem = (size_t)nw * Kr * 2 + (size_t)nchunk * 5;
-    // the block metadata (5 bytes per 16 positions) is staged whole; the shared-memory budget bounds it
-    if (line_is_row && nw >= 1 && nchunk <= kMetaMaxChunks16 && smem <= 200 * 1024 && bm1 >= 1 && bm1 <= 7) {
-      const int16_t* X16 = reinterpret_cast<const int16_t*>(X);
+    int nw = 0;
+    size_t smem = 0;
+    if (line_is_row && bm1 >= 1 && bm1 <= 7 && staged_shape(K, sizeof(T), nchunk, &nw, &smem)) {
       const int64_t ng = outer ? zj.ngrp : 0;
-      imq_status s;
-      switch (bm1) {
-        case 1: s = launch_lines16<1>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-        case 2: s = launch_lines16<2>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-        case 3: s = launch_lines16<3>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-        case 4: s = launch_lines16<4>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-        case 5: s = launch_lines16<5>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-        case 6: s = launch_lines16<6>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-        default: s = launch_lines16<7>(X16, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st); break;
-      }
+      const imq_status s = launch_staged<T>(bm1, X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out,
+                                            zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st, nullptr, 1);
       *zeroed = s == IMQ_OK;
       return s;
     }
@@ -758,7 +865,9 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
         if (grid > ctas) grid = ctas;
         IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
         k_unpack_lines<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, P, nw, outer, lvl, pos, tK, lk, blk16,
-                                                             K_unp, bm1, meta_smem, out, nullptr);
+                                                             K_unp, bm1, meta_smem, out, zj.grpL, zj.grpN,
+                                                             outer ? zj.ngrp : 0, zj.G, nullptr);
+        *zeroed = true;
         return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
       }
     }
@@ -871,27 +980,15 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
   if (nlines == 0 || nchunk == 0) return IMQ_OK;
   void* dj = nullptr;
   imq_status s = IMQ_OK;
-  if (sizeof(T) == 2 && line_is_row && bm1 >= 1 && bm1 <= 7) {
-    const int64_t Kr = (K + 15) / 16 * 16;
-    int nw = (int)((64 * 1024) / (Kr * 2));
-    if (nw < 1) nw = (int)((192 * 1024) / (Kr * 2)) >= 1 ? 1 : 0;
-    if (nw > 8) nw = 8;
-    const size_t smem = (size_t)nw * Kr * 2 + (size_t)nchunk * 5;
-    if (nw >= 1 && nchunk <= kMetaMaxChunks16 && smem <= 200 * 1024) {
+  {
+    int nw = 0;
+    size_t smem = 0;
+    if (line_is_row && bm1 >= 1 && bm1 <= 7 && staged_shape(K, sizeof(T), nchunk, &nw, &smem)) {
       s = upload_table(jobs.data(), sizeof(LineJob) * (size_t)n, &dj, st);
       if (s != IMQ_OK) return s;
-      const int16_t* X0 = static_cast<const int16_t*>(src[0]);
-      const LineJob* J = static_cast<const LineJob*>(dj);
-      const int G = side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP;
-      switch (bm1) {
-        case 1: s = launch_lines16<1>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-        case 2: s = launch_lines16<2>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-        case 3: s = launch_lines16<3>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-        case 4: s = launch_lines16<4>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-        case 5: s = launch_lines16<5>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-        case 6: s = launch_lines16<6>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-        default: s = launch_lines16<7>(X0, nlines, K, ld, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, G, smem, num_sms, st, J, n); break;
-      }
+      s = launch_staged<T>(bm1, static_cast<const T*>(src[0]), nlines, K, ld, nw, 0, nullptr, nullptr, nullptr,
+                           nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP,
+                           smem, num_sms, st, static_cast<const LineJob*>(dj), n);
       cudaFreeAsync(dj, st);
       return s;
     }
@@ -913,17 +1010,11 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
       IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
       k_unpack_lines<T><<<dim3((unsigned)grid, (unsigned)n), 256, smem, st>>>(
           static_cast<const T*>(src[0]), nlines, K, ld, P, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, bm1,
-          meta_smem, nullptr, static_cast<const LineJob*>(dj));
+          meta_smem, nullptr, nullptr, nullptr, 0, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP,
+          static_cast<const LineJob*>(dj));
       s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
       cudaFreeAsync(dj, st);
-      if (s != IMQ_OK) return s;
-      // this kernel does not zero the unused lines of OUTER groups
-      for (int h = 0; h < n; ++h)
-        if (jobs[h].outer && jobs[h].ngrp > 0)
-          k_zero_unused<<<(unsigned)(jobs[h].ngrp < 4096 ? jobs[h].ngrp : 4096), 256, 0, st>>>(
-              jobs[h].grpL, jobs[h].grpN, jobs[h].ngrp, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP, jobs[h].K_unp,
-              jobs[h].out);
-      return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+      return s;
     }
   }
   // anything else: problem by problem
