@@ -84,8 +84,8 @@ struct imq_plan {
   int32_t* tK;      // [K_unp] source inner index, -1 on padding
   int8_t* lAk;      // [K_unp] digit level of A at that inner position
   int8_t* lBk;      // [K_unp] digit level of B
-  int32_t* blk16;   // [K_unp/16] first source index t0 when positions 16c..16c+15 hold t0..t0+15 with
-                    // t0 % 16 == 0 and one (lA, lB) pair, else -1 (the unpacker copies such blocks)
+  int32_t* blk16;   // [K_unp/16] when positions 16c..16c+15 hold t0..t0+15 with one (lA, lB) pair: t0
+                    // if t0 % 16 == 0, else -(t0 + 2); otherwise -1 (the unpackers copy runs)
   int32_t* posA;    // [M] first unpacked row of each source row (A OUTER)
   int32_t* srcA;    // [M_unp] source row of each unpacked row, -1 unused (A OUTER)
   int32_t* grpA_L;  // [M_unp / IMQ_A_GROUP] level of each row group

@@ -685,10 +685,12 @@ __device__ void inner_map_group(const InnerGroup grp, const InnerSeg* __restrict
   for (int64_t c = grp.k0 / 16 + threadIdx.x; c < (grp.k0 + grp.kpad) / 16; c += blockDim.x) {
     const int32_t* t = tK + c * 16;
     const int32_t t0 = t[0];
-    bool ok = t0 >= 0 && (t0 & 15) == 0;
-    for (int k = 1; k < 16 && ok; ++k)
-      ok = t[k] == t0 + k && lAk[c * 16 + k] == lAk[c * 16] && lBk[c * 16 + k] == lBk[c * 16];
-    blk16[c] = ok ? t0 : -1;
+    bool run = t0 >= 0;
+    for (int k = 1; k < 16 && run; ++k)
+      run = t[k] == t0 + k && lAk[c * 16 + k] == lAk[c * 16] && lBk[c * 16 + k] == lBk[c * 16];
+    // t0 for an aligned run, -(t0 + 2) for a run starting elsewhere (the staged unpacker reads those
+    // with unaligned loads; every other reader treats a negative entry as a gathered block), else -1
+    blk16[c] = !run ? -1 : ((t0 & 15) == 0 ? t0 : -(t0 + 2));
   }
 }
 

@@ -445,12 +445,15 @@ struct Mag16w {
   uint32_t m[16];
   uint32_t neg;  // bit k: entry k is negative
 };
+// v16 may start anywhere (16-byte loads when it is 16-byte aligned).
 __device__ __forceinline__ Mag16w mag16_i32(const int32_t* v16) {
   Mag16w r;
   r.neg = 0;
+  const bool al = (reinterpret_cast<uintptr_t>(v16) & 15) == 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int4 w = reinterpret_cast<const int4*>(v16)[q];
+    const int4 w = al ? reinterpret_cast<const int4*>(v16)[q]
+                      : make_int4(v16[4 * q], v16[4 * q + 1], v16[4 * q + 2], v16[4 * q + 3]);
     const int32_t e[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -478,6 +481,23 @@ __device__ __forceinline__ uint4 digits16_i32(const Mag16w& m, int l, int bm1) {
     o[q] = packed;
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The 16 int16 entries row[t0 .. t0 + 15] of a staged line at any t0, as 8 words of two entries (low
+// half first): 16-byte loads when t0 % 8 == 0, else 32-bit loads and a funnel shift for odd t0.
+__device__ __forceinline__ void load16_i16(const int16_t* row, int t0, uint32_t (&w)[8]) {
+  if ((t0 & 7) == 0) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + t0), b = *reinterpret_cast<const uint4*>(row + t0 + 8);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+    const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row + (t0 & ~1));
+    uint32_t v[9];
+#pragma unroll
+    for (int i = 0; i < 9; ++i) v[i] = r32[i];  // the 9th word is inside the 32-byte padded line
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = (t0 & 1) ? __funnelshift_r(v[i], v[i + 1], 16) : v[i];
+  }
 }
 
 constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take the unrolled path
@@ -538,18 +558,18 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
 #pragma unroll
         for (int l = 0; l < kFastLevels; ++l) ol[l] = o0 + (int64_t)l * K_unp;
         for (int c = c_first; c < nchunk; c += c_step) {
-          const int t0 = s_blk[c];
+          const int tb = s_blk[c];
+          const int t0 = tb >= 0 ? tb : -tb - 2;  // first source index of a run (aligned or not)
           const int p = c * 16;
           uint4 d[kFastLevels];
-          if (t0 >= 0) {
+          if (tb != -1) {
             const int lk0 = s_lk0[c];
             if (L > 1 && lk0 > 0) {
 #pragma unroll
               for (int l = 0; l < kFastLevels; ++l) d[l] = make_uint4(0u, 0u, 0u, 0u);
             } else if constexpr (sizeof(T) == 2) {
-              const uint4 w0 = *reinterpret_cast<const uint4*>(row + t0);
-              const uint4 w1 = *reinterpret_cast<const uint4*>(row + t0 + 8);
-              const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              uint32_t w[8];
+              load16_i16(reinterpret_cast<const int16_t*>(row), t0, w);
               const Mag16 m = mag16_i16(w);
               if (L == 1) {
                 d[0] = digits16_from(m, lk0, kBm1);
@@ -568,8 +588,52 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
                 for (int l = 0; l < kFastLevels; ++l) d[l] = l < L ? digits16_i32(m, l, kBm1) : make_uint4(0u, 0u, 0u, 0u);
               }
             }
+          } else if (const uint4 lq = *reinterpret_cast<const uint4*>(lk + p);
+                     lq.x == lq.y && lq.y == lq.z && lq.z == lq.w && (lq.x & 0xFFu) * 0x01010101u == lq.x) {
+            // a block of scattered source indices with one inner level (a sparse segment): its 16 entries
+            // gathered from the staged line (padding positions read as 0), then split like a run
+            const int lr = (int)(int8_t)(lq.x & 0xFFu);
+            const int4* tq = reinterpret_cast<const int4*>(tK + p);
+            int32_t tt[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int4 v = tq[q];
+              tt[4 * q] = v.x; tt[4 * q + 1] = v.y; tt[4 * q + 2] = v.z; tt[4 * q + 3] = v.w;
+            }
+            if (L > 1 && lr > 0) {
+#pragma unroll
+              for (int l = 0; l < kFastLevels; ++l) d[l] = make_uint4(0u, 0u, 0u, 0u);
+            } else if constexpr (sizeof(T) == 2) {
+              uint32_t w[8];
+#pragma unroll
+              for (int h = 0; h < 8; ++h) {
+                const uint32_t lo = tt[2 * h] >= 0 ? (uint32_t)(uint16_t)row[tt[2 * h]] : 0u;
+                const uint32_t hi = tt[2 * h + 1] >= 0 ? (uint32_t)(uint16_t)row[tt[2 * h + 1]] : 0u;
+                w[h] = lo | (hi << 16);
+              }
+              const Mag16 m = mag16_i16(w);
+              if (L == 1) {
+                d[0] = digits16_from(m, lr, kBm1);
+              } else {
+                d[0] = digits16_fixed<kBm1, 0>(m);
+                d[1] = digits16_fixed<kBm1, 1>(m);
+                if (L > 2) d[2] = digits16_fixed<kBm1, 2>(m);
+                if (L > 3) d[3] = digits16_fixed<kBm1, 3>(m);
+              }
+            } else {
+              int32_t g16[16];
+#pragma unroll
+              for (int k = 0; k < 16; ++k) g16[k] = tt[k] >= 0 ? (int32_t)row[tt[k]] : 0;
+              const Mag16w m = mag16_i32(g16);
+              if (L == 1) {
+                d[0] = digits16_i32(m, lr, kBm1);
+              } else {
+#pragma unroll
+                for (int l = 0; l < kFastLevels; ++l) d[l] = l < L ? digits16_i32(m, l, kBm1) : make_uint4(0u, 0u, 0u, 0u);
+              }
+            }
           } else {
-            // gathered entry by entry (block boundaries of segments and padding; rare)
+            // gathered entry by entry (blocks across segment boundaries and padding; rare)
 #pragma unroll
             for (int l = 0; l < kFastLevels; ++l) {
               uint32_t wv[4] = {0u, 0u, 0u, 0u};
@@ -598,18 +662,18 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
       } else {
         // lines of more levels (small b): one output line at a time
         for (int c = c_first; c < nchunk; c += c_step) {
-          const int t0 = s_blk[c];
+          const int tb = s_blk[c];
+          const int t0 = tb >= 0 ? tb : -tb - 2;
           const int p = c * 16;
-          const int lk0 = t0 >= 0 ? s_lk0[c] : 0;
+          const int lk0 = tb != -1 ? s_lk0[c] : 0;
           for (int l = 0; l < L; ++l) {
             uint4 dv;
-            if (t0 >= 0) {
+            if (tb != -1) {
               if (lk0 > 0) {
                 dv = make_uint4(0u, 0u, 0u, 0u);
               } else if constexpr (sizeof(T) == 2) {
-                const uint4 w0 = *reinterpret_cast<const uint4*>(row + t0);
-                const uint4 w1 = *reinterpret_cast<const uint4*>(row + t0 + 8);
-                const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t w[8];
+                load16_i16(reinterpret_cast<const int16_t*>(row), t0, w);
                 dv = digits16_i16(w, l, kBm1);
               } else {
                 dv = digits16_i32(mag16_i32(reinterpret_cast<const int32_t*>(row + t0)), l, kBm1);
