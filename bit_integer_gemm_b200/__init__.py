@@ -18,11 +18,12 @@ from collections import namedtuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libimq.so")
+# IMQ_LIB=debug selects the IMQ_DEBUG build (index checks after every plan); anything else the release one
+LIB_PATH = os.path.join(_HERE, "libimq_debug.so" if os.environ.get("IMQ_LIB") == "debug" else "libimq.so")
 
 # status codes
 IMQ_OK, IMQ_ERR_ARG, IMQ_ERR_NONFINITE, IMQ_ERR_RANGE = 0, 1, 2, 3
-IMQ_ERR_BUFFER, IMQ_ERR_TIMEOUT, IMQ_ERR_CUDA, IMQ_ERR_UNSUPPORTED, IMQ_ERR_PLAN = 4, 5, 6, 7, 8
+IMQ_ERR_BUFFER, IMQ_ERR_TIMEOUT, IMQ_ERR_CUDA, IMQ_ERR_UNSUPPORTED, IMQ_ERR_PLAN, IMQ_ERR_BOUNDS = 4, 5, 6, 7, 8, 9
 # dtypes
 IMQ_F32, IMQ_BF16, IMQ_I16, IMQ_I32, IMQ_I64 = 0, 1, 2, 3, 4
 # quantisation groups
@@ -116,7 +117,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m bit_integer_gemm_b200.build`")
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m bit_integer_gemm_b200.build`"
+                               + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
         L = ctypes.CDLL(LIB_PATH)
         for name, args in SIGNATURES.items():
             fn = getattr(L, name)

@@ -559,6 +559,7 @@ const char* imq_status_str(imq_status s) {
     case IMQ_ERR_CUDA: return "CUDA runtime error";
     case IMQ_ERR_UNSUPPORTED: return "unsupported input";
     case IMQ_ERR_PLAN: return "input not covered by the plan";
+    case IMQ_ERR_BOUNDS: return "plan index outside the plan's sizes (debug build)";
   }
   return "unknown status";
 }

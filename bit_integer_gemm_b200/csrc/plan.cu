@@ -796,6 +796,101 @@ __global__ void __launch_bounds__(1024) k_plan_maps(const __grid_constant__ Maps
   outer_map_class(cls[j.cls0 + ci], j.lv, j.n, j.G, j.pos, j.src, j.grpL, j.grpN);
 }
 
+#ifdef IMQ_DEBUG
+// ------------------------------------------------------------------------------------------------
+// Debug build only: every index of a finished plan that the unpack and GEMM kernels read, checked
+// against the plan's sizes.  A violation records IMQ_ERR_BOUNDS in the status word (nothing traps and
+// nothing else changes); the checks run right after the maps kernel, in stream order.
+// ------------------------------------------------------------------------------------------------
+struct CheckGroup {
+  int64_t off, len, padded;
+  int32_t e;
+};
+struct CheckOuter {
+  int on;                 // the operand is unpacked OUTER
+  int64_t n, n_unp, ngrp;  // source lines, unpacked lines, groups of IMQ_*_GROUP lines
+  const int8_t* lv;        // levels of the source lines
+  const int32_t* pos;
+  const int32_t* src;
+  const int32_t* grpL;
+  const int32_t* grpN;
+};
+struct CheckArgs {
+  int64_t K, K_unp;
+  int a_inner, b_inner;
+  const int8_t* lva;  // levels of A's columns
+  const int8_t* lvb;  // levels of B's rows
+  const int32_t* tK;
+  const int8_t* lAk;
+  const int8_t* lBk;
+  const int32_t* blk16;
+  int ng;
+  CheckGroup grp[IMQ_MAX_GROUPS];
+  CheckOuter o[2];
+  int32_t* status;
+};
+
+__device__ __forceinline__ void check(bool ok, int32_t* status) {
+  if (!ok) set_status(status, IMQ_ERR_BOUNDS);
+}
+
+__global__ void __launch_bounds__(256) k_plan_check(const __grid_constant__ CheckArgs c) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  // inner positions: source index, levels, exponent and padding of their group
+  for (int64_t p = i0; p < c.K_unp; p += stride) {
+    int g = -1;
+    for (int k = 0; k < c.ng; ++k)
+      if (p >= c.grp[k].off && p < c.grp[k].off + c.grp[k].padded) g = k;
+    check(g >= 0, c.status);
+    if (g < 0) continue;
+    const int32_t t = c.tK[p];
+    const bool real = p < c.grp[g].off + c.grp[g].len;
+    check(real ? (t >= 0 && t < c.K) : t == -1, c.status);
+    if (t < 0 || t >= c.K) continue;
+    const int la = c.a_inner ? c.lva[t] : 1, lb = c.b_inner ? c.lvb[t] : 1;
+    const int lA = c.lAk[p], lB = c.lBk[p];
+    check(lA >= 0 && lA < la && lB >= 0 && lB < lb && lA + lB == c.grp[g].e, c.status);
+  }
+  // 16-position blocks: a run entry must describe the positions exactly
+  for (int64_t b = i0; b < c.K_unp / 16; b += stride) {
+    const int32_t v = c.blk16[b];
+    if (v == -1) continue;
+    const int32_t t0 = v >= 0 ? v : -v - 2;
+    check(v < 0 || (t0 & 15) == 0, c.status);
+    check(t0 >= 0 && t0 + 16 <= c.K, c.status);
+    for (int k = 0; k < 16; ++k)
+      check(c.tK[b * 16 + k] == t0 + k && c.lAk[b * 16 + k] == c.lAk[b * 16] && c.lBk[b * 16 + k] == c.lBk[b * 16],
+            c.status);
+  }
+  // OUTER lines: every source line's L lines inside the unpacked operand and inside one group of its level,
+  // every used unpacked line pointing back at its source, every group's level and count in range
+  for (int o = 0; o < 2; ++o) {
+    const CheckOuter& q = c.o[o];
+    if (!q.on) continue;
+    check(q.ngrp * 32 == q.n_unp, c.status);
+    for (int64_t i = i0; i < q.n; i += stride) {
+      const int L = q.lv[i];
+      const int64_t u = q.pos[i];
+      check(L >= 1 && L <= 31 && u >= 0 && u + L <= q.n_unp, c.status);
+      if (!(L >= 1 && L <= 31 && u >= 0 && u + L <= q.n_unp)) continue;
+      check(u / 32 == (u + L - 1) / 32 && q.grpL[u / 32] == L && (u % 32) % L == 0 && (u % 32) / L < q.grpN[u / 32],
+            c.status);
+      for (int l = 0; l < L; ++l) check(q.src[u + l] == (int32_t)i, c.status);
+    }
+    for (int64_t u = i0; u < q.n_unp; u += stride) {
+      const int32_t s = q.src[u];
+      check(s >= -1 && s < q.n, c.status);
+      if (s >= 0 && s < q.n) check(q.pos[s] <= u && u < q.pos[s] + q.lv[s], c.status);
+    }
+    for (int64_t g = i0; g < q.ngrp; g += stride) {
+      const int L = q.grpL[g], nn = q.grpN[g];
+      check(L >= 1 && L <= 31 && nn >= 0 && nn * L <= 32, c.status);
+    }
+  }
+}
+#endif
+
 // ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
@@ -1512,6 +1607,42 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
     if (blocks > 0) k_plan_maps<<<blocks, 1024, 0, st>>>(m);
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
+#ifdef IMQ_DEBUG
+  {
+    // the exponent groups on the host: contiguous, padded to IMQ_INNER_PAD, filling K_unp
+    int64_t next = 0;
+    for (int g = 0; g < ng; ++g) {
+      const imq_group& gr = pl->groups[g];
+      if (gr.k_offset != next || gr.k_len > gr.k_len_padded || gr.k_len_padded % IMQ_INNER_PAD ||
+          gr.k_len_padded - gr.k_len >= IMQ_INNER_PAD)
+        return fail(IMQ_ERR_BOUNDS);
+      next += gr.k_len_padded;
+    }
+    if (next != I.K_unp) return fail(IMQ_ERR_BOUNDS);
+    CheckArgs c;
+    memset(&c, 0, sizeof(c));
+    c.K = K;
+    c.K_unp = I.K_unp;
+    c.a_inner = a_inner;
+    c.b_inner = b_inner;
+    c.lva = pl->lv_a_col;
+    c.lvb = pl->lv_b_row;
+    c.tK = pl->tK;
+    c.lAk = pl->lAk;
+    c.lBk = pl->lBk;
+    c.blk16 = pl->blk16;
+    c.ng = ng;
+    for (int g = 0; g < ng; ++g)
+      c.grp[g] = CheckGroup{pl->groups[g].k_offset, pl->groups[g].k_len, pl->groups[g].k_len_padded, pl->groups[g].e};
+    c.o[0] = CheckOuter{a_outer ? 1 : 0, M, I.M_unp, pl->n_grp_a, pl->lv_a_row, pl->posA, pl->srcA, pl->grpA_L,
+                        pl->grpA_n};
+    c.o[1] = CheckOuter{b_outer ? 1 : 0, N, I.N_unp, pl->n_grp_b, pl->lv_b_col, pl->posB, pl->srcB, pl->grpB_L,
+                        pl->grpB_n};
+    c.status = ds->status;
+    k_plan_check<<<(unsigned)ds->num_sms, 256, 0, st>>>(c);
+    if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  }
+#endif
   *out = pl;
   return IMQ_OK;
 }

@@ -54,7 +54,8 @@ typedef enum {
   IMQ_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out                                    */
   IMQ_ERR_CUDA = 6,        /* a CUDA runtime call failed                                                 */
   IMQ_ERR_UNSUPPORTED = 7, /* legal input outside what the kernels implement (see imq_plan)             */
-  IMQ_ERR_PLAN = 8         /* imq_rtn_quantize_unpack: a quantised entry above the plan's max |A[:, t]| */
+  IMQ_ERR_PLAN = 8,        /* imq_rtn_quantize_unpack: a quantised entry above the plan's max |A[:, t]| */
+  IMQ_ERR_BOUNDS = 9       /* debug build (IMQ_DEBUG) only: a plan index outside the plan's sizes        */
 } imq_status;
 
 typedef enum { IMQ_F32 = 0, IMQ_BF16 = 1, IMQ_I16 = 2, IMQ_I32 = 3, IMQ_I64 = 4 } imq_dtype;

@@ -38,6 +38,13 @@ def test_library_builds_and_exports_every_declared_symbol():
         assert len(imq.SIGNATURES[name]) == nargs, f"{name}: binding has {len(imq.SIGNATURES[name])} args, header {nargs}"
 
 
+def test_debug_library_builds_and_exports_every_declared_symbol():
+    from bit_integer_gemm_b200 import build as b
+    lib = ctypes.CDLL(b.build(debug=True))
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} not exported by the debug build"
+
+
 def test_struct_layouts_match_header():
     import bit_integer_gemm_b200 as imq
     # imq_plan_info: 4 int32, 9 int64, 2 double, 6 int32, 8 int64, size_t
