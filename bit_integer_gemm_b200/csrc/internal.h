@@ -84,8 +84,14 @@ struct imq_plan {
   int32_t* tK;      // [K_unp] source inner index, -1 on padding
   int8_t* lAk;      // [K_unp] digit level of A at that inner position
   int8_t* lBk;      // [K_unp] digit level of B
-  int32_t* blk16;   // [K_unp/16] when positions 16c..16c+15 hold t0..t0+15 with one (lA, lB) pair: t0
-                    // if t0 % 16 == 0, else -(t0 + 2); otherwise -1 (the unpackers copy runs)
+  int32_t* perm;    // [K] staging order: the inner index at each staging position (indices grouped by
+                    // their (A column, B row) level class); null when the order is the identity
+  int32_t* pinv;    // [K] staging position of each inner index; null with perm
+  int32_t* tJ;      // [K_unp] staging position of the index at each inner position, -1 on padding (tK
+                    // itself when perm is null)
+  int32_t* blk16;   // [K_unp/16] when positions 16c..16c+15 hold the indices at staging positions
+                    // j0..j0+15 with one (lA, lB) pair: j0 if j0 % 16 == 0, else -(j0 + 2); otherwise -1
+                    // (the unpackers stage a source line in staging order and copy runs)
   int32_t* posA;    // [M] first unpacked row of each source row (A OUTER)
   int32_t* srcA;    // [M_unp] source row of each unpacked row, -1 unused (A OUTER)
   int32_t* grpA_L;  // [M_unp / IMQ_A_GROUP] level of each row group

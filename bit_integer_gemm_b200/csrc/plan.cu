@@ -13,9 +13,12 @@
 //                  histograms, the joint histogram of (level of A column t, level of B row t), and the
 //                  exact 128-bit bound sum_t max|A[:,t]| * max|B[t,:]|
 //   -- the summary (a few KB) is read back; the host fixes directions, groups and sizes --
-//   k_plan_maps    one launch: one CTA per exponent group of the inner dimension (stream compaction of
-//                  the inner indices of each of its (lA, lB) segments, padding, 16-position blocks) and
-//                  one CTA per OUTER level class (stable compaction of the lines of that level into groups)
+//   k_plan_order   (plans that use a staging order) one CTA per (A column, B row) level class: the
+//                  class's inner indices at their staging positions
+//   k_plan_maps    one launch: one CTA per exponent group of the inner dimension (each of its (lA, lB)
+//                  segments as ranges of the staging order, padding, 16-position blocks) and one CTA per
+//                  OUTER level class (stable compaction of the lines of that level into groups)
+#include <math.h>
 #include <stddef.h>
 #include <string.h>
 
@@ -644,53 +647,109 @@ struct InnerGroup {
   int32_t seg0, nseg;
 };
 
-// The inner map of one exponent group (one CTA of 1024 threads): each segment's inner indices t (with
-// line levels la > seg.la and lb > seg.lb) in increasing order, then the padding, then blk16 for the
-// group's 16-position blocks: blk16[c] = t0 when block c holds t0..t0+15 (t0 % 16 == 0) with one
-// (lA, lB) pair, else -1.
-__device__ void inner_map_group(const InnerGroup grp, const InnerSeg* __restrict__ segs,
+// The staging order of the inner indices.  Index t belongs to class (ea, eb): ea = level of A column t
+// when A is unpacked INNER (else 1), eb = level of B row t when B is (else 1).  The staging order lists
+// the classes in descending (ea, eb), each class's indices ascending, so that the indices a segment
+// (lA, lB) holds -- every class with ea > lA and eb > lB -- are, for each ea, one contiguous range of
+// staging positions.  E[ea * ew + s] (ew = maxlb + 1) is the first staging position past the classes
+// (ea, eb) with eb > s: class (ea, eb) occupies [E[ea*ew + eb], E[ea*ew + eb - 1]).  perm[j] is the index at
+// staging position j and pinv its inverse; both are null when the order is the identity (one class, or
+// a plan whose segments keep most 16-position blocks runs in index order).
+struct StageOrder {
+  const int32_t* E;
+  int ew;
+  int maxla, maxlb;
+  int32_t* perm;
+  int32_t* pinv;
+};
+
+// The staging order of one class (one CTA of 1024 threads): its indices, ascending, at its positions.
+__device__ void stage_class(int ea, int eb, const StageOrder& so, const int8_t* __restrict__ lva,
+                            const int8_t* __restrict__ lvb, int a_inner, int b_inner, int64_t K) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int64_t j0 = so.E[ea * so.ew + eb];
+  if (so.E[ea * so.ew + eb - 1] == j0) return;  // empty class
+  int64_t rank0 = 0;
+  for (int64_t t0 = 0; t0 < K; t0 += 1024) {
+    const int64_t t = t0 + threadIdx.x;
+    int pred = 0;
+    if (t < K) pred = (a_inner ? lva[t] : 1) == ea && (b_inner ? lvb[t] : 1) == eb;
+    const int r = block_rank(pred, warp_tot, &total);
+    if (pred) {
+      const int64_t j = j0 + rank0 + r;
+      so.perm[j] = (int32_t)t;
+      so.pinv[t] = (int32_t)j;
+    }
+    __syncthreads();
+    rank0 += total;
+    __syncthreads();
+  }
+}
+
+// The inner map of one exponent group (one CTA of 1024 threads): each segment (lA, lB) holds the inner
+// indices of the classes ea > lA, eb > lB -- with a staging order, in that order (for each ea, from the
+// largest, one range of staging positions), else ascending -- then the padding, then blk16 for the
+// group's 16-position blocks: blk16[c] = j0
+// when block c holds the indices at staging positions j0..j0+15 with one (lA, lB) pair (j0 % 16 == 0),
+// -(j0 + 2) for such a run at any other j0, else -1.  tJ[p] = staging position of position p's index.
+__device__ void inner_map_group(const InnerGroup grp, const InnerSeg* __restrict__ segs, const StageOrder& so,
                                 const int8_t* __restrict__ lva, const int8_t* __restrict__ lvb, int a_inner,
-                                int b_inner, int64_t K, int32_t* __restrict__ tK, int8_t* __restrict__ lAk,
+                                int b_inner, int64_t K, int32_t* tK, int32_t* tJ, int8_t* __restrict__ lAk,
                                 int8_t* __restrict__ lBk, int32_t* __restrict__ blk16) {
   __shared__ int warp_tot[32];
   __shared__ int total;
   int64_t base = grp.k0;
   for (int si = 0; si < grp.nseg; ++si) {
     const InnerSeg sg = segs[grp.seg0 + si];
-    for (int64_t t0 = 0; t0 < K; t0 += 1024) {
-      const int64_t t = t0 + threadIdx.x;
-      int pred = 0;
-      if (t < K) {
-        const int la = a_inner ? lva[t] : 1;
-        const int lb = b_inner ? lvb[t] : 1;
-        pred = (la > sg.la) && (lb > sg.lb);
+    if (so.perm) {
+      // the segment's ranges of the staging order, one per A level ea > lA
+      for (int ea = so.maxla; ea > sg.la; --ea) {
+        const int64_t jb = so.E[ea * so.ew + so.maxlb], je = so.E[ea * so.ew + sg.lb];
+        for (int64_t i = threadIdx.x; i < je - jb; i += blockDim.x) {
+          const int64_t j = jb + i, q = base + i;
+          tK[q] = so.perm[j];
+          tJ[q] = (int32_t)j;
+          lAk[q] = (int8_t)sg.la;
+          lBk[q] = (int8_t)sg.lb;
+        }
+        base += je - jb;
       }
-      const int r = block_rank(pred, warp_tot, &total);
-      if (pred) {
-        tK[base + r] = (int32_t)t;
-        lAk[base + r] = (int8_t)sg.la;
-        lBk[base + r] = (int8_t)sg.lb;
+    } else {
+      // index order: the segment's indices by stream compaction
+      for (int64_t t0 = 0; t0 < K; t0 += 1024) {
+        const int64_t t = t0 + threadIdx.x;
+        int pred = 0;
+        if (t < K) pred = ((a_inner ? lva[t] : 1) > sg.la) && ((b_inner ? lvb[t] : 1) > sg.lb);
+        const int r = block_rank(pred, warp_tot, &total);
+        if (pred) {
+          tK[base + r] = (int32_t)t;
+          tJ[base + r] = (int32_t)t;
+          lAk[base + r] = (int8_t)sg.la;
+          lBk[base + r] = (int8_t)sg.lb;
+        }
+        __syncthreads();
+        base += total;
+        __syncthreads();
       }
-      __syncthreads();
-      base += total;
-      __syncthreads();
     }
   }
   for (int64_t q = base + threadIdx.x; q < grp.k0 + grp.kpad; q += blockDim.x) {
     tK[q] = -1;
+    tJ[q] = -1;
     lAk[q] = 0;
     lBk[q] = 0;
   }
   __syncthreads();  // the block's writes above are visible to all its threads after this
   for (int64_t c = grp.k0 / 16 + threadIdx.x; c < (grp.k0 + grp.kpad) / 16; c += blockDim.x) {
-    const int32_t* t = tK + c * 16;
-    const int32_t t0 = t[0];
-    bool run = t0 >= 0;
+    const int32_t* j = tJ + c * 16;
+    const int32_t j0 = j[0];
+    bool run = j0 >= 0;
     for (int k = 1; k < 16 && run; ++k)
-      run = t[k] == t0 + k && lAk[c * 16 + k] == lAk[c * 16] && lBk[c * 16 + k] == lBk[c * 16];
-    // t0 for an aligned run, -(t0 + 2) for a run starting elsewhere (the staged unpacker reads those
-    // with unaligned loads; every other reader treats a negative entry as a gathered block), else -1
-    blk16[c] = !run ? -1 : ((t0 & 15) == 0 ? t0 : -(t0 + 2));
+      run = j[k] == j0 + k && lAk[c * 16 + k] == lAk[c * 16] && lBk[c * 16 + k] == lBk[c * 16];
+    // the staged unpackers read an unaligned run with unaligned loads; every other reader treats a
+    // negative entry as a gathered block
+    blk16[c] = !run ? -1 : ((j0 & 15) == 0 ? j0 : -(j0 + 2));
   }
 }
 
@@ -752,25 +811,34 @@ __device__ void outer_map_class(const OuterClass c, const int8_t* __restrict__ l
 constexpr int kParamSegs = 24;
 constexpr int kParamCls = 24;
 constexpr int kParamGrps = 16;
+constexpr int kParamE = 100;
 struct MapsTables {
   InnerSeg segs[kParamSegs];
   OuterClass cls[kParamCls];
   InnerGroup grps[kParamGrps];
+  int32_t E[kParamE];
 };
 
-// Stage 2 of a plan in one launch: blocks [0, ngrp) build the inner map of one exponent group each, the
-// next a.ncls blocks one OUTER class of A each, the rest one OUTER class of B each.
+// Stage 2 of a plan.  k_plan_order (only when the staging order is not the identity): one CTA per class
+// (ea, eb), blockIdx.x = (maxla - ea) * maxlb + (maxlb - eb).  Then k_plan_maps: blocks [0, ngrp) build the
+// inner map of one exponent group each, the next a.ncls blocks one OUTER class of A each, the rest one
+// OUTER class of B each.
 struct MapsArgs {
-  int inline_tables;       // 1: the tables are `t` below, 0: the device copies at grps / segs / cls
+  int inline_tables;       // 1: the tables are `t` below, 0: the device copies at grps / segs / cls / E
   const InnerGroup* grps;
   int ngrp;
   const InnerSeg* segs;
   const OuterClass* cls;
+  const int32_t* E;
+  int ew, maxla, maxlb;
   const int8_t* lva;
   const int8_t* lvb;
   int a_inner, b_inner;
   int64_t K;
+  int32_t* perm;
+  int32_t* pinv;
   int32_t* tK;
+  int32_t* tJ;
   int8_t* lAk;
   int8_t* lBk;
   int32_t* blk16;
@@ -780,13 +848,24 @@ struct MapsArgs {
 // kernel parameters above 4 KB need CUDA 12.1 or later; the limit there is 32 764 bytes
 static_assert(sizeof(MapsArgs) <= 32764, "plan tables exceed the kernel parameter limit");
 
+__device__ __forceinline__ StageOrder stage_order(const MapsArgs& m) {
+  return StageOrder{m.inline_tables ? m.t.E : m.E, m.ew, m.maxla, m.maxlb, m.perm, m.pinv};
+}
+
+__global__ void __launch_bounds__(1024) k_plan_order(const __grid_constant__ MapsArgs m) {
+  const int bx = (int)blockIdx.x;
+  const int ea = m.maxla - bx / m.maxlb, eb = m.maxlb - bx % m.maxlb;
+  stage_class(ea, eb, stage_order(m), m.lva, m.lvb, m.a_inner, m.b_inner, m.K);
+}
+
 __global__ void __launch_bounds__(1024) k_plan_maps(const __grid_constant__ MapsArgs m) {
   const InnerSeg* segs = m.inline_tables ? m.t.segs : m.segs;
   const OuterClass* cls = m.inline_tables ? m.t.cls : m.cls;
   const InnerGroup* grps = m.inline_tables ? m.t.grps : m.grps;
   const int bx = (int)blockIdx.x;
   if (bx < m.ngrp) {
-    inner_map_group(grps[bx], segs, m.lva, m.lvb, m.a_inner, m.b_inner, m.K, m.tK, m.lAk, m.lBk, m.blk16);
+    inner_map_group(grps[bx], segs, stage_order(m), m.lva, m.lvb, m.a_inner, m.b_inner, m.K, m.tK, m.tJ, m.lAk,
+                    m.lBk, m.blk16);
     return;
   }
   const int ob = bx - m.ngrp;
@@ -821,6 +900,9 @@ struct CheckArgs {
   const int8_t* lva;  // levels of A's columns
   const int8_t* lvb;  // levels of B's rows
   const int32_t* tK;
+  const int32_t* tJ;    // staging position of each inner position's index (tK itself when perm is null)
+  const int32_t* perm;  // staging order (null: the identity)
+  const int32_t* pinv;
   const int8_t* lAk;
   const int8_t* lBk;
   const int32_t* blk16;
@@ -847,20 +929,31 @@ __global__ void __launch_bounds__(256) k_plan_check(const __grid_constant__ Chec
     const int32_t t = c.tK[p];
     const bool real = p < c.grp[g].off + c.grp[g].len;
     check(real ? (t >= 0 && t < c.K) : t == -1, c.status);
+    check(c.tJ[p] == (t >= 0 && t < c.K && c.pinv ? c.pinv[t] : t), c.status);
     if (t < 0 || t >= c.K) continue;
     const int la = c.a_inner ? c.lva[t] : 1, lb = c.b_inner ? c.lvb[t] : 1;
     const int lA = c.lAk[p], lB = c.lBk[p];
     check(lA >= 0 && lA < la && lB >= 0 && lB < lb && lA + lB == c.grp[g].e, c.status);
   }
-  // 16-position blocks: a run entry must describe the positions exactly
+  // the staging order: a permutation of the inner indices
+  if (c.perm) {
+    for (int64_t j = i0; j < c.K; j += stride) {
+      const int32_t t = c.perm[j];
+      check(t >= 0 && t < c.K, c.status);
+      if (t >= 0 && t < c.K) check(c.pinv[t] == (int32_t)j, c.status);
+    }
+  }
+  // 16-position blocks: a run entry must describe the positions exactly (staging positions j0..j0+15)
   for (int64_t b = i0; b < c.K_unp / 16; b += stride) {
     const int32_t v = c.blk16[b];
     if (v == -1) continue;
-    const int32_t t0 = v >= 0 ? v : -v - 2;
-    check(v < 0 || (t0 & 15) == 0, c.status);
-    check(t0 >= 0 && t0 + 16 <= c.K, c.status);
+    const int32_t j0 = v >= 0 ? v : -v - 2;
+    check(v < 0 || (j0 & 15) == 0, c.status);
+    check(j0 >= 0 && j0 + 16 <= c.K, c.status);
+    if (!(j0 >= 0 && j0 + 16 <= c.K)) continue;
     for (int k = 0; k < 16; ++k)
-      check(c.tK[b * 16 + k] == t0 + k && c.lAk[b * 16 + k] == c.lAk[b * 16] && c.lBk[b * 16 + k] == c.lBk[b * 16],
+      check(c.tK[b * 16 + k] == (c.perm ? c.perm[j0 + k] : j0 + k) && c.tJ[b * 16 + k] == j0 + k &&
+                c.lAk[b * 16 + k] == c.lAk[b * 16] && c.lBk[b * 16 + k] == c.lBk[b * 16],
             c.status);
   }
   // OUTER lines: every source line's L lines inside the unpacked operand and inside one group of its level,
@@ -978,7 +1071,7 @@ struct PlanJob {
   imq_plan_t* pl = nullptr;
   char* blk1 = nullptr;
   Summary* dsum = nullptr;
-  size_t o_segs = 0, o_cls = 0, o_grps = 0;
+  size_t o_segs = 0, o_cls = 0, o_grps = 0, o_E = 0;
   uint32_t seq = 0;
 };
 
@@ -995,7 +1088,8 @@ imq_status plan_fail(imq_plan_t* pl, imq_status e, cudaStream_t st) {
 // Makes sure the pinned summary slots and table staging of this device exist (nslots slots).
 imq_status pinned_ready(Pinned& pin, int nslots) {
   const size_t staging_bytes = align_up(sizeof(InnerSeg) * kLv * kLv, 256) +
-                               align_up(sizeof(OuterClass) * 2 * kLv, 256) + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
+                               align_up(sizeof(OuterClass) * 2 * kLv, 256) +
+                               align_up(sizeof(InnerGroup) * IMQ_MAX_GROUPS, 256) + sizeof(int32_t) * kLv * kLv;
   if (pin.cap < nslots) {
     // every earlier plan has read its summary before returning, so the old slots are idle
     if (pin.sum) cudaFreeHost(pin.sum);
@@ -1026,8 +1120,8 @@ imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaS
   const imq_strategy strategy = job.strategy;
   const int32_t *a_rowmax = job.a_rowmax, *a_colmax = job.a_colmax, *b_rowmax = job.b_rowmax,
                 *b_colmax = job.b_colmax;
-  const size_t tables_bytes =
-      sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv + sizeof(InnerGroup) * IMQ_MAX_GROUPS;
+  const size_t tables_bytes = sizeof(InnerSeg) * kLv * kLv + sizeof(OuterClass) * 2 * kLv +
+                              sizeof(InnerGroup) * IMQ_MAX_GROUPS + sizeof(int32_t) * kLv * kLv;
   imq_plan_t* pl = new imq_plan_t;
   memset(pl, 0, sizeof(*pl));
   pl->host_tables = malloc(tables_bytes);
@@ -1064,6 +1158,8 @@ imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaS
   off = align_up(off + sizeof(OuterClass) * 2 * kLv, 256);
   const size_t o_grps = off;
   off = align_up(off + sizeof(InnerGroup) * IMQ_MAX_GROUPS, 256);
+  const size_t o_E = off;
+  off = align_up(off + sizeof(int32_t) * kLv * kLv, 256);
   // hybrid scratch: per matrix (A: M outer lines, B: N outer lines; K inner indices each) the counts and
   // the two histograms (zeroed together), then the least-count tables (filled with kHybInf), then the
   // threshold and the carried levels
@@ -1237,6 +1333,7 @@ imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaS
   job.o_segs = o_segs;
   job.o_cls = o_cls;
   job.o_grps = o_grps;
+  job.o_E = o_E;
   job.seq = la.seq;
   return IMQ_OK;
 }
@@ -1292,8 +1389,9 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
   InnerSeg* hsegs = static_cast<InnerSeg*>(pl->host_tables);
   OuterClass* hcls = reinterpret_cast<OuterClass*>(hsegs + kLv * kLv);
   InnerGroup* hgrps = reinterpret_cast<InnerGroup*>(hcls + 2 * kLv);
+  int32_t* hE = reinterpret_cast<int32_t*>(hgrps + IMQ_MAX_GROUPS);
   char* blk1 = job.blk1;
-  const size_t o_segs = job.o_segs, o_cls = job.o_cls, o_grps = job.o_grps;
+  const size_t o_segs = job.o_segs, o_cls = job.o_cls, o_grps = job.o_grps, o_E = job.o_E;
   // a pending kernel error (e.g. a non-finite quantiser input) is reported before planning
   if (S.status != IMQ_OK) return fail((imq_status)S.status);
 
@@ -1391,6 +1489,7 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
   };
   int nseg = 0;
   int64_t koff = 0, keff = 0;
+  double scattered = 0.0;
   int ng = 0;
   for (int e = 0; e <= maxla + maxlb - 2; ++e) {
     int64_t glen = 0;
@@ -1400,6 +1499,9 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
       if (sb < 0 || sb >= maxlb) continue;
       const int64_t n = seg_len(sa, sb);
       if (n == 0) continue;
+      // positions of this segment expected outside 16-long runs of consecutive indices, were its indices
+      // placed at random among the K (a segment of density d keeps a block a run with probability d^15)
+      scattered += (double)n * (1.0 - pow((double)n / (double)K, 15.0));
       hsegs[nseg].la = sa;
       hsegs[nseg].lb = sb;
       hsegs[nseg].off = koff + glen;
@@ -1423,6 +1525,34 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
   I.n_groups = ng;
   I.K_unp = koff;
   I.K_eff = keff;
+
+  // The staging order of the inner indices (StageOrder): classes (ea, eb) in descending order, their sizes
+  // from the joint level histogram.  With one non-empty class the order is the identity.
+  const int ew = maxlb + 1;
+  int nonempty = 0;
+  {
+    std::vector<int64_t> ccount((size_t)(maxla + 1) * ew, 0);
+    for (int x = 1; x <= (int)lmax[1]; ++x)
+      for (int y = 1; y <= (int)lmax[2]; ++y) {
+        const int ea = a_inner ? x : 1, eb = b_inner ? y : 1;
+        ccount[(size_t)ea * ew + eb] += S.joint[x][y];
+      }
+    int64_t j = 0;
+    for (int ea = maxla; ea >= 1; --ea) {
+      hE[ea * ew + maxlb] = (int32_t)j;
+      for (int eb = maxlb; eb >= 1; --eb) {
+        const int64_t c = ccount[(size_t)ea * ew + eb];
+        nonempty += c > 0;
+        j += c;
+        hE[ea * ew + eb - 1] = (int32_t)j;
+      }
+    }
+    for (int e2 = 0; e2 < ew; ++e2) hE[e2] = (int32_t)j;  // row 0: past every class
+    if (j != K) return fail(IMQ_ERR_CUDA);                // the histogram counts every inner index once
+  }
+  // The staging order costs a scattered staging of every source line; it pays when index order would leave
+  // many blocks gathered (segments of middling density: both operands unpacked INNER, typically).
+  const bool permuted = nonempty > 1 && koff > 0 && scattered > 0.25 * (double)keff;
 
   // outer sizes
   int ncls = 0;
@@ -1530,6 +1660,12 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
   const size_t o_lAk = off2; off2 = align_up(off2 + (size_t)I.K_unp, 256);
   const size_t o_lBk = off2; off2 = align_up(off2 + (size_t)I.K_unp, 256);
   const size_t o_blk = off2; off2 = align_up(off2 + (size_t)(I.K_unp / 16) * 4, 256);
+  size_t o_perm = 0, o_pinv = 0, o_tJ = 0;
+  if (permuted) {
+    o_perm = off2; off2 = align_up(off2 + (size_t)K * 4, 256);
+    o_pinv = off2; off2 = align_up(off2 + (size_t)K * 4, 256);
+    o_tJ = off2; off2 = align_up(off2 + (size_t)I.K_unp * 4, 256);
+  }
   size_t o_posA = 0, o_srcA = 0, o_gLA = 0, o_gNA = 0, o_posB = 0, o_srcB = 0, o_gLB = 0, o_gNB = 0;
   if (a_outer) {
     o_posA = off2; off2 = align_up(off2 + (size_t)M * 4, 256);
@@ -1554,6 +1690,9 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
   pl->lAk = reinterpret_cast<int8_t*>(b2 + o_lAk);
   pl->lBk = reinterpret_cast<int8_t*>(b2 + o_lBk);
   pl->blk16 = reinterpret_cast<int32_t*>(b2 + o_blk);
+  pl->perm = permuted ? reinterpret_cast<int32_t*>(b2 + o_perm) : nullptr;
+  pl->pinv = permuted ? reinterpret_cast<int32_t*>(b2 + o_pinv) : nullptr;
+  pl->tJ = permuted ? reinterpret_cast<int32_t*>(b2 + o_tJ) : pl->tK;
   if (a_outer) {
     pl->posA = reinterpret_cast<int32_t*>(b2 + o_posA);
     pl->srcA = reinterpret_cast<int32_t*>(b2 + o_srcA);
@@ -1568,11 +1707,13 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
   }
   if (ng > 0 || ncls > 0) {
     MapsArgs m;
-    m.inline_tables = (nseg <= kParamSegs && ncls <= kParamCls && ng <= kParamGrps) ? 1 : 0;
+    const int nE = (maxla + 1) * ew;
+    m.inline_tables = (nseg <= kParamSegs && ncls <= kParamCls && ng <= kParamGrps && nE <= kParamE) ? 1 : 0;
     if (m.inline_tables) {
       memcpy(m.t.segs, hsegs, sizeof(InnerSeg) * (size_t)nseg);
       memcpy(m.t.cls, hcls, sizeof(OuterClass) * (size_t)ncls);
       memcpy(m.t.grps, hgrps, sizeof(InnerGroup) * (size_t)ng);
+      memcpy(m.t.E, hE, sizeof(int32_t) * (size_t)nE);
     } else {
       // one upload from pinned staging (an asynchronous copy; pageable memory would be staged by the
       // driver first); the staging is reused once the previous plan's upload has completed
@@ -1581,7 +1722,8 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
       memcpy(stg, hsegs, sizeof(InnerSeg) * (size_t)nseg);
       memcpy(stg + (o_cls - o_segs), hcls, sizeof(OuterClass) * (size_t)ncls);
       memcpy(stg + (o_grps - o_segs), hgrps, sizeof(InnerGroup) * (size_t)ng);
-      if (cudaMemcpyAsync(dsegs, stg, (o_grps - o_segs) + sizeof(InnerGroup) * (size_t)ng, cudaMemcpyHostToDevice,
+      memcpy(stg + (o_E - o_segs), hE, sizeof(int32_t) * (size_t)nE);
+      if (cudaMemcpyAsync(dsegs, stg, (o_E - o_segs) + sizeof(int32_t) * (size_t)nE, cudaMemcpyHostToDevice,
                           st) != cudaSuccess ||
           cudaEventRecord(pin.tables_done, st) != cudaSuccess)
         return fail(IMQ_ERR_CUDA);
@@ -1590,12 +1732,19 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
     m.cls = dcls;
     m.ngrp = ng;
     m.segs = dsegs;
+    m.E = reinterpret_cast<const int32_t*>(blk1 + o_E);
+    m.ew = ew;
+    m.maxla = maxla;
+    m.maxlb = maxlb;
     m.lva = pl->lv_a_col;
     m.lvb = pl->lv_b_row;
     m.a_inner = a_inner;
     m.b_inner = b_inner;
     m.K = K;
+    m.perm = pl->perm;
+    m.pinv = pl->pinv;
     m.tK = pl->tK;
+    m.tJ = pl->tJ;
     m.lAk = pl->lAk;
     m.lBk = pl->lBk;
     m.blk16 = pl->blk16;
@@ -1603,6 +1752,7 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
            pl->grpA_L, pl->grpA_n};
     m.b = {cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
            pl->grpB_L, pl->grpB_n};
+    if (permuted) k_plan_order<<<maxla * maxlb, 1024, 0, st>>>(m);
     const int blocks = ng + m.a.ncls + m.b.ncls;
     if (blocks > 0) k_plan_maps<<<blocks, 1024, 0, st>>>(m);
   }
@@ -1628,6 +1778,9 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
     c.lva = pl->lv_a_col;
     c.lvb = pl->lv_b_row;
     c.tK = pl->tK;
+    c.tJ = pl->tJ;
+    c.perm = pl->perm;
+    c.pinv = pl->pinv;
     c.lAk = pl->lAk;
     c.lBk = pl->lBk;
     c.blk16 = pl->blk16;

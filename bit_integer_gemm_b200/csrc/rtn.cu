@@ -907,36 +907,35 @@ __global__ void __launch_bounds__(NT) k_rtn_rows_reg(const uint16_t* __restrict_
   }
 }
 
-// bf16 transpose through shared memory: X (rows x cols, leading dimension ld) into Y (cols x rows, dense),
-// 64 x 64 tiles, 16-byte loads and stores (rows and cols multiples of 8, X and ld 16-byte aligned).
+// Word k (0..3) of a 16-byte vector (k known at compile time after unrolling).
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int k) {
+  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+}
+
+// bf16 transpose in registers: X (rows x cols, leading dimension ld) into Y (cols x rows, dense).  A
+// thread moves one 8 x 8 block: eight 16-byte row loads, the 8 x 8 transpose of its 16-bit entries by
+// byte permutes (one per output word: the same half of one word of two consecutive input rows), eight
+// 16-byte stores.  A warp covers 64 rows x 32 columns (lane = 4 column blocks x 8 row blocks), so that a
+// load instruction reads 64 contiguous bytes of each of 8 rows and a store instruction 128 contiguous
+// bytes of each of 4 output rows; a CTA of 8 warps covers 64 rows x 256 columns.  No shared memory.
+// rows and cols are multiples of 8; X, ld and Y 16-byte aligned.
 __global__ void __launch_bounds__(256) k_transpose_bf16(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
                                                         int64_t ld, uint16_t* __restrict__ Y) {
-  __shared__ uint16_t tile[64][64 + 8];
-  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
-  const int tid = threadIdx.x;
-  // load: 64 rows x 8 vectors of 8 entries, two per thread
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t r = (int64_t)blockIdx.y * 64 + (lane >> 2) * 8;
+  const int64_t c = (int64_t)blockIdx.x * 256 + warp * 32 + (lane & 3) * 8;
+  if (r >= rows || c >= cols) return;  // blocks are whole: rows and cols are multiples of 8
+  uint4 w[8];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int i = tid + k * 256, rr = i >> 3, cv = (i & 7) * 8;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if (r0 + rr < rows && c0 + cv < cols) w = __ldcs(reinterpret_cast<const uint4*>(X + (r0 + rr) * ld + c0 + cv));
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+  for (int i = 0; i < 8; ++i) w[i] = __ldcs(reinterpret_cast<const uint4*>(X + (r + i) * ld + c));
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      tile[rr][cv + 2 * e] = (uint16_t)(ww[e] & 0xFFFFu);
-      tile[rr][cv + 2 * e + 1] = (uint16_t)(ww[e] >> 16);
-    }
-  }
-  __syncthreads();
-  // store: 64 output rows (columns of X) x 8 vectors of 8 entries (rows of X)
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int i = tid + k * 256, cc = i >> 3, rv = (i & 7) * 8;
-    if (c0 + cc >= cols || r0 + rv >= rows) continue;
+  for (int j = 0; j < 8; ++j) {
+    // output row c + j holds entries (r + 0..7, c + j): word j/2 of every input row, low half for even j
+    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
     uint32_t o[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = (uint32_t)tile[rv + 2 * e][cc] | ((uint32_t)tile[rv + 2 * e + 1][cc] << 16);
-    *reinterpret_cast<uint4*>(Y + (c0 + cc) * rows + r0 + rv) = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int q = 0; q < 4; ++q) o[q] = __byte_perm(word_of(w[2 * q], j >> 1), word_of(w[2 * q + 1], j >> 1), sel);
+    *reinterpret_cast<uint4*>(Y + (c + j) * rows + r) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -1385,7 +1384,7 @@ imq_status run(const T* X, int64_t rows, int64_t cols, int64_t ld, imq_gran g, d
       StreamScratch tp;
       if (tp.alloc(ds, (size_t)rows * cols * 2, st) != IMQ_OK) return IMQ_ERR_CUDA;
       uint16_t* Y = static_cast<uint16_t*>(tp.p);
-      const dim3 tg((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+      const dim3 tg((unsigned)((cols + 255) / 256), (unsigned)((rows + 63) / 64));
       k_transpose_bf16<<<tg, 256, 0, st>>>(reinterpret_cast<const uint16_t*>(X), rows, cols, ld, Y);
       if (cudaGetLastError() != cudaSuccess) return IMQ_ERR_CUDA;
       if (try_rows_reg<kOut16>(Y, cols, rows, rows, (unsigned long long)nearest_rank(rows, p), beta, Xint, ldq, delta,
@@ -1612,7 +1611,9 @@ imq_status launch_rtn_quantize_rows_noalloc(const void* X, imq_dtype xt, int64_t
 // shared memory, its percentile selected and its values quantised (as in k_rtn_rows) into an int16 row
 // that never leaves shared memory; the warp then writes the row's unpacked line in the plan's layout (a
 // 16-position block the plan marked contiguous is one digit plane of 16 consecutive entries, computed
-// from two 16-byte reads; any other block is gathered entry by entry).  Each quantised entry is checked
+// from two 16-byte reads; any other block is gathered entry by entry).  With a staging order the int16
+// row is held in that order (entry t at staging position pinv[t]), which the plan's runs refer to.  Each
+// quantised entry is checked
 // against the plan's maximum |A[:, t]|: one above it may need a digit the layout does not hold, or break
 // the plan's accumulator bound, and sets IMQ_ERR_PLAN.
 // ------------------------------------------------------------------------------------------------
@@ -1620,7 +1621,8 @@ namespace {
 struct FusedArgs {
   int64_t rows, cols, ld;  // X, row-major
   int64_t K_unp;
-  const int32_t* tK;
+  const int32_t* pinv;  // staging position of each inner index (null: the identity)
+  const int32_t* tJ;    // staging position of the index at each inner position
   const int8_t* lAk;
   const int32_t* blk16;
   const int32_t* amax;  // [cols] max |A[:, t]| of the plan
@@ -1632,12 +1634,12 @@ struct FusedArgs {
   int32_t* status;
 };
 
-// Bytes of shared memory one warp of k_rtn_unpack_rows uses: the staged row and, for fp32 input, a
-// separate int16 row (a bf16 row is quantised in place: each lane reads its 8 entries before writing
-// their 8 int16 values at the same address).
+// Bytes of shared memory one warp of k_rtn_unpack_rows uses: the staged row and, for fp32 input or a
+// staging order, a separate int16 row (a bf16 row in index order is quantised in place: each lane reads
+// its 8 entries before writing their 8 int16 values at the same address).
 template <typename T>
-__host__ __device__ constexpr int64_t fused_warp_bytes(int64_t cols) {
-  return (cols * (int64_t)sizeof(T) + 15) / 16 * 16 + (sizeof(T) == 2 ? 0 : (cols * 2 + 31) / 32 * 32);
+__host__ __device__ constexpr int64_t fused_warp_bytes(int64_t cols, bool permuted) {
+  return (cols * (int64_t)sizeof(T) + 15) / 16 * 16 + (sizeof(T) == 2 && !permuted ? 0 : (cols * 2 + 31) / 32 * 32);
 }
 constexpr int64_t kFusedMetaMaxChunks = 4096;
 
@@ -1646,7 +1648,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
                                                               int meta_smem) {
   extern __shared__ __align__(16) unsigned char dsm[];
   const int64_t row_bytes = (f.cols * (int64_t)sizeof(T) + 15) / 16 * 16;
-  const int64_t wbytes = fused_warp_bytes<T>(f.cols);
+  const int64_t wbytes = fused_warp_bytes<T>(f.cols, f.pinv != nullptr);
   __shared__ uint32_t hist_all[kThreads / 32][kSelWords];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t nchunk = f.K_unp / 16;
@@ -1662,8 +1664,8 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
   }
   if (warp >= nwarps) return;
   T* row = reinterpret_cast<T*>(dsm + (int64_t)warp * wbytes);
-  int16_t* qv = sizeof(T) == 2 ? reinterpret_cast<int16_t*>(row)
-                               : reinterpret_cast<int16_t*>(dsm + (int64_t)warp * wbytes + row_bytes);
+  int16_t* qv = sizeof(T) == 2 && !f.pinv ? reinterpret_cast<int16_t*>(row)
+                                          : reinterpret_cast<int16_t*>(dsm + (int64_t)warp * wbytes + row_bytes);
   uint32_t* hist = hist_all[warp];
   constexpr int V = 16 / sizeof(T);
   const int n = (int)f.cols;
@@ -1710,15 +1712,23 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
         v[j] = quant_val<true>(Key<T>::value(e), s, f.status, 0);
         over |= (v[j] < 0 ? -v[j] : v[j]) > mm[j];
       }
-      uint32_t pk[4];
+      if (f.pinv) {
+        const int4 j0 = *reinterpret_cast<const int4*>(f.pinv + g * 8);
+        const int4 j1 = *reinterpret_cast<const int4*>(f.pinv + g * 8 + 4);
+        const int32_t jj[8] = {j0.x, j0.y, j0.z, j0.w, j1.x, j1.y, j1.z, j1.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) pk[j] = ((uint32_t)v[2 * j] & 0xFFFFu) | ((uint32_t)v[2 * j + 1] << 16);
-      *reinterpret_cast<uint4*>(qv + g * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int j = 0; j < 8; ++j) qv[jj[j]] = (int16_t)v[j];
+      } else {
+        uint32_t pk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pk[j] = ((uint32_t)v[2 * j] & 0xFFFFu) | ((uint32_t)v[2 * j + 1] << 16);
+        *reinterpret_cast<uint4*>(qv + g * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
     }
     for (int c = n8 * 8 + lane; c < n; c += 32) {
       const int32_t v = quant_val<true>(Key<T>::value(row[c]), s, f.status, 0);
       over |= (v < 0 ? -v : v) > f.amax[c];
-      qv[c] = (int16_t)v;
+      qv[f.pinv ? f.pinv[c] : c] = (int16_t)v;
     }
     if (over) set_status(f.status, IMQ_ERR_PLAN);
     __syncwarp();
@@ -1733,7 +1743,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         o = digits16_i16(w, meta_smem ? s_lk0[c] : f.lAk[p], f.bm1);
       } else {
-        const int4* tq = reinterpret_cast<const int4*>(f.tK + p);
+        const int4* tq = reinterpret_cast<const int4*>(f.tJ + p);
         const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
         const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
                                 tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
@@ -1761,7 +1771,7 @@ __global__ void __launch_bounds__(kThreads) k_rtn_unpack_rows(const T* __restric
 
 template <typename T>
 imq_status run_rtn_unpack(const T* X, const FusedArgs& f, DeviceState* ds, cudaStream_t st) {
-  const int64_t per_warp = fused_warp_bytes<T>(f.cols);
+  const int64_t per_warp = fused_warp_bytes<T>(f.cols, f.pinv != nullptr);
   const int64_t nchunk = f.K_unp / 16;
   const int meta_smem = nchunk <= kFusedMetaMaxChunks ? 1 : 0;
   const size_t meta = meta_smem ? (size_t)nchunk * 5 : 0;
@@ -1808,7 +1818,8 @@ imq_status launch_rtn_quantize_unpack(const imq_plan_t* pl, const void* X, imq_d
   f.cols = I.K;
   f.ld = ld;
   f.K_unp = I.K_unp;
-  f.tK = pl->tK;
+  f.pinv = pl->pinv;
+  f.tJ = pl->tJ;
   f.lAk = pl->lAk;
   f.blk16 = pl->blk16;
   f.amax = pl->max_a_col;

@@ -52,6 +52,24 @@ __device__ __forceinline__ void warp_copy16_global(const uint4* __restrict__ src
   }
 }
 
+// Staging positions of the 8 entries t .. t+7 (the identity without a staging order; -1 past K).
+__device__ __forceinline__ void octet_positions(const int32_t* __restrict__ pinv, int64_t t, int64_t K, int32_t (&pj)[8]) {
+#pragma unroll
+  for (int r = 0; r < 8; ++r) pj[r] = t + r < K ? (pinv ? pinv[t + r] : (int32_t)(t + r)) : -1;
+}
+// Stores the 8 digit bytes (lo: entries 0-3, hi: 4-7) of an octet at plane row prow: one 8-byte store in
+// index order, or byte by byte at the entries' staging positions.
+__device__ __forceinline__ void store_octet(int8_t* prow, int64_t t, uint32_t lo, uint32_t hi, bool permuted,
+                                            const int32_t (&pj)[8]) {
+  if (!permuted) {
+    *reinterpret_cast<uint2*>(prow + t) = make_uint2(lo, hi);
+    return;
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (pj[r] >= 0) prow[pj[r]] = (int8_t)(((r < 4 ? lo : hi) >> (8 * (r & 3))) & 0xFFu);
+}
+
 // Row gather: a CTA takes a batch of NL source lines and writes their digit planes to shared memory,
 // plane[b][l][t] = d_l(line b, entry t) for the P levels the batch needs, one byte each.  Then each
 // lane writes 16 consecutive inner positions of an output line: a block the plan marked contiguous
@@ -60,7 +78,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, int64_t nlines, int64_t K,
                                                      int64_t ld, int NL, int P, int outer,
                                                      const int8_t* __restrict__ lvl, const int32_t* __restrict__ pos,
-                                                     const int32_t* __restrict__ tK, const int8_t* __restrict__ lk,
+                                                     const int32_t* __restrict__ pinv, const int32_t* __restrict__ tJ,
+                                                     const int8_t* __restrict__ lk,
                                                      const int32_t* __restrict__ blk16, int64_t K_unp, int bm1,
                                                      int8_t* __restrict__ out) {
   extern __shared__ __align__(16) unsigned char dsm[];
@@ -117,7 +136,9 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
         if (f >= nq) continue;
         const int32_t b = (int32_t)f / (int32_t)q_line;
         const int64_t t = (f - (int64_t)b * q_line) * 8;
-        int8_t* pb = planes + (int64_t)b * P * Kp + t;
+        int8_t* pb = planes + (int64_t)b * P * Kp;
+        int32_t pj[8];
+        octet_positions(pinv, t, K, pj);
         uint32_t a[8], sg[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
@@ -134,7 +155,7 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
             lo |= (((d0 ^ sg[r]) - sg[r]) & 0xFFu) << (8 * r);
             hi |= (((d1 ^ sg[r + 4]) - sg[r + 4]) & 0xFFu) << (8 * r);
           }
-          *reinterpret_cast<uint2*>(pb + (int64_t)l * Kp) = make_uint2(lo, hi);
+          store_octet(pb + (int64_t)l * Kp, t, lo, hi, pinv != nullptr, pj);
         }
       }
     }
@@ -154,7 +175,7 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
           }
         }
       } else {
-        const int4* tq = reinterpret_cast<const int4*>(tK + p);
+        const int4* tq = reinterpret_cast<const int4*>(tJ + p);
         const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
         const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
                                 tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
@@ -193,7 +214,8 @@ __global__ void __launch_bounds__(256) k_unpack_rows(const T* __restrict__ X, in
 // no byte borrows).  Digits of level l with l * bm1 >= 16 are zero for int16 magnitudes.  The line is
 // 16-byte aligned and K a multiple of 8; entries K .. Kp-1 of the planes are written as zeros.
 __device__ __forceinline__ void digit_planes_i16(const int16_t* __restrict__ xr, int64_t K, int64_t Kp, int P,
-                                                 int bm1, int8_t* __restrict__ planes, int lane) {
+                                                 int bm1, const int32_t* __restrict__ pinv,
+                                                 int8_t* __restrict__ planes, int lane) {
   const uint32_t mask = (1u << bm1) - 1u;
   const int64_t nq = Kp / 8;
   constexpr int kU = 8;
@@ -208,6 +230,8 @@ __device__ __forceinline__ void digit_planes_i16(const int16_t* __restrict__ xr,
     for (int u = 0; u < kU; ++u) {
       const int64_t t = (q0 + u * 32 + lane) * 8;
       if (t >= Kp) continue;
+      int32_t pj[8];
+      octet_positions(pinv, t, K, pj);
       const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
       uint32_t A[4], S[4];
 #pragma unroll
@@ -230,7 +254,7 @@ __device__ __forceinline__ void digit_planes_i16(const int16_t* __restrict__ xr,
           lo = (plo & ~Mlo) | (nlo & Mlo);
           hi = (phi & ~Mhi) | (nhi & Mhi);
         }
-        *reinterpret_cast<uint2*>(planes + (int64_t)l * Kp + t) = make_uint2(lo, hi);
+        store_octet(planes + (int64_t)l * Kp, t, lo, hi, pinv != nullptr, pj);
       }
     }
   }
@@ -253,7 +277,8 @@ struct LineJob {
   int outer;
   const int8_t* lvl;
   const int32_t* pos;
-  const int32_t* tK;
+  const int32_t* pinv;  // staging position of each inner index (null: the identity)
+  const int32_t* tJ;    // staging position of the index at each inner position
   const int8_t* lk;
   const int32_t* blk16;
   int64_t K_unp;
@@ -269,7 +294,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines, int64_t K,
                                                       int64_t ld, int P, int nwarps, int outer,
                                                       const int8_t* lvl, const int32_t* pos,
-                                                      const int32_t* tK, const int8_t* lk,
+                                                      const int32_t* pinv, const int32_t* tJ, const int8_t* lk,
                                                       const int32_t* blk16, int64_t K_unp, int bm1,
                                                       int meta_smem, int8_t* out, const int32_t* grpL,
                                                       const int32_t* grpN, int64_t ngrp, int G,
@@ -281,7 +306,8 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
     outer = jb.outer;
     lvl = jb.lvl;
     pos = jb.pos;
-    tK = jb.tK;
+    pinv = jb.pinv;
+    tJ = jb.tJ;
     lk = jb.lk;
     blk16 = jb.blk16;
     K_unp = jb.K_unp;
@@ -325,7 +351,7 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
     bool planes_done = false;
     if constexpr (sizeof(T) == 2) {
       if (vec8) {
-        digit_planes_i16(reinterpret_cast<const int16_t*>(xr), K, Kp, P, bm1, planes, lane);
+        digit_planes_i16(reinterpret_cast<const int16_t*>(xr), K, Kp, P, bm1, pinv, planes, lane);
         planes_done = true;
       }
     }
@@ -357,6 +383,8 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
       for (int u = 0; u < kU; ++u) {
         const int64_t t = (q0 + u * 32 + lane) * 8;
         if (t >= Kp) continue;
+        int32_t pj[8];
+        octet_positions(pinv, t, K, pj);
         uint32_t a[8], sg[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
@@ -373,7 +401,7 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
             lo |= (((d0 ^ sg[r]) - sg[r]) & 0xFFu) << (8 * r);
             hi |= (((d1 ^ sg[r + 4]) - sg[r + 4]) & 0xFFu) << (8 * r);
           }
-          *reinterpret_cast<uint2*>(planes + (int64_t)l * Kp + t) = make_uint2(lo, hi);
+          store_octet(planes + (int64_t)l * Kp, t, lo, hi, pinv != nullptr, pj);
         }
       }
     }
@@ -391,7 +419,7 @@ __global__ void __launch_bounds__(256) k_unpack_lines(const T* X, int64_t nlines
           *reinterpret_cast<uint4*>(out + (base + l) * K_unp + p) = w;
         }
       } else {
-        const int4* tq = reinterpret_cast<const int4*>(tK + p);
+        const int4* tq = reinterpret_cast<const int4*>(tJ + p);
         const int4 ta = tq[0], tb = tq[1], tc = tq[2], td = tq[3];
         const int32_t tt[16] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w,
                                 tc.x, tc.y, tc.z, tc.w, td.x, td.y, td.z, td.w};
@@ -440,30 +468,64 @@ __device__ __forceinline__ uint4 digits16_fixed(const Mag16& m) {
   }
 }
 
-// Magnitudes and signs of 16 consecutive int32 entries (shared memory), for their digits of any level.
+// Magnitudes and signs of 16 int32 entries, for their digits of any level: per 4 entries a byte mask
+// (0xFF where the entry is negative) in entry order.
 struct Mag16w {
   uint32_t m[16];
-  uint32_t neg;  // bit k: entry k is negative
+  uint32_t neg[4];
 };
-// v16 may start anywhere (16-byte loads when it is 16-byte aligned).
-__device__ __forceinline__ Mag16w mag16_i32(const int32_t* v16) {
+__device__ __forceinline__ Mag16w mag16_i32(const int32_t (&e)[16]) {
   Mag16w r;
-  r.neg = 0;
-  const bool al = (reinterpret_cast<uintptr_t>(v16) & 15) == 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int4 w = al ? reinterpret_cast<const int4*>(v16)[q]
-                      : make_int4(v16[4 * q], v16[4 * q + 1], v16[4 * q + 2], v16[4 * q + 3]);
-    const int32_t e[4] = {w.x, w.y, w.z, w.w};
+    uint32_t nm = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      r.m[4 * q + k] = e[k] < 0 ? (uint32_t)(-(int64_t)e[k]) : (uint32_t)e[k];
-      r.neg |= (uint32_t)(e[k] < 0) << (4 * q + k);
+      const int32_t v = e[4 * q + k];
+      r.m[4 * q + k] = v < 0 ? 0u - (uint32_t)v : (uint32_t)v;
+      nm |= ((uint32_t)(v >> 31) & 0xFFu) << (8 * k);
     }
+    r.neg[q] = nm;
   }
   return r;
 }
-// Digit l (base 2^bm1, sign-magnitude) of the 16 entries as 16 bytes in entry order.
+// The 16 int32 entries row[t0 .. t0 + 15] of a staged line (16-byte loads when t0 % 4 == 0).
+__device__ __forceinline__ void load16_i32(const int32_t* row, int t0, int32_t (&e)[16]) {
+  if ((t0 & 3) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int4 w = reinterpret_cast<const int4*>(row + t0)[q];
+      e[4 * q] = w.x; e[4 * q + 1] = w.y; e[4 * q + 2] = w.z; e[4 * q + 3] = w.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) e[k] = row[t0 + k];
+  }
+}
+// The 16 entries at staging positions j[0..15] of a staged line (0 where j < 0: padding).
+__device__ __forceinline__ void gather16_i32(const int32_t* row, const int32_t* __restrict__ j, int32_t (&e)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int4 v = reinterpret_cast<const int4*>(j)[q];
+    e[4 * q] = v.x >= 0 ? row[v.x] : 0;
+    e[4 * q + 1] = v.y >= 0 ? row[v.y] : 0;
+    e[4 * q + 2] = v.z >= 0 ? row[v.z] : 0;
+    e[4 * q + 3] = v.w >= 0 ? row[v.w] : 0;
+  }
+}
+__device__ __forceinline__ void gather16_i16(const int16_t* row, const int32_t* __restrict__ j, uint32_t (&w)[8]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int4 v = reinterpret_cast<const int4*>(j)[q];
+    const uint32_t e0 = v.x >= 0 ? (uint32_t)(uint16_t)row[v.x] : 0u, e1 = v.y >= 0 ? (uint32_t)(uint16_t)row[v.y] : 0u;
+    const uint32_t e2 = v.z >= 0 ? (uint32_t)(uint16_t)row[v.z] : 0u, e3 = v.w >= 0 ? (uint32_t)(uint16_t)row[v.w] : 0u;
+    w[2 * q] = e0 | (e1 << 16);
+    w[2 * q + 1] = e2 | (e3 << 16);
+  }
+}
+// Digit l (base 2^bm1, sign-magnitude) of the 16 entries as 16 bytes in entry order: four digits
+// gathered into one word by byte permutes, the negative entries' digits negated byte-wise as
+// (0x80808080 - d) ^ 0x80808080 (a digit is at most 127, so no byte borrows).
 __device__ __forceinline__ uint4 digits16_i32(const Mag16w& m, int l, int bm1) {
   const int sh = l * bm1;
   if (sh >= 31) return make_uint4(0u, 0u, 0u, 0u);
@@ -471,14 +533,11 @@ __device__ __forceinline__ uint4 digits16_i32(const Mag16w& m, int l, int bm1) {
   uint32_t o[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint32_t packed = 0;
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int k = 4 * q + r;
-      const uint32_t d = (m.m[k] >> sh) & mask;
-      packed |= (((m.neg >> k) & 1u) ? ((0u - d) & 0xFFu) : d) << (8 * r);
-    }
-    o[q] = packed;
+    const uint32_t d0 = (m.m[4 * q] >> sh) & mask, d1 = (m.m[4 * q + 1] >> sh) & mask;
+    const uint32_t d2 = (m.m[4 * q + 2] >> sh) & mask, d3 = (m.m[4 * q + 3] >> sh) & mask;
+    const uint32_t pd = __byte_perm(__byte_perm(d0, d1, 0x0040), __byte_perm(d2, d3, 0x0040), 0x5410);
+    const uint32_t nd = (0x80808080u - pd) ^ 0x80808080u;
+    o[q] = (pd & ~m.neg[q]) | (nd & m.neg[q]);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -502,23 +561,65 @@ __device__ __forceinline__ void load16_i16(const int16_t* row, int t0, uint32_t 
 
 constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take the unrolled path
 
-// Row gather for int16 sources, one warp per source line (base 2^kBm1 fixed at compile time).  The warp
-// stages its line in its own shared memory (16-byte loads, all of a lane's in flight) and writes the
-// line's L unpacked lines, 16 inner positions per lane and step: a block the plan marked contiguous
-// (t0..t0+15, t0 % 16 == 0, one inner level lk0) takes the magnitudes and signs of its 16 entries once
-// and emits the digit (l + lk0) for every output line l from them; any other block is gathered entry by
-// entry.  The per-block plan metadata is staged in shared memory once per CTA.  Lines are dealt to the
-// CTAs in turn (line i to CTA i mod gridDim.x).  After its lines, each CTA zeroes the unused lines of the
-// OUTER groups dealt to it (group g to CTA g mod gridDim.x), lines n*L .. G-1 of a group of n sources of
-// level L, which no source line writes.  cta_line: lines too long for a line per warp (more than 8192
-// entries) are staged one at a time per CTA by all its threads, and all its threads write its blocks.
+// Stages source line xr (K entries) in staging order: entry t at row[pinv[t]].  Threads i0, i0 + step, ...
+// take 16-byte pieces (vec: K, the row start and the line stride allow them), four in flight before their
+// scattered shared-memory stores.
+template <typename T>
+__device__ __forceinline__ void stage_permuted(const T* __restrict__ xr, int64_t K, bool vec,
+                                               const int32_t* __restrict__ pinv, T* row, int i0, int step) {
+  constexpr int V = 16 / (int)sizeof(T);
+  constexpr int kBatch = 2;
+  if (vec) {
+    const int64_t nq = K / V;
+    for (int64_t q0 = i0; q0 < nq; q0 += (int64_t)step * kBatch) {
+      uint4 w[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t q = q0 + (int64_t)u * step;
+        if (q < nq) w[u] = reinterpret_cast<const uint4*>(xr)[q];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t q = q0 + (int64_t)u * step;
+        if (q >= nq) continue;
+        const int4* pj = reinterpret_cast<const int4*>(pinv + q * V);
+        if constexpr (sizeof(T) == 2) {
+          const int4 a = pj[0], b = pj[1];
+          row[a.x] = (T)(w[u].x & 0xFFFFu); row[a.y] = (T)(w[u].x >> 16);
+          row[a.z] = (T)(w[u].y & 0xFFFFu); row[a.w] = (T)(w[u].y >> 16);
+          row[b.x] = (T)(w[u].z & 0xFFFFu); row[b.y] = (T)(w[u].z >> 16);
+          row[b.z] = (T)(w[u].w & 0xFFFFu); row[b.w] = (T)(w[u].w >> 16);
+        } else {
+          const int4 a = pj[0];
+          row[a.x] = (T)w[u].x; row[a.y] = (T)w[u].y; row[a.z] = (T)w[u].z; row[a.w] = (T)w[u].w;
+        }
+      }
+    }
+  } else {
+    for (int64_t t = i0; t < K; t += step) row[pinv[t]] = xr[t];
+  }
+}
+
+// Row gather for int16 and int32 sources, the base 2^kBm1 fixed at compile time.  Each source line is
+// staged in shared memory in the plan's staging order (one line per warp, or per CTA for long lines) and
+// the line's L unpacked lines are written 16 inner positions per lane and step.  A block the plan marked
+// a run (the indices at staging positions j0..j0+15, one inner level lk0) takes the magnitudes and signs
+// of its 16 staged entries once and emits digit (l + lk0) for every output line l from them.  The few
+// other blocks (those across a segment or range boundary, and padding) are taken by the whole warp after
+// the runs of its step: a half-warp per block, one position per lane, read through the plan's staging
+// positions tJ.  The per-block plan metadata is staged in shared memory once per CTA.  Lines are dealt to
+// the CTAs in turn (line i to CTA i mod gridDim.x).  After its lines, each CTA zeroes the unused lines of
+// the OUTER groups dealt to it (group g to CTA g mod gridDim.x), lines n*L .. G-1 of a group of n sources
+// of level L, which no source line writes.  cta_line: lines too long for a line per warp are staged one
+// at a time per CTA by all its threads, and all its threads write its blocks.
 template <typename T, int kBm1>
 __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(const T* X, int64_t nlines, int64_t K,
                                                            int64_t ld, int nwarps, int outer, const int8_t* lvl,
-                                                           const int32_t* pos, const int32_t* tK, const int8_t* lk,
-                                                           const int32_t* blk16, int64_t K_unp, int8_t* out,
-                                                           const int32_t* grpL, const int32_t* grpN, int64_t ngrp,
-                                                           int G, int cta_line, const LineJob* __restrict__ jobs) {
+                                                           const int32_t* pos, const int32_t* pinv, const int32_t* tJ,
+                                                           const int8_t* lk, const int32_t* blk16, int64_t K_unp,
+                                                           int8_t* out, const int32_t* grpL, const int32_t* grpN,
+                                                           int64_t ngrp, int G, int cta_line,
+                                                           const LineJob* __restrict__ jobs) {
   extern __shared__ __align__(16) unsigned char dsm[];
   if (jobs) {
     const LineJob& jb = jobs[blockIdx.y];
@@ -526,7 +627,8 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
     outer = jb.outer;
     lvl = jb.lvl;
     pos = jb.pos;
-    tK = jb.tK;
+    pinv = jb.pinv;
+    tJ = jb.tJ;
     lk = jb.lk;
     blk16 = jb.blk16;
     K_unp = jb.K_unp;
@@ -538,160 +640,86 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t Kr = (K + 15) / 16 * 16;  // staged line length in entries (32-byte multiple)
   const int nchunk = (int)(K_unp / 16);
-  // [lines of nwarps warps (one line in cta_line mode), int16 x Kr][block starts, int32 x nchunk]
+  // [lines of nwarps warps (one line in cta_line mode), T x Kr][block starts, int32 x nchunk]
   // [first inner levels, int8 x nchunk]
   int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)(cta_line ? 1 : nwarps) * Kr * (int64_t)sizeof(T));
-  int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);
+  int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);  // inner level of each block, -1 mixed
   for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
     s_blk[c] = blk16[c];
-    s_lk0[c] = lk[(int64_t)c * 16];
+    // the block's inner level, or -1 when its 16 positions do not share one
+    const uint4 q = *reinterpret_cast<const uint4*>(lk + (int64_t)c * 16);
+    const uint32_t b0 = (q.x & 0xFFu) * 0x01010101u;
+    s_lk0[c] = (q.x == b0 && q.y == b0 && q.z == b0 && q.w == b0) ? (int8_t)(q.x & 0xFFu) : (int8_t)-1;
   }
   __syncthreads();
   constexpr int kPer16 = 16 / (int)sizeof(T);  // entries per 16-byte load
   const bool vec8 = (K % kPer16 == 0) && (ld % kPer16 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
-  // The unpacked lines of source line `line`, staged in `row`: blocks c_first, c_first + c_step, ...
-  auto emit = [&](int64_t line, const T* row, int c_first, int c_step) {
+  // Warp-cooperative write of the irregular blocks flagged in `irr` (bit k: block cb + k): lanes 0-15 take
+  // one block, lanes 16-31 the next, one position per lane and a byte store per output line.
+  auto irregular = [&](const T* row, int8_t* o0, int L, int cb, unsigned irr) {
+    while (irr) {
+      const int k0 = __ffs(irr) - 1;
+      irr &= irr - 1;
+      int k1 = -1;
+      if (irr) {
+        k1 = __ffs(irr) - 1;
+        irr &= irr - 1;
+      }
+      const int kk = lane < 16 ? k0 : k1;
+      if (kk < 0) continue;
+      const int64_t pp = (int64_t)(cb + kk) * 16 + (lane & 15);
+      const int32_t j = tJ[pp];
+      const int lr = lk[pp];
+      const int32_t v = j >= 0 ? (int32_t)row[j] : 0;
+      const bool use = j >= 0 && (L == 1 || lr == 0);
+      for (int l = 0; l < L; ++l) o0[(int64_t)l * K_unp + pp] = (int8_t)(use ? digit_of(v, l + lr, kBm1) : 0);
+    }
+  };
+  // The unpacked lines of source line `line`, staged in `row`: the warp's blocks cb0 + lane, cb0 + lane +
+  // c_step, ... (cb0 and c_step the same for all its lanes).
+  auto emit = [&](int64_t line, const T* row, int cb0, int c_step) {
       const int L = outer ? (int)lvl[line] : 1;
       int8_t* o0 = out + (outer ? (int64_t)pos[line] : line) * K_unp;
-      if (L <= kFastLevels) {
-        int8_t* ol[kFastLevels];
-#pragma unroll
-        for (int l = 0; l < kFastLevels; ++l) ol[l] = o0 + (int64_t)l * K_unp;
-        for (int c = c_first; c < nchunk; c += c_step) {
-          const int tb = s_blk[c];
-          const int t0 = tb >= 0 ? tb : -tb - 2;  // first source index of a run (aligned or not)
-          const int p = c * 16;
-          uint4 d[kFastLevels];
-          if (tb != -1) {
-            const int lk0 = s_lk0[c];
-            if (L > 1 && lk0 > 0) {
-#pragma unroll
-              for (int l = 0; l < kFastLevels; ++l) d[l] = make_uint4(0u, 0u, 0u, 0u);
-            } else if constexpr (sizeof(T) == 2) {
-              uint32_t w[8];
-              load16_i16(reinterpret_cast<const int16_t*>(row), t0, w);
-              const Mag16 m = mag16_i16(w);
-              if (L == 1) {
-                d[0] = digits16_from(m, lk0, kBm1);
-              } else {
-                d[0] = digits16_fixed<kBm1, 0>(m);
-                d[1] = digits16_fixed<kBm1, 1>(m);
-                if (L > 2) d[2] = digits16_fixed<kBm1, 2>(m);
-                if (L > 3) d[3] = digits16_fixed<kBm1, 3>(m);
-              }
+      for (int cb = cb0; cb < nchunk; cb += c_step) {
+        const int c = cb + lane;
+        const int tb = c < nchunk ? s_blk[c] : -1;
+        const int lk0 = c < nchunk ? s_lk0[c] : -1;
+        // a run, or a block of one inner level gathered through tJ: the lane's own block, the digits
+        // computed the same way for both; any other block is taken by the whole warp below
+        const bool uni = c < nchunk && (tb != -1 || lk0 >= 0);
+        if (uni) {
+          const int64_t p = (int64_t)c * 16;
+          const int t0 = tb >= 0 ? tb : -tb - 2;  // first staging position of a run (aligned or not)
+          if (L > 1 && lk0 > 0) {
+            for (int l = 0; l < L; ++l) *reinterpret_cast<uint4*>(o0 + (int64_t)l * K_unp + p) = make_uint4(0u, 0u, 0u, 0u);
+          } else if constexpr (sizeof(T) == 2) {
+            uint32_t w[8];
+            if (tb != -1) load16_i16(reinterpret_cast<const int16_t*>(row), t0, w);
+            else gather16_i16(reinterpret_cast<const int16_t*>(row), tJ + p, w);
+            const Mag16 m = mag16_i16(w);
+            if (L == 1) {
+              *reinterpret_cast<uint4*>(o0 + p) = digits16_from(m, lk0, kBm1);
+            } else if (L <= kFastLevels) {
+              *reinterpret_cast<uint4*>(o0 + p) = digits16_fixed<kBm1, 0>(m);
+              *reinterpret_cast<uint4*>(o0 + K_unp + p) = digits16_fixed<kBm1, 1>(m);
+              if (L > 2) *reinterpret_cast<uint4*>(o0 + 2 * K_unp + p) = digits16_fixed<kBm1, 2>(m);
+              if (L > 3) *reinterpret_cast<uint4*>(o0 + 3 * K_unp + p) = digits16_fixed<kBm1, 3>(m);
             } else {
-              const Mag16w m = mag16_i32(reinterpret_cast<const int32_t*>(row + t0));
-              if (L == 1) {
-                d[0] = digits16_i32(m, lk0, kBm1);
-              } else {
-#pragma unroll
-                for (int l = 0; l < kFastLevels; ++l) d[l] = l < L ? digits16_i32(m, l, kBm1) : make_uint4(0u, 0u, 0u, 0u);
-              }
-            }
-          } else if (const uint4 lq = *reinterpret_cast<const uint4*>(lk + p);
-                     lq.x == lq.y && lq.y == lq.z && lq.z == lq.w && (lq.x & 0xFFu) * 0x01010101u == lq.x) {
-            // a block of scattered source indices with one inner level (a sparse segment): its 16 entries
-            // gathered from the staged line (padding positions read as 0), then split like a run
-            const int lr = (int)(int8_t)(lq.x & 0xFFu);
-            const int4* tq = reinterpret_cast<const int4*>(tK + p);
-            int32_t tt[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int4 v = tq[q];
-              tt[4 * q] = v.x; tt[4 * q + 1] = v.y; tt[4 * q + 2] = v.z; tt[4 * q + 3] = v.w;
-            }
-            if (L > 1 && lr > 0) {
-#pragma unroll
-              for (int l = 0; l < kFastLevels; ++l) d[l] = make_uint4(0u, 0u, 0u, 0u);
-            } else if constexpr (sizeof(T) == 2) {
-              uint32_t w[8];
-#pragma unroll
-              for (int h = 0; h < 8; ++h) {
-                const uint32_t lo = tt[2 * h] >= 0 ? (uint32_t)(uint16_t)row[tt[2 * h]] : 0u;
-                const uint32_t hi = tt[2 * h + 1] >= 0 ? (uint32_t)(uint16_t)row[tt[2 * h + 1]] : 0u;
-                w[h] = lo | (hi << 16);
-              }
-              const Mag16 m = mag16_i16(w);
-              if (L == 1) {
-                d[0] = digits16_from(m, lr, kBm1);
-              } else {
-                d[0] = digits16_fixed<kBm1, 0>(m);
-                d[1] = digits16_fixed<kBm1, 1>(m);
-                if (L > 2) d[2] = digits16_fixed<kBm1, 2>(m);
-                if (L > 3) d[3] = digits16_fixed<kBm1, 3>(m);
-              }
-            } else {
-              int32_t g16[16];
-#pragma unroll
-              for (int k = 0; k < 16; ++k) g16[k] = tt[k] >= 0 ? (int32_t)row[tt[k]] : 0;
-              const Mag16w m = mag16_i32(g16);
-              if (L == 1) {
-                d[0] = digits16_i32(m, lr, kBm1);
-              } else {
-#pragma unroll
-                for (int l = 0; l < kFastLevels; ++l) d[l] = l < L ? digits16_i32(m, l, kBm1) : make_uint4(0u, 0u, 0u, 0u);
-              }
+              for (int l = 0; l < L; ++l) *reinterpret_cast<uint4*>(o0 + (int64_t)l * K_unp + p) = digits16_from(m, l, kBm1);
             }
           } else {
-            // gathered entry by entry (blocks across segment boundaries and padding; rare)
-#pragma unroll
-            for (int l = 0; l < kFastLevels; ++l) {
-              uint32_t wv[4] = {0u, 0u, 0u, 0u};
-              if (l < L) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const int4 tq = reinterpret_cast<const int4*>(tK + p)[q];
-                  const uint32_t lq = reinterpret_cast<const uint32_t*>(lk + p)[q];
-                  const int32_t tt[4] = {tq.x, tq.y, tq.z, tq.w};
-#pragma unroll
-                  for (int r = 0; r < 4; ++r) {
-                    const int lr = (int)(int8_t)(lq >> (8 * r));
-                    const int32_t dg =
-                        (tt[r] >= 0 && (L == 1 || lr == 0)) ? digit_of((int32_t)row[tt[r]], l + lr, kBm1) : 0;
-                    wv[q] |= ((uint32_t)(uint8_t)(int8_t)dg) << (8 * r);
-                  }
-                }
-              }
-              d[l] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
-          }
-#pragma unroll
-          for (int l = 0; l < kFastLevels; ++l)
-            if (l < L) *reinterpret_cast<uint4*>(ol[l] + p) = d[l];
-        }
-      } else {
-        // lines of more levels (small b): one output line at a time
-        for (int c = c_first; c < nchunk; c += c_step) {
-          const int tb = s_blk[c];
-          const int t0 = tb >= 0 ? tb : -tb - 2;
-          const int p = c * 16;
-          const int lk0 = tb != -1 ? s_lk0[c] : 0;
-          for (int l = 0; l < L; ++l) {
-            uint4 dv;
-            if (tb != -1) {
-              if (lk0 > 0) {
-                dv = make_uint4(0u, 0u, 0u, 0u);
-              } else if constexpr (sizeof(T) == 2) {
-                uint32_t w[8];
-                load16_i16(reinterpret_cast<const int16_t*>(row), t0, w);
-                dv = digits16_i16(w, l, kBm1);
-              } else {
-                dv = digits16_i32(mag16_i32(reinterpret_cast<const int32_t*>(row + t0)), l, kBm1);
-              }
+            int32_t e[16];
+            if (tb != -1) load16_i32(reinterpret_cast<const int32_t*>(row), t0, e);
+            else gather16_i32(reinterpret_cast<const int32_t*>(row), tJ + p, e);
+            const Mag16w m = mag16_i32(e);
+            if (L == 1) {
+              *reinterpret_cast<uint4*>(o0 + p) = digits16_i32(m, lk0, kBm1);
             } else {
-              uint32_t wv[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const int32_t t = tK[p + k];
-                const int lr = lk[p + k];
-                const int32_t dg = (t >= 0 && lr == 0) ? digit_of((int32_t)row[t], l, kBm1) : 0;
-                wv[k >> 2] |= ((uint32_t)(uint8_t)(int8_t)dg) << (8 * (k & 3));
-              }
-              dv = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+              for (int l = 0; l < L; ++l) *reinterpret_cast<uint4*>(o0 + (int64_t)l * K_unp + p) = digits16_i32(m, l, kBm1);
             }
-            *reinterpret_cast<uint4*>(o0 + (int64_t)l * K_unp + p) = dv;
           }
         }
+        irregular(row, o0, L, cb, __ballot_sync(0xffffffffu, c < nchunk && !uni));
       }
   };
   if (cta_line) {
@@ -700,7 +728,9 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
     for (int64_t line = blockIdx.x; line < nlines; line += gridDim.x) {
       const T* xr = X + line * ld;
       __syncthreads();  // the previous line has been read
-      if (vec8) {
+      if (pinv) {
+        stage_permuted<T>(xr, K, vec8, pinv, row, (int)threadIdx.x, (int)blockDim.x);
+      } else if (vec8) {
         const uint4* src = reinterpret_cast<const uint4*>(xr);
         uint4* dst = reinterpret_cast<uint4*>(row);
         for (int64_t q = threadIdx.x; q < K / kPer16; q += blockDim.x) dst[q] = src[q];
@@ -708,21 +738,23 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
         for (int64_t t = threadIdx.x; t < K; t += blockDim.x) row[t] = xr[t];
       }
       __syncthreads();
-      emit(line, row, (int)threadIdx.x, (int)blockDim.x);
+      emit(line, row, warp * 32, (int)blockDim.x);
     }
   } else if (warp < nwarps) {
     T* row = reinterpret_cast<T*>(dsm) + (int64_t)warp * Kr;
     for (int64_t line = (int64_t)warp * gridDim.x + blockIdx.x; line < nlines;
          line += (int64_t)gridDim.x * nwarps) {
       const T* xr = X + line * ld;
-      if (vec8) {
+      if (pinv) {
+        stage_permuted<T>(xr, K, vec8, pinv, row, lane, 32);
+      } else if (vec8) {
         warp_copy16_global<4>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), (int)(K / kPer16),
                               lane);
       } else {
         for (int64_t t = lane; t < K; t += 32) row[t] = xr[t];
       }
       __syncwarp();
-      emit(line, row, lane, 32);
+      emit(line, row, 0, 32);
       __syncwarp();
     }
   }
@@ -738,10 +770,10 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
 // nprob > 1: `jobs` (device) holds the per-problem arguments and the ones given here are ignored.
 template <typename T, int kBm1>
 imq_status launch_lines16(const T* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
-                          const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
-                          const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL, const int32_t* grpN,
-                          int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs = nullptr,
-                          int nprob = 1) {
+                          const int8_t* lvl, const int32_t* pos, const int32_t* pinv, const int32_t* tJ,
+                          const int8_t* lk, const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL,
+                          const int32_t* grpN, int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st,
+                          const LineJob* jobs = nullptr, int nprob = 1) {
   auto kern = k_unpack_lines16<T, kBm1>;
   IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
   int per_sm = 0;
@@ -750,28 +782,32 @@ imq_status launch_lines16(const T* X, int64_t nlines, int64_t K, int64_t ld, int
   // every resident slot once over the whole batch
   int64_t grid = ((int64_t)num_sms * per_sm + nprob - 1) / nprob;
   if (grid > nlines) grid = nlines;
-  kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16,
-                                                                 K_unp, out, grpL, grpN, ngrp, G, nw == 0 ? 1 : 0,
-                                                                 jobs);
+  kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, pinv, tJ, lk,
+                                                                 blk16, K_unp, out, grpL, grpN, ngrp, G,
+                                                                 nw == 0 ? 1 : 0, jobs);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
 // The staged-line kernel for base 2^bm1 (bm1 in 1..7), the base fixed at compile time.
 template <typename T>
 imq_status launch_staged(int bm1, const T* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
-                         const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
-                         const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL, const int32_t* grpN,
-                         int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs,
-                         int nprob) {
+                         const int8_t* lvl, const int32_t* pos, const int32_t* pinv, const int32_t* tJ,
+                         const int8_t* lk, const int32_t* blk16, int64_t K_unp, int8_t* out, const int32_t* grpL,
+                         const int32_t* grpN, int64_t ngrp, int G, size_t smem, int num_sms, cudaStream_t st,
+                         const LineJob* jobs, int nprob) {
+#define IMQ_STAGED(B) \
+  launch_lines16<T, B>(X, nlines, K, ld, nw, outer, lvl, pos, pinv, tJ, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, \
+                       num_sms, st, jobs, nprob)
   switch (bm1) {
-    case 1: return launch_lines16<T, 1>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
-    case 2: return launch_lines16<T, 2>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
-    case 3: return launch_lines16<T, 3>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
-    case 4: return launch_lines16<T, 4>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
-    case 5: return launch_lines16<T, 5>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
-    case 6: return launch_lines16<T, 6>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
-    default: return launch_lines16<T, 7>(X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out, grpL, grpN, ngrp, G, smem, num_sms, st, jobs, nprob);
+    case 1: return IMQ_STAGED(1);
+    case 2: return IMQ_STAGED(2);
+    case 3: return IMQ_STAGED(3);
+    case 4: return IMQ_STAGED(4);
+    case 5: return IMQ_STAGED(5);
+    case 6: return IMQ_STAGED(6);
+    default: return IMQ_STAGED(7);
   }
+#undef IMQ_STAGED
 }
 
 // Launch shape of the staged-line kernel for lines of K entries of T and nchunk 16-position blocks: a
@@ -892,8 +928,9 @@ struct ZeroJob {
 // One operand.  *zeroed is set when the launch also zeroed the operand's unused OUTER lines.
 template <typename T>
 imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool line_is_row, int outer, int P,
-                      const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int8_t* lk,
-                      const int32_t* blk16, int64_t K_unp, int bm1, int8_t* out, int num_sms, cudaStream_t st,
+                      const int8_t* lvl, const int32_t* pos, const int32_t* tK, const int32_t* pinv,
+                      const int32_t* tJ, const int8_t* lk, const int32_t* blk16, int64_t K_unp, int bm1, int8_t* out,
+                      int num_sms, cudaStream_t st,
                       const ZeroJob& zj, bool* zeroed) {
   *zeroed = false;
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
@@ -904,7 +941,7 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
     size_t smem = 0;
     if (line_is_row && bm1 >= 1 && bm1 <= 7 && staged_shape(K, sizeof(T), nchunk, &nw, &smem)) {
       const int64_t ng = outer ? zj.ngrp : 0;
-      const imq_status s = launch_staged<T>(bm1, X, nlines, K, ld, nw, outer, lvl, pos, tK, lk, blk16, K_unp, out,
+      const imq_status s = launch_staged<T>(bm1, X, nlines, K, ld, nw, outer, lvl, pos, pinv, tJ, lk, blk16, K_unp, out,
                                             zj.grpL, zj.grpN, ng, zj.G, smem, num_sms, st, nullptr, 1);
       *zeroed = s == IMQ_OK;
       return s;
@@ -928,7 +965,7 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
         int64_t grid = (int64_t)num_sms * (per_sm > 8 ? 8 : per_sm);
         if (grid > ctas) grid = ctas;
         IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
-        k_unpack_lines<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, P, nw, outer, lvl, pos, tK, lk, blk16,
+        k_unpack_lines<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, P, nw, outer, lvl, pos, pinv, tJ, lk, blk16,
                                                              K_unp, bm1, meta_smem, out, zj.grpL, zj.grpN,
                                                              outer ? zj.ngrp : 0, zj.G, nullptr);
         *zeroed = true;
@@ -953,7 +990,7 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
     int64_t grid = (int64_t)num_sms * (per_sm > 8 ? 8 : per_sm);
     if (grid > batches) grid = batches;
     IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_rows<T>), smem));
-    k_unpack_rows<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, NL, P, outer, lvl, pos, tK, lk, blk16,
+    k_unpack_rows<T><<<(unsigned)grid, 256, smem, st>>>(X, nlines, K, ld, NL, P, outer, lvl, pos, pinv, tJ, lk, blk16,
                                                         K_unp, bm1, out);
   } else {
     const dim3 grid((unsigned)((nlines + 31) / 32), (unsigned)(K_unp / 128));
@@ -982,11 +1019,11 @@ imq_status unpack_typed(const imq_plan_t* pl, const T* A, const T* B, int8_t* Au
   if (b_outer) zb = ZeroJob{pl->grpB_L, pl->grpB_n, pl->n_grp_b, IMQ_B_GROUP};
   bool za_done = false, zb_done = false;
   imq_status s = unpack_one<T>(A, I.M, I.K, pl->lda, !pl->transA, a_outer, pa, pl->lv_a_row, pl->posA, pl->tK,
-                               pl->lAk, pl->blk16, I.K_unp, bm1, Au, num_sms, st, za, &za_done);
+                               pl->pinv, pl->tJ, pl->lAk, pl->blk16, I.K_unp, bm1, Au, num_sms, st, za, &za_done);
   if (s != IMQ_OK) return s;
   // B'^T lines are the logical columns of B: stored rows only when B is given transposed
-  s = unpack_one<T>(B, I.N, I.K, pl->ldb, pl->transB != 0, b_outer, pb, pl->lv_b_col, pl->posB, pl->tK, pl->lBk,
-                    pl->blk16, I.K_unp, bm1, Bu, num_sms, st, zb, &zb_done);
+  s = unpack_one<T>(B, I.N, I.K, pl->ldb, pl->transB != 0, b_outer, pb, pl->lv_b_col, pl->posB, pl->tK, pl->pinv,
+                    pl->tJ, pl->lBk, pl->blk16, I.K_unp, bm1, Bu, num_sms, st, zb, &zb_done);
   if (s != IMQ_OK) return s;
   if (I.K_unp > 0) {
     if (a_outer && pl->n_grp_a > 0 && !za_done)
@@ -1031,7 +1068,8 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
     j.outer = outer;
     j.lvl = side == 0 ? pl->lv_a_row : pl->lv_b_col;
     j.pos = side == 0 ? pl->posA : pl->posB;
-    j.tK = pl->tK;
+    j.pinv = pl->pinv;
+    j.tJ = pl->tJ;
     j.lk = side == 0 ? pl->lAk : pl->lBk;
     j.blk16 = pl->blk16;
     j.K_unp = I.K_unp;
@@ -1051,7 +1089,8 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
       s = upload_table(jobs.data(), sizeof(LineJob) * (size_t)n, &dj, st);
       if (s != IMQ_OK) return s;
       s = launch_staged<T>(bm1, static_cast<const T*>(src[0]), nlines, K, ld, nw, 0, nullptr, nullptr, nullptr,
-                           nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP,
+                           nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0,
+                           side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP,
                            smem, num_sms, st, static_cast<const LineJob*>(dj), n);
       cudaFreeAsync(dj, st);
       return s;
@@ -1073,7 +1112,8 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
       if (s != IMQ_OK) return s;
       IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(k_unpack_lines<T>), smem));
       k_unpack_lines<T><<<dim3((unsigned)grid, (unsigned)n), 256, smem, st>>>(
-          static_cast<const T*>(src[0]), nlines, K, ld, P, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0, bm1,
+          static_cast<const T*>(src[0]), nlines, K, ld, P, nw, 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+          0, bm1,
           meta_smem, nullptr, nullptr, nullptr, 0, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP,
           static_cast<const LineJob*>(dj));
       s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
@@ -1088,8 +1128,8 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
     ZeroJob zj;
     if (j.outer) zj = ZeroJob{j.grpL, j.grpN, j.ngrp, side == 0 ? IMQ_A_GROUP : IMQ_B_GROUP};
     bool zeroed = false;
-    s = unpack_one<T>(static_cast<const T*>(j.X), nlines, K, ld, line_is_row, j.outer, P, j.lvl, j.pos, pl->tK, j.lk,
-                      pl->blk16, j.K_unp, bm1, j.out, num_sms, st, zj, &zeroed);
+    s = unpack_one<T>(static_cast<const T*>(j.X), nlines, K, ld, line_is_row, j.outer, P, j.lvl, j.pos, pl->tK,
+                      pl->pinv, pl->tJ, j.lk, pl->blk16, j.K_unp, bm1, j.out, num_sms, st, zj, &zeroed);
     if (s != IMQ_OK) return s;
     if (j.outer && j.ngrp > 0 && !zeroed && j.K_unp > 0)
       k_zero_unused<<<(unsigned)(j.ngrp < 4096 ? j.ngrp : 4096), 256, 0, st>>>(j.grpL, j.grpN, j.ngrp, zj.G, j.K_unp,

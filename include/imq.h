@@ -287,7 +287,12 @@ imq_status imq_plan_destroy(imq_plan_t *plan);
  * Layout (READING: the page fixes no operand order; this one is the library's):
  *   inner index p enumerates pairs (t, lA, lB) with lA < la_t, lB < lb_t (la_t = level of A column t
  *   when A is INNER else 1, lb_t = level of B row t when B is INNER else 1), ordered by exponent
- *   e = lA + lB, then lA, then t; each exponent group padded with zeros to IMQ_INNER_PAD.
+ *   e = lA + lB, then lA, then t -- or, in a plan that groups the inner indices by class, by the class
+ *   (la_t, lb_t) in descending order (la_t first) and then t; each exponent group padded with zeros to
+ *   IMQ_INNER_PAD.  (Grouping by class makes each (lA, lB) segment a few ranges of one fixed order of
+ *   the inner indices, in which the unpack kernels stage a source line, so that most 16-position blocks
+ *   are runs of consecutive staged entries; the plan groups when index order would leave many blocks
+ *   scattered.  imq_plan_maps gives the order a plan took.)
  *   OUTER rows of A: source rows sorted by level L (stable), floor(IMQ_A_GROUP / L) source rows per
  *   group of IMQ_A_GROUP unpacked rows, lines (source, level) consecutive, unused rows zero.
  *   OUTER columns of B: the same with IMQ_B_GROUP.
@@ -323,7 +328,8 @@ imq_status imq_unpack(const imq_plan_t *plan, const void *A, const void *B,
  * deltaA  device fp32[M]: the dequantisation step of every row.
  * Errors: IMQ_ERR_ARG at once; IMQ_ERR_NONFINITE, IMQ_ERR_RANGE (an entry above 32767), IMQ_ERR_PLAN
  *         through the device status word.  IMQ_ERR_UNSUPPORTED when a row (input and int16 copy) does
- *         not fit in shared memory (K above about 33 000 for BF16).  Asynchronous; allocates nothing.
+ *         not fit in shared memory (K above about 33 000 for F32 input, 50 000 for BF16).
+ *         Asynchronous; allocates nothing.
  */
 imq_status imq_rtn_quantize_unpack(const imq_plan_t *plan, const void *X, imq_dtype xt, int64_t ld,
                                    double p, int32_t beta, int8_t *A_unp, float *deltaA,

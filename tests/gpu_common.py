@@ -108,20 +108,30 @@ def check_unpacked(plan, pl: oracle.Plan, Au: np.ndarray, Bu: np.ndarray, A: np.
 
 def check_layout(plan, mp=None):
     """The library's documented layout (imq_unpack), from its own maps: inner positions grouped by
-    exponent e ascending, each group's triples ordered by (lA, t) and padded with -1 to a multiple of
-    IMQ_INNER_PAD; OUTER lines in groups of 32 holding floor(32 / L) sources of one level L, the L lines
-    of a source consecutive with levels 0..L-1, sources sorted by (level, index); unused lines last in a
-    group.  This checks the library against its own specification, not against the oracle."""
+    exponent e ascending, each group's triples ordered by lA and then either by t, or by the class
+    (la_t, lb_t) of t descending and then t (one of the two for the whole plan), and padded with -1 to a
+    multiple of IMQ_INNER_PAD; OUTER lines in groups of 32
+    holding floor(32 / L) sources of one level L, the L lines of a source consecutive with levels
+    0..L-1, sources sorted by (level, index); unused lines last in a group.  This checks the library
+    against its own specification, not against the oracle."""
     I = plan.info
     mp = plan.maps() if mp is None else mp
     lv = plan.levels()
+    # class of each inner index: its A column level when A is unpacked INNER, its B row level when B is
+    cla = lv["a_col"].astype(np.int64) if I["dir_a"] & 2 else np.ones(I["K"], np.int64)
+    clb = lv["b_row"].astype(np.int64) if I["dir_b"] & 2 else np.ones(I["K"], np.int64)
+    in_order = {True: True, False: True}  # whether every group so far follows the index / class order
     for e, off, n, padded in plan.groups():
         assert off % 128 == 0 and padded % 128 == 0 and 0 <= padded - n < 128
         t, la, lb = mp["tK"][off:off + n], mp["lAk"][off:off + n], mp["lBk"][off:off + n]
         assert (t >= 0).all() and np.all(la.astype(int) + lb == e)
-        key = la.astype(np.int64) * (1 << 32) + t
-        assert np.all(np.diff(key) > 0)
+        tt = t.astype(np.int64)
+        by_index = la.astype(np.int64) * (1 << 32) + tt
+        by_class = la.astype(np.int64) * (1 << 60) + (63 - cla[tt]) * (1 << 54) + (63 - clb[tt]) * (1 << 48) + tt
+        in_order[False] &= bool(np.all(np.diff(by_index) > 0))
+        in_order[True] &= bool(np.all(np.diff(by_class) > 0))
         assert np.all(mp["tK"][off + n:off + padded] == -1)
+    assert in_order[True] or in_order[False], "inner positions follow neither documented order"
     assert sum(g[3] for g in plan.groups()) == I["K_unp"]
     for src, lvl, lines, dirv in ((mp["srcA"], mp["lvlA"], lv["a_row"], I["dir_a"]),
                                   (mp["srcB"], mp["lvlB"], lv["b_col"], I["dir_b"])):
