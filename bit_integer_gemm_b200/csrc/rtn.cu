@@ -769,22 +769,38 @@ __global__ void __launch_bounds__(NT) k_rtn_rows_reg(const uint16_t* __restrict_
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
     for (int c = 0; c < CW; ++c) cm[j][c] = 0;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const uint16_t* xr = X + r * ld;
-    uint4 w[VPT];
-    uint32_t kmax = 0, bad = 0;
+  // Rows are dealt to the CTAs in turn.  With kPrefetch the loads of a CTA's next row are issued as soon as
+  // its current row is in registers, so that they complete while the current row is selected and
+  // quantised (registers for two rows); otherwise each row is loaded when its turn comes.
+  constexpr bool kPrefetch = VPT <= 6;
+  uint4 w[VPT];
+  auto load_row = [&](int64_t rr, uint4 (&dst)[VPT]) {
+    const uint16_t* xr = X + rr * ld;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = tid + j * NT;
-      w[j] = v < nvec ? __ldcs(reinterpret_cast<const uint4*>(xr) + v) : make_uint4(0u, 0u, 0u, 0u);
-      const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t k0 = ww[q] & 0x7FFFu, k1 = (ww[q] >> 16) & 0x7FFFu;
-        kmax = max(kmax, max(k0, k1));
-      }
+      dst[j] = v < nvec ? __ldcs(reinterpret_cast<const uint4*>(xr) + v) : make_uint4(0u, 0u, 0u, 0u);
     }
-    bad = kmax >= 0x7F80u;  // an Inf or NaN among this thread's entries (padding vectors are zeros)
+  };
+  if (kPrefetch && (int64_t)blockIdx.x < rows) load_row(blockIdx.x, w);
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    uint4 wn[VPT];
+    if constexpr (kPrefetch) {
+      if (r + gridDim.x < rows) load_row(r + gridDim.x, wn);
+    } else {
+      load_row(r, w);
+    }
+    // largest key of this thread's entries, two 15-bit keys per word at a time
+    uint32_t kmax2 = 0;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      kmax2 = __vmaxu2(kmax2, w[j].x & 0x7FFF7FFFu);
+      kmax2 = __vmaxu2(kmax2, w[j].y & 0x7FFF7FFFu);
+      kmax2 = __vmaxu2(kmax2, w[j].z & 0x7FFF7FFFu);
+      kmax2 = __vmaxu2(kmax2, w[j].w & 0x7FFF7FFFu);
+    }
+    const uint32_t kmax = max(kmax2 & 0xFFFFu, kmax2 >> 16);
+    const uint32_t bad = kmax >= 0x7F80u;  // an Inf or NaN among this thread's entries (padding is zero)
     for (int i = tid; i < 256; i += NT) hist[i] = 0;
     const uint32_t rkmax = block_reduce_max<NT>(kmax, red);  // also orders the zeroing before the counts
     if (NT == 32) __syncwarp();
@@ -885,6 +901,10 @@ __global__ void __launch_bounds__(NT) k_rtn_rows_reg(const uint16_t* __restrict_
           __stcs(o + 1, make_int4(q[4], q[5], q[6], q[7]));
         }
       }
+    }
+    if constexpr (kPrefetch) {
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) w[j] = wn[j];
     }
   }
   if (part) {

@@ -489,36 +489,53 @@ __device__ __forceinline__ Mag16w mag16_i32(const int32_t (&e)[16]) {
   }
   return r;
 }
-// The 16 int32 entries row[t0 .. t0 + 15] of a staged line (16-byte loads when t0 % 4 == 0).
-__device__ __forceinline__ void load16_i32(const int32_t* row, int t0, int32_t (&e)[16]) {
-  if ((t0 & 3) == 0) {
+// Lines staged one per team of warps (long lines) keep a 4-byte pad word after every 16 entries (pad = 4 /
+// sizeof(T) entries, else 0): a lane's 16-position block starts 32 (int16) or 64 (int32) bytes after its
+// neighbour's, which without the pad puts a warp's loads on 4 or 2 of the 32 banks; with it neighbouring
+// lanes are 9 or 17 words apart and every bank is used once.
+__device__ __forceinline__ int slot(int j, int pad) { return j + (j >> 4) * pad; }
+// Entries a staged line of K entries occupies (a padded line with 8 spare entries; the ninth word of a
+// block's loads may reach one word past a line, which stays inside the shared memory of the launch: the
+// next line or the block metadata).
+__host__ __device__ constexpr int64_t staged_len(int64_t K, int pad) {
+  return (K + 15) / 16 * (16 + pad) + (pad ? 8 : 0);
+}
+
+// The 16 int32 entries at staging positions t0 .. t0 + 15 of a staged line (16-byte loads for an unpadded
+// line and t0 % 4 == 0).
+__device__ __forceinline__ void load16_i32(const int32_t* row, int t0, int pad, int32_t (&e)[16]) {
+  if (pad == 0 && (t0 & 3) == 0) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int4 w = reinterpret_cast<const int4*>(row + t0)[q];
       e[4 * q] = w.x; e[4 * q + 1] = w.y; e[4 * q + 2] = w.z; e[4 * q + 3] = w.w;
     }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 16; ++k) e[k] = row[t0 + k];
+    return;
   }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) e[k] = row[slot(t0 + k, pad)];
 }
 // The 16 entries at staging positions j[0..15] of a staged line (0 where j < 0: padding).
-__device__ __forceinline__ void gather16_i32(const int32_t* row, const int32_t* __restrict__ j, int32_t (&e)[16]) {
+__device__ __forceinline__ void gather16_i32(const int32_t* row, const int32_t* __restrict__ j, int pad,
+                                             int32_t (&e)[16]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int4 v = reinterpret_cast<const int4*>(j)[q];
-    e[4 * q] = v.x >= 0 ? row[v.x] : 0;
-    e[4 * q + 1] = v.y >= 0 ? row[v.y] : 0;
-    e[4 * q + 2] = v.z >= 0 ? row[v.z] : 0;
-    e[4 * q + 3] = v.w >= 0 ? row[v.w] : 0;
+    e[4 * q] = v.x >= 0 ? row[slot(v.x, pad)] : 0;
+    e[4 * q + 1] = v.y >= 0 ? row[slot(v.y, pad)] : 0;
+    e[4 * q + 2] = v.z >= 0 ? row[slot(v.z, pad)] : 0;
+    e[4 * q + 3] = v.w >= 0 ? row[slot(v.w, pad)] : 0;
   }
 }
-__device__ __forceinline__ void gather16_i16(const int16_t* row, const int32_t* __restrict__ j, uint32_t (&w)[8]) {
+__device__ __forceinline__ void gather16_i16(const int16_t* row, const int32_t* __restrict__ j, int pad,
+                                             uint32_t (&w)[8]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int4 v = reinterpret_cast<const int4*>(j)[q];
-    const uint32_t e0 = v.x >= 0 ? (uint32_t)(uint16_t)row[v.x] : 0u, e1 = v.y >= 0 ? (uint32_t)(uint16_t)row[v.y] : 0u;
-    const uint32_t e2 = v.z >= 0 ? (uint32_t)(uint16_t)row[v.z] : 0u, e3 = v.w >= 0 ? (uint32_t)(uint16_t)row[v.w] : 0u;
+    const uint32_t e0 = v.x >= 0 ? (uint32_t)(uint16_t)row[slot(v.x, pad)] : 0u;
+    const uint32_t e1 = v.y >= 0 ? (uint32_t)(uint16_t)row[slot(v.y, pad)] : 0u;
+    const uint32_t e2 = v.z >= 0 ? (uint32_t)(uint16_t)row[slot(v.z, pad)] : 0u;
+    const uint32_t e3 = v.w >= 0 ? (uint32_t)(uint16_t)row[slot(v.w, pad)] : 0u;
     w[2 * q] = e0 | (e1 << 16);
     w[2 * q + 1] = e2 | (e3 << 16);
   }
@@ -542,31 +559,32 @@ __device__ __forceinline__ uint4 digits16_i32(const Mag16w& m, int l, int bm1) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// The 16 int16 entries row[t0 .. t0 + 15] of a staged line at any t0, as 8 words of two entries (low
-// half first): 16-byte loads when t0 % 8 == 0, else 32-bit loads and a funnel shift for odd t0.
-__device__ __forceinline__ void load16_i16(const int16_t* row, int t0, uint32_t (&w)[8]) {
-  if ((t0 & 7) == 0) {
+// The 16 int16 entries at staging positions t0 .. t0 + 15 of a staged line at any t0, as 8 words of two
+// entries (low half first): two 16-byte loads for an unpadded line and t0 % 8 == 0, else nine 32-bit loads
+// of entry pairs (a pair never straddles a pad word) and a funnel shift for odd t0.
+__device__ __forceinline__ void load16_i16(const int16_t* row, int t0, int pad, uint32_t (&w)[8]) {
+  if (pad == 0 && (t0 & 7) == 0) {
     const uint4 a = *reinterpret_cast<const uint4*>(row + t0), b = *reinterpret_cast<const uint4*>(row + t0 + 8);
     w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
     w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-  } else {
-    const uint32_t* r32 = reinterpret_cast<const uint32_t*>(row + (t0 & ~1));
-    uint32_t v[9];
-#pragma unroll
-    for (int i = 0; i < 9; ++i) v[i] = r32[i];  // the 9th word is inside the 32-byte padded line
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = (t0 & 1) ? __funnelshift_r(v[i], v[i + 1], 16) : v[i];
+    return;
   }
+  const int e0 = t0 & ~1;
+  uint32_t v[9];
+#pragma unroll
+  for (int i = 0; i < 9; ++i) v[i] = *reinterpret_cast<const uint32_t*>(row + slot(e0 + 2 * i, pad));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = (t0 & 1) ? __funnelshift_r(v[i], v[i + 1], 16) : v[i];
 }
 
 constexpr int kFastLevels = 4;  // OUTER lines of up to this many levels take the unrolled path
 
-// Stages source line xr (K entries) in staging order: entry t at row[pinv[t]].  Threads i0, i0 + step, ...
-// take 16-byte pieces (vec: K, the row start and the line stride allow them), four in flight before their
-// scattered shared-memory stores.
+// Stages source line xr (K entries) in the padded staged layout: entry t at row[slot(t)], or with a
+// staging order at row[slot(pinv[t])].  Threads i0, i0 + step, ... take 16-byte pieces (vec: K, the row
+// start and the line stride allow them), two in flight before their shared-memory stores.
 template <typename T>
-__device__ __forceinline__ void stage_permuted(const T* __restrict__ xr, int64_t K, bool vec,
-                                               const int32_t* __restrict__ pinv, T* row, int i0, int step) {
+__device__ __forceinline__ void stage_line(const T* __restrict__ xr, int64_t K, bool vec,
+                                           const int32_t* __restrict__ pinv, int pad, T* row, int i0, int step) {
   constexpr int V = 16 / (int)sizeof(T);
   constexpr int kBatch = 2;
   if (vec) {
@@ -582,22 +600,38 @@ __device__ __forceinline__ void stage_permuted(const T* __restrict__ xr, int64_t
       for (int u = 0; u < kBatch; ++u) {
         const int64_t q = q0 + (int64_t)u * step;
         if (q >= nq) continue;
-        const int4* pj = reinterpret_cast<const int4*>(pinv + q * V);
-        if constexpr (sizeof(T) == 2) {
+        const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        if (!pinv) {
+          // a piece lies inside one group of 16 entries: four word stores from its first slot
+          uint32_t* d = reinterpret_cast<uint32_t*>(row + slot((int)(q * V), pad));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) d[k] = ww[k];
+        } else if constexpr (sizeof(T) == 2) {
+          const int4* pj = reinterpret_cast<const int4*>(pinv + q * V);
           const int4 a = pj[0], b = pj[1];
-          row[a.x] = (T)(w[u].x & 0xFFFFu); row[a.y] = (T)(w[u].x >> 16);
-          row[a.z] = (T)(w[u].y & 0xFFFFu); row[a.w] = (T)(w[u].y >> 16);
-          row[b.x] = (T)(w[u].z & 0xFFFFu); row[b.y] = (T)(w[u].z >> 16);
-          row[b.z] = (T)(w[u].w & 0xFFFFu); row[b.w] = (T)(w[u].w >> 16);
+          row[slot(a.x, pad)] = (T)(ww[0] & 0xFFFFu); row[slot(a.y, pad)] = (T)(ww[0] >> 16);
+          row[slot(a.z, pad)] = (T)(ww[1] & 0xFFFFu); row[slot(a.w, pad)] = (T)(ww[1] >> 16);
+          row[slot(b.x, pad)] = (T)(ww[2] & 0xFFFFu); row[slot(b.y, pad)] = (T)(ww[2] >> 16);
+          row[slot(b.z, pad)] = (T)(ww[3] & 0xFFFFu); row[slot(b.w, pad)] = (T)(ww[3] >> 16);
         } else {
-          const int4 a = pj[0];
-          row[a.x] = (T)w[u].x; row[a.y] = (T)w[u].y; row[a.z] = (T)w[u].z; row[a.w] = (T)w[u].w;
+          const int4 a = *reinterpret_cast<const int4*>(pinv + q * V);
+          row[slot(a.x, pad)] = (T)ww[0]; row[slot(a.y, pad)] = (T)ww[1];
+          row[slot(a.z, pad)] = (T)ww[2]; row[slot(a.w, pad)] = (T)ww[3];
         }
       }
     }
   } else {
-    for (int64_t t = i0; t < K; t += step) row[pinv[t]] = xr[t];
+    for (int64_t t = i0; t < K; t += step) row[slot(pinv ? pinv[t] : (int)t, pad)] = xr[t];
   }
+}
+
+// Named barrier 1 (id 1) or 2 (any other id) over `n` threads (a team of the CTA).  The ids are immediates,
+// so that a CTA reserves three barriers rather than all sixteen (which would cap the CTAs per SM).
+__device__ __forceinline__ void team_sync(int id, int n) {
+  if (id == 1)
+    asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory");
+  else
+    asm volatile("bar.sync 2, %0;" ::"r"(n) : "memory");
 }
 
 // Row gather for int16 and int32 sources, the base 2^kBm1 fixed at compile time.  Each source line is
@@ -610,15 +644,17 @@ __device__ __forceinline__ void stage_permuted(const T* __restrict__ xr, int64_t
 // positions tJ.  The per-block plan metadata is staged in shared memory once per CTA.  Lines are dealt to
 // the CTAs in turn (line i to CTA i mod gridDim.x).  After its lines, each CTA zeroes the unused lines of
 // the OUTER groups dealt to it (group g to CTA g mod gridDim.x), lines n*L .. G-1 of a group of n sources
-// of level L, which no source line writes.  cta_line: lines too long for a line per warp are staged one
-// at a time per CTA by all its threads, and all its threads write its blocks.
+// of level L, which no source line writes.  teams > 0: lines too long for a line per warp are taken one
+// at a time by each of `teams` teams of warps of the CTA (each with its own staged line, padded against
+// bank conflicts, and its own named barrier), whose threads stage the line and write its blocks; one
+// team's staging overlaps another's writes.
 template <typename T, int kBm1>
 __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(const T* X, int64_t nlines, int64_t K,
                                                            int64_t ld, int nwarps, int outer, const int8_t* lvl,
                                                            const int32_t* pos, const int32_t* pinv, const int32_t* tJ,
                                                            const int8_t* lk, const int32_t* blk16, int64_t K_unp,
                                                            int8_t* out, const int32_t* grpL, const int32_t* grpN,
-                                                           int64_t ngrp, int G, int cta_line,
+                                                           int64_t ngrp, int G, int teams,
                                                            const LineJob* __restrict__ jobs) {
   extern __shared__ __align__(16) unsigned char dsm[];
   if (jobs) {
@@ -638,11 +674,12 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
     ngrp = jb.ngrp;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t Kr = (K + 15) / 16 * 16;  // staged line length in entries (32-byte multiple)
+  const int pad = teams ? 4 / (int)sizeof(T) : 0;
+  const int64_t SL = staged_len(K, pad);  // staged line length in entries
   const int nchunk = (int)(K_unp / 16);
-  // [lines of nwarps warps (one line in cta_line mode), T x Kr][block starts, int32 x nchunk]
+  // [staged lines of nwarps warps or of the teams, T x SL][block starts, int32 x nchunk]
   // [first inner levels, int8 x nchunk]
-  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)(cta_line ? 1 : nwarps) * Kr * (int64_t)sizeof(T));
+  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)(teams ? teams : nwarps) * SL * (int64_t)sizeof(T));
   int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);  // inner level of each block, -1 mixed
   for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
     s_blk[c] = blk16[c];
@@ -670,7 +707,7 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
       const int64_t pp = (int64_t)(cb + kk) * 16 + (lane & 15);
       const int32_t j = tJ[pp];
       const int lr = lk[pp];
-      const int32_t v = j >= 0 ? (int32_t)row[j] : 0;
+      const int32_t v = j >= 0 ? (int32_t)row[slot(j, pad)] : 0;
       const bool use = j >= 0 && (L == 1 || lr == 0);
       for (int l = 0; l < L; ++l) o0[(int64_t)l * K_unp + pp] = (int8_t)(use ? digit_of(v, l + lr, kBm1) : 0);
     }
@@ -694,8 +731,8 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
             for (int l = 0; l < L; ++l) *reinterpret_cast<uint4*>(o0 + (int64_t)l * K_unp + p) = make_uint4(0u, 0u, 0u, 0u);
           } else if constexpr (sizeof(T) == 2) {
             uint32_t w[8];
-            if (tb != -1) load16_i16(reinterpret_cast<const int16_t*>(row), t0, w);
-            else gather16_i16(reinterpret_cast<const int16_t*>(row), tJ + p, w);
+            if (tb != -1) load16_i16(reinterpret_cast<const int16_t*>(row), t0, pad, w);
+            else gather16_i16(reinterpret_cast<const int16_t*>(row), tJ + p, pad, w);
             const Mag16 m = mag16_i16(w);
             if (L == 1) {
               *reinterpret_cast<uint4*>(o0 + p) = digits16_from(m, lk0, kBm1);
@@ -709,8 +746,8 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
             }
           } else {
             int32_t e[16];
-            if (tb != -1) load16_i32(reinterpret_cast<const int32_t*>(row), t0, e);
-            else gather16_i32(reinterpret_cast<const int32_t*>(row), tJ + p, e);
+            if (tb != -1) load16_i32(reinterpret_cast<const int32_t*>(row), t0, pad, e);
+            else gather16_i32(reinterpret_cast<const int32_t*>(row), tJ + p, pad, e);
             const Mag16w m = mag16_i32(e);
             if (L == 1) {
               *reinterpret_cast<uint4*>(o0 + p) = digits16_i32(m, lk0, kBm1);
@@ -722,31 +759,24 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
         irregular(row, o0, L, cb, __ballot_sync(0xffffffffu, c < nchunk && !uni));
       }
   };
-  if (cta_line) {
-    // long lines: one line at a time per CTA, staged by all its threads, its blocks spread over all of them
-    T* row = reinterpret_cast<T*>(dsm);
-    for (int64_t line = blockIdx.x; line < nlines; line += gridDim.x) {
-      const T* xr = X + line * ld;
-      __syncthreads();  // the previous line has been read
-      if (pinv) {
-        stage_permuted<T>(xr, K, vec8, pinv, row, (int)threadIdx.x, (int)blockDim.x);
-      } else if (vec8) {
-        const uint4* src = reinterpret_cast<const uint4*>(xr);
-        uint4* dst = reinterpret_cast<uint4*>(row);
-        for (int64_t q = threadIdx.x; q < K / kPer16; q += blockDim.x) dst[q] = src[q];
-      } else {
-        for (int64_t t = threadIdx.x; t < K; t += blockDim.x) row[t] = xr[t];
-      }
-      __syncthreads();
-      emit(line, row, warp * 32, (int)blockDim.x);
+  if (teams) {
+    // long lines: one at a time per team, staged by the team's threads, its blocks spread over them
+    const int tpt = (int)blockDim.x / teams;  // threads per team (a multiple of 32)
+    const int team = (int)threadIdx.x / tpt, ti = (int)threadIdx.x % tpt;
+    T* row = reinterpret_cast<T*>(dsm) + (int64_t)team * SL;
+    for (int64_t line = (int64_t)blockIdx.x * teams + team; line < nlines; line += (int64_t)gridDim.x * teams) {
+      team_sync(1 + team, tpt);  // the team's previous line has been read
+      stage_line<T>(X + line * ld, K, vec8, pinv, pad, row, ti, tpt);
+      team_sync(1 + team, tpt);
+      emit(line, row, (ti >> 5) * 32, tpt);
     }
   } else if (warp < nwarps) {
-    T* row = reinterpret_cast<T*>(dsm) + (int64_t)warp * Kr;
+    T* row = reinterpret_cast<T*>(dsm) + (int64_t)warp * SL;
     for (int64_t line = (int64_t)warp * gridDim.x + blockIdx.x; line < nlines;
          line += (int64_t)gridDim.x * nwarps) {
       const T* xr = X + line * ld;
       if (pinv) {
-        stage_permuted<T>(xr, K, vec8, pinv, row, lane, 32);
+        stage_line<T>(xr, K, vec8, pinv, 0, row, lane, 32);
       } else if (vec8) {
         warp_copy16_global<4>(reinterpret_cast<const uint4*>(xr), reinterpret_cast<uint4*>(row), (int)(K / kPer16),
                               lane);
@@ -767,6 +797,304 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 2) k_unpack_lines16(
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Digit planes for lines unpacked INNER (one unpacked line per source line, the digit level set by the
+// inner position).  An entry appears at several inner positions, once per (lA, lB) segment it belongs
+// to, so its digits are computed once per line into byte planes -- plane[l][j] = digit l of the staged
+// entry at staging position j -- and every 16-position block of one inner level is then a copy of 16
+// plane bytes: a run from consecutive staging positions, or a gather through tJ.
+// ------------------------------------------------------------------------------------------------
+// Byte offset of staging position j in a plane: 4 pad bytes after every 16, so that lanes copying runs
+// 16 bytes apart read words 5 apart and every bank once.
+__device__ __forceinline__ int pslot(int j) { return j + ((j >> 4) << 2); }
+// Bytes of one plane of K positions: 20 per group of 16 and one spare group, rounded up to 16.
+__host__ __device__ constexpr int64_t plane_bytes(int64_t K) { return (((K + 15) / 16 + 1) * 20 + 15) / 16 * 16; }
+// Entries of the staged line (a 16-byte multiple).
+template <typename T>
+__host__ __device__ constexpr int64_t plane_row_len(int64_t K) {
+  return (K + 15) / 16 * 16;
+}
+
+// Digit l of 8 entries as two words (bytes in entry order): magnitudes in `a` (int16: two per word, four
+// words; int32: one per word, eight words) and byte masks of the negative entries in `neg`.
+template <typename T>
+__device__ __forceinline__ void digits8(const uint32_t* a, const uint32_t (&neg)[2], int l, int bm1,
+                                        uint32_t& lo, uint32_t& hi) {
+  const int sh = l * bm1;
+  uint32_t pd[2];
+  if constexpr (sizeof(T) == 2) {
+    if (sh >= 16) {
+      lo = hi = 0u;
+      return;
+    }
+    const uint32_t m2 = ((((1u << bm1) - 1u) << sh) & 0xFFFFu) * 0x00010001u;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      pd[h] = __byte_perm((a[2 * h] & m2) >> sh, (a[2 * h + 1] & m2) >> sh, 0x6420);
+  } else {
+    if (sh >= 31) {
+      lo = hi = 0u;
+      return;
+    }
+    const uint32_t mask = (1u << bm1) - 1u;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t d0 = (a[4 * h] >> sh) & mask, d1 = (a[4 * h + 1] >> sh) & mask;
+      const uint32_t d2 = (a[4 * h + 2] >> sh) & mask, d3 = (a[4 * h + 3] >> sh) & mask;
+      pd[h] = __byte_perm(__byte_perm(d0, d1, 0x0040), __byte_perm(d2, d3, 0x0040), 0x5410);
+    }
+  }
+  const uint32_t n0 = (0x80808080u - pd[0]) ^ 0x80808080u, n1 = (0x80808080u - pd[1]) ^ 0x80808080u;
+  lo = (pd[0] & ~neg[0]) | (n0 & neg[0]);
+  hi = (pd[1] & ~neg[1]) | (n1 & neg[1]);
+}
+
+// Teams of warps (`teams` per CTA, named barriers 1 .. teams) take one source line at a time: stage it in
+// staging order, write its P digit planes, then write its unpacked line.  Lines are dealt to the teams in
+// turn.  Blocks of one inner level copy plane bytes; blocks that mix levels (segment boundaries, padding)
+// are taken by the whole warp, one position per lane.
+template <typename T, int kBm1>
+__global__ void __launch_bounds__(256, 2) k_unpack_planes(const T* X, int64_t nlines, int64_t K, int64_t ld, int P,
+                                                          int teams, const int32_t* pinv, const int32_t* tJ,
+                                                          const int8_t* lk, const int32_t* blk16, int64_t K_unp,
+                                                          int8_t* out, const LineJob* __restrict__ jobs) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  if (jobs) {
+    const LineJob& jb = jobs[blockIdx.y];
+    X = static_cast<const T*>(jb.X);
+    pinv = jb.pinv;
+    tJ = jb.tJ;
+    lk = jb.lk;
+    blk16 = jb.blk16;
+    K_unp = jb.K_unp;
+    out = jb.out;
+  }
+  const int lane = threadIdx.x & 31;
+  const int64_t RL = plane_row_len<T>(K), PB = plane_bytes(K);
+  const int64_t team_bytes = RL * (int64_t)sizeof(T) + (int64_t)P * PB;
+  const int nchunk = (int)(K_unp / 16);
+  // [teams x (staged line, T x RL | P planes of PB bytes)][block starts, int32 x nchunk][levels, int8 x nchunk]
+  int32_t* s_blk = reinterpret_cast<int32_t*>(dsm + (int64_t)teams * team_bytes);
+  int8_t* s_lk0 = reinterpret_cast<int8_t*>(s_blk + nchunk);  // inner level of each block, -1 mixed
+  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
+    s_blk[c] = blk16[c];
+    const uint4 q = *reinterpret_cast<const uint4*>(lk + (int64_t)c * 16);
+    const uint32_t b0 = (q.x & 0xFFu) * 0x01010101u;
+    s_lk0[c] = (q.x == b0 && q.y == b0 && q.z == b0 && q.w == b0) ? (int8_t)(q.x & 0xFFu) : (int8_t)-1;
+  }
+  __syncthreads();
+  const int tpt = (int)blockDim.x / teams;  // threads per team (a multiple of 32)
+  const int team = (int)threadIdx.x / tpt, ti = (int)threadIdx.x % tpt;
+  T* row = reinterpret_cast<T*>(dsm + (int64_t)team * team_bytes);
+  uint8_t* planes = reinterpret_cast<uint8_t*>(row + RL);
+  constexpr int kPer16 = 16 / (int)sizeof(T);
+  const bool vec = (K % kPer16 == 0) && (ld % kPer16 == 0) && ((reinterpret_cast<uintptr_t>(X) & 15) == 0);
+  // The team's next line is loaded into registers (up to kPF 16-byte pieces per thread) while the current
+  // one is split and written, so that its load latency is hidden; pieces beyond that are loaded when the
+  // line is staged.
+  constexpr int kPF = 8;
+  const int64_t nq = vec ? K / kPer16 : 0;
+  uint4 pf[kPF];
+  auto prefetch = [&](int64_t ln) {
+    const uint4* src = reinterpret_cast<const uint4*>(X + ln * ld);
+#pragma unroll
+    for (int k = 0; k < kPF; ++k) {
+      const int64_t q = ti + (int64_t)k * tpt;
+      if (q < nq) pf[k] = __ldcs(src + q);
+    }
+  };
+  // piece q (entries q * kPer16 ...) into the staged line, in staging order when there is one
+  auto put = [&](int64_t q, const uint4& w) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    if (!pinv) {
+      *reinterpret_cast<uint4*>(row + q * kPer16) = w;
+    } else if constexpr (sizeof(T) == 2) {
+      const int4* pj = reinterpret_cast<const int4*>(pinv + q * kPer16);
+      const int4 a = pj[0], b = pj[1];
+      row[a.x] = (T)(ww[0] & 0xFFFFu); row[a.y] = (T)(ww[0] >> 16);
+      row[a.z] = (T)(ww[1] & 0xFFFFu); row[a.w] = (T)(ww[1] >> 16);
+      row[b.x] = (T)(ww[2] & 0xFFFFu); row[b.y] = (T)(ww[2] >> 16);
+      row[b.z] = (T)(ww[3] & 0xFFFFu); row[b.w] = (T)(ww[3] >> 16);
+    } else {
+      const int4 a = *reinterpret_cast<const int4*>(pinv + q * kPer16);
+      row[a.x] = (T)ww[0]; row[a.y] = (T)ww[1]; row[a.z] = (T)ww[2]; row[a.w] = (T)ww[3];
+    }
+  };
+  const int64_t first = (int64_t)blockIdx.x * teams + team, stride = (int64_t)gridDim.x * teams;
+  if (vec && first < nlines) prefetch(first);
+  for (int64_t line = first; line < nlines; line += stride) {
+    team_sync(1 + team, tpt);  // the team's previous line and planes have been read
+    if (vec) {
+#pragma unroll
+      for (int k = 0; k < kPF; ++k) {
+        const int64_t q = ti + (int64_t)k * tpt;
+        if (q < nq) put(q, pf[k]);
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(X + line * ld);
+      for (int64_t q = ti + (int64_t)kPF * tpt; q < nq; q += tpt) put(q, src[q]);
+      if (line + stride < nlines) prefetch(line + stride);
+    } else {
+      stage_line<T>(X + line * ld, K, false, pinv, 0, row, ti, tpt);
+    }
+    team_sync(1 + team, tpt);
+    // planes: 8 staging positions per thread and step
+    for (int m = ti; m < (int)(RL / 8); m += tpt) {
+      uint32_t a[sizeof(T) == 2 ? 4 : 8];
+      uint32_t neg[2];
+      if constexpr (sizeof(T) == 2) {
+        const uint4 w = reinterpret_cast<const uint4*>(row)[m];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        uint32_t S[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const uint32_t sgn = (ww[h] >> 15) & 0x00010001u;
+          S[h] = sgn * 0xFFFFu;
+          a[h] = (ww[h] ^ S[h]) + sgn;
+        }
+        neg[0] = __byte_perm(S[0], S[1], 0x6420);
+        neg[1] = __byte_perm(S[2], S[3], 0x6420);
+      } else {
+        const int4 w0 = reinterpret_cast<const int4*>(row)[2 * m], w1 = reinterpret_cast<const int4*>(row)[2 * m + 1];
+        const int32_t e[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t nm = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int32_t v = e[4 * h + k];
+            a[4 * h + k] = v < 0 ? 0u - (uint32_t)v : (uint32_t)v;
+            nm |= ((uint32_t)(v >> 31) & 0xFFu) << (8 * k);
+          }
+          neg[h] = nm;
+        }
+      }
+      uint32_t* dst = reinterpret_cast<uint32_t*>(planes + pslot(8 * m));
+      for (int l = 0; l < P; ++l) {
+        uint32_t lo, hi;
+        digits8<T>(a, neg, l, kBm1, lo, hi);
+        dst[0] = lo;
+        dst[1] = hi;
+        dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(dst) + PB);
+      }
+    }
+    team_sync(1 + team, tpt);
+    int8_t* o0 = out + line * K_unp;
+    for (int cb = (ti >> 5) * 32; cb < nchunk; cb += tpt) {
+      const int c = cb + lane;
+      const int tb = c < nchunk ? s_blk[c] : -1;
+      const int lk0 = c < nchunk ? s_lk0[c] : -1;
+      const bool uni = c < nchunk && (tb != -1 || lk0 >= 0);
+      if (uni) {
+        const uint8_t* pl = planes + (int64_t)lk0 * PB;
+        uint4 o;
+        if (tb != -1) {
+          // a run: staging positions j0 .. j0 + 15 -- five words of the padded plane, shifted by j0 % 4 bytes
+          const int j0 = tb >= 0 ? tb : -tb - 2;
+          const int v0 = j0 >> 2, sh = (j0 & 3) * 8;
+          uint32_t wv[5];
+#pragma unroll
+          for (int i = 0; i < 5; ++i) {
+            const int vw = v0 + i;
+            wv[i] = reinterpret_cast<const uint32_t*>(pl)[vw + (vw >> 2)];
+          }
+          o.x = __funnelshift_r(wv[0], wv[1], sh);
+          o.y = __funnelshift_r(wv[1], wv[2], sh);
+          o.z = __funnelshift_r(wv[2], wv[3], sh);
+          o.w = __funnelshift_r(wv[3], wv[4], sh);
+        } else {
+          // one inner level at scattered staging positions
+          uint32_t wv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int4 jj = reinterpret_cast<const int4*>(tJ + (int64_t)c * 16)[q];
+            const uint32_t b0 = jj.x >= 0 ? pl[pslot(jj.x)] : 0u, b1 = jj.y >= 0 ? pl[pslot(jj.y)] : 0u;
+            const uint32_t b2 = jj.z >= 0 ? pl[pslot(jj.z)] : 0u, b3 = jj.w >= 0 ? pl[pslot(jj.w)] : 0u;
+            wv[q] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+          }
+          o = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        *reinterpret_cast<uint4*>(o0 + (int64_t)c * 16) = o;
+      }
+      unsigned irr = __ballot_sync(0xffffffffu, c < nchunk && !uni);
+      while (irr) {
+        // two mixed blocks per pass: lanes 0-15 the first, 16-31 the second, one position per lane
+        const int k0 = __ffs(irr) - 1;
+        irr &= irr - 1;
+        int k1 = -1;
+        if (irr) {
+          k1 = __ffs(irr) - 1;
+          irr &= irr - 1;
+        }
+        const int kk = lane < 16 ? k0 : k1;
+        if (kk < 0) continue;
+        const int64_t pp = (int64_t)(cb + kk) * 16 + (lane & 15);
+        const int32_t j = tJ[pp];
+        const int lr = lk[pp];
+        o0[pp] = (int8_t)(j >= 0 ? planes[(int64_t)lr * PB + pslot(j)] : 0u);
+      }
+    }
+  }
+}
+
+// Whether INNER lines of K entries, P digit planes and K_unp unpacked positions take the plane kernel:
+// the lines are long (a team per line spends its barriers on enough output) and an entry appears at
+// enough positions (K_unp / K) to repay writing its P plane bytes once.
+__host__ __device__ constexpr bool planes_pay(int64_t K, int P, int64_t K_unp) {
+  return K >= 1024 && 2 * K_unp >= (int64_t)(P + 1) * K;
+}
+
+// Launch shape of the plane kernel for lines of K entries of T, P planes and nchunk blocks: two teams of
+// four warps when both teams' lines and planes and the metadata fit about half an SM (two CTAs per SM),
+// else one team of eight within the budget.  False when neither fits.
+bool planes_shape(int64_t K, size_t elem, int P, int64_t nchunk, int* teams, size_t* smem) {
+  const size_t team = (size_t)plane_row_len<int16_t>(K) * elem + (size_t)P * (size_t)plane_bytes(K);
+  const size_t meta = (size_t)nchunk * 5;
+  if (2 * team + meta <= 110 * 1024) {
+    *teams = 2;
+  } else if (team + meta <= 200 * 1024) {
+    *teams = 1;
+  } else {
+    return false;
+  }
+  *smem = (size_t)*teams * team + meta;
+  return nchunk <= kMetaMaxChunks16;
+}
+
+template <typename T, int kBm1>
+imq_status launch_planes_b(const T* X, int64_t nlines, int64_t K, int64_t ld, int P, int teams, const int32_t* pinv,
+                           const int32_t* tJ, const int8_t* lk, const int32_t* blk16, int64_t K_unp, int8_t* out,
+                           size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs, int nprob) {
+  auto kern = k_unpack_planes<T, kBm1>;
+  IMQ_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
+  int per_sm = 0;
+  IMQ_CUDA_TRY(blocks_per_sm(reinterpret_cast<const void*>(kern), 256, smem, &per_sm));
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = ((int64_t)num_sms * per_sm + nprob - 1) / nprob;
+  const int64_t need = (nlines + teams - 1) / teams;
+  if (grid > need) grid = need;
+  kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, P, teams, pinv, tJ, lk, blk16,
+                                                                 K_unp, out, jobs);
+  return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+}
+
+template <typename T>
+imq_status launch_planes(int bm1, const T* X, int64_t nlines, int64_t K, int64_t ld, int P, int teams,
+                         const int32_t* pinv, const int32_t* tJ, const int8_t* lk, const int32_t* blk16, int64_t K_unp,
+                         int8_t* out, size_t smem, int num_sms, cudaStream_t st, const LineJob* jobs, int nprob) {
+#define IMQ_PLANES(B) \
+  launch_planes_b<T, B>(X, nlines, K, ld, P, teams, pinv, tJ, lk, blk16, K_unp, out, smem, num_sms, st, jobs, nprob)
+  switch (bm1) {
+    case 1: return IMQ_PLANES(1);
+    case 2: return IMQ_PLANES(2);
+    case 3: return IMQ_PLANES(3);
+    case 4: return IMQ_PLANES(4);
+    case 5: return IMQ_PLANES(5);
+    case 6: return IMQ_PLANES(6);
+    default: return IMQ_PLANES(7);
+  }
+#undef IMQ_PLANES
+}
+
 // nprob > 1: `jobs` (device) holds the per-problem arguments and the ones given here are ignored.
 template <typename T, int kBm1>
 imq_status launch_lines16(const T* X, int64_t nlines, int64_t K, int64_t ld, int nw, int outer,
@@ -779,12 +1107,14 @@ imq_status launch_lines16(const T* X, int64_t nlines, int64_t K, int64_t ld, int
   int per_sm = 0;
   IMQ_CUDA_TRY(blocks_per_sm(reinterpret_cast<const void*>(kern), 256, smem, &per_sm));
   if (per_sm < 1) per_sm = 1;
-  // every resident slot once over the whole batch
+  // every resident slot once over the whole batch; a CTA takes a line per warp or per team at a time
+  const int teams = nw < 0 ? -nw : 0;
   int64_t grid = ((int64_t)num_sms * per_sm + nprob - 1) / nprob;
-  if (grid > nlines) grid = nlines;
-  kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, nw, outer, lvl, pos, pinv, tJ, lk,
-                                                                 blk16, K_unp, out, grpL, grpN, ngrp, G,
-                                                                 nw == 0 ? 1 : 0, jobs);
+  const int64_t need = teams ? (nlines + teams - 1) / teams : nlines;
+  if (grid > need) grid = need;
+  kern<<<dim3((unsigned)grid, (unsigned)nprob), 256, smem, st>>>(X, nlines, K, ld, nw > 0 ? nw : 0, outer, lvl, pos,
+                                                                 pinv, tJ, lk, blk16, K_unp, out, grpL, grpN, ngrp,
+                                                                 G, teams, jobs);
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
@@ -811,18 +1141,28 @@ imq_status launch_staged(int bm1, const T* X, int64_t nlines, int64_t K, int64_t
 }
 
 // Launch shape of the staged-line kernel for lines of K entries of T and nchunk 16-position blocks: a
-// line per warp (8 warps while their lines fit in 64 KB, so that three CTAs share an SM), or for lines
-// above 16 KB one line per CTA (nw = 0: all 8 warps stage it and write its blocks).  False when the
-// line and the block metadata (5 bytes per block, staged whole) do not fit the shared-memory budget.
+// line per warp (*nw_out > 0 warps, 8 while their lines fit in 64 KB, so that three CTAs share an SM),
+// or for lines above 16 KB a line per team (*nw_out = -teams: two teams of four warps when two padded
+// lines and the metadata fit the budget, else one of eight).  False when nothing fits the shared-memory
+// budget or the block metadata (5 bytes per block, staged whole) is too long.
 bool staged_shape(int64_t K, size_t elem, int64_t nchunk, int* nw_out, size_t* smem_out) {
-  const int64_t line_bytes = (K + 15) / 16 * 16 * (int64_t)elem;
-  const bool cta_line = line_bytes > 16 * 1024;
-  int nw = cta_line ? 0 : (int)((64 * 1024) / line_bytes);
-  if (nw > 8) nw = 8;
-  const size_t smem = (size_t)(cta_line ? 1 : nw) * line_bytes + (size_t)nchunk * 5;
-  *nw_out = nw;
+  constexpr size_t kBudget = 200 * 1024;
+  const size_t meta = (size_t)nchunk * 5;
+  const int64_t plain = staged_len(K, 0) * (int64_t)elem;
+  size_t smem;
+  if (plain <= 16 * 1024) {
+    int nw = (int)((64 * 1024) / plain);
+    if (nw > 8) nw = 8;
+    *nw_out = nw;
+    smem = (size_t)nw * plain + meta;
+  } else {
+    const size_t padded = (size_t)staged_len(K, 4 / (int)elem) * elem;
+    const int teams = 2 * padded + meta <= kBudget ? 2 : 1;
+    *nw_out = -teams;
+    smem = (size_t)teams * padded + meta;
+  }
   *smem_out = smem;
-  return nchunk <= kMetaMaxChunks16 && smem <= 200 * 1024;
+  return nchunk <= kMetaMaxChunks16 && smem <= kBudget;
 }
 
 // Row gather for lines too long for shared-memory planes: digits are computed from the source line in
@@ -934,6 +1274,14 @@ imq_status unpack_one(const T* X, int64_t nlines, int64_t K, int64_t ld, bool li
                       const ZeroJob& zj, bool* zeroed) {
   *zeroed = false;
   if (nlines == 0 || K_unp == 0) return IMQ_OK;
+  // long rows unpacked INNER: the digit-plane kernel
+  if (line_is_row && !outer && bm1 >= 1 && bm1 <= 7 && planes_pay(K, P, K_unp)) {
+    int teams = 0;
+    size_t smem = 0;
+    if (planes_shape(K, sizeof(T), P, K_unp / 16, &teams, &smem))
+      return launch_planes<T>(bm1, X, nlines, K, ld, P, teams, pinv, tJ, lk, blk16, K_unp, out, smem, num_sms, st,
+                              nullptr, 1);
+  }
   // rows (int16 or int32): the staged-line kernel, which also zeroes the unused OUTER lines
   {
     const int64_t nchunk = K_unp / 16;
@@ -1082,6 +1430,44 @@ imq_status unpack_side_batch(const imq_plan_t* const* pls, int n, const void* co
   if (nlines == 0 || nchunk == 0) return IMQ_OK;
   void* dj = nullptr;
   imq_status s = IMQ_OK;
+  if (line_is_row && bm1 >= 1 && bm1 <= 7 && K >= 1024) {
+    // the problems whose lines are unpacked INNER take the digit-plane kernel in one launch; the others
+    // (OUTER lines) follow as a batch of their own
+    std::vector<LineJob> in_jobs;
+    std::vector<const imq_plan_t*> o_pls;
+    std::vector<const void*> o_src;
+    std::vector<int8_t*> o_dst;
+    int P_in = 1;
+    int64_t nchunk_in = 0;
+    for (int h = 0; h < n; ++h) {
+      const imq_plan_info& Ih = pls[h]->info;
+      const int pih = ((side == 0 ? Ih.dir_a : Ih.dir_b) & IMQ_DIR_INNER) ? (side == 0 ? Ih.lmax_a_col : Ih.lmax_b_row) : 1;
+      if (jobs[h].outer || !planes_pay(K, pih, Ih.K_unp)) {
+        o_pls.push_back(pls[h]);
+        o_src.push_back(src[h]);
+        o_dst.push_back(dst[h]);
+        continue;
+      }
+      const imq_plan_info& I = pls[h]->info;
+      const int dir = side == 0 ? I.dir_a : I.dir_b;
+      const int pi = (dir & IMQ_DIR_INNER) ? (side == 0 ? I.lmax_a_col : I.lmax_b_row) : 1;
+      P_in = P_in > pi ? P_in : pi;
+      nchunk_in = nchunk_in > I.K_unp / 16 ? nchunk_in : I.K_unp / 16;
+      in_jobs.push_back(jobs[h]);
+    }
+    int teams = 0;
+    size_t smem = 0;
+    if (!in_jobs.empty() && planes_shape(K, sizeof(T), P_in, nchunk_in, &teams, &smem)) {
+      s = upload_table(in_jobs.data(), sizeof(LineJob) * in_jobs.size(), &dj, st);
+      if (s != IMQ_OK) return s;
+      s = launch_planes<T>(bm1, static_cast<const T*>(src[0]), nlines, K, ld, P_in, teams, nullptr, nullptr, nullptr,
+                           nullptr, 0, nullptr, smem, num_sms, st, static_cast<const LineJob*>(dj),
+                           (int)in_jobs.size());
+      cudaFreeAsync(dj, st);
+      if (s != IMQ_OK || o_pls.empty()) return s;
+      return unpack_side_batch<T>(o_pls.data(), (int)o_pls.size(), o_src.data(), o_dst.data(), side, num_sms, st);
+    }
+  }
   {
     int nw = 0;
     size_t smem = 0;
