@@ -106,6 +106,81 @@ __global__ void __launch_bounds__(256) k_line_max(const T* __restrict__ X, int64
       if (cmax[c]) atomicMax(colmax + c, (int32_t)cmax[c]);
 }
 
+// The line maxima of the matrices of a batch of plans in one launch (blockIdx.y = matrix): a block per
+// stored row at a time, 16-byte loads where the matrix allows; column maxima through shared memory, then
+// atomicMax into colmax, which k_zero_batch has cleared.  Rows are written whole (0 for empty rows).
+struct LineMaxJob {
+  const void* X;
+  int64_t rows, cols, ld;
+  int32_t* rowmax;
+  int32_t* colmax;
+};
+template <typename T>
+__global__ void __launch_bounds__(256) k_line_max_batch(const LineMaxJob* __restrict__ jobs) {
+  extern __shared__ uint32_t cmax_s[];
+  __shared__ uint32_t red[8];
+  const LineMaxJob J = jobs[blockIdx.y];
+  const T* X = static_cast<const T*>(J.X);
+  const int tid = threadIdx.x;
+  constexpr int V = 16 / (int)sizeof(T);
+  const bool vec = J.cols % V == 0 && J.ld % V == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+  for (int64_t c = tid; c < J.cols; c += 256) cmax_s[c] = 0;
+  __syncthreads();
+  for (int64_t r = blockIdx.x; r < J.rows; r += gridDim.x) {
+    uint32_t m = 0;
+    if (vec) {
+      const uint4* xr = reinterpret_cast<const uint4*>(X + r * J.ld);
+      for (int64_t q = tid; q < J.cols / V; q += 256) {
+        const uint4 w = __ldcs(xr + q);
+        const T* e = reinterpret_cast<const T*>(&w);
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+          const int64_t v = e[k];
+          const uint32_t a = (uint32_t)(v < 0 ? -v : v);
+          m = max(m, a);
+          cmax_s[q * V + k] = max(cmax_s[q * V + k], a);
+        }
+      }
+    } else {
+      for (int64_t c = tid; c < J.cols; c += 256) {
+        const int64_t v = X[r * J.ld + c];
+        const uint32_t a = (uint32_t)(v < 0 ? -v : v);
+        m = max(m, a);
+        cmax_s[c] = max(cmax_s[c], a);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t r2 = 0;
+      for (int w = 0; w < 8; ++w) r2 = max(r2, red[w]);
+      J.rowmax[r] = (int32_t)r2;
+    }
+    __syncthreads();
+  }
+  for (int64_t c = tid; c < J.cols; c += 256)
+    if (cmax_s[c]) atomicMax(J.colmax + c, (int32_t)cmax_s[c]);
+}
+
+// Clears the byte ranges of a batch (blockIdx.y = range; every range 16-byte aligned, a 4-byte multiple).
+struct ZeroSpan {
+  void* p;
+  int64_t bytes;
+};
+__global__ void __launch_bounds__(256) k_zero_batch(const ZeroSpan* __restrict__ spans) {
+  const ZeroSpan z = spans[blockIdx.y];
+  uint4* q = static_cast<uint4*>(z.p);
+  const int64_t n16 = z.bytes / 16;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
+    q[i] = make_uint4(0u, 0u, 0u, 0u);
+  uint32_t* w = static_cast<uint32_t*>(z.p);
+  for (int64_t i = n16 * 4 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < z.bytes / 4;
+       i += (int64_t)gridDim.x * blockDim.x)
+    w[i] = 0u;
+}
+
 // ------------------------------------------------------------------------------------------------
 // levels and summary.  Vectors: 0 = A rows (M), 1 = A cols (K), 2 = B rows (K), 3 = B cols (N).
 // ------------------------------------------------------------------------------------------------
@@ -120,9 +195,10 @@ struct LevelArgs {
   const int32_t* status;  // the device status word, copied into the summary by block 0
   HostSummary* hsum;      // device address of the mapped host copy
   uint32_t seq;           // written to hsum->seq once hsum->s is complete
+  uint32_t nblk;          // blocks of this plan's level kernel (the last one publishes the summary)
 };
 
-__global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
+__device__ __forceinline__ void levels_body(const LevelArgs& a) {
   __shared__ unsigned int hist[4][kLv];
   __shared__ unsigned int joint[kLv][kLv];
   __shared__ unsigned long long ssum[4], soor[4];
@@ -138,7 +214,7 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
     slmax[tid] = 0;
   }
   __syncthreads();
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t stride = (int64_t)a.nblk * blockDim.x;
   unsigned long long bsum[4] = {0, 0, 0, 0}, boor[4] = {0, 0, 0, 0};
   unsigned int blmax[4] = {0, 0, 0, 0};
   // the bound sum_t max|A[:,t]| * max|B[t,:]| as two 64-bit sums, of the products' low 32-bit halves and
@@ -227,7 +303,7 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   __shared__ bool last;
   __threadfence();
   __syncthreads();
-  if (tid == 0) last = atomicAdd(&a.sum->done, 1u) == gridDim.x - 1;
+  if (tid == 0) last = atomicAdd(&a.sum->done, 1u) == a.nblk - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
@@ -236,6 +312,16 @@ __global__ void __launch_bounds__(256) k_levels(LevelArgs a) {
   __syncthreads();
   // the fence above orders the summary before `seq`; nothing after it needs to wait for the write
   if (tid == 0) *reinterpret_cast<volatile uint32_t*>(&a.hsum->seq) = a.seq;
+}
+
+__global__ void __launch_bounds__(256) k_levels(LevelArgs a) { levels_body(a); }
+
+// The level kernels of a batch of plans in one launch: blockIdx.y = plan, its blocks blockIdx.x <
+// nblk[plan] (the others return at once).
+__global__ void __launch_bounds__(256) k_levels_batch(const LevelArgs* __restrict__ args, const int* __restrict__ nblk) {
+  if ((int)blockIdx.x >= nblk[blockIdx.y]) return;
+  const LevelArgs a = args[blockIdx.y];
+  levels_body(a);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -858,11 +944,29 @@ __global__ void __launch_bounds__(1024) k_plan_order(const __grid_constant__ Map
   stage_class(ea, eb, stage_order(m), m.lva, m.lvb, m.a_inner, m.b_inner, m.K);
 }
 
-__global__ void __launch_bounds__(1024) k_plan_maps(const __grid_constant__ MapsArgs m) {
+__device__ __forceinline__ void maps_body(const MapsArgs& m, int bx);
+
+__global__ void __launch_bounds__(1024) k_plan_maps(const __grid_constant__ MapsArgs m) { maps_body(m, (int)blockIdx.x); }
+
+// The order and maps kernels of a batch of plans in one launch each: blockIdx.y = plan, reading its
+// arguments from a device table; blocks past the plan's own count return at once.
+__global__ void __launch_bounds__(1024) k_plan_order_batch(const MapsArgs* __restrict__ tab) {
+  const MapsArgs& m = tab[blockIdx.y];
+  if (!m.perm || (int)blockIdx.x >= m.maxla * m.maxlb) return;
+  const int bx = (int)blockIdx.x;
+  const int ea = m.maxla - bx / m.maxlb, eb = m.maxlb - bx % m.maxlb;
+  stage_class(ea, eb, stage_order(m), m.lva, m.lvb, m.a_inner, m.b_inner, m.K);
+}
+__global__ void __launch_bounds__(1024) k_plan_maps_batch(const MapsArgs* __restrict__ tab) {
+  const MapsArgs& m = tab[blockIdx.y];
+  if ((int)blockIdx.x >= m.ngrp + m.a.ncls + m.b.ncls) return;
+  maps_body(m, (int)blockIdx.x);
+}
+
+__device__ __forceinline__ void maps_body(const MapsArgs& m, int bx) {
   const InnerSeg* segs = m.inline_tables ? m.t.segs : m.segs;
   const OuterClass* cls = m.inline_tables ? m.t.cls : m.cls;
   const InnerGroup* grps = m.inline_tables ? m.t.grps : m.grps;
-  const int bx = (int)blockIdx.x;
   if (bx < m.ngrp) {
     inner_map_group(grps[bx], segs, stage_order(m), m.lva, m.lvb, m.a_inner, m.b_inner, m.K, m.tK, m.tJ, m.lAk,
                     m.lBk, m.blk16);
@@ -1050,6 +1154,14 @@ imq_status launch_line_max(const void* X, imq_dtype it, int64_t rows, int64_t co
   return cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
 }
 
+// The maps kernels of a batch run as one launch, except in the debug build, whose index checks follow each
+// plan's own maps.
+#ifdef IMQ_DEBUG
+constexpr bool kBatchMaps = false;
+#else
+constexpr bool kBatchMaps = true;
+#endif
+
 // One plan in the making: its arguments and what its first stage leaves for the second.
 struct PlanJob {
   const void* A;
@@ -1067,12 +1179,24 @@ struct PlanJob {
   const int32_t* b_rowmax;
   const int32_t* b_colmax;
   int slot;  // summary slot of the batch
+  // batched: this plan's kernels are queued by build_plans together with the other plans' of its batch
+  // (one launch per kind); plan_begin and plan_finish only record their arguments
+  bool batched = false;
   // state after plan_begin
   imq_plan_t* pl = nullptr;
   char* blk1 = nullptr;
   Summary* dsum = nullptr;
   size_t o_segs = 0, o_cls = 0, o_grps = 0, o_E = 0;
   uint32_t seq = 0;
+  LevelArgs la{};
+  int nlm = 0;  // line maxima to compute (batched)
+  LineMaxJob lm[2]{};
+  int nzero = 0;
+  ZeroSpan zero[3]{};
+  // state after plan_finish (batched)
+  bool has_maps = false;
+  int order_blocks = 0, maps_blocks = 0;
+  MapsArgs maps{};
 };
 
 // Frees a plan that failed before it was returned.
@@ -1216,6 +1340,12 @@ imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaS
     lmx[1] = a_colmax;
     lmx[2] = b_rowmax;
     lmx[3] = b_colmax;
+  } else if (job.batched) {
+    // recorded for the batch's line-maxima launch; the column maxima are cleared first
+    job.lm[0] = transA ? LineMaxJob{A, K, M, lda, mx[1], mx[0]} : LineMaxJob{A, M, K, lda, mx[0], mx[1]};
+    job.lm[1] = transB ? LineMaxJob{B, N, K, ldb, mx[3], mx[2]} : LineMaxJob{B, K, N, ldb, mx[2], mx[3]};
+    job.nlm = 2;
+    for (int q = 0; q < 2; ++q) job.zero[job.nzero++] = ZeroSpan{job.lm[q].colmax, job.lm[q].cols * 4};
   } else {
     // A stored M x K (or K x M when transposed); B stored K x N (or N x K)
     imq_status e = transA ? launch_line_max(A, it, K, M, lda, mx[1], mx[0], st)
@@ -1231,7 +1361,11 @@ imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaS
       if (N && cudaMemsetAsync(mx[3], 0, (size_t)N * 4, st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
     }
   }
-  if (cudaMemsetAsync(dsum, 0, sizeof(Summary), st) != cudaSuccess) return fail(IMQ_ERR_CUDA);
+  if (job.batched) {
+    job.zero[job.nzero++] = ZeroSpan{dsum, (int64_t)sizeof(Summary)};
+  } else if (cudaMemsetAsync(dsum, 0, sizeof(Summary), st) != cudaSuccess) {
+    return fail(IMQ_ERR_CUDA);
+  }
   LevelArgs la;
   la.keep_a_col = have_max ? mx[1] : nullptr;  // k_levels copies the caller's A column maxima there
   for (int v = 0; v < 4; ++v) {
@@ -1324,7 +1458,11 @@ imq_status plan_begin(PlanJob& job, Pinned& pin, DeviceState* ds, int dev, cudaS
     int64_t grid = (nmax + 255) / 256;
     if (grid > ds->num_sms * 2) grid = ds->num_sms * 2;
     if (grid < 1) grid = 1;
-    k_levels<<<(unsigned)grid, 256, 0, st>>>(la);
+    la.nblk = (uint32_t)grid;
+    if (job.batched)
+      job.la = la;
+    else
+      k_levels<<<(unsigned)grid, 256, 0, st>>>(la);
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
   job.pl = pl;
@@ -1752,9 +1890,16 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
            pl->grpA_L, pl->grpA_n};
     m.b = {cls_b0, b_outer ? cls_b1 - cls_b0 : 0, pl->lv_b_col, N, IMQ_B_GROUP, pl->posB, pl->srcB,
            pl->grpB_L, pl->grpB_n};
-    if (permuted) k_plan_order<<<maxla * maxlb, 1024, 0, st>>>(m);
     const int blocks = ng + m.a.ncls + m.b.ncls;
-    if (blocks > 0) k_plan_maps<<<blocks, 1024, 0, st>>>(m);
+    if (job.batched && kBatchMaps) {
+      job.has_maps = true;
+      job.order_blocks = permuted ? maxla * maxlb : 0;
+      job.maps_blocks = blocks;
+      job.maps = m;
+    } else {
+      if (permuted) k_plan_order<<<maxla * maxlb, 1024, 0, st>>>(m);
+      if (blocks > 0) k_plan_maps<<<blocks, 1024, 0, st>>>(m);
+    }
   }
   if (cudaGetLastError() != cudaSuccess) return fail(IMQ_ERR_CUDA);
 #ifdef IMQ_DEBUG
@@ -1805,6 +1950,88 @@ imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B,
                        int32_t b, imq_strategy strategy, const int32_t* a_rowmax, const int32_t* a_colmax,
                        const int32_t* b_rowmax, const int32_t* b_colmax, imq_plan_t** out, cudaStream_t st);
 
+// Stage 1 of a batch of plans: the summaries and column maxima cleared, the line maxima, the level
+// kernels -- one launch each for the whole batch.
+imq_status launch_stage1_batch(std::vector<PlanJob>& jobs, imq_dtype it, DeviceState* ds, cudaStream_t st) {
+  std::vector<ZeroSpan> zero;
+  std::vector<LineMaxJob> lm;
+  std::vector<LevelArgs> la;
+  std::vector<int> nblk;
+  int64_t max_rows = 1, max_cols = 0;
+  int max_blk = 1;
+  int64_t max_bytes = 16;
+  for (PlanJob& j : jobs) {
+    for (int q = 0; q < j.nzero; ++q) {
+      zero.push_back(j.zero[q]);
+      max_bytes = j.zero[q].bytes > max_bytes ? j.zero[q].bytes : max_bytes;
+    }
+    for (int q = 0; q < j.nlm; ++q) {
+      lm.push_back(j.lm[q]);
+      max_rows = j.lm[q].rows > max_rows ? j.lm[q].rows : max_rows;
+      max_cols = j.lm[q].cols > max_cols ? j.lm[q].cols : max_cols;
+    }
+    la.push_back(j.la);
+    nblk.push_back((int)j.la.nblk);
+    max_blk = (int)j.la.nblk > max_blk ? (int)j.la.nblk : max_blk;
+  }
+  void* dz = nullptr;
+  void* dl = nullptr;
+  void* da = nullptr;
+  void* dn = nullptr;
+  imq_status s = upload_table(zero.data(), sizeof(ZeroSpan) * zero.size(), &dz, st);
+  if (s == IMQ_OK && !lm.empty()) s = upload_table(lm.data(), sizeof(LineMaxJob) * lm.size(), &dl, st);
+  if (s == IMQ_OK) s = upload_table(la.data(), sizeof(LevelArgs) * la.size(), &da, st);
+  if (s == IMQ_OK) s = upload_table(nblk.data(), sizeof(int) * nblk.size(), &dn, st);
+  if (s == IMQ_OK) {
+    const int64_t zb = (max_bytes / 16 + 255) / 256;
+    k_zero_batch<<<dim3((unsigned)(zb < 64 ? zb : 64), (unsigned)zero.size()), 256, 0, st>>>(
+        static_cast<const ZeroSpan*>(dz));
+    if (!lm.empty()) {
+      // about eight blocks per SM over the whole batch, at most one per row
+      int64_t gx = ((int64_t)ds->num_sms * 8 + (int64_t)lm.size() - 1) / (int64_t)lm.size();
+      if (gx > max_rows) gx = max_rows;
+      const size_t smem = (size_t)max_cols * 4;
+      const dim3 g((unsigned)gx, (unsigned)lm.size());
+      if (it == IMQ_I16) {
+        if (ensure_smem(reinterpret_cast<const void*>(k_line_max_batch<int16_t>), smem) != cudaSuccess) s = IMQ_ERR_CUDA;
+        else k_line_max_batch<int16_t><<<g, 256, smem, st>>>(static_cast<const LineMaxJob*>(dl));
+      } else {
+        if (ensure_smem(reinterpret_cast<const void*>(k_line_max_batch<int32_t>), smem) != cudaSuccess) s = IMQ_ERR_CUDA;
+        else k_line_max_batch<int32_t><<<g, 256, smem, st>>>(static_cast<const LineMaxJob*>(dl));
+      }
+    }
+    if (s == IMQ_OK)
+      k_levels_batch<<<dim3((unsigned)max_blk, (unsigned)la.size()), 256, 0, st>>>(static_cast<const LevelArgs*>(da),
+                                                                                  static_cast<const int*>(dn));
+    if (cudaGetLastError() != cudaSuccess) s = IMQ_ERR_CUDA;
+  }
+  for (void* p : {dz, dl, da, dn})
+    if (p) cudaFreeAsync(p, st);
+  return s;
+}
+
+// Stage 2 of a batch of plans: the order kernels, then the maps kernels, one launch each.
+imq_status launch_stage2_batch(std::vector<PlanJob>& jobs, cudaStream_t st) {
+  std::vector<MapsArgs> tab;
+  int max_order = 0, max_maps = 0;
+  for (PlanJob& j : jobs) {
+    if (!j.has_maps) continue;
+    tab.push_back(j.maps);
+    max_order = j.order_blocks > max_order ? j.order_blocks : max_order;
+    max_maps = j.maps_blocks > max_maps ? j.maps_blocks : max_maps;
+  }
+  if (tab.empty() || (max_order == 0 && max_maps == 0)) return IMQ_OK;
+  void* dt = nullptr;
+  imq_status s = upload_table(tab.data(), sizeof(MapsArgs) * tab.size(), &dt, st);
+  if (s != IMQ_OK) return s;
+  const MapsArgs* t = static_cast<const MapsArgs*>(dt);
+  if (max_order > 0) k_plan_order_batch<<<dim3((unsigned)max_order, (unsigned)tab.size()), 1024, 0, st>>>(t);
+  if (max_maps > 0) k_plan_maps_batch<<<dim3((unsigned)max_maps, (unsigned)tab.size()), 1024, 0, st>>>(t);
+  s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+  cudaFreeAsync(dt, st);
+  return s;
+}
+
 // Builds a plan; see imq_plan in include/imq.h.
 imq_status build_plan(const void* A, const void* B, imq_dtype it, int64_t M, int64_t K, int64_t N,
                       int32_t transA, int64_t lda, int32_t transB, int64_t ldb, int32_t b,
@@ -1848,8 +2075,12 @@ imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B,
       }
     return e;
   };
+  // A batch queues each kind of plan kernel once for all its plans (the hybrid's choice kernels stay per
+  // plan; the debug build's index checks follow each plan's maps, so there stage 2 stays per plan too).
+  const bool batched = batch > 1 && strategy != IMQ_HYBRID && (have_max || (M <= 32768 && K <= 32768 && N <= 32768));
   for (int h = 0; h < batch; ++h) {
     PlanJob& j = jobs[h];
+    j.batched = batched;
     j.A = static_cast<const char*>(A) + (size_t)h * strideA * esz;
     j.B = static_cast<const char*>(B) + (size_t)h * strideB * esz;
     j.it = it;
@@ -1870,6 +2101,10 @@ imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B,
     s = plan_begin(j, pin, ds, dev, st);
     if (s != IMQ_OK) return drop(h, s);
   }
+  if (batched) {
+    s = launch_stage1_batch(jobs, it, ds, st);
+    if (s != IMQ_OK) return drop(batch, s);
+  }
   std::vector<Summary> sums((size_t)batch);
   for (int h = 0; h < batch; ++h) {
     s = plan_wait(jobs[h], pin, st, &sums[h]);
@@ -1877,6 +2112,10 @@ imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B,
   }
   for (int h = 0; h < batch; ++h) {
     s = plan_finish(jobs[h], sums[h], pin, ds, st, &out[h]);
+    if (s != IMQ_OK) return drop(batch, s);
+  }
+  if (batched) {
+    s = launch_stage2_batch(jobs, st);
     if (s != IMQ_OK) return drop(batch, s);
   }
   return IMQ_OK;
