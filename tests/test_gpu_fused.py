@@ -75,6 +75,55 @@ def test_fused_matches_separate_path_and_oracle(imq, dtype, shape, b):
     plan.destroy()
 
 
+def _class_ordered(plan):
+    """True when some segment of the plan's inner layout is not in index order (the plan grouped its inner
+    indices by level class: the staging order)."""
+    mp = plan.maps()
+    for e, off, n, padded in plan.groups():
+        t = mp["tK"][off:off + n].astype(np.int64)
+        la = mp["lAk"][off:off + n].astype(np.int64)
+        key = la * (1 << 32) + t
+        if not np.all(np.diff(key) > 0):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fused_with_class_ordered_plan(imq, dtype):
+    """A plan whose inner indices are grouped by level class (half the columns of X and half the rows of W
+    scaled down, so that every segment beyond the first is about half dense): the fused path stages its
+    int16 row in that order and must still equal the separate path, the oracle and the exact product."""
+    M, K, N, b, p, beta = 300, 520, 270, 3, 0.95, 15
+    rng = np.random.default_rng(2024)
+    X = rng.standard_normal((M, K), dtype=np.float32)
+    X[:, rng.permutation(K)[:K // 2]] *= np.float32(0.4)
+    W = rng.standard_normal((K, N), dtype=np.float32) * np.float32(0.02)
+    W[rng.permutation(K)[:K // 2], :] *= np.float32(0.4)
+    Xs = workloads.Stored("X", workloads.f32_to_bf16_bits(X) if dtype == "bf16" else X, dtype)
+    Ws = workloads.Stored("W", workloads.f32_to_bf16_bits(W), "bf16")
+    Xd, Wd = to_device(Xs), to_device(Ws)
+    qx = imq.imq_rtn_quantize(Xd, imq.IMQ_PER_ROW, p, beta)
+    qw = _weight(imq, Wd, p, beta)
+    plan = imq.imq_plan(qx.xint, qw.xint, b, imq.IMQ_COL_ROW, transB=True,
+                        maxes=(qx.rowmax, qx.colmax, qw.rowmax, qw.colmax))
+    assert _class_ordered(plan), "the case was built to take the class-grouped order"
+    Au, Bu = imq.imq_unpack(plan, qx.xint, qw.xint)
+    Af, dAf = imq.imq_rtn_quantize_unpack(plan, Xd, p, beta)
+    torch.cuda.synchronize()
+    assert imq.imq_device_status(clear=True) == imq.IMQ_OK
+    assert torch.equal(Af, Au), "fused A' differs from quantise + unpack"
+    xi, dx, _ = oracle.rtn_quantize(oracle.as_f32(Xs.data, dtype), oracle.PER_ROW, p, beta)
+    wi, dw, _ = oracle.rtn_quantize(oracle.as_f32(Ws.data, "bf16"), oracle.PER_COL, p, beta)
+    pl = oracle.plan(xi, wi, b, oracle.COL_ROW)
+    check_unpacked(plan, pl, Af.cpu().numpy(), Bu.cpu().numpy(), xi, wi)
+    C, Cf = imq.imq_gemm_unpacked(plan, Af, Bu, dAf, imq.IMQ_PER_ROW, qw.delta, imq.IMQ_PER_COL)
+    torch.cuda.synchronize()
+    want = oracle.gemm_exact(xi, wi)
+    assert np.array_equal(C.cpu().numpy().astype(np.int64), want)
+    assert_f32_close(Cf.cpu().numpy(), oracle.dequant(want, dx, oracle.PER_ROW, dw, oracle.PER_COL))
+    plan.destroy()
+
+
 def test_fused_q_proj_kept_weight_new_batches(imq):
     """q_proj shapes: the plan is made once with widened column maxima (each raised to the largest value
     with the same number of base-R digits, R^L - 1) and W' is unpacked once; three new activation batches
