@@ -10,16 +10,18 @@
 // the digits of every inner level); for the pure strategies one of L > 1, lk > 0 never holds.
 //
 // Both unpacked operands are K-major (the inner index contiguous) because that is what the tcgen05
-// GEMM reads through TMA.  The kernels cover the two storage orders of a source matrix:
-//   k_unpack_lines16  int16 source lines that are stored rows (A, or B given as B^T): one warp per line
-//                  with the line staged, digits computed per 16-position block for every output level;
-//                  it also zeroes the unused lines of OUTER groups.
-//   k_unpack_lines / k_unpack_rows  the same for int32 sources (and lines too long to stage): digit
-//                  planes in shared memory, 16-byte copies out of them.
-//   k_unpack_rows  the source line is a stored row (A, or B given as B^T): a CTA writes the digit planes
-//                  of a batch of lines to shared memory and streams out their unpacked lines, 16-byte
-//                  copies for the inner blocks the plan marked contiguous (k_unpack_rows_direct gathers
-//                  from global memory when the planes do not fit).
+// GEMM reads through TMA.  A source line is staged in the plan's staging order (index order, or its
+// inner indices grouped by level class when the plan chose that), so that most 16-position blocks are
+// runs of consecutive staged entries.  The kernels:
+//   k_unpack_planes   long stored rows unpacked INNER (one unpacked line per source line): a team of
+//                  warps per line writes each entry's digits once into byte planes, then copies every
+//                  block out of them; the team's next line is loaded meanwhile.
+//   k_unpack_lines16  other stored rows (A, or B given as B^T), int16 or int32: a line per warp (or per
+//                  team of warps for long lines); per block of one inner level the magnitudes of its 16
+//                  entries are taken once and the digit of every output line emitted; blocks that mix
+//                  levels are taken by the whole warp; it also zeroes the unused lines of OUTER groups.
+//   k_unpack_lines / k_unpack_rows  fallbacks with per-line digit planes (lines too long for the
+//                  kernels above); k_unpack_rows_direct gathers from global memory when planes do not fit.
 //   k_unpack_cols  the source line is a stored column (B, or A given as A^T): a CTA transposes a
 //                  128 (inner) x 32 (lines) tile through shared memory, reading 64-byte row segments
 //                  and writing 128-byte segments of unpacked lines.
