@@ -37,6 +37,7 @@
 
 #include <mutex>
 #include <type_traits>
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -53,6 +54,7 @@ constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr int kMaxSplits = 16;   // K splits of one output tile
 constexpr int kMaxPieces = kMaxJobs + kMaxSplits;  // a split boundary cuts at most one step in two
 constexpr int kMaxProbs = 64;    // problems of one launch (larger batches take several launches)
+constexpr int kMaxInlineOrder = 2048;  // tile columns whose order a single-problem launch carries inline
 
 // Epilogue shape per accumulation width: with int32 values two warps share each TMEM lane quarter (each
 // takes every other chunk), with int64 values one warp per quarter (its transpose buffer is twice as
@@ -72,6 +74,12 @@ struct Epi {
 struct alignas(64) GemmProb {
   CUtensorMap tmA, tmB;
   int32_t tiles_m, tiles_n, splits, n_pieces;
+  // tile column order: the k-th column of tiles in schedule order is order[order_off + k] (order_off < 0:
+  // k), the order array being GemmLaunch::order for a single problem and the int32 array after the problem
+  // table for a table launch.  With B unpacked OUTER its line groups are sorted by level class, so tiles of
+  // different classes cover the same output columns; the order interleaves them by position, so that the
+  // tiles completing a 32-byte sector of C and Cf run at about the same time.
+  int32_t order_off;
   int32_t split_off[kMaxSplits + 1];
   int32_t pc_kb0[kMaxPieces];    // first 128-deep k-block of the piece
   int32_t pc_nkb[kMaxPieces];    // its k-blocks
@@ -114,6 +122,7 @@ struct GemmLaunch {
   uint64_t timeout_ns;
   const GemmProb* probs;  // nullptr: the problem is `one`
   GemmProb one;
+  int32_t order[kMaxInlineOrder];  // the single problem's tile column order (see GemmProb::order_off)
 };
 // kernel parameters above 4 KB need CUDA 12.1 or later; the limit there is 32 764 bytes
 static_assert(sizeof(GemmLaunch) <= 32764, "GEMM parameters exceed the kernel parameter limit");
@@ -177,6 +186,12 @@ __device__ Unit unit_of(const GemmLaunch& L, int u) {
   r.pb = pb;
   r.mt = tile % pb->tiles_m;
   r.nt = tile / pb->tiles_m;
+  if (pb->order_off >= 0) {
+    if constexpr (kMulti)
+      r.nt = reinterpret_cast<const int32_t*>(L.probs + L.nprob)[pb->order_off + r.nt];
+    else
+      r.nt = L.order[pb->order_off + r.nt];
+  }
   r.pc0 = pb->split_off[s];
   r.npc = pb->split_off[s + 1] - r.pc0;
   return r;
@@ -990,6 +1005,29 @@ imq_status launch_group(const GemmSpec* const* specs, int n, DeviceState* ds, cu
     while (S > 1 && kblocks / S < 16) --S;
   }
 
+  // tile column orders of the problems with B unpacked OUTER: columns sorted by the mean position of their
+  // line groups (stable), all problems' orders in one upload
+  std::vector<int32_t> orders;
+  std::vector<int64_t> order_off((size_t)n, -1);
+  for (int i = 0; i < n; ++i) {
+    const imq_plan_t* pl = specs[i]->plan;
+    std::vector<float> gpos;
+    const int64_t tn = (pl->info.N_unp + bn - 1) / bn;
+    if (tn < 2 || !b_group_positions(pl, &gpos)) continue;
+    const int64_t gpt = bn / 32;  // line groups per tile column
+    std::vector<std::pair<float, int32_t>> key((size_t)tn);
+    for (int64_t t = 0; t < tn; ++t) {
+      double sum = 0.0;
+      int64_t cnt = 0;
+      for (int64_t g = t * gpt; g < (t + 1) * gpt && g < (int64_t)gpos.size(); ++g, ++cnt) sum += gpos[(size_t)g];
+      key[(size_t)t] = {cnt ? (float)(sum / (double)cnt) : 1.0f, (int32_t)t};
+    }
+    std::stable_sort(key.begin(), key.end(),
+                     [](const std::pair<float, int32_t>& x, const std::pair<float, int32_t>& y) { return x.first < y.first; });
+    order_off[(size_t)i] = (int64_t)orders.size();
+    for (const auto& kv : key) orders.push_back(kv.second);
+  }
+
   GemmLaunch* Lp = new GemmLaunch;
   GemmLaunch& L = *Lp;
   memset(&L, 0, sizeof(L));
@@ -1003,6 +1041,14 @@ imq_status launch_group(const GemmSpec* const* specs, int n, DeviceState* ds, cu
     memset(&g, 0, sizeof(g));
     g.tiles_m = (int32_t)((I.M_unp + tm - 1) / tm);
     g.tiles_n = (int32_t)((I.N_unp + bn - 1) / bn);
+    g.order_off = (int32_t)order_off[(size_t)i];
+    if (n == 1 && g.order_off >= 0) {
+      // a single problem carries its order in the parameters, when it fits
+      if ((int64_t)orders.size() <= kMaxInlineOrder)
+        memcpy(L.order, orders.data(), sizeof(int32_t) * orders.size());
+      else
+        g.order_off = -1;
+    }
     if (!build_pieces(pl, S, &g)) {
       delete Lp;
       return IMQ_ERR_UNSUPPORTED;
@@ -1068,8 +1114,12 @@ imq_status launch_group(const GemmSpec* const* specs, int n, DeviceState* ds, cu
   imq_status s = IMQ_OK;
   GemmProb* dtab = nullptr;
   if (n > 1) {
+    // the problem table, then the problems' tile column orders (int32), in one upload
+    std::vector<char> blob(sizeof(GemmProb) * (size_t)n + sizeof(int32_t) * orders.size());
+    memcpy(blob.data(), tab.data(), sizeof(GemmProb) * (size_t)n);
+    if (!orders.empty()) memcpy(blob.data() + sizeof(GemmProb) * (size_t)n, orders.data(), sizeof(int32_t) * orders.size());
     void* d = nullptr;
-    s = upload_table(tab.data(), sizeof(GemmProb) * (size_t)n, &d, st);
+    s = upload_table(blob.data(), blob.size(), &d, st);
     dtab = static_cast<GemmProb*>(d);
     L.probs = dtab;
   }

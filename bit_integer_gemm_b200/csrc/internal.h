@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <vector>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -101,6 +102,7 @@ struct imq_plan {
   int32_t* grpB_L;  // [N_unp / IMQ_B_GROUP]
   int32_t* grpB_n;
   int64_t n_grp_a, n_grp_b;
+  int32_t cls_b0, cls_b1;  // B's OUTER level classes: entries cls_b0 .. cls_b1 - 1 of the host class table
   imq_group groups[IMQ_MAX_GROUPS];
   // GEMM schedule of one output tile (see gemm.cu): a sequence of steps, each one exponent group (or a
   // K-slice of one) accumulated into the tile's TMEM slot.  Consecutive steps of a chunk follow Horner's
@@ -148,6 +150,10 @@ struct GemmSpec {
   float* Cf;
   int64_t ldcf;
 };
+// For B unpacked OUTER: the relative position in N of each group of B'^T's lines, the middle rank of its
+// sources within their level class over the class's size (sources are spread over N, so groups of equal
+// position in different classes cover about the same output columns).  False when B is not OUTER (plan.cu).
+bool b_group_positions(const imq_plan_t* pl, std::vector<float>* pos);
 // The GEMMs of n problems in as few launches as the problem table allows (gemm.cu).
 imq_status launch_gemm_multi(const GemmSpec* specs, int n, cudaStream_t stream);
 }  // namespace imq

@@ -1724,6 +1724,8 @@ imq_status plan_finish(PlanJob& job, const Summary& S, Pinned& pin, DeviceState*
     cls_b0 = ncls;
     outer_classes(3, IMQ_B_GROUP, &pl->n_grp_b);
     cls_b1 = ncls;
+    pl->cls_b0 = cls_b0;
+    pl->cls_b1 = cls_b1;
     I.N_unp = pl->n_grp_b * IMQ_B_GROUP;
     I.N_eff = (int64_t)S.sum[3];
   } else {
@@ -2030,6 +2032,23 @@ imq_status launch_stage2_batch(std::vector<PlanJob>& jobs, cudaStream_t st) {
   s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
   cudaFreeAsync(dt, st);
   return s;
+}
+
+// See internal.h.
+bool b_group_positions(const imq_plan_t* pl, std::vector<float>* pos) {
+  if (!(pl->info.dir_b & IMQ_DIR_OUTER) || pl->n_grp_b <= 0 || !pl->host_tables) return false;
+  const InnerSeg* hsegs = static_cast<const InnerSeg*>(pl->host_tables);
+  const OuterClass* hcls = reinterpret_cast<const OuterClass*>(hsegs + kLv * kLv);
+  pos->assign((size_t)pl->n_grp_b, 0.0f);
+  for (int c = pl->cls_b0; c < pl->cls_b1; ++c) {
+    const OuterClass& k = hcls[c];
+    const int64_t ng = (k.count + k.per - 1) / k.per;
+    for (int64_t g = 0; g < ng && k.grp0 + g < pl->n_grp_b; ++g) {
+      const double first = (double)(g * k.per), n_in = (double)(g < ng - 1 ? k.per : k.count - (ng - 1) * k.per);
+      (*pos)[(size_t)(k.grp0 + g)] = (float)((first + 0.5 * n_in) / (double)k.count);
+    }
+  }
+  return true;
 }
 
 // Builds a plan; see imq_plan in include/imq.h.
