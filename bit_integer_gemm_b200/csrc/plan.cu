@@ -933,6 +933,8 @@ struct MapsArgs {
 };
 // kernel parameters above 4 KB need CUDA 12.1 or later; the limit there is 32 764 bytes
 static_assert(sizeof(MapsArgs) <= 32764, "plan tables exceed the kernel parameter limit");
+// a batch's maps launch uploads the arguments of up to 64 plans through one 256 KB staging buffer
+static_assert(sizeof(MapsArgs) * 64 <= 256 * 1024, "64 plans' maps arguments exceed a staging buffer");
 
 __device__ __forceinline__ StageOrder stage_order(const MapsArgs& m) {
   return StageOrder{m.inline_tables ? m.t.E : m.E, m.ew, m.maxla, m.maxlb, m.perm, m.pinv};
@@ -2012,26 +2014,37 @@ imq_status launch_stage1_batch(std::vector<PlanJob>& jobs, imq_dtype it, DeviceS
   return s;
 }
 
-// Stage 2 of a batch of plans: the order kernels, then the maps kernels, one launch each.
+// Stage 2 of a batch of plans: the order kernels, then the maps kernels, one launch each per 64 plans (the
+// argument table of 64 plans stays within one staging buffer of the upload).
 imq_status launch_stage2_batch(std::vector<PlanJob>& jobs, cudaStream_t st) {
-  std::vector<MapsArgs> tab;
-  int max_order = 0, max_maps = 0;
+  std::vector<MapsArgs> all;
+  std::vector<int> order_blocks, maps_blocks;
   for (PlanJob& j : jobs) {
     if (!j.has_maps) continue;
-    tab.push_back(j.maps);
-    max_order = j.order_blocks > max_order ? j.order_blocks : max_order;
-    max_maps = j.maps_blocks > max_maps ? j.maps_blocks : max_maps;
+    all.push_back(j.maps);
+    order_blocks.push_back(j.order_blocks);
+    maps_blocks.push_back(j.maps_blocks);
   }
-  if (tab.empty() || (max_order == 0 && max_maps == 0)) return IMQ_OK;
-  void* dt = nullptr;
-  imq_status s = upload_table(tab.data(), sizeof(MapsArgs) * tab.size(), &dt, st);
-  if (s != IMQ_OK) return s;
-  const MapsArgs* t = static_cast<const MapsArgs*>(dt);
-  if (max_order > 0) k_plan_order_batch<<<dim3((unsigned)max_order, (unsigned)tab.size()), 1024, 0, st>>>(t);
-  if (max_maps > 0) k_plan_maps_batch<<<dim3((unsigned)max_maps, (unsigned)tab.size()), 1024, 0, st>>>(t);
-  s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
-  cudaFreeAsync(dt, st);
-  return s;
+  constexpr size_t kChunk = 64;
+  for (size_t c0 = 0; c0 < all.size(); c0 += kChunk) {
+    const size_t n = all.size() - c0 < kChunk ? all.size() - c0 : kChunk;
+    int max_order = 0, max_maps = 0;
+    for (size_t i = c0; i < c0 + n; ++i) {
+      max_order = order_blocks[i] > max_order ? order_blocks[i] : max_order;
+      max_maps = maps_blocks[i] > max_maps ? maps_blocks[i] : max_maps;
+    }
+    if (max_order == 0 && max_maps == 0) continue;
+    void* dt = nullptr;
+    imq_status s = upload_table(all.data() + c0, sizeof(MapsArgs) * n, &dt, st);
+    if (s != IMQ_OK) return s;
+    const MapsArgs* t = static_cast<const MapsArgs*>(dt);
+    if (max_order > 0) k_plan_order_batch<<<dim3((unsigned)max_order, (unsigned)n), 1024, 0, st>>>(t);
+    if (max_maps > 0) k_plan_maps_batch<<<dim3((unsigned)max_maps, (unsigned)n), 1024, 0, st>>>(t);
+    s = cudaGetLastError() == cudaSuccess ? IMQ_OK : IMQ_ERR_CUDA;
+    cudaFreeAsync(dt, st);
+    if (s != IMQ_OK) return s;
+  }
+  return IMQ_OK;
 }
 
 // See internal.h.
@@ -2096,7 +2109,9 @@ imq_status build_plans(int batch, const void* A, int64_t strideA, const void* B,
   };
   // A batch queues each kind of plan kernel once for all its plans (the hybrid's choice kernels stay per
   // plan; the debug build's index checks follow each plan's maps, so there stage 2 stays per plan too).
-  const bool batched = batch > 1 && strategy != IMQ_HYBRID && (have_max || (M <= 32768 && K <= 32768 && N <= 32768));
+  // (up to 256 plans: their stage-1 argument tables stay within one staging buffer of the upload)
+  const bool batched = batch > 1 && batch <= 256 && strategy != IMQ_HYBRID &&
+                       (have_max || (M <= 32768 && K <= 32768 && N <= 32768));
   for (int h = 0; h < batch; ++h) {
     PlanJob& j = jobs[h];
     j.batched = batched;
