@@ -418,7 +418,10 @@ imq_status imq_plan_unpack(const void *A, const void *B, imq_dtype it, int64_t M
  * with imq_plan_destroy).  Arguments as imq_plan; the four line-maxima vectors, when all are given,
  * hold batch consecutive vectors (problem h's a_rowmax at a_rowmax + h * M, a_colmax at + h * K,
  * b_rowmax at + h * K, b_colmax at + h * N); when any is NULL each plan computes its own.  Synchronises
- * once for the whole batch.  On an error no plan is returned (every entry of plans is NULL).
+ * once for the whole batch.  Every plan is made as by imq_plan.  Up to 256 plans (except with
+ * IMQ_HYBRID) share their device launches: one per kind of plan kernel for the whole batch.  Larger
+ * batches queue each plan's kernels in turn.  On an error no plan is returned (every entry of plans is
+ * NULL).
  */
 imq_status imq_plan_batched(int32_t batch, const void *A, int64_t strideA, const void *B, int64_t strideB,
                             imq_dtype it, int64_t M, int64_t K, int64_t N, int32_t transA, int64_t lda,
